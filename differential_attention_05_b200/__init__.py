@@ -1,0 +1,27 @@
+"""B200-native differential attention (DIFF Transformer V1 / V2 operator).
+
+The compute path is the C-ABI library libdiffattn.so (hand-written sm_100a kernels,
+declared in include/diffattn.h). This package is a thin ctypes binding over it; the
+functions load the library on first use and raise if it is missing.
+"""
+from ._binding import (  # noqa: F401
+    DiffattnError,
+    diffattn_lambda,
+    diffattn_fwd_prefill,
+    diffattn_fwd_decode,
+    diffattn_decode_workspace_size,
+    diffattn_status_string,
+    library_path,
+    load_library,
+)
+
+__all__ = [
+    "DiffattnError",
+    "diffattn_lambda",
+    "diffattn_fwd_prefill",
+    "diffattn_fwd_decode",
+    "diffattn_decode_workspace_size",
+    "diffattn_status_string",
+    "library_path",
+    "load_library",
+]

@@ -1,0 +1,262 @@
+"""ctypes binding over libdiffattn.so (include/diffattn.h).
+
+Argument marshalling only: tensors become pointers, shapes and element strides become
+the parameter structs, and the current torch CUDA stream becomes the launch stream.
+Every step of the operator runs in the library's kernels. There is no fallback: if the
+library is missing or a call fails, these functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libdiffattn.so"
+
+DIFFATTN_F32, DIFFATTN_BF16 = 0, 1
+DIFFATTN_V1, DIFFATTN_V2 = 1, 2
+
+STATUS = {
+    0: "DIFFATTN_OK",
+    -1: "DIFFATTN_ERR_INVALID_ARG",
+    -2: "DIFFATTN_ERR_UNSUPPORTED",
+    -3: "DIFFATTN_ERR_MISALIGNED",
+    -4: "DIFFATTN_ERR_WORKSPACE",
+    -5: "DIFFATTN_ERR_CUDA",
+    -6: "DIFFATTN_ERR_TIMEOUT",
+}
+
+# every symbol include/diffattn.h declares
+EXPORTS = (
+    "diffattn_version",
+    "diffattn_status_string",
+    "diffattn_lambda",
+    "diffattn_fwd_prefill",
+    "diffattn_decode_workspace_size",
+    "diffattn_fwd_decode",
+)
+
+
+class DiffattnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} returned {status} ({STATUS.get(status, 'unknown')})")
+
+
+class PrefillParams(ctypes.Structure):
+    _fields_ = [
+        ("variant", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("batch", ctypes.c_int32),
+        ("seqlen", ctypes.c_int32),
+        ("n_q_heads", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("causal", ctypes.c_int32),
+        ("apply_norm", ctypes.c_int32),
+        ("norm_eps", ctypes.c_float),
+        ("q_strides", ctypes.c_int64 * 3),
+        ("k_strides", ctypes.c_int64 * 3),
+        ("v_strides", ctypes.c_int64 * 3),
+        ("o_strides", ctypes.c_int64 * 3),
+    ]
+
+
+class DecodeParams(ctypes.Structure):
+    _fields_ = [
+        ("variant", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("batch", ctypes.c_int32),
+        ("max_kv_len", ctypes.c_int32),
+        ("n_q_heads", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("num_splits", ctypes.c_int32),
+        ("q_strides", ctypes.c_int64 * 2),
+        ("kv_strides", ctypes.c_int64 * 3),
+        ("o_strides", ctypes.c_int64 * 2),
+    ]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return os.environ.get("DIFFATTN_LIBRARY", os.path.join(_HERE, _LIB_NAME))
+
+
+def load_library():
+    """Load libdiffattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m differential_attention_05_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    vp, i32, f32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
+    lib.diffattn_version.restype = i32
+    lib.diffattn_version.argtypes = []
+    lib.diffattn_status_string.restype = ctypes.c_char_p
+    lib.diffattn_status_string.argtypes = [i32]
+    lib.diffattn_lambda.restype = i32
+    lib.diffattn_lambda.argtypes = [f32p, f32p, f32p, f32p, i32, i32, i32, f32p, f32p, vp]
+    lib.diffattn_fwd_prefill.restype = i32
+    lib.diffattn_fwd_prefill.argtypes = [ctypes.POINTER(PrefillParams), vp, vp, vp, f32p, f32p,
+                                         vp, vp, vp]
+    lib.diffattn_decode_workspace_size.restype = i32
+    lib.diffattn_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeParams),
+                                                   ctypes.POINTER(ctypes.c_size_t)]
+    lib.diffattn_fwd_decode.restype = i32
+    lib.diffattn_fwd_decode.argtypes = [ctypes.POINTER(DecodeParams), vp, vp, vp, vp, f32p, vp,
+                                        vp, ctypes.c_size_t, vp, vp]
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise DiffattnError(fn, rc)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return DIFFATTN_BF16
+    if t.dtype == torch.float32:
+        return DIFFATTN_F32
+    raise DiffattnError("dtype", -2)
+
+
+def diffattn_status_string(status: int) -> str:
+    return load_library().diffattn_status_string(int(status)).decode()
+
+
+def diffattn_lambda(lq1, lk1, lq2, lk2, depth: int, lambda_out=None, lambda_init_out=None,
+                    stream=None):
+    """lambda[h] = exp(lq1[h].lk1[h]) - exp(lq2[h].lk2[h]) + lambda_init(depth), on device.
+    lq*, lk*: float32 CUDA tensors [n_heads, dim]. Returns (lambda_out, lambda_init_out)."""
+    import torch
+    lib = load_library()
+    H, dim = lq1.shape
+    if lambda_out is None:
+        lambda_out = torch.empty(H, dtype=torch.float32, device=lq1.device)
+    if lambda_init_out is None:
+        lambda_init_out = torch.empty(1, dtype=torch.float32, device=lq1.device)
+    for t in (lq1, lk1, lq2, lk2):
+        if not t.is_contiguous():
+            raise DiffattnError("diffattn_lambda", -1)
+    rc = lib.diffattn_lambda(_ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), H, dim, int(depth),
+                             _ptr(lambda_out), _ptr(lambda_init_out), _stream(stream))
+    _check("diffattn_lambda", rc)
+    return lambda_out, lambda_init_out
+
+
+def prefill_params(q, k, v, out, causal=True, apply_norm=None, norm_eps=1e-5) -> PrefillParams:
+    """Build the prefill parameter struct from tensor shapes and strides.
+    V1: q,k [B,N,H,2,d], v,out [B,N,H,2d]. V2: q [B,N,Hq,d], k,v [B,N,Hkv,d], out [B,N,Hq/2,d]."""
+    p = PrefillParams()
+    if q.dim() == 5:
+        B, N, H, two, d = q.shape
+        p.variant, p.n_q_heads, p.n_kv_heads = DIFFATTN_V1, H, H
+        if two != 2:
+            raise DiffattnError("diffattn_fwd_prefill", -1)
+        p.apply_norm = 1 if apply_norm is None else int(bool(apply_norm))
+        qs, ks = q.stride(), k.stride()
+        p.q_strides[:] = (qs[0], qs[1], qs[2])
+        p.k_strides[:] = (ks[0], ks[1], ks[2])
+        if qs[3] != d or ks[3] != d or qs[4] != 1 or ks[4] != 1:
+            raise DiffattnError("diffattn_fwd_prefill", -1)
+    elif q.dim() == 4:
+        B, N, Hq, d = q.shape
+        p.variant, p.n_q_heads, p.n_kv_heads = DIFFATTN_V2, Hq, k.shape[2]
+        p.apply_norm = 0 if apply_norm is None else int(bool(apply_norm))
+        p.q_strides[:] = q.stride()[:3]
+        p.k_strides[:] = k.stride()[:3]
+        if q.stride(3) != 1 or k.stride(3) != 1:
+            raise DiffattnError("diffattn_fwd_prefill", -1)
+    else:
+        raise DiffattnError("diffattn_fwd_prefill", -1)
+    if v.stride(-1) != 1 or out.stride(-1) != 1:
+        raise DiffattnError("diffattn_fwd_prefill", -1)
+    p.dtype = _dtype_code(q)
+    p.batch, p.seqlen, p.head_dim = B, N, d
+    p.causal = int(bool(causal))
+    p.norm_eps = float(norm_eps)
+    p.v_strides[:] = v.stride()[:3]
+    p.o_strides[:] = out.stride()[:3]
+    return p
+
+
+def diffattn_fwd_prefill(q, k, v, lam, lambda_init=None, out=None, causal=True, apply_norm=None,
+                         norm_eps=1e-5, dev_status=None, stream=None):
+    """Fused differential attention prefill (see include/diffattn.h for layouts)."""
+    import torch
+    lib = load_library()
+    if out is None:
+        if q.dim() == 5:
+            B, N, H, _, d = q.shape
+            out = torch.empty((B, N, H, 2 * d), dtype=q.dtype, device=q.device)
+        else:
+            B, N, Hq, d = q.shape
+            out = torch.empty((B, N, Hq // 2, d), dtype=q.dtype, device=q.device)
+    p = prefill_params(q, k, v, out, causal, apply_norm, norm_eps)
+    rc = lib.diffattn_fwd_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                                  _ptr(lambda_init), _ptr(out), _ptr(dev_status), _stream(stream))
+    _check("diffattn_fwd_prefill", rc)
+    return out
+
+
+def decode_params(q, k_cache, v_cache, out, num_splits=0) -> DecodeParams:
+    p = DecodeParams()
+    B, Hq, d = q.shape
+    _, L, Hkv, _ = k_cache.shape
+    if tuple(k_cache.stride()) != tuple(v_cache.stride()):
+        raise DiffattnError("diffattn_fwd_decode", -1)
+    p.variant, p.dtype = DIFFATTN_V2, _dtype_code(q)
+    p.batch, p.max_kv_len, p.n_q_heads, p.n_kv_heads, p.head_dim = B, L, Hq, Hkv, d
+    p.num_splits = int(num_splits)
+    p.q_strides[:] = q.stride()[:2]
+    p.kv_strides[:] = k_cache.stride()[:3]
+    p.o_strides[:] = out.stride()[:2]
+    return p
+
+
+def diffattn_decode_workspace_size(p: DecodeParams) -> int:
+    n = ctypes.c_size_t(0)
+    _check("diffattn_decode_workspace_size",
+           load_library().diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return int(n.value)
+
+
+def diffattn_fwd_decode(q, k_cache, v_cache, lam, kv_len=None, out=None, workspace=None,
+                        num_splits=0, dev_status=None, stream=None):
+    """Split-KV differential decode (V2). q [B,Hq,d], caches [B,L,Hkv,d] -> out [B,Hq/2,d]."""
+    import torch
+    lib = load_library()
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq // 2, d), dtype=q.dtype, device=q.device)
+    p = decode_params(q, k_cache, v_cache, out, num_splits)
+    need = diffattn_decode_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib.diffattn_fwd_decode(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                 _ptr(kv_len), _ptr(lam), _ptr(out), _ptr(workspace), ws_bytes,
+                                 _ptr(dev_status), _stream(stream))
+    _check("diffattn_fwd_decode", rc)
+    return out

@@ -1,0 +1,198 @@
+/*
+ * diffattn.h -- C ABI of the B200 (sm_100a) differential attention library.
+ *
+ * The operator (DIFF Transformer attention) as the pages state it:
+ *
+ *   A_1 = softmax(Q_1 K_1^T / sqrt(d)),  A_2 = softmax(Q_2 K_2^T / sqrt(d))
+ *   DiffAttn = (A_1 - lambda * A_2) V
+ *     -- "Differential Attention (V2)" lesson (AI Engineering from Scratch, Phase 10),
+ *        The Concept, "The difference idea"; "Attention Variants: Sliding Window, Sparse,
+ *        Differential", Build It, Step 4 (diff_attention(Q1, K1, Q2, K2, V, lam)).
+ *   lambda = exp(lq1 . lk1) - exp(lq2 . lk2) + lambda_init, one scalar per head
+ *     -- "Differential Attention (V2)", The Concept; Key Terms, "lambda".
+ *   lambda_init = 0.8 - 0.6 * exp(-0.3 * (depth - 1))
+ *     -- skill-diff-attention-integrator, "Architecture diff".
+ *   V1: head dim halved per branch, V of width 2d, per-head RMSNorm after the
+ *       subtraction, then the (1 - lambda_init) output scale
+ *     -- "Differential Attention (V2)", "V1 vs V2"; Key Terms, "Per-head RMSNorm";
+ *        Hugging Face post on the DIFF Transformer, "How?" (GroupNorm per head).
+ *   V2: twice the query heads over unchanged KV heads (GQA); query heads 2p and 2p+1
+ *       are the two branches of pair p and share one KV head; no per-head norm
+ *     -- "Differential Attention (V2)", "V1 vs V2"; compatibility table ("GQA: yes").
+ *   Causal: query i sees keys j <= i
+ *     -- "Attention Variants", Build It, Step 1 (causal_mask).
+ *
+ * Conventions for every entry point
+ *   - Pointers are DEVICE pointers unless marked "host". The caller owns every buffer;
+ *     the library allocates nothing, frees nothing and keeps no pointer after a call.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     The library never synchronizes.
+ *   - Arguments are validated on the host before anything is launched. On any error
+ *     status nothing is launched and no output is written.
+ *   - CUDA launch failures return DIFFATTN_ERR_CUDA. Conditions a kernel detects while
+ *     running (a bounded wait that gave up) are written to `dev_status` (a device int,
+ *     nullable), which the caller reads after synchronizing; 0 means success, otherwise
+ *     a diffattn_status value. Kernels never trap.
+ *   - No C++ exception crosses this boundary.
+ *   - Element strides are in elements, not bytes. The innermost dimension is always
+ *     contiguous (stride 1).
+ */
+#ifndef DIFFATTN_H_
+#define DIFFATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DIFFATTN_OK = 0,
+  DIFFATTN_ERR_INVALID_ARG = -1, /* null pointer, negative size, inconsistent shape */
+  DIFFATTN_ERR_UNSUPPORTED = -2, /* valid request this build does not implement */
+  DIFFATTN_ERR_MISALIGNED = -3,  /* pointer or stride violates the alignment rules */
+  DIFFATTN_ERR_WORKSPACE = -4,   /* workspace missing or smaller than required */
+  DIFFATTN_ERR_CUDA = -5,        /* a CUDA runtime / driver call failed */
+  DIFFATTN_ERR_TIMEOUT = -6      /* a kernel's bounded wait gave up (dev_status only) */
+} diffattn_status;
+
+typedef enum { DIFFATTN_F32 = 0, DIFFATTN_BF16 = 1 } diffattn_dtype;
+typedef enum { DIFFATTN_V1 = 1, DIFFATTN_V2 = 2 } diffattn_variant;
+
+/* Library ABI version (major * 100 + minor). */
+int diffattn_version(void);
+
+/* Static description of a status code. Never NULL. */
+const char* diffattn_status_string(int status);
+
+/*
+ * diffattn_lambda -- the lambda re-parameterisation, on the device.
+ *
+ *   lambda_out[h] = exp(lq1[h,:] . lk1[h,:]) - exp(lq2[h,:] . lk2[h,:]) + lambda_init
+ *   lambda_init   = 0.8 - 0.6 * exp(-0.3 * (depth - 1))
+ * ("Differential Attention (V2)", The Concept; skill-diff-attention-integrator,
+ * "Architecture diff"). lambda may be negative; nothing is clamped.
+ *
+ * lq1, lk1, lq2, lk2 : float32 [n_heads, dim], row-major, 16-byte aligned
+ *                      (n_heads = V1 heads, or V2 pairs)
+ * lambda_out         : float32 [n_heads]
+ * lambda_init_out    : float32 [1] or NULL
+ * depth              : layer depth, >= 1
+ * Sizes: 1 <= n_heads <= 65535, 1 <= dim <= 4096.
+ * Arithmetic: fp32 dot products in a fixed order, fp32 expf.
+ */
+int diffattn_lambda(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
+                    int n_heads, int dim, int depth, float* lambda_out, float* lambda_init_out,
+                    void* stream);
+
+/*
+ * Prefill parameters.
+ *
+ * V1 (variant = DIFFATTN_V1): n_q_heads = n_kv_heads = H differential heads,
+ *   head_dim = d per branch (d = 64 for bf16; any 1..128 multiple of 4 for f32).
+ *   q, k : [B, N, H, 2, d]   branch 1 at index 0, branch 2 at index 1 (contiguous, so
+ *                            each (token, head) row holds q1 then q2)
+ *   v    : [B, N, H, 2d]
+ *   out  : [B, N, H, 2d]
+ *   lambda: [H]. apply_norm = 1 applies the per-head RMSNorm (over the 2d channels,
+ *   eps = norm_eps, unit gain) and then multiplies by (1 - lambda_init[0]).
+ * V2 (variant = DIFFATTN_V2): n_q_heads = Hq (even), n_kv_heads = Hkv with Hq/Hkv even;
+ *   head_dim = d (128 for bf16; any 1..128 multiple of 4 for f32).
+ *   q    : [B, N, Hq, d]     query heads 2p, 2p+1 = branches 1, 2 of pair p
+ *   k, v : [B, N, Hkv, d]    query head h reads KV head h / (Hq / Hkv)
+ *   out  : [B, N, Hq/2, d]
+ *   lambda: [Hq/2]. apply_norm must be 0.
+ * Strides (elements) are {batch, token, head}; the branch axis (V1) and the channel
+ * axis are contiguous. bf16: q/k/v base pointers 16-byte aligned and every stride a
+ * multiple of 8 elements (TMA rules); f32: 16-byte aligned, strides multiple of 4.
+ * out must not alias q, k or v.
+ * causal = 1: query i attends keys 0..i (queries and keys share positions 0..N-1);
+ * causal = 0: every query attends all N keys.
+ */
+typedef struct {
+  int32_t variant;    /* diffattn_variant */
+  int32_t dtype;      /* diffattn_dtype of q, k, v and out */
+  int32_t batch;      /* B >= 0 */
+  int32_t seqlen;     /* N >= 0 (queries = keys = N) */
+  int32_t n_q_heads;  /* V1: H; V2: Hq */
+  int32_t n_kv_heads; /* V1: H; V2: Hkv */
+  int32_t head_dim;   /* d per branch */
+  int32_t causal;     /* 1 = causal, 0 = full */
+  int32_t apply_norm; /* V1: 1 = RMSNorm + (1 - lambda_init) scale; V2: 0 */
+  float norm_eps;     /* RMSNorm epsilon (1e-5) */
+  int64_t q_strides[3];
+  int64_t k_strides[3];
+  int64_t v_strides[3];
+  int64_t o_strides[3];
+} diffattn_prefill_params;
+
+/*
+ * diffattn_fwd_prefill -- fused causal/full differential attention forward.
+ * One pass over the keys; both attention maps stay on chip (never written to memory).
+ * bf16: tcgen05 tensor-core kernel, fp32 accumulation, P rounded to bf16 as an MMA
+ * operand only; fp32: exact-fp32 SIMT kernel.
+ *
+ * lambda      : float32 [n_units] (V1 heads / V2 pairs), device
+ * lambda_init : float32 [1], device; read only when apply_norm = 1 (may be NULL otherwise)
+ * dev_status  : nullable device int, see the conventions above
+ * B == 0 or N == 0 launches nothing and returns DIFFATTN_OK.
+ */
+int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const void* k,
+                         const void* v, const float* lambda, const float* lambda_init, void* out,
+                         int* dev_status, void* stream);
+
+/*
+ * Decode parameters (V2 only; bf16 only).
+ *   q       : [B, Hq, d]        one new query token per batch entry
+ *   k_cache : [B, L, Hkv, d]    L = max_kv_len (cache capacity)
+ *   v_cache : [B, L, Hkv, d]    same strides as k_cache
+ *   kv_len  : int32 [B] or NULL (NULL = every entry holds L keys); 0 <= kv_len[b] <= L
+ *   out     : [B, Hq/2, d]
+ * The new query attends every cached key 0 .. kv_len[b]-1 (its own key is expected to be
+ * in the cache already). Hq / Hkv must be 8 and d = 128 in this build.
+ * Strides (elements): q {batch, head}, kv {batch, token, head}, out {batch, pair};
+ * 16-byte aligned base pointers, strides multiples of 8 elements.
+ */
+typedef struct {
+  int32_t variant;    /* DIFFATTN_V2 */
+  int32_t dtype;      /* DIFFATTN_BF16 */
+  int32_t batch;      /* B >= 0 */
+  int32_t max_kv_len; /* L >= 0 */
+  int32_t n_q_heads;  /* Hq */
+  int32_t n_kv_heads; /* Hkv */
+  int32_t head_dim;   /* d */
+  int32_t num_splits; /* KV splits per (batch, KV head); 0 = chosen by the library */
+  int64_t q_strides[2];
+  int64_t kv_strides[3];
+  int64_t o_strides[2];
+} diffattn_decode_params;
+
+/*
+ * diffattn_decode_workspace_size -- device workspace bytes diffattn_fwd_decode needs
+ * for these parameters (written to *bytes, a HOST pointer). The workspace holds the
+ * per-split partial softmax states; its contents need no initialisation.
+ */
+int diffattn_decode_workspace_size(const diffattn_decode_params* p, size_t* bytes);
+
+/*
+ * diffattn_fwd_decode -- split-KV differential decode. Each (batch, KV head, split)
+ * block streams its slice of the cache once with 128-bit loads and scores it for all
+ * query heads of the GQA group (both branches of every pair), keeping one running
+ * (max, sum, output) state per query head. A second, small kernel merges the per-split
+ * states of each head and applies O = O_1/l_1 - lambda * O_2/l_2 per pair.
+ *
+ * lambda     : float32 [Hq/2], device
+ * workspace  : device buffer of at least diffattn_decode_workspace_size() bytes,
+ *              256-byte aligned; calls sharing a workspace must not overlap in time
+ * dev_status : nullable device int
+ */
+int diffattn_fwd_decode(const diffattn_decode_params* p, const void* q, const void* k_cache,
+                        const void* v_cache, const int32_t* kv_len, const float* lambda, void* out,
+                        void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIFFATTN_H_ */

@@ -1,0 +1,188 @@
+"""Float64 CPU oracle for differential attention (ctypes wrapper over diffattn_oracle.c).
+
+TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the benchmark's
+CPU-baseline / reference leg may import this module. The product package never imports
+it, and nothing here is shared with the CUDA path.
+
+The C source states, function by function, which passage of the pages each step
+follows. This wrapper only converts numpy arrays to contiguous float64 and calls it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "diffattn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_libs: dict = {}
+_active = None
+
+
+def compile_source(src: str, out: str) -> str:
+    """gcc, IEEE float64, no fast-math, no FMA contraction."""
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.check_call(
+        ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+         "-fno-fast-math", "-o", tmp, src, "-lm", "-lpthread"])
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile diffattn_oracle.c into oracle/liboracle.so."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        compile_source(_SRC, _LIB)
+    return _LIB
+
+
+class use_library:
+    """Context manager that points this module at another build of the oracle source
+    (used by the tests that plant a mistake in a copy of the oracle)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _active
+        self._prev = _active
+        _active = self.path
+        return self
+
+    def __exit__(self, *exc):
+        global _active
+        _active = self._prev
+        return False
+
+
+def _load():
+    path = _active or build()
+    lib = _libs.get(path)
+    if lib is None:
+        lib = ctypes.CDLL(os.path.abspath(path))
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.oracle_lambda_init.restype = ctypes.c_double
+        lib.oracle_lambda_init.argtypes = [ctypes.c_int]
+        lib.oracle_lambda.restype = ctypes.c_int
+        lib.oracle_lambda.argtypes = [dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, dp]
+        lib.oracle_prefill_v1.restype = ctypes.c_int
+        lib.oracle_prefill_v1.argtypes = [dp, dp, dp, dp, ctypes.c_double] + [ctypes.c_int] * 6 + [
+            ctypes.c_double, ip, ctypes.c_int, dp, ctypes.c_int]
+        lib.oracle_prefill_v2.restype = ctypes.c_int
+        lib.oracle_prefill_v2.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 6 + [
+            ip, ctypes.c_int, dp, ctypes.c_int]
+        lib.oracle_decode_v2.restype = ctypes.c_int
+        lib.oracle_decode_v2.argtypes = [dp, dp, dp, ip, dp] + [ctypes.c_int] * 5 + [dp, ctypes.c_int]
+        lib.oracle_map_row_v2.restype = ctypes.c_int
+        lib.oracle_map_row_v2.argtypes = [dp, dp] + [ctypes.c_int] * 6 + [dp, dp]
+        _libs[path] = lib
+    return lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _dp(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _ip(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
+def default_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return max(1, os.cpu_count() or 1)
+
+
+def lambda_init(depth: int) -> float:
+    return float(_load().oracle_lambda_init(int(depth)))
+
+
+def lambda_(lq1, lk1, lq2, lk2, depth: int) -> np.ndarray:
+    """lambda per head from the four [H, d] re-parameterisation vectors."""
+    a = [_f64(x) for x in (lq1, lk1, lq2, lk2)]
+    H, d = a[0].shape
+    out = np.zeros(H, dtype=np.float64)
+    rc = _load().oracle_lambda(*[_dp(x) for x in a], H, d, int(depth), _dp(out))
+    if rc != 0:
+        raise ValueError(f"oracle_lambda failed: {rc}")
+    return out
+
+
+def _rows(rows, N):
+    if rows is None:
+        return None, N
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    return r, int(r.size)
+
+
+def prefill_v1(q, k, v, lam, lambda_init_value: float, causal=True, apply_norm=True,
+               eps=1e-5, rows=None, threads=None) -> np.ndarray:
+    """V1 prefill. q,k: [B,N,H,2,d]; v: [B,N,H,2d]; lam: [H] -> out [B,R,H,2d]."""
+    q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
+    B, N, H, two, d = q.shape
+    assert two == 2 and k.shape == q.shape and v.shape == (B, N, H, 2 * d) and lam.shape == (H,)
+    r, R = _rows(rows, N)
+    out = np.zeros((B, R, H, 2 * d), dtype=np.float64)
+    rc = _load().oracle_prefill_v1(_dp(q), _dp(k), _dp(v), _dp(lam), float(lambda_init_value),
+                                   B, N, H, d, int(bool(causal)), int(bool(apply_norm)), float(eps),
+                                   _ip(r), R, _dp(out), int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_prefill_v1 failed: {rc}")
+    return out
+
+
+def prefill_v2(q, k, v, lam, causal=True, rows=None, threads=None) -> np.ndarray:
+    """V2 prefill. q: [B,N,Hq,d]; k,v: [B,N,Hkv,d]; lam: [Hq/2] -> out [B,R,Hq/2,d]."""
+    q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    assert k.shape == (B, N, Hkv, d) and v.shape == k.shape and lam.shape == (Hq // 2,)
+    r, R = _rows(rows, N)
+    out = np.zeros((B, R, Hq // 2, d), dtype=np.float64)
+    rc = _load().oracle_prefill_v2(_dp(q), _dp(k), _dp(v), _dp(lam), B, N, Hq, Hkv, d,
+                                   int(bool(causal)), _ip(r), R, _dp(out),
+                                   int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_prefill_v2 failed: {rc}")
+    return out
+
+
+def decode_v2(q, k, v, lam, kv_len=None, threads=None) -> np.ndarray:
+    """V2 decode. q: [B,Hq,d]; k,v: [B,L,Hkv,d]; kv_len: [B] or None -> out [B,Hq/2,d]."""
+    q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
+    B, Hq, d = q.shape
+    L, Hkv = k.shape[1], k.shape[2]
+    assert k.shape == (B, L, Hkv, d) and v.shape == k.shape and lam.shape == (Hq // 2,)
+    kl = None if kv_len is None else np.ascontiguousarray(np.asarray(kv_len, dtype=np.int32))
+    out = np.zeros((B, Hq // 2, d), dtype=np.float64)
+    rc = _load().oracle_decode_v2(_dp(q), _dp(k), _dp(v), _ip(kl), _dp(lam), B, L, Hq, Hkv, d,
+                                  _dp(out), int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_decode_v2 failed: {rc}")
+    return out
+
+
+def map_row_v2(q, k, p: int, i: int):
+    """The two softmax rows (A_1[i, :i+1], A_2[i, :i+1]) of pair p, one batch entry.
+    q: [N,Hq,d]; k: [N,Hkv,d]."""
+    q, k = _f64(q), _f64(k)
+    N, Hq, d = q.shape
+    Hkv = k.shape[1]
+    a1 = np.zeros(i + 1, dtype=np.float64)
+    a2 = np.zeros(i + 1, dtype=np.float64)
+    rc = _load().oracle_map_row_v2(_dp(q), _dp(k), N, Hq, Hkv, d, int(p), int(i), _dp(a1), _dp(a2))
+    if rc != 0:
+        raise ValueError(f"oracle_map_row_v2 failed: {rc}")
+    return a1, a2

@@ -1,0 +1,287 @@
+"""Pins of the float64 oracle to things other than itself.
+
+Each pin raises AssertionError when the oracle disagrees with what the pages or the
+mathematics fix. tests/test_oracle_pins.py runs them against the oracle as built, and
+tests/test_oracle_mutants.py runs them against copies of the oracle source with one
+planted mistake each, expecting every mutant to fail at least one pin.
+
+Independent references used here (none of them is the oracle's code):
+  * torch.nn.functional.scaled_dot_product_attention in float64 on the CPU -- lambda = 0
+    reduces differential attention to standard (causal) softmax attention;
+  * torch.softmax / matmul / rms_norm in float64 -- the printed operator
+    (A_1 - lambda A_2) V ("Attention Variants", Build It, Step 4) evaluated by a library;
+  * mpmath at 40 digits, exp / sum without max-subtraction -- brute force on tiny inputs;
+  * closed forms: row sums, identical branches, the first causal row, lambda values for
+    chosen vectors, the lambda_init schedule's end points;
+  * the pages' noise-cancellation claim on a length-1024 signal-plus-noise sequence.
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+from differential_attention_05_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _sdpa(q, k, v, causal):
+    """q [B,H,N,d] f64 -> standard softmax attention (library routine)."""
+    d = q.shape[-1]
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), is_causal=causal,
+        scale=1.0 / math.sqrt(d)).numpy()
+
+
+def _close(a, b, tol, what):
+    err = float(np.max(np.abs(np.asarray(a) - np.asarray(b)))) if np.size(a) else 0.0
+    assert err <= tol, f"{what}: max abs err {err:.3e} > {tol:.1e}"
+
+
+# ---- lambda and lambda_init ----------------------------------------------------------
+
+def pin_lambda_init_schedule():
+    rows = [ln.split() for ln in open(os.path.join(GOLDEN, "lambda_init.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    for depth, value, tol in rows:
+        dep = 400 if depth == "inf" else int(depth)
+        _close(oracle.lambda_init(dep), float(value), float(tol), f"lambda_init(depth={depth})")
+    vals = [oracle.lambda_init(dd) for dd in range(1, 40)]
+    assert all(b > a for a, b in zip(vals, vals[1:])), "lambda_init must rise with depth"
+
+
+def pin_lambda_closed_form():
+    """Vectors whose dot products are ln 3 and ln 2 give exp terms 3 and 2 exactly;
+    cross products (lq1.lk2, lq2.lk1) are zero, so a swapped pairing gives 0."""
+    d = 6
+    lq1 = np.zeros((3, d)); lk1 = np.zeros((3, d)); lq2 = np.zeros((3, d)); lk2 = np.zeros((3, d))
+    # head 0: lambda = 3 - 2 + li
+    lq1[0, 0], lk1[0, 0] = math.log(3.0), 1.0
+    lq2[0, 1], lk2[0, 1] = 2.0, math.log(2.0) / 2.0
+    # head 1: all zero -> 1 - 1 + li
+    # head 2: lambda = 1 - 5 + li  (negative: "can be negative")
+    lq2[2, 3], lk2[2, 3] = math.log(5.0), 1.0
+    for depth in (1, 7):
+        li = oracle.lambda_init(depth)
+        lam = oracle.lambda_(lq1, lk1, lq2, lk2, depth)
+        _close(lam, [1.0 + li, li, -4.0 + li], 1e-14, f"lambda closed form (depth {depth})")
+        assert lam[2] < 0
+
+
+# ---- softmax attention special case (lambda = 0) -------------------------------------
+
+def pin_lambda0_is_softmax_attention_v1():
+    r = _rng(1)
+    B, N, H, d = 2, 37, 3, 8
+    q = r.standard_normal((B, N, H, 2, d)); k = r.standard_normal((B, N, H, 2, d))
+    v = r.standard_normal((B, N, H, 2 * d))
+    lam = np.zeros(H)
+    for causal in (True, False):
+        out = oracle.prefill_v1(q, k, v, lam, 0.3, causal=causal, apply_norm=False, threads=2)
+        ref = _sdpa(q[:, :, :, 0].transpose(0, 2, 1, 3).copy(), k[:, :, :, 0].transpose(0, 2, 1, 3).copy(),
+                    v.transpose(0, 2, 1, 3).copy(), causal).transpose(0, 2, 1, 3)
+        _close(out, ref, 1e-12, f"V1 lambda=0 vs SDPA (causal={causal})")
+
+
+def pin_lambda0_is_softmax_attention_v2():
+    r = _rng(2)
+    B, N, Hq, Hkv, d = 2, 29, 8, 2, 16
+    q = r.standard_normal((B, N, Hq, d)); k = r.standard_normal((B, N, Hkv, d))
+    v = r.standard_normal((B, N, Hkv, d))
+    lam = np.zeros(Hq // 2)
+    group = Hq // Hkv
+    for causal in (True, False):
+        out = oracle.prefill_v2(q, k, v, lam, causal=causal, threads=2)
+        kk = np.repeat(k, group, axis=2)  # query head h reads KV head h // group
+        vv = np.repeat(v, group, axis=2)
+        ref = _sdpa(q.transpose(0, 2, 1, 3).copy(), kk.transpose(0, 2, 1, 3).copy(),
+                    vv.transpose(0, 2, 1, 3).copy(), causal).transpose(0, 2, 1, 3)
+        _close(out, ref[:, :, 0::2], 1e-12, f"V2 lambda=0 vs SDPA on heads 2p (causal={causal})")
+
+
+def pin_lambda0_decode_is_softmax_attention():
+    r = _rng(3)
+    B, L, Hq, Hkv, d = 3, 41, 8, 2, 16
+    q = r.standard_normal((B, Hq, d)); k = r.standard_normal((B, L, Hkv, d))
+    v = r.standard_normal((B, L, Hkv, d))
+    kv_len = np.array([41, 1, 17], dtype=np.int32)
+    out = oracle.decode_v2(q, k, v, np.zeros(Hq // 2), kv_len=kv_len, threads=2)
+    group = Hq // Hkv
+    for b in range(B):
+        n = kv_len[b]
+        kk = np.repeat(k[b, :n], group, axis=1).transpose(1, 0, 2)[None].copy()
+        vv = np.repeat(v[b, :n], group, axis=1).transpose(1, 0, 2)[None].copy()
+        ref = _sdpa(q[b][None, :, None, :].copy(), kk, vv, False)[0, :, 0, :]
+        _close(out[b], ref[0::2], 1e-12, f"decode lambda=0 vs SDPA (b={b}, kv_len={n})")
+
+
+# ---- invariants of the difference -----------------------------------------------------
+
+def pin_identical_branches_cancel():
+    """Q1 = Q2, K1 = K2 and lambda = 1: (A_1 - A_2) V = 0 before the norm."""
+    r = _rng(4)
+    B, N, H, d = 1, 23, 2, 8
+    q1 = r.standard_normal((B, N, H, 1, d)); k1 = r.standard_normal((B, N, H, 1, d))
+    q = np.concatenate([q1, q1], axis=3); k = np.concatenate([k1, k1], axis=3)
+    v = r.standard_normal((B, N, H, 2 * d))
+    out = oracle.prefill_v1(q, k, v, np.ones(H), 0.2, apply_norm=False, threads=1)
+    _close(out, 0.0, 1e-15, "V1 identical branches, lambda=1")
+    Hq, Hkv = 4, 2
+    qv = r.standard_normal((B, N, Hq // 2, d))
+    q2 = np.repeat(qv, 2, axis=2)  # heads 2p and 2p+1 equal
+    k2 = r.standard_normal((B, N, Hkv, d)); v2 = r.standard_normal((B, N, Hkv, d))
+    out2 = oracle.prefill_v2(q2, k2, v2, np.ones(Hq // 2), threads=1)
+    _close(out2, 0.0, 1e-15, "V2 identical branches, lambda=1")
+
+
+def pin_rows_sum_to_one_minus_lambda():
+    """Every softmax row sums to 1, so with V = 1 each output channel is 1 - lambda."""
+    r = _rng(5)
+    B, N, H, d = 1, 19, 3, 4
+    q = r.standard_normal((B, N, H, 2, d)) * 3; k = r.standard_normal((B, N, H, 2, d)) * 3
+    v = np.ones((B, N, H, 2 * d))
+    lam = np.array([0.0, 0.8, -1.7])
+    for causal in (True, False):
+        out = oracle.prefill_v1(q, k, v, lam, 0.2, causal=causal, apply_norm=False, threads=1)
+        _close(out, np.broadcast_to((1.0 - lam)[None, None, :, None], out.shape), 1e-13,
+               f"V1 rows sum to 1 - lambda (causal={causal})")
+    Hq, Hkv = 8, 4
+    q2 = r.standard_normal((B, N, Hq, d)); k2 = r.standard_normal((B, N, Hkv, d))
+    lam2 = np.array([0.5, 1.0, 0.2, -0.3])
+    out2 = oracle.prefill_v2(q2, k2, np.ones((B, N, Hkv, d)), lam2, threads=1)
+    _close(out2, np.broadcast_to((1.0 - lam2)[None, None, :, None], out2.shape), 1e-13,
+           "V2 rows sum to 1 - lambda")
+    out3 = oracle.decode_v2(q2[:, 0], k2, np.ones((B, N, Hkv, d)), lam2, kv_len=[7], threads=1)
+    _close(out3, np.broadcast_to((1.0 - lam2)[None, :, None], out3.shape), 1e-13,
+           "decode rows sum to 1 - lambda")
+
+
+def pin_norm_first_row_closed_form():
+    """Causal row 0 sees only key 0: o = (1-lambda) v0, then RMSNorm and (1 - lambda_init):
+    out_0 = (1-lambda) v0 / sqrt((1-lambda)^2 mean(v0^2) + eps) * (1 - lambda_init).
+    The second case makes mean(o^2) comparable to eps so a dropped eps shows."""
+    r = _rng(6)
+    B, N, H, d = 1, 5, 2, 8
+    q = r.standard_normal((B, N, H, 2, d)); k = r.standard_normal((B, N, H, 2, d))
+    lam = np.array([0.35, -0.6])
+    li, eps = 0.43, 1e-5
+    for vscale in (1.0, 2e-3):
+        v = r.standard_normal((B, N, H, 2 * d)) * vscale
+        out = oracle.prefill_v1(q, k, v, lam, li, apply_norm=True, eps=eps, threads=1)
+        for h in range(H):
+            v0 = v[0, 0, h]
+            o = (1 - lam[h]) * v0
+            ref = o / np.sqrt(np.mean(o * o) + eps) * (1 - li)
+            _close(out[0, 0, h], ref, 1e-13, f"first-row norm closed form (scale {vscale})")
+
+
+def pin_printed_operator_with_library_ops():
+    """(A_1 - lambda A_2) V with A_b from torch.softmax over the causal mask, then
+    torch's rms_norm and the (1 - lambda_init) factor -- for V1 with distinct branches."""
+    r = _rng(7)
+    B, N, H, d = 1, 33, 2, 8
+    q = r.standard_normal((B, N, H, 2, d)); k = r.standard_normal((B, N, H, 2, d))
+    v = r.standard_normal((B, N, H, 2 * d))
+    lam = np.array([0.7, 0.25]); li, eps = 0.6, 1e-5
+    T = torch.from_numpy
+    mask = torch.ones(N, N, dtype=torch.bool).tril()
+    ref = np.zeros((B, N, H, 2 * d))
+    for h in range(H):
+        def amap(b):
+            s = T(q[0, :, h, b]) @ T(k[0, :, h, b]).T / math.sqrt(d)
+            return torch.softmax(s.masked_fill(~mask, float("-inf")), dim=-1)
+        o = (amap(0) - lam[h] * amap(1)) @ T(v[0, :, h])
+        o = torch.nn.functional.rms_norm(o, (2 * d,), eps=eps) * (1 - li)
+        ref[0, :, h] = o.numpy()
+    out = oracle.prefill_v1(q, k, v, lam, li, apply_norm=True, eps=eps, threads=2)
+    _close(out, ref, 1e-12, "printed operator via torch ops")
+    rows = [0, 5, 32, 17]
+    out_rows = oracle.prefill_v1(q, k, v, lam, li, apply_norm=True, eps=eps, rows=rows, threads=1)
+    _close(out_rows, ref[:, rows], 1e-12, "row-sampled oracle")
+
+
+def pin_brute_force_tiny():
+    """N <= 8, d in {1, 2, 4}: 40-digit mpmath, exp and sums taken directly (no maximum
+    subtracted), weights A_1 - lambda A_2 formed explicitly."""
+    import mpmath
+    mpmath.mp.dps = 40
+    r = _rng(8)
+    for (N, d) in ((1, 1), (2, 1), (5, 2), (8, 4)):
+        B, H = 1, 1
+        q = r.standard_normal((B, N, H, 2, d)); k = r.standard_normal((B, N, H, 2, d))
+        v = r.standard_normal((B, N, H, 2 * d))
+        lam = np.array([0.77])
+        out = oracle.prefill_v1(q, k, v, lam, 0.1, apply_norm=False, threads=1)
+        for i in range(N):
+            def row(b):
+                e = [mpmath.e ** (mpmath.fsum(mpmath.mpf(q[0, i, 0, b, c]) * mpmath.mpf(k[0, j, 0, b, c])
+                                              for c in range(d)) / mpmath.sqrt(d)) for j in range(i + 1)]
+                s = mpmath.fsum(e)
+                return [x / s for x in e]
+            a1, a2 = row(0), row(1)
+            w = [a1[j] - mpmath.mpf(lam[0]) * a2[j] for j in range(i + 1)]
+            ref = [float(mpmath.fsum(w[j] * mpmath.mpf(v[0, j, 0, c]) for j in range(i + 1)))
+                   for c in range(2 * d)]
+            _close(out[0, i, 0], ref, 1e-14, f"brute force N={N} d={d} row {i}")
+
+
+# ---- noise cancellation (the pages' measurement) --------------------------------------
+
+def _snr_gains(lam, stride=37):
+    """Median SNR gain (differential over plain softmax) over query rows past the planted
+    key. SNR = weight on the signal key / mean |weight| on unrelated keys."""
+    cfg = {ln.split()[0]: ln.split()[1] for ln in open(os.path.join(GOLDEN, "snr_claim.txt"))
+           if ln.strip() and not ln.startswith("#")}
+    N = int(cfg["length"])
+    inp = synth.signal_plus_noise(N=N, Hq=8, Hkv=1, d=128, seed=5)
+    q = inp.as_f64("q")[0]; k = inp.as_f64("k")[0]
+    pos = inp.extra["planted_pos"]
+    gains, plain_mass, diff_mass = [], [], []
+    for p in range(4):
+        s = int(pos[0, p])
+        for i in range(s + 1, N, stride):
+            a1, a2 = oracle.map_row_v2(q, k, p, i)
+            w = a1 - lam * a2
+            n = i  # unrelated keys visible to row i
+            plain = a1[s] / ((a1.sum() - a1[s]) / n)
+            diff = w[s] / ((np.abs(w).sum() - abs(w[s])) / n)
+            gains.append(diff / plain)
+            plain_mass.append(a1.sum() - a1[s])
+            diff_mass.append(w.sum() - w[s])
+    return float(np.median(gains)), float(np.mean(plain_mass)), float(np.mean(diff_mass)), cfg
+
+
+def pin_noise_cancellation():
+    g0, plain_mass, _, cfg = _snr_gains(0.0)
+    assert abs(g0 - 1.0) < 1e-12, "lambda = 0 must be plain softmax"
+    assert plain_mass > 0.5, f"plain softmax noise mass {plain_mass:.3f} should be O(1)"
+    lam = float(cfg["lambda"])
+    g, _, diff_mass, _ = _snr_gains(lam)
+    assert float(cfg["gain_min"]) <= g <= float(cfg["gain_max"]), f"SNR gain {g:.2f} outside claim"
+    assert abs(diff_mass) < 0.25 * plain_mass, (
+        f"differential noise mass {diff_mass:.3f} not well below plain {plain_mass:.3f}")
+    sweep = [_snr_gains(x)[0] for x in (0.0, 0.5, 0.8, 0.9)]
+    assert all(b > a for a, b in zip(sweep, sweep[1:])), f"lambda ablation not rising: {sweep}"
+
+
+ALL_PINS = [
+    pin_lambda_init_schedule,
+    pin_lambda_closed_form,
+    pin_lambda0_is_softmax_attention_v1,
+    pin_lambda0_is_softmax_attention_v2,
+    pin_lambda0_decode_is_softmax_attention,
+    pin_identical_branches_cancel,
+    pin_rows_sum_to_one_minus_lambda,
+    pin_norm_first_row_closed_form,
+    pin_printed_operator_with_library_ops,
+    pin_brute_force_tiny,
+    pin_noise_cancellation,
+]
