@@ -1,0 +1,223 @@
+// api.cu -- the C ABI (include/diffattn.h): host-side validation and dispatch.
+// Nothing is launched unless every argument passes; no entry point allocates memory.
+#include <math.h>
+#include <string.h>
+
+#include "../../include/diffattn.h"
+#include "kernels.h"
+
+using namespace diffattn;
+
+namespace {
+
+constexpr int kAbiVersion = 100;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return DIFFATTN_OK;
+  if (e == cudaErrorNotSupported) return DIFFATTN_ERR_UNSUPPORTED;
+  return DIFFATTN_ERR_CUDA;
+}
+
+// Largest element offset reachable through strides s for extents n (all >= 1).
+inline bool strides_ok(const int64_t* s, int n) {
+  for (int i = 0; i < n; ++i)
+    if (s[i] < 0) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int diffattn_version(void) { return kAbiVersion; }
+
+const char* diffattn_status_string(int status) {
+  switch (status) {
+    case DIFFATTN_OK: return "ok";
+    case DIFFATTN_ERR_INVALID_ARG: return "invalid argument";
+    case DIFFATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DIFFATTN_ERR_MISALIGNED: return "misaligned pointer or stride";
+    case DIFFATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case DIFFATTN_ERR_CUDA: return "CUDA error";
+    case DIFFATTN_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int diffattn_lambda(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
+                    int n_heads, int dim, int depth, float* lambda_out, float* lambda_init_out,
+                    void* stream) {
+  if (!lq1 || !lk1 || !lq2 || !lk2 || !lambda_out) return DIFFATTN_ERR_INVALID_ARG;
+  if (n_heads < 1 || n_heads > 65535 || dim < 1 || dim > 4096 || depth < 1)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(lq1) || !aligned16(lk1) || !aligned16(lq2) || !aligned16(lk2))
+    return DIFFATTN_ERR_MISALIGNED;
+  return from_cuda(launch_lambda(lq1, lk1, lq2, lk2, n_heads, dim, depth, lambda_out,
+                                 lambda_init_out, static_cast<cudaStream_t>(stream)));
+}
+
+int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const void* k,
+                         const void* v, const float* lambda, const float* lambda_init, void* out,
+                         int* dev_status, void* stream) {
+  if (!p) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->seqlen < 0 || p->head_dim < 1) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->variant != DIFFATTN_V1 && p->variant != DIFFATTN_V2) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->dtype != DIFFATTN_F32 && p->dtype != DIFFATTN_BF16) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->causal != 0 && p->causal != 1) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->apply_norm != 0 && p->apply_norm != 1) return DIFFATTN_ERR_INVALID_ARG;
+  if (!strides_ok(p->q_strides, 3) || !strides_ok(p->k_strides, 3) ||
+      !strides_ok(p->v_strides, 3) || !strides_ok(p->o_strides, 3))
+    return DIFFATTN_ERR_INVALID_ARG;
+
+  PrefillArgs a;
+  memset(&a, 0, sizeof(a));
+  a.variant = p->variant;
+  a.B = p->batch;
+  a.N = p->seqlen;
+  a.d = p->head_dim;
+  a.causal = p->causal;
+  a.apply_norm = p->apply_norm;
+  a.eps = p->norm_eps;
+  if (p->variant == DIFFATTN_V1) {
+    if (p->n_q_heads < 1 || p->n_kv_heads != p->n_q_heads) return DIFFATTN_ERR_INVALID_ARG;
+    a.units = p->n_q_heads;
+    a.Hq = a.Hkv = p->n_q_heads;
+    a.group = 1;
+    a.dv = 2 * a.d;
+  } else {
+    if (p->n_q_heads < 2 || p->n_kv_heads < 1 || p->n_q_heads % p->n_kv_heads != 0 ||
+        (p->n_q_heads / p->n_kv_heads) % 2 != 0)
+      return DIFFATTN_ERR_INVALID_ARG;
+    if (p->apply_norm) return DIFFATTN_ERR_INVALID_ARG;  // V2 has no per-head norm
+    a.units = p->n_q_heads / 2;
+    a.Hq = p->n_q_heads;
+    a.Hkv = p->n_kv_heads;
+    a.group = p->n_q_heads / p->n_kv_heads;
+    a.dv = a.d;
+  }
+  if (a.apply_norm && !(p->norm_eps >= 0.f && isfinite(p->norm_eps))) return DIFFATTN_ERR_INVALID_ARG;
+  if (a.units > 65535 || a.B > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  if (a.B == 0 || a.N == 0) return DIFFATTN_OK;
+  if (!q || !k || !v || !lambda || !out) return DIFFATTN_ERR_INVALID_ARG;
+  if (a.apply_norm && !lambda_init) return DIFFATTN_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return DIFFATTN_ERR_MISALIGNED;
+  const int vec = p->dtype == DIFFATTN_BF16 ? 8 : 4;  // elements per 16 bytes
+  for (int i = 0; i < 3; ++i) {
+    if (p->q_strides[i] % vec || p->k_strides[i] % vec || p->v_strides[i] % vec ||
+        p->o_strides[i] % vec)
+      return DIFFATTN_ERR_MISALIGNED;
+  }
+  memcpy(a.qs, p->q_strides, sizeof(a.qs));
+  memcpy(a.ks, p->k_strides, sizeof(a.ks));
+  memcpy(a.vs, p->v_strides, sizeof(a.vs));
+  memcpy(a.os, p->o_strides, sizeof(a.os));
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.lambda = lambda;
+  a.lambda_init = lambda_init;
+  a.out = out;
+  a.dev_status = dev_status;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  if (p->dtype == DIFFATTN_F32) {
+    if (a.d > 128 || a.d % 4 != 0) return DIFFATTN_ERR_UNSUPPORTED;
+    return from_cuda(launch_prefill_f32(a, s));
+  }
+  // bf16: tcgen05 kernel (V1: d = 64; V2: d = 128)
+  if (p->variant == DIFFATTN_V1 && a.d != 64) return DIFFATTN_ERR_UNSUPPORTED;
+  if (p->variant == DIFFATTN_V2 && a.d != 128) return DIFFATTN_ERR_UNSUPPORTED;
+  if (a.N > (1 << 24)) return DIFFATTN_ERR_UNSUPPORTED;
+  return from_cuda(launch_prefill_tc(a, s));
+}
+
+static int decode_check(const diffattn_decode_params* p, int* splits, int* split_len) {
+  if (!p) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->max_kv_len < 0 || p->n_q_heads < 1 || p->n_kv_heads < 1 ||
+      p->head_dim < 1 || p->num_splits < 0)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (p->variant != DIFFATTN_V2) return p->variant == DIFFATTN_V1 ? DIFFATTN_ERR_UNSUPPORTED
+                                                                  : DIFFATTN_ERR_INVALID_ARG;
+  if (p->dtype != DIFFATTN_BF16) return p->dtype == DIFFATTN_F32 ? DIFFATTN_ERR_UNSUPPORTED
+                                                                 : DIFFATTN_ERR_INVALID_ARG;
+  if (p->n_q_heads % p->n_kv_heads != 0 || (p->n_q_heads / p->n_kv_heads) % 2 != 0)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (p->n_q_heads / p->n_kv_heads != 8 || p->head_dim != 128) return DIFFATTN_ERR_UNSUPPORTED;
+  if (!strides_ok(p->q_strides, 2) || !strides_ok(p->kv_strides, 3) || !strides_ok(p->o_strides, 2))
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (p->batch > 65535 || p->n_kv_heads > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  int s = p->num_splits ? p->num_splits : decode_default_splits(p->batch, p->max_kv_len, p->n_kv_heads);
+  const int L = p->max_kv_len;
+  int len = (L + s - 1) / (s > 0 ? s : 1);
+  len = ((len + kDecodeChunk - 1) / kDecodeChunk) * kDecodeChunk;
+  if (len < kDecodeChunk) len = kDecodeChunk;
+  s = (L + len - 1) / len;
+  if (s < 1) s = 1;
+  if (s > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  *splits = s;
+  *split_len = len;
+  return DIFFATTN_OK;
+}
+
+static size_t decode_ws_bytes(const diffattn_decode_params* p, int splits) {
+  const size_t recs = (size_t)p->batch * p->n_q_heads * splits;
+  const size_t o_bytes = ((recs * p->head_dim * sizeof(float)) + 255) & ~(size_t)255;
+  return o_bytes + recs * 2 * sizeof(float);
+}
+
+int diffattn_decode_workspace_size(const diffattn_decode_params* p, size_t* bytes) {
+  if (!bytes) return DIFFATTN_ERR_INVALID_ARG;
+  int splits = 0, len = 0;
+  int rc = decode_check(p, &splits, &len);
+  if (rc != DIFFATTN_OK) return rc;
+  *bytes = decode_ws_bytes(p, splits);
+  return DIFFATTN_OK;
+}
+
+int diffattn_fwd_decode(const diffattn_decode_params* p, const void* q, const void* k_cache,
+                        const void* v_cache, const int32_t* kv_len, const float* lambda, void* out,
+                        void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  int splits = 0, len = 0;
+  int rc = decode_check(p, &splits, &len);
+  if (rc != DIFFATTN_OK) return rc;
+  if (p->batch == 0) return DIFFATTN_OK;
+  if (!q || !k_cache || !v_cache || !lambda || !out) return DIFFATTN_ERR_INVALID_ARG;
+  const size_t need = decode_ws_bytes(p, splits);
+  if (!workspace || workspace_bytes < need) return DIFFATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIFFATTN_ERR_MISALIGNED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return DIFFATTN_ERR_MISALIGNED;
+  if (p->q_strides[0] % 8 || p->q_strides[1] % 8 || p->kv_strides[0] % 8 || p->kv_strides[1] % 8 ||
+      p->kv_strides[2] % 8 || p->o_strides[0] % 8 || p->o_strides[1] % 8)
+    return DIFFATTN_ERR_MISALIGNED;
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = p->batch;
+  a.L = p->max_kv_len;
+  a.Hq = p->n_q_heads;
+  a.Hkv = p->n_kv_heads;
+  a.d = p->head_dim;
+  a.splits = splits;
+  a.split_len = len;
+  memcpy(a.qs, p->q_strides, sizeof(a.qs));
+  memcpy(a.kvs, p->kv_strides, sizeof(a.kvs));
+  memcpy(a.os, p->o_strides, sizeof(a.os));
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.kv_len = kv_len;
+  a.lambda = lambda;
+  a.out = out;
+  const size_t recs = (size_t)a.B * a.Hq * splits;
+  a.ws_o = static_cast<float*>(workspace);
+  a.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                     (((recs * a.d * sizeof(float)) + 255) & ~(size_t)255));
+  a.dev_status = dev_status;
+  return from_cuda(launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,59 @@
+// kernels.h -- internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace diffattn {
+
+// Resolved prefill problem (validated by the API layer).
+struct PrefillArgs {
+  int variant;       // DIFFATTN_V1 / DIFFATTN_V2
+  int B, N;
+  int units;         // V1 heads / V2 pairs
+  int Hq, Hkv;       // head counts as given
+  int group;         // V2: Hq / Hkv (query heads per KV head); V1: 1
+  int d, dv;         // branch width, value width
+  int causal, apply_norm;
+  float eps;
+  int64_t qs[3], ks[3], vs[3], os[3];  // element strides {batch, token, head}
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* lambda;
+  const float* lambda_init;
+  void* out;
+  int* dev_status;
+};
+
+struct DecodeArgs {
+  int B, L, Hq, Hkv, d;
+  int splits, split_len;  // keys per split (multiple of the chunk size)
+  int64_t qs[2], kvs[3], os[2];
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* kv_len;
+  const float* lambda;
+  void* out;
+  float* ws_o;   // [B, Hq, splits, d]
+  float* ws_ml;  // [B, Hq, splits, 2]
+  int* dev_status;
+};
+
+cudaError_t launch_lambda(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
+                          int n_heads, int dim, int depth, float* lam, float* lam_init,
+                          cudaStream_t stream);
+
+cudaError_t launch_prefill_f32(const PrefillArgs& a, cudaStream_t stream);
+
+// tcgen05 bf16 prefill; returns cudaErrorNotSupported for shapes it does not handle.
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream);
+
+// split-KV decode (V2, bf16, d = 128, 8 query heads per KV head)
+constexpr int kDecodeChunk = 64;  // keys per pipeline stage
+int decode_default_splits(int B, int L, int Hkv);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+}  // namespace diffattn

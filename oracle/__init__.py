@@ -85,7 +85,10 @@ def _load():
 
 
 def _f64(a) -> np.ndarray:
-    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        raise TypeError("bf16 bit patterns must be converted to values before the oracle sees them")
+    return np.ascontiguousarray(a, dtype=np.float64)
 
 
 def _dp(a: np.ndarray):

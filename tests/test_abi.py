@@ -1,0 +1,152 @@
+"""The C-ABI library (no GPU needed): it loads, exports every entry point the header
+declares, and rejects bad arguments on the host before launching anything. No call here
+reaches a kernel launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import differential_attention_05_b200 as da
+from differential_attention_05_b200 import _binding as B
+from differential_attention_05_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "diffattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return da.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w[\w\s\*]*?\b(diffattn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    assert set(declared_functions()) == set(B.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} missing from {da.library_path()}"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.diffattn_version() == 100
+    for code in range(-6, 1):
+        assert da.diffattn_status_string(code)
+    assert da.diffattn_status_string(-99) == "unknown status"
+
+
+def _prefill_params(**kw):
+    p = B.PrefillParams()
+    p.variant, p.dtype, p.batch, p.seqlen = B.DIFFATTN_V2, B.DIFFATTN_BF16, 1, 256
+    p.n_q_heads, p.n_kv_heads, p.head_dim = 16, 2, 128
+    p.causal, p.apply_norm, p.norm_eps = 1, 0, 1e-5
+    N = p.seqlen
+    p.q_strides[:] = (N * 16 * 128, 16 * 128, 128)
+    p.k_strides[:] = (N * 2 * 128, 2 * 128, 128)
+    p.v_strides[:] = (N * 2 * 128, 2 * 128, 128)
+    p.o_strides[:] = (N * 8 * 128, 8 * 128, 128)
+    for k_, v_ in kw.items():
+        setattr(p, k_, v_)
+    return p
+
+
+GOOD = 1 << 20  # a 16-byte-aligned stand-in address; validation never dereferences it
+
+
+def _call_prefill(lib, p, q=GOOD, k=GOOD + 4096, v=GOOD + 8192, lam=GOOD + 12288, li=None,
+                  out=GOOD + 16384):
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.diffattn_fwd_prefill(ctypes.byref(p), vp(q), vp(k), vp(v), vp(lam), vp(li), vp(out),
+                                    None, None)
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("variant", 3, -1), ("dtype", 7, -1), ("batch", -1, -1), ("seqlen", -5, -1),
+    ("n_kv_heads", 3, -1),    # 16 % 3 != 0
+    ("n_kv_heads", 16, -1),   # group of 1 cannot hold a pair
+    ("apply_norm", 1, -1),    # V2 has no per-head norm
+    ("causal", 2, -1),
+    ("head_dim", 96, -2),     # bf16 V2 needs d = 128
+])
+def test_prefill_rejects(lib, field, value, code):
+    assert _call_prefill(lib, _prefill_params(**{field: value})) == code
+
+
+def test_prefill_rejects_null_and_alias_and_misalignment(lib):
+    p = _prefill_params()
+    assert lib.diffattn_fwd_prefill(None, None, None, None, None, None, None, None, None) == -1
+    assert _call_prefill(lib, p, q=None) == -1
+    assert _call_prefill(lib, p, out=GOOD) == -1                 # out aliases q
+    assert _call_prefill(lib, p, k=GOOD + 4098) == -3            # not 16-byte aligned
+    p2 = _prefill_params()
+    p2.q_strides[1] = 16 * 128 + 4                               # token stride not 16 B multiple
+    assert _call_prefill(lib, p2) == -3
+
+
+def test_prefill_empty_problem_launches_nothing(lib):
+    assert _call_prefill(lib, _prefill_params(batch=0), q=None, k=None, v=None, out=None) == 0
+    assert _call_prefill(lib, _prefill_params(seqlen=0), q=None, k=None, v=None, out=None) == 0
+
+
+def test_v1_requires_lambda_init_when_normalising(lib):
+    p = _prefill_params(variant=B.DIFFATTN_V1, n_q_heads=4, n_kv_heads=4, head_dim=64, apply_norm=1)
+    assert _call_prefill(lib, p, li=None) == -1
+
+
+def _decode_params(B_=4, L=1000, Hq=64, Hkv=8, d=128, splits=0):
+    p = B.DecodeParams()
+    p.variant, p.dtype = B.DIFFATTN_V2, B.DIFFATTN_BF16
+    p.batch, p.max_kv_len, p.n_q_heads, p.n_kv_heads, p.head_dim, p.num_splits = B_, L, Hq, Hkv, d, splits
+    p.q_strides[:] = (Hq * d, d)
+    p.kv_strides[:] = (L * Hkv * d, Hkv * d, d)
+    p.o_strides[:] = (Hq // 2 * d, d)
+    return p
+
+
+def test_decode_workspace_size(lib):
+    n = ctypes.c_size_t(0)
+    p = _decode_params(B_=4, L=1000, splits=3)
+    assert lib.diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    # 3 splits of 384 keys (rounded up to the 64-key chunk): 4 * 64 heads * 3 records
+    recs = 4 * 64 * 3
+    assert n.value == ((recs * 128 * 4 + 255) // 256) * 256 + recs * 2 * 4
+    p = _decode_params(Hq=64, Hkv=16)  # group of 4: not this build's decode shape
+    assert lib.diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == -2
+    p = _decode_params()
+    p.variant = B.DIFFATTN_V1
+    assert lib.diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == -2
+
+
+def test_decode_rejects_small_workspace(lib):
+    p = _decode_params(B_=2, L=512)
+    n = ctypes.c_size_t(0)
+    assert lib.diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    vp = ctypes.c_void_p
+    args = [vp(GOOD), vp(GOOD + 4096), vp(GOOD + 8192), None, vp(GOOD + 12288), vp(GOOD + 16384)]
+    assert lib.diffattn_fwd_decode(ctypes.byref(p), *args, vp(GOOD * 4), n.value - 1, None, None) == -4
+    assert lib.diffattn_fwd_decode(ctypes.byref(p), *args, None, n.value, None, None) == -4
+    assert lib.diffattn_fwd_decode(ctypes.byref(p), *args, vp(GOOD * 4 + 16), n.value, None, None) == -3
+
+
+def test_lambda_rejects(lib):
+    vp = ctypes.c_void_p
+    f = lib.diffattn_lambda
+    assert f(None, vp(GOOD), vp(GOOD), vp(GOOD), 4, 64, 1, vp(GOOD), None, None) == -1
+    assert f(vp(GOOD), vp(GOOD), vp(GOOD), vp(GOOD), 0, 64, 1, vp(GOOD), None, None) == -1
+    assert f(vp(GOOD), vp(GOOD), vp(GOOD), vp(GOOD), 4, 64, 0, vp(GOOD), None, None) == -1
+    assert f(vp(GOOD + 4), vp(GOOD), vp(GOOD), vp(GOOD), 4, 64, 1, vp(GOOD), None, None) == -3
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setenv("DIFFATTN_LIBRARY", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(B, "_lib", None)
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        B.load_library()
