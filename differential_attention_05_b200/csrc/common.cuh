@@ -16,11 +16,17 @@ namespace diffattn {
 
 // ---- status --------------------------------------------------------------------------
 
-// Spin bound for every mbarrier / flag wait (try_wait iterations, each of which may
-// suspend for a hardware-chosen interval). Around a second or more at 1.9 GHz.
-#ifndef DIFFATTN_WAIT_LIMIT
-#define DIFFATTN_WAIT_LIMIT (1u << 26)
+// Time bound for every mbarrier / flag wait, in nanoseconds of %globaltimer. No wait in
+// these kernels legitimately lasts more than a few milliseconds.
+#ifndef DIFFATTN_WAIT_NS
+#define DIFFATTN_WAIT_NS 2000000000ull
 #endif
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ void report_status(int* dev_status, int code) {
   if (dev_status) atomicCAS(dev_status, 0, code);
@@ -94,14 +100,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
 }
 
 // Bounded wait for the barrier phase with parity `phase` to complete. Returns false if
-// the bound ran out or *abort was raised by another thread (then the caller stops).
+// the time bound ran out (then it raises *abort) or *abort was raised by another thread;
+// the caller then stops issuing work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, volatile int* abort) {
-  for (uint32_t it = 0; it < DIFFATTN_WAIT_LIMIT; ++it) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, phase)) return true;
-    if ((it & 63u) == 63u && *abort) return false;
+    if ((it & 31u) == 0) {
+      if (*abort) return false;
+      if (global_ns() - t0 > DIFFATTN_WAIT_NS) {
+        *abort = 1;
+        return false;
+      }
+    }
   }
-  *abort = 1;
-  return false;
+}
+
+// Bounded wait that ignores the abort flag: used to drain copies / MMAs already in
+// flight before a CTA gives back its shared memory and TMEM.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t phase) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, phase)) return true;
+    if ((it & 31u) == 31u && global_ns() - t0 > DIFFATTN_WAIT_NS) return false;
+  }
 }
 
 // ---- cp.async (16-byte, zero-fill when src_bytes == 0) --------------------------------

@@ -152,10 +152,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (*abort_flag) {
         // let the copies already in flight land before the CTA's shared memory goes away
+        mbar_wait_drain(&ms.q_full, 0);
         for (int j = max(0, issued_k - KSTAGES); j < issued_k; ++j)
-          mbar_wait(&ms.k_full[j % KSTAGES], (j / KSTAGES) & 1, abort_flag), (void)0;
+          mbar_wait_drain(&ms.k_full[j % KSTAGES], (j / KSTAGES) & 1);
         for (int j = max(0, issued_v - VSTAGES); j < issued_v; ++j)
-          mbar_wait(&ms.v_full[j % VSTAGES], (j / VSTAGES) & 1, abort_flag), (void)0;
+          mbar_wait_drain(&ms.v_full[j % VSTAGES], (j / VSTAGES) & 1);
       }
     }
   } else if (warp == 9) {
@@ -248,7 +249,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
 
     for (int j = 0; j < n_kt; ++j) {
-      if (!(ok = mbar_wait(&ms.s_full[br], j & 1, abort_flag))) break;
+      ok = mbar_wait(&ms.s_full[br], j & 1, abort_flag);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;  // tcgen05.ld/st below are warp-wide
       tc_fence_after();
       float s[BN];
 #pragma unroll
@@ -270,24 +272,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       float mx = -INFINITY;
 #pragma unroll
       for (int e = 0; e < BN; ++e) mx = fmaxf(mx, s[e]);
-      if (mx > m + RESCALE_LOG2 || m == -INFINITY) {
-        const float mn = fmaxf(mx, m);
-        if (j > 0 && m != -INFINITY) {
-          const float alpha = ex2(m - mn);
-          l *= alpha;
-          // O_br row *= alpha (its last P.V MMA completed before S_br(j) did)
+      // raise the running max only when it grew by more than 2^8 (or was unset); the
+      // decision is per row, the O rescale below is done by the whole warp when any of
+      // its rows needs it (rows that do not use alpha = 1)
+      const bool raise = (mx > m + RESCALE_LOG2) || (m == -INFINITY);
+      const float mn = raise ? fmaxf(mx, m) : m;
+      const float alpha = (raise && m != -INFINITY) ? ex2(m - mn) : 1.f;
+      if (__any_sync(0xffffffffu, raise && m != -INFINITY)) {
+        // O_br row *= alpha (its last P.V MMA completed before S_br(j) did)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(o_col + c * 32, r);
-            tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(o_col + c * 32, r);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(o_col + c * 32, r);
-          }
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(o_col + c * 32, r);
         }
-        m = mn;
       }
+      l *= alpha;
+      m = mn;
       const float mref = (m == -INFINITY) ? 0.f : m;  // fully masked row: all p = 0
       float ps = 0.f;
 #pragma unroll
@@ -310,6 +314,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     // ------------------------------- epilogue ----------------------------------------
     if (ok) ok = mbar_wait(&ms.o_full, 0, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
     ms.l_x[br][row] = l;
     named_bar_sync(1, 256);
     if (ok) {
@@ -363,9 +368,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 9) {
     if (*abort_flag) {
       // wait (bounded) for any MMA still in flight before giving TMEM back
-      uint32_t it = 0;
-      while (!mbar_try_wait(&ms.o_full, 0) && ++it < DIFFATTN_WAIT_LIMIT) {
-      }
+      mbar_wait_drain(&ms.o_full, 0);
       if (threadIdx.x == 9 * 32) report_status(a.dev_status, DIFFATTN_ERR_TIMEOUT);
     }
     tc_fence_after();
