@@ -1,0 +1,557 @@
+#!/usr/bin/env python
+"""Benchmark of the differential attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload c2|c3|c4|c5] [--no-secondary]
+
+A step is one pass of the hot path over one batch of synthetic input: the on-device
+lambda re-parameterisation followed by the fused prefill (or the split-KV decode for the
+decode workload). Default workload: the V1 bf16 layer (B=2, 16 heads, N=4096, d=64).
+Inputs are the seeded synthetic tensors of differential_attention_05_b200.synth.
+
+Timing: W untimed warm-up steps, then K steps between a barrier + synchronize on both
+sides; every step is bracketed by CUDA events on the launching stream and L2 is flushed
+(256 MB write) between steps when the inputs fit in L2. The maximum over ranks is taken.
+Rank 0 prints one JSON line.
+
+--impl reference times the float64 CPU oracle (the checker the kernels are held to) on
+the host cores, on a bounded sample of the same workload, and prints the same line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------------------
+# workloads and their algorithmic work
+
+def workload_inputs(name: str):
+    from differential_attention_05_b200 import synth
+    return {"c2": synth.config2, "c3": synth.config3, "c4": synth.config4, "c5": synth.config5}[name]()
+
+
+def prefill_flops(inp) -> float:
+    """Algorithmic FLOPs: per causal (i, j) pair, 12 d per V1 head (two d-wide QK^T dot
+    products and two 2d-wide P.V rows, 2 flops per multiply-add) and 4 d per V2 query
+    head; masked pairs, exp and the norm are not counted."""
+    pairs = inp.N * (inp.N + 1) / 2 if inp.causal else float(inp.N) * inp.N
+    per = 12 * inp.d * inp.H if inp.variant == 1 else 4 * inp.d * inp.H
+    return float(inp.B) * pairs * per
+
+
+def decode_bytes(B, L, Hkv, d) -> float:
+    """Algorithmic bytes: the K and V caches read once (bf16)."""
+    return float(B) * L * Hkv * d * 2 * 2
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        self.out.flush()
+        try:
+            lines = open(self.out.name).read().strip().splitlines()
+        except OSError:
+            lines = []
+        os.unlink(self.out.name)
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------
+# the GPU arm
+
+def run_ours(args, rank, world, device):
+    import torch
+
+    import differential_attention_05_b200 as da
+
+    torch.cuda.set_device(device)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+    peaks = load_peaks()
+    inp = workload_inputs(args.workload)
+
+    def dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    q, k, v = dev(inp.q), dev(inp.k), dev(inp.v)
+    vecs = [dev(getattr(inp, n)) for n in ("lq1", "lk1", "lq2", "lk2")]
+    lam = torch.empty(inp.n_units, dtype=torch.float32, device=device)
+    li = torch.empty(1, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    decode = inp.mode == "decode"
+    if decode:
+        out = torch.empty((inp.B, inp.H // 2, inp.d), dtype=torch.bfloat16, device=device)
+        p = da._binding.decode_params(q, k, v, out)
+        ws = torch.empty(da._binding.diffattn_decode_workspace_size(p), dtype=torch.uint8,
+                         device=device)
+        work = decode_bytes(inp.B, inp.N, inp.Hkv, inp.d)
+        unit, metric = "GB/s", "diff-attn decode KV GB/s at 1 B200"
+    else:
+        out = (torch.empty((inp.B, inp.N, inp.H, 2 * inp.d), dtype=torch.bfloat16, device=device)
+               if inp.variant == 1 else
+               torch.empty((inp.B, inp.N, inp.H // 2, inp.d), dtype=torch.bfloat16, device=device))
+        work = prefill_flops(inp)
+        unit, metric = "TFLOP/s", "diff-attn prefill TFLOP/s (% bf16 peak)"
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    flush = in_bytes < 2 * L2_BYTES
+    scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device) if flush else None
+
+    def lambda_step():
+        da.diffattn_lambda(*vecs, depth=inp.depth, lambda_out=lam, lambda_init_out=li)
+
+    def main_kernel():
+        if decode:
+            da.diffattn_fwd_decode(q, k, v, lam, out=out, workspace=ws)
+        else:
+            da.diffattn_fwd_prefill(q, k, v, lam, li, out=out, causal=inp.causal,
+                                    apply_norm=inp.apply_norm, norm_eps=inp.eps)
+
+    launches_per_step = 1 + (2 if decode else 1)
+
+    for _ in range(args.warmup):
+        lambda_step()
+        main_kernel()
+        if flush:
+            scratch.zero_()
+    torch.cuda.synchronize(device)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            lambda_step()
+            ev[i][1].record(stream)
+            main_kernel()
+            ev[i][2].record(stream)
+            if flush:
+                scratch.zero_()  # outside the timed events
+        torch.cuda.synchronize(device)
+        if dist is not None:
+            dist.barrier()
+        t_wall = time.perf_counter() - t_wall
+        time.sleep(0.25)
+    clocks = clk.summary()
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    kern_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = float(sum(step_ms))
+    kern_avg = float(sum(kern_ms) / len(kern_ms))
+    if dist is not None:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    if decode:
+        value = world * work * args.steps / (total_ms * 1e-3) / 1e9
+        achieved = work / (kern_avg * 1e-3) / 1e9
+        peak, bound, runit = peaks["hbm_gbs"], "hbm", "GB/s"
+    else:
+        value = world * work * args.steps / (total_ms * 1e-3) / 1e12
+        achieved = work / (kern_avg * 1e-3) / 1e12
+        peak, bound, runit = peaks["bf16_tflops"], "tensor", "TFLOP/s"
+
+    # end to end through the public API: pinned host inputs -> device, hot path, result -> host
+    host_in = [torch.from_numpy(inp.q.view(np.int16) if inp.q.dtype == np.uint16 else inp.q).pin_memory(),
+               torch.from_numpy(inp.k.view(np.int16) if inp.k.dtype == np.uint16 else inp.k).pin_memory(),
+               torch.from_numpy(inp.v.view(np.int16) if inp.v.dtype == np.uint16 else inp.v).pin_memory()]
+    host_vec = [torch.from_numpy(np.ascontiguousarray(getattr(inp, n))).pin_memory()
+                for n in ("lq1", "lk1", "lq2", "lk2")]
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in + host_vec)
+    d2h = host_out.numel() * host_out.element_size()
+    e2e_steps = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        for src, dst in zip(host_in, (q, k, v)):
+            dst.view(src.dtype).copy_(src, non_blocking=True)
+        for src, dst in zip(host_vec, vecs):
+            dst.copy_(src, non_blocking=True)
+        lambda_step()
+        main_kernel()
+        host_out.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_val = world * work * e2e_steps / (e2e_ms * 1e-3) / (1e9 if decode else 1e12)
+
+    line = {
+        "metric": metric,
+        "value": round(value, 3),
+        "unit": unit,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded numpy PCG64, bf16-rounded; shapes and distributions of the workload)",
+        "config": {
+            "workload": inp.name,
+            "batch": inp.B, "seq_len": inp.N, "heads": inp.H, "kv_heads": inp.Hkv,
+            "head_dim": inp.d, "causal": bool(inp.causal), "depth": inp.depth,
+            "tokens_per_step": inp.B * (1 if decode else inp.N),
+            "l2": ("flushed between steps (256 MB write, outside the timed events)" if flush
+                   else "inputs larger than L2"),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "tokens_per_s": round(world * inp.B * (1 if decode else inp.N) * args.steps / (total_ms * 1e-3), 1),
+        "roofline": {
+            "bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": runit,
+            "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": f"{peaks['source']} ({'burst bf16' if bound == 'tensor' else 'HBM copy'})",
+            "kernel": "decode_split_kernel + decode_combine_kernel" if decode else "prefill_tc_kernel",
+            "avg_kernel_ms": round(kern_avg, 5),
+        },
+        "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "wall_s_timed": round(t_wall, 4),
+    }
+    del q, k, v, out
+    torch.cuda.empty_cache()
+    if not args.no_secondary and not decode and args.workload == "c2":
+        line["secondary"] = secondary(device, peaks, torch, da)
+    return line
+
+
+def secondary(device, peaks, torch, da):
+    """Other rows of the hot path, timed alone: V2 prefill (64/8 heads, d=128, N=16384)
+    and V2 decode (batch 64, cache 32768). Inputs are drawn on the device (seeded N(0,1),
+    same shapes) to keep the run short; both exceed L2."""
+    res = {}
+    g = torch.Generator(device=device)
+    g.manual_seed(1002)
+    N, Hq, Hkv, d = 16384, 64, 8, 128
+    q = torch.randn((1, N, Hq, d), generator=g, device=device).bfloat16()
+    k = torch.randn((1, N, Hkv, d), generator=g, device=device).bfloat16()
+    v = torch.randn((1, N, Hkv, d), generator=g, device=device).bfloat16()
+    lam = torch.full((Hq // 2,), 0.8, dtype=torch.float32, device=device)
+    out = torch.empty((1, N, Hq // 2, d), dtype=torch.bfloat16, device=device)
+    for _ in range(3):
+        da.diffattn_fwd_prefill(q, k, v, lam, out=out)
+    es = [(torch.cuda.Event(True), torch.cuda.Event(True)) for _ in range(10)]
+    for a, b in es:
+        a.record()
+        da.diffattn_fwd_prefill(q, k, v, lam, out=out)
+        b.record()
+    torch.cuda.synchronize(device)
+    ms = statistics.median(a.elapsed_time(b) for a, b in es)
+    fl = 4.0 * d * Hq * N * (N + 1) / 2
+    res["v2_prefill"] = {"workload": "v2_bf16_prefill_b1_n16384_hq64_hkv8_d128", "ms": round(ms, 4),
+                         "TFLOP/s": round(fl / ms / 1e9, 2),
+                         "frac_of_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
+    del q, k, v, out
+    B, L = 64, 32768
+    q = torch.randn((B, Hq, d), generator=g, device=device).bfloat16()
+    k = torch.randn((B, L, Hkv, d), generator=g, device=device).bfloat16()
+    v = torch.randn((B, L, Hkv, d), generator=g, device=device).bfloat16()
+    out = torch.empty((B, Hq // 2, d), dtype=torch.bfloat16, device=device)
+    p = da._binding.decode_params(q, k, v, out)
+    ws = torch.empty(da._binding.diffattn_decode_workspace_size(p), dtype=torch.uint8, device=device)
+    for _ in range(3):
+        da.diffattn_fwd_decode(q, k, v, lam, out=out, workspace=ws)
+    es = [(torch.cuda.Event(True), torch.cuda.Event(True)) for _ in range(10)]
+    for a, b in es:
+        a.record()
+        da.diffattn_fwd_decode(q, k, v, lam, out=out, workspace=ws)
+        b.record()
+    torch.cuda.synchronize(device)
+    ms = statistics.median(a.elapsed_time(b) for a, b in es)
+    by = decode_bytes(B, L, Hkv, d)
+    res["decode"] = {"workload": "v2_bf16_decode_b64_l32768_hq64_hkv8_d128", "ms": round(ms, 4),
+                     "GB/s": round(by / ms / 1e6, 1),
+                     "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    del q, k, v, out, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------------------------------
+# the oracle, timed on the host cores (cpu_baseline and the reference arm)
+
+class OracleRows:
+    """The oracle on chosen query rows of a prefill workload; inputs converted to float64
+    once, the oracle call itself is what gets timed."""
+
+    def __init__(self, inp):
+        import oracle
+        from differential_attention_05_b200 import synth
+        self.inp = inp
+        self.lam = oracle.lambda_(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.depth)
+        self.li = oracle.lambda_init(inp.depth)
+        self.k, self.v = inp.as_f64("k"), inp.as_f64("v")
+        self._q = (lambda rows: synth.bf16_to_f32(inp.q[:, rows]).astype(np.float64)) \
+            if inp.q.dtype == np.uint16 else (lambda rows: inp.q[:, rows].astype(np.float64))
+        self.units = inp.B * (inp.H if inp.variant == 1 else inp.H // 2)
+        self.per_pair = 12 * inp.d if inp.variant == 1 else 8 * inp.d  # flops per (i, j) per unit
+
+    def flops(self, rows):
+        inp = self.inp
+        return float(sum((r + 1) if inp.causal else inp.N for r in rows)) * self.per_pair * self.units
+
+    def run(self, rows):
+        import oracle
+        inp, qr = self.inp, self._q(rows)
+        if inp.variant == 1:
+            return oracle.prefill_v1(None, self.k, self.v, self.lam, self.li, causal=inp.causal,
+                                     apply_norm=inp.apply_norm, eps=inp.eps, rows=rows, q_rows=qr)
+        return oracle.prefill_v2(None, self.k, self.v, self.lam, causal=inp.causal, rows=rows,
+                                 q_rows=qr)
+
+    def sample(self, seconds: float, seed: int = 7):
+        """Seeded query rows sized so that one oracle call takes about `seconds`."""
+        inp = self.inp
+        rng = np.random.default_rng(seed)
+        n = 8
+        for _ in range(3):
+            rows = sorted(rng.choice(inp.N, size=min(n, inp.N), replace=False).tolist())
+            t0 = time.perf_counter()
+            self.run(rows)
+            dt = time.perf_counter() - t0
+            if dt >= 0.5 * seconds or n >= inp.N:
+                break
+            n = int(min(inp.N, max(n + 1, n * seconds / max(dt, 1e-3))))
+        rows = sorted(np.random.default_rng(seed + 1).choice(inp.N, size=min(n, inp.N),
+                                                             replace=False).tolist())
+        desc = f"{len(rows)} seeded query rows of every one of the {self.units} units of {inp.name}"
+        return rows, desc
+
+
+def oracle_decode_sample(inp, seconds):
+    import oracle
+    from differential_attention_05_b200 import synth
+    lam = oracle.lambda_(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.depth)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        b = n % inp.B
+        oracle.decode_v2(synth.bf16_to_f32(inp.q[b:b + 1]), synth.bf16_to_f32(inp.k[b:b + 1]),
+                         synth.bf16_to_f32(inp.v[b:b + 1]), lam)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return n, dt
+
+
+def cpu_baseline(inp, seconds=12.0):
+    import oracle
+    cores = oracle.default_threads()
+    if inp.mode == "decode":
+        n, dt = oracle_decode_sample(inp, seconds)
+        val = n * decode_bytes(1, inp.N, inp.Hkv, inp.d) / dt / 1e9
+        return {"value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                "sample": f"{n} batch entries of {inp.name}, {dt:.1f} s"}
+    orc = OracleRows(inp)
+    rows, desc = orc.sample(seconds)
+    t0 = time.perf_counter()
+    orc.run(rows)
+    dt = time.perf_counter() - t0
+    return {"value": round(orc.flops(rows) / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle", "sample": f"{desc}, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    import oracle
+    oracle.build()
+    inp = workload_inputs(args.workload)
+    cores = oracle.default_threads()
+    decode = inp.mode == "decode"
+    per_step_s = max(0.5, min(8.0, 120.0 / max(1, args.steps + args.warmup)))
+    if decode:
+        times = []
+        for i in range(args.warmup + args.steps):
+            n, dt = oracle_decode_sample(inp, per_step_s)
+            if i >= args.warmup:
+                times.append((n, dt))
+        total_units = sum(n for n, _ in times)
+        total_s = sum(dt for _, dt in times)
+        value = total_units * decode_bytes(1, inp.N, inp.Hkv, inp.d) / total_s / 1e9
+        unit, metric = "GB/s", "diff-attn decode KV GB/s at 1 B200"
+        sample = f"whole batch entries of {inp.name} ({total_units} in {total_s:.1f} s)"
+    else:
+        orc = OracleRows(inp)
+        rows, desc = orc.sample(per_step_s)
+        flops = orc.flops(rows)
+        ts = []
+        for i in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            orc.run(rows)
+            if i >= args.warmup:
+                ts.append(time.perf_counter() - t0)
+        total_s = sum(ts)
+        value = flops * len(ts) / total_s / 1e12
+        unit, metric = "TFLOP/s", "diff-attn prefill TFLOP/s (% bf16 peak)"
+        sample = desc
+    ms_per_step = 1e3 * total_s / args.steps
+    return {
+        "impl": "reference",
+        "metric": metric, "value": round(value, 6), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded numpy PCG64, bf16-rounded; shapes and distributions of the workload)",
+        "config": {"workload": inp.name, "batch": inp.B, "seq_len": inp.N, "heads": inp.H,
+                   "kv_heads": inp.Hkv, "head_dim": inp.d, "causal": bool(inp.causal)},
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+# ---------------------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=("c2", "c3", "c4", "c5"), default="c2")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle timing (profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        # the oracle runs on the host of rank 0 only; other ranks have nothing to do
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return 0
+
+    import torch
+    from datetime import timedelta
+
+    device = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", rank=rank, world_size=world, device_id=device,
+                                timeout=timedelta(seconds=300))
+    try:
+        line = run_ours(args, rank, world, device)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            inp = workload_inputs(args.workload)
+            line["cpu_baseline"] = cpu_baseline(inp, args.cpu_seconds)
+        elif rank == 0:
+            line["cpu_baseline"] = None
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -50,6 +50,8 @@ cudaError_t launch_prefill_f32(const PrefillArgs& a, cudaStream_t stream);
 
 // tcgen05 bf16 prefill; returns cudaErrorNotSupported for shapes it does not handle.
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream);
+// V1 (d = 64, V width 128, per-head RMSNorm): two-pass tcgen05 kernel
+cudaError_t launch_prefill_tc_v1(const PrefillArgs& a, cudaStream_t stream);
 
 // split-KV decode (V2, bf16, d = 128, 8 query heads per KV head)
 constexpr int kDecodeChunk = 64;  // keys per pipeline stage

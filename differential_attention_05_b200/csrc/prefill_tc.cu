@@ -13,7 +13,8 @@
 //     (V2) and every V tile (V1 and V2). TMEM holds S_1, S_2, O_1, O_2 (4 x 128 columns,
 //     the full 512). P_b is written back over S_b as bf16 and fed to the P.V MMA straight
 //     from TMEM, so neither map ever leaves the SM.
-//   * warp 8 (one lane) issues TMA tile loads (128-byte swizzle, no multicast) into a
+//   * 384 threads; after launch the registers are re-split (setmaxnreg) towards the
+//     softmax warpgroups. warp 8 (one lane) issues TMA tile loads (128-byte swizzle, no multicast) into a
 //     2-stage K ring and a 2-stage V ring; warp 9 (one lane) allocates TMEM and issues all
 //     tcgen05.mma; warps 0-3 run the online softmax of branch 1, warps 4-7 of branch 2
 //     (thread t owns TMEM lane t = query row t, so row max and row sum need no shuffles).
@@ -31,6 +32,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tma_host.cuh"
 
 namespace diffattn {
 
@@ -44,7 +46,10 @@ constexpr int K_OFF = 4 * BLK_BYTES;       // 64K
 constexpr int V_OFF = K_OFF + KSTAGES * 2 * BLK_BYTES;
 constexpr int MISC_OFF = V_OFF + VSTAGES * 2 * BLK_BYTES;  // 192K
 constexpr int SMEM_BYTES = MISC_OFF + 4096 + 1024;         // + misc + alignment slack
-constexpr int NUM_THREADS = 320;           // 8 softmax warps + TMA warp + MMA warp
+constexpr int NUM_THREADS = 384;           // 8 softmax warps + TMA warp + MMA warp + 2 idle
+// register split after launch (168 per thread): softmax warpgroups 208, the third 88;
+// 2 * 208 + 88 = 3 * 168, so the increases are exactly covered by the decrease
+constexpr int REGS_SOFTMAX = 208, REGS_OTHER = 88;
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t COL_S1 = 0, COL_S2 = 128, COL_O1 = 256, COL_O2 = 384;
 constexpr float RESCALE_LOG2 = 8.0f;       // lazy-rescale threshold (factor 256)
@@ -62,10 +67,6 @@ struct Misc {
 };
 static_assert(sizeof(Misc) <= 4096, "misc region");
 }  // namespace
-
-struct TcMaps {
-  CUtensorMap q, k, v;
-};
 
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -116,6 +117,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     qh1 = 2 * u; qh2 = 2 * u + 1; kvh = (2 * u) / a.group;
   }
 
+  if (warp >= 8) {
+    // third warpgroup: gives registers to the softmax warpgroups, then TMA / MMA roles
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
   if (warp == 8) {
     // ------------------------------ TMA producer -------------------------------------
     if (lane == 0) {
@@ -236,7 +240,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_commit(&ms.o_full);  // arrives once every MMA issued above has completed
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
     // ------------------------- softmax warpgroups (branch br) -------------------------
     const int br = warp >> 2;              // 0: warps 0-3, 1: warps 4-7
     const int row = (warp & 3) * 32 + lane;  // TMEM lane == query row in the tile
@@ -252,15 +258,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ok = mbar_wait(&ms.s_full[br], j & 1, abort_flag);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;  // tcgen05.ld/st below are warp-wide
       tc_fence_after();
+      // S row (raw scores) -> registers: four loads in flight, one wait
       float s[BN];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(s_col + c * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]) * sl2;
-      }
+      for (int c = 0; c < BN / 32; ++c) tmem_ld32f(s_col + c * 32, s + c * 32);
+      tmem_wait_ld();
       // mask: causal diagonal tile, or keys past N when not causal
       const int k0 = j * BN;
       const int lim = a.causal ? (qi - k0) : (a.N - 1 - k0);  // last visible key offset
@@ -269,9 +271,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int e = 0; e < BN; ++e)
           if (e > lim) s[e] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row max: four independent chains of 3-input max
+      float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < BN; ++e) mx = fmaxf(mx, s[e]);
+      for (int e = 0; e < BN; e += 8) {
+        c0 = fmax3(c0, s[e + 0], s[e + 1]);
+        c1 = fmax3(c1, s[e + 2], s[e + 3]);
+        c2 = fmax3(c2, s[e + 4], s[e + 5]);
+        c3 = fmax3(c3, s[e + 6], s[e + 7]);
+      }
+      const float mx = fmax3(fmaxf(c0, c1), c2, c3) * sl2;  // log2 domain
       // raise the running max only when it grew by more than 2^8 (or was unset); the
       // decision is per row, the O rescale below is done by the whole warp when any of
       // its rows needs it (rows that do not use alpha = 1)
@@ -292,20 +301,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       l *= alpha;
       m = mn;
-      const float mref = (m == -INFINITY) ? 0.f : m;  // fully masked row: all p = 0
-      float ps = 0.f;
+      // P = 2^(s * log2(e)/sqrt(d) - m), summed in fp32, stored as bf16 over S_br
+      const float nm = (m == -INFINITY) ? 0.f : -m;  // fully masked row: all p = 0
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, a4 = 0.f, a5 = 0.f, a6 = 0.f, a7 = 0.f;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float p0 = ex2(s[c * 64 + 2 * e] - mref);
-          const float p1 = ex2(s[c * 64 + 2 * e + 1] - mref);
-          ps += p0 + p1;
+        for (int e = 0; e < 32; e += 2) {
+          float x0, x1, x2, x3;
+          ffma2(x0, x1, s[c * 64 + 2 * e], s[c * 64 + 2 * e + 1], sl2, sl2, nm, nm);
+          ffma2(x2, x3, s[c * 64 + 2 * e + 2], s[c * 64 + 2 * e + 3], sl2, sl2, nm, nm);
+          const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+          if ((e & 2) == 0) {
+            fadd2(a0, a1, a0, a1, p0, p1);
+            fadd2(a2, a3, a2, a3, p2, p3);
+          } else {
+            fadd2(a4, a5, a4, a5, p0, p1);
+            fadd2(a6, a7, a6, a7, p2, p3);
+          }
           pk[e] = pack_bf16(p0, p1);
+          pk[e + 1] = pack_bf16(p2, p3);
         }
         tmem_st32(s_col + c * 32, pk);
       }
+      const float ps = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
       l += ps;
       tmem_wait_st();
       tc_fence_before();
@@ -329,9 +349,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld32(lane_addr + COL_O1 + br * 64 + c * 32, r1);
         tmem_ld32(lane_addr + COL_O2 + br * 64 + c * 32, r2);
         tmem_wait_ld();
+        // a_b = O_b / l_b rounded on its own, then one fused a_1 - lambda a_2: identical
+        // branches with lambda = 1 give exactly 0 (no contraction across the subtraction)
 #pragma unroll
         for (int e = 0; e < 32; ++e)
-          y[c * 32 + e] = __uint_as_float(r1[e]) * inv1 - lam * (__uint_as_float(r2[e]) * inv2);
+          y[c * 32 + e] = __fmaf_rn(-lam, __fmul_rn(__uint_as_float(r2[e]), inv2),
+                                    __fmul_rn(__uint_as_float(r1[e]), inv1));
       }
       if (VARIANT == DIFFATTN_V1 && a.apply_norm) {
         float ss = 0.f;
@@ -381,39 +404,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 4-D bf16 map {C (contiguous), heads, tokens, batch}, box {64, 1, 128, 1}, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, int C, int heads, int N, int B,
-              const int64_t* strides /* batch, token, head (elements) */) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)heads, (cuuint64_t)N, (cuuint64_t)B};
-  int64_t hs = strides[2], ts = strides[1], bs = strides[0];
-  // extents of 1 may carry any stride; give TMA a well-formed one
-  if (heads == 1) hs = C;
-  if (N == 1) ts = hs * heads;
-  if (B == 1) bs = ts * N;
-  cuuint64_t gstr[3] = {(cuuint64_t)hs * 2, (cuuint64_t)ts * 2, (cuuint64_t)bs * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
-  cuuint32_t es[4] = {1, 1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, gstr, box,
-                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int VARIANT>
 cudaError_t launch_variant(const PrefillArgs& a, cudaStream_t stream) {
   TcMaps maps;
@@ -444,7 +434,7 @@ cudaError_t launch_variant(const PrefillArgs& a, cudaStream_t stream) {
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
   if (a.variant == DIFFATTN_V1) {
     if (a.d != 64) return cudaErrorNotSupported;
-    return launch_variant<DIFFATTN_V1>(a, stream);
+    return launch_prefill_tc_v1(a, stream);  // two-pass kernel (prefill_tc_v1.cu)
   }
   if (a.d != 128 || a.group % 2 != 0) return cudaErrorNotSupported;
   return launch_variant<DIFFATTN_V2>(a, stream);

@@ -72,10 +72,10 @@ def _load():
         lib.oracle_lambda.argtypes = [dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, dp]
         lib.oracle_prefill_v1.restype = ctypes.c_int
         lib.oracle_prefill_v1.argtypes = [dp, dp, dp, dp, ctypes.c_double] + [ctypes.c_int] * 6 + [
-            ctypes.c_double, ip, ctypes.c_int, dp, ctypes.c_int]
+            ctypes.c_double, ip, ctypes.c_int, ctypes.c_int, dp, ctypes.c_int]
         lib.oracle_prefill_v2.restype = ctypes.c_int
         lib.oracle_prefill_v2.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 6 + [
-            ip, ctypes.c_int, dp, ctypes.c_int]
+            ip, ctypes.c_int, ctypes.c_int, dp, ctypes.c_int]
         lib.oracle_decode_v2.restype = ctypes.c_int
         lib.oracle_decode_v2.argtypes = [dp, dp, dp, ip, dp] + [ctypes.c_int] * 5 + [dp, ctypes.c_int]
         lib.oracle_map_row_v2.restype = ctypes.c_int
@@ -131,31 +131,51 @@ def _rows(rows, N):
 
 
 def prefill_v1(q, k, v, lam, lambda_init_value: float, causal=True, apply_norm=True,
-               eps=1e-5, rows=None, threads=None) -> np.ndarray:
-    """V1 prefill. q,k: [B,N,H,2,d]; v: [B,N,H,2d]; lam: [H] -> out [B,R,H,2d]."""
-    q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
-    B, N, H, two, d = q.shape
-    assert two == 2 and k.shape == q.shape and v.shape == (B, N, H, 2 * d) and lam.shape == (H,)
+               eps=1e-5, rows=None, threads=None, q_rows=None) -> np.ndarray:
+    """V1 prefill. q,k: [B,N,H,2,d]; v: [B,N,H,2d]; lam: [H] -> out [B,R,H,2d].
+    With rows and q_rows ([B,R,H,2,d], the queries at those positions), q may be None."""
+    k, v, lam = _f64(k), _f64(v), _f64(lam)
+    B, N, H, two, d = k.shape
+    assert two == 2 and v.shape == (B, N, H, 2 * d) and lam.shape == (H,)
     r, R = _rows(rows, N)
+    compact = q_rows is not None
+    if compact:
+        assert r is not None
+        q = _f64(q_rows)
+        assert q.shape == (B, R, H, 2, d)
+    else:
+        q = _f64(q)
+        assert q.shape == k.shape
     out = np.zeros((B, R, H, 2 * d), dtype=np.float64)
     rc = _load().oracle_prefill_v1(_dp(q), _dp(k), _dp(v), _dp(lam), float(lambda_init_value),
                                    B, N, H, d, int(bool(causal)), int(bool(apply_norm)), float(eps),
-                                   _ip(r), R, _dp(out), int(threads or default_threads()))
+                                   _ip(r), R, int(compact), _dp(out),
+                                   int(threads or default_threads()))
     if rc != 0:
         raise ValueError(f"oracle_prefill_v1 failed: {rc}")
     return out
 
 
-def prefill_v2(q, k, v, lam, causal=True, rows=None, threads=None) -> np.ndarray:
-    """V2 prefill. q: [B,N,Hq,d]; k,v: [B,N,Hkv,d]; lam: [Hq/2] -> out [B,R,Hq/2,d]."""
-    q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
-    B, N, Hq, d = q.shape
-    Hkv = k.shape[2]
-    assert k.shape == (B, N, Hkv, d) and v.shape == k.shape and lam.shape == (Hq // 2,)
+def prefill_v2(q, k, v, lam, causal=True, rows=None, threads=None, q_rows=None) -> np.ndarray:
+    """V2 prefill. q: [B,N,Hq,d]; k,v: [B,N,Hkv,d]; lam: [Hq/2] -> out [B,R,Hq/2,d].
+    With rows and q_rows ([B,R,Hq,d], the queries at those positions), q may be None."""
+    k, v, lam = _f64(k), _f64(v), _f64(lam)
+    B, N, Hkv, d = k.shape
+    assert v.shape == k.shape
     r, R = _rows(rows, N)
+    compact = q_rows is not None
+    if compact:
+        assert r is not None
+        q = _f64(q_rows)
+        assert q.shape[:2] == (B, R) and q.shape[3] == d
+    else:
+        q = _f64(q)
+        assert q.shape[:2] == (B, N) and q.shape[3] == d
+    Hq = q.shape[2]
+    assert lam.shape == (Hq // 2,)
     out = np.zeros((B, R, Hq // 2, d), dtype=np.float64)
     rc = _load().oracle_prefill_v2(_dp(q), _dp(k), _dp(v), _dp(lam), B, N, Hq, Hkv, d,
-                                   int(bool(causal)), _ip(r), R, _dp(out),
+                                   int(bool(causal)), _ip(r), R, int(compact), _dp(out),
                                    int(threads or default_threads()))
     if rc != 0:
         raise ValueError(f"oracle_prefill_v2 failed: {rc}")

@@ -142,6 +142,7 @@ struct job {
   const int* kv_len;
   const int* rows;
   int n_rows;
+  int q_compact; /* 1: q holds only the sampled rows, [B, n_rows, ...] */
   int B, N, H, Hq, Hkv, d, causal, apply_norm;
   double eps, lambda_init;
   double* out;
@@ -210,6 +211,7 @@ static int run_job(const job* jb, int nthreads) {
  * v    : [B, N, H, 2d]
  * lam  : [H]
  * out  : [B, n_rows, H, 2d]; output row r is query position rows[r] (all N when rows==NULL)
+ * q_compact = 1 (with rows): q holds only the sampled query rows, [B, n_rows, H, 2, d].
  * One unit = (b, h).
  */
 static void v1_unit(const job* jb, long unit, double* a1, double* a2) {
@@ -217,13 +219,14 @@ static void v1_unit(const job* jb, long unit, double* a1, double* a2) {
   int N = jb->N, H = jb->H, d = jb->d, dv = 2 * d;
   long tok_q = (long)H * 2 * d; /* element stride between tokens in q and k */
   long tok_v = (long)H * dv;
-  const double* qb = jb->q + (long)b * N * tok_q + (long)h * 2 * d;
+  int n_rows = jb->rows ? jb->n_rows : N;
+  int nq = jb->q_compact ? n_rows : N; /* query rows stored per batch entry */
+  const double* qb = jb->q + (long)b * nq * tok_q + (long)h * 2 * d;
   const double* kb = jb->k + (long)b * N * tok_q + (long)h * 2 * d;
   const double* vb = jb->v + (long)b * N * tok_v + (long)h * dv;
-  int n_rows = jb->rows ? jb->n_rows : N;
   for (int r = 0; r < n_rows; ++r) {
     int i = jb->rows ? jb->rows[r] : r;
-    const double* q1 = qb + (long)i * tok_q;
+    const double* q1 = qb + (long)(jb->q_compact ? r : i) * tok_q;
     const double* q2 = q1 + d;
     int n_keys = jb->causal ? i + 1 : N;
     double* o = jb->out + (((long)b * n_rows + r) * H + h) * dv;
@@ -234,7 +237,8 @@ static void v1_unit(const job* jb, long unit, double* a1, double* a2) {
 
 int oracle_prefill_v1(const double* q, const double* k, const double* v, const double* lam,
                       double lambda_init, int B, int N, int H, int d, int causal, int apply_norm,
-                      double eps, const int* rows, int n_rows, double* out, int nthreads) {
+                      double eps, const int* rows, int n_rows, int q_compact, double* out,
+                      int nthreads) {
   if (!q || !k || !v || !lam || !out || B < 0 || N < 0 || H < 0 || d <= 0) return ORACLE_ERR_ARG;
   if (rows) {
     for (int r = 0; r < n_rows; ++r)
@@ -244,7 +248,7 @@ int oracle_prefill_v1(const double* q, const double* k, const double* v, const d
   memset(&jb, 0, sizeof(jb));
   jb.variant = 1;
   jb.q = q; jb.k = k; jb.v = v; jb.lam = lam;
-  jb.rows = rows; jb.n_rows = n_rows;
+  jb.rows = rows; jb.n_rows = n_rows; jb.q_compact = rows ? q_compact : 0;
   jb.B = B; jb.N = N; jb.H = H; jb.d = d; jb.causal = causal; jb.apply_norm = apply_norm;
   jb.eps = eps; jb.lambda_init = lambda_init; jb.out = out;
   jb.n_units = (long)B * H;
@@ -258,6 +262,7 @@ int oracle_prefill_v1(const double* q, const double* k, const double* v, const d
  * k, v : [B, N, Hkv, d]; query head hq reads KV head hq / (Hq / Hkv)
  * lam  : [Hq/2]
  * out  : [B, n_rows, Hq/2, d]
+ * q_compact = 1 (with rows): q holds only the sampled query rows, [B, n_rows, Hq, d].
  * One unit = (b, p).
  */
 static void v2_unit(const job* jb, long unit, double* a1, double* a2) {
@@ -268,14 +273,16 @@ static void v2_unit(const job* jb, long unit, double* a1, double* a2) {
   int h1 = 2 * p, h2 = 2 * p + 1;
   int g1 = h1 / group, g2 = h2 / group;
   long tok_q = (long)jb->Hq * d, tok_kv = (long)jb->Hkv * d;
-  const double* qb = jb->q + (long)b * N * tok_q;
+  int n_rows = jb->rows ? jb->n_rows : N;
+  int nq = jb->q_compact ? n_rows : N;
+  const double* qb = jb->q + (long)b * nq * tok_q;
   const double* kb = jb->k + (long)b * N * tok_kv;
   const double* vb = jb->v + (long)b * N * tok_kv;
-  int n_rows = jb->rows ? jb->n_rows : N;
   for (int r = 0; r < n_rows; ++r) {
     int i = jb->rows ? jb->rows[r] : r;
-    const double* q1 = qb + (long)i * tok_q + (long)h1 * d;
-    const double* q2 = qb + (long)i * tok_q + (long)h2 * d;
+    long qr = jb->q_compact ? r : i;
+    const double* q1 = qb + qr * tok_q + (long)h1 * d;
+    const double* q2 = qb + qr * tok_q + (long)h2 * d;
     int n_keys = jb->causal ? i + 1 : N;
     double* o = jb->out + (((long)b * n_rows + r) * P + p) * d;
     /* both branches of a pair read the same KV head when Hq/Hkv is even */
@@ -286,7 +293,7 @@ static void v2_unit(const job* jb, long unit, double* a1, double* a2) {
 
 int oracle_prefill_v2(const double* q, const double* k, const double* v, const double* lam,
                       int B, int N, int Hq, int Hkv, int d, int causal, const int* rows,
-                      int n_rows, double* out, int nthreads) {
+                      int n_rows, int q_compact, double* out, int nthreads) {
   if (!q || !k || !v || !lam || !out || B < 0 || N < 0 || Hq <= 0 || Hkv <= 0 || d <= 0)
     return ORACLE_ERR_ARG;
   if (Hq % 2 != 0 || Hq % Hkv != 0 || (Hq / Hkv) % 2 != 0) return ORACLE_ERR_ARG;
@@ -298,7 +305,7 @@ int oracle_prefill_v2(const double* q, const double* k, const double* v, const d
   memset(&jb, 0, sizeof(jb));
   jb.variant = 2;
   jb.q = q; jb.k = k; jb.v = v; jb.lam = lam;
-  jb.rows = rows; jb.n_rows = n_rows;
+  jb.rows = rows; jb.n_rows = n_rows; jb.q_compact = rows ? q_compact : 0;
   jb.B = B; jb.N = N; jb.Hq = Hq; jb.Hkv = Hkv; jb.d = d; jb.causal = causal;
   jb.out = out;
   jb.n_units = (long)B * (Hq / 2);

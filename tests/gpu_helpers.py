@@ -2,6 +2,9 @@
 library through its C ABI binding, and compare with the oracle."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -47,9 +50,17 @@ def errors(gpu: np.ndarray, ref: np.ndarray):
     return max_abs, rel_rms
 
 
+def _log(what, max_abs, rel_rms):
+    path = os.environ.get("DIFFATTN_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": what, "max_abs": max_abs, "rel_rms": rel_rms}) + "\n")
+
+
 def assert_parity(gpu: np.ndarray, ref: np.ndarray, dtype: str, what: str = ""):
     assert np.all(np.isfinite(gpu)), f"{what}: non-finite output"
     max_abs, rel_rms = errors(gpu, ref)
+    _log(what, max_abs, rel_rms)
     if dtype == "f32":
         assert max_abs <= F32_ATOL, f"{what}: max abs {max_abs:.3e} > {F32_ATOL}"
     else:

@@ -285,3 +285,26 @@ ALL_PINS = [
     pin_brute_force_tiny,
     pin_noise_cancellation,
 ]
+
+
+def pin_compact_query_rows():
+    """Sampled rows given as a compact query array equal the same rows of the full run
+    (bookkeeping check of the row-sampling path used at full sizes)."""
+    r = _rng(9)
+    B, N, H, d = 2, 40, 2, 8
+    q = r.standard_normal((B, N, H, 2, d)); k = r.standard_normal((B, N, H, 2, d))
+    v = r.standard_normal((B, N, H, 2 * d))
+    lam = np.array([0.4, 0.9])
+    rows = [39, 0, 17]
+    full = oracle.prefill_v1(q, k, v, lam, 0.5, threads=1)
+    comp = oracle.prefill_v1(None, k, v, lam, 0.5, rows=rows, q_rows=q[:, rows], threads=1)
+    _close(comp, full[:, rows], 0.0, "V1 compact rows")
+    Hq, Hkv = 8, 2
+    q2 = r.standard_normal((B, N, Hq, d)); k2 = r.standard_normal((B, N, Hkv, d))
+    v2 = r.standard_normal((B, N, Hkv, d)); lam2 = r.standard_normal(Hq // 2)
+    full2 = oracle.prefill_v2(q2, k2, v2, lam2, threads=1)
+    comp2 = oracle.prefill_v2(None, k2, v2, lam2, rows=rows, q_rows=q2[:, rows], threads=1)
+    _close(comp2, full2[:, rows], 0.0, "V2 compact rows")
+
+
+ALL_PINS.append(pin_compact_query_rows)
