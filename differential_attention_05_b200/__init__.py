@@ -9,6 +9,7 @@ from ._binding import (  # noqa: F401
     diffattn_lambda,
     diffattn_fwd_prefill,
     diffattn_fwd_decode,
+    diffattn_fwd_decode_static,
     diffattn_decode_workspace_size,
     diffattn_status_string,
     library_path,
@@ -20,6 +21,7 @@ __all__ = [
     "diffattn_lambda",
     "diffattn_fwd_prefill",
     "diffattn_fwd_decode",
+    "diffattn_fwd_decode_static",
     "diffattn_decode_workspace_size",
     "diffattn_status_string",
     "library_path",

@@ -34,6 +34,7 @@ EXPORTS = (
     "diffattn_fwd_prefill",
     "diffattn_decode_workspace_size",
     "diffattn_fwd_decode",
+    "diffattn_fwd_decode_static",
 )
 
 
@@ -112,6 +113,9 @@ def load_library():
     lib.diffattn_fwd_decode.restype = i32
     lib.diffattn_fwd_decode.argtypes = [ctypes.POINTER(DecodeParams), vp, vp, vp, vp, f32p, vp,
                                         vp, ctypes.c_size_t, vp, vp]
+    lib.diffattn_fwd_decode_static.restype = i32
+    lib.diffattn_fwd_decode_static.argtypes = [ctypes.POINTER(DecodeParams), vp, vp, vp, vp, f32p,
+                                               vp, vp, vp]
     _lib = lib
     return lib
 
@@ -259,4 +263,22 @@ def diffattn_fwd_decode(q, k_cache, v_cache, lam, kv_len=None, out=None, workspa
                                  _ptr(kv_len), _ptr(lam), _ptr(out), _ptr(workspace), ws_bytes,
                                  _ptr(dev_status), _stream(stream))
     _check("diffattn_fwd_decode", rc)
+    return out
+
+
+def diffattn_fwd_decode_static(q, k_cache, v_cache, lam, kv_len=None, out=None, num_splits=0,
+                               dev_status=None, stream=None):
+    """diffattn_fwd_decode with the partial states in the library's own device array, for
+    callers that cannot allocate a workspace (see include/diffattn.h). Calls that overlap
+    on the GPU share that array and must be ordered."""
+    import torch
+    lib = load_library()
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq // 2, d), dtype=q.dtype, device=q.device)
+    p = decode_params(q, k_cache, v_cache, out, num_splits)
+    rc = lib.diffattn_fwd_decode_static(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(kv_len), _ptr(lam), _ptr(out), _ptr(dev_status),
+                                        _stream(stream))
+    _check("diffattn_fwd_decode_static", rc)
     return out

@@ -191,6 +191,34 @@ int diffattn_fwd_decode(const diffattn_decode_params* p, const void* q, const vo
                         const void* v_cache, const int32_t* kv_len, const float* lambda, void* out,
                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
 
+/*
+ * diffattn_fwd_decode_static -- diffattn_fwd_decode without a caller-provided workspace.
+ * (A convenience of this library; the pages describe no counterpart.)
+ *
+ * For callers that cannot allocate device memory when they call: for example a serving
+ * loop that runs from a device-memory budget fixed at start-up and must not allocate per
+ * request, or a plugin whose host application owns all device memory through its own
+ * pool. The per-split partial states live in a 16 MiB array inside the library instead.
+ * This entry point itself allocates nothing (no cudaMalloc / cudaFree, no allocating
+ * library call).
+ *
+ * Arguments, layouts and results are those of diffattn_fwd_decode. Differences:
+ *   - num_splits = 0 picks the automatic split count when its partial states fit in the
+ *     16 MiB array, otherwise the largest count that fits; an explicit num_splits whose
+ *     states do not fit, or a problem that does not fit even unsplit (about
+ *     B * Hq > 32000 at d = 128), returns DIFFATTN_ERR_WORKSPACE before any CUDA call.
+ *   - The array is one per device and shared by every call on that device, and it keeps
+ *     the previous call's contents. Nothing in it needs to start at zero (each call writes
+ *     every state it reads), but two calls whose kernels overlap on the GPU (for example
+ *     on two streams without ordering between them) race on it: order them.
+ *   - The first call made with a given device current looks up the array's device
+ *     address (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture. Every GPU that loads the library holds the array until exit.
+ */
+int diffattn_fwd_decode_static(const diffattn_decode_params* p, const void* q,
+                               const void* k_cache, const void* v_cache, const int32_t* kv_len,
+                               const float* lambda, void* out, int* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
