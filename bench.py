@@ -41,8 +41,11 @@ L2_BYTES = 126 * 1024 * 1024
 # ---------------------------------------------------------------------------------------
 # workloads and their algorithmic work
 
-def workload_inputs(name: str):
+def workload_inputs(name: str, batch: int = 0):
+    """The named workload; `batch` > 0 shrinks the decode workload's batch (profiling runs)."""
     from differential_attention_05_b200 import synth
+    if name == "c4" and batch:
+        return synth.v2_decode(B=batch, name=f"v2_bf16_decode_b{batch}_l32768_hq64_hkv8_d128")
     return {"c2": synth.config2, "c3": synth.config3, "c4": synth.config4, "c5": synth.config5}[name]()
 
 
@@ -71,6 +74,31 @@ def load_peaks():
     except (OSError, KeyError, ValueError):
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                 "source": "fallback"}
+
+
+def measured_traffic(kernel: str, workload_batch_scale: float = 1.0):
+    """DRAM bytes per launch of `kernel` from the committed ncu record (profiles/traffic.txt),
+    or None when the kernel's sources changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    csrc = os.path.join(ROOT, "differential_attention_05_b200", "csrc")
+    try:
+        lines = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    except OSError:
+        return None
+    for f in lines:
+        if len(f) != 5 or f[0] != kernel:
+            continue
+        m = hashlib.sha256()
+        try:
+            for src in f[3].split(","):
+                m.update(open(os.path.join(csrc, src), "rb").read())
+        except OSError:
+            return None
+        if m.hexdigest()[:16] != f[2]:
+            return None
+        return float(f[4]) * workload_batch_scale
+    return None
 
 
 # ---------------------------------------------------------------------------------------
@@ -146,7 +174,7 @@ def run_ours(args, rank, world, device):
         import torch.distributed as dist_mod
         dist = dist_mod
     peaks = load_peaks()
-    inp = workload_inputs(args.workload)
+    inp = workload_inputs(args.workload, args.batch)
 
     def dev(a):
         if a.dtype == np.uint16:
@@ -270,6 +298,13 @@ def run_ours(args, rank, world, device):
         e2e_ms = float(t.item())
     e2e_val = world * work * e2e_steps / (e2e_ms * 1e-3) / (1e9 if decode else 1e12)
 
+    kernel_name = ("decode_split_kernel" if decode else
+                   "prefill_tc_v1_kernel" if inp.variant == 1 else "prefill_tc_kernel<V2>")
+    # decode traffic was captured at batch 8 and grows in proportion to the batch
+    traffic = measured_traffic(kernel_name, inp.B / 8.0 if decode else 1.0)
+    if traffic is not None and not decode and inp.name not in (
+            "v1_bf16_layer_b2_h16_n4096_d64", "v2_bf16_prefill_b1_n16384_hq64_hkv8_d128"):
+        traffic = None
     line = {
         "metric": metric,
         "value": round(value, 3),
@@ -295,9 +330,10 @@ def run_ours(args, rank, world, device):
         "tokens_per_s": round(world * inp.B * (1 if decode else inp.N) * args.steps / (total_ms * 1e-3), 1),
         "roofline": {
             "bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": runit,
-            "frac": round(achieved / peak, 4), "traffic": None,
+            "frac": round(achieved / peak, 4), "traffic": traffic,
             "peak_source": f"{peaks['source']} ({'burst bf16' if bound == 'tensor' else 'HBM copy'})",
-            "kernel": "decode_split_kernel + decode_combine_kernel" if decode else "prefill_tc_kernel",
+            "kernel": ("decode_split_kernel + decode_combine_kernel" if decode else
+                       "prefill_tc_v1_kernel" if inp.variant == 1 else "prefill_tc_kernel<V2>"),
             "avg_kernel_ms": round(kern_avg, 5),
         },
         "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": int(h2d),
@@ -453,7 +489,7 @@ def cpu_baseline(inp, seconds=12.0):
 def run_reference(args, rank, world):
     import oracle
     oracle.build()
-    inp = workload_inputs(args.workload)
+    inp = workload_inputs(args.workload, args.batch)
     cores = oracle.default_threads()
     decode = inp.mode == "decode"
     per_step_s = max(0.5, min(8.0, 120.0 / max(1, args.steps + args.warmup)))
@@ -509,6 +545,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", choices=("c2", "c3", "c4", "c5"), default="c2")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="decode workload only: smaller batch (profiling runs)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (profiling runs)")
@@ -539,7 +577,7 @@ def main():
     try:
         line = run_ours(args, rank, world, device)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            inp = workload_inputs(args.workload)
+            inp = workload_inputs(args.workload, args.batch)
             line["cpu_baseline"] = cpu_baseline(inp, args.cpu_seconds)
         elif rank == 0:
             line["cpu_baseline"] = None
