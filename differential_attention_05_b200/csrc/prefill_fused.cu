@@ -1,0 +1,511 @@
+// prefill_fused.cu -- single-pass fused differential attention prefill on the sm_100a
+// tensor cores, V1 and V2.
+//
+// What it computes, per differential unit (V1 head / V2 query-head pair) and query row i:
+//   A_b = softmax(Q_b K_b^T / sqrt(d)) over keys j <= i (causal) or all keys,  b = 1, 2
+//   o   = (A_1 - lambda A_2) V                      (V2: K_1 = K_2 and one V per KV head)
+//   V1: o <- o / sqrt(mean(o^2) + eps) * (1 - lambda_init)
+// ("Differential Attention (V2)", The Concept, "The difference idea" and "V1 vs V2";
+//  "Attention Variants", Build It, Steps 1 and 4; Hugging Face post, "How?").
+//
+// Rounding the two branches' probabilities to bf16 separately and subtracting afterwards
+// loses the difference when the branches nearly cancel (lambda near 1, similar maps): the
+// 2^-9 rounding error of each map is amplified by about 1/(1 - lambda). So each thread
+// handles both branches of its keys and the kernel accumulates, per row,
+//   D   = sum_j (p1_j - c p2_j) v_j      with c near lambda l_1 / l_2
+//   O_2 = sum_j p2_j v_j
+// where p_b = 2^(s_b log2(e)/sqrt(d) - m_b) and m_b is branch b's running maximum. The
+// operand p1 - c p2 is formed in fp32 from the exact p1, p2 and rounded once, so it carries
+// an error relative to the (small) difference itself. At the end
+//   o = O_1/l_1 - lambda O_2/l_2 = D/l_1 + O_2 (c/l_1 - lambda/l_2),
+// and the rounding error of O_2 enters only through c/l_1 - lambda/l_2, which vanishes as
+// c is set to lambda l_1 / l_2 from the first key tile's sums and follows the running sums
+// (exchanged every tile, so both halves hold the same c). D = O_1 - c O_2 is kept exact across updates: raising m_1
+// (factor a_1) or m_2 (factor a_2) and moving c to c' maps D -> a_1 D + (a_1 c - a_2 c') O_2
+// and O_2 -> a_2 O_2, done lazily -- a maximum is raised only when it grows by more than
+// 2^8, and c is reset only when it leaves [0.8, 1.25] times its target.
+//
+// Layout of the work (one CTA per 128-query tile of one unit, heaviest causal tiles first):
+//   * keys in tiles of 64; S_1 = Q_1 K_1^T and S_2 = Q_2 K_2^T of a tile share one TMEM
+//     buffer (2 x 64 columns), double-buffered, so the tensor core computes tile j+1 while
+//     tile j is in the softmax; D and O_2 take the other 256 TMEM columns.
+//   * warps 0-3 and 4-7 (two warpgroups) take the left / right 32 keys of every tile for
+//     both branches (thread t owns TMEM lane t = query row t); the two halves exchange their
+//     row maxima through shared memory once per tile. The operands p1 - c p2 and p2 are
+//     written back over the S buffer as bf16 and read by the P.V MMAs straight from TMEM.
+//   * warp 8: TMA loads (128-byte swizzle, no multicast) of Q once and K, V in 4-stage
+//     rings; each K tile feeds both branches (V2), each V tile both P.V products.
+//   * warp 9: TMEM allocation and every tcgen05.mma / commit.
+//   * registers are re-split after launch (setmaxnreg): 208 for the softmax warpgroups,
+//     88 for the third; 2 * 208 + 88 = 3 * 168, the launch allocation.
+//   * every mbarrier wait is bounded; a timeout raises an abort flag so every role stops
+//     issuing (the softmax warpgroups still pass the same number of named barriers), drains
+//     copies and MMAs in flight, frees TMEM and reports DIFFATTN_ERR_TIMEOUT.
+#include "common.cuh"
+#include "kernels.h"
+#include "tma_host.cuh"
+
+namespace diffattn {
+
+namespace {
+constexpr int BM = 128;                  // queries per tile
+constexpr int BN = 64;                   // keys per tile
+constexpr int HALF = BN / 2;             // keys per softmax warpgroup per tile
+constexpr int QBLK = 128 * 128;          // [128 rows x 64 bf16], 128-byte swizzle
+constexpr int KBLK = 64 * 128;           // [64 rows x 64 bf16]
+constexpr int STAGES = 4;
+constexpr int Q_OFF = 0;                 // Q_1 blocks at 0 (,16K); Q_2 at 32K (,48K)
+constexpr int K_OFF = 4 * QBLK;
+constexpr int V_OFF = K_OFF + STAGES * 2 * KBLK;
+constexpr int MISC_OFF = V_OFF + STAGES * 2 * KBLK;
+constexpr int MISC_BYTES = 12288;
+constexpr int SMEM_BYTES = MISC_OFF + MISC_BYTES + 1024;
+constexpr int NUM_THREADS = 384;
+constexpr int REGS_SOFTMAX = 208, REGS_OTHER = 88;
+constexpr int TMEM_COLS = 512;
+constexpr uint32_t COL_D = 256, COL_O2 = 384;
+constexpr float RESCALE_LOG2 = 8.0f;
+
+struct Misc {
+  uint64_t q_full;
+  uint64_t k_full[STAGES], k_empty[STAGES];
+  uint64_t v_full[STAGES], v_empty[STAGES];
+  uint64_t s_full[2];
+  uint64_t p_full;   // both warpgroups wrote the P.V operands of the current tile
+  uint64_t pv_done;  // the P.V MMAs of a tile have completed
+  uint64_t o_full;   // every MMA has completed
+  uint32_t tmem_base;
+  int abort;
+  float mx[2][2][2][BM];  // [tile parity][warpgroup][branch][row] partial row maxima
+  float ls[2][2][2][BM];  // [tile parity][warpgroup][branch][row] partial row sums so far
+  float lx[2][2][BM];     // [warpgroup][branch][row] partial row sums
+  float ssx[2][BM];       // V1 norm: partial sums of squares
+};
+static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+}  // namespace
+
+__device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// row max of 32 values, four independent chains of 3-input max:
+// s[0..11] seed the chains, s[12..27] in two rounds of 8, s[28..31] close two chains
+__device__ __forceinline__ float max32(const float* s) {
+  float c0 = fmax3(s[0], s[1], s[2]), c1 = fmax3(s[3], s[4], s[5]);
+  float c2 = fmax3(s[6], s[7], s[8]), c3 = fmax3(s[9], s[10], s[11]);
+#pragma unroll
+  for (int e = 12; e < 28; e += 8) {
+    c0 = fmax3(c0, s[e + 0], s[e + 1]);
+    c1 = fmax3(c1, s[e + 2], s[e + 3]);
+    c2 = fmax3(c2, s[e + 4], s[e + 5]);
+    c3 = fmax3(c3, s[e + 6], s[e + 7]);
+  }
+  c0 = fmax3(c0, s[28], s[29]);
+  c1 = fmax3(c1, s[30], s[31]);
+  return fmax3(fmaxf(c0, c1), c2, c3);
+}
+
+template <int VARIANT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    prefill_fused_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Misc& ms = *reinterpret_cast<Misc*>(smem + MISC_OFF);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // tile -> (q-tile, unit, batch); the largest causal tiles are handed out first
+  const int n_qt = (a.N + BM - 1) / BM;
+  const int per_qt = a.units * a.B;
+  const int qt = a.causal ? (n_qt - 1 - (int)(blockIdx.x / per_qt)) : (int)(blockIdx.x / per_qt);
+  const int u = (int)(blockIdx.x % per_qt) % a.units;
+  const int b = (int)(blockIdx.x % per_qt) / a.units;
+  const int q0 = qt * BM;
+  const int kend = a.causal ? min(q0 + BM, a.N) : a.N;  // keys this tile can see
+  const int n_kt = (kend + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ms.q_full, 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ms.k_full[s], 1); mbar_init(&ms.k_empty[s], 1);
+      mbar_init(&ms.v_full[s], 1); mbar_init(&ms.v_empty[s], 1);
+    }
+    mbar_init(&ms.s_full[0], 1);
+    mbar_init(&ms.s_full[1], 1);
+    mbar_init(&ms.p_full, 2 * BM);
+    mbar_init(&ms.pv_done, 1);
+    mbar_init(&ms.o_full, 1);
+    ms.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&ms.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms.tmem_base;
+  volatile int* abort_flag = &ms.abort;
+
+  // TMA coordinates: V1 -> head u, branch 1 / 2 at columns 0 / 64 of the [2d] row;
+  // V2 -> query heads 2u, 2u+1 and their KV head
+  const int qh1 = VARIANT == DIFFATTN_V1 ? u : 2 * u;
+  const int qh2 = VARIANT == DIFFATTN_V1 ? u : 2 * u + 1;
+  const int kvh = VARIANT == DIFFATTN_V1 ? u : (2 * u) / a.group;
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
+    if (warp == 8 && lane == 0) {
+      // ------------------------------ TMA producer -----------------------------------
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.k);
+      tma_prefetch_desc(&maps.v);
+      if (VARIANT == DIFFATTN_V2) {
+        mbar_arrive_expect_tx(&ms.q_full, 4 * QBLK);
+        tma_load_4d(smem + Q_OFF + 0 * QBLK, &maps.q, &ms.q_full, 0, qh1, q0, b);
+        tma_load_4d(smem + Q_OFF + 1 * QBLK, &maps.q, &ms.q_full, 64, qh1, q0, b);
+        tma_load_4d(smem + Q_OFF + 2 * QBLK, &maps.q, &ms.q_full, 0, qh2, q0, b);
+        tma_load_4d(smem + Q_OFF + 3 * QBLK, &maps.q, &ms.q_full, 64, qh2, q0, b);
+      } else {
+        mbar_arrive_expect_tx(&ms.q_full, 2 * QBLK);
+        tma_load_4d(smem + Q_OFF + 0 * QBLK, &maps.q, &ms.q_full, 0, qh1, q0, b);   // q_1
+        tma_load_4d(smem + Q_OFF + 2 * QBLK, &maps.q, &ms.q_full, 64, qh1, q0, b);  // q_2
+      }
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < n_kt && !*abort_flag; ++j) {
+        const int st = j % STAGES;
+        const uint32_t par = ((j / STAGES) & 1) ^ 1;
+        if (!mbar_wait(&ms.k_empty[st], par, abort_flag)) break;
+        mbar_arrive_expect_tx(&ms.k_full[st], 2 * KBLK);
+        uint8_t* kd = smem + K_OFF + st * 2 * KBLK;  // V1: k_1 | k_2; V2: d 0..63 | 64..127
+        tma_load_4d(kd, &maps.k, &ms.k_full[st], 0, kvh, j * BN, b);
+        tma_load_4d(kd + KBLK, &maps.k, &ms.k_full[st], 64, kvh, j * BN, b);
+        issued_k = j + 1;
+        if (!mbar_wait(&ms.v_empty[st], par, abort_flag)) break;
+        mbar_arrive_expect_tx(&ms.v_full[st], 2 * KBLK);
+        uint8_t* vd = smem + V_OFF + st * 2 * KBLK;
+        tma_load_4d(vd, &maps.v, &ms.v_full[st], 0, kvh, j * BN, b);
+        tma_load_4d(vd + KBLK, &maps.v, &ms.v_full[st], 64, kvh, j * BN, b);
+        issued_v = j + 1;
+      }
+      if (*abort_flag) {
+        // let the copies already in flight land before the CTA's shared memory goes away
+        mbar_wait_drain(&ms.q_full, 0);
+        for (int j = max(0, issued_k - STAGES); j < issued_k; ++j)
+          mbar_wait_drain(&ms.k_full[j % STAGES], (j / STAGES) & 1);
+        for (int j = max(0, issued_v - STAGES); j < issued_v; ++j)
+          mbar_wait_drain(&ms.v_full[j % STAGES], (j / STAGES) & 1);
+      }
+    } else if (warp == 9 && lane == 0) {
+      // ------------------------------ MMA issuer -------------------------------------
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, 128, false, true);
+      const uint32_t qbase = smem_u32(smem + Q_OFF);
+      const uint32_t kbase = smem_u32(smem + K_OFF);
+      const uint32_t vbase = smem_u32(smem + V_OFF);
+      // S_1, S_2 of key tile j into buffer f (columns 128 f, 128 f + 64)
+      auto issue_s = [&](int f, int j) {
+        const uint32_t kst = kbase + (j % STAGES) * 2 * KBLK;
+#pragma unroll
+        for (int br = 0; br < 2; ++br) {
+          const uint32_t d = tmem + 128u * f + 64u * br;
+          const uint32_t qb = qbase + br * 2 * QBLK;
+          if (VARIANT == DIFFATTN_V2) {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_ss(d, sw128_desc(qb + (kk >> 2) * QBLK + (kk & 3) * 32, 16, 1024),
+                      sw128_desc(kst + (kk >> 2) * KBLK + (kk & 3) * 32, 16, 1024), IDESC_S,
+                      kk > 0);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_ss(d, sw128_desc(qb + kk * 32, 16, 1024),
+                      sw128_desc(kst + br * KBLK + kk * 32, 16, 1024), IDESC_S, kk > 0);
+          }
+        }
+        tc_commit(&ms.s_full[f]);
+      };
+      bool ok = mbar_wait(&ms.q_full, 0, abort_flag);
+      for (int j = 0; j < 2 && j < n_kt && ok; ++j) {
+        if (!(ok = mbar_wait(&ms.k_full[j], 0, abort_flag))) break;
+        tc_fence_after();
+        issue_s(j, j);
+        tc_commit(&ms.k_empty[j]);
+      }
+      for (int j = 0; j < n_kt && ok; ++j) {
+        const int f = j & 1, st = j % STAGES;
+        if (!(ok = mbar_wait(&ms.v_full[st], (j / STAGES) & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(&ms.p_full, j & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t vst = vbase + st * 2 * KBLK;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          // B = V: MN-major, 16 keys per k-step (2048 B), column blocks 8 KB apart
+          const uint64_t vd = sw128_desc(vst + kk * 2048, KBLK, 1024);
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+          umma_ts(tmem + COL_D, tmem + 128u * f + kk * 8, vd, IDESC_PV, acc);
+          umma_ts(tmem + COL_O2, tmem + 128u * f + 64u + kk * 8, vd, IDESC_PV, acc);
+        }
+        tc_commit(&ms.pv_done);
+        tc_commit(&ms.v_empty[st]);
+        if (j + 2 < n_kt) {
+          const int s2 = (j + 2) % STAGES;
+          if (!(ok = mbar_wait(&ms.k_full[s2], ((j + 2) / STAGES) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_s(f, j + 2);  // buffer f is free once the P.V MMAs above have read it
+          tc_commit(&ms.k_empty[s2]);
+        }
+      }
+      tc_commit(&ms.o_full);  // arrives once every MMA issued above has completed
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
+    // --------------------------- softmax warpgroups ------------------------------------
+    const int wg = warp >> 2;                 // key half of every tile
+    const int row = (warp & 3) * 32 + lane;   // TMEM lane == query row
+    const int qi = q0 + row;
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const float sl2 = 1.4426950408889634f * rsqrtf((float)a.d);  // log2(e)/sqrt(d)
+    const float lam = a.lambda[u];
+    float m1 = -INFINITY, m2 = -INFINITY, l1 = 0.f, l2 = 0.f, c = 0.f;
+    bool ok = true;
+
+    for (int j = 0; j < n_kt; ++j) {
+      const int f = j & 1;
+      const uint32_t sb = lane_addr + 128u * f;
+      if (ok) ok = mbar_wait(&ms.s_full[f], (j >> 1) & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      float s1[HALF], s2[HALF];
+      float pm1 = -INFINITY, pm2 = -INFINITY;
+      const int k0 = j * BN + wg * HALF;
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32f(sb + wg * HALF, s1);
+        tmem_ld32f(sb + 64 + wg * HALF, s2);
+        tmem_wait_ld();
+        const int lim = (a.causal ? qi : a.N - 1) - k0;  // last visible key offset
+        if (lim < HALF - 1) {
+#pragma unroll
+          for (int e = 0; e < HALF; ++e)
+            if (e > lim) { s1[e] = -INFINITY; s2[e] = -INFINITY; }
+        }
+        pm1 = max32(s1);
+        pm2 = max32(s2);
+      }
+      ms.mx[f][wg][0][row] = pm1;
+      ms.mx[f][wg][1][row] = pm2;
+      ms.ls[f][wg][0][row] = l1;
+      ms.ls[f][wg][1][row] = l2;
+      tc_fence_before();
+      bar_softmax();  // both halves loaded: the operand writes below may reuse the buffer
+      tc_fence_after();
+      if (!ok) {
+        if (j == 0) { bar_softmax(); bar_softmax(); }  // keep the barrier count of tile 0
+        continue;
+      }
+      const float t1 = fmaxf(pm1, ms.mx[f][wg ^ 1][0][row]) * sl2;
+      const float t2 = fmaxf(pm2, ms.mx[f][wg ^ 1][1][row]) * sl2;
+      const float L1 = l1 + ms.ls[f][wg ^ 1][0][row];  // row sums over tiles 0..j-1
+      const float L2 = l2 + ms.ls[f][wg ^ 1][1][row];
+      // lazy maxima: raise only on growth by more than 2^8 (or when unset)
+      const bool r1 = (t1 > m1 + RESCALE_LOG2) || (m1 == -INFINITY);
+      const bool r2 = (t2 > m2 + RESCALE_LOG2) || (m2 == -INFINITY);
+      const float n1 = r1 ? fmaxf(t1, m1) : m1;
+      const float n2 = r2 ? fmaxf(t2, m2) : m2;
+      const float a1 = (r1 && m1 != -INFINITY) ? ex2(m1 - n1) : 1.f;
+      const float a2 = (r2 && m2 != -INFINITY) ? ex2(m2 - n2) : 1.f;
+      // c: D = O_1 - c O_2 is best conditioned with c near lambda l_1 / l_2 (then the O_2
+      // term of the result vanishes). Tile 0 sets it from tile 0's own sums (below, after
+      // the exponentials). Later, under max updates c follows c a_1 / a_2, which leaves D
+      // unchanged, and it is reset to lambda L_1 / L_2 (sums so far) when it drifts outside
+      // [0.8, 1.25] times that target.
+      float cn = 0.f, kc = 0.f;
+      if (j > 0) {
+        const float cev = (a1 == a2) ? c : c * (a1 / a2);
+        const float cst = lam * ((L1 * a1) / (L2 * a2));
+        const float ra = fabsf(cev), rt = fabsf(cst);
+        const bool reset = (lam != 0.f) && !(ra >= 0.8f * rt && ra <= 1.25f * rt);
+        cn = reset ? cst : cev;
+        if (reset) kc = __fsub_rn(__fmul_rn(a1, c), __fmul_rn(a2, cn));
+      }
+      if (j > 0) {
+        const bool need = (a1 != 1.f) || (a2 != 1.f) || (kc != 0.f);
+        if (__any_sync(0xffffffffu, need)) {
+          // D <- a1 D + kc O_2, O_2 <- a2 O_2 on this half's 64 output columns; the
+          // P.V MMAs of the previous tile must have completed
+          ok = mbar_wait(&ms.pv_done, (j - 1) & 1, abort_flag);
+          ok = __all_sync(0xffffffffu, ok);
+          if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+              const uint32_t col = wg * 64 + ch * 32;
+              float dv[32], ov[32];
+              tmem_ld32f(lane_addr + COL_D + col, dv);
+              tmem_ld32f(lane_addr + COL_O2 + col, ov);
+              tmem_wait_ld();
+              uint32_t rd[32], ro[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                rd[e] = __float_as_uint(fmaf(kc, ov[e], a1 * dv[e]));
+                ro[e] = __float_as_uint(a2 * ov[e]);
+              }
+              tmem_st32(lane_addr + COL_D + col, rd);
+              tmem_st32(lane_addr + COL_O2 + col, ro);
+            }
+          }
+        }
+      }
+      if (!ok) {
+        if (j == 0) { bar_softmax(); bar_softmax(); }  // keep the barrier count of tile 0
+        continue;
+      }
+      l1 *= a1;
+      l2 *= a2;
+      m1 = n1;
+      m2 = n2;
+      if (j > 0) c = cn;
+      // p_b = 2^(s_b sl2 - m_b), in place
+      float s10 = 0.f, s11 = 0.f, s20 = 0.f, s21 = 0.f;
+      const float nm1 = -m1, nm2 = -m2;
+#pragma unroll
+      for (int e = 0; e < HALF; e += 2) {
+        float x0, x1, y0, y1;
+        ffma2(x0, x1, s1[e], s1[e + 1], sl2, sl2, nm1, nm1);
+        ffma2(y0, y1, s2[e], s2[e + 1], sl2, sl2, nm2, nm2);
+        s1[e] = ex2(x0);
+        s1[e + 1] = ex2(x1);
+        s2[e] = ex2(y0);
+        s2[e + 1] = ex2(y1);
+        fadd2(s10, s11, s10, s11, s1[e], s1[e + 1]);
+        fadd2(s20, s21, s20, s21, s2[e], s2[e + 1]);
+      }
+      const float t1sum = s10 + s11, t2sum = s20 + s21;
+      l1 += t1sum;
+      l2 += t2sum;
+      if (j == 0) {
+        // tile 0: c = lambda l_1 / l_2 from this tile's complete row sums
+        ms.lx[wg][0][row] = t1sum;
+        ms.lx[wg][1][row] = t2sum;
+        bar_softmax();
+        const float z1 = t1sum + ms.lx[wg ^ 1][0][row], z2 = t2sum + ms.lx[wg ^ 1][1][row];
+        c = (lam == 0.f) ? 0.f : lam * (z1 / z2);
+        bar_softmax();  // lx is reused by the epilogue
+      }
+      // operands p1 - c p2 and p2 as bf16 over this half of the buffer
+      uint32_t pa[HALF / 2], pb[HALF / 2];
+      const float nc = -c;
+#pragma unroll
+      for (int e = 0; e < HALF; e += 2) {
+        float w0, w1;
+        ffma2(w0, w1, s2[e], s2[e + 1], nc, nc, s1[e], s1[e + 1]);  // p1 - c p2
+        pa[e / 2] = pack_bf16(w0, w1);
+        pb[e / 2] = pack_bf16(s2[e], s2[e + 1]);
+      }
+      tmem_st16(sb + wg * (HALF / 2), pa);
+      tmem_st16(sb + 64 + wg * (HALF / 2), pb);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&ms.p_full);
+    }
+
+    // ------------------------------- epilogue ----------------------------------------
+    if (ok) ok = mbar_wait(&ms.o_full, 0, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    ms.lx[wg][0][row] = l1;
+    ms.lx[wg][1][row] = l2;
+    bar_softmax();
+    const float L1 = ms.lx[0][0][row] + ms.lx[1][0][row];
+    const float L2 = ms.lx[0][1][row] + ms.lx[1][1][row];
+    const float inv1 = 1.f / L1, inv2 = 1.f / L2;
+    // o = D / l_1 + O_2 (c / l_1 - lambda / l_2); products rounded on their own so that
+    // identical branches with lambda = 1 give exactly 0
+    const float coef = __fsub_rn(__fmul_rn(c, inv1), __fmul_rn(lam, inv2));
+    float y[64];
+    float ss = 0.f;
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        float dv[32], ov[32];
+        tmem_ld32f(lane_addr + COL_D + wg * 64 + ch * 32, dv);
+        tmem_ld32f(lane_addr + COL_O2 + wg * 64 + ch * 32, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) y[ch * 32 + e] = __fmaf_rn(ov[e], coef, __fmul_rn(dv[e], inv1));
+      }
+#pragma unroll
+      for (int e = 0; e < 64; ++e) ss = fmaf(y[e], y[e], ss);
+    }
+    float sc = 1.f;
+    if (VARIANT == DIFFATTN_V1) {
+      ms.ssx[wg][row] = ss;
+      bar_softmax();
+      if (a.apply_norm)
+        sc = rsqrtf((ms.ssx[0][row] + ms.ssx[1][row]) * (1.f / 128.f) + a.eps) *
+             (1.f - a.lambda_init[0]);
+    }
+    if (ok && qi < a.N) {
+      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)b * a.os[0] +
+                          (int64_t)qi * a.os[1] + (int64_t)u * a.os[2] + wg * 64;
+      uint4* o4 = reinterpret_cast<uint4*>(ob);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        uint4 w;
+        w.x = pack_bf16(y[v * 8 + 0] * sc, y[v * 8 + 1] * sc);
+        w.y = pack_bf16(y[v * 8 + 2] * sc, y[v * 8 + 3] * sc);
+        w.z = pack_bf16(y[v * 8 + 4] * sc, y[v * 8 + 5] * sc);
+        w.w = pack_bf16(y[v * 8 + 6] * sc, y[v * 8 + 7] * sc);
+        o4[v] = w;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    if (*abort_flag) {
+      mbar_wait_drain(&ms.o_full, 0);
+      if (lane == 0) report_status(a.dev_status, DIFFATTN_ERR_TIMEOUT);
+    }
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+template <int VARIANT>
+static cudaError_t launch_fused(const PrefillArgs& a, cudaStream_t stream) {
+  TcMaps maps;
+  // V1: q, k viewed as [B, N, H, 128] (branch 1 in columns 0..63, branch 2 in 64..127) and
+  // v as [B, N, H, 2d = 128]; V2: q [B, N, Hq, 128], k, v [B, N, Hkv, 128]
+  const int hq = VARIANT == DIFFATTN_V1 ? a.units : a.Hq;
+  const int hkv = VARIANT == DIFFATTN_V1 ? a.units : a.Hkv;
+  if (!make_map(&maps.q, a.q, 128, hq, a.N, a.B, a.qs, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, 128, hkv, a.N, a.B, a.ks, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, 128, hkv, a.N, a.B, a.vs, BN)) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  if (dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(prefill_fused_kernel<VARIANT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set[dev] = true;
+  }
+  const long long tiles = (long long)((a.N + BM - 1) / BM) * a.units * a.B;
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  prefill_fused_kernel<VARIANT><<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_fused(const PrefillArgs& a, cudaStream_t stream) {
+  if (a.variant == DIFFATTN_V1) {
+    if (a.d != 64) return cudaErrorNotSupported;
+    return launch_fused<DIFFATTN_V1>(a, stream);
+  }
+  if (a.d != 128 || a.group % 2 != 0) return cudaErrorNotSupported;
+  return launch_fused<DIFFATTN_V2>(a, stream);
+}
+
+}  // namespace diffattn
