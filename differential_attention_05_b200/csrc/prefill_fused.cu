@@ -19,8 +19,7 @@
 // an error relative to the (small) difference itself. At the end
 //   o = O_1/l_1 - lambda O_2/l_2 = D/l_1 + O_2 (c/l_1 - lambda/l_2),
 // and the rounding error of O_2 enters only through c/l_1 - lambda/l_2, which vanishes as
-// c is set to lambda l_1 / l_2 from the first key tile's sums and follows the running sums
-// (exchanged every tile, so both halves hold the same c). D = O_1 - c O_2 is kept exact across updates: raising m_1
+// c is set to lambda l_1 / l_2 from the running sums (including the current key tile). D = O_1 - c O_2 is kept exact across updates: raising m_1
 // (factor a_1) or m_2 (factor a_2) and moving c to c' maps D -> a_1 D + (a_1 c - a_2 c') O_2
 // and O_2 -> a_2 O_2, done lazily -- a maximum is raised only when it grows by more than
 // 2^8, and c is reset only when it leaves [0.8, 1.25] times its target.
@@ -29,17 +28,21 @@
 //   * keys in tiles of 64; S_1 = Q_1 K_1^T and S_2 = Q_2 K_2^T of a tile share one TMEM
 //     buffer (2 x 64 columns), double-buffered, so the tensor core computes tile j+1 while
 //     tile j is in the softmax; D and O_2 take the other 256 TMEM columns.
-//   * warps 0-3 and 4-7 (two warpgroups) take the left / right 32 keys of every tile for
-//     both branches (thread t owns TMEM lane t = query row t); the two halves exchange their
-//     row maxima through shared memory once per tile. The operands p1 - c p2 and p2 are
-//     written back over the S buffer as bf16 and read by the P.V MMAs straight from TMEM.
+//   * warps 4-7 own branch 2: for every key tile they form p2 over the tile's 64 keys,
+//     write it in fp32 over their own score columns and post (max, rescale factor, sum) of
+//     each row through shared memory and an mbarrier, then move on to the next tile.
+//     Warps 0-3 own branch 1: they form p1, take branch 2's tile, choose c, keep D exact
+//     (rescales), and write both bf16 operands over S_1; the P.V MMAs read them straight
+//     from TMEM. Thread t owns TMEM lane t = query row t, so row max and row sum need no
+//     shuffles, and branch 2 running a tile ahead keeps both warpgroups busy.
 //   * warp 8: TMA loads (128-byte swizzle, no multicast) of Q once and K, V in 4-stage
 //     rings; each K tile feeds both branches (V2), each V tile both P.V products.
+//   * only the branch-1 warpgroup and the MMA warp rescale / read the accumulators.
 //   * warp 9: TMEM allocation and every tcgen05.mma / commit.
 //   * registers are re-split after launch (setmaxnreg): 208 for the softmax warpgroups,
 //     88 for the third; 2 * 208 + 88 = 3 * 168, the launch allocation.
 //   * every mbarrier wait is bounded; a timeout raises an abort flag so every role stops
-//     issuing (the softmax warpgroups still pass the same number of named barriers), drains
+//     issuing (the softmax warpgroups pass the same number of named barriers), drains
 //     copies and MMAs in flight, frees TMEM and reports DIFFATTN_ERR_TIMEOUT.
 #include "common.cuh"
 #include "kernels.h"
@@ -50,7 +53,6 @@ namespace diffattn {
 namespace {
 constexpr int BM = 128;                  // queries per tile
 constexpr int BN = 64;                   // keys per tile
-constexpr int HALF = BN / 2;             // keys per softmax warpgroup per tile
 constexpr int QBLK = 128 * 128;          // [128 rows x 64 bf16], 128-byte swizzle
 constexpr int KBLK = 64 * 128;           // [64 rows x 64 bf16]
 constexpr int STAGES = 4;
@@ -71,14 +73,18 @@ struct Misc {
   uint64_t k_full[STAGES], k_empty[STAGES];
   uint64_t v_full[STAGES], v_empty[STAGES];
   uint64_t s_full[2];
-  uint64_t p_full;   // both warpgroups wrote the P.V operands of the current tile
+  // one per S buffer: a buffer is reused two tiles later only after these were consumed,
+  // so a waiter can never see two completed phases of the same barrier
+  uint64_t p2_ready[2];  // branch 2 posted p2 (TMEM) and its row state (below) for a tile
+  uint64_t p_full[2];    // the P.V operands of a tile are in TMEM
   uint64_t pv_done;  // the P.V MMAs of a tile have completed
   uint64_t o_full;   // every MMA has completed
   uint32_t tmem_base;
   int abort;
-  float mx[2][2][2][BM];  // [tile parity][warpgroup][branch][row] partial row maxima
-  float ls[2][2][2][BM];  // [tile parity][warpgroup][branch][row] partial row sums so far
-  float lx[2][2][BM];     // [warpgroup][branch][row] partial row sums
+  float h_a2[2][BM];      // [tile parity][row] branch 2: rescale factor of the tile
+  float h_l2[2][BM];      //                    running sum including the tile
+  float ex_l[2][BM];      // epilogue: [branch][row] row sums
+  float ex_c[BM];         // epilogue: c
   float ssx[2][BM];       // V1 norm: partial sums of squares
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
@@ -86,23 +92,6 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 }  // namespace
 
 __device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
-// row max of 32 values, four independent chains of 3-input max:
-// s[0..11] seed the chains, s[12..27] in two rounds of 8, s[28..31] close two chains
-__device__ __forceinline__ float max32(const float* s) {
-  float c0 = fmax3(s[0], s[1], s[2]), c1 = fmax3(s[3], s[4], s[5]);
-  float c2 = fmax3(s[6], s[7], s[8]), c3 = fmax3(s[9], s[10], s[11]);
-#pragma unroll
-  for (int e = 12; e < 28; e += 8) {
-    c0 = fmax3(c0, s[e + 0], s[e + 1]);
-    c1 = fmax3(c1, s[e + 2], s[e + 3]);
-    c2 = fmax3(c2, s[e + 4], s[e + 5]);
-    c3 = fmax3(c3, s[e + 6], s[e + 7]);
-  }
-  c0 = fmax3(c0, s[28], s[29]);
-  c1 = fmax3(c1, s[30], s[31]);
-  return fmax3(fmaxf(c0, c1), c2, c3);
-}
 
 template <int VARIANT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -131,7 +120,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(&ms.s_full[0], 1);
     mbar_init(&ms.s_full[1], 1);
-    mbar_init(&ms.p_full, 2 * BM);
+    for (int f = 0; f < 2; ++f) {
+      mbar_init(&ms.p2_ready[f], BM);
+      mbar_init(&ms.p_full[f], BM);
+    }
     mbar_init(&ms.pv_done, 1);
     mbar_init(&ms.o_full, 1);
     ms.abort = 0;
@@ -235,7 +227,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int j = 0; j < n_kt && ok; ++j) {
         const int f = j & 1, st = j % STAGES;
         if (!(ok = mbar_wait(&ms.v_full[st], (j / STAGES) & 1, abort_flag))) break;
-        if (!(ok = mbar_wait(&ms.p_full, j & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(&ms.p_full[f], (j >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t vst = vbase + st * 2 * KBLK;
 #pragma unroll
@@ -244,7 +236,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t vd = sw128_desc(vst + kk * 2048, KBLK, 1024);
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
           umma_ts(tmem + COL_D, tmem + 128u * f + kk * 8, vd, IDESC_PV, acc);
-          umma_ts(tmem + COL_O2, tmem + 128u * f + 64u + kk * 8, vd, IDESC_PV, acc);
+          umma_ts(tmem + COL_O2, tmem + 128u * f + 32u + kk * 8, vd, IDESC_PV, acc);
         }
         tc_commit(&ms.pv_done);
         tc_commit(&ms.v_empty[st]);
@@ -261,162 +253,155 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
     // --------------------------- softmax warpgroups ------------------------------------
-    const int wg = warp >> 2;                 // key half of every tile
+    const int wg = warp >> 2;                 // 0: branch 1 (+ operands), 1: branch 2
     const int row = (warp & 3) * 32 + lane;   // TMEM lane == query row
     const int qi = q0 + row;
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sl2 = 1.4426950408889634f * rsqrtf((float)a.d);  // log2(e)/sqrt(d)
     const float lam = a.lambda[u];
-    float m1 = -INFINITY, m2 = -INFINITY, l1 = 0.f, l2 = 0.f, c = 0.f;
+    const int vis = a.causal ? qi : a.N - 1;  // last visible key
+    float m = -INFINITY, l = 0.f;             // this warpgroup's branch
+    float c = 0.f;                            // branch 1 warpgroup only
     bool ok = true;
 
     for (int j = 0; j < n_kt; ++j) {
       const int f = j & 1;
-      const uint32_t sb = lane_addr + 128u * f;
+      const uint32_t sb = lane_addr + 128u * f;  // S_1 at +0, S_2 at +64
       if (ok) ok = mbar_wait(&ms.s_full[f], (j >> 1) & 1, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      float s1[HALF], s2[HALF];
-      float pm1 = -INFINITY, pm2 = -INFINITY;
-      const int k0 = j * BN + wg * HALF;
-      if (ok) {
-        tc_fence_after();
-        tmem_ld32f(sb + wg * HALF, s1);
-        tmem_ld32f(sb + 64 + wg * HALF, s2);
-        tmem_wait_ld();
-        const int lim = (a.causal ? qi : a.N - 1) - k0;  // last visible key offset
-        if (lim < HALF - 1) {
-#pragma unroll
-          for (int e = 0; e < HALF; ++e)
-            if (e > lim) { s1[e] = -INFINITY; s2[e] = -INFINITY; }
-        }
-        pm1 = max32(s1);
-        pm2 = max32(s2);
-      }
-      ms.mx[f][wg][0][row] = pm1;
-      ms.mx[f][wg][1][row] = pm2;
-      ms.ls[f][wg][0][row] = l1;
-      ms.ls[f][wg][1][row] = l2;
-      tc_fence_before();
-      bar_softmax();  // both halves loaded: the operand writes below may reuse the buffer
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
-      if (!ok) {
-        if (j == 0) { bar_softmax(); bar_softmax(); }  // keep the barrier count of tile 0
+      // this branch's 64 scores of the tile
+      float p[BN];
+      tmem_ld32f(sb + 64u * wg, p);
+      tmem_ld32f(sb + 64u * wg + 32, p + 32);
+      tmem_wait_ld();
+      const int lim = vis - j * BN;
+      if (lim < BN - 1) {
+#pragma unroll
+        for (int e = 0; e < BN; ++e)
+          if (e > lim) p[e] = -INFINITY;
+      }
+      float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < BN; e += 8) {
+        c0 = fmax3(c0, p[e + 0], p[e + 1]);
+        c1 = fmax3(c1, p[e + 2], p[e + 3]);
+        c2 = fmax3(c2, p[e + 4], p[e + 5]);
+        c3 = fmax3(c3, p[e + 6], p[e + 7]);
+      }
+      const float t = fmax3(fmaxf(c0, c1), c2, c3) * sl2;
+      // lazy maximum: raised only on growth by more than 2^8 (or when unset)
+      const bool r = (t > m + RESCALE_LOG2) || (m == -INFINITY);
+      const float n = r ? fmaxf(t, m) : m;
+      const float al = (r && m != -INFINITY) ? ex2(m - n) : 1.f;
+      m = n;
+      // p = 2^(s sl2 - m), in place
+      float sa = 0.f, sb2 = 0.f, sc2 = 0.f, sd = 0.f;
+      const float nm = -m;
+#pragma unroll
+      for (int e = 0; e < BN; e += 4) {
+        float x0, x1, x2, x3;
+        ffma2(x0, x1, p[e], p[e + 1], sl2, sl2, nm, nm);
+        ffma2(x2, x3, p[e + 2], p[e + 3], sl2, sl2, nm, nm);
+        p[e] = ex2(x0);
+        p[e + 1] = ex2(x1);
+        p[e + 2] = ex2(x2);
+        p[e + 3] = ex2(x3);
+        fadd2(sa, sb2, sa, sb2, p[e], p[e + 1]);
+        fadd2(sc2, sd, sc2, sd, p[e + 2], p[e + 3]);
+      }
+      l = l * al + ((sa + sb2) + (sc2 + sd));
+
+      if (wg == 1) {
+        // ---- branch 2: p2 (fp32) over its own score columns, row state to shared memory
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t rr[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(p[ch * 32 + e]);
+          tmem_st32(sb + 64 + ch * 32, rr);
+        }
+        ms.h_a2[f][row] = al;
+        ms.h_l2[f][row] = l;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&ms.p2_ready[f]);
         continue;
       }
-      const float t1 = fmaxf(pm1, ms.mx[f][wg ^ 1][0][row]) * sl2;
-      const float t2 = fmaxf(pm2, ms.mx[f][wg ^ 1][1][row]) * sl2;
-      const float L1 = l1 + ms.ls[f][wg ^ 1][0][row];  // row sums over tiles 0..j-1
-      const float L2 = l2 + ms.ls[f][wg ^ 1][1][row];
-      // lazy maxima: raise only on growth by more than 2^8 (or when unset)
-      const bool r1 = (t1 > m1 + RESCALE_LOG2) || (m1 == -INFINITY);
-      const bool r2 = (t2 > m2 + RESCALE_LOG2) || (m2 == -INFINITY);
-      const float n1 = r1 ? fmaxf(t1, m1) : m1;
-      const float n2 = r2 ? fmaxf(t2, m2) : m2;
-      const float a1 = (r1 && m1 != -INFINITY) ? ex2(m1 - n1) : 1.f;
-      const float a2 = (r2 && m2 != -INFINITY) ? ex2(m2 - n2) : 1.f;
-      // c: D = O_1 - c O_2 is best conditioned with c near lambda l_1 / l_2 (then the O_2
-      // term of the result vanishes). Tile 0 sets it from tile 0's own sums (below, after
-      // the exponentials). Later, under max updates c follows c a_1 / a_2, which leaves D
-      // unchanged, and it is reset to lambda L_1 / L_2 (sums so far) when it drifts outside
-      // [0.8, 1.25] times that target.
-      float cn = 0.f, kc = 0.f;
+
+      // ---- branch 1: take branch 2's tile, choose c, keep D = O_1 - c O_2, write operands
+      ok = mbar_wait(&ms.p2_ready[f], (j >> 1) & 1, abort_flag);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      tc_fence_after();
+      const float a2 = ms.h_a2[f][row];
+      const float l2 = ms.h_l2[f][row];
+      // target c = lambda l_1 / l_2 (sums including this tile); under max updates c follows
+      // c a_1 / a_2, which leaves D unchanged; reset to the target when it leaves
+      // [0.8, 1.25] times it (tile 0 always takes the target)
+      const float cst = lam * __fdiv_rn(l, l2);  // exact ratio: identical branches give c = lambda
+      float cn = cst, kc = 0.f;
       if (j > 0) {
-        const float cev = (a1 == a2) ? c : c * (a1 / a2);
-        const float cst = lam * ((L1 * a1) / (L2 * a2));
+        const float cev = (al == a2) ? c : c * __fdividef(al, a2);
         const float ra = fabsf(cev), rt = fabsf(cst);
-        const bool reset = (lam != 0.f) && !(ra >= 0.8f * rt && ra <= 1.25f * rt);
+        const bool reset = !(ra >= 0.8f * rt && ra <= 1.25f * rt);
         cn = reset ? cst : cev;
-        if (reset) kc = __fsub_rn(__fmul_rn(a1, c), __fmul_rn(a2, cn));
-      }
-      if (j > 0) {
-        const bool need = (a1 != 1.f) || (a2 != 1.f) || (kc != 0.f);
+        if (reset) kc = __fsub_rn(__fmul_rn(al, c), __fmul_rn(a2, cn));
+        const bool need = (al != 1.f) || (a2 != 1.f) || (kc != 0.f);
         if (__any_sync(0xffffffffu, need)) {
-          // D <- a1 D + kc O_2, O_2 <- a2 O_2 on this half's 64 output columns; the
-          // P.V MMAs of the previous tile must have completed
+          // D <- a_1 D + kc O_2, O_2 <- a_2 O_2 over all 128 output columns; the P.V MMAs
+          // of the previous tile must have completed
           ok = mbar_wait(&ms.pv_done, (j - 1) & 1, abort_flag);
-          ok = __all_sync(0xffffffffu, ok);
-          if (ok) {
-            tc_fence_after();
+          if (!(ok = __all_sync(0xffffffffu, ok))) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int ch = 0; ch < 4; ++ch) {
+            float dv[32], ov[32];
+            tmem_ld32f(lane_addr + COL_D + ch * 32, dv);
+            tmem_ld32f(lane_addr + COL_O2 + ch * 32, ov);
+            tmem_wait_ld();
+            uint32_t rd[32], ro[32];
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-              const uint32_t col = wg * 64 + ch * 32;
-              float dv[32], ov[32];
-              tmem_ld32f(lane_addr + COL_D + col, dv);
-              tmem_ld32f(lane_addr + COL_O2 + col, ov);
-              tmem_wait_ld();
-              uint32_t rd[32], ro[32];
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                rd[e] = __float_as_uint(fmaf(kc, ov[e], a1 * dv[e]));
-                ro[e] = __float_as_uint(a2 * ov[e]);
-              }
-              tmem_st32(lane_addr + COL_D + col, rd);
-              tmem_st32(lane_addr + COL_O2 + col, ro);
+            for (int e = 0; e < 32; ++e) {
+              rd[e] = __float_as_uint(fmaf(kc, ov[e], al * dv[e]));
+              ro[e] = __float_as_uint(a2 * ov[e]);
             }
+            tmem_st32(lane_addr + COL_D + ch * 32, rd);
+            tmem_st32(lane_addr + COL_O2 + ch * 32, ro);
           }
         }
       }
-      if (!ok) {
-        if (j == 0) { bar_softmax(); bar_softmax(); }  // keep the barrier count of tile 0
-        continue;
-      }
-      l1 *= a1;
-      l2 *= a2;
-      m1 = n1;
-      m2 = n2;
-      if (j > 0) c = cn;
-      // p_b = 2^(s_b sl2 - m_b), in place
-      float s10 = 0.f, s11 = 0.f, s20 = 0.f, s21 = 0.f;
-      const float nm1 = -m1, nm2 = -m2;
-#pragma unroll
-      for (int e = 0; e < HALF; e += 2) {
-        float x0, x1, y0, y1;
-        ffma2(x0, x1, s1[e], s1[e + 1], sl2, sl2, nm1, nm1);
-        ffma2(y0, y1, s2[e], s2[e + 1], sl2, sl2, nm2, nm2);
-        s1[e] = ex2(x0);
-        s1[e + 1] = ex2(x1);
-        s2[e] = ex2(y0);
-        s2[e + 1] = ex2(y1);
-        fadd2(s10, s11, s10, s11, s1[e], s1[e + 1]);
-        fadd2(s20, s21, s20, s21, s2[e], s2[e + 1]);
-      }
-      const float t1sum = s10 + s11, t2sum = s20 + s21;
-      l1 += t1sum;
-      l2 += t2sum;
-      if (j == 0) {
-        // tile 0: c = lambda l_1 / l_2 from this tile's complete row sums
-        ms.lx[wg][0][row] = t1sum;
-        ms.lx[wg][1][row] = t2sum;
-        bar_softmax();
-        const float z1 = t1sum + ms.lx[wg ^ 1][0][row], z2 = t2sum + ms.lx[wg ^ 1][1][row];
-        c = (lam == 0.f) ? 0.f : lam * (z1 / z2);
-        bar_softmax();  // lx is reused by the epilogue
-      }
-      // operands p1 - c p2 and p2 as bf16 over this half of the buffer
-      uint32_t pa[HALF / 2], pb[HALF / 2];
+      c = cn;
+      // operands: p1 - c p2 -> columns 0..31, p2 -> columns 32..63 (bf16 over S_1)
       const float nc = -c;
 #pragma unroll
-      for (int e = 0; e < HALF; e += 2) {
-        float w0, w1;
-        ffma2(w0, w1, s2[e], s2[e + 1], nc, nc, s1[e], s1[e + 1]);  // p1 - c p2
-        pa[e / 2] = pack_bf16(w0, w1);
-        pb[e / 2] = pack_bf16(s2[e], s2[e + 1]);
+      for (int ch = 0; ch < 2; ++ch) {
+        float q2[32];
+        tmem_ld32f(sb + 64 + ch * 32, q2);
+        tmem_wait_ld();
+        uint32_t pa[16], pb[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float w0, w1;
+          ffma2(w0, w1, q2[e], q2[e + 1], nc, nc, p[ch * 32 + e], p[ch * 32 + e + 1]);
+          pa[e / 2] = pack_bf16(w0, w1);
+          pb[e / 2] = pack_bf16(q2[e], q2[e + 1]);
+        }
+        tmem_st16(sb + ch * 16, pa);
+        tmem_st16(sb + 32 + ch * 16, pb);
       }
-      tmem_st16(sb + wg * (HALF / 2), pa);
-      tmem_st16(sb + 64 + wg * (HALF / 2), pb);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&ms.p_full);
+      mbar_arrive(&ms.p_full[f]);
     }
 
     // ------------------------------- epilogue ----------------------------------------
     if (ok) ok = mbar_wait(&ms.o_full, 0, abort_flag);
     ok = __all_sync(0xffffffffu, ok);
-    ms.lx[wg][0][row] = l1;
-    ms.lx[wg][1][row] = l2;
+    ms.ex_l[wg][row] = l;
+    if (wg == 0) ms.ex_c[row] = c;
     bar_softmax();
-    const float L1 = ms.lx[0][0][row] + ms.lx[1][0][row];
-    const float L2 = ms.lx[0][1][row] + ms.lx[1][1][row];
+    c = ms.ex_c[row];
+    const float L1 = ms.ex_l[0][row], L2 = ms.ex_l[1][row];
     const float inv1 = 1.f / L1, inv2 = 1.f / L2;
     // o = D / l_1 + O_2 (c / l_1 - lambda / l_2); products rounded on their own so that
     // identical branches with lambda = 1 give exactly 0
