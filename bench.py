@@ -298,7 +298,7 @@ def run_ours(args, rank, world, device):
         e2e_ms = float(t.item())
     e2e_val = world * work * e2e_steps / (e2e_ms * 1e-3) / (1e9 if decode else 1e12)
 
-    kernel_name = "decode_split_kernel" if decode else f"prefill_fused_kernel<V{inp.variant}>"
+    kernel_name = "decode_split_kernel" if decode else f"prefill_v{inp.variant}_kernel"
     # decode traffic was captured at batch 8 and grows in proportion to the batch
     traffic = measured_traffic(kernel_name, inp.B / 8.0 if decode else 1.0)
     if traffic is not None and not decode and inp.name not in (
@@ -331,8 +331,7 @@ def run_ours(args, rank, world, device):
             "bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": runit,
             "frac": round(achieved / peak, 4), "traffic": traffic,
             "peak_source": f"{peaks['source']} ({'burst bf16' if bound == 'tensor' else 'HBM copy'})",
-            "kernel": ("decode_split_kernel + decode_combine_kernel" if decode else
-                       f"prefill_fused_kernel<V{inp.variant}>"),
+            "kernel": ("decode_split_kernel + decode_combine_kernel" if decode else kernel_name),
             "avg_kernel_ms": round(kern_avg, 5),
         },
         "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": int(h2d),

@@ -132,7 +132,7 @@ int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   if (p->variant == DIFFATTN_V1 && a.d != 64) return DIFFATTN_ERR_UNSUPPORTED;
   if (p->variant == DIFFATTN_V2 && a.d != 128) return DIFFATTN_ERR_UNSUPPORTED;
   if (a.N > (1 << 24)) return DIFFATTN_ERR_UNSUPPORTED;
-  return from_cuda(launch_prefill_fused(a, s));
+  return from_cuda(a.variant == DIFFATTN_V1 ? launch_prefill_v1(a, s) : launch_prefill_v2(a, s));
 }
 
 static int decode_check(const diffattn_decode_params* p, int* splits, int* split_len) {

@@ -76,6 +76,31 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float x0, float x1, 
       : "f"(x0), "f"(x1), "f"(y0), "f"(y1));
 }
 
+// 2^x for a pair of floats on the FMA pipe, leaving the MUFU unit to ex2 (which it can
+// only issue at a quarter of the FMA rate). Range reduction x = n + f with n = rint(x),
+// f in [-0.5, 0.5] (adding 1.5 * 2^23 rounds x to an integer held in the low mantissa
+// bits); 2^f from a degree-4 polynomial fitted here for relative error on [-0.5, 0.5]
+// (max 2.7e-6 in fp32 Horner evaluation); n is then added to the exponent field. x is
+// clamped to >= -125 so the exponent never underflows: a masked key (x = -inf) gets
+// 2^-125 (2.4e-38) instead of 0, which is below every sum it enters by 38 decades.
+__device__ __forceinline__ void exp2_fma2(float& y0, float& y1, float x0, float x1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999992847442627f, c1 = 0.6931217908859253f, c2 = 0.240247443318367f,
+                  c3 = 0.05591785907745361f, c4 = 0.009570101276040077f;
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  float t0, t1, n0, n1, f0, f1, p0, p1;
+  fadd2(t0, t1, x0, x1, kShift, kShift);
+  fadd2(n0, n1, t0, t1, -kShift, -kShift);
+  ffma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);
+  ffma2(p0, p1, c4, c4, f0, f1, c3, c3);
+  ffma2(p0, p1, p0, p1, f0, f1, c2, c2);
+  ffma2(p0, p1, p0, p1, f0, f1, c1, c1);
+  ffma2(p0, p1, p0, p1, f0, f1, c0, c0);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
   return *reinterpret_cast<uint32_t*>(&v);
@@ -116,6 +141,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test: has the phase with parity `phase` completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(phase)
@@ -261,6 +299,36 @@ __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float* f) {
         "=f"(f[20]), "=f"(f[21]), "=f"(f[22]), "=f"(f[23]), "=f"(f[24]), "=f"(f[25]),
         "=f"(f[26]), "=f"(f[27]), "=f"(f[28]), "=f"(f[29]), "=f"(f[30]), "=f"(f[31])
       : "r"(taddr));
+}
+
+// 16 lanes x 32 bits, twice, 32 consecutive columns: with `taddr` at lane L0 (a multiple of
+// 16), threads t and t + 16 of the warp both get lane L0 + t, columns col .. col+31 (the
+// second half's column offset is 0). Lets lanes 0-15 of a 32-lane group read lanes 16-31.
+__device__ __forceinline__ void tmem_ld16x2_32f(uint32_t taddr, float* f) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 0;"
+      : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3]), "=f"(f[4]), "=f"(f[5]), "=f"(f[6]),
+        "=f"(f[7]), "=f"(f[8]), "=f"(f[9]), "=f"(f[10]), "=f"(f[11]), "=f"(f[12]), "=f"(f[13]),
+        "=f"(f[14]), "=f"(f[15]), "=f"(f[16]), "=f"(f[17]), "=f"(f[18]), "=f"(f[19]),
+        "=f"(f[20]), "=f"(f[21]), "=f"(f[22]), "=f"(f[23]), "=f"(f[24]), "=f"(f[25]),
+        "=f"(f[26]), "=f"(f[27]), "=f"(f[28]), "=f"(f[29]), "=f"(f[30]), "=f"(f[31])
+      : "r"(taddr));
+}
+
+// 32 lanes x 32 bits, 32 consecutive columns from 32 consecutive floats of a register array
+__device__ __forceinline__ void tmem_st32f(uint32_t taddr, const float* f) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "f"(f[0]), "f"(f[1]), "f"(f[2]), "f"(f[3]), "f"(f[4]), "f"(f[5]), "f"(f[6]), "f"(f[7]),
+      "f"(f[8]), "f"(f[9]), "f"(f[10]), "f"(f[11]), "f"(f[12]), "f"(f[13]), "f"(f[14]),
+      "f"(f[15]), "f"(f[16]), "f"(f[17]), "f"(f[18]), "f"(f[19]), "f"(f[20]), "f"(f[21]),
+      "f"(f[22]), "f"(f[23]), "f"(f[24]), "f"(f[25]), "f"(f[26]), "f"(f[27]), "f"(f[28]),
+      "f"(f[29]), "f"(f[30]), "f"(f[31])
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {

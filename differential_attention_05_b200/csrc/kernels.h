@@ -48,9 +48,11 @@ cudaError_t launch_lambda(const float* lq1, const float* lk1, const float* lq2, 
 
 cudaError_t launch_prefill_f32(const PrefillArgs& a, cudaStream_t stream);
 
-// bf16 prefill on tcgen05 (V1: d = 64; V2: d = 128), single pass with the (p1 - c p2, p2)
-// operand split; returns cudaErrorNotSupported for shapes it does not handle.
-cudaError_t launch_prefill_fused(const PrefillArgs& a, cudaStream_t stream);
+// bf16 prefill on tcgen05, single pass with the (p1 - c p2, p2) operand split: V1 with
+// d = 64 (prefill_v1.cu), V2 with d = 128 and an even number of query heads per KV head
+// (prefill_v2.cu); each returns cudaErrorNotSupported for shapes it does not handle.
+cudaError_t launch_prefill_v1(const PrefillArgs& a, cudaStream_t stream);
+cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream);
 
 // split-KV decode (V2, bf16, d = 128, 8 query heads per KV head)
 constexpr int kDecodeChunk = 64;  // keys per pipeline stage

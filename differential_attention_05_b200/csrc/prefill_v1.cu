@@ -1,17 +1,17 @@
-// prefill_fused.cu -- single-pass fused differential attention prefill on the sm_100a
-// tensor cores, V1 and V2.
+// prefill_v1.cu -- single-pass fused differential attention prefill on the sm_100a tensor
+// cores, V1 (branch width d = 64, value width 2d = 128). V2 runs on the kernel in
+// prefill_v2.cu.
 //
-// What it computes, per differential unit (V1 head / V2 query-head pair) and query row i:
+// What it computes, per head and query row i:
 //   A_b = softmax(Q_b K_b^T / sqrt(d)) over keys j <= i (causal) or all keys,  b = 1, 2
-//   o   = (A_1 - lambda A_2) V                      (V2: K_1 = K_2 and one V per KV head)
-//   V1: o <- o / sqrt(mean(o^2) + eps) * (1 - lambda_init)
+//   o   = (A_1 - lambda A_2) V,   then   o <- o / sqrt(mean(o^2) + eps) * (1 - lambda_init)
 // ("Differential Attention (V2)", The Concept, "The difference idea" and "V1 vs V2";
 //  "Attention Variants", Build It, Steps 1 and 4; Hugging Face post, "How?").
 //
 // Rounding the two branches' probabilities to bf16 separately and subtracting afterwards
 // loses the difference when the branches nearly cancel (lambda near 1, similar maps): the
-// 2^-9 rounding error of each map is amplified by about 1/(1 - lambda). So each thread
-// handles both branches of its keys and the kernel accumulates, per row,
+// 2^-9 rounding error of each map is amplified by about 1/(1 - lambda), and the per-head
+// RMSNorm amplifies it again. So the kernel accumulates, per row,
 //   D   = sum_j (p1_j - c p2_j) v_j      with c near lambda l_1 / l_2
 //   O_2 = sum_j p2_j v_j
 // where p_b = 2^(s_b log2(e)/sqrt(d) - m_b) and m_b is branch b's running maximum. The
@@ -19,15 +19,19 @@
 // an error relative to the (small) difference itself. At the end
 //   o = O_1/l_1 - lambda O_2/l_2 = D/l_1 + O_2 (c/l_1 - lambda/l_2),
 // and the rounding error of O_2 enters only through c/l_1 - lambda/l_2, which vanishes as
-// c is set to lambda l_1 / l_2 from the running sums (including the current key tile). D = O_1 - c O_2 is kept exact across updates: raising m_1
-// (factor a_1) or m_2 (factor a_2) and moving c to c' maps D -> a_1 D + (a_1 c - a_2 c') O_2
-// and O_2 -> a_2 O_2, done lazily -- a maximum is raised only when it grows by more than
-// 2^8, and c is reset only when it leaves [0.8, 1.25] times its target.
+// c is set to lambda l_1 / l_2 from the running sums (including the current key tile).
+// D = O_1 - c O_2 is kept exact across updates: raising m_1 (factor a_1) or m_2 (factor a_2)
+// and moving c to c' maps D -> a_1 D + (a_1 c - a_2 c') O_2 and O_2 -> a_2 O_2, done lazily
+// -- a maximum is raised only when it grows by more than 2^8, and c is reset only when it
+// leaves [0.8, 1.25] times its target.
 //
-// Layout of the work (one CTA per 128-query tile of one unit, heaviest causal tiles first):
+// Layout of the work (one CTA per 128-query tile of one head, heaviest causal tiles first):
 //   * keys in tiles of 64; S_1 = Q_1 K_1^T and S_2 = Q_2 K_2^T of a tile share one TMEM
 //     buffer (2 x 64 columns), double-buffered, so the tensor core computes tile j+1 while
-//     tile j is in the softmax; D and O_2 take the other 256 TMEM columns.
+//     tile j is in the softmax; D and O_2 take the other 256 TMEM columns. (Stacking both
+//     branches of 64 queries into one 128-row MMA, as the V2 kernel does, gains nothing
+//     here: with K_1 != K_2 the score MMAs would be two M = 64 instructions, which cost
+//     what the M = 128, N = 64 ones do.)
 //   * warps 4-7 own branch 2: for every key tile they form p2 over the tile's 64 keys,
 //     write it in fp32 over their own score columns and post (max, rescale factor, sum) of
 //     each row through shared memory and an mbarrier, then move on to the next tile.
@@ -36,7 +40,7 @@
 //     from TMEM. Thread t owns TMEM lane t = query row t, so row max and row sum need no
 //     shuffles, and branch 2 running a tile ahead keeps both warpgroups busy.
 //   * warp 8: TMA loads (128-byte swizzle, no multicast) of Q once and K, V in 4-stage
-//     rings; each K tile feeds both branches (V2), each V tile both P.V products.
+//     rings; each V tile feeds both P.V products.
 //   * only the branch-1 warpgroup and the MMA warp rescale / read the accumulators.
 //   * warp 9: TMEM allocation and every tcgen05.mma / commit.
 //   * registers are re-split after launch (setmaxnreg): 208 for the softmax warpgroups,
@@ -93,9 +97,8 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
 __device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-template <int VARIANT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    prefill_fused_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
+    prefill_v1_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -139,11 +142,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem = ms.tmem_base;
   volatile int* abort_flag = &ms.abort;
 
-  // TMA coordinates: V1 -> head u, branch 1 / 2 at columns 0 / 64 of the [2d] row;
-  // V2 -> query heads 2u, 2u+1 and their KV head
-  const int qh1 = VARIANT == DIFFATTN_V1 ? u : 2 * u;
-  const int qh2 = VARIANT == DIFFATTN_V1 ? u : 2 * u + 1;
-  const int kvh = VARIANT == DIFFATTN_V1 ? u : (2 * u) / a.group;
+  // TMA coordinates: head u, branch 1 / 2 at columns 0 / 64 of the [2d] rows of q and k
 
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
@@ -152,32 +151,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&maps.q);
       tma_prefetch_desc(&maps.k);
       tma_prefetch_desc(&maps.v);
-      if (VARIANT == DIFFATTN_V2) {
-        mbar_arrive_expect_tx(&ms.q_full, 4 * QBLK);
-        tma_load_4d(smem + Q_OFF + 0 * QBLK, &maps.q, &ms.q_full, 0, qh1, q0, b);
-        tma_load_4d(smem + Q_OFF + 1 * QBLK, &maps.q, &ms.q_full, 64, qh1, q0, b);
-        tma_load_4d(smem + Q_OFF + 2 * QBLK, &maps.q, &ms.q_full, 0, qh2, q0, b);
-        tma_load_4d(smem + Q_OFF + 3 * QBLK, &maps.q, &ms.q_full, 64, qh2, q0, b);
-      } else {
-        mbar_arrive_expect_tx(&ms.q_full, 2 * QBLK);
-        tma_load_4d(smem + Q_OFF + 0 * QBLK, &maps.q, &ms.q_full, 0, qh1, q0, b);   // q_1
-        tma_load_4d(smem + Q_OFF + 2 * QBLK, &maps.q, &ms.q_full, 64, qh1, q0, b);  // q_2
-      }
+      mbar_arrive_expect_tx(&ms.q_full, 2 * QBLK);
+      tma_load_4d(smem + Q_OFF + 0 * QBLK, &maps.q, &ms.q_full, 0, u, q0, b);   // q_1
+      tma_load_4d(smem + Q_OFF + 2 * QBLK, &maps.q, &ms.q_full, 64, u, q0, b);  // q_2
       int issued_k = 0, issued_v = 0;
       for (int j = 0; j < n_kt && !*abort_flag; ++j) {
         const int st = j % STAGES;
         const uint32_t par = ((j / STAGES) & 1) ^ 1;
         if (!mbar_wait(&ms.k_empty[st], par, abort_flag)) break;
         mbar_arrive_expect_tx(&ms.k_full[st], 2 * KBLK);
-        uint8_t* kd = smem + K_OFF + st * 2 * KBLK;  // V1: k_1 | k_2; V2: d 0..63 | 64..127
-        tma_load_4d(kd, &maps.k, &ms.k_full[st], 0, kvh, j * BN, b);
-        tma_load_4d(kd + KBLK, &maps.k, &ms.k_full[st], 64, kvh, j * BN, b);
+        uint8_t* kd = smem + K_OFF + st * 2 * KBLK;  // k_1 | k_2
+        tma_load_4d(kd, &maps.k, &ms.k_full[st], 0, u, j * BN, b);
+        tma_load_4d(kd + KBLK, &maps.k, &ms.k_full[st], 64, u, j * BN, b);
         issued_k = j + 1;
         if (!mbar_wait(&ms.v_empty[st], par, abort_flag)) break;
         mbar_arrive_expect_tx(&ms.v_full[st], 2 * KBLK);
         uint8_t* vd = smem + V_OFF + st * 2 * KBLK;
-        tma_load_4d(vd, &maps.v, &ms.v_full[st], 0, kvh, j * BN, b);
-        tma_load_4d(vd + KBLK, &maps.v, &ms.v_full[st], 64, kvh, j * BN, b);
+        tma_load_4d(vd, &maps.v, &ms.v_full[st], 0, u, j * BN, b);
+        tma_load_4d(vd + KBLK, &maps.v, &ms.v_full[st], 64, u, j * BN, b);
         issued_v = j + 1;
       }
       if (*abort_flag) {
@@ -202,18 +193,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int br = 0; br < 2; ++br) {
           const uint32_t d = tmem + 128u * f + 64u * br;
           const uint32_t qb = qbase + br * 2 * QBLK;
-          if (VARIANT == DIFFATTN_V2) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              umma_ss(d, sw128_desc(qb + (kk >> 2) * QBLK + (kk & 3) * 32, 16, 1024),
-                      sw128_desc(kst + (kk >> 2) * KBLK + (kk & 3) * 32, 16, 1024), IDESC_S,
-                      kk > 0);
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_ss(d, sw128_desc(qb + kk * 32, 16, 1024),
-                      sw128_desc(kst + br * KBLK + kk * 32, 16, 1024), IDESC_S, kk > 0);
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ss(d, sw128_desc(qb + kk * 32, 16, 1024),
+                    sw128_desc(kst + br * KBLK + kk * 32, 16, 1024), IDESC_S, kk > 0);
         }
         tc_commit(&ms.s_full[f]);
       };
@@ -423,13 +406,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int e = 0; e < 64; ++e) ss = fmaf(y[e], y[e], ss);
     }
     float sc = 1.f;
-    if (VARIANT == DIFFATTN_V1) {
-      ms.ssx[wg][row] = ss;
-      bar_softmax();
-      if (a.apply_norm)
-        sc = rsqrtf((ms.ssx[0][row] + ms.ssx[1][row]) * (1.f / 128.f) + a.eps) *
-             (1.f - a.lambda_init[0]);
-    }
+    ms.ssx[wg][row] = ss;
+    bar_softmax();
+    if (a.apply_norm)
+      sc = rsqrtf((ms.ssx[0][row] + ms.ssx[1][row]) * (1.f / 128.f) + a.eps) *
+           (1.f - a.lambda_init[0]);
     if (ok && qi < a.N) {
       __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)b * a.os[0] +
                           (int64_t)qi * a.os[1] + (int64_t)u * a.os[2] + wg * 64;
@@ -458,39 +439,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-template <int VARIANT>
-static cudaError_t launch_fused(const PrefillArgs& a, cudaStream_t stream) {
+cudaError_t launch_prefill_v1(const PrefillArgs& a, cudaStream_t stream) {
+  if (a.variant != DIFFATTN_V1 || a.d != 64) return cudaErrorNotSupported;
   TcMaps maps;
-  // V1: q, k viewed as [B, N, H, 128] (branch 1 in columns 0..63, branch 2 in 64..127) and
-  // v as [B, N, H, 2d = 128]; V2: q [B, N, Hq, 128], k, v [B, N, Hkv, 128]
-  const int hq = VARIANT == DIFFATTN_V1 ? a.units : a.Hq;
-  const int hkv = VARIANT == DIFFATTN_V1 ? a.units : a.Hkv;
-  if (!make_map(&maps.q, a.q, 128, hq, a.N, a.B, a.qs, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.k, a.k, 128, hkv, a.N, a.B, a.ks, BN)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.v, a.v, 128, hkv, a.N, a.B, a.vs, BN)) return cudaErrorInvalidValue;
+  // q, k viewed as [B, N, H, 128] (branch 1 in columns 0..63, branch 2 in 64..127) and v as
+  // [B, N, H, 2d = 128]
+  if (!make_map(&maps.q, a.q, 128, a.units, a.N, a.B, a.qs, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, 128, a.units, a.N, a.B, a.ks, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, 128, a.units, a.N, a.B, a.vs, BN)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   if (dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(prefill_fused_kernel<VARIANT>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    e = cudaFuncSetAttribute(prefill_v1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set[dev] = true;
   }
   const long long tiles = (long long)((a.N + BM - 1) / BM) * a.units * a.B;
   if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  prefill_fused_kernel<VARIANT><<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  prefill_v1_kernel<<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   return cudaGetLastError();
-}
-
-cudaError_t launch_prefill_fused(const PrefillArgs& a, cudaStream_t stream) {
-  if (a.variant == DIFFATTN_V1) {
-    if (a.d != 64) return cudaErrorNotSupported;
-    return launch_fused<DIFFATTN_V1>(a, stream);
-  }
-  if (a.d != 128 || a.group % 2 != 0) return cudaErrorNotSupported;
-  return launch_fused<DIFFATTN_V2>(a, stream);
 }
 
 }  // namespace diffattn

@@ -1,0 +1,481 @@
+// prefill_v2.cu -- single-pass fused differential attention prefill on the sm_100a tensor
+// cores, V2 (query-head pairs sharing a KV head, d = 128). V1 runs on prefill_v1.cu.
+//
+// What it computes, per query-head pair (2u, 2u+1) and query row i:
+//   A_b = softmax(Q_b K^T / sqrt(d)) over keys j <= i (causal) or all keys,  b = 1, 2
+//   o   = (A_1 - lambda A_2) V          (K, V of the pair's KV head)
+// ("Differential Attention (V2)", The Concept, "The difference idea" and "V1 vs V2";
+//  "Attention Variants", Build It, Steps 1 and 4).
+//
+// Precision. Rounding the two branches' probabilities to bf16 separately and subtracting
+// afterwards loses the difference when the branches nearly cancel (lambda near 1, similar
+// maps): the 2^-9 rounding error of each map is amplified by about 1/(1 - lambda). So the
+// kernel accumulates, per query,
+//   D   = sum_j (p1_j - c p2_j) v_j      with c near lambda l_1 / l_2
+//   O_2 = sum_j p2_j v_j
+// where p_b = 2^(s_b log2(e)/sqrt(d) - m_b) and m_b is branch b's running maximum. The
+// operand p1 - c p2 is formed in fp32 from the exact p1, p2 and rounded once, so it carries
+// an error relative to the (small) difference itself. At the end
+//   o = O_1/l_1 - lambda O_2/l_2 = D/l_1 + O_2 (c/l_1 - lambda/l_2),
+// and the rounding error of O_2 enters only through c/l_1 - lambda/l_2, which is small as
+// c tracks lambda l_1 / l_2. D = O_1 - c O_2 is kept exact across updates: raising m_1
+// (factor a_1) or m_2 (factor a_2) and moving c to c' maps D -> a_1 D + (a_1 c - a_2 c') O_2
+// and O_2 -> a_2 O_2. With c' = c a_1 / a_2 the cross term vanishes; c is reset to its
+// target (cross term included) only when it leaves [0.8, 1.25] times the target. Maxima are
+// raised lazily, only when they grow by more than 2^8.
+//
+// Tensor-core shape. A tcgen05.mma costs about the same time for any N up to 128, so the
+// products run at M = 128, N = 128: both branches share K, so one score MMA covers 64
+// queries x both branches x 128 keys, and one P.V MMA 64 queries x both branches x 128 value
+// columns (half the score instructions of a layout with a row per query and 64-key tiles).
+//   * TMEM lane / operand row of (query t, branch b) in a 64-query sub-tile:
+//     (t % 16) + 32 (t / 16) + 16 b; the Q rows are loaded in this order (16-row boxes
+//     alternating the two heads of the pair).
+//   * Warp w of a softmax warpgroup owns queries 16w..16w+15: lanes 0-15 branch 1, lanes
+//     16-31 branch 2 of the same queries. Every lane writes its p (fp32) over its own score
+//     columns; the 16-lane paired TMEM load then hands lanes 0-15 the row of lane + 16
+//     (exact p2 of the same keys). Branch 1 writes p1 - c p2 as its bf16 P row, branch 2
+//     writes p2; the P.V MMA (A = P from TMEM) leaves D in the branch-1 lanes and O_2 in
+//     the branch-2 lanes.
+//   * Two 64-query sub-tiles per CTA (128 queries share every K/V tile) ping-pong: while
+//     one warpgroup turns its scores into P, the tensor core runs the other sub-tile's
+//     products. TMEM: S/P of sub-tile 0 | O of sub-tile 0 | S/P of 1 | O of 1 (4 x 128
+//     columns). P (bf16) overwrites the first 64 columns of its S block; the next score
+//     MMA of that sub-tile is issued after its P.V MMA, and tcgen05 MMAs run in order.
+//   * Exponentials: in every 8 keys one pair is evaluated on the FMA pipe (exp2_fma2), the
+//     rest on the MUFU unit.
+//   * warp 8: TMA loads (128-byte swizzle, no multicast) of Q once and of K, V per 128-key
+//     tile into 2-stage rings; warp 9: TMEM allocation and every tcgen05.mma / commit.
+//     Registers are re-split after launch (setmaxnreg): 200 for the softmax warpgroups, 104
+//     for the third; 2 * 200 + 104 = 3 * 168, the launch allocation.
+//   * every mbarrier wait is bounded; a timeout raises an abort flag so every role stops
+//     issuing, drains copies and MMAs in flight, frees TMEM and reports
+//     DIFFATTN_ERR_TIMEOUT.
+#include "common.cuh"
+#include "kernels.h"
+#include "tma_host.cuh"
+
+namespace diffattn {
+
+namespace {
+constexpr int BM = 128;                  // queries per CTA
+constexpr int SUB = 64;                  // queries per sub-tile
+constexpr int BN = 128;                  // keys per tile
+constexpr int HALF = 128 * 128;          // one [128 rows x 64 bf16] swizzled block (16 KB)
+constexpr int KSTAGES = 2, VSTAGES = 2;
+constexpr int Q_OFF = 0;                 // sub-tile x at x * 2 * HALF
+constexpr int K_OFF = Q_OFF + 4 * HALF;  // stage s: 2 blocks (d halves)
+constexpr int V_OFF = K_OFF + KSTAGES * 2 * HALF;  // stage s: 2 blocks (value column halves)
+constexpr int MISC_OFF = V_OFF + VSTAGES * 2 * HALF;
+constexpr int MISC_BYTES = 1024;
+constexpr int SMEM_BYTES = MISC_OFF + MISC_BYTES + 1024;
+constexpr int NUM_THREADS = 384;
+constexpr int REGS_SOFTMAX = 200, REGS_OTHER = 104;
+constexpr int TMEM_COLS = 512;
+constexpr float RESCALE_LOG2 = 8.0f;
+constexpr int POLY_PAIRS = 1;          // of every 4 pairs of exponentials, on the FMA pipe
+
+struct Misc {
+  uint64_t q_full[2];
+  uint64_t k_full[KSTAGES], k_empty[KSTAGES];
+  uint64_t v_full[VSTAGES], v_empty[VSTAGES];
+  uint64_t s_full[2];  // [sub-tile] scores of the current key tile are in TMEM
+  uint64_t p_full[2];  // [sub-tile] P of the current key tile is in TMEM (128 arrivals)
+  uint64_t o_full[2];  // [sub-tile] its last P.V MMA has completed
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_OTHER == NUM_THREADS * 168, "register split");
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// descriptor of the same operand layout `bytes` further on (start address field, bits 0-13;
+// shared-memory addresses stay below 2^18, so the field never carries)
+__device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+}  // namespace
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    prefill_v2_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Misc& ms = *reinterpret_cast<Misc*>(smem + MISC_OFF);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // tile -> (q-tile, unit, batch); the largest causal tiles are handed out first
+  const int n_qt = (a.N + BM - 1) / BM;
+  const int per_qt = a.units * a.B;
+  const int qt = a.causal ? (n_qt - 1 - (int)(blockIdx.x / per_qt)) : (int)(blockIdx.x / per_qt);
+  const int u = (int)(blockIdx.x % per_qt) % a.units;
+  const int b = (int)(blockIdx.x % per_qt) / a.units;
+  const int q0 = qt * BM;
+  const int kend = a.causal ? min(q0 + BM, a.N) : a.N;  // keys this tile can see
+  const int n_kt = (kend + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&ms.q_full[x], 1);
+      mbar_init(&ms.s_full[x], 1);
+      mbar_init(&ms.p_full[x], 128);
+      mbar_init(&ms.o_full[x], 1);
+    }
+    for (int s = 0; s < KSTAGES; ++s) {
+      mbar_init(&ms.k_full[s], 1);
+      mbar_init(&ms.k_empty[s], 1);
+    }
+    for (int s = 0; s < VSTAGES; ++s) {
+      mbar_init(&ms.v_full[s], 1);
+      mbar_init(&ms.v_empty[s], 1);
+    }
+    ms.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&ms.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms.tmem_base;
+  volatile int* abort_flag = &ms.abort;
+
+  // query heads 2u, 2u+1 and their KV head
+  const int kvh = (2 * u) / a.group;
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
+    if (warp == 8 && lane == 0) {
+      // ------------------------------ TMA producer -----------------------------------
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.k);
+      tma_prefetch_desc(&maps.v);
+      for (int x = 0; x < 2; ++x) {
+        uint8_t* qd = smem + Q_OFF + x * 2 * HALF;
+        const int t0 = q0 + x * SUB;
+        // rows in TMEM-lane order: 16-row groups alternate branch 1 / branch 2
+        mbar_arrive_expect_tx(&ms.q_full[x], 2 * HALF);
+        for (int hf = 0; hf < 2; ++hf)
+          for (int g = 0; g < 8; ++g)
+            tma_load_4d(qd + hf * HALF + g * 2048, &maps.q, &ms.q_full[x], 64 * hf,
+                        2 * u + (g & 1), t0 + 16 * (g >> 1), b);
+      }
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < n_kt && !*abort_flag; ++j) {
+        const int ks = j % KSTAGES;
+        if (!mbar_wait(&ms.k_empty[ks], ((j / KSTAGES) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&ms.k_full[ks], 2 * HALF);
+        uint8_t* kd = smem + K_OFF + ks * 2 * HALF;
+        tma_load_4d(kd, &maps.k, &ms.k_full[ks], 0, kvh, j * BN, b);
+        tma_load_4d(kd + HALF, &maps.k, &ms.k_full[ks], 64, kvh, j * BN, b);
+        issued_k = j + 1;
+        const int vs = j % VSTAGES;
+        if (!mbar_wait(&ms.v_empty[vs], ((j / VSTAGES) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&ms.v_full[vs], 2 * HALF);
+        uint8_t* vd = smem + V_OFF + vs * 2 * HALF;
+        tma_load_4d(vd, &maps.v, &ms.v_full[vs], 0, kvh, j * BN, b);
+        tma_load_4d(vd + HALF, &maps.v, &ms.v_full[vs], 64, kvh, j * BN, b);
+        issued_v = j + 1;
+      }
+      if (*abort_flag) {
+        // let the copies already in flight land before the CTA's shared memory goes away
+        mbar_wait_drain(&ms.q_full[0], 0);
+        mbar_wait_drain(&ms.q_full[1], 0);
+        for (int j = max(0, issued_k - KSTAGES); j < issued_k; ++j)
+          mbar_wait_drain(&ms.k_full[j % KSTAGES], (j / KSTAGES) & 1);
+        for (int j = max(0, issued_v - VSTAGES); j < issued_v; ++j)
+          mbar_wait_drain(&ms.v_full[j % VSTAGES], (j / VSTAGES) & 1);
+      }
+    } else if (warp == 9 && lane == 0) {
+      // ------------------------------ MMA issuer -------------------------------------
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, false, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, 128, false, true);
+      // K-major operands (Q, K): 8-row groups 1024 B apart, k-step = 32 B inside the swizzle
+      // atom. V (B of P.V) is MN-major: 16 keys per k-step (2048 B), column blocks HALF apart.
+      const uint64_t qdesc = sw128_desc(smem_u32(smem + Q_OFF), 16, 1024);
+      const uint64_t kdesc = sw128_desc(smem_u32(smem + K_OFF), 16, 1024);
+      const uint64_t vdesc = sw128_desc(smem_u32(smem + V_OFF), HALF, 1024);
+      auto issue_s = [&](int x, int j) {
+        const uint64_t kd = desc_at(kdesc, (j % KSTAGES) * 2 * HALF);
+        const uint64_t qd = desc_at(qdesc, x * 2 * HALF);
+        const uint32_t d = tmem + 256u * x;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+          umma_ss(d, desc_at(qd, off), desc_at(kd, off), IDESC_S, kk > 0);
+        }
+        tc_commit(&ms.s_full[x]);
+      };
+      auto issue_pv = [&](int x, int j) {
+        const uint64_t vd = desc_at(vdesc, (j % VSTAGES) * 2 * HALF);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + 256u * x + 128u, tmem + 256u * x + kk * 8, desc_at(vd, kk * 2048),
+                  IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool done0 = false, done1 = false;
+      bool ok = mbar_wait(&ms.q_full[0], 0, abort_flag) && mbar_wait(&ms.k_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        ok = mbar_wait(&ms.q_full[1], 0, abort_flag);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_s(1, 0);
+        tc_commit(&ms.k_empty[0]);
+      }
+      for (int j = 0; j < n_kt && ok; ++j) {
+        const int vs = j % VSTAGES;
+        const int ks = (j + 1) % KSTAGES;
+        if (!(ok = mbar_wait(&ms.v_full[vs], (j / VSTAGES) & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(&ms.p_full[0], j & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (j + 1 == n_kt) {
+          tc_commit(&ms.o_full[0]);
+          done0 = true;
+        } else {
+          if (!(ok = mbar_wait(&ms.k_full[ks], ((j + 1) / KSTAGES) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_s(0, j + 1);  // S/P block 0 is rewritten after the P.V MMAs above read it
+        }
+        if (!(ok = mbar_wait(&ms.p_full[1], j & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        tc_commit(&ms.v_empty[vs]);
+        if (j + 1 == n_kt) {
+          tc_commit(&ms.o_full[1]);
+          done1 = true;
+        } else {
+          issue_s(1, j + 1);
+          tc_commit(&ms.k_empty[ks]);
+        }
+      }
+      // on an abort, these still arrive once every MMA issued above has completed
+      if (!done0) tc_commit(&ms.o_full[0]);
+      if (!done1) tc_commit(&ms.o_full[1]);
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
+    // --------------------------- softmax warpgroups ------------------------------------
+    const int x = warp >> 2;                       // sub-tile
+    const int wq = warp & 3;                       // 32-lane group of TMEM
+    const int h = (lane >> 4) & 1;                 // 0: branch 1, 1: branch 2
+    const int tq = wq * 16 + (lane & 15);          // query within the sub-tile
+    const int qi = q0 + x * SUB + tq;
+    const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
+    const uint32_t s_addr = lane_addr + 256u * x;  // S, then P over its first 64 columns
+    const uint32_t o_addr = s_addr + 128u;         // D (branch-1 lanes) / O_2 (branch 2)
+    const float sl2 = 1.4426950408889634f * rsqrtf((float)a.d);  // log2(e)/sqrt(d)
+    const float lam = a.lambda[u];
+    const int vis = a.causal ? min(qi, a.N - 1) : a.N - 1;  // last visible key
+    float m = -INFINITY, l = 0.f;  // this lane's branch
+    float c = 0.f;                 // identical in both lanes of a query
+    bool ok = true;
+
+    for (int j = 0; j < n_kt; ++j) {
+      if (ok) ok = mbar_wait(&ms.s_full[x], j & 1, abort_flag);
+      if (!(ok = __all_sync(FULL, ok))) break;
+      tc_fence_after();
+      float p[BN];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_ld32f(s_addr + 32 * i, p + 32 * i);
+      tmem_wait_ld();
+      const int lim = vis - j * BN;
+      if (lim < BN - 1) {
+#pragma unroll
+        for (int e = 0; e < BN; ++e)
+          if (e > lim) p[e] = -INFINITY;
+      }
+      float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < BN; e += 8) {
+        c0 = fmax3(c0, p[e + 0], p[e + 1]);
+        c1 = fmax3(c1, p[e + 2], p[e + 3]);
+        c2 = fmax3(c2, p[e + 4], p[e + 5]);
+        c3 = fmax3(c3, p[e + 6], p[e + 7]);
+      }
+      const float t = fmax3(fmaxf(c0, c1), c2, c3) * sl2;
+      // lazy maximum: raised only on growth by more than 2^8 (or when unset)
+      const bool r = (t > m + RESCALE_LOG2) || (m == -INFINITY);
+      const float n = r ? fmaxf(t, m) : m;
+      const float al = (r && m != -INFINITY) ? ex2(m - n) : 1.f;
+      m = n;
+      // p = 2^(s sl2 - m), in place; in every group of 8 keys the last POLY_PAIRS pairs go
+      // to the FMA pipe, the rest to the MUFU unit
+      float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
+      const float nm = -m;
+#pragma unroll
+      for (int e = 0; e < BN; e += 8) {
+        float xv[8];
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) ffma2(xv[i], xv[i + 1], p[e + i], p[e + i + 1], sl2, sl2, nm, nm);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+          if (i >= 8 - 2 * POLY_PAIRS) {
+            exp2_fma2(p[e + i], p[e + i + 1], xv[i], xv[i + 1]);
+          } else {
+            p[e + i] = ex2(xv[i]);
+            p[e + i + 1] = ex2(xv[i + 1]);
+          }
+        }
+        fadd2(sa, sb, sa, sb, p[e], p[e + 1]);
+        fadd2(sc, sd, sc, sd, p[e + 2], p[e + 3]);
+        fadd2(sa, sb, sa, sb, p[e + 4], p[e + 5]);
+        fadd2(sc, sd, sc, sd, p[e + 6], p[e + 7]);
+      }
+      l = l * al + ((sa + sb) + (sc + sd));
+
+      // the query's two branches: this lane and lane ^ 16
+      const float al_o = __shfl_xor_sync(FULL, al, 16);
+      const float l_o = __shfl_xor_sync(FULL, l, 16);
+      const float a1 = h ? al_o : al, a2 = h ? al : al_o;
+      const float l1 = h ? l_o : l, l2 = h ? l : l_o;
+      // target c = lambda l_1 / l_2 (sums including this tile); under max updates c follows
+      // c a_1 / a_2, which leaves D unchanged; reset to the target when it leaves
+      // [0.8, 1.25] times it (tile 0 always takes the target). Both lanes compute the same.
+      const float cst = lam * __fdiv_rn(l1, l2);  // exact ratio: identical branches give c = lambda
+      float cn = cst, kc = 0.f;
+      if (j > 0) {
+        const float cev = (a1 == a2) ? c : c * __fdividef(a1, a2);
+        const float ra = fabsf(cev), rt = fabsf(cst);
+        const bool reset = !(ra >= 0.8f * rt && ra <= 1.25f * rt);
+        cn = reset ? cst : cev;
+        if (reset) kc = __fsub_rn(__fmul_rn(a1, c), __fmul_rn(a2, cn));
+        const bool need = (al != 1.f) || (kc != 0.f);
+        if (__any_sync(FULL, need)) {
+          // D <- a_1 D + kc O_2, O_2 <- a_2 O_2 over all 128 value columns. The score MMA
+          // that filled S was issued after this sub-tile's previous P.V MMAs, so its
+          // completion implies theirs.
+          const float kx = h ? 0.f : kc;
+#pragma unroll 1
+          for (int ch = 0; ch < 4; ++ch) {
+            float ov[32];
+            tmem_ld32f(o_addr + ch * 32, ov);
+            tmem_wait_ld();
+            uint32_t ro[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float other = __shfl_xor_sync(FULL, ov[e], 16);
+              ro[e] = __float_as_uint(fmaf(kx, other, al * ov[e]));
+            }
+            tmem_st32(o_addr + ch * 32, ro);
+          }
+        }
+      }
+      c = cn;
+      // P row: branch 1 writes p1 - c p2, branch 2 writes p2. Every lane first puts its p
+      // (fp32) over its own score columns; the 16-lane paired load then hands lanes 0-15 the
+      // row of lane + 16 (branch 2 of the same query) and lanes 16-31 their own row.
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_st32f(s_addr + ch * 32, p + ch * 32);
+      tmem_wait_st();
+      const float nc = h ? 0.f : -c;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        float q2[32];
+        tmem_ld16x2_32f(s_addr + (16u << 16) + ch * 32, q2);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float w0, w1;
+          ffma2(w0, w1, q2[e], q2[e + 1], nc, nc, p[ch * 32 + e], p[ch * 32 + e + 1]);
+          pk[e / 2] = pack_bf16(w0, w1);
+        }
+        // bf16 pairs land on columns 16 ch .. 16 ch + 15, all read already
+        tmem_st16(s_addr + ch * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&ms.p_full[x]);
+    }
+
+    // ------------------------------- epilogue ----------------------------------------
+    if (ok) ok = mbar_wait(&ms.o_full[x], 0, abort_flag);
+    ok = __all_sync(FULL, ok);
+    const float l_o = __shfl_xor_sync(FULL, l, 16);
+    const float L1 = h ? l_o : l, L2 = h ? l : l_o;
+    const float inv1 = 1.f / L1, inv2 = 1.f / L2;
+    // o = D / l_1 + O_2 (c / l_1 - lambda / l_2); products rounded on their own so that
+    // identical branches with lambda = 1 give exactly 0
+    const float coef = __fsub_rn(__fmul_rn(c, inv1), __fmul_rn(lam, inv2));
+    // this lane writes value columns 64 h .. 64 h + 63 of its query; D and O_2 of a column
+    // sit in the two lanes of the query
+    float y[64];
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        float v0[32], v1[32];
+        tmem_ld32f(o_addr + ch * 32, v0);
+        tmem_ld32f(o_addr + 64 + ch * 32, v1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float mine = h ? v1[e] : v0[e];
+          const float other = __shfl_xor_sync(FULL, h ? v0[e] : v1[e], 16);
+          const float dv = h ? other : mine, ov = h ? mine : other;
+          y[ch * 32 + e] = __fmaf_rn(ov, coef, __fmul_rn(dv, inv1));
+        }
+      }
+    }
+    if (ok && qi < a.N) {
+      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)b * a.os[0] +
+                          (int64_t)qi * a.os[1] + (int64_t)u * a.os[2] + h * 64;
+      uint4* o4 = reinterpret_cast<uint4*>(ob);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        uint4 w;
+        w.x = pack_bf16(y[v * 8 + 0], y[v * 8 + 1]);
+        w.y = pack_bf16(y[v * 8 + 2], y[v * 8 + 3]);
+        w.z = pack_bf16(y[v * 8 + 4], y[v * 8 + 5]);
+        w.w = pack_bf16(y[v * 8 + 6], y[v * 8 + 7]);
+        o4[v] = w;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    if (*abort_flag) {
+      mbar_wait_drain(&ms.o_full[0], 0);
+      mbar_wait_drain(&ms.o_full[1], 0);
+      if (lane == 0) report_status(a.dev_status, DIFFATTN_ERR_TIMEOUT);
+    }
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream) {
+  if (a.variant != DIFFATTN_V2 || a.d != 128 || a.group % 2 != 0) return cudaErrorNotSupported;
+  TcMaps maps;
+  // q [B, N, Hq, 128], k, v [B, N, Hkv, 128]; Q boxes of 16 queries of one head (the
+  // TMEM-lane row order), K and V boxes of 128 keys
+  if (!make_map(&maps.q, a.q, 128, a.Hq, a.N, a.B, a.qs, 16)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, 128, a.Hkv, a.N, a.B, a.ks, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, 128, a.Hkv, a.N, a.B, a.vs, BN)) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  if (dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(prefill_v2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set[dev] = true;
+  }
+  const long long tiles = (long long)((a.N + BM - 1) / BM) * a.units * a.B;
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  prefill_v2_kernel<<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  return cudaGetLastError();
+}
+
+}  // namespace diffattn
