@@ -102,6 +102,26 @@ def measured_traffic(kernel: str, workload_batch_scale: float = 1.0):
 
 
 # ---------------------------------------------------------------------------------------
+# across ranks
+
+def max_over_ranks(ms: float, dist=None, device=None) -> float:
+    """The slowest rank's time: every rank times its own device with CUDA events and the
+    job's time is the maximum (one rank: `ms` itself)."""
+    if dist is None:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, work_per_rank: float, steps: int, max_ms: float, scale: float) -> float:
+    """Whole-job throughput: the work all ranks processed (each rank runs its own replica of
+    the workload) divided by the slowest rank's time, in units of `scale` per second."""
+    return world * work_per_rank * steps / (max_ms * 1e-3) / scale
+
+
+# ---------------------------------------------------------------------------------------
 # clocks during the timed region
 
 class ClockSampler:
@@ -247,17 +267,14 @@ def run_ours(args, rank, world, device):
     kern_ms = [e[1].elapsed_time(e[2]) for e in ev]
     total_ms = float(sum(step_ms))
     kern_avg = float(sum(kern_ms) / len(kern_ms))
-    if dist is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, device)
     ms_per_step = total_ms / args.steps
     if decode:
-        value = world * work * args.steps / (total_ms * 1e-3) / 1e9
+        value = job_rate(world, work, args.steps, total_ms, 1e9)
         achieved = work / (kern_avg * 1e-3) / 1e9
         peak, bound, runit = peaks["hbm_gbs"], "hbm", "GB/s"
     else:
-        value = world * work * args.steps / (total_ms * 1e-3) / 1e12
+        value = job_rate(world, work, args.steps, total_ms, 1e12)
         achieved = work / (kern_avg * 1e-3) / 1e12
         peak, bound, runit = peaks["bf16_tflops"], "tensor", "TFLOP/s"
 
@@ -292,11 +309,8 @@ def run_ours(args, rank, world, device):
     e1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_val = world * work * e2e_steps / (e2e_ms * 1e-3) / (1e9 if decode else 1e12)
+    e2e_ms = max_over_ranks(e2e_ms, dist, device)
+    e2e_val = job_rate(world, work, e2e_steps, e2e_ms, 1e9 if decode else 1e12)
 
     kernel_name = "decode_split_kernel" if decode else f"prefill_v{inp.variant}_kernel"
     # decode traffic was captured at batch 8 and grows in proportion to the batch

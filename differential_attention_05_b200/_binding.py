@@ -35,6 +35,7 @@ EXPORTS = (
     "diffattn_decode_workspace_size",
     "diffattn_fwd_decode",
     "diffattn_fwd_decode_static",
+    "diffattn_selftest_timeout",
 )
 
 
@@ -116,6 +117,8 @@ def load_library():
     lib.diffattn_fwd_decode_static.restype = i32
     lib.diffattn_fwd_decode_static.argtypes = [ctypes.POINTER(DecodeParams), vp, vp, vp, vp, f32p,
                                                vp, vp, vp]
+    lib.diffattn_selftest_timeout.restype = i32
+    lib.diffattn_selftest_timeout.argtypes = [vp, i32, vp]
     _lib = lib
     return lib
 
@@ -282,3 +285,12 @@ def diffattn_fwd_decode_static(q, k_cache, v_cache, lam, kv_len=None, out=None, 
                                         _stream(stream))
     _check("diffattn_fwd_decode_static", rc)
     return out
+
+
+def diffattn_selftest_timeout(dev_status, timeout_ms=200, stream=None):
+    """Launch the bounded-wait self-test (see include/diffattn.h): a wait that nothing
+    completes runs out after `timeout_ms` and DIFFATTN_ERR_TIMEOUT lands in `dev_status`
+    (a device int32 tensor) when the block finishes."""
+    lib = load_library()
+    rc = lib.diffattn_selftest_timeout(_ptr(dev_status), int(timeout_ms), _stream(stream))
+    _check("diffattn_selftest_timeout", rc)

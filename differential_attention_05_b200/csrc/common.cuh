@@ -162,16 +162,17 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t phase) {
 }
 
 // Bounded wait for the barrier phase with parity `phase` to complete. Returns false if
-// the time bound ran out (then it raises *abort) or *abort was raised by another thread;
-// the caller then stops issuing work.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, volatile int* abort) {
+// the time bound (`limit_ns`, by default DIFFATTN_WAIT_NS) ran out (then it raises *abort)
+// or *abort was raised by another thread; the caller then stops issuing work.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase, volatile int* abort,
+                                          uint64_t limit_ns = DIFFATTN_WAIT_NS) {
   if (mbar_try_wait(bar, phase)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, phase)) return true;
     if ((it & 31u) == 0) {
       if (*abort) return false;
-      if (global_ns() - t0 > DIFFATTN_WAIT_NS) {
+      if (global_ns() - t0 > limit_ns) {
         *abort = 1;
         return false;
       }

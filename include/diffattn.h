@@ -219,6 +219,26 @@ int diffattn_fwd_decode_static(const diffattn_decode_params* p, const void* q,
                                const void* k_cache, const void* v_cache, const int32_t* kv_len,
                                const float* lambda, void* out, int* dev_status, void* stream);
 
+/*
+ * diffattn_selftest_timeout -- exercises the kernels' bounded-wait path on purpose.
+ * (A diagnostic of this library, for tests; it computes nothing.)
+ *
+ * Every mbarrier wait in the kernels above gives up after a time bound and then reports
+ * DIFFATTN_ERR_TIMEOUT through the status word instead of hanging the GPU. This entry
+ * point launches one block of 128 threads that waits, with the same wait routine, for a
+ * barrier phase that nothing completes, bounded by timeout_ms instead of the kernels'
+ * 2-second bound. The wait runs out, the block writes DIFFATTN_ERR_TIMEOUT to *dev_status
+ * (left untouched if it already holds a non-zero code) and returns; the CUDA context stays
+ * usable.
+ *
+ *   dev_status  device int, required.
+ *   timeout_ms  1 .. 10000.
+ * Returns DIFFATTN_ERR_INVALID_ARG for a null status pointer or a timeout outside that
+ * range, DIFFATTN_ERR_CUDA if the launch fails, else DIFFATTN_OK (the timeout itself is
+ * reported on the device, when the block finishes).
+ */
+int diffattn_selftest_timeout(int* dev_status, int timeout_ms, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -150,3 +150,11 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "_lib", None)
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         B.load_library()
+
+
+def test_selftest_timeout_rejects(lib):
+    vp = ctypes.c_void_p
+    f = lib.diffattn_selftest_timeout
+    assert f(None, 100, None) == -1
+    assert f(vp(GOOD), 0, None) == -1
+    assert f(vp(GOOD), 10001, None) == -1
