@@ -78,6 +78,9 @@ def _load():
             ip, ctypes.c_int, ctypes.c_int, dp, ctypes.c_int]
         lib.oracle_decode_v2.restype = ctypes.c_int
         lib.oracle_decode_v2.argtypes = [dp, dp, dp, ip, dp] + [ctypes.c_int] * 5 + [dp, ctypes.c_int]
+        lib.oracle_decode_v1.restype = ctypes.c_int
+        lib.oracle_decode_v1.argtypes = [dp, dp, dp, ip, dp, ctypes.c_double] + [ctypes.c_int] * 5 + [
+            ctypes.c_double, dp, ctypes.c_int]
         lib.oracle_map_row_v2.restype = ctypes.c_int
         lib.oracle_map_row_v2.argtypes = [dp, dp] + [ctypes.c_int] * 6 + [dp, dp]
         _libs[path] = lib
@@ -194,6 +197,25 @@ def decode_v2(q, k, v, lam, kv_len=None, threads=None) -> np.ndarray:
                                   _dp(out), int(threads or default_threads()))
     if rc != 0:
         raise ValueError(f"oracle_decode_v2 failed: {rc}")
+    return out
+
+
+def decode_v1(q, k, v, lam, lambda_init_value: float, kv_len=None, apply_norm=True, eps=1e-5,
+              threads=None) -> np.ndarray:
+    """V1 decode. q: [B,H,2,d]; k: [B,L,H,2,d]; v: [B,L,H,2d]; kv_len: [B] or None
+    -> out [B,H,2d] (per-head RMSNorm and (1 - lambda_init) scale when apply_norm)."""
+    q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
+    B, H, two, d = q.shape
+    L = k.shape[1]
+    assert two == 2 and k.shape == (B, L, H, 2, d) and v.shape == (B, L, H, 2 * d)
+    assert lam.shape == (H,)
+    kl = None if kv_len is None else np.ascontiguousarray(np.asarray(kv_len, dtype=np.int32))
+    out = np.zeros((B, H, 2 * d), dtype=np.float64)
+    rc = _load().oracle_decode_v1(_dp(q), _dp(k), _dp(v), _ip(kl), _dp(lam), float(lambda_init_value),
+                                  B, L, H, d, int(bool(apply_norm)), float(eps), _dp(out),
+                                  int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_decode_v1 failed: {rc}")
     return out
 
 

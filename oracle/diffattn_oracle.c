@@ -137,7 +137,7 @@ typedef struct job job;
 typedef void (*unit_fn)(const job*, long unit, double* a1, double* a2);
 
 struct job {
-  int variant; /* 1 = V1 prefill, 2 = V2 prefill, 3 = V2 decode */
+  int variant; /* 1 = V1 prefill, 2 = V2 prefill, 3 = V2 decode, 4 = V1 decode */
   const double *q, *k, *v, *lam;
   const int* kv_len;
   const int* rows;
@@ -360,6 +360,52 @@ int oracle_decode_v2(const double* q, const double* k, const double* v, const in
   jb.n_units = (long)B * (Hq / 2);
   jb.scratch_len = L;
   jb.fn = dec_unit;
+  return run_job(&jb, nthreads);
+}
+
+/* ---- V1 decode ----------------------------------------------------------------------
+ * One new query per batch entry and head attends every cached key 0 .. kv_len[b]-1 of
+ * that head; both branches read their own cached keys and the one cached value row.
+ * q    : [B, H, 2, d]      (index 0 of the branch axis is branch 1)
+ * k    : [B, L, H, 2, d]   (L = cache capacity)
+ * v    : [B, L, H, 2d]
+ * kv_len : [B] or NULL (= L)
+ * lam  : [H]
+ * out  : [B, H, 2d], per-head RMSNorm and (1 - lambda_init) scale when apply_norm
+ * One unit = (b, h).
+ */
+static void dec1_unit(const job* jb, long unit, double* a1, double* a2) {
+  int H = jb->H;
+  int b = (int)(unit / H), h = (int)(unit % H);
+  int L = jb->N, d = jb->d, dv = 2 * d;
+  long tok_k = (long)H * 2 * d, tok_v = (long)H * dv;
+  const double* kb = jb->k + (long)b * L * tok_k + (long)h * 2 * d;
+  const double* vb = jb->v + (long)b * L * tok_v + (long)h * dv;
+  const double* q1 = jb->q + ((long)b * H + h) * 2 * d;
+  const double* q2 = q1 + d;
+  int n_keys = jb->kv_len ? jb->kv_len[b] : L;
+  double* o = jb->out + ((long)b * H + h) * dv;
+  diff_row(q1, q2, kb, kb + d, tok_k, vb, tok_v, n_keys, d, dv, jb->lam[h], a1, a2, o);
+  if (jb->apply_norm) rmsnorm_scale(o, dv, jb->eps, jb->lambda_init);
+}
+
+int oracle_decode_v1(const double* q, const double* k, const double* v, const int* kv_len,
+                     const double* lam, double lambda_init, int B, int L, int H, int d,
+                     int apply_norm, double eps, double* out, int nthreads) {
+  if (!q || !k || !v || !lam || !out || B < 0 || L < 0 || H <= 0 || d <= 0) return ORACLE_ERR_ARG;
+  if (kv_len) {
+    for (int b = 0; b < B; ++b)
+      if (kv_len[b] < 0 || kv_len[b] > L) return ORACLE_ERR_ARG;
+  }
+  job jb;
+  memset(&jb, 0, sizeof(jb));
+  jb.variant = 4;
+  jb.q = q; jb.k = k; jb.v = v; jb.lam = lam; jb.kv_len = kv_len;
+  jb.B = B; jb.N = L; jb.H = H; jb.d = d; jb.apply_norm = apply_norm;
+  jb.eps = eps; jb.lambda_init = lambda_init; jb.out = out;
+  jb.n_units = (long)B * H;
+  jb.scratch_len = L;
+  jb.fn = dec1_unit;
   return run_job(&jb, nthreads);
 }
 

@@ -123,6 +123,40 @@ def pin_lambda0_decode_is_softmax_attention():
         _close(out[b], ref[0::2], 1e-12, f"decode lambda=0 vs SDPA (b={b}, kv_len={n})")
 
 
+def pin_lambda0_decode_v1_is_softmax_attention():
+    """V1 decode with lambda = 0 and no norm: branch 1's softmax attention over the cache
+    (K_1 from the first half of each cached key row, V the whole 2d row)."""
+    r = _rng(11)
+    B, L, H, d = 2, 29, 3, 8
+    q = r.standard_normal((B, H, 2, d)); k = r.standard_normal((B, L, H, 2, d))
+    v = r.standard_normal((B, L, H, 2 * d))
+    kv_len = np.array([29, 5], dtype=np.int32)
+    out = oracle.decode_v1(q, k, v, np.zeros(H), 0.3, kv_len=kv_len, apply_norm=False, threads=2)
+    for b in range(B):
+        n = kv_len[b]
+        ref = _sdpa(q[b, :, 0][None, :, None, :].copy(), k[b, :n, :, 0].transpose(1, 0, 2)[None].copy(),
+                    v[b, :n].transpose(1, 0, 2)[None].copy(), False)[0, :, 0, :]
+        _close(out[b], ref, 1e-12, f"V1 decode lambda=0 vs SDPA (b={b}, kv_len={n})")
+
+
+def pin_decode_v1_is_last_prefill_row():
+    """A V1 decode step for a query at cache position n - 1 equals the last causal prefill
+    row over the same n keys, norm and scale included."""
+    r = _rng(12)
+    B, L, H, d = 2, 24, 2, 8
+    k = r.standard_normal((B, L, H, 2, d)); v = r.standard_normal((B, L, H, 2 * d))
+    q = r.standard_normal((B, H, 2, d))
+    lam = np.array([0.7, -0.4])
+    kv_len = np.array([24, 9], dtype=np.int32)
+    out = oracle.decode_v1(q, k, v, lam, 0.55, kv_len=kv_len, threads=2)
+    for b in range(B):
+        n = kv_len[b]
+        qq = r.standard_normal((1, n, H, 2, d))
+        qq[0, n - 1] = q[b]
+        pre = oracle.prefill_v1(qq, k[b:b + 1, :n], v[b:b + 1, :n], lam, 0.55, threads=1)
+        _close(out[b], pre[0, n - 1], 1e-13, f"V1 decode vs last prefill row (b={b})")
+
+
 # ---- invariants of the difference -----------------------------------------------------
 
 def pin_identical_branches_cancel():
@@ -140,6 +174,8 @@ def pin_identical_branches_cancel():
     k2 = r.standard_normal((B, N, Hkv, d)); v2 = r.standard_normal((B, N, Hkv, d))
     out2 = oracle.prefill_v2(q2, k2, v2, np.ones(Hq // 2), threads=1)
     _close(out2, 0.0, 1e-15, "V2 identical branches, lambda=1")
+    out3 = oracle.decode_v1(q[:, 5], k, v, np.ones(H), 0.2, kv_len=[17], apply_norm=False, threads=1)
+    _close(out3, 0.0, 1e-15, "V1 decode identical branches, lambda=1")
 
 
 def pin_rows_sum_to_one_minus_lambda():
@@ -162,6 +198,9 @@ def pin_rows_sum_to_one_minus_lambda():
     out3 = oracle.decode_v2(q2[:, 0], k2, np.ones((B, N, Hkv, d)), lam2, kv_len=[7], threads=1)
     _close(out3, np.broadcast_to((1.0 - lam2)[None, :, None], out3.shape), 1e-13,
            "decode rows sum to 1 - lambda")
+    out4 = oracle.decode_v1(q[:, 3], q, v, lam, 0.2, kv_len=[11], apply_norm=False, threads=1)
+    _close(out4, np.broadcast_to((1.0 - lam)[None, :, None], out4.shape), 1e-13,
+           "V1 decode rows sum to 1 - lambda")
 
 
 def pin_norm_first_row_closed_form():
@@ -278,6 +317,8 @@ ALL_PINS = [
     pin_lambda0_is_softmax_attention_v1,
     pin_lambda0_is_softmax_attention_v2,
     pin_lambda0_decode_is_softmax_attention,
+    pin_lambda0_decode_v1_is_softmax_attention,
+    pin_decode_v1_is_last_prefill_row,
     pin_identical_branches_cancel,
     pin_rows_sum_to_one_minus_lambda,
     pin_norm_first_row_closed_form,

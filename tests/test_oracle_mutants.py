@@ -28,15 +28,24 @@ MUTANTS = {
                              "d2 += lq2[(long)h * dim + c] * lk1[(long)h * dim + c];"),
     "lambda_init_rate": ("return 0.8 - 0.6 * exp(-0.3 * (double)(depth - 1));",
                          "return 0.8 - 0.6 * exp(-0.3 * (double)depth);"),
-    "v1_q2_is_q1": ("const double* q2 = q1 + d;", "const double* q2 = q1;"),
+    "v1_q2_is_q1": ("const double* q2 = q1 + d;\n    int n_keys = jb->causal", "const double* q2 = q1;\n    int n_keys = jb->causal"),
+    "v1_decode_q2_is_q1": ("const double* q2 = q1 + d;\n  int n_keys = jb->kv_len", "const double* q2 = q1;\n  int n_keys = jb->kv_len"),
     "v1_value_of_other_head": ("const double* vb = jb->v + (long)b * N * tok_v + (long)h * dv;",
                                "const double* vb = jb->v + (long)b * N * tok_v + (long)((h + 1) % H) * dv;"),
     "v2_gqa_modulo": ("int g1 = h1 / group, g2 = h2 / group;\n  long tok_q",
                       "int g1 = h1 % jb->Hkv, g2 = h2 % jb->Hkv;\n  long tok_q"),
     "v2_pairing_halves": ("int h1 = 2 * p, h2 = 2 * p + 1;\n  int g1 = h1 / group, g2 = h2 / group;\n  long tok_q",
                           "int h1 = p, h2 = p + P;\n  int g1 = h1 / group, g2 = h2 / group;\n  long tok_q"),
-    "decode_drops_last_key": ("int n_keys = jb->kv_len ? jb->kv_len[b] : L;",
-                              "int n_keys = jb->kv_len ? jb->kv_len[b] - 1 : L;"),
+    "decode_drops_last_key": ("int n_keys = jb->kv_len ? jb->kv_len[b] : L;\n  double* o = jb->out + ((long)b * P + p) * d;",
+                              "int n_keys = jb->kv_len ? jb->kv_len[b] - 1 : L;\n  double* o = jb->out + ((long)b * P + p) * d;"),
+    "v1_decode_drops_last_key": ("int n_keys = jb->kv_len ? jb->kv_len[b] : L;\n  double* o = jb->out + ((long)b * H + h) * dv;",
+                                 "int n_keys = jb->kv_len ? jb->kv_len[b] - 1 : L;\n  double* o = jb->out + ((long)b * H + h) * dv;"),
+    "v1_decode_branch2_reads_k1": ("diff_row(q1, q2, kb, kb + d, tok_k, vb, tok_v",
+                                   "diff_row(q1, q2, kb, kb, tok_k, vb, tok_v"),
+    "v1_decode_drops_norm": ("  if (jb->apply_norm) rmsnorm_scale(o, dv, jb->eps, jb->lambda_init);\n}\n\nint oracle_decode_v1",
+                             "}\n\nint oracle_decode_v1"),
+    "v1_decode_key_of_other_head": ("const double* kb = jb->k + (long)b * L * tok_k + (long)h * 2 * d;",
+                                    "const double* kb = jb->k + (long)b * L * tok_k + (long)((h + 1) % H) * 2 * d;"),
     "value_channel_shift": ("for (int c = 0; c < dv; ++c) o[c] += w * vj[c];",
                                "for (int c = 0; c < dv; ++c) o[c] += w * vj[(c + 1) % dv];"),
 }
