@@ -2,7 +2,7 @@
 """Benchmark of the differential attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload c2|c3|c4|c5] [--no-secondary]
+                    [--workload c2|c3|c4|c5|d1] [--no-secondary]
 
 A step is one pass of the hot path over one batch of synthetic input: the on-device
 lambda re-parameterisation followed by the fused prefill (or the split-KV decode for the
@@ -46,6 +46,8 @@ def workload_inputs(name: str, batch: int = 0):
     from differential_attention_05_b200 import synth
     if name == "c4" and batch:
         return synth.v2_decode(B=batch, name=f"v2_bf16_decode_b{batch}_l32768_hq64_hkv8_d128")
+    if name == "d1":
+        return synth.v1_decode(B=batch) if batch else synth.v1_decode()
     return {"c2": synth.config2, "c3": synth.config3, "c4": synth.config4, "c5": synth.config5}[name]()
 
 
@@ -56,6 +58,14 @@ def prefill_flops(inp) -> float:
     pairs = inp.N * (inp.N + 1) / 2 if inp.causal else float(inp.N) * inp.N
     per = 12 * inp.d * inp.H if inp.variant == 1 else 4 * inp.d * inp.H
     return float(inp.B) * pairs * per
+
+
+def workload_decode_bytes(inp) -> float:
+    """Cache bytes one decode step reads: V2 K and V of width d per KV head; V1 K rows
+    (K_1 | K_2, 2d) and V rows (2d) per head."""
+    if inp.variant == 1:
+        return decode_bytes(inp.B, inp.N, inp.H, 2 * inp.d)
+    return decode_bytes(inp.B, inp.N, inp.Hkv, inp.d)
 
 
 def decode_bytes(B, L, Hkv, d) -> float:
@@ -208,11 +218,15 @@ def run_ours(args, rank, world, device):
     stream = torch.cuda.current_stream(device)
     decode = inp.mode == "decode"
     if decode:
-        out = torch.empty((inp.B, inp.H // 2, inp.d), dtype=torch.bfloat16, device=device)
-        p = da._binding.decode_params(q, k, v, out)
+        if inp.variant == 1:
+            out = torch.empty((inp.B, inp.H, 2 * inp.d), dtype=torch.bfloat16, device=device)
+            p = da._binding.decode_params_v1(q, k, v, out)
+        else:
+            out = torch.empty((inp.B, inp.H // 2, inp.d), dtype=torch.bfloat16, device=device)
+            p = da._binding.decode_params(q, k, v, out)
         ws = torch.empty(da._binding.diffattn_decode_workspace_size(p), dtype=torch.uint8,
                          device=device)
-        work = decode_bytes(inp.B, inp.N, inp.Hkv, inp.d)
+        work = workload_decode_bytes(inp)
         unit, metric = "GB/s", "diff-attn decode KV GB/s at 1 B200"
     else:
         out = (torch.empty((inp.B, inp.N, inp.H, 2 * inp.d), dtype=torch.bfloat16, device=device)
@@ -228,7 +242,10 @@ def run_ours(args, rank, world, device):
         da.diffattn_lambda(*vecs, depth=inp.depth, lambda_out=lam, lambda_init_out=li)
 
     def main_kernel():
-        if decode:
+        if decode and inp.variant == 1:
+            da.diffattn_fwd_decode_v1(q, k, v, lam, li, out=out, apply_norm=inp.apply_norm,
+                                      norm_eps=inp.eps, workspace=ws)
+        elif decode:
             da.diffattn_fwd_decode(q, k, v, lam, out=out, workspace=ws)
         else:
             da.diffattn_fwd_prefill(q, k, v, lam, li, out=out, causal=inp.causal,
@@ -312,7 +329,8 @@ def run_ours(args, rank, world, device):
     e2e_ms = max_over_ranks(e2e_ms, dist, device)
     e2e_val = job_rate(world, work, e2e_steps, e2e_ms, 1e9 if decode else 1e12)
 
-    kernel_name = "decode_split_kernel" if decode else f"prefill_v{inp.variant}_kernel"
+    kernel_name = (("decode_v1_split_kernel" if inp.variant == 1 else "decode_split_kernel")
+                   if decode else f"prefill_v{inp.variant}_kernel")
     # decode traffic was captured at batch 8 and grows in proportion to the batch
     traffic = measured_traffic(kernel_name, inp.B / 8.0 if decode else 1.0)
     if traffic is not None and not decode and inp.name not in (
@@ -345,7 +363,8 @@ def run_ours(args, rank, world, device):
             "bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": runit,
             "frac": round(achieved / peak, 4), "traffic": traffic,
             "peak_source": f"{peaks['source']} ({'burst bf16' if bound == 'tensor' else 'HBM copy'})",
-            "kernel": ("decode_split_kernel + decode_combine_kernel" if decode else kernel_name),
+            "kernel": (kernel_name + (" + decode_v1_combine_kernel" if inp.variant == 1 else
+                                      " + decode_combine_kernel") if decode else kernel_name),
             "avg_kernel_ms": round(kern_avg, 5),
         },
         "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": int(h2d),
@@ -362,9 +381,10 @@ def run_ours(args, rank, world, device):
 
 
 def secondary(device, peaks, torch, da):
-    """Other rows of the hot path, timed alone: V2 prefill (64/8 heads, d=128, N=16384)
-    and V2 decode (batch 64, cache 32768). Inputs are drawn on the device (seeded N(0,1),
-    same shapes) to keep the run short; both exceed L2."""
+    """Other rows of the hot path, timed alone: V2 prefill (64/8 heads, d=128, N=16384),
+    V2 decode (batch 64, cache 32768) and V1 decode (batch 32, cache 32768, 16 heads,
+    d=64). Inputs are drawn on the device (seeded N(0,1), same shapes) to keep the run
+    short; all exceed L2."""
     res = {}
     g = torch.Generator(device=device)
     g.manual_seed(1002)
@@ -408,6 +428,31 @@ def secondary(device, peaks, torch, da):
     res["decode"] = {"workload": "v2_bf16_decode_b64_l32768_hq64_hkv8_d128", "ms": round(ms, 4),
                      "GB/s": round(by / ms / 1e6, 1),
                      "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    del q, k, v, out, ws
+    torch.cuda.empty_cache()
+    # V1 decode: batch 32, cache 32768, 16 heads, d = 64 (the same cache bytes as above)
+    B, L, H, d1 = 32, 32768, 16, 64
+    q = (torch.randn((B, H, 2, d1), generator=g, device=device) / 8).bfloat16()
+    k = (torch.randn((B, L, H, 2, d1), generator=g, device=device) / 8).bfloat16()
+    v = (torch.randn((B, L, H, 2 * d1), generator=g, device=device) / 8).bfloat16()
+    lam1 = torch.full((H,), 0.8, dtype=torch.float32, device=device)
+    li = torch.full((1,), 0.78, dtype=torch.float32, device=device)
+    out = torch.empty((B, H, 2 * d1), dtype=torch.bfloat16, device=device)
+    p = da._binding.decode_params_v1(q, k, v, out)
+    ws = torch.empty(da._binding.diffattn_decode_workspace_size(p), dtype=torch.uint8, device=device)
+    for _ in range(3):
+        da.diffattn_fwd_decode_v1(q, k, v, lam1, li, out=out, workspace=ws)
+    es = [(torch.cuda.Event(True), torch.cuda.Event(True)) for _ in range(10)]
+    for a, b in es:
+        a.record()
+        da.diffattn_fwd_decode_v1(q, k, v, lam1, li, out=out, workspace=ws)
+        b.record()
+    torch.cuda.synchronize(device)
+    ms = statistics.median(a.elapsed_time(b) for a, b in es)
+    by = decode_bytes(B, L, H, 2 * d1)
+    res["decode_v1"] = {"workload": "v1_bf16_decode_b32_l32768_h16_d64", "ms": round(ms, 4),
+                        "GB/s": round(by / ms / 1e6, 1),
+                        "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
     del q, k, v, out, ws
     torch.cuda.empty_cache()
     return res
@@ -472,8 +517,13 @@ def oracle_decode_sample(inp, seconds):
     n = 0
     while True:
         b = n % inp.B
-        oracle.decode_v2(synth.bf16_to_f32(inp.q[b:b + 1]), synth.bf16_to_f32(inp.k[b:b + 1]),
-                         synth.bf16_to_f32(inp.v[b:b + 1]), lam)
+        if inp.variant == 1:
+            oracle.decode_v1(synth.bf16_to_f32(inp.q[b:b + 1]), synth.bf16_to_f32(inp.k[b:b + 1]),
+                             synth.bf16_to_f32(inp.v[b:b + 1]), lam, oracle.lambda_init(inp.depth),
+                             apply_norm=inp.apply_norm, eps=inp.eps)
+        else:
+            oracle.decode_v2(synth.bf16_to_f32(inp.q[b:b + 1]), synth.bf16_to_f32(inp.k[b:b + 1]),
+                             synth.bf16_to_f32(inp.v[b:b + 1]), lam)
         n += 1
         if time.perf_counter() - t0 >= seconds:
             break
@@ -486,7 +536,7 @@ def cpu_baseline(inp, seconds=12.0):
     cores = oracle.default_threads()
     if inp.mode == "decode":
         n, dt = oracle_decode_sample(inp, seconds)
-        val = n * decode_bytes(1, inp.N, inp.Hkv, inp.d) / dt / 1e9
+        val = n * workload_decode_bytes(inp) / inp.B / dt / 1e9
         return {"value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                 "sample": f"{n} batch entries of {inp.name}, {dt:.1f} s"}
     orc = OracleRows(inp)
@@ -513,7 +563,7 @@ def run_reference(args, rank, world):
                 times.append((n, dt))
         total_units = sum(n for n, _ in times)
         total_s = sum(dt for _, dt in times)
-        value = total_units * decode_bytes(1, inp.N, inp.Hkv, inp.d) / total_s / 1e9
+        value = total_units * workload_decode_bytes(inp) / inp.B / total_s / 1e9
         unit, metric = "GB/s", "diff-attn decode KV GB/s at 1 B200"
         sample = f"whole batch entries of {inp.name} ({total_units} in {total_s:.1f} s)"
     else:
@@ -555,7 +605,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("c2", "c3", "c4", "c5"), default="c2")
+    ap.add_argument("--workload", choices=("c2", "c3", "c4", "c5", "d1"), default="c2")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="decode workload only: smaller batch (profiling runs)")

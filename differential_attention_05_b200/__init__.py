@@ -10,6 +10,7 @@ from ._binding import (  # noqa: F401
     diffattn_fwd_prefill,
     diffattn_fwd_decode,
     diffattn_fwd_decode_static,
+    diffattn_fwd_decode_v1,
     diffattn_selftest_timeout,
     diffattn_decode_workspace_size,
     diffattn_status_string,
@@ -23,6 +24,7 @@ __all__ = [
     "diffattn_fwd_prefill",
     "diffattn_fwd_decode",
     "diffattn_fwd_decode_static",
+    "diffattn_fwd_decode_v1",
     "diffattn_selftest_timeout",
     "diffattn_decode_workspace_size",
     "diffattn_status_string",

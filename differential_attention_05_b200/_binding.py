@@ -35,6 +35,7 @@ EXPORTS = (
     "diffattn_decode_workspace_size",
     "diffattn_fwd_decode",
     "diffattn_fwd_decode_static",
+    "diffattn_fwd_decode_v1",
     "diffattn_selftest_timeout",
 )
 
@@ -117,6 +118,9 @@ def load_library():
     lib.diffattn_fwd_decode_static.restype = i32
     lib.diffattn_fwd_decode_static.argtypes = [ctypes.POINTER(DecodeParams), vp, vp, vp, vp, f32p,
                                                vp, vp, vp]
+    lib.diffattn_fwd_decode_v1.restype = i32
+    lib.diffattn_fwd_decode_v1.argtypes = [ctypes.POINTER(DecodeParams), vp, vp, vp, vp, f32p, f32p,
+                                           i32, ctypes.c_float, vp, vp, ctypes.c_size_t, vp, vp]
     lib.diffattn_selftest_timeout.restype = i32
     lib.diffattn_selftest_timeout.argtypes = [vp, i32, vp]
     _lib = lib
@@ -242,6 +246,22 @@ def decode_params(q, k_cache, v_cache, out, num_splits=0) -> DecodeParams:
     return p
 
 
+def decode_params_v1(q, k_cache, v_cache, out, num_splits=0) -> DecodeParams:
+    """V1: q [B,H,2,d], k_cache [B,L,H,2,d], v_cache [B,L,H,2d], out [B,H,2d]."""
+    p = DecodeParams()
+    B, H, two, d = q.shape
+    _, L = k_cache.shape[:2]
+    if two != 2 or tuple(k_cache.stride()[:3]) != tuple(v_cache.stride()[:3]):
+        raise DiffattnError("diffattn_fwd_decode_v1", -1)
+    p.variant, p.dtype = DIFFATTN_V1, _dtype_code(q)
+    p.batch, p.max_kv_len, p.n_q_heads, p.n_kv_heads, p.head_dim = B, L, H, H, d
+    p.num_splits = int(num_splits)
+    p.q_strides[:] = q.stride()[:2]
+    p.kv_strides[:] = k_cache.stride()[:3]
+    p.o_strides[:] = out.stride()[:2]
+    return p
+
+
 def diffattn_decode_workspace_size(p: DecodeParams) -> int:
     n = ctypes.c_size_t(0)
     _check("diffattn_decode_workspace_size",
@@ -266,6 +286,30 @@ def diffattn_fwd_decode(q, k_cache, v_cache, lam, kv_len=None, out=None, workspa
                                  _ptr(kv_len), _ptr(lam), _ptr(out), _ptr(workspace), ws_bytes,
                                  _ptr(dev_status), _stream(stream))
     _check("diffattn_fwd_decode", rc)
+    return out
+
+
+def diffattn_fwd_decode_v1(q, k_cache, v_cache, lam, lambda_init=None, kv_len=None, out=None,
+                           apply_norm=True, norm_eps=1e-5, workspace=None, num_splits=0,
+                           dev_status=None, stream=None):
+    """Split-KV differential decode (V1). q [B,H,2,d], k_cache [B,L,H,2,d],
+    v_cache [B,L,H,2d] -> out [B,H,2d], per-head RMSNorm and (1 - lambda_init) scale when
+    apply_norm."""
+    import torch
+    lib = load_library()
+    B, H, _, d = q.shape
+    if out is None:
+        out = torch.empty((B, H, 2 * d), dtype=q.dtype, device=q.device)
+    p = decode_params_v1(q, k_cache, v_cache, out, num_splits)
+    need = diffattn_decode_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib.diffattn_fwd_decode_v1(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(kv_len), _ptr(lam), _ptr(lambda_init), int(bool(apply_norm)),
+                                    float(norm_eps), _ptr(out), _ptr(workspace), ws_bytes,
+                                    _ptr(dev_status), _stream(stream))
+    _check("diffattn_fwd_decode_v1", rc)
     return out
 
 

@@ -163,7 +163,41 @@ static int decode_check(const diffattn_decode_params* p, int* splits, int* split
   return DIFFATTN_OK;
 }
 
+// V1 decode: one (K_1 | K_2, V) cache per differential head, d = 64.
+static int decode_v1_check(const diffattn_decode_params* p, int* splits, int* split_len) {
+  if (!p) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->max_kv_len < 0 || p->n_q_heads < 1 || p->n_kv_heads < 1 ||
+      p->head_dim < 1 || p->num_splits < 0)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (p->variant != DIFFATTN_V1) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->dtype != DIFFATTN_BF16) return p->dtype == DIFFATTN_F32 ? DIFFATTN_ERR_UNSUPPORTED
+                                                                 : DIFFATTN_ERR_INVALID_ARG;
+  if (p->n_q_heads != p->n_kv_heads) return DIFFATTN_ERR_INVALID_ARG;  // one cache per head
+  if (p->head_dim != 64) return DIFFATTN_ERR_UNSUPPORTED;
+  if (!strides_ok(p->q_strides, 2) || !strides_ok(p->kv_strides, 3) || !strides_ok(p->o_strides, 2))
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (p->batch > 65535 || p->n_q_heads > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  int s = p->num_splits ? p->num_splits
+                        : decode_v1_default_splits(p->batch, p->max_kv_len, p->n_q_heads);
+  const int L = p->max_kv_len;
+  int len = (L + s - 1) / (s > 0 ? s : 1);
+  len = ((len + kDecodeChunk - 1) / kDecodeChunk) * kDecodeChunk;
+  if (len < kDecodeChunk) len = kDecodeChunk;
+  s = (L + len - 1) / len;
+  if (s < 1) s = 1;
+  if (s > 65535) return DIFFATTN_ERR_UNSUPPORTED;
+  *splits = s;
+  *split_len = len;
+  return DIFFATTN_OK;
+}
+
 static size_t decode_ws_bytes(const diffattn_decode_params* p, int splits) {
+  if (p->variant == DIFFATTN_V1) {
+    // per (b, h, split) and branch: 2d partial outputs, then (max, sum)
+    const size_t recs = (size_t)p->batch * p->n_q_heads * splits * 2;
+    const size_t o_bytes = ((recs * 2 * p->head_dim * sizeof(float)) + 255) & ~(size_t)255;
+    return o_bytes + recs * 2 * sizeof(float);
+  }
   const size_t recs = (size_t)p->batch * p->n_q_heads * splits;
   const size_t o_bytes = ((recs * p->head_dim * sizeof(float)) + 255) & ~(size_t)255;
   return o_bytes + recs * 2 * sizeof(float);
@@ -172,7 +206,8 @@ static size_t decode_ws_bytes(const diffattn_decode_params* p, int splits) {
 int diffattn_decode_workspace_size(const diffattn_decode_params* p, size_t* bytes) {
   if (!bytes) return DIFFATTN_ERR_INVALID_ARG;
   int splits = 0, len = 0;
-  int rc = decode_check(p, &splits, &len);
+  int rc = (p && p->variant == DIFFATTN_V1) ? decode_v1_check(p, &splits, &len)
+                                            : decode_check(p, &splits, &len);
   if (rc != DIFFATTN_OK) return rc;
   *bytes = decode_ws_bytes(p, splits);
   return DIFFATTN_OK;
@@ -218,6 +253,56 @@ int diffattn_fwd_decode(const diffattn_decode_params* p, const void* q, const vo
                                      (((recs * a.d * sizeof(float)) + 255) & ~(size_t)255));
   a.dev_status = dev_status;
   return from_cuda(launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+int diffattn_fwd_decode_v1(const diffattn_decode_params* p, const void* q, const void* k_cache,
+                           const void* v_cache, const int32_t* kv_len, const float* lambda,
+                           const float* lambda_init, int apply_norm, float norm_eps, void* out,
+                           void* workspace, size_t workspace_bytes, int* dev_status,
+                           void* stream) {
+  int splits = 0, len = 0;
+  int rc = decode_v1_check(p, &splits, &len);
+  if (rc != DIFFATTN_OK) return rc;
+  if (apply_norm != 0 && apply_norm != 1) return DIFFATTN_ERR_INVALID_ARG;
+  if (apply_norm && !(norm_eps >= 0.f && isfinite(norm_eps))) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->batch == 0) return DIFFATTN_OK;
+  if (!q || !k_cache || !v_cache || !lambda || !out) return DIFFATTN_ERR_INVALID_ARG;
+  if (apply_norm && !lambda_init) return DIFFATTN_ERR_INVALID_ARG;
+  const size_t need = decode_ws_bytes(p, splits);
+  if (!workspace || workspace_bytes < need) return DIFFATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIFFATTN_ERR_MISALIGNED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+    return DIFFATTN_ERR_MISALIGNED;
+  if (p->q_strides[0] % 8 || p->q_strides[1] % 8 || p->kv_strides[0] % 8 || p->kv_strides[1] % 8 ||
+      p->kv_strides[2] % 8 || p->o_strides[0] % 8 || p->o_strides[1] % 8)
+    return DIFFATTN_ERR_MISALIGNED;
+  DecodeArgs a;
+  memset(&a, 0, sizeof(a));
+  a.B = p->batch;
+  a.L = p->max_kv_len;
+  a.Hq = p->n_q_heads;
+  a.Hkv = p->n_kv_heads;
+  a.d = p->head_dim;
+  a.splits = splits;
+  a.split_len = len;
+  memcpy(a.qs, p->q_strides, sizeof(a.qs));
+  memcpy(a.kvs, p->kv_strides, sizeof(a.kvs));
+  memcpy(a.os, p->o_strides, sizeof(a.os));
+  a.q = q;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.kv_len = kv_len;
+  a.lambda = lambda;
+  a.lambda_init = lambda_init;
+  a.apply_norm = apply_norm;
+  a.eps = norm_eps;
+  a.out = out;
+  const size_t recs = (size_t)a.B * a.Hq * splits * 2;
+  a.ws_o = static_cast<float*>(workspace);
+  a.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                     (((recs * 2 * a.d * sizeof(float)) + 255) & ~(size_t)255));
+  a.dev_status = dev_status;
+  return from_cuda(launch_decode_v1(a, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -28,7 +28,7 @@ struct PrefillArgs {
 };
 
 struct DecodeArgs {
-  int B, L, Hq, Hkv, d;
+  int B, L, Hq, Hkv, d;   // V1: Hq = Hkv = H differential heads, d = branch width
   int splits, split_len;  // keys per split (multiple of the chunk size)
   int64_t qs[2], kvs[3], os[2];
   const void* q;
@@ -36,9 +36,12 @@ struct DecodeArgs {
   const void* v;
   const int32_t* kv_len;
   const float* lambda;
+  const float* lambda_init;  // V1, read when apply_norm
+  int apply_norm;            // V1
+  float eps;                 // V1
   void* out;
-  float* ws_o;   // [B, Hq, splits, d]
-  float* ws_ml;  // [B, Hq, splits, 2]
+  float* ws_o;   // V2: [B, Hq, splits, d]; V1: [B, H, splits, 2 branches, 2d]
+  float* ws_ml;  // V2: [B, Hq, splits, 2];  V1: [B, H, splits, 2 branches, 2]
   int* dev_status;
 };
 
@@ -58,5 +61,10 @@ cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream);
 constexpr int kDecodeChunk = 64;  // keys per pipeline stage
 int decode_default_splits(int B, int L, int Hkv);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// split-KV decode, V1 (bf16, d = 64: K rows K_1 | K_2, value rows of 2d), fp32 on the CUDA
+// cores; per-head RMSNorm and (1 - lambda_init) scale in the merge
+int decode_v1_default_splits(int B, int L, int H);
+cudaError_t launch_decode_v1(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace diffattn

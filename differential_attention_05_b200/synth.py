@@ -187,6 +187,31 @@ def decode_cache_slice(b: int, L=32768, Hkv=8, d=128, seed=1003):
     return k, v
 
 
+def v1_decode(B=32, L=32768, H=16, d=64, depth=12, seed=1006, kv_len=None, name=None,
+              scale=None) -> Inputs:
+    """V1 decode, bf16: q [B,H,2,d]; cache k [B,L,H,2,d], v [B,L,H,2d]; the V1 layer's
+    heads and widths (C2: 16 heads, d = 64, depth 12) over a decode cache holding the same
+    bytes as the V2 decode workload (8.6 GB at B=32, L=32768). Values N(0,1) scaled by
+    1/sqrt(d) like the V1 layer inputs; one stream per batch entry (see
+    decode_cache_slice_v1)."""
+    sc = scale if scale is not None else 1.0 / math.sqrt(d)
+    q = _normal_sliced(seed, _T_Q, (B, H, 2, d), sc)
+    k = _normal_sliced(seed, _T_K, (B, L, H, 2, d), sc)
+    v = _normal_sliced(seed, _T_V, (B, L, H, 2 * d), sc)
+    kl = None if kv_len is None else np.asarray(kv_len, dtype=np.int32)
+    return Inputs(name or f"v1_bf16_decode_b{B}_l{L}_h{H}_d{d}", 1, "decode", "bf16",
+                  B, L, H, H, d, depth, q, k, v, *_lambda_vectors(seed, H, d),
+                  causal=False, apply_norm=True, kv_len=kl)
+
+
+def decode_cache_slice_v1(b: int, L=32768, H=16, d=64, seed=1006, scale=None):
+    """Batch entry b of the V1 decode cache (k, v) as bf16 bits, identical to v1_decode's."""
+    sc = scale if scale is not None else 1.0 / math.sqrt(d)
+    k = bf16_bits(_normal(seed, _T_K, (L, H, 2, d), sc, slice_=b))
+    v = bf16_bits(_normal(seed, _T_V, (L, H, 2 * d), sc, slice_=b))
+    return k, v
+
+
 def signal_plus_noise(N=65536, Hq=64, Hkv=8, d=128, depth=24, seed=1004, name=None) -> Inputs:
     """Long-context signal-plus-noise workload (bf16, causal, B=1).
 

@@ -143,7 +143,8 @@ int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const 
                          int* dev_status, void* stream);
 
 /*
- * Decode parameters (V2 only; bf16 only).
+ * Decode parameters (bf16 only). V2 (diffattn_fwd_decode) below; V1 uses the same struct
+ * with the layouts given at diffattn_fwd_decode_v1.
  *   q       : [B, Hq, d]        one new query token per batch entry
  *   k_cache : [B, L, Hkv, d]    L = max_kv_len (cache capacity)
  *   v_cache : [B, L, Hkv, d]    same strides as k_cache
@@ -155,7 +156,7 @@ int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const 
  * 16-byte aligned base pointers, strides multiples of 8 elements.
  */
 typedef struct {
-  int32_t variant;    /* DIFFATTN_V2 */
+  int32_t variant;    /* DIFFATTN_V2 (diffattn_fwd_decode) or DIFFATTN_V1 (_v1) */
   int32_t dtype;      /* DIFFATTN_BF16 */
   int32_t batch;      /* B >= 0 */
   int32_t max_kv_len; /* L >= 0 */
@@ -169,8 +170,8 @@ typedef struct {
 } diffattn_decode_params;
 
 /*
- * diffattn_decode_workspace_size -- device workspace bytes diffattn_fwd_decode needs
- * for these parameters (written to *bytes, a HOST pointer). The workspace holds the
+ * diffattn_decode_workspace_size -- device workspace bytes diffattn_fwd_decode (V2) or
+ * diffattn_fwd_decode_v1 (V1, by p->variant) needs for these parameters (written to *bytes, a HOST pointer). The workspace holds the
  * per-split partial softmax states; its contents need no initialisation.
  */
 int diffattn_decode_workspace_size(const diffattn_decode_params* p, size_t* bytes);
@@ -190,6 +191,38 @@ int diffattn_decode_workspace_size(const diffattn_decode_params* p, size_t* byte
 int diffattn_fwd_decode(const diffattn_decode_params* p, const void* q, const void* k_cache,
                         const void* v_cache, const int32_t* kv_len, const float* lambda, void* out,
                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+
+/*
+ * diffattn_fwd_decode_v1 -- split-KV differential decode for V1 ("Differential Attention
+ * (V2)", "V1 vs V2": each V1 head has two query/key branches of width d and one value
+ * of width 2d; the per-head RMSNorm and the (1 - lambda_init) scale follow the
+ * difference). Each (batch, head, split) block streams its slice of the cache once --
+ * the value rows serve both branches -- and keeps one running (max, sum, output) per
+ * branch; a second kernel merges the splits, forms O_1/l_1 - lambda O_2/l_2, and applies
+ * the norm and scale. fp32 arithmetic throughout (no bf16 rounding of probabilities).
+ *
+ * Parameters: diffattn_decode_params with variant = DIFFATTN_V1, dtype = DIFFATTN_BF16,
+ * n_q_heads = n_kv_heads = H (differential heads), head_dim = d = 64 in this build.
+ *   q       : [B, H, 2, d]      branch 2 at +d inside each head's row
+ *   k_cache : [B, L, H, 2, d]   branch 2's key at +d inside each cached row
+ *   v_cache : [B, L, H, 2d]     same strides as k_cache
+ *   kv_len  : int32 [B] or NULL (NULL = L); the query attends keys 0 .. kv_len[b]-1
+ *   out     : [B, H, 2d]
+ * Strides (elements): q {batch, head}, kv {batch, token, head}, out {batch, head};
+ * 16-byte aligned base pointers, strides multiples of 8 elements.
+ *   lambda      : float32 [H], device
+ *   lambda_init : float32 [1], device; read only when apply_norm = 1 (may be NULL otherwise)
+ *   apply_norm  : 1 = RMSNorm over the 2d channels (eps = norm_eps >= 0, unit gain) and
+ *                 x (1 - lambda_init); 0 = the plain difference
+ *   workspace   : >= diffattn_decode_workspace_size(p) bytes, 256-byte aligned
+ * kv_len[b] = 0 gives a zero output row. Errors as for diffattn_fwd_decode; a V2 parameter
+ * set returns DIFFATTN_ERR_INVALID_ARG.
+ */
+int diffattn_fwd_decode_v1(const diffattn_decode_params* p, const void* q, const void* k_cache,
+                           const void* v_cache, const int32_t* kv_len, const float* lambda,
+                           const float* lambda_init, int apply_norm, float norm_eps, void* out,
+                           void* workspace, size_t workspace_bytes, int* dev_status,
+                           void* stream);
 
 /*
  * diffattn_fwd_decode_static -- diffattn_fwd_decode without a caller-provided workspace.

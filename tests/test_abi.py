@@ -121,8 +121,52 @@ def test_decode_workspace_size(lib):
     p = _decode_params(Hq=64, Hkv=16)  # group of 4: not this build's decode shape
     assert lib.diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == -2
     p = _decode_params()
-    p.variant = B.DIFFATTN_V1
+    p.variant = B.DIFFATTN_V1  # V1 needs one cache per head (Hq == Hkv)
+    assert lib.diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == -1
+
+
+def _decode_params_v1(B_=4, L=1000, H=16, d=64, splits=0):
+    p = B.DecodeParams()
+    p.variant, p.dtype = B.DIFFATTN_V1, B.DIFFATTN_BF16
+    p.batch, p.max_kv_len, p.n_q_heads, p.n_kv_heads, p.head_dim, p.num_splits = B_, L, H, H, d, splits
+    p.q_strides[:] = (H * 2 * d, 2 * d)
+    p.kv_strides[:] = (L * H * 2 * d, H * 2 * d, 2 * d)
+    p.o_strides[:] = (H * 2 * d, 2 * d)
+    return p
+
+
+def test_decode_v1_workspace_size(lib):
+    n = ctypes.c_size_t(0)
+    p = _decode_params_v1(B_=4, L=1000, H=16, splits=3)
+    assert lib.diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    # 3 splits; per (b, h, split) two branch records of 2d = 128 floats and (max, sum)
+    recs = 4 * 16 * 3 * 2
+    assert n.value == ((recs * 128 * 4 + 255) // 256) * 256 + recs * 2 * 4
+    p = _decode_params_v1(d=128)  # this build's V1 decode takes d = 64
     assert lib.diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == -2
+
+
+def test_decode_v1_rejects(lib):
+    vp = ctypes.c_void_p
+    f = lib.diffattn_fwd_decode_v1
+    p = _decode_params_v1(B_=2, L=512, H=4)
+    n = ctypes.c_size_t(0)
+    assert lib.diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    ptrs = [vp(GOOD), vp(GOOD + 4096), vp(GOOD + 8192), None, vp(GOOD + 12288)]
+    ws = vp(GOOD * 4)
+    # V2 parameters through the V1 entry point
+    p2 = _decode_params(B_=2, L=512)
+    assert f(ctypes.byref(p2), *ptrs, vp(GOOD), 1, 1e-5, vp(GOOD + 16384), ws, n.value, None, None) == -1
+    # apply_norm without lambda_init, a bad flag, a bad eps
+    assert f(ctypes.byref(p), *ptrs, None, 1, 1e-5, vp(GOOD + 16384), ws, n.value, None, None) == -1
+    assert f(ctypes.byref(p), *ptrs, vp(GOOD), 2, 1e-5, vp(GOOD + 16384), ws, n.value, None, None) == -1
+    assert f(ctypes.byref(p), *ptrs, vp(GOOD), 1, -1.0, vp(GOOD + 16384), ws, n.value, None, None) == -1
+    # workspace too small / missing / misaligned; misaligned query
+    assert f(ctypes.byref(p), *ptrs, vp(GOOD), 1, 1e-5, vp(GOOD + 16384), ws, n.value - 1, None, None) == -4
+    assert f(ctypes.byref(p), *ptrs, vp(GOOD), 1, 1e-5, vp(GOOD + 16384), None, n.value, None, None) == -4
+    assert f(ctypes.byref(p), *ptrs, vp(GOOD), 1, 1e-5, vp(GOOD + 16384), vp(GOOD * 4 + 16), n.value, None, None) == -3
+    bad = [vp(GOOD + 2)] + ptrs[1:]
+    assert f(ctypes.byref(p), *bad, vp(GOOD), 1, 1e-5, vp(GOOD + 16384), ws, n.value, None, None) == -3
 
 
 def test_decode_rejects_small_workspace(lib):
