@@ -76,6 +76,12 @@ def _load():
         lib.oracle_prefill_v2.restype = ctypes.c_int
         lib.oracle_prefill_v2.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 6 + [
             ip, ctypes.c_int, ctypes.c_int, dp, ctypes.c_int]
+        lib.oracle_prefill_v1_range.restype = ctypes.c_int
+        lib.oracle_prefill_v1_range.argtypes = [dp, dp, dp, dp, ctypes.c_double] + [ctypes.c_int] * 8 + [
+            ctypes.c_double, ip, ctypes.c_int, ctypes.c_int, dp, ctypes.c_int]
+        lib.oracle_prefill_v2_range.restype = ctypes.c_int
+        lib.oracle_prefill_v2_range.argtypes = [dp, dp, dp, dp] + [ctypes.c_int] * 8 + [
+            ip, ctypes.c_int, ctypes.c_int, dp, ctypes.c_int]
         lib.oracle_decode_v2.restype = ctypes.c_int
         lib.oracle_decode_v2.argtypes = [dp, dp, dp, ip, dp] + [ctypes.c_int] * 5 + [dp, ctypes.c_int]
         lib.oracle_decode_v1.restype = ctypes.c_int
@@ -134,54 +140,65 @@ def _rows(rows, N):
 
 
 def prefill_v1(q, k, v, lam, lambda_init_value: float, causal=True, apply_norm=True,
-               eps=1e-5, rows=None, threads=None, q_rows=None) -> np.ndarray:
-    """V1 prefill. q,k: [B,N,H,2,d]; v: [B,N,H,2d]; lam: [H] -> out [B,R,H,2d].
-    With rows and q_rows ([B,R,H,2,d], the queries at those positions), q may be None."""
+               eps=1e-5, rows=None, threads=None, q_rows=None, window=0,
+               n_queries=None) -> np.ndarray:
+    """V1 prefill. q: [B,Nq,H,2,d]; k: [B,Nk,H,2,d]; v: [B,Nk,H,2d]; lam: [H]
+    -> out [B,R,H,2d]. Nq <= Nk queries are the last Nq positions (chunked prefill); a
+    causal sliding window of `window` keys when window > 0. With rows and q_rows
+    ([B,R,H,2,d], the queries at those positions), q may be None (then Nq = n_queries,
+    default Nk)."""
     k, v, lam = _f64(k), _f64(v), _f64(lam)
-    B, N, H, two, d = k.shape
-    assert two == 2 and v.shape == (B, N, H, 2 * d) and lam.shape == (H,)
-    r, R = _rows(rows, N)
+    B, Nk, H, two, d = k.shape
+    assert two == 2 and v.shape == (B, Nk, H, 2 * d) and lam.shape == (H,)
     compact = q_rows is not None
     if compact:
+        Nq = int(n_queries or Nk)
+        r, R = _rows(rows, Nq)
         assert r is not None
         q = _f64(q_rows)
         assert q.shape == (B, R, H, 2, d)
     else:
         q = _f64(q)
-        assert q.shape == k.shape
+        Nq = q.shape[1]
+        r, R = _rows(rows, Nq)
+        assert q.shape == (B, Nq, H, 2, d)
     out = np.zeros((B, R, H, 2 * d), dtype=np.float64)
-    rc = _load().oracle_prefill_v1(_dp(q), _dp(k), _dp(v), _dp(lam), float(lambda_init_value),
-                                   B, N, H, d, int(bool(causal)), int(bool(apply_norm)), float(eps),
-                                   _ip(r), R, int(compact), _dp(out),
-                                   int(threads or default_threads()))
+    rc = _load().oracle_prefill_v1_range(_dp(q), _dp(k), _dp(v), _dp(lam), float(lambda_init_value),
+                                         B, Nq, Nk, H, d, int(bool(causal)), int(window),
+                                         int(bool(apply_norm)), float(eps), _ip(r), R, int(compact),
+                                         _dp(out), int(threads or default_threads()))
     if rc != 0:
-        raise ValueError(f"oracle_prefill_v1 failed: {rc}")
+        raise ValueError(f"oracle_prefill_v1_range failed: {rc}")
     return out
 
 
-def prefill_v2(q, k, v, lam, causal=True, rows=None, threads=None, q_rows=None) -> np.ndarray:
-    """V2 prefill. q: [B,N,Hq,d]; k,v: [B,N,Hkv,d]; lam: [Hq/2] -> out [B,R,Hq/2,d].
-    With rows and q_rows ([B,R,Hq,d], the queries at those positions), q may be None."""
+def prefill_v2(q, k, v, lam, causal=True, rows=None, threads=None, q_rows=None, window=0,
+               n_queries=None) -> np.ndarray:
+    """V2 prefill. q: [B,Nq,Hq,d]; k,v: [B,Nk,Hkv,d]; lam: [Hq/2] -> out [B,R,Hq/2,d].
+    Nq <= Nk, window as for prefill_v1. With rows and q_rows ([B,R,Hq,d]), q may be None."""
     k, v, lam = _f64(k), _f64(v), _f64(lam)
-    B, N, Hkv, d = k.shape
+    B, Nk, Hkv, d = k.shape
     assert v.shape == k.shape
-    r, R = _rows(rows, N)
     compact = q_rows is not None
     if compact:
+        Nq = int(n_queries or Nk)
+        r, R = _rows(rows, Nq)
         assert r is not None
         q = _f64(q_rows)
         assert q.shape[:2] == (B, R) and q.shape[3] == d
     else:
         q = _f64(q)
-        assert q.shape[:2] == (B, N) and q.shape[3] == d
+        Nq = q.shape[1]
+        r, R = _rows(rows, Nq)
+        assert q.shape[0] == B and q.shape[3] == d
     Hq = q.shape[2]
     assert lam.shape == (Hq // 2,)
     out = np.zeros((B, R, Hq // 2, d), dtype=np.float64)
-    rc = _load().oracle_prefill_v2(_dp(q), _dp(k), _dp(v), _dp(lam), B, N, Hq, Hkv, d,
-                                   int(bool(causal)), _ip(r), R, int(compact), _dp(out),
-                                   int(threads or default_threads()))
+    rc = _load().oracle_prefill_v2_range(_dp(q), _dp(k), _dp(v), _dp(lam), B, Nq, Nk, Hq, Hkv, d,
+                                         int(bool(causal)), int(window), _ip(r), R, int(compact),
+                                         _dp(out), int(threads or default_threads()))
     if rc != 0:
-        raise ValueError(f"oracle_prefill_v2 failed: {rc}")
+        raise ValueError(f"oracle_prefill_v2_range failed: {rc}")
     return out
 
 

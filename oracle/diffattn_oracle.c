@@ -27,6 +27,9 @@
  *
  *   causal: key j is visible to query i iff j <= i ("Attention Variants: Sliding
  *   Window, Sparse, Differential", Build It, Step 1 causal_mask; Step 4 diff_attention).
+ *   With Nk keys and Nq <= Nk queries (a chunk of new queries after Nk - Nq cached ones)
+ *   query i sits at position i + Nk - Nq. A sliding window of W keys (same page, Build
+ *   It, sliding-window mask) keeps keys j with pos - W < j <= pos.
  *
  *   lambda = exp(lq1 . lk1) - exp(lq2 . lk2) + lambda_init   ("Differential Attention (V2)",
  *            The Concept, "The difference idea"; Key Terms "lambda")
@@ -144,6 +147,8 @@ struct job {
   int n_rows;
   int q_compact; /* 1: q holds only the sampled rows, [B, n_rows, ...] */
   int B, N, H, Hq, Hkv, d, causal, apply_norm;
+  int Nk;     /* keys per batch entry (>= N, the queries); prefill only */
+  int window; /* causal sliding window in keys; 0 = none */
   double eps, lambda_init;
   double* out;
   long n_units;
@@ -222,39 +227,54 @@ static void v1_unit(const job* jb, long unit, double* a1, double* a2) {
   int n_rows = jb->rows ? jb->n_rows : N;
   int nq = jb->q_compact ? n_rows : N; /* query rows stored per batch entry */
   const double* qb = jb->q + (long)b * nq * tok_q + (long)h * 2 * d;
-  const double* kb = jb->k + (long)b * N * tok_q + (long)h * 2 * d;
-  const double* vb = jb->v + (long)b * N * tok_v + (long)h * dv;
+  const double* kb = jb->k + (long)b * jb->Nk * tok_q + (long)h * 2 * d;
+  const double* vb = jb->v + (long)b * jb->Nk * tok_v + (long)h * dv;
   for (int r = 0; r < n_rows; ++r) {
     int i = jb->rows ? jb->rows[r] : r;
     const double* q1 = qb + (long)(jb->q_compact ? r : i) * tok_q;
     const double* q2 = q1 + d;
-    int n_keys = jb->causal ? i + 1 : N;
+    int hi = jb->causal ? i + (jb->Nk - N) : jb->Nk - 1; /* last visible key */
+    int lo = (jb->causal && jb->window > 0 && hi - jb->window + 1 > 0) ? hi - jb->window + 1 : 0;
     double* o = jb->out + (((long)b * n_rows + r) * H + h) * dv;
-    diff_row(q1, q2, kb, kb + d, tok_q, vb, tok_v, n_keys, d, dv, jb->lam[h], a1, a2, o);
+    diff_row(q1, q2, kb + (long)lo * tok_q, kb + (long)lo * tok_q + d, tok_q, vb + (long)lo * tok_v,
+             tok_v, hi - lo + 1, d, dv, jb->lam[h], a1, a2, o);
     if (jb->apply_norm) rmsnorm_scale(o, dv, jb->eps, jb->lambda_init);
   }
 }
 
-int oracle_prefill_v1(const double* q, const double* k, const double* v, const double* lam,
-                      double lambda_init, int B, int N, int H, int d, int causal, int apply_norm,
-                      double eps, const int* rows, int n_rows, int q_compact, double* out,
-                      int nthreads) {
-  if (!q || !k || !v || !lam || !out || B < 0 || N < 0 || H < 0 || d <= 0) return ORACLE_ERR_ARG;
+/* Nq queries (the last Nq of Nk positions when causal), Nk keys, causal sliding window of
+ * `window` keys (0 = none; only with causal). */
+int oracle_prefill_v1_range(const double* q, const double* k, const double* v, const double* lam,
+                            double lambda_init, int B, int Nq, int Nk, int H, int d, int causal,
+                            int window, int apply_norm, double eps, const int* rows, int n_rows,
+                            int q_compact, double* out, int nthreads) {
+  if (!q || !k || !v || !lam || !out || B < 0 || Nq < 0 || Nk < Nq || H < 0 || d <= 0 || window < 0)
+    return ORACLE_ERR_ARG;
+  if (window > 0 && !causal) return ORACLE_ERR_ARG;
   if (rows) {
     for (int r = 0; r < n_rows; ++r)
-      if (rows[r] < 0 || rows[r] >= N) return ORACLE_ERR_ARG;
+      if (rows[r] < 0 || rows[r] >= Nq) return ORACLE_ERR_ARG;
   }
   job jb;
   memset(&jb, 0, sizeof(jb));
   jb.variant = 1;
   jb.q = q; jb.k = k; jb.v = v; jb.lam = lam;
   jb.rows = rows; jb.n_rows = n_rows; jb.q_compact = rows ? q_compact : 0;
-  jb.B = B; jb.N = N; jb.H = H; jb.d = d; jb.causal = causal; jb.apply_norm = apply_norm;
+  jb.B = B; jb.N = Nq; jb.Nk = Nk; jb.window = window; jb.H = H; jb.d = d; jb.causal = causal;
+  jb.apply_norm = apply_norm;
   jb.eps = eps; jb.lambda_init = lambda_init; jb.out = out;
   jb.n_units = (long)B * H;
-  jb.scratch_len = N;
+  jb.scratch_len = Nk;
   jb.fn = v1_unit;
   return run_job(&jb, nthreads);
+}
+
+int oracle_prefill_v1(const double* q, const double* k, const double* v, const double* lam,
+                      double lambda_init, int B, int N, int H, int d, int causal, int apply_norm,
+                      double eps, const int* rows, int n_rows, int q_compact, double* out,
+                      int nthreads) {
+  return oracle_prefill_v1_range(q, k, v, lam, lambda_init, B, N, N, H, d, causal, 0, apply_norm,
+                                 eps, rows, n_rows, q_compact, out, nthreads);
 }
 
 /* ---- V2 prefill ---------------------------------------------------------------------
@@ -276,42 +296,55 @@ static void v2_unit(const job* jb, long unit, double* a1, double* a2) {
   int n_rows = jb->rows ? jb->n_rows : N;
   int nq = jb->q_compact ? n_rows : N;
   const double* qb = jb->q + (long)b * nq * tok_q;
-  const double* kb = jb->k + (long)b * N * tok_kv;
-  const double* vb = jb->v + (long)b * N * tok_kv;
+  const double* kb = jb->k + (long)b * jb->Nk * tok_kv;
+  const double* vb = jb->v + (long)b * jb->Nk * tok_kv;
   for (int r = 0; r < n_rows; ++r) {
     int i = jb->rows ? jb->rows[r] : r;
     long qr = jb->q_compact ? r : i;
     const double* q1 = qb + qr * tok_q + (long)h1 * d;
     const double* q2 = qb + qr * tok_q + (long)h2 * d;
-    int n_keys = jb->causal ? i + 1 : N;
+    int hi = jb->causal ? i + (jb->Nk - N) : jb->Nk - 1; /* last visible key */
+    int lo = (jb->causal && jb->window > 0 && hi - jb->window + 1 > 0) ? hi - jb->window + 1 : 0;
     double* o = jb->out + (((long)b * n_rows + r) * P + p) * d;
+    const double* k0 = kb + (long)lo * tok_kv;
+    const double* v0 = vb + (long)lo * tok_kv;
     /* both branches of a pair read the same KV head when Hq/Hkv is even */
-    diff_row(q1, q2, kb + (long)g1 * d, kb + (long)g2 * d, tok_kv, vb + (long)g1 * d, tok_kv,
-             n_keys, d, d, jb->lam[p], a1, a2, o);
+    diff_row(q1, q2, k0 + (long)g1 * d, k0 + (long)g2 * d, tok_kv, v0 + (long)g1 * d, tok_kv,
+             hi - lo + 1, d, d, jb->lam[p], a1, a2, o);
   }
 }
 
-int oracle_prefill_v2(const double* q, const double* k, const double* v, const double* lam,
-                      int B, int N, int Hq, int Hkv, int d, int causal, const int* rows,
-                      int n_rows, int q_compact, double* out, int nthreads) {
-  if (!q || !k || !v || !lam || !out || B < 0 || N < 0 || Hq <= 0 || Hkv <= 0 || d <= 0)
+int oracle_prefill_v2_range(const double* q, const double* k, const double* v, const double* lam,
+                            int B, int Nq, int Nk, int Hq, int Hkv, int d, int causal, int window,
+                            const int* rows, int n_rows, int q_compact, double* out, int nthreads) {
+  if (!q || !k || !v || !lam || !out || B < 0 || Nq < 0 || Nk < Nq || Hq <= 0 || Hkv <= 0 ||
+      d <= 0 || window < 0)
     return ORACLE_ERR_ARG;
+  if (window > 0 && !causal) return ORACLE_ERR_ARG;
   if (Hq % 2 != 0 || Hq % Hkv != 0 || (Hq / Hkv) % 2 != 0) return ORACLE_ERR_ARG;
   if (rows) {
     for (int r = 0; r < n_rows; ++r)
-      if (rows[r] < 0 || rows[r] >= N) return ORACLE_ERR_ARG;
+      if (rows[r] < 0 || rows[r] >= Nq) return ORACLE_ERR_ARG;
   }
   job jb;
   memset(&jb, 0, sizeof(jb));
   jb.variant = 2;
   jb.q = q; jb.k = k; jb.v = v; jb.lam = lam;
   jb.rows = rows; jb.n_rows = n_rows; jb.q_compact = rows ? q_compact : 0;
-  jb.B = B; jb.N = N; jb.Hq = Hq; jb.Hkv = Hkv; jb.d = d; jb.causal = causal;
+  jb.B = B; jb.N = Nq; jb.Nk = Nk; jb.window = window; jb.Hq = Hq; jb.Hkv = Hkv; jb.d = d;
+  jb.causal = causal;
   jb.out = out;
   jb.n_units = (long)B * (Hq / 2);
-  jb.scratch_len = N;
+  jb.scratch_len = Nk;
   jb.fn = v2_unit;
   return run_job(&jb, nthreads);
+}
+
+int oracle_prefill_v2(const double* q, const double* k, const double* v, const double* lam,
+                      int B, int N, int Hq, int Hkv, int d, int causal, const int* rows,
+                      int n_rows, int q_compact, double* out, int nthreads) {
+  return oracle_prefill_v2_range(q, k, v, lam, B, N, N, Hq, Hkv, d, causal, 0, rows, n_rows,
+                                 q_compact, out, nthreads);
 }
 
 /* ---- V2 decode ----------------------------------------------------------------------

@@ -349,3 +349,68 @@ def pin_compact_query_rows():
 
 
 ALL_PINS.append(pin_compact_query_rows)
+
+
+def pin_chunked_prefill_is_last_rows():
+    """Nq < Nk queries (a chunk after Nk - Nq cached positions) equal the last Nq rows of
+    the full causal prefill whose last Nq queries are the chunk's (V1 and V2)."""
+    r = _rng(13)
+    B, Nk, Nq, H, d = 2, 45, 17, 2, 8
+    qf = r.standard_normal((B, Nk, H, 2, d)); k = r.standard_normal((B, Nk, H, 2, d))
+    v = r.standard_normal((B, Nk, H, 2 * d)); lam = np.array([0.6, -0.2])
+    full = oracle.prefill_v1(qf, k, v, lam, 0.4, threads=1)
+    part = oracle.prefill_v1(qf[:, Nk - Nq:].copy(), k, v, lam, 0.4, threads=1)
+    _close(part, full[:, Nk - Nq:], 1e-13, "V1 chunk = last rows")
+    Hq, Hkv = 8, 2
+    qf2 = r.standard_normal((B, Nk, Hq, d)); k2 = r.standard_normal((B, Nk, Hkv, d))
+    v2 = r.standard_normal((B, Nk, Hkv, d)); lam2 = r.standard_normal(Hq // 2)
+    full2 = oracle.prefill_v2(qf2, k2, v2, lam2, threads=1)
+    part2 = oracle.prefill_v2(qf2[:, Nk - Nq:].copy(), k2, v2, lam2, threads=1)
+    _close(part2, full2[:, Nk - Nq:], 1e-13, "V2 chunk = last rows")
+
+
+def pin_window_lambda0_is_banded_attention():
+    """lambda = 0 with a causal sliding window of W keys: softmax attention under the band
+    mask pos - W < j <= pos (torch SDPA with an explicit boolean mask), chunked queries
+    included."""
+    r = _rng(14)
+    B, Nk, Nq, H, d, W = 1, 40, 25, 2, 8, 7
+    q = r.standard_normal((B, Nq, H, 2, d)); k = r.standard_normal((B, Nk, H, 2, d))
+    v = r.standard_normal((B, Nk, H, 2 * d))
+    out = oracle.prefill_v1(q, k, v, np.zeros(H), 0.3, apply_norm=False, window=W, threads=1)
+    pos = np.arange(Nq)[:, None] + (Nk - Nq)
+    j = np.arange(Nk)[None, :]
+    mask = torch.from_numpy((j <= pos) & (j > pos - W))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q[:, :, :, 0].transpose(0, 2, 1, 3).copy()),
+        torch.from_numpy(k[:, :, :, 0].transpose(0, 2, 1, 3).copy()),
+        torch.from_numpy(v.transpose(0, 2, 1, 3).copy()), attn_mask=mask,
+        scale=1.0 / math.sqrt(d)).numpy().transpose(0, 2, 1, 3)
+    _close(out, ref, 1e-12, "V1 window lambda=0 vs banded SDPA")
+    Hq, Hkv = 4, 2
+    q2 = r.standard_normal((B, Nq, Hq, d)); k2 = r.standard_normal((B, Nk, Hkv, d))
+    v2 = r.standard_normal((B, Nk, Hkv, d))
+    out2 = oracle.prefill_v2(q2, k2, v2, np.zeros(Hq // 2), window=W, threads=1)
+    kk = np.repeat(k2, 2, axis=2).transpose(0, 2, 1, 3).copy()
+    vv = np.repeat(v2, 2, axis=2).transpose(0, 2, 1, 3).copy()
+    ref2 = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q2.transpose(0, 2, 1, 3).copy()), torch.from_numpy(kk),
+        torch.from_numpy(vv), attn_mask=mask, scale=1.0 / math.sqrt(d)).numpy().transpose(0, 2, 1, 3)
+    _close(out2, ref2[:, :, 0::2], 1e-12, "V2 window lambda=0 vs banded SDPA")
+
+
+def pin_window_extremes():
+    """A window as long as the sequence changes nothing; a window of one key leaves
+    o = (1 - lambda) v_pos (then the V1 norm and scale)."""
+    r = _rng(15)
+    B, N, H, d = 1, 21, 2, 8
+    q = r.standard_normal((B, N, H, 2, d)); k = r.standard_normal((B, N, H, 2, d))
+    v = r.standard_normal((B, N, H, 2 * d)); lam = np.array([0.3, 0.9])
+    plain = oracle.prefill_v1(q, k, v, lam, 0.5, threads=1)
+    _close(oracle.prefill_v1(q, k, v, lam, 0.5, window=N, threads=1), plain, 0.0, "window = N")
+    one = oracle.prefill_v1(q, k, v, lam, 0.5, apply_norm=False, window=1, threads=1)
+    _close(one, (1.0 - lam)[None, None, :, None] * v, 1e-14, "window = 1")
+
+
+ALL_PINS += [pin_chunked_prefill_is_last_rows, pin_window_lambda0_is_banded_attention,
+             pin_window_extremes]

@@ -15,10 +15,16 @@ MUTANTS = {
     "branch2_reads_k1": ("a2[j] = dot(q2, k2 + (long)j * ks, d)", "a2[j] = dot(q2, k1 + (long)j * ks, d)"),
     "scale_1_over_d": ("double inv_sqrt_d = 1.0 / sqrt((double)d);\n  for (int j = 0; j < n_keys",
                        "double inv_sqrt_d = 1.0 / (double)d;\n  for (int j = 0; j < n_keys"),
-    "causal_off_by_one_v1": ("int n_keys = jb->causal ? i + 1 : N;\n    double* o = jb->out + (((long)b * n_rows + r) * H",
-                             "int n_keys = jb->causal ? i : N;\n    double* o = jb->out + (((long)b * n_rows + r) * H"),
-    "causal_off_by_one_v2": ("int n_keys = jb->causal ? i + 1 : N;\n    double* o = jb->out + (((long)b * n_rows + r) * P",
-                             "int n_keys = jb->causal ? i : N;\n    double* o = jb->out + (((long)b * n_rows + r) * P"),
+    "causal_off_by_one_v1": ("int hi = jb->causal ? i + (jb->Nk - N) : jb->Nk - 1; /* last visible key */\n    int lo = (jb->causal && jb->window > 0 && hi - jb->window + 1 > 0) ? hi - jb->window + 1 : 0;\n    double* o = jb->out + (((long)b * n_rows + r) * H",
+                             "int hi = jb->causal ? i - 1 + (jb->Nk - N) : jb->Nk - 1; /* last visible key */\n    int lo = (jb->causal && jb->window > 0 && hi - jb->window + 1 > 0) ? hi - jb->window + 1 : 0;\n    double* o = jb->out + (((long)b * n_rows + r) * H"),
+    "causal_off_by_one_v2": ("int hi = jb->causal ? i + (jb->Nk - N) : jb->Nk - 1; /* last visible key */\n    int lo = (jb->causal && jb->window > 0 && hi - jb->window + 1 > 0) ? hi - jb->window + 1 : 0;\n    double* o = jb->out + (((long)b * n_rows + r) * P",
+                             "int hi = jb->causal ? i - 1 + (jb->Nk - N) : jb->Nk - 1; /* last visible key */\n    int lo = (jb->causal && jb->window > 0 && hi - jb->window + 1 > 0) ? hi - jb->window + 1 : 0;\n    double* o = jb->out + (((long)b * n_rows + r) * P"),
+    "chunk_offset_dropped_v1": ("int hi = jb->causal ? i + (jb->Nk - N) : jb->Nk - 1; /* last visible key */\n    int lo = (jb->causal && jb->window > 0 && hi - jb->window + 1 > 0) ? hi - jb->window + 1 : 0;\n    double* o = jb->out + (((long)b * n_rows + r) * H",
+                                "int hi = jb->causal ? i : jb->Nk - 1; /* last visible key */\n    int lo = (jb->causal && jb->window > 0 && hi - jb->window + 1 > 0) ? hi - jb->window + 1 : 0;\n    double* o = jb->out + (((long)b * n_rows + r) * H"),
+    "window_off_by_one_v1": ("int lo = (jb->causal && jb->window > 0 && hi - jb->window + 1 > 0) ? hi - jb->window + 1 : 0;\n    double* o = jb->out + (((long)b * n_rows + r) * H",
+                             "int lo = (jb->causal && jb->window > 0 && hi - jb->window > 0) ? hi - jb->window : 0;\n    double* o = jb->out + (((long)b * n_rows + r) * H"),
+    "window_ignored_v2": ("int lo = (jb->causal && jb->window > 0 && hi - jb->window + 1 > 0) ? hi - jb->window + 1 : 0;\n    double* o = jb->out + (((long)b * n_rows + r) * P",
+                          "int lo = 0;\n    double* o = jb->out + (((long)b * n_rows + r) * P"),
     "branch2_no_softmax": ("softmax_row(a2, n_keys);", ""),
     "norm_drops_scale": ("o[c] = o[c] / r * (1.0 - lambda_init);", "o[c] = o[c] / r;"),
     "norm_drops_eps": ("double r = sqrt(ss / (double)n + eps);", "double r = sqrt(ss / (double)n);"),
@@ -28,10 +34,10 @@ MUTANTS = {
                              "d2 += lq2[(long)h * dim + c] * lk1[(long)h * dim + c];"),
     "lambda_init_rate": ("return 0.8 - 0.6 * exp(-0.3 * (double)(depth - 1));",
                          "return 0.8 - 0.6 * exp(-0.3 * (double)depth);"),
-    "v1_q2_is_q1": ("const double* q2 = q1 + d;\n    int n_keys = jb->causal", "const double* q2 = q1;\n    int n_keys = jb->causal"),
+    "v1_q2_is_q1": ("const double* q2 = q1 + d;\n    int hi = jb->causal", "const double* q2 = q1;\n    int hi = jb->causal"),
     "v1_decode_q2_is_q1": ("const double* q2 = q1 + d;\n  int n_keys = jb->kv_len", "const double* q2 = q1;\n  int n_keys = jb->kv_len"),
-    "v1_value_of_other_head": ("const double* vb = jb->v + (long)b * N * tok_v + (long)h * dv;",
-                               "const double* vb = jb->v + (long)b * N * tok_v + (long)((h + 1) % H) * dv;"),
+    "v1_value_of_other_head": ("const double* vb = jb->v + (long)b * jb->Nk * tok_v + (long)h * dv;",
+                               "const double* vb = jb->v + (long)b * jb->Nk * tok_v + (long)((h + 1) % H) * dv;"),
     "v2_gqa_modulo": ("int g1 = h1 / group, g2 = h2 / group;\n  long tok_q",
                       "int g1 = h1 % jb->Hkv, g2 = h2 % jb->Hkv;\n  long tok_q"),
     "v2_pairing_halves": ("int h1 = 2 * p, h2 = 2 * p + 1;\n  int g1 = h1 / group, g2 = h2 / group;\n  long tok_q",
