@@ -62,6 +62,8 @@ class PrefillParams(ctypes.Structure):
         ("k_strides", ctypes.c_int64 * 3),
         ("v_strides", ctypes.c_int64 * 3),
         ("o_strides", ctypes.c_int64 * 3),
+        ("kv_seqlen", ctypes.c_int32),
+        ("window", ctypes.c_int32),
     ]
 
 
@@ -176,9 +178,12 @@ def diffattn_lambda(lq1, lk1, lq2, lk2, depth: int, lambda_out=None, lambda_init
     return lambda_out, lambda_init_out
 
 
-def prefill_params(q, k, v, out, causal=True, apply_norm=None, norm_eps=1e-5) -> PrefillParams:
+def prefill_params(q, k, v, out, causal=True, apply_norm=None, norm_eps=1e-5,
+                   window=0) -> PrefillParams:
     """Build the prefill parameter struct from tensor shapes and strides.
-    V1: q,k [B,N,H,2,d], v,out [B,N,H,2d]. V2: q [B,N,Hq,d], k,v [B,N,Hkv,d], out [B,N,Hq/2,d]."""
+    V1: q [B,N,H,2,d], k [B,Nk,H,2,d], v [B,Nk,H,2d], out [B,N,H,2d].
+    V2: q [B,N,Hq,d], k,v [B,Nk,Hkv,d], out [B,N,Hq/2,d]. Nk >= N: the queries are the last
+    N positions (chunked prefill)."""
     p = PrefillParams()
     if q.dim() == 5:
         B, N, H, two, d = q.shape
@@ -207,14 +212,19 @@ def prefill_params(q, k, v, out, causal=True, apply_norm=None, norm_eps=1e-5) ->
     p.batch, p.seqlen, p.head_dim = B, N, d
     p.causal = int(bool(causal))
     p.norm_eps = float(norm_eps)
+    if k.shape[1] != v.shape[1]:
+        raise DiffattnError("diffattn_fwd_prefill", -1)
+    p.kv_seqlen = int(k.shape[1])
+    p.window = int(window)
     p.v_strides[:] = v.stride()[:3]
     p.o_strides[:] = out.stride()[:3]
     return p
 
 
 def diffattn_fwd_prefill(q, k, v, lam, lambda_init=None, out=None, causal=True, apply_norm=None,
-                         norm_eps=1e-5, dev_status=None, stream=None):
-    """Fused differential attention prefill (see include/diffattn.h for layouts)."""
+                         norm_eps=1e-5, dev_status=None, stream=None, window=0):
+    """Fused differential attention prefill (see include/diffattn.h for layouts). k and v
+    may hold more positions than q (chunked prefill); window > 0 is a causal sliding window."""
     import torch
     lib = load_library()
     if out is None:
@@ -224,7 +234,7 @@ def diffattn_fwd_prefill(q, k, v, lam, lambda_init=None, out=None, causal=True, 
         else:
             B, N, Hq, d = q.shape
             out = torch.empty((B, N, Hq // 2, d), dtype=q.dtype, device=q.device)
-    p = prefill_params(q, k, v, out, causal, apply_norm, norm_eps)
+    p = prefill_params(q, k, v, out, causal, apply_norm, norm_eps, window)
     rc = lib.diffattn_fwd_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
                                   _ptr(lambda_init), _ptr(out), _ptr(dev_status), _stream(stream))
     _check("diffattn_fwd_prefill", rc)

@@ -67,6 +67,10 @@ int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   if (p->dtype != DIFFATTN_F32 && p->dtype != DIFFATTN_BF16) return DIFFATTN_ERR_INVALID_ARG;
   if (p->causal != 0 && p->causal != 1) return DIFFATTN_ERR_INVALID_ARG;
   if (p->apply_norm != 0 && p->apply_norm != 1) return DIFFATTN_ERR_INVALID_ARG;
+  // chunked prefill: kv_seqlen >= seqlen keys (0 reads as seqlen); window only when causal
+  const int nk = p->kv_seqlen == 0 ? p->seqlen : p->kv_seqlen;
+  if (nk < p->seqlen || p->window < 0 || (p->window > 0 && !p->causal))
+    return DIFFATTN_ERR_INVALID_ARG;
   if (!strides_ok(p->q_strides, 3) || !strides_ok(p->k_strides, 3) ||
       !strides_ok(p->v_strides, 3) || !strides_ok(p->o_strides, 3))
     return DIFFATTN_ERR_INVALID_ARG;
@@ -76,6 +80,8 @@ int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   a.variant = p->variant;
   a.B = p->batch;
   a.N = p->seqlen;
+  a.Nk = nk;
+  a.window = p->window;
   a.d = p->head_dim;
   a.causal = p->causal;
   a.apply_norm = p->apply_norm;
@@ -131,7 +137,7 @@ int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   // bf16: tcgen05 kernel (V1: d = 64; V2: d = 128)
   if (p->variant == DIFFATTN_V1 && a.d != 64) return DIFFATTN_ERR_UNSUPPORTED;
   if (p->variant == DIFFATTN_V2 && a.d != 128) return DIFFATTN_ERR_UNSUPPORTED;
-  if (a.N > (1 << 24)) return DIFFATTN_ERR_UNSUPPORTED;
+  if (a.Nk > (1 << 24)) return DIFFATTN_ERR_UNSUPPORTED;
   return from_cuda(a.variant == DIFFATTN_V1 ? launch_prefill_v1(a, s) : launch_prefill_v2(a, s));
 }
 

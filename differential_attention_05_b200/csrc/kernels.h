@@ -10,7 +10,9 @@ namespace diffattn {
 // Resolved prefill problem (validated by the API layer).
 struct PrefillArgs {
   int variant;       // DIFFATTN_V1 / DIFFATTN_V2
-  int B, N;
+  int B, N;          // N queries (the last N of the Nk key positions)
+  int Nk;            // keys; Nk >= N
+  int window;        // causal sliding window in keys (0: none)
   int units;         // V1 heads / V2 pairs
   int Hq, Hkv;       // head counts as given
   int group;         // V2: Hq / Hkv (query heads per KV head); V1: 1

@@ -61,8 +61,11 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_f32_kernel(PrefillArgs a)
 #pragma unroll
   for (int t = 0; t < kPerLane; ++t) acc1[t] = acc2[t] = 0.f;
 
-  const int n_keys = a.causal ? i + 1 : a.N;
-  for (int j0 = 0; j0 < n_keys; j0 += 32) {
+  // visible keys key_lo .. n_keys - 1: query i sits at position i + Nk - N; causal stops at
+  // its own position, a sliding window keeps the last `window` of those
+  const int n_keys = a.causal ? i + (a.Nk - a.N) + 1 : a.Nk;
+  const int key_lo = (a.causal && a.window > 0) ? max(0, n_keys - a.window) : 0;
+  for (int j0 = key_lo; j0 < n_keys; j0 += 32) {
     const int j = j0 + lane;
     float s1 = -INFINITY, s2 = -INFINITY;
     if (j < n_keys) {

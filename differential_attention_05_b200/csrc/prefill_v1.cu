@@ -112,8 +112,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int u = (int)(blockIdx.x % per_qt) % a.units;
   const int b = (int)(blockIdx.x % per_qt) / a.units;
   const int q0 = qt * BM;
-  const int kend = a.causal ? min(q0 + BM, a.N) : a.N;  // keys this tile can see
-  const int n_kt = (kend + BN - 1) / BN;
+  // query i sits at key position i + off (chunked prefill: the last N of Nk positions);
+  // this tile sees keys klo .. khi, in key tiles j_lo .. j_lo + n_kt - 1
+  const int off = a.Nk - a.N;
+  const int khi = a.causal ? min(q0 + BM - 1 + off, a.Nk - 1) : a.Nk - 1;
+  const int klo = (a.causal && a.window > 0) ? max(0, q0 + off - a.window + 1) : 0;
+  const int j_lo = klo / BN;
+  const int n_kt = (khi + BN) / BN - j_lo;
 
   if (threadIdx.x == 0) {
     mbar_init(&ms.q_full, 1);
@@ -161,14 +166,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&ms.k_empty[st], par, abort_flag)) break;
         mbar_arrive_expect_tx(&ms.k_full[st], 2 * KBLK);
         uint8_t* kd = smem + K_OFF + st * 2 * KBLK;  // k_1 | k_2
-        tma_load_4d(kd, &maps.k, &ms.k_full[st], 0, u, j * BN, b);
-        tma_load_4d(kd + KBLK, &maps.k, &ms.k_full[st], 64, u, j * BN, b);
+        tma_load_4d(kd, &maps.k, &ms.k_full[st], 0, u, (j_lo + j) * BN, b);
+        tma_load_4d(kd + KBLK, &maps.k, &ms.k_full[st], 64, u, (j_lo + j) * BN, b);
         issued_k = j + 1;
         if (!mbar_wait(&ms.v_empty[st], par, abort_flag)) break;
         mbar_arrive_expect_tx(&ms.v_full[st], 2 * KBLK);
         uint8_t* vd = smem + V_OFF + st * 2 * KBLK;
-        tma_load_4d(vd, &maps.v, &ms.v_full[st], 0, u, j * BN, b);
-        tma_load_4d(vd + KBLK, &maps.v, &ms.v_full[st], 64, u, j * BN, b);
+        tma_load_4d(vd, &maps.v, &ms.v_full[st], 0, u, (j_lo + j) * BN, b);
+        tma_load_4d(vd + KBLK, &maps.v, &ms.v_full[st], 64, u, (j_lo + j) * BN, b);
         issued_v = j + 1;
       }
       if (*abort_flag) {
@@ -242,7 +247,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sl2 = 1.4426950408889634f * rsqrtf((float)a.d);  // log2(e)/sqrt(d)
     const float lam = a.lambda[u];
-    const int vis = a.causal ? qi : a.N - 1;  // last visible key
+    // visible keys of this row: vlo .. vis (causal: up to its own position; window: the
+    // last `window` of those)
+    const int vis = a.causal ? min(qi + off, a.Nk - 1) : a.Nk - 1;
+    const int vlo = (a.causal && a.window > 0) ? max(0, vis - a.window + 1) : 0;
+    // the same bounds relative to the first key of this tile's range
+    const int vis0 = vis - j_lo * BN, vlo0 = vlo - j_lo * BN;
     float m = -INFINITY, l = 0.f;             // this warpgroup's branch
     float c = 0.f;                            // branch 1 warpgroup only
     bool ok = true;
@@ -258,11 +268,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_ld32f(sb + 64u * wg, p);
       tmem_ld32f(sb + 64u * wg + 32, p + 32);
       tmem_wait_ld();
-      const int lim = vis - j * BN;
-      if (lim < BN - 1) {
+      const int lim = vis0 - j * BN, llim = vlo0 - j * BN;
+      if (lim < BN - 1 || llim > 0) {
 #pragma unroll
         for (int e = 0; e < BN; ++e)
-          if (e > lim) p[e] = -INFINITY;
+          if (e > lim || e < llim) p[e] = -INFINITY;
       }
       float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
 #pragma unroll
@@ -274,13 +284,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const float t = fmax3(fmaxf(c0, c1), c2, c3) * sl2;
       // lazy maximum: raised only on growth by more than 2^8 (or when unset)
-      const bool r = (t > m + RESCALE_LOG2) || (m == -INFINITY);
+      const bool had = m != -INFINITY;  // the row saw a visible key in an earlier tile
+      const bool r = (t > m + RESCALE_LOG2) || !had;
       const float n = r ? fmaxf(t, m) : m;
-      const float al = (r && m != -INFINITY) ? ex2(m - n) : 1.f;
+      const float al = (r && had) ? ex2(m - n) : 1.f;
       m = n;
-      // p = 2^(s sl2 - m), in place
+      // p = 2^(s sl2 - m), in place (0 for every key while the row has none visible)
       float sa = 0.f, sb2 = 0.f, sc2 = 0.f, sd = 0.f;
-      const float nm = -m;
+      const float nm = m == -INFINITY ? 0.f : -m;
 #pragma unroll
       for (int e = 0; e < BN; e += 4) {
         float x0, x1, x2, x3;
@@ -320,16 +331,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float l2 = ms.h_l2[f][row];
       // target c = lambda l_1 / l_2 (sums including this tile); under max updates c follows
       // c a_1 / a_2, which leaves D unchanged; reset to the target when it leaves
-      // [0.8, 1.25] times it (tile 0 always takes the target)
-      const float cst = lam * __fdiv_rn(l, l2);  // exact ratio: identical branches give c = lambda
+      // [0.8, 1.25] times it (the row's first tile with a visible key always takes the
+      // target: D and O_2 are still 0)
+      const float cst = l2 > 0.f ? lam * __fdiv_rn(l, l2) : lam;  // exact ratio: identical branches give c = lambda
       float cn = cst, kc = 0.f;
-      if (j > 0) {
+      bool need = false;
+      if (had) {
         const float cev = (al == a2) ? c : c * __fdividef(al, a2);
         const float ra = fabsf(cev), rt = fabsf(cst);
         const bool reset = !(ra >= 0.8f * rt && ra <= 1.25f * rt);
         cn = reset ? cst : cev;
         if (reset) kc = __fsub_rn(__fmul_rn(al, c), __fmul_rn(a2, cn));
-        const bool need = (al != 1.f) || (a2 != 1.f) || (kc != 0.f);
+        need = (al != 1.f) || (a2 != 1.f) || (kc != 0.f);
+      }
+      {
+        // the whole warp rescales (a row with nothing to do has al = a2 = 1, kc = 0)
         if (__any_sync(0xffffffffu, need)) {
           // D <- a_1 D + kc O_2, O_2 <- a_2 O_2 over all 128 output columns; the P.V MMAs
           // of the previous tile must have completed
@@ -445,8 +461,8 @@ cudaError_t launch_prefill_v1(const PrefillArgs& a, cudaStream_t stream) {
   // q, k viewed as [B, N, H, 128] (branch 1 in columns 0..63, branch 2 in 64..127) and v as
   // [B, N, H, 2d = 128]
   if (!make_map(&maps.q, a.q, 128, a.units, a.N, a.B, a.qs, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.k, a.k, 128, a.units, a.N, a.B, a.ks, BN)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.v, a.v, 128, a.units, a.N, a.B, a.vs, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, 128, a.units, a.Nk, a.B, a.ks, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, 128, a.units, a.Nk, a.B, a.vs, BN)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

@@ -113,8 +113,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int u = (int)(blockIdx.x % per_qt) % a.units;
   const int b = (int)(blockIdx.x % per_qt) / a.units;
   const int q0 = qt * BM;
-  const int kend = a.causal ? min(q0 + BM, a.N) : a.N;  // keys this tile can see
-  const int n_kt = (kend + BN - 1) / BN;
+  // query i sits at key position i + off (chunked prefill: the last N of Nk positions);
+  // this tile sees keys klo .. khi, in key tiles j_lo .. j_lo + n_kt - 1
+  const int off = a.Nk - a.N;
+  const int khi = a.causal ? min(q0 + BM - 1 + off, a.Nk - 1) : a.Nk - 1;
+  const int klo = (a.causal && a.window > 0) ? max(0, q0 + off - a.window + 1) : 0;
+  const int j_lo = klo / BN;
+  const int n_kt = (khi + BN) / BN - j_lo;
 
   if (threadIdx.x == 0) {
     for (int x = 0; x < 2; ++x) {
@@ -170,15 +175,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&ms.k_empty[ks], ((j / KSTAGES) & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&ms.k_full[ks], 2 * HALF);
         uint8_t* kd = smem + K_OFF + ks * 2 * HALF;
-        tma_load_4d(kd, &maps.k, &ms.k_full[ks], 0, kvh, j * BN, b);
-        tma_load_4d(kd + HALF, &maps.k, &ms.k_full[ks], 64, kvh, j * BN, b);
+        tma_load_4d(kd, &maps.k, &ms.k_full[ks], 0, kvh, (j_lo + j) * BN, b);
+        tma_load_4d(kd + HALF, &maps.k, &ms.k_full[ks], 64, kvh, (j_lo + j) * BN, b);
         issued_k = j + 1;
         const int vs = j % VSTAGES;
         if (!mbar_wait(&ms.v_empty[vs], ((j / VSTAGES) & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&ms.v_full[vs], 2 * HALF);
         uint8_t* vd = smem + V_OFF + vs * 2 * HALF;
-        tma_load_4d(vd, &maps.v, &ms.v_full[vs], 0, kvh, j * BN, b);
-        tma_load_4d(vd + HALF, &maps.v, &ms.v_full[vs], 64, kvh, j * BN, b);
+        tma_load_4d(vd, &maps.v, &ms.v_full[vs], 0, kvh, (j_lo + j) * BN, b);
+        tma_load_4d(vd + HALF, &maps.v, &ms.v_full[vs], 64, kvh, (j_lo + j) * BN, b);
         issued_v = j + 1;
       }
       if (*abort_flag) {
@@ -273,7 +278,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t o_addr = s_addr + 128u;         // D (branch-1 lanes) / O_2 (branch 2)
     const float sl2 = 1.4426950408889634f * rsqrtf((float)a.d);  // log2(e)/sqrt(d)
     const float lam = a.lambda[u];
-    const int vis = a.causal ? min(qi, a.N - 1) : a.N - 1;  // last visible key
+    // visible keys of this query: vlo .. vis (causal: up to its own position, clamped for
+    // the padding rows of the last tile; window: the last `window` of those)
+    const int vis = a.causal ? min(qi + off, a.Nk - 1) : a.Nk - 1;
+    const int vlo = (a.causal && a.window > 0) ? max(0, vis - a.window + 1) : 0;
     float m = -INFINITY, l = 0.f;  // this lane's branch
     float c = 0.f;                 // identical in both lanes of a query
     bool ok = true;
@@ -286,11 +294,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) tmem_ld32f(s_addr + 32 * i, p + 32 * i);
       tmem_wait_ld();
-      const int lim = vis - j * BN;
-      if (lim < BN - 1) {
+      const int lim = vis - (j_lo + j) * BN, llim = vlo - (j_lo + j) * BN;
+      if (lim < BN - 1 || llim > 0) {
 #pragma unroll
         for (int e = 0; e < BN; ++e)
-          if (e > lim) p[e] = -INFINITY;
+          if (e > lim || e < llim) p[e] = -INFINITY;
       }
       float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
 #pragma unroll
@@ -302,14 +310,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const float t = fmax3(fmaxf(c0, c1), c2, c3) * sl2;
       // lazy maximum: raised only on growth by more than 2^8 (or when unset)
-      const bool r = (t > m + RESCALE_LOG2) || (m == -INFINITY);
+      const bool had = m != -INFINITY;  // the query saw a visible key in an earlier tile
+      const bool r = (t > m + RESCALE_LOG2) || !had;
       const float n = r ? fmaxf(t, m) : m;
-      const float al = (r && m != -INFINITY) ? ex2(m - n) : 1.f;
+      const float al = (r && had) ? ex2(m - n) : 1.f;
       m = n;
-      // p = 2^(s sl2 - m), in place; in every group of 8 keys the last POLY_PAIRS pairs go
-      // to the FMA pipe, the rest to the MUFU unit
+      // p = 2^(s sl2 - m), in place (0 for every key while the query has none visible); in
+      // every group of 8 keys the last POLY_PAIRS pairs go to the FMA pipe, the rest to MUFU
       float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
-      const float nm = -m;
+      const float nm = m == -INFINITY ? 0.f : -m;
 #pragma unroll
       for (int e = 0; e < BN; e += 8) {
         float xv[8];
@@ -338,16 +347,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float l1 = h ? l_o : l, l2 = h ? l : l_o;
       // target c = lambda l_1 / l_2 (sums including this tile); under max updates c follows
       // c a_1 / a_2, which leaves D unchanged; reset to the target when it leaves
-      // [0.8, 1.25] times it (tile 0 always takes the target). Both lanes compute the same.
-      const float cst = lam * __fdiv_rn(l1, l2);  // exact ratio: identical branches give c = lambda
+      // [0.8, 1.25] times it (the query's first tile with a visible key always takes the
+      // target: D and O_2 are still 0). Both lanes compute the same.
+      const float cst = l2 > 0.f ? lam * __fdiv_rn(l1, l2) : lam;  // exact ratio: identical branches give c = lambda
       float cn = cst, kc = 0.f;
-      if (j > 0) {
+      bool need = false;
+      if (had) {
         const float cev = (a1 == a2) ? c : c * __fdividef(a1, a2);
         const float ra = fabsf(cev), rt = fabsf(cst);
         const bool reset = !(ra >= 0.8f * rt && ra <= 1.25f * rt);
         cn = reset ? cst : cev;
         if (reset) kc = __fsub_rn(__fmul_rn(a1, c), __fmul_rn(a2, cn));
-        const bool need = (al != 1.f) || (kc != 0.f);
+        need = (al != 1.f) || (kc != 0.f);
+      }
+      {
+        // the whole warp rescales (a query with nothing to do has al = 1, kc = 0)
         if (__any_sync(FULL, need)) {
           // D <- a_1 D + kc O_2, O_2 <- a_2 O_2 over all 128 value columns. The score MMA
           // that filled S was issued after this sub-tile's previous P.V MMAs, so its
@@ -460,8 +474,8 @@ cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream) {
   // q [B, N, Hq, 128], k, v [B, N, Hkv, 128]; Q boxes of 16 queries of one head (the
   // TMEM-lane row order), K and V boxes of 128 keys
   if (!make_map(&maps.q, a.q, 128, a.Hq, a.N, a.B, a.qs, 16)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.k, a.k, 128, a.Hkv, a.N, a.B, a.ks, BN)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.v, a.v, 128, a.Hkv, a.N, a.B, a.vs, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, 128, a.Hkv, a.Nk, a.B, a.ks, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, 128, a.Hkv, a.Nk, a.B, a.vs, BN)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

@@ -91,30 +91,36 @@ int diffattn_lambda(const float* lq1, const float* lk1, const float* lq2, const 
  *
  * V1 (variant = DIFFATTN_V1): n_q_heads = n_kv_heads = H differential heads,
  *   head_dim = d per branch (d = 64 for bf16; any 1..128 multiple of 4 for f32).
- *   q, k : [B, N, H, 2, d]   branch 1 at index 0, branch 2 at index 1 (contiguous, so
+ *   q    : [B, N, H, 2, d]   branch 1 at index 0, branch 2 at index 1 (contiguous, so
  *                            each (token, head) row holds q1 then q2)
- *   v    : [B, N, H, 2d]
+ *   k    : [B, Nk, H, 2, d]
+ *   v    : [B, Nk, H, 2d]
  *   out  : [B, N, H, 2d]
  *   lambda: [H]. apply_norm = 1 applies the per-head RMSNorm (over the 2d channels,
  *   eps = norm_eps, unit gain) and then multiplies by (1 - lambda_init[0]).
  * V2 (variant = DIFFATTN_V2): n_q_heads = Hq (even), n_kv_heads = Hkv with Hq/Hkv even;
  *   head_dim = d (128 for bf16; any 1..128 multiple of 4 for f32).
  *   q    : [B, N, Hq, d]     query heads 2p, 2p+1 = branches 1, 2 of pair p
- *   k, v : [B, N, Hkv, d]    query head h reads KV head h / (Hq / Hkv)
+ *   k, v : [B, Nk, Hkv, d]   query head h reads KV head h / (Hq / Hkv)
  *   out  : [B, N, Hq/2, d]
  *   lambda: [Hq/2]. apply_norm must be 0.
  * Strides (elements) are {batch, token, head}; the branch axis (V1) and the channel
  * axis are contiguous. bf16: q/k/v base pointers 16-byte aligned and every stride a
  * multiple of 8 elements (TMA rules); f32: 16-byte aligned, strides multiple of 4.
  * out must not alias q, k or v.
- * causal = 1: query i attends keys 0..i (queries and keys share positions 0..N-1);
- * causal = 0: every query attends all N keys.
+ * Nk = kv_seqlen (0 reads as N) >= N. The N queries are the LAST N of the Nk positions
+ * (chunked prefill: a chunk of new tokens attends the earlier ones and itself), so query i
+ * sits at position i + Nk - N.
+ * causal = 1: query i attends keys 0..i + Nk - N; causal = 0: every query attends all Nk
+ * keys. window = W > 0 (causal only) keeps the last W of those keys (a causal sliding
+ * window: keys i + Nk - N - W + 1 .. i + Nk - N); window = 0 keeps all.
+ * Nk < N, window < 0, or window > 0 with causal = 0 return DIFFATTN_ERR_INVALID_ARG.
  */
 typedef struct {
   int32_t variant;    /* diffattn_variant */
   int32_t dtype;      /* diffattn_dtype of q, k, v and out */
   int32_t batch;      /* B >= 0 */
-  int32_t seqlen;     /* N >= 0 (queries = keys = N) */
+  int32_t seqlen;     /* N >= 0 queries */
   int32_t n_q_heads;  /* V1: H; V2: Hq */
   int32_t n_kv_heads; /* V1: H; V2: Hkv */
   int32_t head_dim;   /* d per branch */
@@ -125,6 +131,8 @@ typedef struct {
   int64_t k_strides[3];
   int64_t v_strides[3];
   int64_t o_strides[3];
+  int32_t kv_seqlen;  /* Nk >= N keys; 0 = N */
+  int32_t window;     /* causal sliding window in keys; 0 = none */
 } diffattn_prefill_params;
 
 /*

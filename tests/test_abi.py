@@ -75,6 +75,8 @@ def _call_prefill(lib, p, q=GOOD, k=GOOD + 4096, v=GOOD + 8192, lam=GOOD + 12288
     ("apply_norm", 1, -1),    # V2 has no per-head norm
     ("causal", 2, -1),
     ("head_dim", 96, -2),     # bf16 V2 needs d = 128
+    ("kv_seqlen", 255, -1),   # fewer keys than queries
+    ("window", -1, -1),
 ])
 def test_prefill_rejects(lib, field, value, code):
     assert _call_prefill(lib, _prefill_params(**{field: value})) == code
@@ -89,6 +91,16 @@ def test_prefill_rejects_null_and_alias_and_misalignment(lib):
     p2 = _prefill_params()
     p2.q_strides[1] = 16 * 128 + 4                               # token stride not 16 B multiple
     assert _call_prefill(lib, p2) == -3
+
+
+def test_prefill_window_needs_causal(lib):
+    assert _call_prefill(lib, _prefill_params(causal=0, window=16)) == -1
+
+
+def test_prefill_params_layout():
+    """The two chunked-prefill fields sit after the stride arrays (ABI append-only)."""
+    assert B.PrefillParams.kv_seqlen.offset == B.PrefillParams.o_strides.offset + 24
+    assert B.PrefillParams.window.offset == B.PrefillParams.kv_seqlen.offset + 4
 
 
 def test_prefill_empty_problem_launches_nothing(lib):
