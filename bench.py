@@ -60,6 +60,18 @@ def prefill_flops(inp) -> float:
     return float(inp.B) * pairs * per
 
 
+def visible_pairs(Nq: int, Nk: int, causal: bool = True, window: int = 0) -> float:
+    """(query, key) pairs a prefill attends: queries at the last Nq of Nk positions, each
+    seeing keys up to its own position (causal), the last `window` of them when window > 0."""
+    if not causal:
+        return float(Nq) * Nk
+    off = Nk - Nq
+    seen = np.arange(off + 1, Nk + 1, dtype=np.float64)  # keys 0 .. i + off
+    if window > 0:
+        seen = np.minimum(seen, window)
+    return float(seen.sum())
+
+
 def workload_decode_bytes(inp) -> float:
     """Cache bytes one decode step reads: V2 K and V of width d per KV head; V1 K rows
     (K_1 | K_2, 2d) and V rows (2d) per head."""
@@ -407,6 +419,23 @@ def secondary(device, peaks, torch, da):
     res["v2_prefill"] = {"workload": "v2_bf16_prefill_b1_n16384_hq64_hkv8_d128", "ms": round(ms, 4),
                          "TFLOP/s": round(fl / ms / 1e9, 2),
                          "frac_of_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
+    # the same tensors as a sliding-window layer (4096 keys) and as a 2048-query chunk at
+    # the end of the 16384-key context; FLOPs count the attended pairs only
+    for name, Nq, window in (("v2_prefill_window4096", N, 4096), ("v2_prefill_chunk2048", 2048, 0)):
+        qq = q[:, N - Nq:]
+        oo = out[:, N - Nq:]
+        for _ in range(3):
+            da.diffattn_fwd_prefill(qq, k, v, lam, out=oo, window=window)
+        for a, b in es:
+            a.record()
+            da.diffattn_fwd_prefill(qq, k, v, lam, out=oo, window=window)
+            b.record()
+        torch.cuda.synchronize(device)
+        ms = statistics.median(a.elapsed_time(b) for a, b in es)
+        fl = 4.0 * d * Hq * visible_pairs(Nq, N, True, window)
+        res[name] = {"queries": Nq, "keys": N, "window": window, "ms": round(ms, 4),
+                     "TFLOP/s": round(fl / ms / 1e9, 2),
+                     "frac_of_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
     del q, k, v, out
     B, L = 64, 32768
     q = torch.randn((B, Hq, d), generator=g, device=device).bfloat16()

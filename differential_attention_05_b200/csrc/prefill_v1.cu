@@ -97,6 +97,10 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
 __device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
+// WINDOW: a causal sliding window (a.window > 0). Without one every row sees key 0, the
+// first key of the first tile, so the row state is set after tile 0 and the masks have
+// only an upper end; that case compiles without the lower-end and unset-row checks.
+template <bool WINDOW>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_v1_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -116,7 +120,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // this tile sees keys klo .. khi, in key tiles j_lo .. j_lo + n_kt - 1
   const int off = a.Nk - a.N;
   const int khi = a.causal ? min(q0 + BM - 1 + off, a.Nk - 1) : a.Nk - 1;
-  const int klo = (a.causal && a.window > 0) ? max(0, q0 + off - a.window + 1) : 0;
+  const int klo = WINDOW ? max(0, q0 + off - a.window + 1) : 0;
   const int j_lo = klo / BN;
   const int n_kt = (khi + BN) / BN - j_lo;
 
@@ -250,7 +254,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // visible keys of this row: vlo .. vis (causal: up to its own position; window: the
     // last `window` of those)
     const int vis = a.causal ? min(qi + off, a.Nk - 1) : a.Nk - 1;
-    const int vlo = (a.causal && a.window > 0) ? max(0, vis - a.window + 1) : 0;
+    const int vlo = WINDOW ? max(0, vis - a.window + 1) : 0;
     // the same bounds relative to the first key of this tile's range
     const int vis0 = vis - j_lo * BN, vlo0 = vlo - j_lo * BN;
     float m = -INFINITY, l = 0.f;             // this warpgroup's branch
@@ -269,10 +273,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_ld32f(sb + 64u * wg + 32, p + 32);
       tmem_wait_ld();
       const int lim = vis0 - j * BN, llim = vlo0 - j * BN;
-      if (lim < BN - 1 || llim > 0) {
+      if (lim < BN - 1 || (WINDOW && llim > 0)) {
 #pragma unroll
         for (int e = 0; e < BN; ++e)
-          if (e > lim || e < llim) p[e] = -INFINITY;
+          if (e > lim || (WINDOW && e < llim)) p[e] = -INFINITY;
       }
       float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
 #pragma unroll
@@ -284,14 +288,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const float t = fmax3(fmaxf(c0, c1), c2, c3) * sl2;
       // lazy maximum: raised only on growth by more than 2^8 (or when unset)
-      const bool had = m != -INFINITY;  // the row saw a visible key in an earlier tile
+      const bool had = WINDOW ? m != -INFINITY : j > 0;  // the row saw a visible key before
       const bool r = (t > m + RESCALE_LOG2) || !had;
       const float n = r ? fmaxf(t, m) : m;
       const float al = (r && had) ? ex2(m - n) : 1.f;
       m = n;
       // p = 2^(s sl2 - m), in place (0 for every key while the row has none visible)
       float sa = 0.f, sb2 = 0.f, sc2 = 0.f, sd = 0.f;
-      const float nm = m == -INFINITY ? 0.f : -m;
+      const float nm = (WINDOW && m == -INFINITY) ? 0.f : -m;
 #pragma unroll
       for (int e = 0; e < BN; e += 4) {
         float x0, x1, x2, x3;
@@ -333,7 +337,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // c a_1 / a_2, which leaves D unchanged; reset to the target when it leaves
       // [0.8, 1.25] times it (the row's first tile with a visible key always takes the
       // target: D and O_2 are still 0)
-      const float cst = l2 > 0.f ? lam * __fdiv_rn(l, l2) : lam;  // exact ratio: identical branches give c = lambda
+      const float cst = (WINDOW && !(l2 > 0.f)) ? lam : lam * __fdiv_rn(l, l2);  // exact ratio: identical branches give c = lambda
       float cn = cst, kc = 0.f;
       bool need = false;
       if (had) {
@@ -344,7 +348,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (reset) kc = __fsub_rn(__fmul_rn(al, c), __fmul_rn(a2, cn));
         need = (al != 1.f) || (a2 != 1.f) || (kc != 0.f);
       }
-      {
+      if (WINDOW || j > 0) {
         // the whole warp rescales (a row with nothing to do has al = a2 = 1, kc = 0)
         if (__any_sync(0xffffffffu, need)) {
           // D <- a_1 D + kc O_2, O_2 <- a_2 O_2 over all 128 output columns; the P.V MMAs
@@ -468,14 +472,20 @@ cudaError_t launch_prefill_v1(const PrefillArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   if (dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(prefill_v1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(prefill_v1_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(prefill_v1_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set[dev] = true;
   }
   const long long tiles = (long long)((a.N + BM - 1) / BM) * a.units * a.B;
   if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  prefill_v1_kernel<<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  if (a.causal && a.window > 0)
+    prefill_v1_kernel<true><<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  else
+    prefill_v1_kernel<false><<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   return cudaGetLastError();
 }
 

@@ -98,6 +98,10 @@ __device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t bytes) {
 }
 }  // namespace
 
+// WINDOW: a causal sliding window (a.window > 0). Without one every row sees key 0, the
+// first key of the first tile, so the row state is set after tile 0 and the masks have
+// only an upper end; that case compiles without the lower-end and unset-row checks.
+template <bool WINDOW>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_v2_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -117,7 +121,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // this tile sees keys klo .. khi, in key tiles j_lo .. j_lo + n_kt - 1
   const int off = a.Nk - a.N;
   const int khi = a.causal ? min(q0 + BM - 1 + off, a.Nk - 1) : a.Nk - 1;
-  const int klo = (a.causal && a.window > 0) ? max(0, q0 + off - a.window + 1) : 0;
+  const int klo = WINDOW ? max(0, q0 + off - a.window + 1) : 0;
   const int j_lo = klo / BN;
   const int n_kt = (khi + BN) / BN - j_lo;
 
@@ -281,7 +285,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // visible keys of this query: vlo .. vis (causal: up to its own position, clamped for
     // the padding rows of the last tile; window: the last `window` of those)
     const int vis = a.causal ? min(qi + off, a.Nk - 1) : a.Nk - 1;
-    const int vlo = (a.causal && a.window > 0) ? max(0, vis - a.window + 1) : 0;
+    const int vlo = WINDOW ? max(0, vis - a.window + 1) : 0;
     float m = -INFINITY, l = 0.f;  // this lane's branch
     float c = 0.f;                 // identical in both lanes of a query
     bool ok = true;
@@ -295,10 +299,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int i = 0; i < 4; ++i) tmem_ld32f(s_addr + 32 * i, p + 32 * i);
       tmem_wait_ld();
       const int lim = vis - (j_lo + j) * BN, llim = vlo - (j_lo + j) * BN;
-      if (lim < BN - 1 || llim > 0) {
+      if (lim < BN - 1 || (WINDOW && llim > 0)) {
 #pragma unroll
         for (int e = 0; e < BN; ++e)
-          if (e > lim || e < llim) p[e] = -INFINITY;
+          if (e > lim || (WINDOW && e < llim)) p[e] = -INFINITY;
       }
       float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
 #pragma unroll
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       const float t = fmax3(fmaxf(c0, c1), c2, c3) * sl2;
       // lazy maximum: raised only on growth by more than 2^8 (or when unset)
-      const bool had = m != -INFINITY;  // the query saw a visible key in an earlier tile
+      const bool had = WINDOW ? m != -INFINITY : j > 0;  // the query saw a visible key before
       const bool r = (t > m + RESCALE_LOG2) || !had;
       const float n = r ? fmaxf(t, m) : m;
       const float al = (r && had) ? ex2(m - n) : 1.f;
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // p = 2^(s sl2 - m), in place (0 for every key while the query has none visible); in
       // every group of 8 keys the last POLY_PAIRS pairs go to the FMA pipe, the rest to MUFU
       float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
-      const float nm = m == -INFINITY ? 0.f : -m;
+      const float nm = (WINDOW && m == -INFINITY) ? 0.f : -m;
 #pragma unroll
       for (int e = 0; e < BN; e += 8) {
         float xv[8];
@@ -349,7 +353,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // c a_1 / a_2, which leaves D unchanged; reset to the target when it leaves
       // [0.8, 1.25] times it (the query's first tile with a visible key always takes the
       // target: D and O_2 are still 0). Both lanes compute the same.
-      const float cst = l2 > 0.f ? lam * __fdiv_rn(l1, l2) : lam;  // exact ratio: identical branches give c = lambda
+      const float cst = (WINDOW && !(l2 > 0.f)) ? lam : lam * __fdiv_rn(l1, l2);  // exact ratio: identical branches give c = lambda
       float cn = cst, kc = 0.f;
       bool need = false;
       if (had) {
@@ -360,7 +364,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (reset) kc = __fsub_rn(__fmul_rn(a1, c), __fmul_rn(a2, cn));
         need = (al != 1.f) || (kc != 0.f);
       }
-      {
+      if (WINDOW || j > 0) {
         // the whole warp rescales (a query with nothing to do has al = 1, kc = 0)
         if (__any_sync(FULL, need)) {
           // D <- a_1 D + kc O_2, O_2 <- a_2 O_2 over all 128 value columns. The score MMA
@@ -481,14 +485,20 @@ cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   if (dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(prefill_v2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(prefill_v2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(prefill_v2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set[dev] = true;
   }
   const long long tiles = (long long)((a.N + BM - 1) / BM) * a.units * a.B;
   if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  prefill_v2_kernel<<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  if (a.causal && a.window > 0)
+    prefill_v2_kernel<true><<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  else
+    prefill_v2_kernel<false><<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   return cudaGetLastError();
 }
 

@@ -71,3 +71,18 @@ def test_reference_arm_other_ranks_exit_silently():
                          env=env, capture_output=True, text=True, timeout=120)
     assert out.returncode == 0
     assert out.stdout.strip() == ""
+
+
+def test_visible_pairs_brute_force():
+    """The attended (query, key) pair count against enumeration on small shapes."""
+    import bench
+    for Nq, Nk, causal, window in [(5, 5, True, 0), (3, 9, True, 0), (9, 9, True, 4),
+                                   (4, 11, True, 3), (6, 7, False, 0), (1, 1, True, 1)]:
+        off = Nk - Nq
+        n = 0
+        for i in range(Nq):
+            for j in range(Nk):
+                hi = i + off if causal else Nk - 1
+                lo = hi - window + 1 if window > 0 else 0
+                n += lo <= j <= hi
+        assert bench.visible_pairs(Nq, Nk, causal, window) == n
