@@ -8,9 +8,11 @@ from ._binding import (  # noqa: F401
     DiffattnError,
     diffattn_lambda,
     diffattn_fwd_prefill,
+    diffattn_fwd_prefill_varlen,
     diffattn_fwd_decode,
     diffattn_fwd_decode_static,
     diffattn_fwd_decode_v1,
+    diffattn_fwd_decode_paged,
     diffattn_selftest_timeout,
     diffattn_decode_workspace_size,
     diffattn_status_string,
@@ -22,9 +24,11 @@ __all__ = [
     "DiffattnError",
     "diffattn_lambda",
     "diffattn_fwd_prefill",
+    "diffattn_fwd_prefill_varlen",
     "diffattn_fwd_decode",
     "diffattn_fwd_decode_static",
     "diffattn_fwd_decode_v1",
+    "diffattn_fwd_decode_paged",
     "diffattn_selftest_timeout",
     "diffattn_decode_workspace_size",
     "diffattn_status_string",

@@ -32,10 +32,12 @@ EXPORTS = (
     "diffattn_status_string",
     "diffattn_lambda",
     "diffattn_fwd_prefill",
+    "diffattn_fwd_prefill_varlen",
     "diffattn_decode_workspace_size",
     "diffattn_fwd_decode",
     "diffattn_fwd_decode_static",
     "diffattn_fwd_decode_v1",
+    "diffattn_fwd_decode_paged",
     "diffattn_selftest_timeout",
 )
 
@@ -111,6 +113,9 @@ def load_library():
     lib.diffattn_fwd_prefill.restype = i32
     lib.diffattn_fwd_prefill.argtypes = [ctypes.POINTER(PrefillParams), vp, vp, vp, f32p, f32p,
                                          vp, vp, vp]
+    lib.diffattn_fwd_prefill_varlen.restype = i32
+    lib.diffattn_fwd_prefill_varlen.argtypes = [ctypes.POINTER(PrefillParams), vp, vp, i32, vp, vp,
+                                                vp, f32p, f32p, vp, vp, vp]
     lib.diffattn_decode_workspace_size.restype = i32
     lib.diffattn_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeParams),
                                                    ctypes.POINTER(ctypes.c_size_t)]
@@ -123,6 +128,10 @@ def load_library():
     lib.diffattn_fwd_decode_v1.restype = i32
     lib.diffattn_fwd_decode_v1.argtypes = [ctypes.POINTER(DecodeParams), vp, vp, vp, vp, f32p, f32p,
                                            i32, ctypes.c_float, vp, vp, ctypes.c_size_t, vp, vp]
+    lib.diffattn_fwd_decode_paged.restype = i32
+    lib.diffattn_fwd_decode_paged.argtypes = [ctypes.POINTER(DecodeParams), ctypes.POINTER(PagedKV),
+                                              vp, vp, vp, vp, vp, f32p, f32p, i32, ctypes.c_float,
+                                              vp, vp, ctypes.c_size_t, vp, vp]
     lib.diffattn_selftest_timeout.restype = i32
     lib.diffattn_selftest_timeout.argtypes = [vp, i32, vp]
     _lib = lib
@@ -241,6 +250,39 @@ def diffattn_fwd_prefill(q, k, v, lam, lambda_init=None, out=None, causal=True, 
     return out
 
 
+def diffattn_fwd_prefill_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, lam,
+                                lambda_init=None, out=None, causal=True, apply_norm=None,
+                                norm_eps=1e-5, window=0, dev_status=None, stream=None):
+    """Prefill over packed sequences of different lengths (see include/diffattn.h).
+    V1: q [Tq,H,2,d], k [Tk,H,2,d], v [Tk,H,2d] -> out [Tq,H,2d]. V2: q [Tq,Hq,d],
+    k,v [Tk,Hkv,d] -> out [Tq,Hq/2,d]. cu_seqlens_q / _k: int32 [S+1] device offsets;
+    max_seqlen_q: the longest sequence's query count (host int)."""
+    import torch
+    lib = load_library()
+    if out is None:
+        if q.dim() == 4:
+            T, H, _, d = q.shape
+            out = torch.empty((T, H, 2 * d), dtype=q.dtype, device=q.device)
+        else:
+            T, Hq, d = q.shape
+            out = torch.empty((T, Hq // 2, d), dtype=q.dtype, device=q.device)
+    # the packed tensors viewed with a batch axis of one: the fixed-length struct applies
+    p = prefill_params(q.unsqueeze(0), k.unsqueeze(0), v.unsqueeze(0), out.unsqueeze(0), causal,
+                       apply_norm, norm_eps, window)
+    p.batch = int(cu_seqlens_q.numel()) - 1
+    if p.batch < 0 or cu_seqlens_k.numel() != cu_seqlens_q.numel():
+        raise DiffattnError("diffattn_fwd_prefill_varlen", -1)
+    p.seqlen, p.kv_seqlen = int(q.shape[0]), int(k.shape[0])
+    for st in (p.q_strides, p.k_strides, p.v_strides, p.o_strides):
+        st[0] = 0
+    rc = lib.diffattn_fwd_prefill_varlen(ctypes.byref(p), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+                                         int(max_seqlen_q), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                                         _ptr(lambda_init), _ptr(out), _ptr(dev_status),
+                                         _stream(stream))
+    _check("diffattn_fwd_prefill_varlen", rc)
+    return out
+
+
 def decode_params(q, k_cache, v_cache, out, num_splits=0) -> DecodeParams:
     p = DecodeParams()
     B, Hq, d = q.shape
@@ -320,6 +362,72 @@ def diffattn_fwd_decode_v1(q, k_cache, v_cache, lam, lambda_init=None, kv_len=No
                                     float(norm_eps), _ptr(out), _ptr(workspace), ws_bytes,
                                     _ptr(dev_status), _stream(stream))
     _check("diffattn_fwd_decode_v1", rc)
+    return out
+
+
+class PagedKV(ctypes.Structure):
+    _fields_ = [
+        ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("max_pages_per_seq", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("page_strides", ctypes.c_int64 * 3),
+    ]
+
+
+def paged_kv(k_pages, v_pages, block_table) -> PagedKV:
+    """Pool geometry from the page tensors ([P, page_size, heads, ...]) and the block table
+    ([B, max_pages_per_seq])."""
+    if tuple(k_pages.stride()[:3]) != tuple(v_pages.stride()[:3]) or k_pages.shape[:2] != v_pages.shape[:2]:
+        raise DiffattnError("diffattn_fwd_decode_paged", -1)
+    pk = PagedKV()
+    pk.num_pages, pk.page_size = int(k_pages.shape[0]), int(k_pages.shape[1])
+    pk.max_pages_per_seq = int(block_table.shape[1])
+    pk.page_strides[:] = k_pages.stride()[:3]
+    return pk
+
+
+def diffattn_fwd_decode_paged(q, k_pages, v_pages, block_table, lam, kv_len=None, lambda_init=None,
+                              out=None, apply_norm=None, norm_eps=1e-5, workspace=None,
+                              num_splits=0, max_kv_len=None, dev_status=None, stream=None):
+    """Split-KV differential decode over a paged cache (block table [B, max_pages_per_seq],
+    int32). V2: q [B,Hq,d], pages [P,page,Hkv,d] -> out [B,Hq/2,d]. V1: q [B,H,2,d],
+    k_pages [P,page,H,2,d], v_pages [P,page,H,2d] -> out [B,H,2d] (norm and scale when
+    apply_norm, default on). max_kv_len defaults to page_size * max_pages_per_seq."""
+    import torch
+    lib = load_library()
+    pk = paged_kv(k_pages, v_pages, block_table)
+    p = DecodeParams()
+    v1 = q.dim() == 4
+    B = q.shape[0]
+    if v1:
+        _, H, two, d = q.shape
+        if two != 2:
+            raise DiffattnError("diffattn_fwd_decode_paged", -1)
+        p.variant, p.n_q_heads, p.n_kv_heads = DIFFATTN_V1, H, H
+        oshape = (B, H, 2 * d)
+        norm = True if apply_norm is None else bool(apply_norm)
+    else:
+        _, Hq, d = q.shape
+        p.variant, p.n_q_heads, p.n_kv_heads = DIFFATTN_V2, Hq, int(k_pages.shape[2])
+        oshape = (B, Hq // 2, d)
+        norm = False if apply_norm is None else bool(apply_norm)
+    if out is None:
+        out = torch.empty(oshape, dtype=q.dtype, device=q.device)
+    p.dtype = _dtype_code(q)
+    p.batch, p.head_dim, p.num_splits = B, d, int(num_splits)
+    p.max_kv_len = int(max_kv_len if max_kv_len is not None else pk.page_size * pk.max_pages_per_seq)
+    p.q_strides[:] = q.stride()[:2]
+    p.o_strides[:] = out.stride()[:2]
+    need = diffattn_decode_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib.diffattn_fwd_decode_paged(ctypes.byref(p), ctypes.byref(pk), _ptr(q), _ptr(k_pages),
+                                       _ptr(v_pages), _ptr(block_table), _ptr(kv_len), _ptr(lam),
+                                       _ptr(lambda_init), int(norm), float(norm_eps), _ptr(out),
+                                       _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
+    _check("diffattn_fwd_decode_paged", rc)
     return out
 
 

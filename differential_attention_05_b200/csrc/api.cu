@@ -58,19 +58,28 @@ int diffattn_lambda(const float* lq1, const float* lk1, const float* lq2, const 
                                  lambda_init_out, static_cast<cudaStream_t>(stream)));
 }
 
-int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const void* k,
-                         const void* v, const float* lambda, const float* lambda_init, void* out,
-                         int* dev_status, void* stream) {
+}  // extern "C"
+
+// The body shared by the fixed-length and the variable-length prefill. cu_q = nullptr:
+// p->batch sequences of p->seqlen queries and kv_seqlen keys. Otherwise p->batch packed
+// sequences with offsets cu_q / cu_k (device), p->seqlen / kv_seqlen the packed row counts
+// and max_q the longest query count.
+static int prefill_run(const diffattn_prefill_params* p, const int32_t* cu_q, const int32_t* cu_k,
+                       int max_q, const void* q, const void* k, const void* v, const float* lambda,
+                       const float* lambda_init, void* out, int* dev_status, void* stream) {
   if (!p) return DIFFATTN_ERR_INVALID_ARG;
   if (p->batch < 0 || p->seqlen < 0 || p->head_dim < 1) return DIFFATTN_ERR_INVALID_ARG;
   if (p->variant != DIFFATTN_V1 && p->variant != DIFFATTN_V2) return DIFFATTN_ERR_INVALID_ARG;
   if (p->dtype != DIFFATTN_F32 && p->dtype != DIFFATTN_BF16) return DIFFATTN_ERR_INVALID_ARG;
   if (p->causal != 0 && p->causal != 1) return DIFFATTN_ERR_INVALID_ARG;
   if (p->apply_norm != 0 && p->apply_norm != 1) return DIFFATTN_ERR_INVALID_ARG;
-  // chunked prefill: kv_seqlen >= seqlen keys (0 reads as seqlen); window only when causal
+  const bool varlen = cu_q != nullptr;
+  // keys: kv_seqlen (0 reads as seqlen); fixed length needs at least as many keys as
+  // queries (chunked prefill); a window only when causal
   const int nk = p->kv_seqlen == 0 ? p->seqlen : p->kv_seqlen;
-  if (nk < p->seqlen || p->window < 0 || (p->window > 0 && !p->causal))
+  if (nk < 0 || (!varlen && nk < p->seqlen) || p->window < 0 || (p->window > 0 && !p->causal))
     return DIFFATTN_ERR_INVALID_ARG;
+  if (varlen && (max_q < 0 || !cu_k)) return DIFFATTN_ERR_INVALID_ARG;
   if (!strides_ok(p->q_strides, 3) || !strides_ok(p->k_strides, 3) ||
       !strides_ok(p->v_strides, 3) || !strides_ok(p->o_strides, 3))
     return DIFFATTN_ERR_INVALID_ARG;
@@ -79,13 +88,19 @@ int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   memset(&a, 0, sizeof(a));
   a.variant = p->variant;
   a.B = p->batch;
-  a.N = p->seqlen;
+  a.N = varlen ? max_q : p->seqlen;
   a.Nk = nk;
   a.window = p->window;
   a.d = p->head_dim;
   a.causal = p->causal;
   a.apply_norm = p->apply_norm;
   a.eps = p->norm_eps;
+  if (varlen) {
+    a.cu_q = cu_q;
+    a.cu_k = cu_k;
+    a.total_q = p->seqlen;
+    a.total_k = nk;
+  }
   if (p->variant == DIFFATTN_V1) {
     if (p->n_q_heads < 1 || p->n_kv_heads != p->n_q_heads) return DIFFATTN_ERR_INVALID_ARG;
     a.units = p->n_q_heads;
@@ -105,11 +120,13 @@ int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   }
   if (a.apply_norm && !(p->norm_eps >= 0.f && isfinite(p->norm_eps))) return DIFFATTN_ERR_INVALID_ARG;
   if (a.units > 65535 || a.B > 65535) return DIFFATTN_ERR_UNSUPPORTED;
-  if (a.B == 0 || a.N == 0) return DIFFATTN_OK;
+  if (a.B == 0 || a.N == 0 || (varlen && p->seqlen == 0)) return DIFFATTN_OK;
   if (!q || !k || !v || !lambda || !out) return DIFFATTN_ERR_INVALID_ARG;
   if (a.apply_norm && !lambda_init) return DIFFATTN_ERR_INVALID_ARG;
   if (out == q || out == k || out == v) return DIFFATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return DIFFATTN_ERR_MISALIGNED;
+  if (varlen && ((reinterpret_cast<uintptr_t>(cu_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_k) & 3u)))
     return DIFFATTN_ERR_MISALIGNED;
   const int vec = p->dtype == DIFFATTN_BF16 ? 8 : 4;  // elements per 16 bytes
   for (int i = 0; i < 3; ++i) {
@@ -137,8 +154,26 @@ int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   // bf16: tcgen05 kernel (V1: d = 64; V2: d = 128)
   if (p->variant == DIFFATTN_V1 && a.d != 64) return DIFFATTN_ERR_UNSUPPORTED;
   if (p->variant == DIFFATTN_V2 && a.d != 128) return DIFFATTN_ERR_UNSUPPORTED;
-  if (a.Nk > (1 << 24)) return DIFFATTN_ERR_UNSUPPORTED;
+  if (a.Nk > (1 << 24) || p->seqlen > (1 << 24)) return DIFFATTN_ERR_UNSUPPORTED;
   return from_cuda(a.variant == DIFFATTN_V1 ? launch_prefill_v1(a, s) : launch_prefill_v2(a, s));
+}
+
+extern "C" {
+
+int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const void* k,
+                         const void* v, const float* lambda, const float* lambda_init, void* out,
+                         int* dev_status, void* stream) {
+  return prefill_run(p, nullptr, nullptr, 0, q, k, v, lambda, lambda_init, out, dev_status, stream);
+}
+
+int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t* cu_seqlens_q,
+                                const int32_t* cu_seqlens_k, int max_seqlen_q, const void* q,
+                                const void* k, const void* v, const float* lambda,
+                                const float* lambda_init, void* out, int* dev_status,
+                                void* stream) {
+  if (!cu_seqlens_q || !cu_seqlens_k) return DIFFATTN_ERR_INVALID_ARG;
+  return prefill_run(p, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, q, k, v, lambda, lambda_init,
+                     out, dev_status, stream);
 }
 
 static int decode_check(const diffattn_decode_params* p, int* splits, int* split_len) {
@@ -219,21 +254,44 @@ int diffattn_decode_workspace_size(const diffattn_decode_params* p, size_t* byte
   return DIFFATTN_OK;
 }
 
-int diffattn_fwd_decode(const diffattn_decode_params* p, const void* q, const void* k_cache,
-                        const void* v_cache, const int32_t* kv_len, const float* lambda, void* out,
-                        void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+}  // extern "C"
+
+// The body shared by the decode entry points: checks by variant, the paged-cache checks
+// when pk is given, then the launch.
+static int decode_run(const diffattn_decode_params* p, const diffattn_paged_kv* pk,
+                      const void* q, const void* k, const void* v, const int32_t* block_table,
+                      const int32_t* kv_len, const float* lambda, const float* lambda_init,
+                      int apply_norm, float norm_eps, void* out, void* workspace,
+                      size_t workspace_bytes, int* dev_status, void* stream) {
   int splits = 0, len = 0;
-  int rc = decode_check(p, &splits, &len);
+  const bool v1 = p->variant == DIFFATTN_V1;
+  int rc = v1 ? decode_v1_check(p, &splits, &len) : decode_check(p, &splits, &len);
   if (rc != DIFFATTN_OK) return rc;
+  if (apply_norm != 0 && apply_norm != 1) return DIFFATTN_ERR_INVALID_ARG;
+  if (!v1 && apply_norm) return DIFFATTN_ERR_INVALID_ARG;  // V2 has no per-head norm
+  if (apply_norm && !(norm_eps >= 0.f && isfinite(norm_eps))) return DIFFATTN_ERR_INVALID_ARG;
+  int page_shift = 0;
+  if (pk) {
+    if (pk->page_size < 1 || pk->page_size > 65536 || (pk->page_size & (pk->page_size - 1)))
+      return DIFFATTN_ERR_INVALID_ARG;
+    if (pk->num_pages < 1 || pk->max_pages_per_seq < 1 || pk->reserved != 0 ||
+        !strides_ok(pk->page_strides, 3))
+      return DIFFATTN_ERR_INVALID_ARG;
+    if ((int64_t)pk->max_pages_per_seq * pk->page_size < p->max_kv_len) return DIFFATTN_ERR_INVALID_ARG;
+    while ((1 << page_shift) < pk->page_size) ++page_shift;
+  }
   if (p->batch == 0) return DIFFATTN_OK;
-  if (!q || !k_cache || !v_cache || !lambda || !out) return DIFFATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !lambda || !out) return DIFFATTN_ERR_INVALID_ARG;
+  if (pk && !block_table) return DIFFATTN_ERR_INVALID_ARG;
+  if (apply_norm && !lambda_init) return DIFFATTN_ERR_INVALID_ARG;
   const size_t need = decode_ws_bytes(p, splits);
   if (!workspace || workspace_bytes < need) return DIFFATTN_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIFFATTN_ERR_MISALIGNED;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return DIFFATTN_ERR_MISALIGNED;
-  if (p->q_strides[0] % 8 || p->q_strides[1] % 8 || p->kv_strides[0] % 8 || p->kv_strides[1] % 8 ||
-      p->kv_strides[2] % 8 || p->o_strides[0] % 8 || p->o_strides[1] % 8)
+  const int64_t* kvs = pk ? pk->page_strides : p->kv_strides;
+  if (p->q_strides[0] % 8 || p->q_strides[1] % 8 || kvs[0] % 8 || kvs[1] % 8 || kvs[2] % 8 ||
+      p->o_strides[0] % 8 || p->o_strides[1] % 8)
     return DIFFATTN_ERR_MISALIGNED;
   DecodeArgs a;
   memset(&a, 0, sizeof(a));
@@ -245,20 +303,44 @@ int diffattn_fwd_decode(const diffattn_decode_params* p, const void* q, const vo
   a.splits = splits;
   a.split_len = len;
   memcpy(a.qs, p->q_strides, sizeof(a.qs));
-  memcpy(a.kvs, p->kv_strides, sizeof(a.kvs));
+  memcpy(a.kvs, kvs, sizeof(a.kvs));
   memcpy(a.os, p->o_strides, sizeof(a.os));
   a.q = q;
-  a.k = k_cache;
-  a.v = v_cache;
+  a.k = k;
+  a.v = v;
   a.kv_len = kv_len;
   a.lambda = lambda;
+  a.lambda_init = lambda_init;
+  a.apply_norm = apply_norm;
+  a.eps = norm_eps;
   a.out = out;
-  const size_t recs = (size_t)a.B * a.Hq * splits;
+  if (pk) {
+    a.block_table = block_table;
+    a.bt_stride = pk->max_pages_per_seq;
+    a.page_shift = page_shift;
+    a.num_pages = pk->num_pages;
+  }
+  // per (b, head, split): V2 one record of d floats; V1 two (one per branch) of 2d
+  const size_t recs = (size_t)a.B * a.Hq * splits * (v1 ? 2 : 1);
+  const size_t rec_floats = v1 ? 2 * (size_t)a.d : (size_t)a.d;
   a.ws_o = static_cast<float*>(workspace);
   a.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                     (((recs * a.d * sizeof(float)) + 255) & ~(size_t)255));
+                                     (((recs * rec_floats * sizeof(float)) + 255) & ~(size_t)255));
   a.dev_status = dev_status;
-  return from_cuda(launch_decode(a, static_cast<cudaStream_t>(stream)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return from_cuda(v1 ? launch_decode_v1(a, s) : launch_decode(a, s));
+}
+
+extern "C" {
+
+int diffattn_fwd_decode(const diffattn_decode_params* p, const void* q, const void* k_cache,
+                        const void* v_cache, const int32_t* kv_len, const float* lambda, void* out,
+                        void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  if (!p) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->variant != DIFFATTN_V2) return p->variant == DIFFATTN_V1 ? DIFFATTN_ERR_UNSUPPORTED
+                                                                  : DIFFATTN_ERR_INVALID_ARG;
+  return decode_run(p, nullptr, q, k_cache, v_cache, nullptr, kv_len, lambda, nullptr, 0, 0.f, out,
+                    workspace, workspace_bytes, dev_status, stream);
 }
 
 int diffattn_fwd_decode_v1(const diffattn_decode_params* p, const void* q, const void* k_cache,
@@ -266,49 +348,22 @@ int diffattn_fwd_decode_v1(const diffattn_decode_params* p, const void* q, const
                            const float* lambda_init, int apply_norm, float norm_eps, void* out,
                            void* workspace, size_t workspace_bytes, int* dev_status,
                            void* stream) {
-  int splits = 0, len = 0;
-  int rc = decode_v1_check(p, &splits, &len);
-  if (rc != DIFFATTN_OK) return rc;
-  if (apply_norm != 0 && apply_norm != 1) return DIFFATTN_ERR_INVALID_ARG;
-  if (apply_norm && !(norm_eps >= 0.f && isfinite(norm_eps))) return DIFFATTN_ERR_INVALID_ARG;
-  if (p->batch == 0) return DIFFATTN_OK;
-  if (!q || !k_cache || !v_cache || !lambda || !out) return DIFFATTN_ERR_INVALID_ARG;
-  if (apply_norm && !lambda_init) return DIFFATTN_ERR_INVALID_ARG;
-  const size_t need = decode_ws_bytes(p, splits);
-  if (!workspace || workspace_bytes < need) return DIFFATTN_ERR_WORKSPACE;
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIFFATTN_ERR_MISALIGNED;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-    return DIFFATTN_ERR_MISALIGNED;
-  if (p->q_strides[0] % 8 || p->q_strides[1] % 8 || p->kv_strides[0] % 8 || p->kv_strides[1] % 8 ||
-      p->kv_strides[2] % 8 || p->o_strides[0] % 8 || p->o_strides[1] % 8)
-    return DIFFATTN_ERR_MISALIGNED;
-  DecodeArgs a;
-  memset(&a, 0, sizeof(a));
-  a.B = p->batch;
-  a.L = p->max_kv_len;
-  a.Hq = p->n_q_heads;
-  a.Hkv = p->n_kv_heads;
-  a.d = p->head_dim;
-  a.splits = splits;
-  a.split_len = len;
-  memcpy(a.qs, p->q_strides, sizeof(a.qs));
-  memcpy(a.kvs, p->kv_strides, sizeof(a.kvs));
-  memcpy(a.os, p->o_strides, sizeof(a.os));
-  a.q = q;
-  a.k = k_cache;
-  a.v = v_cache;
-  a.kv_len = kv_len;
-  a.lambda = lambda;
-  a.lambda_init = lambda_init;
-  a.apply_norm = apply_norm;
-  a.eps = norm_eps;
-  a.out = out;
-  const size_t recs = (size_t)a.B * a.Hq * splits * 2;
-  a.ws_o = static_cast<float*>(workspace);
-  a.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                     (((recs * 2 * a.d * sizeof(float)) + 255) & ~(size_t)255));
-  a.dev_status = dev_status;
-  return from_cuda(launch_decode_v1(a, static_cast<cudaStream_t>(stream)));
+  if (!p) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->variant != DIFFATTN_V1) return DIFFATTN_ERR_INVALID_ARG;
+  return decode_run(p, nullptr, q, k_cache, v_cache, nullptr, kv_len, lambda, lambda_init,
+                    apply_norm, norm_eps, out, workspace, workspace_bytes, dev_status, stream);
+}
+
+int diffattn_fwd_decode_paged(const diffattn_decode_params* p, const diffattn_paged_kv* pk,
+                              const void* q, const void* k_pages, const void* v_pages,
+                              const int32_t* block_table, const int32_t* kv_len,
+                              const float* lambda, const float* lambda_init, int apply_norm,
+                              float norm_eps, void* out, void* workspace, size_t workspace_bytes,
+                              int* dev_status, void* stream) {
+  if (!p || !pk) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->variant != DIFFATTN_V1 && p->variant != DIFFATTN_V2) return DIFFATTN_ERR_INVALID_ARG;
+  return decode_run(p, pk, q, k_pages, v_pages, block_table, kv_len, lambda, lambda_init,
+                    apply_norm, norm_eps, out, workspace, workspace_bytes, dev_status, stream);
 }
 
 }  // extern "C"

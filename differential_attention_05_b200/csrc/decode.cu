@@ -74,10 +74,14 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
   const int t_end = min(t_begin + a.split_len, kv_len);
   const int n_chunks = t_end > t_begin ? (t_end - t_begin + CH - 1) / CH : 0;
 
+  // paged cache: this entry's row of the block table; the page stride replaces the batch one
+  const int32_t* bt = a.block_table ? a.block_table + (int64_t)b * a.bt_stride : nullptr;
+  const int64_t boff = bt ? 0 : b * a.kvs[0];
   const __nv_bfloat16* kbase =
-      static_cast<const __nv_bfloat16*>(a.k) + b * a.kvs[0] + (int64_t)g * a.kvs[2];
+      static_cast<const __nv_bfloat16*>(a.k) + boff + (int64_t)g * a.kvs[2];
   const __nv_bfloat16* vbase =
-      static_cast<const __nv_bfloat16*>(a.v) + b * a.kvs[0] + (int64_t)g * a.kvs[2];
+      static_cast<const __nv_bfloat16*>(a.v) + boff + (int64_t)g * a.kvs[2];
+  bool bad_page = false;  // a block-table entry outside the pool: its rows read as zero
 
   // issue the copies of chunk c into stage c % STAGES (zero-fill past t_end)
   auto load_chunk = [&](int c) {
@@ -90,8 +94,17 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
       const int rem = idx % (CH * CHUNKS16_PER_ROW);
       const int row = rem / CHUNKS16_PER_ROW, c16 = rem % CHUNKS16_PER_ROW;
       const int tok = tok0 + row;
-      const bool ok = tok < t_end;
-      const __nv_bfloat16* src = (tensor ? vbase : kbase) + (ok ? (int64_t)tok * a.kvs[1] : 0) + c16 * 8;
+      bool ok = tok < t_end;
+      int64_t roff = (int64_t)tok * a.kvs[1];
+      if (bt) {
+        const int id = ok ? __ldg(bt + (tok >> a.page_shift)) : 0;
+        if ((unsigned)id >= (unsigned)a.num_pages) {
+          bad_page = bad_page || ok;
+          ok = false;
+        }
+        roff = (int64_t)id * a.kvs[0] + (int64_t)(tok & ((1 << a.page_shift) - 1)) * a.kvs[1];
+      }
+      const __nv_bfloat16* src = (tensor ? vbase : kbase) + (ok ? roff : 0) + c16 * 8;
       cp_async_16(st + tensor * TILE_BYTES + swz(row, c16), src, ok ? 16u : 0u);
     }
   };
@@ -194,6 +207,7 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
   }
   cp_async_wait<0>();
   __syncthreads();
+  if (bad_page) report_status(a.dev_status, DIFFATTN_ERR_INVALID_ARG);
 
   // merge the 4 warps' states of each head through shared memory
   float* sm_o = reinterpret_cast<float*>(smem);      // [WARPS][G][D]

@@ -66,10 +66,14 @@ __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs 
   const int t_end = min(t_begin + a.split_len, kv_len);
   const int n_chunks = t_end > t_begin ? (t_end - t_begin + CH - 1) / CH : 0;
 
+  // paged cache: this entry's row of the block table; the page stride replaces the batch one
+  const int32_t* bt = a.block_table ? a.block_table + (int64_t)b * a.bt_stride : nullptr;
+  const int64_t boff = bt ? 0 : b * a.kvs[0];
   const __nv_bfloat16* kbase =
-      static_cast<const __nv_bfloat16*>(a.k) + b * a.kvs[0] + (int64_t)h * a.kvs[2];
+      static_cast<const __nv_bfloat16*>(a.k) + boff + (int64_t)h * a.kvs[2];
   const __nv_bfloat16* vbase =
-      static_cast<const __nv_bfloat16*>(a.v) + b * a.kvs[0] + (int64_t)h * a.kvs[2];
+      static_cast<const __nv_bfloat16*>(a.v) + boff + (int64_t)h * a.kvs[2];
+  bool bad_page = false;  // a block-table entry outside the pool: its rows read as zero
 
   // copies of chunk c into stage c % STAGES (zero-fill past t_end)
   auto load_chunk = [&](int c) {
@@ -82,9 +86,17 @@ __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs 
       const int rem = idx % (CH * C16);
       const int row = rem / C16, c16 = rem % C16;
       const int tok = tok0 + row;
-      const bool ok = tok < t_end;
-      const __nv_bfloat16* src =
-          (tensor ? vbase : kbase) + (ok ? (int64_t)tok * a.kvs[1] : 0) + c16 * 8;
+      bool ok = tok < t_end;
+      int64_t roff = (int64_t)tok * a.kvs[1];
+      if (bt) {
+        const int id = ok ? __ldg(bt + (tok >> a.page_shift)) : 0;
+        if ((unsigned)id >= (unsigned)a.num_pages) {
+          bad_page = bad_page || ok;
+          ok = false;
+        }
+        roff = (int64_t)id * a.kvs[0] + (int64_t)(tok & ((1 << a.page_shift) - 1)) * a.kvs[1];
+      }
+      const __nv_bfloat16* src = (tensor ? vbase : kbase) + (ok ? roff : 0) + c16 * 8;
       cp_async_16(st + tensor * TILE_BYTES + swz_v1(row, c16), src, ok ? 16u : 0u);
     }
   };
@@ -170,6 +182,7 @@ __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs 
     __syncthreads();  // the stage and the scratch are rewritten next iteration
   }
   cp_async_wait<0>();
+  if (bad_page) report_status(a.dev_status, DIFFATTN_ERR_INVALID_ARG);
 
   // add the two key halves and write the split's partial state:
   // ws_o[((b*H + h)*splits + s)*2 + branch][128], ws_ml[...][2] = (m, l)

@@ -27,7 +27,38 @@ struct PrefillArgs {
   const float* lambda_init;
   void* out;
   int* dev_status;
+  // variable-length batch (cu_q != nullptr): sequence b is rows cu_q[b] .. cu_q[b+1] of
+  // q / out and rows cu_k[b] .. cu_k[b+1] of k / v (packed, batch stride unused); N is then
+  // the longest query count the grid covers and total_q / total_k the packed row counts
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int total_q, total_k;
 };
+
+#ifdef __CUDACC__
+// The sequence a tile of batch index b works on: its query and key counts, its first rows
+// in the tensors and its batch coordinate. ok = false for inconsistent varlen offsets.
+struct SeqRange {
+  int nq, nk, qrow0, krow0, bc;
+  bool ok;
+};
+
+__device__ __forceinline__ SeqRange seq_range(const PrefillArgs& a, int b) {
+  SeqRange r;
+  if (!a.cu_q) {
+    r.nq = a.N; r.nk = a.Nk; r.qrow0 = 0; r.krow0 = 0; r.bc = b; r.ok = true;
+    return r;
+  }
+  r.qrow0 = a.cu_q[b];
+  r.nq = a.cu_q[b + 1] - r.qrow0;
+  r.krow0 = a.cu_k[b];
+  r.nk = a.cu_k[b + 1] - r.krow0;
+  r.bc = 0;
+  r.ok = r.qrow0 >= 0 && r.nq >= 0 && r.nq <= a.N && r.qrow0 <= a.total_q - r.nq &&
+         r.krow0 >= 0 && r.nk >= r.nq && r.krow0 <= a.total_k - r.nk;
+  return r;
+}
+#endif
 
 struct DecodeArgs {
   int B, L, Hq, Hkv, d;   // V1: Hq = Hkv = H differential heads, d = branch width
@@ -41,6 +72,12 @@ struct DecodeArgs {
   const float* lambda_init;  // V1, read when apply_norm
   int apply_norm;            // V1
   float eps;                 // V1
+  // paged cache (block_table != nullptr): token t of batch entry b is row t % page_size of
+  // page block_table[b * bt_stride + t / page_size]; kvs = {page, token, head} strides
+  const int32_t* block_table;
+  int64_t bt_stride;
+  int page_shift;            // log2(page_size)
+  int num_pages;
   void* out;
   float* ws_o;   // V2: [B, Hq, splits, d]; V1: [B, H, splits, 2 branches, 2d]
   float* ws_ml;  // V2: [B, Hq, splits, 2];  V1: [B, H, splits, 2 branches, 2]

@@ -27,7 +27,16 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_f32_kernel(PrefillArgs a)
   const int i = blockIdx.x * kWarps + warp;  // query row
   const int u = blockIdx.y;                  // V1 head / V2 pair
   const int b = blockIdx.z;
-  if (i >= a.N) return;
+  // the sequence of this row (a variable-length batch packs several into one tensor)
+  const SeqRange sr = seq_range(a, b);
+  if (!sr.ok) {
+    if (i == 0 && u == 0 && threadIdx.x == 0) report_status(a.dev_status, DIFFATTN_ERR_INVALID_ARG);
+    return;
+  }
+  if (i >= sr.nq) return;
+  const int64_t qrow = (int64_t)sr.bc * a.qs[0] + (int64_t)(sr.qrow0 + i) * a.qs[1];
+  const int64_t krow0 = (int64_t)sr.bc * a.ks[0] + (int64_t)sr.krow0 * a.ks[1];
+  const int64_t vrow0 = (int64_t)sr.bc * a.vs[0] + (int64_t)sr.krow0 * a.vs[1];
   const int d = a.d, dv = a.dv;
   const float* q = static_cast<const float*>(a.q);
   const float* k = static_cast<const float*>(a.k);
@@ -35,19 +44,19 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_f32_kernel(PrefillArgs a)
 
   const float *q1, *q2, *k1, *k2, *vb;
   if (a.variant == DIFFATTN_V1) {
-    q1 = q + b * a.qs[0] + (int64_t)i * a.qs[1] + u * a.qs[2];
+    q1 = q + qrow + u * a.qs[2];
     q2 = q1 + d;
-    k1 = k + b * a.ks[0] + u * a.ks[2];
+    k1 = k + krow0 + u * a.ks[2];
     k2 = k1 + d;
-    vb = v + b * a.vs[0] + u * a.vs[2];
+    vb = v + vrow0 + u * a.vs[2];
   } else {
     const int h1 = 2 * u, h2 = 2 * u + 1;
     const int g1 = h1 / a.group, g2 = h2 / a.group;
-    q1 = q + b * a.qs[0] + (int64_t)i * a.qs[1] + h1 * a.qs[2];
-    q2 = q + b * a.qs[0] + (int64_t)i * a.qs[1] + h2 * a.qs[2];
-    k1 = k + b * a.ks[0] + g1 * a.ks[2];
-    k2 = k + b * a.ks[0] + g2 * a.ks[2];
-    vb = v + b * a.vs[0] + g1 * a.vs[2];
+    q1 = q + qrow + h1 * a.qs[2];
+    q2 = q + qrow + h2 * a.qs[2];
+    k1 = k + krow0 + g1 * a.ks[2];
+    k2 = k + krow0 + g2 * a.ks[2];
+    vb = v + vrow0 + g1 * a.vs[2];
   }
   for (int c = lane; c < d; c += 32) {
     qs[warp][0][c] = q1[c];
@@ -61,9 +70,9 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_f32_kernel(PrefillArgs a)
 #pragma unroll
   for (int t = 0; t < kPerLane; ++t) acc1[t] = acc2[t] = 0.f;
 
-  // visible keys key_lo .. n_keys - 1: query i sits at position i + Nk - N; causal stops at
+  // visible keys key_lo .. n_keys - 1: query i sits at position i + nk - nq; causal stops at
   // its own position, a sliding window keeps the last `window` of those
-  const int n_keys = a.causal ? i + (a.Nk - a.N) + 1 : a.Nk;
+  const int n_keys = a.causal ? i + (sr.nk - sr.nq) + 1 : sr.nk;
   const int key_lo = (a.causal && a.window > 0) ? max(0, n_keys - a.window) : 0;
   for (int j0 = key_lo; j0 < n_keys; j0 += 32) {
     const int j = j0 + lane;
@@ -131,7 +140,8 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_f32_kernel(PrefillArgs a)
 #pragma unroll
     for (int t = 0; t < kPerLane; ++t) o[t] = o[t] / r * sc;
   }
-  float* ob = static_cast<float*>(a.out) + b * a.os[0] + (int64_t)i * a.os[1] + u * a.os[2];
+  float* ob = static_cast<float*>(a.out) + (int64_t)sr.bc * a.os[0] +
+              (int64_t)(sr.qrow0 + i) * a.os[1] + u * a.os[2];
 #pragma unroll
   for (int t = 0; t < kPerLane; ++t) {
     const int c = lane + 32 * t;

@@ -85,6 +85,7 @@ struct Misc {
   uint64_t o_full;   // every MMA has completed
   uint32_t tmem_base;
   int abort;
+  int seq_q0, seq_bc, seq_nq;  // the tile's sequence, for the epilogue's stores
   float h_a2[2][BM];      // [tile parity][row] branch 2: rescale factor of the tile
   float h_l2[2][BM];      //                    running sum including the tile
   float ex_l[2][BM];      // epilogue: [branch][row] row sums
@@ -116,10 +117,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int u = (int)(blockIdx.x % per_qt) % a.units;
   const int b = (int)(blockIdx.x % per_qt) / a.units;
   const int q0 = qt * BM;
-  // query i sits at key position i + off (chunked prefill: the last N of Nk positions);
+  // the sequence of this tile (a variable-length batch packs several into one tensor);
+  // the whole CTA leaves before any setup when the tile lies past its sequence
+  const SeqRange sr = seq_range(a, b);
+  if (!sr.ok || q0 >= sr.nq) {
+    if (!sr.ok && threadIdx.x == 0 && q0 == 0 && u == 0)
+      report_status(a.dev_status, DIFFATTN_ERR_INVALID_ARG);
+    return;
+  }
+  // query i sits at key position i + off (chunked prefill: the last nq of nk positions);
   // this tile sees keys klo .. khi, in key tiles j_lo .. j_lo + n_kt - 1
-  const int off = a.Nk - a.N;
-  const int khi = a.causal ? min(q0 + BM - 1 + off, a.Nk - 1) : a.Nk - 1;
+  const int off = sr.nk - sr.nq;
+  const int khi = a.causal ? min(q0 + BM - 1 + off, sr.nk - 1) : sr.nk - 1;
   const int klo = WINDOW ? max(0, q0 + off - a.window + 1) : 0;
   const int j_lo = klo / BN;
   const int n_kt = (khi + BN) / BN - j_lo;
@@ -139,6 +148,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&ms.pv_done, 1);
     mbar_init(&ms.o_full, 1);
     ms.abort = 0;
+    ms.seq_q0 = sr.qrow0;
+    ms.seq_bc = sr.bc;
+    ms.seq_nq = sr.nq;
     fence_barrier_init();
   }
   if (warp == 9) {
@@ -161,8 +173,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&maps.k);
       tma_prefetch_desc(&maps.v);
       mbar_arrive_expect_tx(&ms.q_full, 2 * QBLK);
-      tma_load_4d(smem + Q_OFF + 0 * QBLK, &maps.q, &ms.q_full, 0, u, q0, b);   // q_1
-      tma_load_4d(smem + Q_OFF + 2 * QBLK, &maps.q, &ms.q_full, 64, u, q0, b);  // q_2
+      tma_load_4d(smem + Q_OFF + 0 * QBLK, &maps.q, &ms.q_full, 0, u, sr.qrow0 + q0, sr.bc);   // q_1
+      tma_load_4d(smem + Q_OFF + 2 * QBLK, &maps.q, &ms.q_full, 64, u, sr.qrow0 + q0, sr.bc);  // q_2
       int issued_k = 0, issued_v = 0;
       for (int j = 0; j < n_kt && !*abort_flag; ++j) {
         const int st = j % STAGES;
@@ -170,14 +182,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&ms.k_empty[st], par, abort_flag)) break;
         mbar_arrive_expect_tx(&ms.k_full[st], 2 * KBLK);
         uint8_t* kd = smem + K_OFF + st * 2 * KBLK;  // k_1 | k_2
-        tma_load_4d(kd, &maps.k, &ms.k_full[st], 0, u, (j_lo + j) * BN, b);
-        tma_load_4d(kd + KBLK, &maps.k, &ms.k_full[st], 64, u, (j_lo + j) * BN, b);
+        tma_load_4d(kd, &maps.k, &ms.k_full[st], 0, u, sr.krow0 + (j_lo + j) * BN, sr.bc);
+        tma_load_4d(kd + KBLK, &maps.k, &ms.k_full[st], 64, u, sr.krow0 + (j_lo + j) * BN, sr.bc);
         issued_k = j + 1;
         if (!mbar_wait(&ms.v_empty[st], par, abort_flag)) break;
         mbar_arrive_expect_tx(&ms.v_full[st], 2 * KBLK);
         uint8_t* vd = smem + V_OFF + st * 2 * KBLK;
-        tma_load_4d(vd, &maps.v, &ms.v_full[st], 0, u, (j_lo + j) * BN, b);
-        tma_load_4d(vd + KBLK, &maps.v, &ms.v_full[st], 64, u, (j_lo + j) * BN, b);
+        tma_load_4d(vd, &maps.v, &ms.v_full[st], 0, u, sr.krow0 + (j_lo + j) * BN, sr.bc);
+        tma_load_4d(vd + KBLK, &maps.v, &ms.v_full[st], 64, u, sr.krow0 + (j_lo + j) * BN, sr.bc);
         issued_v = j + 1;
       }
       if (*abort_flag) {
@@ -253,7 +265,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const float lam = a.lambda[u];
     // visible keys of this row: vlo .. vis (causal: up to its own position; window: the
     // last `window` of those)
-    const int vis = a.causal ? min(qi + off, a.Nk - 1) : a.Nk - 1;
+    const int vis = a.causal ? min(qi + off, sr.nk - 1) : sr.nk - 1;
     const int vlo = WINDOW ? max(0, vis - a.window + 1) : 0;
     // the same bounds relative to the first key of this tile's range
     const int vis0 = vis - j_lo * BN, vlo0 = vlo - j_lo * BN;
@@ -431,9 +443,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (a.apply_norm)
       sc = rsqrtf((ms.ssx[0][row] + ms.ssx[1][row]) * (1.f / 128.f) + a.eps) *
            (1.f - a.lambda_init[0]);
-    if (ok && qi < a.N) {
-      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)b * a.os[0] +
-                          (int64_t)qi * a.os[1] + (int64_t)u * a.os[2] + wg * 64;
+    if (ok && qi < ms.seq_nq) {
+      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)ms.seq_bc * a.os[0] +
+                          (int64_t)(ms.seq_q0 + qi) * a.os[1] + (int64_t)u * a.os[2] + wg * 64;
       uint4* o4 = reinterpret_cast<uint4*>(ob);
 #pragma unroll
       for (int v = 0; v < 8; ++v) {
@@ -464,9 +476,11 @@ cudaError_t launch_prefill_v1(const PrefillArgs& a, cudaStream_t stream) {
   TcMaps maps;
   // q, k viewed as [B, N, H, 128] (branch 1 in columns 0..63, branch 2 in 64..127) and v as
   // [B, N, H, 2d = 128]
-  if (!make_map(&maps.q, a.q, 128, a.units, a.N, a.B, a.qs, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.k, a.k, 128, a.units, a.Nk, a.B, a.ks, BN)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.v, a.v, 128, a.units, a.Nk, a.B, a.vs, BN)) return cudaErrorInvalidValue;
+  // a variable-length batch is one packed sequence of rows to the tensor maps
+  const int rq = a.cu_q ? a.total_q : a.N, rk = a.cu_q ? a.total_k : a.Nk, nb = a.cu_q ? 1 : a.B;
+  if (!make_map(&maps.q, a.q, 128, a.units, rq, nb, a.qs, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, 128, a.units, rk, nb, a.ks, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, 128, a.units, rk, nb, a.vs, BN)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

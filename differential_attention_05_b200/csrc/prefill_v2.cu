@@ -84,6 +84,7 @@ struct Misc {
   uint64_t o_full[2];  // [sub-tile] its last P.V MMA has completed
   uint32_t tmem_base;
   int abort;
+  int seq_q0, seq_bc, seq_nq;  // the tile's sequence, for the epilogue's stores
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -117,10 +118,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int u = (int)(blockIdx.x % per_qt) % a.units;
   const int b = (int)(blockIdx.x % per_qt) / a.units;
   const int q0 = qt * BM;
-  // query i sits at key position i + off (chunked prefill: the last N of Nk positions);
+  // the sequence of this tile (a variable-length batch packs several into one tensor);
+  // the whole CTA leaves before any setup when the tile lies past its sequence
+  const SeqRange sr = seq_range(a, b);
+  if (!sr.ok || q0 >= sr.nq) {
+    if (!sr.ok && threadIdx.x == 0 && q0 == 0 && u == 0)
+      report_status(a.dev_status, DIFFATTN_ERR_INVALID_ARG);
+    return;
+  }
+  // query i sits at key position i + off (chunked prefill: the last nq of nk positions);
   // this tile sees keys klo .. khi, in key tiles j_lo .. j_lo + n_kt - 1
-  const int off = a.Nk - a.N;
-  const int khi = a.causal ? min(q0 + BM - 1 + off, a.Nk - 1) : a.Nk - 1;
+  const int off = sr.nk - sr.nq;
+  const int khi = a.causal ? min(q0 + BM - 1 + off, sr.nk - 1) : sr.nk - 1;
   const int klo = WINDOW ? max(0, q0 + off - a.window + 1) : 0;
   const int j_lo = klo / BN;
   const int n_kt = (khi + BN) / BN - j_lo;
@@ -141,6 +150,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&ms.v_empty[s], 1);
     }
     ms.abort = 0;
+    ms.seq_q0 = sr.qrow0;
+    ms.seq_bc = sr.bc;
+    ms.seq_nq = sr.nq;
     fence_barrier_init();
   }
   if (warp == 9) {
@@ -171,7 +183,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int hf = 0; hf < 2; ++hf)
           for (int g = 0; g < 8; ++g)
             tma_load_4d(qd + hf * HALF + g * 2048, &maps.q, &ms.q_full[x], 64 * hf,
-                        2 * u + (g & 1), t0 + 16 * (g >> 1), b);
+                        2 * u + (g & 1), sr.qrow0 + t0 + 16 * (g >> 1), sr.bc);
       }
       int issued_k = 0, issued_v = 0;
       for (int j = 0; j < n_kt && !*abort_flag; ++j) {
@@ -179,15 +191,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&ms.k_empty[ks], ((j / KSTAGES) & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&ms.k_full[ks], 2 * HALF);
         uint8_t* kd = smem + K_OFF + ks * 2 * HALF;
-        tma_load_4d(kd, &maps.k, &ms.k_full[ks], 0, kvh, (j_lo + j) * BN, b);
-        tma_load_4d(kd + HALF, &maps.k, &ms.k_full[ks], 64, kvh, (j_lo + j) * BN, b);
+        tma_load_4d(kd, &maps.k, &ms.k_full[ks], 0, kvh, sr.krow0 + (j_lo + j) * BN, sr.bc);
+        tma_load_4d(kd + HALF, &maps.k, &ms.k_full[ks], 64, kvh, sr.krow0 + (j_lo + j) * BN, sr.bc);
         issued_k = j + 1;
         const int vs = j % VSTAGES;
         if (!mbar_wait(&ms.v_empty[vs], ((j / VSTAGES) & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&ms.v_full[vs], 2 * HALF);
         uint8_t* vd = smem + V_OFF + vs * 2 * HALF;
-        tma_load_4d(vd, &maps.v, &ms.v_full[vs], 0, kvh, (j_lo + j) * BN, b);
-        tma_load_4d(vd + HALF, &maps.v, &ms.v_full[vs], 64, kvh, (j_lo + j) * BN, b);
+        tma_load_4d(vd, &maps.v, &ms.v_full[vs], 0, kvh, sr.krow0 + (j_lo + j) * BN, sr.bc);
+        tma_load_4d(vd + HALF, &maps.v, &ms.v_full[vs], 64, kvh, sr.krow0 + (j_lo + j) * BN, sr.bc);
         issued_v = j + 1;
       }
       if (*abort_flag) {
@@ -284,7 +296,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const float lam = a.lambda[u];
     // visible keys of this query: vlo .. vis (causal: up to its own position, clamped for
     // the padding rows of the last tile; window: the last `window` of those)
-    const int vis = a.causal ? min(qi + off, a.Nk - 1) : a.Nk - 1;
+    const int vis = a.causal ? min(qi + off, sr.nk - 1) : sr.nk - 1;
     const int vlo = WINDOW ? max(0, vis - a.window + 1) : 0;
     float m = -INFINITY, l = 0.f;  // this lane's branch
     float c = 0.f;                 // identical in both lanes of a query
@@ -443,9 +455,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-    if (ok && qi < a.N) {
-      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)b * a.os[0] +
-                          (int64_t)qi * a.os[1] + (int64_t)u * a.os[2] + h * 64;
+    if (ok && qi < ms.seq_nq) {
+      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)ms.seq_bc * a.os[0] +
+                          (int64_t)(ms.seq_q0 + qi) * a.os[1] + (int64_t)u * a.os[2] + h * 64;
       uint4* o4 = reinterpret_cast<uint4*>(ob);
 #pragma unroll
       for (int v = 0; v < 8; ++v) {
@@ -477,9 +489,11 @@ cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream) {
   TcMaps maps;
   // q [B, N, Hq, 128], k, v [B, N, Hkv, 128]; Q boxes of 16 queries of one head (the
   // TMEM-lane row order), K and V boxes of 128 keys
-  if (!make_map(&maps.q, a.q, 128, a.Hq, a.N, a.B, a.qs, 16)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.k, a.k, 128, a.Hkv, a.Nk, a.B, a.ks, BN)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.v, a.v, 128, a.Hkv, a.Nk, a.B, a.vs, BN)) return cudaErrorInvalidValue;
+  // a variable-length batch is one packed sequence of rows to the tensor maps
+  const int rq = a.cu_q ? a.total_q : a.N, rk = a.cu_q ? a.total_k : a.Nk, nb = a.cu_q ? 1 : a.B;
+  if (!make_map(&maps.q, a.q, 128, a.Hq, rq, nb, a.qs, 16)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, 128, a.Hkv, rk, nb, a.ks, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, 128, a.Hkv, rk, nb, a.vs, BN)) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

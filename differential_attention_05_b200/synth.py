@@ -212,6 +212,36 @@ def decode_cache_slice_v1(b: int, L=32768, H=16, d=64, seed=1006, scale=None):
     return k, v
 
 
+def paginate(caches, page_size: int, seed: int, spare_pages: int = 3, fill: str = "nan"):
+    """Scatter contiguous caches [B, L, ...] (all with the same B and L) into one page pool
+    per cache, in a seeded shuffled page order, as a serving system's paged cache holds
+    them. Returns (pools [P, page_size, ...] per cache, block_table int32 [B, ceil(L /
+    page_size)]). The rows past L in each entry's last page and the spare pages hold NaN
+    (fill="nan") or N(0,1) noise (fill="noise"), so a reader that strays shows it. Inputs
+    and pools are bf16 bit arrays (uint16) or float arrays."""
+    B, L = caches[0].shape[:2]
+    n = -(-L // page_size) if L else 1
+    P = B * n + spare_pages
+    perm = np.random.default_rng(np.random.PCG64(seed)).permutation(P)
+    table = perm[:B * n].reshape(B, n).astype(np.int32)
+    pools = []
+    for ci, c in enumerate(caches):
+        assert c.shape[:2] == (B, L)
+        shape = (P, page_size) + c.shape[2:]
+        if fill == "nan":
+            pool = (np.full(shape, 0x7FC0, dtype=np.uint16) if c.dtype == np.uint16
+                    else np.full(shape, np.nan, dtype=c.dtype))
+        else:
+            noise = _normal(seed, 100 + ci, shape)
+            pool = bf16_bits(noise) if c.dtype == np.uint16 else noise.astype(c.dtype)
+        for b in range(B):
+            for i in range(n):
+                rows = c[b, i * page_size:(i + 1) * page_size]
+                pool[table[b, i], :rows.shape[0]] = rows
+        pools.append(pool)
+    return pools, table
+
+
 def signal_plus_noise(N=65536, Hq=64, Hkv=8, d=128, depth=24, seed=1004, name=None) -> Inputs:
     """Long-context signal-plus-noise workload (bf16, causal, B=1).
 

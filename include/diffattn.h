@@ -151,6 +151,35 @@ int diffattn_fwd_prefill(const diffattn_prefill_params* p, const void* q, const 
                          int* dev_status, void* stream);
 
 /*
+ * diffattn_fwd_prefill_varlen -- diffattn_fwd_prefill over a variable-length batch: S
+ * sequences of different lengths packed back to back in one tensor per operand (no
+ * padding), as a serving system batches prompts of different lengths.
+ *   p->batch      : S, the number of sequences
+ *   p->seqlen     : total packed query rows (the token extent of q and out)
+ *   p->kv_seqlen  : total packed key rows of k and v (0 reads as p->seqlen)
+ *   strides       : the batch strides are ignored; token and head strides as for the
+ *                   fixed-length call, so q is [total_q, H, 2, d] (V1) / [total_q, Hq, d]
+ *                   (V2), k and v likewise over total_k rows, out over total_q rows
+ *   cu_seqlens_q  : int32 [S + 1], device: sequence s owns query (and output) rows
+ *                   cu_seqlens_q[s] .. cu_seqlens_q[s+1] - 1
+ *   cu_seqlens_k  : int32 [S + 1], device: sequence s owns key rows
+ *                   cu_seqlens_k[s] .. cu_seqlens_k[s+1] - 1
+ *   max_seqlen_q  : HOST int, >= every sequence's query count (sizes the launch)
+ * Each sequence is one fixed-length problem: its nq queries are the last nq of its nk
+ * positions (nq <= nk; nq = nk for a plain prompt, nq < nk for a chunk after cached
+ * tokens), with p->causal and p->window as for diffattn_fwd_prefill.
+ * A sequence whose offsets are inconsistent (negative or decreasing counts, nq > nk,
+ * rows past the packed extents, nq > max_seqlen_q) is skipped -- its output rows are not
+ * written -- and DIFFATTN_ERR_INVALID_ARG is written to dev_status. Host-side errors as
+ * for diffattn_fwd_prefill; NULL offsets return DIFFATTN_ERR_INVALID_ARG.
+ */
+int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t* cu_seqlens_q,
+                                const int32_t* cu_seqlens_k, int max_seqlen_q, const void* q,
+                                const void* k, const void* v, const float* lambda,
+                                const float* lambda_init, void* out, int* dev_status,
+                                void* stream);
+
+/*
  * Decode parameters (bf16 only). V2 (diffattn_fwd_decode) below; V1 uses the same struct
  * with the layouts given at diffattn_fwd_decode_v1.
  *   q       : [B, Hq, d]        one new query token per batch entry
@@ -231,6 +260,45 @@ int diffattn_fwd_decode_v1(const diffattn_decode_params* p, const void* q, const
                            const float* lambda_init, int apply_norm, float norm_eps, void* out,
                            void* workspace, size_t workspace_bytes, int* dev_status,
                            void* stream);
+
+/*
+ * Paged KV cache (a block table over a shared page pool, the layout serving systems use
+ * for their caches; the pages name vLLM / SGLang integration as in progress). Page i of
+ * the pool holds page_size consecutive cached tokens of one batch entry, for every head.
+ * Token t of batch entry b lives in row t % page_size of page block_table[b][t / page_size].
+ */
+typedef struct {
+  int32_t page_size;         /* tokens per page: a power of two, 1 .. 65536 */
+  int32_t num_pages;         /* pages in the pool (>= 1) */
+  int32_t max_pages_per_seq; /* columns of block_table; page_size * this >= max_kv_len */
+  int32_t reserved;          /* must be 0 */
+  int64_t page_strides[3];   /* {page, token in page, head}, elements, for both pools */
+} diffattn_paged_kv;
+
+/*
+ * diffattn_fwd_decode_paged -- diffattn_fwd_decode (p->variant = DIFFATTN_V2) or
+ * diffattn_fwd_decode_v1 (DIFFATTN_V1) over a paged cache. Same kernels, arithmetic and
+ * results as the contiguous entry points: only the address of each cached row differs.
+ *   p           : as for the contiguous call; p->kv_strides is ignored
+ *   pk          : HOST pointer, the pool geometry above
+ *   k_pages     : V2 [num_pages, page_size, Hkv, d]; V1 [num_pages, page_size, H, 2, d]
+ *   v_pages     : V2 [num_pages, page_size, Hkv, d]; V1 [num_pages, page_size, H, 2d]
+ *                 (both with pk->page_strides; strides multiples of 8 elements)
+ *   block_table : int32 [B, max_pages_per_seq], device, row-major; entries for pages past
+ *                 kv_len[b] are never read
+ *   kv_len      : int32 [B] or NULL (NULL = max_kv_len), clamped to [0, max_kv_len]
+ *   lambda_init, apply_norm, norm_eps : V1 as for diffattn_fwd_decode_v1; V2: apply_norm = 0
+ *   workspace   : >= diffattn_decode_workspace_size(p) bytes, 256-byte aligned
+ * A block-table entry outside [0, num_pages) that a kernel meets writes
+ * DIFFATTN_ERR_INVALID_ARG to dev_status; the rows of that page read as zeros (no access
+ * outside the pool). Host-side errors as for the contiguous entry points.
+ */
+int diffattn_fwd_decode_paged(const diffattn_decode_params* p, const diffattn_paged_kv* pk,
+                              const void* q, const void* k_pages, const void* v_pages,
+                              const int32_t* block_table, const int32_t* kv_len,
+                              const float* lambda, const float* lambda_init, int apply_norm,
+                              float norm_eps, void* out, void* workspace, size_t workspace_bytes,
+                              int* dev_status, void* stream);
 
 /*
  * diffattn_fwd_decode_static -- diffattn_fwd_decode without a caller-provided workspace.

@@ -202,6 +202,39 @@ def prefill_v2(q, k, v, lam, causal=True, rows=None, threads=None, q_rows=None, 
     return out
 
 
+def _varlen(run, q, k, v, cu_q, cu_k, out_width):
+    """A variable-length batch is its sequences run one by one: sequence s is rows
+    cu_q[s]..cu_q[s+1] of q (and of the result) over rows cu_k[s]..cu_k[s+1] of k, v."""
+    cu_q = np.asarray(cu_q, dtype=np.int64)
+    cu_k = np.asarray(cu_k, dtype=np.int64)
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    out = np.zeros((q.shape[0],) + out_width, dtype=np.float64)
+    for s in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = cu_q[s], cu_q[s + 1], cu_k[s], cu_k[s + 1]
+        if q1 > q0:
+            out[q0:q1] = run(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1])[0]
+    return out
+
+
+def prefill_v1_varlen(q, k, v, cu_q, cu_k, lam, lambda_init_value: float, causal=True,
+                      apply_norm=True, eps=1e-5, window=0, threads=None) -> np.ndarray:
+    """V1 prefill of packed sequences. q: [Tq,H,2,d]; k: [Tk,H,2,d]; v: [Tk,H,2d]
+    -> [Tq,H,2d] (rows of no sequence stay 0)."""
+    H, d = q.shape[1], q.shape[3]
+    run = lambda qq, kk, vv: prefill_v1(qq, kk, vv, lam, lambda_init_value, causal=causal,
+                                        apply_norm=apply_norm, eps=eps, window=window,
+                                        threads=threads)
+    return _varlen(run, q, k, v, cu_q, cu_k, (H, 2 * d))
+
+
+def prefill_v2_varlen(q, k, v, cu_q, cu_k, lam, causal=True, window=0, threads=None) -> np.ndarray:
+    """V2 prefill of packed sequences. q: [Tq,Hq,d]; k,v: [Tk,Hkv,d] -> [Tq,Hq/2,d]."""
+    Hq, d = q.shape[1], q.shape[2]
+    run = lambda qq, kk, vv: prefill_v2(qq, kk, vv, lam, causal=causal, window=window,
+                                        threads=threads)
+    return _varlen(run, q, k, v, cu_q, cu_k, (Hq // 2, d))
+
+
 def decode_v2(q, k, v, lam, kv_len=None, threads=None) -> np.ndarray:
     """V2 decode. q: [B,Hq,d]; k,v: [B,L,Hkv,d]; kv_len: [B] or None -> out [B,Hq/2,d]."""
     q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
@@ -234,6 +267,30 @@ def decode_v1(q, k, v, lam, lambda_init_value: float, kv_len=None, apply_norm=Tr
     if rc != 0:
         raise ValueError(f"oracle_decode_v1 failed: {rc}")
     return out
+
+
+def gather_pages(pool, block_table) -> np.ndarray:
+    """A paged cache read back as a contiguous one: entry b's token t is row t % page_size
+    of page block_table[b, t // page_size]. pool [P, page_size, ...] -> [B, n*page_size, ...]."""
+    pool = np.asarray(pool)
+    bt = np.asarray(block_table, dtype=np.int64)
+    B, n = bt.shape
+    assert bt.min() >= 0 and bt.max() < pool.shape[0]
+    return pool[bt].reshape((B, n * pool.shape[1]) + pool.shape[2:])
+
+
+def decode_v2_paged(q, k_pool, v_pool, block_table, lam, kv_len, threads=None) -> np.ndarray:
+    """V2 decode over a paged cache: the contiguous decode of the gathered cache."""
+    return decode_v2(q, gather_pages(k_pool, block_table), gather_pages(v_pool, block_table), lam,
+                     kv_len=kv_len, threads=threads)
+
+
+def decode_v1_paged(q, k_pool, v_pool, block_table, lam, lambda_init_value: float, kv_len,
+                    apply_norm=True, eps=1e-5, threads=None) -> np.ndarray:
+    """V1 decode over a paged cache: the contiguous decode of the gathered cache."""
+    return decode_v1(q, gather_pages(k_pool, block_table), gather_pages(v_pool, block_table), lam,
+                     lambda_init_value, kv_len=kv_len, apply_norm=apply_norm, eps=eps,
+                     threads=threads)
 
 
 def map_row_v2(q, k, p: int, i: int):

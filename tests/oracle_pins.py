@@ -414,3 +414,66 @@ def pin_window_extremes():
 
 ALL_PINS += [pin_chunked_prefill_is_last_rows, pin_window_lambda0_is_banded_attention,
              pin_window_extremes]
+
+
+# ---- paged KV cache ------------------------------------------------------------------
+
+def pin_paged_decode_is_contiguous_decode():
+    """A paged cache is a storage layout: decoding it over a shuffled page pool gives, bit
+    for bit, the contiguous cache's result. Rows past kv_len and spare pages hold NaN, so a
+    read outside the entry's own keys would show."""
+    r = _rng(16)
+    B, L, Hq, Hkv, d = 3, 37, 8, 2, 4
+    q = r.standard_normal((B, Hq, d)); k = r.standard_normal((B, L, Hkv, d))
+    v = r.standard_normal((B, L, Hkv, d)); lam = r.uniform(-0.5, 1.0, Hq // 2)
+    kv_len = np.array([37, 1, 20], dtype=np.int32)
+    kn, vn = k.copy(), v.copy()
+    for b in range(B):
+        kn[b, kv_len[b]:] = np.nan
+        vn[b, kv_len[b]:] = np.nan
+    for ps in (1, 4, 16, 64):
+        (kp, vp), bt = synth.paginate([kn, vn], ps, seed=ps)
+        got = oracle.decode_v2_paged(q, kp, vp, bt, lam, kv_len, threads=1)
+        _close(got, oracle.decode_v2(q, k, v, lam, kv_len=kv_len, threads=1), 0.0, f"V2 page {ps}")
+    H = 2
+    q1 = r.standard_normal((B, H, 2, d)); k1 = r.standard_normal((B, L, H, 2, d))
+    v1 = r.standard_normal((B, L, H, 2 * d)); lam1 = np.array([0.2, 0.7])
+    k1n, v1n = k1.copy(), v1.copy()
+    for b in range(B):
+        k1n[b, kv_len[b]:] = np.nan
+        v1n[b, kv_len[b]:] = np.nan
+    (kp, vp), bt = synth.paginate([k1n, v1n], 8, seed=3)
+    got = oracle.decode_v1_paged(q1, kp, vp, bt, lam1, 0.4, kv_len, threads=1)
+    want = oracle.decode_v1(q1, k1, v1, lam1, 0.4, kv_len=kv_len, threads=1)
+    _close(got, want, 0.0, "V1 paged")
+
+
+ALL_PINS += [pin_paged_decode_is_contiguous_decode]
+
+
+# ---- variable-length batch -----------------------------------------------------------
+
+def pin_varlen_equal_lengths_is_batched():
+    """Packing B sequences of one length back to back gives the fixed-length batch's rows,
+    for plain prompts (nq = nk) and for chunks (nq < nk), V1 and V2."""
+    r = _rng(17)
+    B, Nq, Nk, H, d = 3, 5, 9, 2, 4
+    lam = np.array([0.4, -0.2])
+    cu_q = np.arange(B + 1) * Nq
+    cu_k = np.arange(B + 1) * Nk
+    q = r.standard_normal((B, Nq, H, 2, d)); k = r.standard_normal((B, Nk, H, 2, d))
+    v = r.standard_normal((B, Nk, H, 2 * d))
+    got = oracle.prefill_v1_varlen(q.reshape(B * Nq, H, 2, d), k.reshape(B * Nk, H, 2, d),
+                                   v.reshape(B * Nk, H, 2 * d), cu_q, cu_k, lam, 0.3, threads=1)
+    want = oracle.prefill_v1(q, k, v, lam, 0.3, threads=1)
+    _close(got, want.reshape(B * Nq, H, 2 * d), 0.0, "V1 packed")
+    Hq, Hkv = 4, 2
+    q2 = r.standard_normal((B, Nq, Hq, d)); k2 = r.standard_normal((B, Nk, Hkv, d))
+    v2 = r.standard_normal((B, Nk, Hkv, d))
+    got = oracle.prefill_v2_varlen(q2.reshape(B * Nq, Hq, d), k2.reshape(B * Nk, Hkv, d),
+                                   v2.reshape(B * Nk, Hkv, d), cu_q, cu_k, lam, window=3, threads=1)
+    want = oracle.prefill_v2(q2, k2, v2, lam, window=3, threads=1)
+    _close(got, want.reshape(B * Nq, Hq // 2, d), 0.0, "V2 packed")
+
+
+ALL_PINS += [pin_varlen_equal_lengths_is_batched]

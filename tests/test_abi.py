@@ -214,3 +214,57 @@ def test_selftest_timeout_rejects(lib):
     assert f(None, 100, None) == -1
     assert f(vp(GOOD), 0, None) == -1
     assert f(vp(GOOD), 10001, None) == -1
+
+
+def _paged(page_size=16, num_pages=64, max_pages=8, strides=(16 * 8 * 128, 8 * 128, 128)):
+    pk = B.PagedKV()
+    pk.page_size, pk.num_pages, pk.max_pages_per_seq = page_size, num_pages, max_pages
+    pk.page_strides[:] = strides
+    return pk
+
+
+def test_decode_paged_rejects(lib):
+    vp = ctypes.c_void_p
+    f = lib.diffattn_fwd_decode_paged
+    p = _decode_params(B_=2, L=128)
+    n = ctypes.c_size_t(0)
+    assert lib.diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    ws = vp(GOOD * 4)
+
+    def call(pk, bt=vp(GOOD + 20480), norm=0, params=p):
+        return f(ctypes.byref(params), ctypes.byref(pk), vp(GOOD), vp(GOOD + 4096), vp(GOOD + 8192),
+                 bt, None, vp(GOOD + 12288), None, norm, 1e-5, vp(GOOD + 16384), ws, n.value, None, None)
+
+    assert f(ctypes.byref(p), None, vp(GOOD), vp(GOOD), vp(GOOD), vp(GOOD), None, vp(GOOD), None, 0,
+             1e-5, vp(GOOD), ws, n.value, None, None) == -1             # no pool geometry
+    assert call(_paged(page_size=12)) == -1                             # not a power of two
+    assert call(_paged(page_size=0)) == -1
+    assert call(_paged(max_pages=7)) == -1                               # 7 x 16 < 128 keys
+    assert call(_paged(num_pages=0)) == -1
+    bad = _paged()
+    bad.reserved = 1
+    assert call(bad) == -1
+    assert call(_paged(), bt=None) == -1                                 # no block table
+    assert call(_paged(), norm=1) == -1                                  # V2 has no norm
+    assert call(_paged(strides=(16 * 8 * 128, 8 * 128 + 4, 128))) == -3  # token stride
+    pv1 = _decode_params_v1(B_=2, L=128, H=4)
+    assert call(_paged(), params=pv1, norm=1) == -1                      # V1 norm needs lambda_init
+
+
+def test_prefill_varlen_rejects(lib):
+    vp = ctypes.c_void_p
+    f = lib.diffattn_fwd_prefill_varlen
+    p = _prefill_params()
+    p.batch, p.seqlen, p.kv_seqlen = 3, 256, 300
+    for st in (p.q_strides, p.k_strides, p.v_strides, p.o_strides):
+        st[0] = 0
+    args = [vp(GOOD), vp(GOOD + 4096), vp(GOOD + 8192), vp(GOOD + 12288), None, vp(GOOD + 16384)]
+    cu_q, cu_k = vp(GOOD + 20480), vp(GOOD + 24576)
+    assert f(ctypes.byref(p), None, cu_k, 128, *args, None, None) == -1      # no offsets
+    assert f(ctypes.byref(p), cu_q, None, 128, *args, None, None) == -1
+    assert f(ctypes.byref(p), cu_q, cu_k, -1, *args, None, None) == -1       # bad max length
+    assert f(ctypes.byref(p), vp(GOOD + 20482), cu_k, 128, *args, None, None) == -3  # misaligned
+    p.window, p.causal = 8, 0
+    assert f(ctypes.byref(p), cu_q, cu_k, 128, *args, None, None) == -1      # window needs causal
+    p.window, p.causal = 0, 1
+    assert f(ctypes.byref(p), cu_q, cu_k, 0, *args, None, None) == 0         # nothing to launch
