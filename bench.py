@@ -457,7 +457,23 @@ def secondary(device, peaks, torch, da):
     res["decode"] = {"workload": "v2_bf16_decode_b64_l32768_hq64_hkv8_d128", "ms": round(ms, 4),
                      "GB/s": round(by / ms / 1e6, 1),
                      "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
-    del q, k, v, out, ws
+    # the same cache as a pool of 16-token pages in a shuffled order (block table)
+    ps = 16
+    kp, vp = k.view(B * L // ps, ps, Hkv, d), v.view(B * L // ps, ps, Hkv, d)
+    bt = torch.randperm(B * L // ps, generator=g, device=device).to(torch.int32).view(B, L // ps)
+    for _ in range(3):
+        da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws)
+    for a, b in es:
+        a.record()
+        da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws)
+        b.record()
+    torch.cuda.synchronize(device)
+    ms = statistics.median(a.elapsed_time(b) for a, b in es)
+    res["decode_paged16"] = {"workload": "v2_bf16_decode_b64_l32768_hq64_hkv8_d128, 16-token pages, "
+                             "shuffled block table", "ms": round(ms, 4),
+                             "GB/s": round(by / ms / 1e6, 1),
+                             "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    del q, k, v, out, ws, kp, vp, bt
     torch.cuda.empty_cache()
     # V1 decode: batch 32, cache 32768, 16 heads, d = 64 (the same cache bytes as above)
     B, L, H, d1 = 32, 32768, 16, 64

@@ -62,6 +62,9 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a2
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
+// PAGED: the cache is a page pool addressed through a block table (DecodeArgs); the
+// contiguous instantiation has none of that code.
+template <bool PAGED>
 __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -75,13 +78,31 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
   const int n_chunks = t_end > t_begin ? (t_end - t_begin + CH - 1) / CH : 0;
 
   // paged cache: this entry's row of the block table; the page stride replaces the batch one
-  const int32_t* bt = a.block_table ? a.block_table + (int64_t)b * a.bt_stride : nullptr;
-  const int64_t boff = bt ? 0 : b * a.kvs[0];
+  const int32_t* bt = PAGED ? a.block_table + (int64_t)b * a.bt_stride : nullptr;
+  const int64_t boff = PAGED ? 0 : b * a.kvs[0];
   const __nv_bfloat16* kbase =
       static_cast<const __nv_bfloat16*>(a.k) + boff + (int64_t)g * a.kvs[2];
   const __nv_bfloat16* vbase =
       static_cast<const __nv_bfloat16*>(a.v) + boff + (int64_t)g * a.kvs[2];
   bool bad_page = false;  // a block-table entry outside the pool: its rows read as zero
+
+  // Each thread copies the same ROWS_T rows of every chunk, (tid / CHUNKS16_PER_ROW) + RSTEP i, for K
+  // and for V. With a paged cache their page ids are fetched one chunk ahead (fetch_ids),
+  // so the table reads overlap the work on the current chunk.
+  constexpr int RSTEP = THREADS / CHUNKS16_PER_ROW;               // rows covered by one pass of the block
+  constexpr int ROWS_T = CH / RSTEP;                   // rows per thread and tensor
+  static_assert(THREADS % CHUNKS16_PER_ROW == 0 && CH % RSTEP == 0, "copy layout");
+  int pid[PAGED ? ROWS_T : 1];
+  auto fetch_ids = [&](int c) {
+    if constexpr (PAGED) {
+      const int tok0 = t_begin + c * CH + tid / CHUNKS16_PER_ROW;
+#pragma unroll
+      for (int i = 0; i < ROWS_T; ++i) {
+        const int tok = tok0 + RSTEP * i;
+        pid[i] = tok < t_end ? __ldg(bt + (tok >> a.page_shift)) : 0;
+      }
+    }
+  };
 
   // issue the copies of chunk c into stage c % STAGES (zero-fill past t_end)
   auto load_chunk = [&](int c) {
@@ -92,17 +113,19 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
       const int idx = tid + it * THREADS;
       const int tensor = idx / (CH * CHUNKS16_PER_ROW);
       const int rem = idx % (CH * CHUNKS16_PER_ROW);
-      const int row = rem / CHUNKS16_PER_ROW, c16 = rem % CHUNKS16_PER_ROW;
+      const int row = rem / CHUNKS16_PER_ROW, c16 = rem % CHUNKS16_PER_ROW;  // row = tid / CHUNKS16_PER_ROW + RSTEP (it % ROWS_T)
       const int tok = tok0 + row;
       bool ok = tok < t_end;
-      int64_t roff = (int64_t)tok * a.kvs[1];
-      if (bt) {
-        const int id = ok ? __ldg(bt + (tok >> a.page_shift)) : 0;
+      int64_t roff;
+      if constexpr (PAGED) {
+        const int id = pid[it % ROWS_T];
         if ((unsigned)id >= (unsigned)a.num_pages) {
           bad_page = bad_page || ok;
           ok = false;
         }
         roff = (int64_t)id * a.kvs[0] + (int64_t)(tok & ((1 << a.page_shift) - 1)) * a.kvs[1];
+      } else {
+        roff = (int64_t)tok * a.kvs[1];
       }
       const __nv_bfloat16* src = (tensor ? vbase : kbase) + (ok ? roff : 0) + c16 * 8;
       cp_async_16(st + tensor * TILE_BYTES + swz(row, c16), src, ok ? 16u : 0u);
@@ -130,12 +153,19 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
 
 #pragma unroll
   for (int c = 0; c < STAGES - 1; ++c) {
-    if (c < n_chunks) load_chunk(c);
+    if (c < n_chunks) {
+      fetch_ids(c);
+      load_chunk(c);
+    }
     cp_async_commit();
   }
+  if (STAGES - 1 < n_chunks) fetch_ids(STAGES - 1);
 
   for (int c = 0; c < n_chunks; ++c) {
-    if (c + STAGES - 1 < n_chunks) load_chunk(c + STAGES - 1);
+    if (c + STAGES - 1 < n_chunks) {
+      load_chunk(c + STAGES - 1);
+      if (c + STAGES < n_chunks) fetch_ids(c + STAGES);
+    }
     cp_async_commit();
     cp_async_wait<STAGES - 1>();
     __syncthreads();
@@ -299,13 +329,19 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   if (dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(decode_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set[dev] = true;
   }
   dim3 grid(a.splits, a.Hkv, a.B);
-  decode_split_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(a);
+  if (a.block_table)
+    decode_split_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(a);
+  else
+    decode_split_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 grid2(a.Hq / 2, a.B);

@@ -48,6 +48,9 @@ __device__ __forceinline__ uint32_t swz_v1(int row, int c16) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// PAGED: the cache is a page pool addressed through a block table (DecodeArgs); the
+// contiguous instantiation has none of that code.
+template <bool PAGED>
 __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t smem[];
   float* ps = reinterpret_cast<float*>(smem + RING_BYTES);  // [2][CH] probabilities
@@ -67,15 +70,33 @@ __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs 
   const int n_chunks = t_end > t_begin ? (t_end - t_begin + CH - 1) / CH : 0;
 
   // paged cache: this entry's row of the block table; the page stride replaces the batch one
-  const int32_t* bt = a.block_table ? a.block_table + (int64_t)b * a.bt_stride : nullptr;
-  const int64_t boff = bt ? 0 : b * a.kvs[0];
+  const int32_t* bt = PAGED ? a.block_table + (int64_t)b * a.bt_stride : nullptr;
+  const int64_t boff = PAGED ? 0 : b * a.kvs[0];
   const __nv_bfloat16* kbase =
       static_cast<const __nv_bfloat16*>(a.k) + boff + (int64_t)h * a.kvs[2];
   const __nv_bfloat16* vbase =
       static_cast<const __nv_bfloat16*>(a.v) + boff + (int64_t)h * a.kvs[2];
   bool bad_page = false;  // a block-table entry outside the pool: its rows read as zero
 
-  // copies of chunk c into stage c % STAGES (zero-fill past t_end)
+  // Each thread copies the same ROWS_T rows of every chunk, (tid / C16) + RSTEP i, for K
+  // and for V. With a paged cache their page ids are fetched one chunk ahead (fetch_ids),
+  // so the table reads overlap the work on the current chunk.
+  constexpr int RSTEP = THREADS / C16;               // rows covered by one pass of the block
+  constexpr int ROWS_T = CH / RSTEP;                   // rows per thread and tensor
+  static_assert(THREADS % C16 == 0 && CH % RSTEP == 0, "copy layout");
+  int pid[PAGED ? ROWS_T : 1];
+  auto fetch_ids = [&](int c) {
+    if constexpr (PAGED) {
+      const int tok0 = t_begin + c * CH + tid / C16;
+#pragma unroll
+      for (int i = 0; i < ROWS_T; ++i) {
+        const int tok = tok0 + RSTEP * i;
+        pid[i] = tok < t_end ? __ldg(bt + (tok >> a.page_shift)) : 0;
+      }
+    }
+  };
+
+  // issue the copies of chunk c into stage c % STAGES (zero-fill past t_end)
   auto load_chunk = [&](int c) {
     uint8_t* st = smem + (c % STAGES) * STAGE_BYTES;
     const int tok0 = t_begin + c * CH;
@@ -84,17 +105,19 @@ __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs 
       const int idx = tid + it * THREADS;
       const int tensor = idx / (CH * C16);
       const int rem = idx % (CH * C16);
-      const int row = rem / C16, c16 = rem % C16;
+      const int row = rem / C16, c16 = rem % C16;  // row = tid / C16 + RSTEP (it % ROWS_T)
       const int tok = tok0 + row;
       bool ok = tok < t_end;
-      int64_t roff = (int64_t)tok * a.kvs[1];
-      if (bt) {
-        const int id = ok ? __ldg(bt + (tok >> a.page_shift)) : 0;
+      int64_t roff;
+      if constexpr (PAGED) {
+        const int id = pid[it % ROWS_T];
         if ((unsigned)id >= (unsigned)a.num_pages) {
           bad_page = bad_page || ok;
           ok = false;
         }
         roff = (int64_t)id * a.kvs[0] + (int64_t)(tok & ((1 << a.page_shift) - 1)) * a.kvs[1];
+      } else {
+        roff = (int64_t)tok * a.kvs[1];
       }
       const __nv_bfloat16* src = (tensor ? vbase : kbase) + (ok ? roff : 0) + c16 * 8;
       cp_async_16(st + tensor * TILE_BYTES + swz_v1(row, c16), src, ok ? 16u : 0u);
@@ -122,12 +145,19 @@ __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs 
 
 #pragma unroll
   for (int c = 0; c < STAGES - 1; ++c) {
-    if (c < n_chunks) load_chunk(c);
+    if (c < n_chunks) {
+      fetch_ids(c);
+      load_chunk(c);
+    }
     cp_async_commit();
   }
+  if (STAGES - 1 < n_chunks) fetch_ids(STAGES - 1);
 
   for (int c = 0; c < n_chunks; ++c) {
-    if (c + STAGES - 1 < n_chunks) load_chunk(c + STAGES - 1);
+    if (c + STAGES - 1 < n_chunks) {
+      load_chunk(c + STAGES - 1);
+      if (c + STAGES < n_chunks) fetch_ids(c + STAGES);
+    }
     cp_async_commit();
     cp_async_wait<STAGES - 1>();
     __syncthreads();
@@ -259,12 +289,18 @@ cudaError_t launch_decode_v1(const DecodeArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   if (dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(decode_v1_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_v1_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(decode_v1_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set[dev] = true;
   }
-  decode_v1_split_kernel<<<dim3(a.splits, a.Hq, a.B), THREADS, SMEM_BYTES, stream>>>(a);
+  if (a.block_table)
+    decode_v1_split_kernel<true><<<dim3(a.splits, a.Hq, a.B), THREADS, SMEM_BYTES, stream>>>(a);
+  else
+    decode_v1_split_kernel<false><<<dim3(a.splits, a.Hq, a.B), THREADS, SMEM_BYTES, stream>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_v1_combine_kernel<<<dim3(a.Hq, a.B), DV, 0, stream>>>(a);

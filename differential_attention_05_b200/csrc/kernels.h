@@ -43,9 +43,10 @@ struct SeqRange {
   bool ok;
 };
 
+template <bool VARLEN = true>
 __device__ __forceinline__ SeqRange seq_range(const PrefillArgs& a, int b) {
   SeqRange r;
-  if (!a.cu_q) {
+  if (!VARLEN || !a.cu_q) {
     r.nq = a.N; r.nk = a.Nk; r.qrow0 = 0; r.krow0 = 0; r.bc = b; r.ok = true;
     return r;
   }

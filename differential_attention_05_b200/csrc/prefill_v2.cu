@@ -102,7 +102,9 @@ __device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t bytes) {
 // WINDOW: a causal sliding window (a.window > 0). Without one every row sees key 0, the
 // first key of the first tile, so the row state is set after tile 0 and the masks have
 // only an upper end; that case compiles without the lower-end and unset-row checks.
-template <bool WINDOW>
+// VARLEN: a variable-length batch (a.cu_q != nullptr); the fixed-length instantiation
+// takes its sizes from the parameters alone.
+template <bool WINDOW, bool VARLEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_v2_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -120,8 +122,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int q0 = qt * BM;
   // the sequence of this tile (a variable-length batch packs several into one tensor);
   // the whole CTA leaves before any setup when the tile lies past its sequence
-  const SeqRange sr = seq_range(a, b);
-  if (!sr.ok || q0 >= sr.nq) {
+  const SeqRange sr = seq_range<VARLEN>(a, b);
+  if (VARLEN && (!sr.ok || q0 >= sr.nq)) {
     if (!sr.ok && threadIdx.x == 0 && q0 == 0 && u == 0)
       report_status(a.dev_status, DIFFATTN_ERR_INVALID_ARG);
     return;
@@ -150,9 +152,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&ms.v_empty[s], 1);
     }
     ms.abort = 0;
-    ms.seq_q0 = sr.qrow0;
-    ms.seq_bc = sr.bc;
-    ms.seq_nq = sr.nq;
+    if (VARLEN) {
+      ms.seq_q0 = sr.qrow0;
+      ms.seq_bc = sr.bc;
+      ms.seq_nq = sr.nq;
+    }
     fence_barrier_init();
   }
   if (warp == 9) {
@@ -455,9 +459,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
     }
-    if (ok && qi < ms.seq_nq) {
-      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)ms.seq_bc * a.os[0] +
-                          (int64_t)(ms.seq_q0 + qi) * a.os[1] + (int64_t)u * a.os[2] + h * 64;
+    // (a variable-length tile reads its sequence back from shared memory, keeping the
+    // registers of the key loop free)
+    const int o_nq = VARLEN ? ms.seq_nq : a.N, o_b = VARLEN ? ms.seq_bc : b;
+    const int o_q0 = VARLEN ? ms.seq_q0 : 0;
+    if (ok && qi < o_nq) {
+      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)o_b * a.os[0] +
+                          (int64_t)(o_q0 + qi) * a.os[1] + (int64_t)u * a.os[2] + h * 64;
       uint4* o4 = reinterpret_cast<uint4*>(ob);
 #pragma unroll
       for (int v = 0; v < 8; ++v) {
@@ -499,20 +507,25 @@ cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   if (dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(prefill_v2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(prefill_v2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    const void* fns[4] = {(const void*)prefill_v2_kernel<false, false>, (const void*)prefill_v2_kernel<true, false>,
+                          (const void*)prefill_v2_kernel<false, true>, (const void*)prefill_v2_kernel<true, true>};
+    for (const void* fn : fns) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+    }
     if (dev < 64) attr_set[dev] = true;
   }
   const long long tiles = (long long)((a.N + BM - 1) / BM) * a.units * a.B;
   if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  if (a.causal && a.window > 0)
-    prefill_v2_kernel<true><<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
-  else
-    prefill_v2_kernel<false><<<(unsigned)tiles, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  const bool window = a.causal && a.window > 0, varlen = a.cu_q != nullptr;
+  const dim3 grid((unsigned)tiles);
+  if (varlen) {
+    if (window) prefill_v2_kernel<true, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+    else prefill_v2_kernel<false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  } else {
+    if (window) prefill_v2_kernel<true, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+    else prefill_v2_kernel<false, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  }
   return cudaGetLastError();
 }
 
