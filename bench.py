@@ -98,18 +98,28 @@ def load_peaks():
                 "source": "fallback"}
 
 
-def measured_traffic(kernel: str, workload_batch_scale: float = 1.0):
-    """DRAM bytes per launch of `kernel` from the committed ncu record (profiles/traffic.txt),
-    or None when the kernel's sources changed since the capture."""
+def measured_traffic(kernel: str, workload: str, batch: int, decode: bool):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu record
+    (profiles/traffic.txt), or None when the kernel's sources changed since the capture or
+    no capture covers the workload. A decode capture at a smaller batch of the same cache
+    shape is scaled by the batch ratio (every batch entry reads its own cache once)."""
     import hashlib
+    import re
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     csrc = os.path.join(ROOT, "differential_attention_05_b200", "csrc")
     try:
         lines = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
     except OSError:
         return None
+    strip = lambda w: re.sub(r"_b\d+_", "_b*_", w)
     for f in lines:
         if len(f) != 5 or f[0] != kernel:
+            continue
+        if f[1] == workload:
+            scale = 1.0
+        elif decode and strip(f[1]) == strip(workload):
+            scale = batch / float(re.search(r"_b(\d+)_", f[1]).group(1))
+        else:
             continue
         m = hashlib.sha256()
         try:
@@ -119,7 +129,7 @@ def measured_traffic(kernel: str, workload_batch_scale: float = 1.0):
             return None
         if m.hexdigest()[:16] != f[2]:
             return None
-        return float(f[4]) * workload_batch_scale
+        return float(f[4]) * scale
     return None
 
 
@@ -343,11 +353,7 @@ def run_ours(args, rank, world, device):
 
     kernel_name = (("decode_v1_split_kernel" if inp.variant == 1 else "decode_split_kernel")
                    if decode else f"prefill_v{inp.variant}_kernel")
-    # decode traffic was captured at batch 8 and grows in proportion to the batch
-    traffic = measured_traffic(kernel_name, inp.B / 8.0 if decode else 1.0)
-    if traffic is not None and not decode and inp.name not in (
-            "v1_bf16_layer_b2_h16_n4096_d64", "v2_bf16_prefill_b1_n16384_hq64_hkv8_d128"):
-        traffic = None
+    traffic = measured_traffic(kernel_name, inp.name, inp.B, decode)
     line = {
         "metric": metric,
         "value": round(value, 3),
@@ -457,22 +463,26 @@ def secondary(device, peaks, torch, da):
     res["decode"] = {"workload": "v2_bf16_decode_b64_l32768_hq64_hkv8_d128", "ms": round(ms, 4),
                      "GB/s": round(by / ms / 1e6, 1),
                      "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
-    # the same cache as a pool of 16-token pages in a shuffled order (block table)
-    ps = 16
-    kp, vp = k.view(B * L // ps, ps, Hkv, d), v.view(B * L // ps, ps, Hkv, d)
-    bt = torch.randperm(B * L // ps, generator=g, device=device).to(torch.int32).view(B, L // ps)
-    for _ in range(3):
-        da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws)
-    for a, b in es:
-        a.record()
-        da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws)
-        b.record()
-    torch.cuda.synchronize(device)
-    ms = statistics.median(a.elapsed_time(b) for a, b in es)
-    res["decode_paged16"] = {"workload": "v2_bf16_decode_b64_l32768_hq64_hkv8_d128, 16-token pages, "
-                             "shuffled block table", "ms": round(ms, 4),
-                             "GB/s": round(by / ms / 1e6, 1),
-                             "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    # the same cache as a page pool: 16-token pages in a shuffled order (block table), the
+    # same pages in order (the paging arithmetic alone), 256-token pages shuffled
+    for ps, shuffled in ((16, True), (16, False), (256, True)):
+        kp, vp = k.view(B * L // ps, ps, Hkv, d), v.view(B * L // ps, ps, Hkv, d)
+        ids = (torch.randperm(B * L // ps, generator=g, device=device) if shuffled
+               else torch.arange(B * L // ps, device=device))
+        bt = ids.to(torch.int32).view(B, L // ps)
+        for _ in range(3):
+            da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws)
+        for a, b in es:
+            a.record()
+            da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws)
+            b.record()
+        torch.cuda.synchronize(device)
+        ms = statistics.median(a.elapsed_time(b) for a, b in es)
+        res[f"decode_paged{ps}_{'shuffled' if shuffled else 'in_order'}"] = {
+            "workload": f"v2_bf16_decode_b64_l32768_hq64_hkv8_d128, {ps}-token pages, "
+                        f"{'shuffled' if shuffled else 'in-order'} block table",
+            "ms": round(ms, 4), "GB/s": round(by / ms / 1e6, 1),
+            "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
     del q, k, v, out, ws, kp, vp, bt
     torch.cuda.empty_cache()
     # V1 decode: batch 32, cache 32768, 16 heads, d = 64 (the same cache bytes as above)
