@@ -477,3 +477,93 @@ def pin_varlen_equal_lengths_is_batched():
 
 
 ALL_PINS += [pin_varlen_equal_lengths_is_batched]
+
+
+# ---- backward ------------------------------------------------------------------------
+
+from oracle import backward as OB  # noqa: E402
+
+
+def _fd(f, x, h=1e-5):
+    """Central differences of the scalar function f at every element of array x."""
+    g = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        x0 = x[i]
+        x[i] = x0 + h
+        fp = f()
+        x[i] = x0 - h
+        fm = f()
+        x[i] = x0
+        g[i] = (fp - fm) / (2 * h)
+    return g
+
+
+def pin_backward_finite_differences():
+    """The backward oracle against central differences of the FORWARD C oracle (a separate
+    code base) on tiny inputs: V1 with the norm and a chunk (Nq < Nk), V2 with GQA and a
+    window; then the lambda vectors through the lambda oracle."""
+    r = _rng(18)
+    B, Nq, Nk, H, d = 1, 3, 5, 2, 3
+    q = r.standard_normal((B, Nq, H, 2, d)); k = r.standard_normal((B, Nk, H, 2, d))
+    v = r.standard_normal((B, Nk, H, 2 * d)); lam = np.array([0.35, -0.2]); li = 0.3
+    R = r.standard_normal((B, Nq, H, 2 * d))
+    loss = lambda: float(np.sum(oracle.prefill_v1(q, k, v, lam, li, eps=1e-3, threads=1) * R))
+    dq, dk, dv, dl = OB.prefill_v1_bwd(q, k, v, lam, li, R, eps=1e-3)
+    for name, x, g in (("dq", q, dq), ("dk", k, dk), ("dv", v, dv), ("dlambda", lam, dl)):
+        _close(g, _fd(loss, x), 2e-7, f"V1 {name}")
+    Hq, Hkv, Nq2, Nk2 = 4, 1, 4, 6
+    q = r.standard_normal((B, Nq2, Hq, d)); k = r.standard_normal((B, Nk2, Hkv, d))
+    v = r.standard_normal((B, Nk2, Hkv, d)); lam = np.array([0.6, 0.1])
+    R = r.standard_normal((B, Nq2, Hq // 2, d))
+    loss = lambda: float(np.sum(oracle.prefill_v2(q, k, v, lam, window=3, threads=1) * R))
+    dq, dk, dv, dl = OB.prefill_v2_bwd(q, k, v, lam, R, window=3)
+    for name, x, g in (("dq", q, dq), ("dk", k, dk), ("dv", v, dv), ("dlambda", lam, dl)):
+        _close(g, _fd(loss, x), 2e-7, f"V2 {name}")
+    vecs = [0.3 * r.standard_normal((Hq // 2, 4)) for _ in range(4)]
+    dlam = r.standard_normal(Hq // 2)
+    lossl = lambda: float(np.sum(oracle.lambda_(*vecs, depth=2) * dlam))
+    for x, g in zip(vecs, OB.lambda_bwd(*vecs, dlam)):
+        _close(g, _fd(lossl, x), 2e-7, "lambda vectors")
+
+
+def pin_backward_autograd():
+    """The backward oracle against torch autograd (float64) through the printed operator
+    (softmax, matmul, rms_norm), causal and full, V1 and V2 with GQA."""
+    r = _rng(19)
+    B, N, H, d = 2, 7, 2, 4
+    for causal in (True, False):
+        q = r.standard_normal((B, N, H, 2, d)); k = r.standard_normal((B, N, H, 2, d))
+        v = r.standard_normal((B, N, H, 2 * d)); lam = np.array([0.8, -0.3]); li = 0.45
+        dy = r.standard_normal((B, N, H, 2 * d))
+        tq, tk, tv, tl = (torch.tensor(x, requires_grad=True) for x in (q, k, v, lam))
+        mask = torch.ones(N, N, dtype=torch.bool).tril() if causal else torch.ones(N, N, dtype=torch.bool)
+        def attn(qb, kb):
+            s = torch.einsum("bihd,bjhd->bhij", qb, kb) / math.sqrt(d)
+            return torch.softmax(s.masked_fill(~mask, float("-inf")), dim=-1)
+        a1, a2 = attn(tq[:, :, :, 0], tk[:, :, :, 0]), attn(tq[:, :, :, 1], tk[:, :, :, 1])
+        vv = tv.permute(0, 2, 1, 3)
+        o = (a1 @ vv - tl[None, :, None, None] * (a2 @ vv)).permute(0, 2, 1, 3)
+        y = torch.nn.functional.rms_norm(o, (2 * d,), eps=1e-5) * (1 - li)
+        (y * torch.tensor(dy)).sum().backward()
+        got = OB.prefill_v1_bwd(q, k, v, lam, li, dy, causal=causal)
+        for g, t, name in zip(got, (tq, tk, tv, tl), ("dq", "dk", "dv", "dlambda")):
+            _close(g, t.grad.numpy(), 1e-11, f"V1 autograd {name} causal={causal}")
+        Hq, Hkv = 8, 2
+        q = r.standard_normal((B, N, Hq, d)); k = r.standard_normal((B, N, Hkv, d))
+        v = r.standard_normal((B, N, Hkv, d)); lam = r.uniform(-0.5, 1, Hq // 2)
+        dy = r.standard_normal((B, N, Hq // 2, d))
+        tq, tk, tv, tl = (torch.tensor(x, requires_grad=True) for x in (q, k, v, lam))
+        kr = tk.repeat_interleave(Hq // Hkv, dim=2)
+        vr = tv.repeat_interleave(Hq // Hkv, dim=2)
+        a = attn(tq, kr)                                   # [B, Hq, N, N]
+        o = a @ vr.permute(0, 2, 1, 3)                     # [B, Hq, N, d]
+        y = (o[:, 0::2] - tl[None, :, None, None] * o[:, 1::2]).permute(0, 2, 1, 3)
+        (y * torch.tensor(dy)).sum().backward()
+        got = OB.prefill_v2_bwd(q, k, v, lam, dy, causal=causal)
+        for g, t, name in zip(got, (tq, tk, tv, tl), ("dq", "dk", "dv", "dlambda")):
+            _close(g, t.grad.numpy(), 1e-11, f"V2 autograd {name} causal={causal}")
+
+
+ALL_PINS += [pin_backward_finite_differences, pin_backward_autograd]
