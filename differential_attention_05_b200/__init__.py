@@ -9,6 +9,9 @@ from ._binding import (  # noqa: F401
     diffattn_lambda,
     diffattn_fwd_prefill,
     diffattn_fwd_prefill_varlen,
+    diffattn_bwd_prefill,
+    diffattn_bwd_workspace_size,
+    diffattn_lambda_bwd,
     diffattn_fwd_decode,
     diffattn_fwd_decode_static,
     diffattn_fwd_decode_v1,
@@ -25,6 +28,9 @@ __all__ = [
     "diffattn_lambda",
     "diffattn_fwd_prefill",
     "diffattn_fwd_prefill_varlen",
+    "diffattn_bwd_prefill",
+    "diffattn_bwd_workspace_size",
+    "diffattn_lambda_bwd",
     "diffattn_fwd_decode",
     "diffattn_fwd_decode_static",
     "diffattn_fwd_decode_v1",

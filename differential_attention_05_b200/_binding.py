@@ -33,6 +33,9 @@ EXPORTS = (
     "diffattn_lambda",
     "diffattn_fwd_prefill",
     "diffattn_fwd_prefill_varlen",
+    "diffattn_bwd_workspace_size",
+    "diffattn_bwd_prefill",
+    "diffattn_lambda_bwd",
     "diffattn_decode_workspace_size",
     "diffattn_fwd_decode",
     "diffattn_fwd_decode_static",
@@ -116,6 +119,14 @@ def load_library():
     lib.diffattn_fwd_prefill_varlen.restype = i32
     lib.diffattn_fwd_prefill_varlen.argtypes = [ctypes.POINTER(PrefillParams), vp, vp, i32, vp, vp,
                                                 vp, f32p, f32p, vp, vp, vp]
+    lib.diffattn_bwd_workspace_size.restype = i32
+    lib.diffattn_bwd_workspace_size.argtypes = [ctypes.POINTER(PrefillParams),
+                                                ctypes.POINTER(ctypes.c_size_t)]
+    lib.diffattn_bwd_prefill.restype = i32
+    lib.diffattn_bwd_prefill.argtypes = [ctypes.POINTER(PrefillParams), vp, vp, vp, f32p, f32p, vp,
+                                         vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
+    lib.diffattn_lambda_bwd.restype = i32
+    lib.diffattn_lambda_bwd.argtypes = [f32p, f32p, f32p, f32p, i32, i32, f32p, vp, vp, vp, vp, vp]
     lib.diffattn_decode_workspace_size.restype = i32
     lib.diffattn_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeParams),
                                                    ctypes.POINTER(ctypes.c_size_t)]
@@ -281,6 +292,49 @@ def diffattn_fwd_prefill_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_
                                          _stream(stream))
     _check("diffattn_fwd_prefill_varlen", rc)
     return out
+
+
+def diffattn_bwd_workspace_size(p: PrefillParams) -> int:
+    n = ctypes.c_size_t(0)
+    _check("diffattn_bwd_workspace_size",
+           load_library().diffattn_bwd_workspace_size(ctypes.byref(p), ctypes.byref(n)))
+    return int(n.value)
+
+
+def diffattn_bwd_prefill(q, k, v, lam, dout, lambda_init=None, causal=True, apply_norm=None,
+                         norm_eps=1e-5, window=0, workspace=None, dev_status=None, stream=None):
+    """Gradients of diffattn_fwd_prefill (see include/diffattn.h): dout has the forward
+    output's layout and dtype. Returns float32 (dq, dk, dv, dlambda) in the shapes of q, k,
+    v and lambda."""
+    import torch
+    lib = load_library()
+    p = prefill_params(q, k, v, dout, causal, apply_norm, norm_eps, window)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    dl = torch.empty(lam.shape, dtype=torch.float32, device=q.device)
+    need = diffattn_bwd_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib.diffattn_bwd_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lam),
+                                  _ptr(lambda_init), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                  _ptr(dl), _ptr(workspace), ws_bytes, _ptr(dev_status),
+                                  _stream(stream))
+    _check("diffattn_bwd_prefill", rc)
+    return dq, dk, dv, dl
+
+
+def diffattn_lambda_bwd(lq1, lk1, lq2, lk2, dlambda, stream=None):
+    """Gradients of the four [n_heads, dim] lambda vectors from dL/dlambda [n_heads]."""
+    import torch
+    lib = load_library()
+    H, dim = lq1.shape
+    outs = [torch.empty((H, dim), dtype=torch.float32, device=lq1.device) for _ in range(4)]
+    rc = lib.diffattn_lambda_bwd(_ptr(lq1), _ptr(lk1), _ptr(lq2), _ptr(lk2), H, dim, _ptr(dlambda),
+                                 *[_ptr(o) for o in outs], _stream(stream))
+    _check("diffattn_lambda_bwd", rc)
+    return tuple(outs)
 
 
 def decode_params(q, k_cache, v_cache, out, num_splits=0) -> DecodeParams:

@@ -64,9 +64,13 @@ int diffattn_lambda(const float* lq1, const float* lk1, const float* lq2, const 
 // p->batch sequences of p->seqlen queries and kv_seqlen keys. Otherwise p->batch packed
 // sequences with offsets cu_q / cu_k (device), p->seqlen / kv_seqlen the packed row counts
 // and max_q the longest query count.
-static int prefill_run(const diffattn_prefill_params* p, const int32_t* cu_q, const int32_t* cu_k,
-                       int max_q, const void* q, const void* k, const void* v, const float* lambda,
-                       const float* lambda_init, void* out, int* dev_status, void* stream) {
+// Checks shared by the forward and the backward and the resolved arguments; *empty is set
+// when there is nothing to launch.
+static int prefill_setup(const diffattn_prefill_params* p, const int32_t* cu_q, const int32_t* cu_k,
+                         int max_q, const void* q, const void* k, const void* v,
+                         const float* lambda, const float* lambda_init, const void* out,
+                         int* dev_status, PrefillArgs* pa, bool* empty) {
+  *empty = false;
   if (!p) return DIFFATTN_ERR_INVALID_ARG;
   if (p->batch < 0 || p->seqlen < 0 || p->head_dim < 1) return DIFFATTN_ERR_INVALID_ARG;
   if (p->variant != DIFFATTN_V1 && p->variant != DIFFATTN_V2) return DIFFATTN_ERR_INVALID_ARG;
@@ -84,7 +88,7 @@ static int prefill_run(const diffattn_prefill_params* p, const int32_t* cu_q, co
       !strides_ok(p->v_strides, 3) || !strides_ok(p->o_strides, 3))
     return DIFFATTN_ERR_INVALID_ARG;
 
-  PrefillArgs a;
+  PrefillArgs& a = *pa;
   memset(&a, 0, sizeof(a));
   a.variant = p->variant;
   a.B = p->batch;
@@ -120,7 +124,10 @@ static int prefill_run(const diffattn_prefill_params* p, const int32_t* cu_q, co
   }
   if (a.apply_norm && !(p->norm_eps >= 0.f && isfinite(p->norm_eps))) return DIFFATTN_ERR_INVALID_ARG;
   if (a.units > 65535 || a.B > 65535) return DIFFATTN_ERR_UNSUPPORTED;
-  if (a.B == 0 || a.N == 0 || (varlen && p->seqlen == 0)) return DIFFATTN_OK;
+  if (a.B == 0 || a.N == 0 || (varlen && p->seqlen == 0)) {
+    *empty = true;
+    return DIFFATTN_OK;
+  }
   if (!q || !k || !v || !lambda || !out) return DIFFATTN_ERR_INVALID_ARG;
   if (a.apply_norm && !lambda_init) return DIFFATTN_ERR_INVALID_ARG;
   if (out == q || out == k || out == v) return DIFFATTN_ERR_INVALID_ARG;
@@ -143,10 +150,20 @@ static int prefill_run(const diffattn_prefill_params* p, const int32_t* cu_q, co
   a.v = v;
   a.lambda = lambda;
   a.lambda_init = lambda_init;
-  a.out = out;
+  a.out = const_cast<void*>(out);
   a.dev_status = dev_status;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return DIFFATTN_OK;
+}
 
+static int prefill_run(const diffattn_prefill_params* p, const int32_t* cu_q, const int32_t* cu_k,
+                       int max_q, const void* q, const void* k, const void* v, const float* lambda,
+                       const float* lambda_init, void* out, int* dev_status, void* stream) {
+  PrefillArgs a;
+  bool empty = false;
+  const int rc = prefill_setup(p, cu_q, cu_k, max_q, q, k, v, lambda, lambda_init, out, dev_status,
+                               &a, &empty);
+  if (rc != DIFFATTN_OK || empty) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (p->dtype == DIFFATTN_F32) {
     if (a.d > 128 || a.d % 4 != 0) return DIFFATTN_ERR_UNSUPPORTED;
     return from_cuda(launch_prefill_f32(a, s));
@@ -174,6 +191,74 @@ int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t*
   if (!cu_seqlens_q || !cu_seqlens_k) return DIFFATTN_ERR_INVALID_ARG;
   return prefill_run(p, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, q, k, v, lambda, lambda_init,
                      out, dev_status, stream);
+}
+
+// backward: any d <= 128 with d % 4 == 0, f32 or bf16 inputs, fixed-length batches
+static int bwd_check(const diffattn_prefill_params* p) {
+  if (!p) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->head_dim > 128 || p->head_dim % 4 != 0) return DIFFATTN_ERR_UNSUPPORTED;
+  return DIFFATTN_OK;
+}
+
+int diffattn_bwd_workspace_size(const diffattn_prefill_params* p, size_t* bytes) {
+  if (!bytes) return DIFFATTN_ERR_INVALID_ARG;
+  const int rc = bwd_check(p);
+  if (rc != DIFFATTN_OK) return rc;
+  if (p->batch < 0 || p->seqlen < 0 || p->head_dim < 1) return DIFFATTN_ERR_INVALID_ARG;
+  int units, dv;
+  if (p->variant == DIFFATTN_V1) {
+    if (p->n_q_heads < 1 || p->n_kv_heads != p->n_q_heads) return DIFFATTN_ERR_INVALID_ARG;
+    units = p->n_q_heads;
+    dv = 2 * p->head_dim;
+  } else if (p->variant == DIFFATTN_V2) {
+    if (p->n_q_heads < 2 || p->n_kv_heads < 1 || p->n_q_heads % p->n_kv_heads != 0 ||
+        (p->n_q_heads / p->n_kv_heads) % 2 != 0)
+      return DIFFATTN_ERR_INVALID_ARG;
+    units = p->n_q_heads / 2;
+    dv = p->head_dim;
+  } else {
+    return DIFFATTN_ERR_INVALID_ARG;
+  }
+  *bytes = bwd_workspace_bytes(p->batch, p->seqlen, units, dv);
+  return DIFFATTN_OK;
+}
+
+int diffattn_bwd_prefill(const diffattn_prefill_params* p, const void* q, const void* k,
+                         const void* v, const float* lambda, const float* lambda_init,
+                         const void* dout, float* dq, float* dk, float* dv, float* dlambda,
+                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  int rc = bwd_check(p);
+  if (rc != DIFFATTN_OK) return rc;
+  BwdArgs g;
+  memset(&g, 0, sizeof(g));
+  bool empty = false;
+  rc = prefill_setup(p, nullptr, nullptr, 0, q, k, v, lambda, lambda_init, dout, dev_status, &g.f,
+                     &empty);
+  if (rc != DIFFATTN_OK || empty) return rc;
+  if (!dout || !dq || !dk || !dv || !dlambda) return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return DIFFATTN_ERR_MISALIGNED;
+  const PrefillArgs& a = g.f;
+  const size_t need = bwd_workspace_bytes(a.B, a.N, a.units, a.dv);
+  if (!workspace || workspace_bytes < need) return DIFFATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIFFATTN_ERR_MISALIGNED;
+  g.bf16 = p->dtype == DIFFATTN_BF16;
+  g.dy = dout;
+  memcpy(g.dys, p->o_strides, sizeof(g.dys));
+  g.dq = dq;
+  g.dk = dk;
+  g.dv = dv;
+  g.dlambda = dlambda;
+  return from_cuda(launch_backward(g, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+int diffattn_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
+                        int n_heads, int dim, const float* dlambda, float* dlq1, float* dlk1,
+                        float* dlq2, float* dlk2, void* stream) {
+  if (!lq1 || !lk1 || !lq2 || !lk2 || !dlambda || !dlq1 || !dlk1 || !dlq2 || !dlk2)
+    return DIFFATTN_ERR_INVALID_ARG;
+  if (n_heads < 1 || n_heads > 65535 || dim < 1 || dim > 4096) return DIFFATTN_ERR_INVALID_ARG;
+  return from_cuda(launch_lambda_bwd(lq1, lk1, lq2, lk2, n_heads, dim, dlambda, dlq1, dlk1, dlq2,
+                                     dlk2, static_cast<cudaStream_t>(stream)));
 }
 
 static int decode_check(const diffattn_decode_params* p, int* splits, int* split_len) {

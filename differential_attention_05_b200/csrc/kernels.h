@@ -35,6 +35,23 @@ struct PrefillArgs {
   int total_q, total_k;
 };
 
+// Resolved backward problem: the forward's arguments plus the incoming gradient dy (the
+// layout of out) and the fp32 gradients, dense in the shapes of q, k, v; the workspace
+// pointers are set by launch_backward.
+struct BwdArgs {
+  PrefillArgs f;
+  int bf16;                  // q, k, v, dy are bf16 (else fp32)
+  const void* dy;
+  int64_t dys[3];            // dy strides {batch, token, unit}
+  float* dq;
+  float* dk;
+  float* dv;
+  float* dlambda;            // [units]
+  float* w_do;               // [B, N, units, dv] gradient reaching O
+  float* w_st;               // [B, N, units, 4] lse_1, lse_2, delta_1, delta_2
+  float* w_dl;               // [B, units, N] per-row dlambda shares
+};
+
 #ifdef __CUDACC__
 // The sequence a tile of batch index b works on: its query and key counts, its first rows
 // in the tensors and its batch coordinate. ok = false for inconsistent varlen offsets.
@@ -106,5 +123,11 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // cores; per-head RMSNorm and (1 - lambda_init) scale in the merge
 int decode_v1_default_splits(int B, int L, int H);
 cudaError_t launch_decode_v1(const DecodeArgs& a, cudaStream_t stream);
+size_t bwd_workspace_bytes(int B, int N, int units, int dv);
+cudaError_t launch_backward(BwdArgs g, void* workspace, cudaStream_t stream);
+cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* lq2,
+                              const float* lk2, int n_heads, int dim, const float* dlam,
+                              float* dlq1, float* dlk1, float* dlq2, float* dlk2,
+                              cudaStream_t stream);
 
 }  // namespace diffattn

@@ -180,6 +180,48 @@ int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t*
                                 void* stream);
 
 /*
+ * diffattn_bwd_prefill -- gradients of diffattn_fwd_prefill (training). The pages present
+ * lambda and the projections as learnable in a pre-trained layer ("Differential Attention
+ * (V2)", Key Terms, "lambda"; "V1 vs V2"); the gradient is fixed by the forward:
+ *   dV = (A_1 - lambda A_2)^T dO,  dS_1 = A_1 o (dO V^T - delta_1),
+ *   dS_2 = -lambda A_2 o (dO V^T - delta_2),  dQ_b = dS_b K_b / sqrt(d),
+ *   dK_b = dS_b^T Q_b / sqrt(d),  dlambda = -sum dO o (A_2 V),
+ * with dO the gradient reaching O = A_1 V - lambda A_2 V (V1: through the per-head RMSNorm
+ * and the (1 - lambda_init) scale) and delta_b = rowsum(dO o (A_b V)). The softmax maps are
+ * recomputed, never stored. V2's two branches and the pairs of a GQA group add into the
+ * gradient of their shared KV head.
+ *
+ * p, q, k, v, lambda, lambda_init : exactly as for the forward call (f32 or bf16 inputs,
+ *              kv_seqlen and window as there); head_dim <= 128, a multiple of 4
+ * dout       : dL/dy in the layout and dtype of the forward's out (p->o_strides)
+ * dq, dk, dv : float32, DENSE row-major in the shapes of q, k and v (V1 [B,N,H,2,d],
+ *              [B,Nk,H,2,d], [B,Nk,H,2d]; V2 [B,N,Hq,d], [B,Nk,Hkv,d], [B,Nk,Hkv,d]),
+ *              16-byte aligned; fully overwritten
+ * dlambda    : float32 [units] (V1 heads / V2 pairs), overwritten; feed it to
+ *              diffattn_lambda_bwd for the four lambda vectors
+ * workspace  : >= diffattn_bwd_workspace_size(p) bytes, 256-byte aligned (per row: dO in
+ *              fp32, two log-sum-exps, two deltas, the row's dlambda share)
+ * Arithmetic: fp32 on the CUDA cores for every dtype; deterministic (no atomics: dQ rows,
+ * dK/dV rows and dlambda are each summed by one thread group in a fixed order).
+ * Errors as for diffattn_fwd_prefill, plus DIFFATTN_ERR_WORKSPACE.
+ */
+int diffattn_bwd_workspace_size(const diffattn_prefill_params* p, size_t* bytes);
+int diffattn_bwd_prefill(const diffattn_prefill_params* p, const void* q, const void* k,
+                         const void* v, const float* lambda, const float* lambda_init,
+                         const void* dout, float* dq, float* dk, float* dv, float* dlambda,
+                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+
+/*
+ * diffattn_lambda_bwd -- gradients of the four lambda vectors from dL/dlambda:
+ *   dlq1 = g e1 lk1, dlk1 = g e1 lq1, dlq2 = -g e2 lk2, dlk2 = -g e2 lq2,
+ *   e_b = exp(lq_b . lk_b), g = dlambda[h]   (lambda_init depends on depth only).
+ * Vectors float32 [n_heads, dim] as for diffattn_lambda (device); outputs overwritten.
+ */
+int diffattn_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
+                        int n_heads, int dim, const float* dlambda, float* dlq1, float* dlk1,
+                        float* dlq2, float* dlk2, void* stream);
+
+/*
  * Decode parameters (bf16 only). V2 (diffattn_fwd_decode) below; V1 uses the same struct
  * with the layouts given at diffattn_fwd_decode_v1.
  *   q       : [B, Hq, d]        one new query token per batch entry

@@ -268,3 +268,25 @@ def test_prefill_varlen_rejects(lib):
     assert f(ctypes.byref(p), cu_q, cu_k, 128, *args, None, None) == -1      # window needs causal
     p.window, p.causal = 0, 1
     assert f(ctypes.byref(p), cu_q, cu_k, 0, *args, None, None) == 0         # nothing to launch
+
+
+def test_backward_workspace_and_rejects(lib):
+    vp = ctypes.c_void_p
+    p = _prefill_params()  # V2, B=1, N=256, Hq=16, Hkv=2, d=128
+    n = ctypes.c_size_t(0)
+    assert lib.diffattn_bwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
+    rows = 1 * 256 * 8
+    up = lambda x: (x + 255) // 256 * 256
+    assert n.value == up(rows * 128 * 4) + up(rows * 16) + up(rows * 4)
+    big = _prefill_params(head_dim=256)
+    assert lib.diffattn_bwd_workspace_size(ctypes.byref(big), ctypes.byref(n)) == -2
+    f = lib.diffattn_bwd_prefill
+    ptr = [vp(GOOD), vp(GOOD + 4096), vp(GOOD + 8192), vp(GOOD + 12288), None, vp(GOOD + 16384)]
+    outs = [vp(GOOD + 20480), vp(GOOD + 24576), vp(GOOD + 28672), vp(GOOD + 32768)]
+    need = up(rows * 128 * 4) + up(rows * 16) + up(rows * 4)
+    assert f(ctypes.byref(p), *ptr, *outs, vp(GOOD * 4), need - 1, None, None) == -4
+    assert f(ctypes.byref(p), *ptr, *outs, None, need, None, None) == -4
+    assert f(ctypes.byref(p), *ptr, vp(GOOD + 20484), *outs[1:], vp(GOOD * 4), need, None, None) == -3
+    assert f(ctypes.byref(p), *ptr, None, *outs[1:], vp(GOOD * 4), need, None, None) == -1
+    assert lib.diffattn_lambda_bwd(None, vp(GOOD), vp(GOOD), vp(GOOD), 4, 64, vp(GOOD),
+                                   vp(GOOD), vp(GOOD), vp(GOOD), vp(GOOD), None) == -1

@@ -1,0 +1,113 @@
+"""GPU parity of the backward pass (diffattn_bwd_prefill, diffattn_lambda_bwd) against the
+float64 backward oracle (itself pinned to finite differences of the forward oracle and to
+torch autograd).
+
+Tolerance: the kernels compute in fp32 from the same input values the oracle reads (bf16
+inputs are widened exactly), so the only error is fp32 rounding of sums over at most a few
+thousand terms and of expf/logf: max abs error <= 2e-5 x max|reference| + 1e-6 per tensor."""
+import numpy as np
+import pytest
+import torch
+
+import differential_attention_05_b200 as da
+import oracle
+from oracle import backward as OB
+from differential_attention_05_b200 import synth
+
+from gpu_helpers import dev_tensor, lambda_on_device
+
+pytestmark = pytest.mark.gpu
+
+REL = 2e-5
+ABS = 1e-6
+
+
+def _check(got, ref, what):
+    got = got.detach().float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite"
+    err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
+    bound = REL * float(np.max(np.abs(ref))) + ABS
+    assert err <= bound, f"{what}: max abs err {err:.3e} > {bound:.3e}"
+
+
+def _case(variant, Nq, Nk, dtype, seed, causal=True, window=0, norm=True, Hq=8, Hkv=2, H=2):
+    if variant == 1:
+        inp = synth.v1_small(B=2, N=Nk, H=H, seed=seed, dtype=dtype, causal=causal, apply_norm=norm)
+    else:
+        inp = synth.v2_small(B=2, N=Nk, Hq=Hq, Hkv=Hkv, seed=seed, dtype=dtype, causal=causal)
+    q = dev_tensor(inp.q)[:, Nk - Nq:].contiguous()
+    k, v = dev_tensor(inp.k), dev_tensor(inp.v)
+    lam, li = lambda_on_device(inp)
+    oshape = (2, Nq, H, 2 * inp.d) if variant == 1 else (2, Nq, Hq // 2, inp.d)
+    g = torch.Generator().manual_seed(seed)
+    dy = torch.randn(oshape, generator=g).to(q.dtype).cuda()
+    dq, dk, dv, dl = da.diffattn_bwd_prefill(q, k, v, lam, dy, li, causal=causal,
+                                             apply_norm=inp.apply_norm, norm_eps=inp.eps,
+                                             window=window)
+    torch.cuda.synchronize()
+    lam64 = oracle.lambda_(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.depth)
+    q64 = inp.as_f64("q")[:, Nk - Nq:]
+    k64, v64 = inp.as_f64("k"), inp.as_f64("v")
+    dy64 = dy.float().cpu().numpy().astype(np.float64)
+    if variant == 1:
+        ref = OB.prefill_v1_bwd(q64, k64, v64, lam64, oracle.lambda_init(inp.depth), dy64,
+                                causal=causal, apply_norm=inp.apply_norm, eps=inp.eps, window=window)
+    else:
+        ref = OB.prefill_v2_bwd(q64, k64, v64, lam64, dy64, causal=causal, window=window)
+    tag = f"V{variant} {dtype} Nq={Nq} Nk={Nk} causal={causal} window={window}"
+    for name, t, r in zip(("dq", "dk", "dv", "dlambda"), (dq, dk, dv, dl), ref):
+        _check(t, r, f"{tag} {name}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("variant", [1, 2])
+def test_backward_causal(variant, dtype):
+    _case(variant, 150, 150, dtype, seed=700 + variant)
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+def test_backward_full_chunk_window(variant):
+    _case(variant, 97, 97, "bf16", seed=710 + variant, causal=False)
+    _case(variant, 60, 201, "bf16", seed=720 + variant)
+    _case(variant, 130, 130, "bf16", seed=730 + variant, window=33)
+    _case(variant, 41, 170, "f32", seed=740 + variant, window=50)
+
+
+def test_backward_v1_without_norm():
+    _case(1, 120, 120, "bf16", seed=750, norm=False)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (8, 1), (16, 2)])
+def test_backward_v2_group_sizes(Hq, Hkv):
+    """dK and dV of a KV head sum both branches of every pair in its GQA group."""
+    _case(2, 80, 80, "bf16", seed=760 + Hq, Hq=Hq, Hkv=Hkv)
+
+
+def test_backward_v2_medium():
+    """2048 tokens, 16 query heads over 2 KV heads, d = 128: several hundred keys per
+    row, so rounding of long sums is exercised."""
+    _case(2, 2048, 2048, "bf16", seed=770, Hq=16, Hkv=2)
+
+
+def test_lambda_bwd():
+    inp = synth.v2_small(B=1, N=4, Hq=64, Hkv=8, seed=780)
+    vecs = [dev_tensor(getattr(inp, n)) for n in ("lq1", "lk1", "lq2", "lk2")]
+    dl = torch.randn(32, generator=torch.Generator().manual_seed(1)).cuda()
+    got = da.diffattn_lambda_bwd(*vecs, dl)
+    torch.cuda.synchronize()
+    ref = OB.lambda_bwd(inp.lq1, inp.lk1, inp.lq2, inp.lk2, dl.cpu().numpy())
+    for name, t, r in zip(("dlq1", "dlk1", "dlq2", "dlk2"), got, ref):
+        _check(t, r, name)
+
+
+def test_backward_deterministic():
+    """No atomics: two calls give identical bits."""
+    inp = synth.v2_small(B=1, N=300, Hq=16, Hkv=2, seed=790)
+    q, k, v = (dev_tensor(getattr(inp, n)) for n in ("q", "k", "v"))
+    lam, _ = lambda_on_device(inp)
+    dy = torch.randn((1, 300, 8, 128), generator=torch.Generator().manual_seed(2)).bfloat16().cuda()
+    a = da.diffattn_bwd_prefill(q, k, v, lam, dy)
+    b = da.diffattn_bwd_prefill(q, k, v, lam, dy)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
