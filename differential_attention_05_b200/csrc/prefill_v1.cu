@@ -68,6 +68,7 @@ constexpr int MISC_BYTES = 12288;
 constexpr int SMEM_BYTES = MISC_OFF + MISC_BYTES + 1024;
 constexpr int NUM_THREADS = 384;
 constexpr int REGS_SOFTMAX = 208, REGS_OTHER = 88;
+constexpr int POLY_PAIRS = 0;  // of every 4 pairs of exponentials, on the FMA pipe
 constexpr int TMEM_COLS = 512;
 constexpr uint32_t COL_D = 256, COL_O2 = 384;
 constexpr float RESCALE_LOG2 = 8.0f;
@@ -309,20 +310,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float n = r ? fmaxf(t, m) : m;
       const float al = (r && had) ? ex2(m - n) : 1.f;
       m = n;
-      // p = 2^(s sl2 - m), in place (0 for every key while the row has none visible)
+      // p = 2^(s sl2 - m), in place (0 for every key while the row has none visible); in
+      // every group of 8 keys the last POLY_PAIRS pairs go to the FMA pipe, the rest to MUFU
       float sa = 0.f, sb2 = 0.f, sc2 = 0.f, sd = 0.f;
       const float nm = (WINDOW && m == -INFINITY) ? 0.f : -m;
 #pragma unroll
-      for (int e = 0; e < BN; e += 4) {
-        float x0, x1, x2, x3;
-        ffma2(x0, x1, p[e], p[e + 1], sl2, sl2, nm, nm);
-        ffma2(x2, x3, p[e + 2], p[e + 3], sl2, sl2, nm, nm);
-        p[e] = ex2(x0);
-        p[e + 1] = ex2(x1);
-        p[e + 2] = ex2(x2);
-        p[e + 3] = ex2(x3);
+      for (int e = 0; e < BN; e += 8) {
+        float xv[8];
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) ffma2(xv[i], xv[i + 1], p[e + i], p[e + i + 1], sl2, sl2, nm, nm);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+          if (i >= 8 - 2 * POLY_PAIRS) {
+            exp2_fma2(p[e + i], p[e + i + 1], xv[i], xv[i + 1]);
+          } else {
+            p[e + i] = ex2(xv[i]);
+            p[e + i + 1] = ex2(xv[i + 1]);
+          }
+        }
         fadd2(sa, sb2, sa, sb2, p[e], p[e + 1]);
         fadd2(sc2, sd, sc2, sd, p[e + 2], p[e + 3]);
+        fadd2(sa, sb2, sa, sb2, p[e + 4], p[e + 5]);
+        fadd2(sc2, sd, sc2, sd, p[e + 6], p[e + 7]);
       }
       l = l * al + ((sa + sb2) + (sc2 + sd));
 
