@@ -425,27 +425,24 @@ def secondary(device, peaks, torch, da):
     res["v2_prefill"] = {"workload": "v2_bf16_prefill_b1_n16384_hq64_hkv8_d128", "ms": round(ms, 4),
                          "TFLOP/s": round(fl / ms / 1e9, 2),
                          "frac_of_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
-    # the backward pass on the first 4096 tokens of the same tensors (fp32 SIMT kernels);
-    # algorithmic FLOPs per attended (query head, key) pair: 8 d (recomputed scores 2d, dP d
-    # per head, dQ 2d, dK 2d, dV d per head), against the FP32 FMA rate of the 148 SMs
+    # the backward pass on the first 4096 tokens of the same tensors (tensor-core kernels:
+    # statistics pass, dK/dV, dQ, dlambda sum); algorithmic FLOPs per attended (query head,
+    # key) pair: 8 d (scores 2d, dP d per head, dQ 2d, dK 2d, dV d per head)
     Nb = 4096
     qb, kb, vb = q[:, :Nb].contiguous(), k[:, :Nb].contiguous(), v[:, :Nb].contiguous()
     dyb = torch.randn((1, Nb, Hq // 2, d), generator=g, device=device).bfloat16()
-    for _ in range(2):
+    for _ in range(3):
         da.diffattn_bwd_prefill(qb, kb, vb, lam, dyb)
-    eb = es[:5]
-    for a, b in eb:
+    for a, b in es:
         a.record()
         da.diffattn_bwd_prefill(qb, kb, vb, lam, dyb)
         b.record()
     torch.cuda.synchronize(device)
-    ms = statistics.median(a.elapsed_time(b) for a, b in eb)
+    ms = statistics.median(a.elapsed_time(b) for a, b in es)
     fl = 8.0 * d * Hq * visible_pairs(Nb, Nb)
-    fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
     res["v2_backward_n4096"] = {"workload": "v2_bf16_prefill_b1_n4096_hq64_hkv8_d128 backward",
-                                "ms": round(ms, 3), "TFLOP/s": round(fl / ms / 1e9, 2),
-                                "frac_of_fp32_fma_peak": round(fl / ms / 1e9 / fp32_peak, 4),
-                                "fp32_fma_peak_tflops": round(fp32_peak, 1)}
+                                "ms": round(ms, 4), "TFLOP/s": round(fl / ms / 1e9, 2),
+                                "frac_of_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
     del qb, kb, vb, dyb
     # the same tensors as a sliding-window layer (4096 keys) and as a 2048-query chunk at
     # the end of the 16384-key context; FLOPs count the attended pairs only

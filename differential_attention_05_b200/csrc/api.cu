@@ -193,6 +193,12 @@ int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t*
                      out, dev_status, stream);
 }
 
+// the tensor-core backward covers V2 in bf16 with d = 128; everything else runs on the
+// exact-fp32 SIMT kernels
+static bool bwd_tensor_core(const diffattn_prefill_params* p) {
+  return p->variant == DIFFATTN_V2 && p->dtype == DIFFATTN_BF16 && p->head_dim == 128;
+}
+
 // backward: any d <= 128 with d % 4 == 0, f32 or bf16 inputs, fixed-length batches
 static int bwd_check(const diffattn_prefill_params* p) {
   if (!p) return DIFFATTN_ERR_INVALID_ARG;
@@ -219,7 +225,8 @@ int diffattn_bwd_workspace_size(const diffattn_prefill_params* p, size_t* bytes)
   } else {
     return DIFFATTN_ERR_INVALID_ARG;
   }
-  *bytes = bwd_workspace_bytes(p->batch, p->seqlen, units, dv);
+  *bytes = bwd_tensor_core(p) ? bwd_v2_tc_workspace_bytes(p->batch, p->seqlen, units)
+                              : bwd_workspace_bytes(p->batch, p->seqlen, units, dv);
   return DIFFATTN_OK;
 }
 
@@ -238,7 +245,9 @@ int diffattn_bwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   if (!dout || !dq || !dk || !dv || !dlambda) return DIFFATTN_ERR_INVALID_ARG;
   if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return DIFFATTN_ERR_MISALIGNED;
   const PrefillArgs& a = g.f;
-  const size_t need = bwd_workspace_bytes(a.B, a.N, a.units, a.dv);
+  const bool tc = bwd_tensor_core(p);
+  const size_t need = tc ? bwd_v2_tc_workspace_bytes(a.B, a.N, a.units)
+                         : bwd_workspace_bytes(a.B, a.N, a.units, a.dv);
   if (!workspace || workspace_bytes < need) return DIFFATTN_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIFFATTN_ERR_MISALIGNED;
   g.bf16 = p->dtype == DIFFATTN_BF16;
@@ -248,7 +257,8 @@ int diffattn_bwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   g.dk = dk;
   g.dv = dv;
   g.dlambda = dlambda;
-  return from_cuda(launch_backward(g, workspace, static_cast<cudaStream_t>(stream)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return from_cuda(tc ? launch_backward_v2_tc(g, workspace, s) : launch_backward(g, workspace, s));
 }
 
 int diffattn_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2,

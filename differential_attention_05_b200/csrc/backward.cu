@@ -414,7 +414,11 @@ cudaError_t launch_backward(BwdArgs g, void* workspace, cudaStream_t stream) {
     bwd_rows_kernel<float><<<grid_rows, kWarps * 32, 0, stream>>>(g);
     bwd_keys_kernel<float><<<grid_keys, kWarps * 32, 0, stream>>>(g);
   }
-  bwd_dlambda_kernel<<<a.units, 256, 0, stream>>>(g);
+  return launch_dlambda_reduce(g, stream);
+}
+
+cudaError_t launch_dlambda_reduce(const BwdArgs& g, cudaStream_t stream) {
+  bwd_dlambda_kernel<<<g.f.units, 256, 0, stream>>>(g);
   return cudaGetLastError();
 }
 

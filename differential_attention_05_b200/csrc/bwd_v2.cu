@@ -1,0 +1,607 @@
+// bwd_v2.cu -- backward of the V2 prefill (bf16, d = 128) on the sm_100a tensor cores.
+//
+// The gradient is the forward's calculus (backward.cu states it). Notation per pair u
+// (query heads 2u, 2u+1 over KV head g), scores S_b = Q_b K^T (raw), P_b = 2^(S_b sl2 -
+// lse_b) with sl2 = log2(e)/sqrt(d) and lse_b the row's log2-domain log-sum-exp:
+//   dP = dO V^T (the same for both branches),  dS_1 = P_1 o (dP - delta_1),
+//   dS_2 = -lambda P_2 o (dP - delta_2),       delta_b = rowsum(dO o (P_b V)),
+//   dV  = sum_u (P_1 - lambda P_2)^T dO,       dK = sum_u (dS_1^T Q_1 + dS_2^T Q_2) / sqrt(d),
+//   dQ_b = dS_b K / sqrt(d).
+// Three launches besides the fixed-order dlambda sum:
+//   1. the forward kernel in its statistics mode (prefill_v2.cu) writes lse_1, lse_2,
+//      delta_1, delta_2 and the dlambda share of every (query, pair);
+//   2. bwd_v2_dkdv_kernel: one CTA per (128-key tile, KV head, batch entry) walks the pairs
+//      of the GQA group and the 64-query tiles that see its keys. Per step the tensor core
+//      computes S^T = K [Q_1; Q_2]^T (both branches stacked, N = 128) and dP^T = V dO^T;
+//      one warpgroup (thread = key = TMEM lane) forms (P_1 - lambda P_2)^T and
+//      [dS_1^T | dS_2^T] in bf16 straight into TMEM, and the tensor core accumulates
+//      dV += (P_1 - lambda P_2)^T dO and dK += [dS_1^T | dS_2^T] [Q_1; Q_2] in TMEM (A from
+//      TMEM, B = the same shared tiles read MN-major);
+//   3. bwd_v2_dq_kernel: one CTA per (64-query tile, pair, batch entry) walks the 128-key
+//      tiles its queries see: S = [Q_1; Q_2] K^T and dP = [dO; dO] V^T (branches stacked in
+//      the M = 128 rows), dS_b in bf16 into TMEM, dQ += dS K.
+// No atomics: every dK/dV row and every dQ row is summed inside one CTA in a fixed order.
+// Warps 0-3 form the per-row arithmetic, warp 4 issues the TMA loads (128-byte swizzle, no
+// multicast) and the 1-D bulk copy of the statistics, warp 5 owns TMEM and every MMA.
+// Every mbarrier wait is bounded as in the forward kernels.
+#include "common.cuh"
+#include "kernels.h"
+#include "tma_host.cuh"
+
+namespace diffattn {
+
+namespace {
+constexpr int BLK = 128 * 128;   // [128 rows x 64 bf16] 128-byte-swizzled block (16 KB)
+constexpr int HBLK = 64 * 128;   // [64 rows x 64 bf16] (8 KB)
+constexpr unsigned FULL = 0xffffffffu;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 512;
+
+struct BwdMaps {
+  CUtensorMap q, k, v, dy;
+};
+
+__device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
+// does query i (at position i + Nk - N) attend key j
+__device__ __forceinline__ bool visible(const PrefillArgs& a, int i, int j) {
+  if (i >= a.N || j >= a.Nk) return false;
+  if (!a.causal) return true;
+  const int pos = i + a.Nk - a.N;
+  return j <= pos && (a.window <= 0 || j > pos - a.window);
+}
+
+// ----------------------------------------------------------------------------- dK, dV
+namespace kv {
+constexpr int KT = 128, QT = 64, STAGES = 2;
+constexpr int K_OFF = 0, V_OFF = 2 * BLK;
+constexpr int STAGE_OFF = 4 * BLK;
+constexpr int QS = 0, DO = 2 * BLK, STS = 2 * BLK + 2 * HBLK;  // inside a stage
+constexpr int STAGE_BYTES = 2 * BLK + 2 * HBLK + 1024;         // 49 KB
+constexpr int MISC_OFF = STAGE_OFF + STAGES * STAGE_BYTES;
+constexpr int SMEM_BYTES = MISC_OFF + 1024 + 1024;
+// TMEM columns: S^T (both branches), dP^T (then P_1 - lambda P_2 in bf16 over its first
+// half), [dS_1^T | dS_2^T] in bf16, dV, dK
+constexpr int C_S = 0, C_DP = 128, C_PC = 128, C_DS = 192, C_DV = 256, C_DK = 384;
+struct Misc {
+  uint64_t kv_full, q_full[STAGES], q_empty[STAGES], s_full, p_full, o_full;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(STAGE_BYTES % 1024 == 0 && sizeof(Misc) <= 1024, "layout");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+}  // namespace kv
+}  // namespace
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_v2_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdArgs g) {
+  using namespace kv;
+  const PrefillArgs& a = g.f;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Misc& ms = *reinterpret_cast<Misc*>(smem + MISC_OFF);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per_kt = a.Hkv * a.B;
+  const int kt = (int)(blockIdx.x / per_kt);  // causal: key tile 0 sees the most queries
+  const int gk = (int)(blockIdx.x % per_kt) % a.Hkv;
+  const int b = (int)(blockIdx.x % per_kt) / a.Hkv;
+  const int k0 = kt * KT;
+  const int off = a.Nk - a.N;
+  // queries that see a key of this tile, in 64-query tiles, for every pair of the group
+  int i_lo = 0, i_hi = a.N - 1;
+  if (a.causal) {
+    i_lo = max(0, k0 - off);
+    if (a.window > 0) i_hi = min(a.N - 1, k0 + KT - 1 - off + a.window - 1);
+  }
+  const int qt_lo = i_lo / QT;
+  const int n_qt = i_hi >= i_lo ? i_hi / QT - qt_lo + 1 : 0;
+  const int pairs = a.group / 2, u0 = gk * pairs;
+  const int n_steps = n_qt * pairs;  // step t: pair u0 + t / n_qt, query tile qt_lo + t % n_qt
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ms.kv_full, 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ms.q_full[s], 1);
+      mbar_init(&ms.q_empty[s], 1);
+    }
+    mbar_init(&ms.s_full, 1);
+    mbar_init(&ms.p_full, 128);
+    mbar_init(&ms.o_full, 1);
+    ms.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&ms.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms.tmem_base;
+  volatile int* abort_flag = &ms.abort;
+  const int rows = a.N + 64;  // statistics rows per (batch entry, pair)
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ------------------------------ TMA producer -----------------------------------
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.k);
+      tma_prefetch_desc(&maps.v);
+      tma_prefetch_desc(&maps.dy);
+      mbar_arrive_expect_tx(&ms.kv_full, 4 * BLK);
+      for (int hf = 0; hf < 2; ++hf) {
+        tma_load_4d(smem + K_OFF + hf * BLK, &maps.k, &ms.kv_full, 64 * hf, gk, k0, b);
+        tma_load_4d(smem + V_OFF + hf * BLK, &maps.v, &ms.kv_full, 64 * hf, gk, k0, b);
+      }
+      int issued = 0;
+      for (int t = 0; t < n_steps && !*abort_flag; ++t) {
+        const int s = t % STAGES;
+        if (!mbar_wait(&ms.q_empty[s], ((t / STAGES) & 1) ^ 1, abort_flag)) break;
+        const int u = u0 + t / n_qt, q0 = (qt_lo + t % n_qt) * QT;
+        uint8_t* st = smem + STAGE_OFF + s * STAGE_BYTES;
+        mbar_arrive_expect_tx(&ms.q_full[s], 2 * BLK + 2 * HBLK + 1024);
+        for (int hf = 0; hf < 2; ++hf) {
+          // [Q_1; Q_2]: rows 0-63 branch 1, rows 64-127 branch 2 of each 64-column block
+          tma_load_4d(st + QS + hf * BLK, &maps.q, &ms.q_full[s], 64 * hf, 2 * u, q0, b);
+          tma_load_4d(st + QS + hf * BLK + 64 * 128, &maps.q, &ms.q_full[s], 64 * hf, 2 * u + 1, q0, b);
+          tma_load_4d(st + DO + hf * HBLK, &maps.dy, &ms.q_full[s], 64 * hf, u, q0, b);
+        }
+        bulk_load(st + STS, g.w_st + (((int64_t)b * a.units + u) * rows + q0) * 4, 1024, &ms.q_full[s]);
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        // let the copies in flight land before the CTA's shared memory goes away
+        mbar_wait_drain(&ms.kv_full, 0);
+        for (int t = max(0, issued - STAGES); t < issued; ++t)
+          mbar_wait_drain(&ms.q_full[t % STAGES], (t / STAGES) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ------------------------------ MMA issuer -------------------------------------
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t IDESC_DP = idesc_bf16_f32(128, 64, false, false);
+      constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, false, true);
+      const uint64_t kdesc = sw128_desc(smem_u32(smem + K_OFF), 16, 1024);
+      const uint64_t vdesc = sw128_desc(smem_u32(smem + V_OFF), 16, 1024);
+      auto issue_s_dp = [&](int t) {
+        const uint32_t st = smem_u32(smem + STAGE_OFF + (t % STAGES) * STAGE_BYTES);
+        const uint64_t qd = sw128_desc(st + QS, 16, 1024);
+        const uint64_t dd = sw128_desc(st + DO, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t o = (kk >> 2) * BLK + (kk & 3) * 32;
+          umma_ss(tmem + C_S, desc_at(kdesc, o), desc_at(qd, o), IDESC_S, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t o = (kk >> 2) * BLK + (kk & 3) * 32;
+          const uint32_t od = (kk >> 2) * HBLK + (kk & 3) * 32;
+          umma_ss(tmem + C_DP, desc_at(vdesc, o), desc_at(dd, od), IDESC_DP, kk > 0);
+        }
+        tc_commit(&ms.s_full);
+      };
+      auto issue_dv_dk = [&](int t) {
+        const uint32_t st = smem_u32(smem + STAGE_OFF + (t % STAGES) * STAGE_BYTES);
+        // the same tiles read MN-major: K index = query (16 rows = 2048 B per step)
+        const uint64_t dmn = sw128_desc(st + DO, HBLK, 1024);
+        const uint64_t qmn = sw128_desc(st + QS, BLK, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ts(tmem + C_DV, tmem + C_PC + kk * 8, desc_at(dmn, kk * 2048), IDESC_ACC,
+                  (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + C_DK, tmem + C_DS + kk * 8, desc_at(qmn, kk * 2048), IDESC_ACC,
+                  (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&ms.q_empty[t % STAGES]);
+      };
+      bool ok = mbar_wait(&ms.kv_full, 0, abort_flag);
+      if (ok && n_steps > 0) {
+        ok = mbar_wait(&ms.q_full[0], 0, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_s_dp(0);
+        }
+      }
+      for (int t = 0; t < n_steps && ok; ++t) {
+        if (!(ok = mbar_wait(&ms.p_full, t & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_dv_dk(t);
+        if (t + 1 < n_steps) {
+          if (!(ok = mbar_wait(&ms.q_full[(t + 1) % STAGES], ((t + 1) / STAGES) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_s_dp(t + 1);
+        }
+      }
+      // arrives once every MMA issued above has completed (also on an abort)
+      tc_commit(&ms.o_full);
+    }
+  } else {
+    // ------------------------- per-key arithmetic (warps 0-3) -------------------------
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int j = k0 + (int)threadIdx.x;  // this thread's key (TMEM lane)
+    const float sl2 = 1.4426950408889634f * rsqrtf((float)a.d);
+    bool ok = true;
+    for (int t = 0; t < n_steps; ++t) {
+      const int s = t % STAGES;
+      const int u = u0 + t / n_qt, q0 = (qt_lo + t % n_qt) * QT;
+      const float lam = a.lambda[u];
+      if (ok) ok = mbar_wait(&ms.q_full[s], (t / STAGES) & 1, abort_flag);
+      if (ok) ok = mbar_wait(&ms.s_full, t & 1, abort_flag);
+      if (!(ok = __all_sync(FULL, ok))) break;
+      tc_fence_after();
+      const float4* sts = reinterpret_cast<const float4*>(smem + STAGE_OFF + s * STAGE_BYTES + STS);
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        float s1[32], s2[32], dp[32];
+        tmem_ld32f(lane_addr + C_S + 32 * c, s1);
+        tmem_ld32f(lane_addr + C_S + 64 + 32 * c, s2);
+        tmem_ld32f(lane_addr + C_DP + 32 * c, dp);
+        tmem_wait_ld();
+        uint32_t pc[16], d1[16], d2[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float vpc[2], vd1[2], vd2[2];
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            const int qq = 32 * c + e + x;
+            const float4 st = sts[qq];
+            const bool vis = visible(a, q0 + qq, j);
+            const float p1 = vis ? ex2(s1[e + x] * sl2 - st.x) : 0.f;
+            const float p2 = vis ? ex2(s2[e + x] * sl2 - st.y) : 0.f;
+            vpc[x] = p1 - lam * p2;
+            vd1[x] = vis ? p1 * (dp[e + x] - st.z) : 0.f;
+            vd2[x] = vis ? -lam * p2 * (dp[e + x] - st.w) : 0.f;
+          }
+          pc[e / 2] = pack_bf16(vpc[0], vpc[1]);
+          d1[e / 2] = pack_bf16(vd1[0], vd1[1]);
+          d2[e / 2] = pack_bf16(vd2[0], vd2[1]);
+        }
+        // chunk c's bf16 columns lie below the dP columns still to be read
+        tmem_st16(lane_addr + C_PC + 16 * c, pc);
+        tmem_st16(lane_addr + C_DS + 16 * c, d1);
+        tmem_st16(lane_addr + C_DS + 32 + 16 * c, d2);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&ms.p_full);
+    }
+    // ------------------------------- epilogue ----------------------------------------
+    if (ok) ok = mbar_wait(&ms.o_full, 0, abort_flag);
+    ok = __all_sync(FULL, ok);
+    // the TMEM loads run on the whole warp (they are warp-collective); only the stores
+    // depend on the key being inside the sequence
+    if (ok) {
+      const float scale = rsqrtf((float)a.d);
+      const bool store = j < a.Nk;
+      const int64_t row = ((int64_t)b * a.Nk + (store ? j : 0)) * a.Hkv + gk;
+      float4* dv4 = reinterpret_cast<float4*>(g.dv + row * 128);
+      float4* dk4 = reinterpret_cast<float4*>(g.dk + row * 128);
+      if (n_steps > 0) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float x[32], y[32];
+          tmem_ld32f(lane_addr + C_DV + 32 * c, x);
+          tmem_ld32f(lane_addr + C_DK + 32 * c, y);
+          tmem_wait_ld();
+          if (store) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              dv4[(32 * c + e) / 4] = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+              dk4[(32 * c + e) / 4] = make_float4(y[e] * scale, y[e + 1] * scale,
+                                                  y[e + 2] * scale, y[e + 3] * scale);
+            }
+          }
+        }
+      } else if (store) {
+        for (int e = 0; e < 32; ++e) dv4[e] = dk4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    if (*abort_flag) {
+      mbar_wait_drain(&ms.o_full, 0);
+      if (lane == 0) report_status(a.dev_status, DIFFATTN_ERR_TIMEOUT);
+    }
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------------------------- dQ
+namespace {
+namespace dqk {
+constexpr int QT = 64, KT = 128, STAGES = 2;
+constexpr int QS_OFF = 0;                 // [Q_1; Q_2]: 2 blocks of [128 x 64]
+constexpr int DO_OFF = 2 * BLK;           // [dO; dO]
+constexpr int ST_OFF = 4 * BLK;           // 64 x (lse_1, lse_2, delta_1, delta_2)
+constexpr int KV_OFF = 4 * BLK + 1024;
+constexpr int KV_STAGE = 4 * BLK;         // K (2 blocks), V (2 blocks)
+constexpr int MISC_OFF = KV_OFF + STAGES * KV_STAGE;
+constexpr int SMEM_BYTES = MISC_OFF + 1024 + 1024;
+// TMEM columns: S, dP, dQ, dS (bf16)
+constexpr int C_S = 0, C_DP = 128, C_DQ = 256, C_DS = 384;
+struct Misc {
+  uint64_t q_full, kv_full[STAGES], kv_empty[STAGES], s_full, p_full, o_full;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(KV_OFF % 1024 == 0 && sizeof(Misc) <= 1024, "layout");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+}  // namespace dqk
+}  // namespace
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    bwd_v2_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdArgs g) {
+  using namespace dqk;
+  const PrefillArgs& a = g.f;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  Misc& ms = *reinterpret_cast<Misc*>(smem + MISC_OFF);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_qtiles = (a.N + QT - 1) / QT;
+  const int per_qt = a.units * a.B;
+  // causal: the last query tile sees the most keys, hand it out first
+  const int qt = a.causal ? n_qtiles - 1 - (int)(blockIdx.x / per_qt) : (int)(blockIdx.x / per_qt);
+  const int u = (int)(blockIdx.x % per_qt) % a.units;
+  const int b = (int)(blockIdx.x % per_qt) / a.units;
+  const int q0 = qt * QT;
+  const int gk = (2 * u) / a.group;
+  const int off = a.Nk - a.N;
+  const int khi = a.causal ? min(q0 + QT - 1 + off, a.Nk - 1) : a.Nk - 1;
+  const int klo = (a.causal && a.window > 0) ? max(0, q0 + off - a.window + 1) : 0;
+  const int j_lo = klo / KT;
+  const int n_kt = khi >= klo ? khi / KT - j_lo + 1 : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ms.q_full, 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ms.kv_full[s], 1);
+      mbar_init(&ms.kv_empty[s], 1);
+    }
+    mbar_init(&ms.s_full, 1);
+    mbar_init(&ms.p_full, 128);
+    mbar_init(&ms.o_full, 1);
+    ms.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&ms.tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms.tmem_base;
+  volatile int* abort_flag = &ms.abort;
+  const int rows = a.N + 64;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.k);
+      tma_prefetch_desc(&maps.v);
+      tma_prefetch_desc(&maps.dy);
+      mbar_arrive_expect_tx(&ms.q_full, 4 * BLK + 1024);
+      for (int hf = 0; hf < 2; ++hf) {
+        tma_load_4d(smem + QS_OFF + hf * BLK, &maps.q, &ms.q_full, 64 * hf, 2 * u, q0, b);
+        tma_load_4d(smem + QS_OFF + hf * BLK + 64 * 128, &maps.q, &ms.q_full, 64 * hf, 2 * u + 1, q0, b);
+        // dO in both halves: the branch-2 rows need dP = dO V^T as well
+        tma_load_4d(smem + DO_OFF + hf * BLK, &maps.dy, &ms.q_full, 64 * hf, u, q0, b);
+        tma_load_4d(smem + DO_OFF + hf * BLK + 64 * 128, &maps.dy, &ms.q_full, 64 * hf, u, q0, b);
+      }
+      bulk_load(smem + ST_OFF, g.w_st + (((int64_t)b * a.units + u) * rows + q0) * 4, 1024, &ms.q_full);
+      int issued = 0;
+      for (int t = 0; t < n_kt && !*abort_flag; ++t) {
+        const int s = t % STAGES;
+        if (!mbar_wait(&ms.kv_empty[s], ((t / STAGES) & 1) ^ 1, abort_flag)) break;
+        const int kj = (j_lo + t) * KT;
+        uint8_t* st = smem + KV_OFF + s * KV_STAGE;
+        mbar_arrive_expect_tx(&ms.kv_full[s], 4 * BLK);
+        for (int hf = 0; hf < 2; ++hf) {
+          tma_load_4d(st + hf * BLK, &maps.k, &ms.kv_full[s], 64 * hf, gk, kj, b);
+          tma_load_4d(st + 2 * BLK + hf * BLK, &maps.v, &ms.kv_full[s], 64 * hf, gk, kj, b);
+        }
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait_drain(&ms.q_full, 0);
+        for (int t = max(0, issued - STAGES); t < issued; ++t)
+          mbar_wait_drain(&ms.kv_full[t % STAGES], (t / STAGES) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, false, true);
+      const uint64_t qd = sw128_desc(smem_u32(smem + QS_OFF), 16, 1024);
+      const uint64_t dd = sw128_desc(smem_u32(smem + DO_OFF), 16, 1024);
+      auto issue_s_dp = [&](int t) {
+        const uint32_t st = smem_u32(smem + KV_OFF + (t % STAGES) * KV_STAGE);
+        const uint64_t kd = sw128_desc(st, 16, 1024);
+        const uint64_t vd = sw128_desc(st + 2 * BLK, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t o = (kk >> 2) * BLK + (kk & 3) * 32;
+          umma_ss(tmem + C_S, desc_at(qd, o), desc_at(kd, o), IDESC_SS, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t o = (kk >> 2) * BLK + (kk & 3) * 32;
+          umma_ss(tmem + C_DP, desc_at(dd, o), desc_at(vd, o), IDESC_SS, kk > 0);
+        }
+        tc_commit(&ms.s_full);
+      };
+      auto issue_dq = [&](int t) {
+        const uint32_t st = smem_u32(smem + KV_OFF + (t % STAGES) * KV_STAGE);
+        const uint64_t kmn = sw128_desc(st, BLK, 1024);  // K read MN-major: K index = key
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + C_DQ, tmem + C_DS + kk * 8, desc_at(kmn, kk * 2048), IDESC_ACC,
+                  (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&ms.kv_empty[t % STAGES]);
+      };
+      bool ok = mbar_wait(&ms.q_full, 0, abort_flag);
+      if (ok && n_kt > 0) {
+        ok = mbar_wait(&ms.kv_full[0], 0, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_s_dp(0);
+        }
+      }
+      for (int t = 0; t < n_kt && ok; ++t) {
+        if (!(ok = mbar_wait(&ms.p_full, t & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_dq(t);
+        if (t + 1 < n_kt) {
+          if (!(ok = mbar_wait(&ms.kv_full[(t + 1) % STAGES], ((t + 1) / STAGES) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_s_dp(t + 1);
+        }
+      }
+      tc_commit(&ms.o_full);
+    }
+  } else {
+    // ----------------------- per-(query, branch) arithmetic (warps 0-3) ------------------
+    // row r: branch r / 64 of query q0 + r % 64 (rows 0-63 Q_1, 64-127 Q_2)
+    const int r = (int)threadIdx.x, br = r >> 6;
+    const int qi = q0 + (r & 63);
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const float sl2 = 1.4426950408889634f * rsqrtf((float)a.d);
+    const float lam = a.lambda[u];
+    bool ok = mbar_wait(&ms.q_full, 0, abort_flag);
+    const float4 st = reinterpret_cast<const float4*>(smem + ST_OFF)[r & 63];
+    const float lse = br ? st.y : st.x, del = br ? st.w : st.z, coef = br ? -lam : 1.f;
+    for (int t = 0; t < n_kt; ++t) {
+      if (ok) ok = mbar_wait(&ms.s_full, t & 1, abort_flag);
+      if (!(ok = __all_sync(FULL, ok))) break;
+      tc_fence_after();
+      const int kj0 = (j_lo + t) * KT;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float sv[32], dp[32];
+        tmem_ld32f(lane_addr + C_S + 32 * c, sv);
+        tmem_ld32f(lane_addr + C_DP + 32 * c, dp);
+        tmem_wait_ld();
+        uint32_t ds[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float v2[2];
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            const bool vis = visible(a, qi, kj0 + 32 * c + e + x);
+            const float p = vis ? ex2(sv[e + x] * sl2 - lse) : 0.f;
+            v2[x] = vis ? coef * p * (dp[e + x] - del) : 0.f;
+          }
+          ds[e / 2] = pack_bf16(v2[0], v2[1]);
+        }
+        tmem_st16(lane_addr + C_DS + 16 * c, ds);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&ms.p_full);
+    }
+    if (ok) ok = mbar_wait(&ms.o_full, 0, abort_flag);
+    ok = __all_sync(FULL, ok);
+    // warp-collective TMEM loads; only the stores depend on the query being in range
+    if (ok) {
+      const float scale = rsqrtf((float)a.d);
+      const bool store = qi < a.N;
+      float4* dq4 = reinterpret_cast<float4*>(
+          g.dq + (((int64_t)b * a.N + (store ? qi : 0)) * a.Hq + 2 * u + br) * 128);
+      if (n_kt > 0) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float x[32];
+          tmem_ld32f(lane_addr + C_DQ + 32 * c, x);
+          tmem_wait_ld();
+          if (store) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              dq4[(32 * c + e) / 4] = make_float4(x[e] * scale, x[e + 1] * scale,
+                                                  x[e + 2] * scale, x[e + 3] * scale);
+          }
+        }
+      } else if (store) {
+        for (int e = 0; e < 32; ++e) dq4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    if (*abort_flag) {
+      mbar_wait_drain(&ms.o_full, 0);
+      if (lane == 0) report_status(a.dev_status, DIFFATTN_ERR_TIMEOUT);
+    }
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+size_t bwd_v2_tc_workspace_bytes(int B, int N, int units) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return up((size_t)B * units * (N + 64) * 4 * sizeof(float)) + up((size_t)B * units * N * sizeof(float));
+}
+
+cudaError_t launch_backward_v2_tc(BwdArgs g, void* workspace, cudaStream_t stream) {
+  const PrefillArgs& a = g.f;
+  if (a.variant != DIFFATTN_V2 || a.d != 128 || a.cu_q) return cudaErrorNotSupported;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  g.w_st = reinterpret_cast<float*>(w);
+  g.w_dl = reinterpret_cast<float*>(w + up((size_t)a.B * a.units * (a.N + 64) * 4 * sizeof(float)));
+  g.w_do = nullptr;
+  // 1. statistics: the forward kernel in its statistics mode
+  PrefillArgs fa = a;
+  fa.out = nullptr;
+  fa.st_dy = g.dy;
+  for (int i = 0; i < 3; ++i) fa.st_dys[i] = g.dys[i];
+  fa.st = g.w_st;
+  fa.st_dl = g.w_dl;
+  fa.st_rows = a.N + 64;
+  cudaError_t e = launch_prefill_v2_stats(fa, stream);
+  if (e != cudaSuccess) return e;
+  // 2, 3. dK/dV and dQ
+  BwdMaps maps;
+  if (!make_map(&maps.q, a.q, 128, a.Hq, a.N, a.B, a.qs, 64)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, 128, a.Hkv, a.Nk, a.B, a.ks, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, 128, a.Hkv, a.Nk, a.B, a.vs, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.dy, g.dy, 128, a.units, a.N, a.B, g.dys, 64)) return cudaErrorInvalidValue;
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  if (dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(bwd_v2_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kv::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_v2_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dqk::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_set[dev] = true;
+  }
+  const long long kv_ctas = (long long)((a.Nk + kv::KT - 1) / kv::KT) * a.Hkv * a.B;
+  const long long dq_ctas = (long long)((a.N + dqk::QT - 1) / dqk::QT) * a.units * a.B;
+  if (kv_ctas > 0x7fffffffLL || dq_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  bwd_v2_dkdv_kernel<<<(unsigned)kv_ctas, NUM_THREADS, kv::SMEM_BYTES, stream>>>(maps, g);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_v2_dq_kernel<<<(unsigned)dq_ctas, NUM_THREADS, dqk::SMEM_BYTES, stream>>>(maps, g);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_dlambda_reduce(g, stream);
+}
+
+}  // namespace diffattn

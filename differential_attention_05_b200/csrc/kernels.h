@@ -33,6 +33,15 @@ struct PrefillArgs {
   const int32_t* cu_q;
   const int32_t* cu_k;
   int total_q, total_k;
+  // V2 statistics pass of the backward (launch_prefill_v2_stats): instead of the output,
+  // per (query, pair) the log2-domain log-sum-exps of both branches and
+  // delta_b = dy . (A_b V) go to st[((b * units + u) * st_rows + i) * 4 + 0..3], and the
+  // row's dlambda share -delta_2 to dl[(b * units + u) * N + i]
+  const void* st_dy;
+  int64_t st_dys[3];
+  float* st;
+  float* st_dl;
+  int st_rows;
 };
 
 // Resolved backward problem: the forward's arguments plus the incoming gradient dy (the
@@ -113,6 +122,7 @@ cudaError_t launch_prefill_f32(const PrefillArgs& a, cudaStream_t stream);
 // (prefill_v2.cu); each returns cudaErrorNotSupported for shapes it does not handle.
 cudaError_t launch_prefill_v1(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream);
+cudaError_t launch_prefill_v2_stats(const PrefillArgs& a, cudaStream_t stream);
 
 // split-KV decode (V2, bf16, d = 128, 8 query heads per KV head)
 constexpr int kDecodeChunk = 64;  // keys per pipeline stage
@@ -125,6 +135,9 @@ int decode_v1_default_splits(int B, int L, int H);
 cudaError_t launch_decode_v1(const DecodeArgs& a, cudaStream_t stream);
 size_t bwd_workspace_bytes(int B, int N, int units, int dv);
 cudaError_t launch_backward(BwdArgs g, void* workspace, cudaStream_t stream);
+cudaError_t launch_dlambda_reduce(const BwdArgs& g, cudaStream_t stream);
+size_t bwd_v2_tc_workspace_bytes(int B, int N, int units);
+cudaError_t launch_backward_v2_tc(BwdArgs g, void* workspace, cudaStream_t stream);
 cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* lq2,
                               const float* lk2, int n_heads, int dim, const float* dlam,
                               float* dlq1, float* dlk1, float* dlq2, float* dlk2,

@@ -104,7 +104,9 @@ __device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t bytes) {
 // only an upper end; that case compiles without the lower-end and unset-row checks.
 // VARLEN: a variable-length batch (a.cu_q != nullptr); the fixed-length instantiation
 // takes its sizes from the parameters alone.
-template <bool WINDOW, bool VARLEN>
+// STATS: the statistics pass of the backward (fixed length only): the epilogue writes the
+// log-sum-exps and deltas described at PrefillArgs::st instead of the output.
+template <bool WINDOW, bool VARLEN, bool STATS = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_v2_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -441,9 +443,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const float coef = __fsub_rn(__fmul_rn(c, inv1), __fmul_rn(lam, inv2));
     // this lane writes value columns 64 h .. 64 h + 63 of its query; D and O_2 of a column
     // sit in the two lanes of the query
-    float y[64];
+    float y[64];  // the output, or (STATS) the incoming gradient dy of the same columns
+    float e1 = 0.f, e2 = 0.f;
+    if constexpr (STATS) {
+      if (ok && qi < a.N) {
+        const uint4* g4 = reinterpret_cast<const uint4*>(
+            static_cast<const __nv_bfloat16*>(a.st_dy) + (int64_t)b * a.st_dys[0] +
+            (int64_t)qi * a.st_dys[1] + (int64_t)u * a.st_dys[2] + h * 64);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const uint4 w = g4[v];
+          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            y[v * 8 + 2 * e] = __uint_as_float(wv[e] << 16);
+            y[v * 8 + 2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) y[e] = 0.f;
+      }
+    }
     if (ok) {
       tc_fence_after();
+      const float c1 = c * inv1;
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         float v0[32], v1[32];
@@ -455,15 +479,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const float mine = h ? v1[e] : v0[e];
           const float other = __shfl_xor_sync(FULL, h ? v0[e] : v1[e], 16);
           const float dv = h ? other : mine, ov = h ? mine : other;
-          y[ch * 32 + e] = __fmaf_rn(ov, coef, __fmul_rn(dv, inv1));
+          if constexpr (STATS) {
+            // O_1 / l_1 = (D + c O_2) / l_1 and O_2 / l_2 at this column, against dy
+            e1 = fmaf(y[ch * 32 + e], __fmaf_rn(ov, c1, dv * inv1), e1);
+            e2 = fmaf(y[ch * 32 + e], ov * inv2, e2);
+          } else {
+            y[ch * 32 + e] = __fmaf_rn(ov, coef, __fmul_rn(dv, inv1));
+          }
         }
+      }
+    }
+    if constexpr (STATS) {
+      // the query's two lanes add their column halves; lse_b = m_b + log2 l_b (log2 domain)
+      e1 += __shfl_xor_sync(FULL, e1, 16);
+      e2 += __shfl_xor_sync(FULL, e2, 16);
+      const float lse_own = m + log2f(l);
+      const float lse_oth = __shfl_xor_sync(FULL, lse_own, 16);
+      if (ok && h == 0 && qi < a.N) {
+        const int64_t r = ((int64_t)b * a.units + u) * a.st_rows + qi;
+        *reinterpret_cast<float4*>(a.st + r * 4) = make_float4(lse_own, lse_oth, e1, e2);
+        a.st_dl[((int64_t)b * a.units + u) * a.N + qi] = -e2;
       }
     }
     // (a variable-length tile reads its sequence back from shared memory, keeping the
     // registers of the key loop free)
     const int o_nq = VARLEN ? ms.seq_nq : a.N, o_b = VARLEN ? ms.seq_bc : b;
     const int o_q0 = VARLEN ? ms.seq_q0 : 0;
-    if (ok && qi < o_nq) {
+    if (!STATS && ok && qi < o_nq) {
       __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)o_b * a.os[0] +
                           (int64_t)(o_q0 + qi) * a.os[1] + (int64_t)u * a.os[2] + h * 64;
       uint4* o4 = reinterpret_cast<uint4*>(ob);
@@ -526,6 +568,38 @@ cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream) {
     if (window) prefill_v2_kernel<true, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
     else prefill_v2_kernel<false, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   }
+  return cudaGetLastError();
+}
+
+// The backward's statistics pass over the same tiles (fixed-length batches): st, st_dl and
+// st_dy must be set; out is not written.
+cudaError_t launch_prefill_v2_stats(const PrefillArgs& a, cudaStream_t stream) {
+  if (a.variant != DIFFATTN_V2 || a.d != 128 || a.group % 2 != 0 || a.cu_q) return cudaErrorNotSupported;
+  if (!a.st || !a.st_dl || !a.st_dy) return cudaErrorInvalidValue;
+  TcMaps maps;
+  if (!make_map(&maps.q, a.q, 128, a.Hq, a.N, a.B, a.qs, 16)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, 128, a.Hkv, a.Nk, a.B, a.ks, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, 128, a.Hkv, a.Nk, a.B, a.vs, BN)) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  if (dev >= 64 || !attr_set[dev]) {
+    const void* fns[2] = {(const void*)prefill_v2_kernel<false, false, true>,
+                          (const void*)prefill_v2_kernel<true, false, true>};
+    for (const void* fn : fns) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+    }
+    if (dev < 64) attr_set[dev] = true;
+  }
+  const long long tiles = (long long)((a.N + BM - 1) / BM) * a.units * a.B;
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const dim3 grid((unsigned)tiles);
+  if (a.causal && a.window > 0)
+    prefill_v2_kernel<true, false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  else
+    prefill_v2_kernel<false, false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   return cudaGetLastError();
 }
 

@@ -272,18 +272,22 @@ def test_prefill_varlen_rejects(lib):
 
 def test_backward_workspace_and_rejects(lib):
     vp = ctypes.c_void_p
-    p = _prefill_params()  # V2, B=1, N=256, Hq=16, Hkv=2, d=128
+    p = _prefill_params()  # V2, B=1, N=256, Hq=16, Hkv=2, d=128: tensor-core backward
     n = ctypes.c_size_t(0)
     assert lib.diffattn_bwd_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
     rows = 1 * 256 * 8
     up = lambda x: (x + 255) // 256 * 256
+    # per (entry, pair): N + 64 rows of (lse_1, lse_2, delta_1, delta_2), then N dlambda shares
+    assert n.value == up(8 * (256 + 64) * 16) + up(rows * 4)
+    pf = _prefill_params(dtype=B.DIFFATTN_F32)  # exact-fp32 kernels: dO rows as well
+    assert lib.diffattn_bwd_workspace_size(ctypes.byref(pf), ctypes.byref(n)) == 0
     assert n.value == up(rows * 128 * 4) + up(rows * 16) + up(rows * 4)
     big = _prefill_params(head_dim=256)
     assert lib.diffattn_bwd_workspace_size(ctypes.byref(big), ctypes.byref(n)) == -2
     f = lib.diffattn_bwd_prefill
     ptr = [vp(GOOD), vp(GOOD + 4096), vp(GOOD + 8192), vp(GOOD + 12288), None, vp(GOOD + 16384)]
     outs = [vp(GOOD + 20480), vp(GOOD + 24576), vp(GOOD + 28672), vp(GOOD + 32768)]
-    need = up(rows * 128 * 4) + up(rows * 16) + up(rows * 4)
+    need = up(8 * (256 + 64) * 16) + up(rows * 4)
     assert f(ctypes.byref(p), *ptr, *outs, vp(GOOD * 4), need - 1, None, None) == -4
     assert f(ctypes.byref(p), *ptr, *outs, None, need, None, None) == -4
     assert f(ctypes.byref(p), *ptr, vp(GOOD + 20484), *outs[1:], vp(GOOD * 4), need, None, None) == -3

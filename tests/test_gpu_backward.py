@@ -2,9 +2,14 @@
 float64 backward oracle (itself pinned to finite differences of the forward oracle and to
 torch autograd).
 
-Tolerance: the kernels compute in fp32 from the same input values the oracle reads (bf16
-inputs are widened exactly), so the only error is fp32 rounding of sums over at most a few
-thousand terms and of expf/logf: max abs error <= 2e-5 x max|reference| + 1e-6 per tensor."""
+Tolerances, per tensor:
+  * exact-fp32 kernels (fp32 inputs, V1, any d other than 128): the kernels compute in fp32
+    from the same input values the oracle reads (bf16 inputs are widened exactly), so the
+    only error is fp32 rounding of sums over at most a few thousand terms and of expf/logf:
+    max abs error <= 2e-5 x max|reference| + 1e-6;
+  * tensor-core kernels (V2, bf16, d = 128): the MMA operands P_1 - lambda P_2 and dS_b are
+    rounded to bf16 (relative 2^-9 each, independent across terms), as in the forward:
+    relative RMS error <= 5e-3 and max abs error <= 2e-2 x max|reference|."""
 import numpy as np
 import pytest
 import torch
@@ -22,11 +27,17 @@ REL = 2e-5
 ABS = 1e-6
 
 
-def _check(got, ref, what):
+def _check(got, ref, what, tensor_core=False):
     got = got.detach().float().cpu().numpy().astype(np.float64)
     assert np.all(np.isfinite(got)), f"{what}: non-finite"
     err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
-    bound = REL * float(np.max(np.abs(ref))) + ABS
+    scale = float(np.max(np.abs(ref))) if ref.size else 0.0
+    if tensor_core:
+        rms = float(np.sqrt(np.mean((got - ref) ** 2)) / max(np.sqrt(np.mean(ref ** 2)), 1e-30))
+        assert rms <= 5e-3, f"{what}: rel RMS {rms:.3e} > 5e-3"
+        assert err <= 2e-2 * scale + 1e-6, f"{what}: max abs err {err:.3e} > {2e-2 * scale:.3e}"
+        return
+    bound = REL * scale + ABS
     assert err <= bound, f"{what}: max abs err {err:.3e} > {bound:.3e}"
 
 
@@ -55,8 +66,9 @@ def _case(variant, Nq, Nk, dtype, seed, causal=True, window=0, norm=True, Hq=8, 
     else:
         ref = OB.prefill_v2_bwd(q64, k64, v64, lam64, dy64, causal=causal, window=window)
     tag = f"V{variant} {dtype} Nq={Nq} Nk={Nk} causal={causal} window={window}"
+    tc = variant == 2 and dtype == "bf16"
     for name, t, r in zip(("dq", "dk", "dv", "dlambda"), (dq, dk, dv, dl), ref):
-        _check(t, r, f"{tag} {name}")
+        _check(t, r, f"{tag} {name}", tensor_core=tc)
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
