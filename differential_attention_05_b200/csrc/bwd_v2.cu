@@ -28,6 +28,8 @@
 #include "kernels.h"
 #include "tma_host.cuh"
 
+#include <type_traits>
+
 namespace diffattn {
 
 namespace {
@@ -51,6 +53,14 @@ __device__ __forceinline__ bool visible(const PrefillArgs& a, int i, int j) {
   if (!a.causal) return true;
   const int pos = i + a.Nk - a.N;
   return j <= pos && (a.window <= 0 || j > pos - a.window);
+}
+
+// is every (query, key) pair of queries q0 .. q0+nq-1 and keys k0 .. k0+nk-1 visible
+__device__ __forceinline__ bool tile_visible(const PrefillArgs& a, int q0, int nq, int k0, int nk) {
+  if (q0 + nq > a.N || k0 + nk > a.Nk) return false;
+  if (!a.causal) return true;
+  const int pos_lo = q0 + a.Nk - a.N, pos_hi = pos_lo + nq - 1;
+  return k0 + nk - 1 <= pos_lo && (a.window <= 0 || k0 > pos_hi - a.window);
 }
 
 // ----------------------------------------------------------------------------- dK, dV
@@ -235,8 +245,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!(ok = __all_sync(FULL, ok))) break;
       tc_fence_after();
       const float4* sts = reinterpret_cast<const float4*>(smem + STAGE_OFF + s * STAGE_BYTES + STS);
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      // inside the visible region (most steps of a causal problem) no pair needs a mask
+      const bool full = tile_visible(a, q0, QT, k0, KT);
+      auto chunk = [&](int c, auto all_visible) {
         float s1[32], s2[32], dp[32];
         tmem_ld32f(lane_addr + C_S + 32 * c, s1);
         tmem_ld32f(lane_addr + C_S + 64 + 32 * c, s2);
@@ -250,7 +261,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int x = 0; x < 2; ++x) {
             const int qq = 32 * c + e + x;
             const float4 st = sts[qq];
-            const bool vis = visible(a, q0 + qq, j);
+            const bool vis = decltype(all_visible)::value || visible(a, q0 + qq, j);
             const float p1 = vis ? ex2(s1[e + x] * sl2 - st.x) : 0.f;
             const float p2 = vis ? ex2(s2[e + x] * sl2 - st.y) : 0.f;
             vpc[x] = p1 - lam * p2;
@@ -265,6 +276,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_st16(lane_addr + C_PC + 16 * c, pc);
         tmem_st16(lane_addr + C_DS + 16 * c, d1);
         tmem_st16(lane_addr + C_DS + 32 + 16 * c, d2);
+      };
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        if (full) chunk(c, std::true_type{});
+        else chunk(c, std::false_type{});
       }
       tmem_wait_st();
       tc_fence_before();
@@ -486,8 +502,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!(ok = __all_sync(FULL, ok))) break;
       tc_fence_after();
       const int kj0 = (j_lo + t) * KT;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      const bool full = tile_visible(a, q0, QT, kj0, KT);
+      auto chunk = [&](int c, auto all_visible) {
         float sv[32], dp[32];
         tmem_ld32f(lane_addr + C_S + 32 * c, sv);
         tmem_ld32f(lane_addr + C_DP + 32 * c, dp);
@@ -498,13 +514,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           float v2[2];
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
-            const bool vis = visible(a, qi, kj0 + 32 * c + e + x);
+            const bool vis = decltype(all_visible)::value || visible(a, qi, kj0 + 32 * c + e + x);
             const float p = vis ? ex2(sv[e + x] * sl2 - lse) : 0.f;
             v2[x] = vis ? coef * p * (dp[e + x] - del) : 0.f;
           }
           ds[e / 2] = pack_bf16(v2[0], v2[1]);
         }
         tmem_st16(lane_addr + C_DS + 16 * c, ds);
+      };
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        if (full) chunk(c, std::true_type{});
+        else chunk(c, std::false_type{});
       }
       tmem_wait_st();
       tc_fence_before();
