@@ -2,11 +2,15 @@
 """Benchmark of the differential attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload c2|c3|c4|c5|d1] [--no-secondary]
+                    [--workload c2|c3|c4|c5|d1|b3|p4] [--no-secondary]
 
 A step is one pass of the hot path over one batch of synthetic input: the on-device
 lambda re-parameterisation followed by the fused prefill (or the split-KV decode for the
 decode workload). Default workload: the V1 bf16 layer (B=2, 16 heads, N=4096, d=64).
+Other workloads: c3 V2 prefill (N=16384, 64/8 heads, d=128), c4 V2 decode (batch 64, cache
+32768), c5 V2 long context (N=65536), d1 V1 decode, b3 the backward of a V2 prefill (N=4096,
+64/8 heads; step = lambda + the whole backward), p4 the c4 decode over 16-token pages in a
+shuffled block table.
 Inputs are the seeded synthetic tensors of differential_attention_05_b200.synth.
 
 Timing: W untimed warm-up steps, then K steps between a barrier + synchronize on both
@@ -48,6 +52,10 @@ def workload_inputs(name: str, batch: int = 0):
         return synth.v2_decode(B=batch, name=f"v2_bf16_decode_b{batch}_l32768_hq64_hkv8_d128")
     if name == "d1":
         return synth.v1_decode(B=batch) if batch else synth.v1_decode()
+    if name == "b3":
+        return synth.v2_backward()
+    if name == "p4":
+        return synth.v2_decode(B=batch or 64, name=f"v2_bf16_decode_paged16_b{batch or 64}_l32768_hq64_hkv8_d128")
     return {"c2": synth.config2, "c3": synth.config3, "c4": synth.config4, "c5": synth.config5}[name]()
 
 
@@ -239,6 +247,17 @@ def run_ours(args, rank, world, device):
     li = torch.empty(1, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
     decode = inp.mode == "decode"
+    backward = args.workload == "b3"
+    paged = args.workload == "p4"
+    if paged:
+        # the cache as a pool of 16-token pages in a seeded shuffled order (block table)
+        ps = 16
+        kp = k.view(inp.B * inp.N // ps, ps, inp.Hkv, inp.d)
+        vp = v.view(inp.B * inp.N // ps, ps, inp.Hkv, inp.d)
+        gen = torch.Generator(device=device)
+        gen.manual_seed(1008)
+        bt = torch.randperm(inp.B * inp.N // ps, generator=gen, device=device).to(torch.int32)
+        bt = bt.view(inp.B, inp.N // ps)
     if decode:
         if inp.variant == 1:
             out = torch.empty((inp.B, inp.H, 2 * inp.d), dtype=torch.bfloat16, device=device)
@@ -250,6 +269,19 @@ def run_ours(args, rank, world, device):
                          device=device)
         work = workload_decode_bytes(inp)
         unit, metric = "GB/s", "diff-attn decode KV GB/s at 1 B200"
+    elif backward:
+        dy = dev(inp.extra["dy"])
+        grads = (torch.empty(q.shape, dtype=torch.float32, device=device),
+                 torch.empty(k.shape, dtype=torch.float32, device=device),
+                 torch.empty(v.shape, dtype=torch.float32, device=device),
+                 torch.empty(lam.shape, dtype=torch.float32, device=device))
+        p = da._binding.prefill_params(q, k, v, dy)
+        ws = torch.empty(da._binding.diffattn_bwd_workspace_size(p), dtype=torch.uint8, device=device)
+        out = grads[0]
+        # algorithmic FLOPs per attended (query head, key) pair: 8 d (scores 2d, dP d per
+        # head, dQ 2d, dK 2d, dV d per head)
+        work = 8.0 * inp.d * inp.H * inp.B * visible_pairs(inp.N, inp.N, inp.causal)
+        unit, metric = "TFLOP/s", "diff-attn backward TFLOP/s (% bf16 peak)"
     else:
         out = (torch.empty((inp.B, inp.N, inp.H, 2 * inp.d), dtype=torch.bfloat16, device=device)
                if inp.variant == 1 else
@@ -264,7 +296,11 @@ def run_ours(args, rank, world, device):
         da.diffattn_lambda(*vecs, depth=inp.depth, lambda_out=lam, lambda_init_out=li)
 
     def main_kernel():
-        if decode and inp.variant == 1:
+        if paged:
+            da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws)
+        elif backward:
+            da.diffattn_bwd_prefill(q, k, v, lam, dy, causal=inp.causal, workspace=ws, grads=grads)
+        elif decode and inp.variant == 1:
             da.diffattn_fwd_decode_v1(q, k, v, lam, li, out=out, apply_norm=inp.apply_norm,
                                       norm_eps=inp.eps, workspace=ws)
         elif decode:
@@ -273,7 +309,7 @@ def run_ours(args, rank, world, device):
             da.diffattn_fwd_prefill(q, k, v, lam, li, out=out, causal=inp.causal,
                                     apply_norm=inp.apply_norm, norm_eps=inp.eps)
 
-    launches_per_step = 1 + (2 if decode else 1)
+    launches_per_step = 1 + (2 if decode else (4 if backward else 1))
 
     for _ in range(args.warmup):
         lambda_step()
@@ -323,19 +359,24 @@ def run_ours(args, rank, world, device):
                torch.from_numpy(inp.v.view(np.int16) if inp.v.dtype == np.uint16 else inp.v).pin_memory()]
     host_vec = [torch.from_numpy(np.ascontiguousarray(getattr(inp, n))).pin_memory()
                 for n in ("lq1", "lk1", "lq2", "lk2")]
-    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    if backward:
+        host_in.append(torch.from_numpy(inp.extra["dy"].view(np.int16)).pin_memory())
+    dev_in = (q, k, v, dy) if backward else (q, k, v)
+    dev_out = grads if backward else (out,)
+    host_outs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dev_out]
     h2d = sum(t.numel() * t.element_size() for t in host_in + host_vec)
-    d2h = host_out.numel() * host_out.element_size()
+    d2h = sum(t.numel() * t.element_size() for t in host_outs)
     e2e_steps = max(3, min(args.steps, 10))
 
     def e2e_step():
-        for src, dst in zip(host_in, (q, k, v)):
+        for src, dst in zip(host_in, dev_in):
             dst.view(src.dtype).copy_(src, non_blocking=True)
         for src, dst in zip(host_vec, vecs):
             dst.copy_(src, non_blocking=True)
         lambda_step()
         main_kernel()
-        host_out.copy_(out, non_blocking=True)
+        for dst, src in zip(host_outs, dev_out):
+            dst.copy_(src, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(device)
@@ -354,6 +395,11 @@ def run_ours(args, rank, world, device):
     kernel_name = (("decode_v1_split_kernel" if inp.variant == 1 else "decode_split_kernel")
                    if decode else f"prefill_v{inp.variant}_kernel")
     traffic = measured_traffic(kernel_name, inp.name, inp.B, decode)
+    if backward:
+        # the timed span is the whole backward call (its four launches)
+        kernel_name = ("prefill_v2_kernel (statistics mode) + bwd_v2_dkdv_kernel + "
+                       "bwd_v2_dq_kernel + bwd_dlambda_kernel")
+        traffic = None
     line = {
         "metric": metric,
         "value": round(value, 3),
@@ -391,7 +437,11 @@ def run_ours(args, rank, world, device):
         "clocks": clocks,
         "wall_s_timed": round(t_wall, 4),
     }
-    del q, k, v, out
+    del q, k, v, out, dev_in, dev_out
+    if backward:
+        del dy, grads
+    if paged:
+        del kp, vp, bt
     torch.cuda.empty_cache()
     if not args.no_secondary and not decode and args.workload == "c2":
         line["secondary"] = secondary(device, peaks, torch, da)
@@ -605,9 +655,44 @@ def oracle_decode_sample(inp, seconds):
     return n, dt
 
 
+def oracle_backward_sample(inp, seconds):
+    """The float64 backward oracle on whole query-head pairs (full sequence, every key) of
+    a backward workload, pair after pair until `seconds` have passed; returns (pairs, s)."""
+    import oracle
+    from oracle import backward as OB
+    from differential_attention_05_b200 import synth
+    lam = oracle.lambda_(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.depth)
+    group = inp.H // inp.Hkv
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        p = n % (inp.H // 2)
+        g = (2 * p) // group
+        q = synth.bf16_to_f32(inp.q[:1, :, 2 * p:2 * p + 2]).astype(np.float64)
+        k = synth.bf16_to_f32(inp.k[:1, :, g:g + 1]).astype(np.float64)
+        v = synth.bf16_to_f32(inp.v[:1, :, g:g + 1]).astype(np.float64)
+        dy = synth.bf16_to_f32(inp.extra["dy"][:1, :, p:p + 1]).astype(np.float64)
+        OB.prefill_v2_bwd(q, k, v, lam[p:p + 1], dy, causal=inp.causal)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    return n, time.perf_counter() - t0
+
+
+def backward_pair_flops(inp) -> float:
+    """Algorithmic FLOPs of one pair's backward over one batch entry (8 d per attended
+    (query head, key) pair, two query heads)."""
+    return 8.0 * inp.d * 2 * visible_pairs(inp.N, inp.N, inp.causal)
+
+
 def cpu_baseline(inp, seconds=12.0):
     import oracle
     cores = oracle.default_threads()
+    if "dy" in inp.extra:
+        n, dt = oracle_backward_sample(inp, seconds)
+        return {"value": round(n * backward_pair_flops(inp) / dt / 1e12, 6), "unit": "TFLOP/s",
+                "cores": cores, "kind": "oracle",
+                "sample": f"{n} whole query-head pairs (every row and key) of {inp.name}, {dt:.1f} s"}
     if inp.mode == "decode":
         n, dt = oracle_decode_sample(inp, seconds)
         val = n * workload_decode_bytes(inp) / inp.B / dt / 1e9
@@ -629,7 +714,18 @@ def run_reference(args, rank, world):
     cores = oracle.default_threads()
     decode = inp.mode == "decode"
     per_step_s = max(0.5, min(8.0, 120.0 / max(1, args.steps + args.warmup)))
-    if decode:
+    if "dy" in inp.extra:
+        times = []
+        for i in range(args.warmup + args.steps):
+            n, dt = oracle_backward_sample(inp, per_step_s)
+            if i >= args.warmup:
+                times.append((n, dt))
+        total_units = sum(n for n, _ in times)
+        total_s = sum(dt for _, dt in times)
+        value = total_units * backward_pair_flops(inp) / total_s / 1e12
+        unit, metric = "TFLOP/s", "diff-attn backward TFLOP/s (% bf16 peak)"
+        sample = f"whole query-head pairs of {inp.name} ({total_units} in {total_s:.1f} s)"
+    elif decode:
         times = []
         for i in range(args.warmup + args.steps):
             n, dt = oracle_decode_sample(inp, per_step_s)
@@ -679,7 +775,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("c2", "c3", "c4", "c5", "d1"), default="c2")
+    ap.add_argument("--workload", choices=("c2", "c3", "c4", "c5", "d1", "b3", "p4"), default="c2")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="decode workload only: smaller batch (profiling runs)")

@@ -302,17 +302,21 @@ def diffattn_bwd_workspace_size(p: PrefillParams) -> int:
 
 
 def diffattn_bwd_prefill(q, k, v, lam, dout, lambda_init=None, causal=True, apply_norm=None,
-                         norm_eps=1e-5, window=0, workspace=None, dev_status=None, stream=None):
+                         norm_eps=1e-5, window=0, workspace=None, dev_status=None, stream=None,
+                         grads=None):
     """Gradients of diffattn_fwd_prefill (see include/diffattn.h): dout has the forward
     output's layout and dtype. Returns float32 (dq, dk, dv, dlambda) in the shapes of q, k,
-    v and lambda."""
+    v and lambda (written into `grads` when given: four dense float32 tensors)."""
     import torch
     lib = load_library()
     p = prefill_params(q, k, v, dout, causal, apply_norm, norm_eps, window)
-    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
-    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
-    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
-    dl = torch.empty(lam.shape, dtype=torch.float32, device=q.device)
+    if grads is None:
+        dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+        dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+        dl = torch.empty(lam.shape, dtype=torch.float32, device=q.device)
+    else:
+        dq, dk, dv, dl = grads
     need = diffattn_bwd_workspace_size(p)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)

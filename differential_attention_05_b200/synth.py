@@ -155,6 +155,20 @@ def v2_prefill(B=1, N=16384, Hq=64, Hkv=8, d=128, depth=24, seed=1002, name=None
                   B, N, Hq, Hkv, d, depth, q, k, v, *_lambda_vectors(seed, Hq // 2, d))
 
 
+def grad_out(shape, seed: int) -> np.ndarray:
+    """A seeded incoming gradient dL/dy of the given shape, N(0,1), as bf16 bits."""
+    return _normal_sliced(seed, _T_V + 17, tuple(shape))
+
+
+def v2_backward(B=1, N=4096, Hq=64, Hkv=8, d=128, depth=24, seed=1007, name=None) -> Inputs:
+    """Backward of a V2 prefill: the V2 prefill inputs (iid N(0,1)) plus dy [B,N,Hq/2,d]
+    N(0,1) in extra["dy"]."""
+    inp = v2_prefill(B=B, N=N, Hq=Hq, Hkv=Hkv, d=d, depth=depth, seed=seed,
+                     name=name or f"v2_bf16_backward_b{B}_n{N}_hq{Hq}_hkv{Hkv}_d{d}")
+    inp.extra["dy"] = grad_out((B, N, Hq // 2, d), seed)
+    return inp
+
+
 def config3() -> Inputs:
     """V2 prefill, bf16, causal, GQA: B=1, 64 query heads (32 pairs) over 8 KV heads,
     d=128, N=16384; iid N(0,1); per-pair lambda at depth 24; no norm."""
