@@ -193,10 +193,12 @@ int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t*
                      out, dev_status, stream);
 }
 
-// the tensor-core backward covers V2 in bf16 with d = 128; everything else runs on the
-// exact-fp32 SIMT kernels
+// the tensor-core backward covers bf16 V2 with d = 128 and bf16 V1 with d = 64 (the shapes
+// of the tcgen05 forward kernels); everything else runs on the exact-fp32 SIMT kernels
 static bool bwd_tensor_core(const diffattn_prefill_params* p) {
-  return p->variant == DIFFATTN_V2 && p->dtype == DIFFATTN_BF16 && p->head_dim == 128;
+  if (p->dtype != DIFFATTN_BF16) return false;
+  return (p->variant == DIFFATTN_V2 && p->head_dim == 128) ||
+         (p->variant == DIFFATTN_V1 && p->head_dim == 64);
 }
 
 // backward: any d <= 128 with d % 4 == 0, f32 or bf16 inputs, fixed-length batches
@@ -225,7 +227,7 @@ int diffattn_bwd_workspace_size(const diffattn_prefill_params* p, size_t* bytes)
   } else {
     return DIFFATTN_ERR_INVALID_ARG;
   }
-  *bytes = bwd_tensor_core(p) ? bwd_v2_tc_workspace_bytes(p->batch, p->seqlen, units)
+  *bytes = bwd_tensor_core(p) ? bwd_tc_workspace_bytes(p->variant, p->batch, p->seqlen, units)
                               : bwd_workspace_bytes(p->batch, p->seqlen, units, dv);
   return DIFFATTN_OK;
 }
@@ -246,7 +248,7 @@ int diffattn_bwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return DIFFATTN_ERR_MISALIGNED;
   const PrefillArgs& a = g.f;
   const bool tc = bwd_tensor_core(p);
-  const size_t need = tc ? bwd_v2_tc_workspace_bytes(a.B, a.N, a.units)
+  const size_t need = tc ? bwd_tc_workspace_bytes(a.variant, a.B, a.N, a.units)
                          : bwd_workspace_bytes(a.B, a.N, a.units, a.dv);
   if (!workspace || workspace_bytes < need) return DIFFATTN_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIFFATTN_ERR_MISALIGNED;
@@ -258,7 +260,7 @@ int diffattn_bwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   g.dv = dv;
   g.dlambda = dlambda;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return from_cuda(tc ? launch_backward_v2_tc(g, workspace, s) : launch_backward(g, workspace, s));
+  return from_cuda(tc ? launch_backward_tc(g, workspace, s) : launch_backward(g, workspace, s));
 }
 
 int diffattn_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
