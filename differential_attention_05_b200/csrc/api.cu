@@ -193,12 +193,13 @@ int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t*
                      out, dev_status, stream);
 }
 
-// the tensor-core backward covers bf16 V2 with d = 128 and bf16 V1 with d = 64 (the shapes
-// of the tcgen05 forward kernels); everything else runs on the exact-fp32 SIMT kernels
+// the tensor-core backward serves bf16 V2 with d = 128; everything else runs on the
+// exact-fp32 SIMT kernels. (The tensor-core kernels also take V1, d = 64: its dQ, dK and dV
+// meet the bf16 bounds, but dlambda through the per-head norm's backward measured 0.5-1.1%
+// relative RMS off the float64 reference, above the 5e-3 the other outputs meet, so V1 stays
+// on the exact path.)
 static bool bwd_tensor_core(const diffattn_prefill_params* p) {
-  if (p->dtype != DIFFATTN_BF16) return false;
-  return (p->variant == DIFFATTN_V2 && p->head_dim == 128) ||
-         (p->variant == DIFFATTN_V1 && p->head_dim == 64);
+  return p->dtype == DIFFATTN_BF16 && p->variant == DIFFATTN_V2 && p->head_dim == 128;
 }
 
 // backward: any d <= 128 with d % 4 == 0, f32 or bf16 inputs, fixed-length batches
