@@ -201,8 +201,11 @@ int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t*
  *              diffattn_lambda_bwd for the four lambda vectors
  * workspace  : >= diffattn_bwd_workspace_size(p) bytes, 256-byte aligned (per row: dO in
  *              fp32, two log-sum-exps, two deltas, the row's dlambda share)
- * Arithmetic: fp32 on the CUDA cores for every dtype; deterministic (no atomics: dQ rows,
- * dK/dV rows and dlambda are each summed by one thread group in a fixed order).
+ * Arithmetic: bf16 V2 with d = 128 runs on the tensor cores (fp32 accumulation; the MMA
+ * operands P_1 - lambda P_2 and dS_b rounded to bf16, as the forward rounds its P operand);
+ * every other case (fp32 inputs, V1, other d) runs exact fp32 on the CUDA cores. Both are
+ * deterministic (no atomics: dQ rows, dK/dV rows and dlambda are each summed by one thread
+ * group in a fixed order).
  * Errors as for diffattn_fwd_prefill, plus DIFFATTN_ERR_WORKSPACE.
  */
 int diffattn_bwd_workspace_size(const diffattn_prefill_params* p, size_t* bytes);

@@ -294,3 +294,24 @@ def test_backward_workspace_and_rejects(lib):
     assert f(ctypes.byref(p), *ptr, None, *outs[1:], vp(GOOD * 4), need, None, None) == -1
     assert lib.diffattn_lambda_bwd(None, vp(GOOD), vp(GOOD), vp(GOOD), 4, 64, vp(GOOD),
                                    vp(GOOD), vp(GOOD), vp(GOOD), vp(GOOD), None) == -1
+
+
+def _declared_arity():
+    """Number of parameters of every entry point as include/diffattn.h declares it."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(diffattn_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(lib):
+    """The binding's ctypes signatures have the header's parameter counts (catches an entry
+    point whose C signature changed without its binding)."""
+    arity = _declared_arity()
+    assert set(arity) == set(B.EXPORTS)
+    for name in B.EXPORTS:
+        argtypes = getattr(lib, name).argtypes
+        assert argtypes is not None, f"{name}: no argtypes"
+        assert len(argtypes) == arity[name], f"{name}: binding {len(argtypes)} vs header {arity[name]}"
