@@ -315,3 +315,18 @@ def test_binding_signatures_match_the_header(lib):
         argtypes = getattr(lib, name).argtypes
         assert argtypes is not None, f"{name}: no argtypes"
         assert len(argtypes) == arity[name], f"{name}: binding {len(argtypes)} vs header {arity[name]}"
+
+
+def test_plain_c_program(lib, tmp_path):
+    """A plain C program compiled against include/diffattn.h and linked to the library runs
+    the host-side paths (no GPU): the boundary is a C ABI, not a Python one."""
+    import subprocess
+    src = os.path.join(ROOT, "tests", "c", "abi_host.c")
+    exe = str(tmp_path / "abi_host")
+    libdir = os.path.dirname(da.library_path())
+    subprocess.check_call(["gcc", "-std=c11", "-O1", "-I", os.path.join(ROOT, "include"), src,
+                           "-L", libdir, "-l:" + os.path.basename(da.library_path()),
+                           "-Wl,-rpath," + libdir, "-o", exe])
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert "all checks hold" in r.stdout
