@@ -22,6 +22,13 @@
  *   Causal: query i sees keys j <= i
  *     -- "Attention Variants", Build It, Step 1 (causal_mask).
  *
+ * Entry points: diffattn_lambda; diffattn_fwd_prefill (V1 / V2, bf16 or f32; causal, full,
+ * chunked, sliding window) and diffattn_fwd_prefill_varlen (packed sequences);
+ * diffattn_fwd_decode (V2), diffattn_fwd_decode_v1, diffattn_fwd_decode_paged (block
+ * table), diffattn_fwd_decode_static, diffattn_decode_workspace_size; diffattn_bwd_prefill,
+ * diffattn_bwd_workspace_size, diffattn_lambda_bwd (training); diffattn_selftest_timeout
+ * (the bounded-wait path); diffattn_version, diffattn_status_string.
+ *
  * Conventions for every entry point
  *   - Pointers are DEVICE pointers unless marked "host". The caller owns every buffer;
  *     the library allocates nothing, frees nothing and keeps no pointer after a call.
