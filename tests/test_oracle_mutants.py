@@ -34,6 +34,10 @@ MUTANTS = {
                              "d2 += lq2[(long)h * dim + c] * lk1[(long)h * dim + c];"),
     "lambda_init_rate": ("return 0.8 - 0.6 * exp(-0.3 * (double)(depth - 1));",
                          "return 0.8 - 0.6 * exp(-0.3 * (double)depth);"),
+    "lambda_init_rate_constant": ("return 0.8 - 0.6 * exp(-0.3 * (double)(depth - 1));",
+                                  "return 0.8 - 0.6 * exp(-0.25 * (double)(depth - 1));"),
+    "lambda_init_amplitude": ("return 0.8 - 0.6 * exp(-0.3 * (double)(depth - 1));",
+                              "return 0.8 - 0.5 * exp(-0.3 * (double)(depth - 1));"),
     "v1_q2_is_q1": ("const double* q2 = q1 + d;\n    int hi = jb->causal", "const double* q2 = q1;\n    int hi = jb->causal"),
     "v1_decode_q2_is_q1": ("const double* q2 = q1 + d;\n  int n_keys = jb->kv_len", "const double* q2 = q1;\n  int n_keys = jb->kv_len"),
     "v1_value_of_other_head": ("const double* vb = jb->v + (long)b * jb->Nk * tok_v + (long)h * dv;",
