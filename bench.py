@@ -6,12 +6,16 @@
 
 A step is one pass of the hot path over one batch of synthetic input: the on-device
 lambda re-parameterisation followed by the fused prefill (or the split-KV decode for the
-decode workload). Default workload: the V1 bf16 layer (B=2, 16 heads, N=4096, d=64).
-Other workloads: c3 V2 prefill (N=16384, 64/8 heads, d=128), c4 V2 decode (batch 64, cache
-32768), c5 V2 long context (N=65536), d1 V1 decode, b3 the backward of a V2 prefill (N=4096,
-64/8 heads; step = lambda + the whole backward), p4 the c4 decode over 16-token pages in a
-shuffled block table.
-Inputs are the seeded synthetic tensors of differential_attention_05_b200.synth.
+decode workload). Default workload (the largest one-GPU workload): c5, the V2 long-context
+signal-plus-noise prefill (B=1, N=65536, 64 query heads over 8 KV heads, d=128, causal).
+Other workloads: c2 the V1 bf16 layer (B=2, 16 heads, N=4096, d=64), c3 V2 prefill
+(N=16384, 64/8 heads, d=128), c4 V2 decode (batch 64, cache 32768), d1 V1 decode, b3 the
+backward of a V2 prefill (N=4096, 64/8 heads; step = lambda + the whole backward), p4 the c4
+decode over 16-token pages in a shuffled block table.
+Inputs are the seeded synthetic tensors of differential_attention_05_b200.synth. With the
+default workload the line also carries "secondary": the other rows timed alone (the V1
+layer, the V2 prefill, its window and chunk forms and its backward on the synth tensors; the
+decodes on same-shape seeded draws made on the device, each entry saying which).
 
 Timing: W untimed warm-up steps, then K steps between a barrier + synchronize on both
 sides; every step is bracketed by CUDA events on the launching stream and L2 is flushed
@@ -139,6 +143,21 @@ def measured_traffic(kernel: str, workload: str, batch: int, decode: bool):
             return None
         return float(f[4]) * scale
     return None
+
+
+def workload_config(inp, world: int) -> dict:
+    """The line's "config": the workload and its sizes, identical in both arms."""
+    decode = inp.mode == "decode"
+    in_bytes = inp.q.nbytes + inp.k.nbytes + inp.v.nbytes
+    return {
+        "workload": inp.name,
+        "batch": inp.B, "seq_len": inp.N, "heads": inp.H, "kv_heads": inp.Hkv,
+        "head_dim": inp.d, "causal": bool(inp.causal), "depth": inp.depth,
+        "tokens_per_step": inp.B * (1 if decode else inp.N),
+        "l2": ("flushed between steps (256 MB write, outside the timed events)"
+               if in_bytes < 2 * L2_BYTES else "inputs larger than L2"),
+        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+    }
 
 
 # ---------------------------------------------------------------------------------------
@@ -395,6 +414,10 @@ def run_ours(args, rank, world, device):
     kernel_name = (("decode_v1_split_kernel" if inp.variant == 1 else "decode_split_kernel")
                    if decode else f"prefill_v{inp.variant}_kernel")
     traffic = measured_traffic(kernel_name, inp.name, inp.B, decode)
+    # the bytes the kernel must move at least: its inputs read once and its output written
+    # once (prefill), the caches read once (decode)
+    algo_bytes = (work if decode else
+                  float(in_bytes + out.numel() * out.element_size()))
     if backward:
         # the timed span is the whole backward call (its four launches)
         kernel_name = ("prefill_v2_kernel (statistics mode) + bwd_v2_dkdv_kernel + "
@@ -413,23 +436,19 @@ def run_ours(args, rank, world, device):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded numpy PCG64, bf16-rounded; shapes and distributions of the workload)",
-        "config": {
-            "workload": inp.name,
-            "batch": inp.B, "seq_len": inp.N, "heads": inp.H, "kv_heads": inp.Hkv,
-            "head_dim": inp.d, "causal": bool(inp.causal), "depth": inp.depth,
-            "tokens_per_step": inp.B * (1 if decode else inp.N),
-            "l2": ("flushed between steps (256 MB write, outside the timed events)" if flush
-                   else "inputs larger than L2"),
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-        },
+        "config": workload_config(inp, world),
         "tokens_per_s": round(world * inp.B * (1 if decode else inp.N) * args.steps / (total_ms * 1e-3), 1),
         "roofline": {
             "bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": runit,
             "frac": round(achieved / peak, 4), "traffic": traffic,
+            "traffic_over_algorithmic": (round(traffic / algo_bytes, 3)
+                                         if traffic and algo_bytes else None),
             "peak_source": f"{peaks['source']} ({'burst bf16' if bound == 'tensor' else 'HBM copy'})",
             "kernel": (kernel_name + (" + decode_v1_combine_kernel" if inp.variant == 1 else
                                       " + decode_combine_kernel") if decode else kernel_name),
             "avg_kernel_ms": round(kern_avg, 5),
+            **({"frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                "sustained_peak": peaks["bf16_tflops_sustained"]} if bound == "tensor" else {}),
         },
         "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
@@ -443,95 +462,106 @@ def run_ours(args, rank, world, device):
     if paged:
         del kp, vp, bt
     torch.cuda.empty_cache()
-    if not args.no_secondary and not decode and args.workload == "c2":
+    if not args.no_secondary and args.workload == "c5":
         line["secondary"] = secondary(device, peaks, torch, da)
     return line
 
 
+def _timed(fn, torch, reps=10, warm=3):
+    """Median CUDA-event time (ms) of `fn` on the current stream over `reps` calls."""
+    for _ in range(warm):
+        fn()
+    es = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for a, b in es:
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in es)
+
+
 def secondary(device, peaks, torch, da):
-    """Other rows of the hot path, timed alone: V2 prefill (64/8 heads, d=128, N=16384),
-    V2 decode (batch 64, cache 32768) and V1 decode (batch 32, cache 32768, 16 heads,
-    d=64). Inputs are drawn on the device (seeded N(0,1), same shapes) to keep the run
-    short; all exceed L2."""
+    """Other rows of the hot path, each timed alone (median of 10 launches):
+      * the V1 bf16 layer (B=2, 16 heads, N=4096, d=64) and the V2 prefill (N=16384, 64/8
+        heads, d=128) on their seeded synth tensors, lambda from the lambda kernel; the
+        V2 tensors also as a 4096-key sliding-window layer and as a 2048-query chunk, and
+        the V2 backward on the seeded N=4096 backward workload;
+      * the V2 decode (batch 64, cache 32768; contiguous and over 16/256-token pages) and
+        the V1 decode (batch 32, cache 32768, 16 heads, d=64) on same-shape seeded N(0,1)
+        draws made on the device (the synth caches take minutes to draw on the host), with
+        the synth lambda vectors.
+    TFLOP/s against the measured bf16 peak, GB/s against the measured copy bandwidth."""
+    from differential_attention_05_b200 import synth
     res = {}
-    g = torch.Generator(device=device)
-    g.manual_seed(1002)
-    N, Hq, Hkv, d = 16384, 64, 8, 128
-    q = torch.randn((1, N, Hq, d), generator=g, device=device).bfloat16()
-    k = torch.randn((1, N, Hkv, d), generator=g, device=device).bfloat16()
-    v = torch.randn((1, N, Hkv, d), generator=g, device=device).bfloat16()
-    lam = torch.full((Hq // 2,), 0.8, dtype=torch.float32, device=device)
+    tflops = lambda fl, ms: {"ms": round(ms, 4), "TFLOP/s": round(fl / ms / 1e9, 2),
+                             "frac_of_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
+    gbs = lambda by, ms: {"ms": round(ms, 4), "GB/s": round(by / ms / 1e6, 1),
+                          "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
+
+    def dev(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    def lam_of(vecs, depth):
+        lam = torch.empty(vecs[0].shape[0], dtype=torch.float32, device=device)
+        li = torch.empty(1, dtype=torch.float32, device=device)
+        da.diffattn_lambda(*[dev(x) for x in vecs], depth=depth, lambda_out=lam, lambda_init_out=li)
+        return lam, li
+
+    seeded = "seeded synth tensors"
+    # ---- V1 layer
+    inp = synth.config2()
+    q, k, v = dev(inp.q), dev(inp.k), dev(inp.v)
+    lam, li = lam_of((inp.lq1, inp.lk1, inp.lq2, inp.lk2), inp.depth)
+    out = torch.empty((inp.B, inp.N, inp.H, 2 * inp.d), dtype=torch.bfloat16, device=device)
+    ms = _timed(lambda: da.diffattn_fwd_prefill(q, k, v, lam, li, out=out, apply_norm=True,
+                                                norm_eps=inp.eps), torch)
+    res["v1_layer"] = {"workload": inp.name, "inputs": seeded, **tflops(prefill_flops(inp), ms)}
+    del q, k, v, out
+    # ---- V2 prefill, its window and chunk forms
+    inp = synth.config3()
+    q, k, v = dev(inp.q), dev(inp.k), dev(inp.v)
+    lam, li = lam_of((inp.lq1, inp.lk1, inp.lq2, inp.lk2), inp.depth)
+    N, Hq, Hkv, d = inp.N, inp.H, inp.Hkv, inp.d
     out = torch.empty((1, N, Hq // 2, d), dtype=torch.bfloat16, device=device)
-    for _ in range(3):
-        da.diffattn_fwd_prefill(q, k, v, lam, out=out)
-    es = [(torch.cuda.Event(True), torch.cuda.Event(True)) for _ in range(10)]
-    for a, b in es:
-        a.record()
-        da.diffattn_fwd_prefill(q, k, v, lam, out=out)
-        b.record()
-    torch.cuda.synchronize(device)
-    ms = statistics.median(a.elapsed_time(b) for a, b in es)
-    fl = 4.0 * d * Hq * N * (N + 1) / 2
-    res["v2_prefill"] = {"workload": "v2_bf16_prefill_b1_n16384_hq64_hkv8_d128", "ms": round(ms, 4),
-                         "TFLOP/s": round(fl / ms / 1e9, 2),
-                         "frac_of_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
-    # the backward pass on the first 4096 tokens of the same tensors (tensor-core kernels:
-    # statistics pass, dK/dV, dQ, dlambda sum); algorithmic FLOPs per attended (query head,
-    # key) pair: 8 d (scores 2d, dP d per head, dQ 2d, dK 2d, dV d per head)
-    Nb = 4096
-    qb, kb, vb = q[:, :Nb].contiguous(), k[:, :Nb].contiguous(), v[:, :Nb].contiguous()
-    dyb = torch.randn((1, Nb, Hq // 2, d), generator=g, device=device).bfloat16()
-    for _ in range(3):
-        da.diffattn_bwd_prefill(qb, kb, vb, lam, dyb)
-    for a, b in es:
-        a.record()
-        da.diffattn_bwd_prefill(qb, kb, vb, lam, dyb)
-        b.record()
-    torch.cuda.synchronize(device)
-    ms = statistics.median(a.elapsed_time(b) for a, b in es)
-    fl = 8.0 * d * Hq * visible_pairs(Nb, Nb)
-    res["v2_backward_n4096"] = {"workload": "v2_bf16_prefill_b1_n4096_hq64_hkv8_d128 backward",
-                                "ms": round(ms, 4), "TFLOP/s": round(fl / ms / 1e9, 2),
-                                "frac_of_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
-    del qb, kb, vb, dyb
+    ms = _timed(lambda: da.diffattn_fwd_prefill(q, k, v, lam, out=out), torch)
+    res["v2_prefill"] = {"workload": inp.name, "inputs": seeded, **tflops(prefill_flops(inp), ms)}
     # the same tensors as a sliding-window layer (4096 keys) and as a 2048-query chunk at
     # the end of the 16384-key context; FLOPs count the attended pairs only
     for name, Nq, window in (("v2_prefill_window4096", N, 4096), ("v2_prefill_chunk2048", 2048, 0)):
-        qq = q[:, N - Nq:]
-        oo = out[:, N - Nq:]
-        for _ in range(3):
-            da.diffattn_fwd_prefill(qq, k, v, lam, out=oo, window=window)
-        for a, b in es:
-            a.record()
-            da.diffattn_fwd_prefill(qq, k, v, lam, out=oo, window=window)
-            b.record()
-        torch.cuda.synchronize(device)
-        ms = statistics.median(a.elapsed_time(b) for a, b in es)
-        fl = 4.0 * d * Hq * visible_pairs(Nq, N, True, window)
-        res[name] = {"queries": Nq, "keys": N, "window": window, "ms": round(ms, 4),
-                     "TFLOP/s": round(fl / ms / 1e9, 2),
-                     "frac_of_bf16_peak": round(fl / ms / 1e9 / peaks["bf16_tflops"], 4)}
-    del q, k, v, out
+        qq, oo = q[:, N - Nq:], out[:, N - Nq:]
+        ms = _timed(lambda: da.diffattn_fwd_prefill(qq, k, v, lam, out=oo, window=window), torch)
+        res[name] = {"workload": inp.name, "inputs": seeded, "queries": Nq, "keys": N,
+                     "window": window, **tflops(4.0 * d * Hq * visible_pairs(Nq, N, True, window), ms)}
+    del q, k, v, out, qq, oo
+    # ---- V2 backward (statistics pass, dK/dV, dQ, dlambda sum); algorithmic FLOPs per
+    # attended (query head, key) pair: 8 d (scores 2d, dP d per head, dQ 2d, dK 2d, dV d)
+    inp = synth.v2_backward()
+    q, k, v, dy = dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.extra["dy"])
+    lam, li = lam_of((inp.lq1, inp.lk1, inp.lq2, inp.lk2), inp.depth)
+    ms = _timed(lambda: da.diffattn_bwd_prefill(q, k, v, lam, dy), torch)
+    res["v2_backward_n4096"] = {"workload": inp.name, "inputs": seeded,
+                                **tflops(8.0 * inp.d * inp.H * visible_pairs(inp.N, inp.N), ms)}
+    del q, k, v, dy
+    torch.cuda.empty_cache()
+    # ---- V2 decode: same-shape draws on the device
+    g = torch.Generator(device=device)
+    g.manual_seed(1003)
+    drawn = "same-shape seeded N(0,1) draws on the device (torch generator), synth lambda vectors"
     B, L = 64, 32768
     q = torch.randn((B, Hq, d), generator=g, device=device).bfloat16()
     k = torch.randn((B, L, Hkv, d), generator=g, device=device).bfloat16()
     v = torch.randn((B, L, Hkv, d), generator=g, device=device).bfloat16()
+    lam, _ = lam_of(synth.lambda_vectors(1003, Hq // 2, d), 24)
     out = torch.empty((B, Hq // 2, d), dtype=torch.bfloat16, device=device)
     p = da._binding.decode_params(q, k, v, out)
     ws = torch.empty(da._binding.diffattn_decode_workspace_size(p), dtype=torch.uint8, device=device)
-    for _ in range(3):
-        da.diffattn_fwd_decode(q, k, v, lam, out=out, workspace=ws)
-    es = [(torch.cuda.Event(True), torch.cuda.Event(True)) for _ in range(10)]
-    for a, b in es:
-        a.record()
-        da.diffattn_fwd_decode(q, k, v, lam, out=out, workspace=ws)
-        b.record()
-    torch.cuda.synchronize(device)
-    ms = statistics.median(a.elapsed_time(b) for a, b in es)
     by = decode_bytes(B, L, Hkv, d)
-    res["decode"] = {"workload": "v2_bf16_decode_b64_l32768_hq64_hkv8_d128", "ms": round(ms, 4),
-                     "GB/s": round(by / ms / 1e6, 1),
-                     "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    ms = _timed(lambda: da.diffattn_fwd_decode(q, k, v, lam, out=out, workspace=ws), torch)
+    res["decode"] = {"workload": "v2_bf16_decode_b64_l32768_hq64_hkv8_d128", "inputs": drawn,
+                     **gbs(by, ms)}
     # the same cache as a page pool: 16-token pages in a shuffled order (block table), the
     # same pages in order (the paging arithmetic alone), 256-token pages shuffled
     for ps, shuffled in ((16, True), (16, False), (256, True)):
@@ -539,44 +569,26 @@ def secondary(device, peaks, torch, da):
         ids = (torch.randperm(B * L // ps, generator=g, device=device) if shuffled
                else torch.arange(B * L // ps, device=device))
         bt = ids.to(torch.int32).view(B, L // ps)
-        for _ in range(3):
-            da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws)
-        for a, b in es:
-            a.record()
-            da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws)
-            b.record()
-        torch.cuda.synchronize(device)
-        ms = statistics.median(a.elapsed_time(b) for a, b in es)
+        ms = _timed(lambda: da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws),
+                    torch)
         res[f"decode_paged{ps}_{'shuffled' if shuffled else 'in_order'}"] = {
             "workload": f"v2_bf16_decode_b64_l32768_hq64_hkv8_d128, {ps}-token pages, "
                         f"{'shuffled' if shuffled else 'in-order'} block table",
-            "ms": round(ms, 4), "GB/s": round(by / ms / 1e6, 1),
-            "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
+            "inputs": drawn, **gbs(by, ms)}
     del q, k, v, out, ws, kp, vp, bt
     torch.cuda.empty_cache()
-    # V1 decode: batch 32, cache 32768, 16 heads, d = 64 (the same cache bytes as above)
+    # ---- V1 decode: batch 32, cache 32768, 16 heads, d = 64 (the V2 decode's cache bytes)
     B, L, H, d1 = 32, 32768, 16, 64
     q = (torch.randn((B, H, 2, d1), generator=g, device=device) / 8).bfloat16()
     k = (torch.randn((B, L, H, 2, d1), generator=g, device=device) / 8).bfloat16()
     v = (torch.randn((B, L, H, 2 * d1), generator=g, device=device) / 8).bfloat16()
-    lam1 = torch.full((H,), 0.8, dtype=torch.float32, device=device)
-    li = torch.full((1,), 0.78, dtype=torch.float32, device=device)
+    lam1, li = lam_of(synth.lambda_vectors(1006, H, d1), 12)
     out = torch.empty((B, H, 2 * d1), dtype=torch.bfloat16, device=device)
     p = da._binding.decode_params_v1(q, k, v, out)
     ws = torch.empty(da._binding.diffattn_decode_workspace_size(p), dtype=torch.uint8, device=device)
-    for _ in range(3):
-        da.diffattn_fwd_decode_v1(q, k, v, lam1, li, out=out, workspace=ws)
-    es = [(torch.cuda.Event(True), torch.cuda.Event(True)) for _ in range(10)]
-    for a, b in es:
-        a.record()
-        da.diffattn_fwd_decode_v1(q, k, v, lam1, li, out=out, workspace=ws)
-        b.record()
-    torch.cuda.synchronize(device)
-    ms = statistics.median(a.elapsed_time(b) for a, b in es)
-    by = decode_bytes(B, L, H, 2 * d1)
-    res["decode_v1"] = {"workload": "v1_bf16_decode_b32_l32768_h16_d64", "ms": round(ms, 4),
-                        "GB/s": round(by / ms / 1e6, 1),
-                        "frac_of_hbm": round(by / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    ms = _timed(lambda: da.diffattn_fwd_decode_v1(q, k, v, lam1, li, out=out, workspace=ws), torch)
+    res["decode_v1"] = {"workload": "v1_bf16_decode_b32_l32768_h16_d64", "inputs": drawn,
+                        **gbs(decode_bytes(B, L, H, 2 * d1), ms)}
     del q, k, v, out, ws
     torch.cuda.empty_cache()
     return res
@@ -757,8 +769,7 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded numpy PCG64, bf16-rounded; shapes and distributions of the workload)",
-        "config": {"workload": inp.name, "batch": inp.B, "seq_len": inp.N, "heads": inp.H,
-                   "kv_heads": inp.Hkv, "head_dim": inp.d, "causal": bool(inp.causal)},
+        "config": workload_config(inp, world),
         "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
@@ -775,7 +786,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("c2", "c3", "c4", "c5", "d1", "b3", "p4"), default="c2")
+    ap.add_argument("--workload", choices=("c2", "c3", "c4", "c5", "d1", "b3", "p4"), default="c5")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="decode workload only: smaller batch (profiling runs)")

@@ -42,6 +42,7 @@ EXPORTS = (
     "diffattn_fwd_decode_v1",
     "diffattn_fwd_decode_paged",
     "diffattn_selftest_timeout",
+    "diffattn_selftest_exp2",
 )
 
 
@@ -145,6 +146,8 @@ def load_library():
                                               vp, vp, ctypes.c_size_t, vp, vp]
     lib.diffattn_selftest_timeout.restype = i32
     lib.diffattn_selftest_timeout.argtypes = [vp, i32, vp]
+    lib.diffattn_selftest_exp2.restype = i32
+    lib.diffattn_selftest_exp2.argtypes = [vp, vp, vp, i32, vp]
     _lib = lib
     return lib
 
@@ -514,3 +517,16 @@ def diffattn_selftest_timeout(dev_status, timeout_ms=200, stream=None):
     lib = load_library()
     rc = lib.diffattn_selftest_timeout(_ptr(dev_status), int(timeout_ms), _stream(stream))
     _check("diffattn_selftest_timeout", rc)
+
+
+def diffattn_selftest_exp2(x, stream=None):
+    """Evaluate the V2 prefill's FMA-pipe 2^x and CUDA's exp2f over a device float32 tensor
+    `x` (see include/diffattn.h); returns (y, y_ref), device float32 tensors like x."""
+    import torch
+    lib = load_library()
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 tensor")
+    y, y_ref = torch.empty_like(x), torch.empty_like(x)
+    rc = lib.diffattn_selftest_exp2(_ptr(x), _ptr(y), _ptr(y_ref), int(x.numel()), _stream(stream))
+    _check("diffattn_selftest_exp2", rc)
+    return y, y_ref

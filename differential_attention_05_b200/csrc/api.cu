@@ -20,7 +20,8 @@ inline int from_cuda(cudaError_t e) {
   return DIFFATTN_ERR_CUDA;
 }
 
-// Largest element offset reachable through strides s for extents n (all >= 1).
+// The first n strides are non-negative (the kernels address rows as base + index * stride;
+// alignment of the strides is checked separately, where the kernel needs it).
 inline bool strides_ok(const int64_t* s, int n) {
   for (int i = 0; i < n; ++i)
     if (s[i] < 0) return false;

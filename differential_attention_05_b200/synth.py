@@ -119,6 +119,12 @@ def _lambda_vectors(seed, n_units, dim):
     return tuple(_normal(seed, t, (n_units, dim), 0.1) for t in (_T_LQ1, _T_LK1, _T_LQ2, _T_LK2))
 
 
+def lambda_vectors(seed: int, n_units: int, dim: int):
+    """The four lambda vectors (lq1, lk1, lq2, lk2) float32 [n_units, dim] that the workload
+    with this seed uses, drawn without its other tensors."""
+    return _lambda_vectors(seed, n_units, dim)
+
+
 # ---------------------------------------------------------------------------------------
 # The five workloads of the operator (seed = 1000 + index)
 

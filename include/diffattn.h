@@ -27,7 +27,8 @@
  * diffattn_fwd_decode (V2), diffattn_fwd_decode_v1, diffattn_fwd_decode_paged (block
  * table), diffattn_fwd_decode_static, diffattn_decode_workspace_size; diffattn_bwd_prefill,
  * diffattn_bwd_workspace_size, diffattn_lambda_bwd (training); diffattn_selftest_timeout
- * (the bounded-wait path); diffattn_version, diffattn_status_string.
+ * (the bounded-wait path), diffattn_selftest_exp2 (the FMA-pipe 2^x); diffattn_version,
+ * diffattn_status_string.
  *
  * Conventions for every entry point
  *   - Pointers are DEVICE pointers unless marked "host". The caller owns every buffer;
@@ -271,6 +272,10 @@ int diffattn_decode_workspace_size(const diffattn_decode_params* p, size_t* byte
  * query heads of the GQA group (both branches of every pair), keeping one running
  * (max, sum, output) state per query head. A second, small kernel merges the per-split
  * states of each head and applies O = O_1/l_1 - lambda * O_2/l_2 per pair.
+ *   -- "Differential Attention (V2)", "V1 vs V2": V2 keeps the KV heads of the base model
+ *      and its two branches read the same cache, so decoding loads the KV cache once per
+ *      step (V1 loads the value cache twice); The Concept, "The difference idea", for
+ *      O = (A_1 - lambda A_2) V with one query row per step.
  *
  * lambda     : float32 [Hq/2], device
  * workspace  : device buffer of at least diffattn_decode_workspace_size() bytes,
@@ -372,9 +377,14 @@ int diffattn_fwd_decode_paged(const diffattn_decode_params* p, const diffattn_pa
  *     the previous call's contents. Nothing in it needs to start at zero (each call writes
  *     every state it reads), but two calls whose kernels overlap on the GPU (for example
  *     on two streams without ordering between them) race on it: order them.
- *   - The first call made with a given device current looks up the array's device
- *     address (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture. Every GPU that loads the library holds the array until exit.
+ *   - The array's device memory is committed when the library's module for it is loaded
+ *     on a device: under CUDA's default lazy module loading that is the first call of this
+ *     entry point with that device current (with CUDA_MODULE_LOADING=EAGER, when the
+ *     library's context starts); it is then held until the process exits. That first call
+ *     also looks up the array's device address (cudaGetSymbolAddress) and caches it per
+ *     device and context (a context created after a device reset gets a fresh lookup).
+ *     So make one warm-up call on each device at start-up, before sizing a memory pool
+ *     from the free memory that is left and before any stream capture.
  */
 int diffattn_fwd_decode_static(const diffattn_decode_params* p, const void* q,
                                const void* k_cache, const void* v_cache, const int32_t* kv_len,
@@ -399,6 +409,28 @@ int diffattn_fwd_decode_static(const diffattn_decode_params* p, const void* q,
  * reported on the device, when the block finishes).
  */
 int diffattn_selftest_timeout(int* dev_status, int timeout_ms, void* stream);
+
+/*
+ * diffattn_selftest_exp2 -- evaluates the V2 prefill's FMA-pipe 2^x beside CUDA's exp2f.
+ * (A diagnostic of this library, for tests; the pages fix no precision for the
+ * exponentials, only the max-subtracted softmax of "Differential Attention (V2)",
+ * Build It, Step 1, whose terms are 2^x with x <= 0 in the log2 domain.)
+ *
+ * The V2 prefill evaluates a quarter of its exponentials on the FMA pipe instead of the
+ * MUFU unit: x = n + f with n = rint(x) (exact in fp32), 2^f from a degree-4 polynomial
+ * with minimax relative error on [-0.5, 0.5] (a Remez-exchange fit: the error
+ * equioscillates at six points, |error| <= 2.7e-6), then n added to the exponent field;
+ * x is clamped at -125 first, so 2^x for x <= -125 (a masked key, x = -inf) is 2^-125.
+ * This entry point runs that routine, on pairs as the kernel does, over n inputs.
+ *
+ *   x      device float[n], inputs.
+ *   y      device float[n], out: the polynomial 2^x.
+ *   y_ref  device float[n], out: exp2f(x) on the same device.
+ *   n      >= 0 (0 launches nothing).
+ * Returns DIFFATTN_ERR_INVALID_ARG for n < 0 or a null pointer with n > 0,
+ * DIFFATTN_ERR_CUDA if the launch fails, else DIFFATTN_OK (asynchronous on `stream`).
+ */
+int diffattn_selftest_exp2(const float* x, float* y, float* y_ref, int n, void* stream);
 
 #ifdef __cplusplus
 }

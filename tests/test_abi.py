@@ -216,6 +216,15 @@ def test_selftest_timeout_rejects(lib):
     assert f(vp(GOOD), 10001, None) == -1
 
 
+def test_selftest_exp2_rejects(lib):
+    vp = ctypes.c_void_p
+    f = lib.diffattn_selftest_exp2
+    assert f(vp(GOOD), vp(GOOD), vp(GOOD), -1, None) == -1
+    assert f(None, vp(GOOD), vp(GOOD), 8, None) == -1
+    assert f(vp(GOOD), vp(GOOD), None, 8, None) == -1
+    assert f(None, None, None, 0, None) == 0  # nothing to do, nothing launched
+
+
 def _paged(page_size=16, num_pages=64, max_pages=8, strides=(16 * 8 * 128, 8 * 128, 128)):
     pk = B.PagedKV()
     pk.page_size, pk.num_pages, pk.max_pages_per_seq = page_size, num_pages, max_pages

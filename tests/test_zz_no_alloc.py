@@ -35,13 +35,13 @@ def test_rejects_problems_larger_than_the_static_array():
     rc = lib.diffattn_fwd_decode_static(ctypes.byref(p), None, None, None, None, None, None,
                                         None, None)
     assert rc == -4  # DIFFATTN_ERR_WORKSPACE
-    p.batch, p.num_splits = 8, 4096 // 64  # fits unsplit, not with this explicit split count
+    p.batch, p.num_splits = 16, 4096 // 64  # fits unsplit, not with this explicit split count
     p.max_kv_len = 4096
     n = ctypes.c_size_t(0)
     assert lib.diffattn_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 0
-    if n.value > (16 << 20):
-        assert lib.diffattn_fwd_decode_static(ctypes.byref(p), None, None, None, None, None, None,
-                                              None, None) == -4
+    assert n.value > (16 << 20), "the case must exceed the static array to test the rejection"
+    assert lib.diffattn_fwd_decode_static(ctypes.byref(p), None, None, None, None, None, None,
+                                          None, None) == -4
 
 
 @pytest.mark.gpu
@@ -80,3 +80,22 @@ def test_full_size_decode_fits_with_fewer_splits():
     torch.cuda.synchronize()
     max_abs, rel_rms = errors(out_f64(got), out_f64(ref))
     assert max_abs <= BF16_ATOL and rel_rms <= BF16_REL_RMS, (max_abs, rel_rms)
+
+
+@pytest.mark.gpu
+def test_calls_after_the_first_take_no_device_memory():
+    """After one warm-up call (which loads the library's module and so commits the static
+    array), further calls leave the device's free memory unchanged: nothing is allocated,
+    stream-ordered allocations included."""
+    inp = synth.v2_decode(B=4, L=2048, Hq=64, Hkv=8, seed=204)
+    q, k, v = (dev_tensor(getattr(inp, n)) for n in ("q", "k", "v"))
+    lam, _ = lambda_on_device(inp)
+    out = torch.empty((4, 32, 128), dtype=torch.bfloat16, device="cuda")
+    da.diffattn_fwd_decode_static(q, k, v, lam, out=out)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(5):
+        da.diffattn_fwd_decode_static(q, k, v, lam, out=out)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
