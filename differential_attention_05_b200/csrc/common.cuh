@@ -335,6 +335,55 @@ __device__ __forceinline__ void tmem_ld16x2_32f(uint32_t taddr, float* f) {
       : "r"(taddr));
 }
 
+// 16 lanes x 32 bits, twice, with the second half OFF columns further on: with `taddr` at
+// lane L0 (a multiple of 16) and column C, thread t < 16 gets lane L0 + t, columns C .. C+31,
+// and thread t + 16 gets the same lane, columns C+OFF .. C+OFF+31. So the two halves of a
+// warp hold two column ranges of the same 16 rows.
+template <int OFF>
+__device__ __forceinline__ void tmem_ld16x2_32f_split(uint32_t taddr, float* f) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;"
+      : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3]), "=f"(f[4]), "=f"(f[5]), "=f"(f[6]),
+        "=f"(f[7]), "=f"(f[8]), "=f"(f[9]), "=f"(f[10]), "=f"(f[11]), "=f"(f[12]), "=f"(f[13]),
+        "=f"(f[14]), "=f"(f[15]), "=f"(f[16]), "=f"(f[17]), "=f"(f[18]), "=f"(f[19]),
+        "=f"(f[20]), "=f"(f[21]), "=f"(f[22]), "=f"(f[23]), "=f"(f[24]), "=f"(f[25]),
+        "=f"(f[26]), "=f"(f[27]), "=f"(f[28]), "=f"(f[29]), "=f"(f[30]), "=f"(f[31])
+      : "r"(taddr), "n"(OFF));
+}
+
+// the store counterpart of tmem_ld16x2_32f_split: thread t < 16 writes lane L0 + t, columns
+// C .. C+31, thread t + 16 the same lane, columns C+OFF .. C+OFF+31
+template <int OFF>
+__device__ __forceinline__ void tmem_st16x2_32_split(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, "
+      "{%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};" ::"r"(taddr),
+      "n"(OFF), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+      "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+      "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]),
+      "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// tmem_st16x2_32_split from 32 consecutive floats of a register array
+template <int OFF>
+__device__ __forceinline__ void tmem_st16x2_32f_split(uint32_t taddr, const float* f) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, "
+      "{%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+      "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};" ::"r"(taddr),
+      "n"(OFF), "f"(f[0]), "f"(f[1]), "f"(f[2]), "f"(f[3]), "f"(f[4]), "f"(f[5]), "f"(f[6]),
+      "f"(f[7]), "f"(f[8]), "f"(f[9]), "f"(f[10]), "f"(f[11]), "f"(f[12]), "f"(f[13]),
+      "f"(f[14]), "f"(f[15]), "f"(f[16]), "f"(f[17]), "f"(f[18]), "f"(f[19]), "f"(f[20]),
+      "f"(f[21]), "f"(f[22]), "f"(f[23]), "f"(f[24]), "f"(f[25]), "f"(f[26]), "f"(f[27]),
+      "f"(f[28]), "f"(f[29]), "f"(f[30]), "f"(f[31])
+      : "memory");
+}
+
 // 32 lanes x 32 bits, 32 consecutive columns from 32 consecutive floats of a register array
 __device__ __forceinline__ void tmem_st32f(uint32_t taddr, const float* f) {
   asm volatile(

@@ -290,87 +290,111 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
     // --------------------------- softmax warpgroups ------------------------------------
+    // Thread (warp wq, lane) owns query tq = 16 wq + lane % 16 of its sub-tile and half hh =
+    // lane / 16 of the key tile and of the value columns (64 each): it holds BOTH branches'
+    // scores of those keys (the split 16-lane TMEM loads read the branch-1 row, lanes 32 wq
+    // + lane % 16, and the branch-2 row, 16 lanes further on), so p1 - c p2 is formed in
+    // registers. The two halves of a query exchange only their maxima and sums (lane ^ 16).
     const int x = warp >> 2;                       // sub-tile
     const int wq = warp & 3;                       // 32-lane group of TMEM
-    const int h = (lane >> 4) & 1;                 // 0: branch 1, 1: branch 2
+    const int hh = (lane >> 4) & 1;                // half: keys / value columns 64 hh .. 64 hh + 63
     const int tq = wq * 16 + (lane & 15);          // query within the sub-tile
     const int qi = q0 + x * SUB + tq;
     const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
-    const uint32_t s_addr = lane_addr + 256u * x;  // S, then P over its first 64 columns
-    const uint32_t o_addr = s_addr + 128u;         // D (branch-1 lanes) / O_2 (branch 2)
+    const uint32_t s1_addr = lane_addr + 256u * x;  // branch-1 rows: S, then P over 64 columns
+    const uint32_t s2_addr = s1_addr + (16u << 16); // branch-2 rows
+    const uint32_t o1_addr = s1_addr + 128u;        // D (branch-1 rows)
+    const uint32_t o2_addr = s2_addr + 128u;        // O_2 (branch-2 rows)
     const float sl2 = 1.4426950408889634f * rsqrtf((float)a.d);  // log2(e)/sqrt(d)
     const float lam = a.lambda[u];
     // visible keys of this query: vlo .. vis (causal: up to its own position, clamped for
     // the padding rows of the last tile; window: the last `window` of those)
     const int vis = a.causal ? min(qi + off, sr.nk - 1) : sr.nk - 1;
     const int vlo = WINDOW ? max(0, vis - a.window + 1) : 0;
-    float m = -INFINITY, l = 0.f;  // this lane's branch
-    float c = 0.f;                 // identical in both lanes of a query
+    float m1 = -INFINITY, m2 = -INFINITY, l1 = 0.f, l2 = 0.f;  // identical in both halves
+    float c = 0.f;
     bool ok = true;
 
     for (int j = 0; j < n_kt; ++j) {
       if (ok) ok = mbar_wait(&ms.s_full[x], j & 1, abort_flag);
       if (!(ok = __all_sync(FULL, ok))) break;
       tc_fence_after();
-      float p[BN];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) tmem_ld32f(s_addr + 32 * i, p + 32 * i);
+      float p[2 * SUB];  // p[e]: branch 1, key 64 hh + e; p[64 + e]: branch 2, same key
+      tmem_ld16x2_32f_split<64>(s1_addr, p);
+      tmem_ld16x2_32f_split<64>(s1_addr + 32, p + 32);
+      tmem_ld16x2_32f_split<64>(s2_addr, p + 64);
+      tmem_ld16x2_32f_split<64>(s2_addr + 32, p + 96);
       tmem_wait_ld();
-      const int lim = vis - (j_lo + j) * BN, llim = vlo - (j_lo + j) * BN;
-      if (lim < BN - 1 || (WINDOW && llim > 0)) {
+      const int lim = vis - (j_lo + j) * BN - 64 * hh, llim = vlo - (j_lo + j) * BN - 64 * hh;
+      if (lim < 63 || (WINDOW && llim > 0)) {
 #pragma unroll
-        for (int e = 0; e < BN; ++e)
-          if (e > lim || (WINDOW && e < llim)) p[e] = -INFINITY;
+        for (int e = 0; e < 64; ++e)
+          if (e > lim || (WINDOW && e < llim)) p[e] = p[64 + e] = -INFINITY;
       }
-      float c0 = -INFINITY, c1 = -INFINITY, c2 = -INFINITY, c3 = -INFINITY;
+      float u0 = -INFINITY, u1 = -INFINITY, w0 = -INFINITY, w1 = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < BN; e += 8) {
-        c0 = fmax3(c0, p[e + 0], p[e + 1]);
-        c1 = fmax3(c1, p[e + 2], p[e + 3]);
-        c2 = fmax3(c2, p[e + 4], p[e + 5]);
-        c3 = fmax3(c3, p[e + 6], p[e + 7]);
+      for (int e = 0; e < 64; e += 4) {
+        u0 = fmax3(u0, p[e + 0], p[e + 1]);
+        u1 = fmax3(u1, p[e + 2], p[e + 3]);
+        w0 = fmax3(w0, p[64 + e + 0], p[64 + e + 1]);
+        w1 = fmax3(w1, p[64 + e + 2], p[64 + e + 3]);
       }
-      const float t = fmax3(fmaxf(c0, c1), c2, c3) * sl2;
-      // lazy maximum: raised only on growth by more than 2^8 (or when unset)
-      const bool had = WINDOW ? m != -INFINITY : j > 0;  // the query saw a visible key before
-      const bool r = (t > m + RESCALE_LOG2) || !had;
-      const float n = r ? fmaxf(t, m) : m;
-      const float al = (r && had) ? ex2(m - n) : 1.f;
-      m = n;
+      float t1 = fmaxf(u0, u1), t2 = fmaxf(w0, w1);
+      t1 = fmaxf(t1, __shfl_xor_sync(FULL, t1, 16)) * sl2;
+      t2 = fmaxf(t2, __shfl_xor_sync(FULL, t2, 16)) * sl2;
+      // lazy maxima: raised only on growth by more than 2^8 (or when unset)
+      const bool had = WINDOW ? m1 != -INFINITY : j > 0;  // the query saw a visible key before
+      const bool r1 = (t1 > m1 + RESCALE_LOG2) || !had, r2 = (t2 > m2 + RESCALE_LOG2) || !had;
+      const float n1 = r1 ? fmaxf(t1, m1) : m1, n2 = r2 ? fmaxf(t2, m2) : m2;
+      const float a1 = (r1 && had) ? ex2(m1 - n1) : 1.f, a2 = (r2 && had) ? ex2(m2 - n2) : 1.f;
+      m1 = n1;
+      m2 = n2;
       // p = 2^(s sl2 - m), in place (0 for every key while the query has none visible); in
       // every group of 8 keys the last POLY_PAIRS pairs go to the FMA pipe, the rest to MUFU
+      const float nm1 = (WINDOW && m1 == -INFINITY) ? 0.f : -m1;
+      const float nm2 = (WINDOW && m2 == -INFINITY) ? 0.f : -m2;
       float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
-      const float nm = (WINDOW && m == -INFINITY) ? 0.f : -m;
 #pragma unroll
-      for (int e = 0; e < BN; e += 8) {
-        float xv[8];
+      for (int e = 0; e < 64; e += 8) {
 #pragma unroll
-        for (int i = 0; i < 8; i += 2) ffma2(xv[i], xv[i + 1], p[e + i], p[e + i + 1], sl2, sl2, nm, nm);
+        for (int br = 0; br < 2; ++br) {
+          float* pb = p + 64 * br + e;
+          const float nm = br ? nm2 : nm1;
+          float xv[8];
 #pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-          if (i >= 8 - 2 * POLY_PAIRS) {
-            exp2_fma2(p[e + i], p[e + i + 1], xv[i], xv[i + 1]);
+          for (int i = 0; i < 8; i += 2) ffma2(xv[i], xv[i + 1], pb[i], pb[i + 1], sl2, sl2, nm, nm);
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            if (i >= 8 - 2 * POLY_PAIRS) {
+              exp2_fma2(pb[i], pb[i + 1], xv[i], xv[i + 1]);
+            } else {
+              pb[i] = ex2(xv[i]);
+              pb[i + 1] = ex2(xv[i + 1]);
+            }
+          }
+          if (br == 0) {
+            fadd2(sa, sb, sa, sb, pb[0], pb[1]);
+            fadd2(sa, sb, sa, sb, pb[2], pb[3]);
+            fadd2(sa, sb, sa, sb, pb[4], pb[5]);
+            fadd2(sa, sb, sa, sb, pb[6], pb[7]);
           } else {
-            p[e + i] = ex2(xv[i]);
-            p[e + i + 1] = ex2(xv[i + 1]);
+            fadd2(sc, sd, sc, sd, pb[0], pb[1]);
+            fadd2(sc, sd, sc, sd, pb[2], pb[3]);
+            fadd2(sc, sd, sc, sd, pb[4], pb[5]);
+            fadd2(sc, sd, sc, sd, pb[6], pb[7]);
           }
         }
-        fadd2(sa, sb, sa, sb, p[e], p[e + 1]);
-        fadd2(sc, sd, sc, sd, p[e + 2], p[e + 3]);
-        fadd2(sa, sb, sa, sb, p[e + 4], p[e + 5]);
-        fadd2(sc, sd, sc, sd, p[e + 6], p[e + 7]);
       }
-      l = l * al + ((sa + sb) + (sc + sd));
+      // tile sums over both halves: a + b is the same float in either order, so both halves
+      // of the query keep bit-identical l_1, l_2 (and so take the same decisions below)
+      const float s1h = sa + sb, s2h = sc + sd;
+      l1 = l1 * a1 + (s1h + __shfl_xor_sync(FULL, s1h, 16));
+      l2 = l2 * a2 + (s2h + __shfl_xor_sync(FULL, s2h, 16));
 
-      // the query's two branches: this lane and lane ^ 16
-      const float al_o = __shfl_xor_sync(FULL, al, 16);
-      const float l_o = __shfl_xor_sync(FULL, l, 16);
-      const float a1 = h ? al_o : al, a2 = h ? al : al_o;
-      const float l1 = h ? l_o : l, l2 = h ? l : l_o;
       // target c = lambda l_1 / l_2 (sums including this tile); under max updates c follows
       // c a_1 / a_2, which leaves D unchanged; reset to the target when it leaves
       // [0.8, 1.25] times it (the query's first tile with a visible key always takes the
-      // target: D and O_2 are still 0). Both lanes compute the same.
+      // target: D and O_2 are still 0).
       const float cst = (WINDOW && !(l2 > 0.f)) ? lam : lam * __fdiv_rn(l1, l2);  // exact ratio: identical branches give c = lambda
       float cn = cst, kc = 0.f;
       bool need = false;
@@ -380,52 +404,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool reset = !(ra >= 0.8f * rt && ra <= 1.25f * rt);
         cn = reset ? cst : cev;
         if (reset) kc = __fsub_rn(__fmul_rn(a1, c), __fmul_rn(a2, cn));
-        need = (al != 1.f) || (kc != 0.f);
-      }
-      if (WINDOW || j > 0) {
-        // the whole warp rescales (a query with nothing to do has al = 1, kc = 0)
-        if (__any_sync(FULL, need)) {
-          // D <- a_1 D + kc O_2, O_2 <- a_2 O_2 over all 128 value columns. The score MMA
-          // that filled S was issued after this sub-tile's previous P.V MMAs, so its
-          // completion implies theirs.
-          const float kx = h ? 0.f : kc;
-#pragma unroll 1
-          for (int ch = 0; ch < 4; ++ch) {
-            float ov[32];
-            tmem_ld32f(o_addr + ch * 32, ov);
-            tmem_wait_ld();
-            uint32_t ro[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float other = __shfl_xor_sync(FULL, ov[e], 16);
-              ro[e] = __float_as_uint(fmaf(kx, other, al * ov[e]));
-            }
-            tmem_st32(o_addr + ch * 32, ro);
-          }
-        }
+        need = (a1 != 1.f) || (a2 != 1.f) || (kc != 0.f);
       }
       c = cn;
-      // P row: branch 1 writes p1 - c p2, branch 2 writes p2. Every lane first puts its p
-      // (fp32) over its own score columns; the 16-lane paired load then hands lanes 0-15 the
-      // row of lane + 16 (branch 2 of the same query) and lanes 16-31 their own row.
+      // P rows (bf16 pairs over the first 64 columns of the S block): branch 1 p1 - c p2,
+      // branch 2 p2; this half's 64 keys are columns 32 hh .. 32 hh + 31. Every column
+      // written here was read by this warp's loads above, which have completed.
+      {
+        const float nc = -c;
+        uint32_t pk1[32], pk2[32];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_st32f(s_addr + ch * 32, p + ch * 32);
-      tmem_wait_st();
-      const float nc = h ? 0.f : -c;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        float q2[32];
-        tmem_ld16x2_32f(s_addr + (16u << 16) + ch * 32, q2);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float w0, w1;
-          ffma2(w0, w1, q2[e], q2[e + 1], nc, nc, p[ch * 32 + e], p[ch * 32 + e + 1]);
-          pk[e / 2] = pack_bf16(w0, w1);
+        for (int e = 0; e < 64; e += 2) {
+          float v0, v1;
+          ffma2(v0, v1, p[64 + e], p[64 + e + 1], nc, nc, p[e], p[e + 1]);
+          pk1[e / 2] = pack_bf16(v0, v1);
+          pk2[e / 2] = pack_bf16(p[64 + e], p[64 + e + 1]);
         }
-        // bf16 pairs land on columns 16 ch .. 16 ch + 15, all read already
-        tmem_st16(s_addr + ch * 16, pk);
+        tmem_st16x2_32_split<32>(s1_addr, pk1);
+        tmem_st16x2_32_split<32>(s2_addr, pk2);
+      }
+      if (WINDOW || j > 0) {
+        // the whole warp rescales (a query with nothing to do has a_1 = a_2 = 1, kc = 0):
+        // D <- a_1 D + kc O_2, O_2 <- a_2 O_2 over this half's 64 value columns. The score
+        // MMA that filled S was issued after this sub-tile's previous P.V MMAs, so its
+        // completion implies theirs; the next P.V MMA waits for p_full below.
+        if (__any_sync(FULL, need)) {
+#pragma unroll 1
+          for (int ch = 0; ch < 2; ++ch) {
+            float dv[32], ov[32];
+            tmem_ld16x2_32f_split<64>(o1_addr + ch * 32, dv);
+            tmem_ld16x2_32f_split<64>(o2_addr + ch * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              dv[e] = fmaf(kc, ov[e], a1 * dv[e]);
+              ov[e] *= a2;
+            }
+            tmem_st16x2_32f_split<64>(o1_addr + ch * 32, dv);
+            tmem_st16x2_32f_split<64>(o2_addr + ch * 32, ov);
+          }
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -435,21 +453,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------- epilogue ----------------------------------------
     if (ok) ok = mbar_wait(&ms.o_full[x], 0, abort_flag);
     ok = __all_sync(FULL, ok);
-    const float l_o = __shfl_xor_sync(FULL, l, 16);
-    const float L1 = h ? l_o : l, L2 = h ? l : l_o;
-    const float inv1 = 1.f / L1, inv2 = 1.f / L2;
+    const float inv1 = 1.f / l1, inv2 = 1.f / l2;
     // o = D / l_1 + O_2 (c / l_1 - lambda / l_2); products rounded on their own so that
     // identical branches with lambda = 1 give exactly 0
     const float coef = __fsub_rn(__fmul_rn(c, inv1), __fmul_rn(lam, inv2));
-    // this lane writes value columns 64 h .. 64 h + 63 of its query; D and O_2 of a column
-    // sit in the two lanes of the query
+    // this thread writes value columns 64 hh .. 64 hh + 63 of its query
     float y[64];  // the output, or (STATS) the incoming gradient dy of the same columns
     float e1 = 0.f, e2 = 0.f;
     if constexpr (STATS) {
       if (ok && qi < a.N) {
         const uint4* g4 = reinterpret_cast<const uint4*>(
             static_cast<const __nv_bfloat16*>(a.st_dy) + (int64_t)b * a.st_dys[0] +
-            (int64_t)qi * a.st_dys[1] + (int64_t)u * a.st_dys[2] + h * 64);
+            (int64_t)qi * a.st_dys[1] + (int64_t)u * a.st_dys[2] + hh * 64);
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
           const uint4 w = g4[v];
@@ -470,34 +485,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float c1 = c * inv1;
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
-        float v0[32], v1[32];
-        tmem_ld32f(o_addr + ch * 32, v0);
-        tmem_ld32f(o_addr + 64 + ch * 32, v1);
+        float dv[32], ov[32];
+        tmem_ld16x2_32f_split<64>(o1_addr + ch * 32, dv);
+        tmem_ld16x2_32f_split<64>(o2_addr + ch * 32, ov);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float mine = h ? v1[e] : v0[e];
-          const float other = __shfl_xor_sync(FULL, h ? v0[e] : v1[e], 16);
-          const float dv = h ? other : mine, ov = h ? mine : other;
           if constexpr (STATS) {
             // O_1 / l_1 = (D + c O_2) / l_1 and O_2 / l_2 at this column, against dy
-            e1 = fmaf(y[ch * 32 + e], __fmaf_rn(ov, c1, dv * inv1), e1);
-            e2 = fmaf(y[ch * 32 + e], ov * inv2, e2);
+            e1 = fmaf(y[ch * 32 + e], __fmaf_rn(ov[e], c1, dv[e] * inv1), e1);
+            e2 = fmaf(y[ch * 32 + e], ov[e] * inv2, e2);
           } else {
-            y[ch * 32 + e] = __fmaf_rn(ov, coef, __fmul_rn(dv, inv1));
+            y[ch * 32 + e] = __fmaf_rn(ov[e], coef, __fmul_rn(dv[e], inv1));
           }
         }
       }
     }
     if constexpr (STATS) {
-      // the query's two lanes add their column halves; lse_b = m_b + log2 l_b (log2 domain)
+      // the query's two halves add their column ranges; lse_b = m_b + log2 l_b (log2 domain)
       e1 += __shfl_xor_sync(FULL, e1, 16);
       e2 += __shfl_xor_sync(FULL, e2, 16);
-      const float lse_own = m + log2f(l);
-      const float lse_oth = __shfl_xor_sync(FULL, lse_own, 16);
-      if (ok && h == 0 && qi < a.N) {
+      if (ok && hh == 0 && qi < a.N) {
         const int64_t r = ((int64_t)b * a.units + u) * a.st_rows + qi;
-        *reinterpret_cast<float4*>(a.st + r * 4) = make_float4(lse_own, lse_oth, e1, e2);
+        *reinterpret_cast<float4*>(a.st + r * 4) =
+            make_float4(m1 + log2f(l1), m2 + log2f(l2), e1, e2);
         a.st_dl[((int64_t)b * a.units + u) * a.N + qi] = -e2;
       }
     }
@@ -507,7 +518,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int o_q0 = VARLEN ? ms.seq_q0 : 0;
     if (!STATS && ok && qi < o_nq) {
       __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)o_b * a.os[0] +
-                          (int64_t)(o_q0 + qi) * a.os[1] + (int64_t)u * a.os[2] + h * 64;
+                          (int64_t)(o_q0 + qi) * a.os[1] + (int64_t)u * a.os[2] + hh * 64;
       uint4* o4 = reinterpret_cast<uint4*>(ob);
 #pragma unroll
       for (int v = 0; v < 8; ++v) {
