@@ -28,8 +28,9 @@
 // kernel) also writes the gradient reaching O through the per-head norm, in bf16, which the
 // kernels read in place of dy.
 // No atomics: every dK/dV row and every dQ row is summed inside one CTA in a fixed order.
-// Warps 0-3 form the per-row arithmetic, warp 4 issues the TMA loads (128-byte swizzle, no
-// multicast) and the 1-D bulk copy of the statistics, warp 5 owns TMEM and every MMA.
+// Warps 0-15 (four warpgroups, each taking a quarter of a step's columns) form the per-row
+// arithmetic, warp 16 issues the TMA loads (128-byte swizzle, no multicast) and the 1-D bulk
+// copy of the statistics, warp 17 owns TMEM and every MMA.
 // Every mbarrier wait is bounded as in the forward kernels.
 #include "common.cuh"
 #include "kernels.h"
@@ -43,7 +44,12 @@ namespace {
 constexpr int BLK = 128 * 128;   // [128 rows x 64 bf16] 128-byte-swizzled block (16 KB)
 constexpr int HBLK = 64 * 128;   // [64 rows x 64 bf16] (8 KB)
 constexpr unsigned FULL = 0xffffffffu;
-constexpr int NUM_THREADS = 192;
+// warps 0 .. 4 RW - 1: RW warpgroups of per-row arithmetic, each taking a quarter of a step's
+// columns (so four warps share every TMEM lane quarter and hide each other's latency); then
+// the TMA warp and the MMA warp
+constexpr int RW = 4;
+constexpr int NUM_THREADS = 128 * RW + 64;
+constexpr int W_TMA = 4 * RW, W_MMA = 4 * RW + 1;
 constexpr int TMEM_COLS = 512;
 
 struct BwdMaps {
@@ -126,12 +132,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&ms.q_empty[s], 1);
     }
     mbar_init(&ms.s_full, 1);
-    mbar_init(&ms.p_full, 128);
+    mbar_init(&ms.p_full, 128 * RW);
     mbar_init(&ms.o_full, 1);
     ms.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == W_MMA) {
     tmem_alloc(&ms.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
@@ -151,7 +157,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = &ms.abort;
   const int rows = a.N + 64;  // statistics rows per (batch entry, pair)
 
-  if (warp == 4) {
+  if (warp == W_TMA) {
     if (lane == 0) {
       // ------------------------------ TMA producer -----------------------------------
       tma_prefetch_desc(&maps.q);
@@ -191,7 +197,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mbar_wait_drain(&ms.q_full[t % STAGES], (t / STAGES) & 1);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == W_MMA) {
     if (lane == 0) {
       // ------------------------------ MMA issuer -------------------------------------
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
@@ -223,7 +229,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint64_t qmn = sw128_desc(st + QS, BLK, 1024);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_ts(tmem + C_DV, tmem + C_PC + kk * 8, desc_at(dmn, kk * 2048), IDESC_ACC,
+          umma_ts(tmem + C_DV, tmem + C_PC + kk * 16, desc_at(dmn, kk * 2048), IDESC_ACC,
                   (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -253,9 +259,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_commit(&ms.o_full);
     }
   } else {
-    // ------------------------- per-key arithmetic (warps 0-3) -------------------------
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    const int j = k0 + (int)threadIdx.x;  // this thread's key (TMEM lane)
+    // ------------------------- per-key arithmetic (warps 0 .. 4 RW - 1) --------------
+    // warpgroup wgr takes queries 16 wgr .. 16 wgr + 15 of every 64-query step
+    static_assert(RW == 4, "one 16-query chunk per row warpgroup");
+    const int wgr = warp >> 2;
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const int j = k0 + (warp & 3) * 32 + lane;  // this thread's key (TMEM lane)
     const float sl2 = 1.4426950408889634f * rsqrtf((float)a.d);
     bool ok = true;
     for (int t = 0; t < n_steps; ++t) {
@@ -269,19 +278,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float4* sts = reinterpret_cast<const float4*>(smem + STAGE_OFF + s * STAGE_BYTES + STS);
       // inside the visible region (most steps of a causal problem) no pair needs a mask
       const bool full = tile_visible(a, q0, QT, k0, KT);
-      auto chunk = [&](int c, auto all_visible) {
-        float s1[32], s2[32], dp[32];
-        tmem_ld32f(lane_addr + C_S + 32 * c, s1);
-        tmem_ld32f(lane_addr + C_S + 64 + 32 * c, s2);
-        tmem_ld32f(lane_addr + C_DP + 32 * c, dp);
+      auto chunk = [&](auto all_visible) {
+        const int c = wgr;
+        float s1[16], s2[16], dp[16];
+        tmem_ld16f(lane_addr + C_S + 16 * c, s1);
+        tmem_ld16f(lane_addr + C_S + 64 + 16 * c, s2);
+        tmem_ld16f(lane_addr + C_DP + 16 * c, dp);
         tmem_wait_ld();
-        uint32_t pc[16], d1[16], d2[16];
+        uint32_t pc[8], d1[8], d2[8];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
+        for (int e = 0; e < 16; e += 2) {
           float vpc[2], vd1[2], vd2[2];
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
-            const int qq = 32 * c + e + x;
+            const int qq = 16 * c + e + x;
             const float4 st = sts[qq];
             const bool vis = decltype(all_visible)::value || visible(a, q0 + qq, j);
             const float p1 = vis ? ex2(s1[e + x] * sl2 - st.x) : 0.f;
@@ -294,16 +304,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           d1[e / 2] = pack_bf16(vd1[0], vd1[1]);
           d2[e / 2] = pack_bf16(vd2[0], vd2[1]);
         }
-        // chunk c's bf16 columns lie below the dP columns still to be read
-        tmem_st16(lane_addr + C_PC + 16 * c, pc);
-        tmem_st16(lane_addr + C_DS + 16 * c, d1);
-        tmem_st16(lane_addr + C_DS + 32 + 16 * c, d2);
+        // P_1 - lambda P_2 over this chunk's own dP columns (read above, by this warp only);
+        // dS_1, dS_2 into their 8-column slots of the dS block
+        tmem_st8(lane_addr + C_PC + 16 * c, pc);
+        tmem_st8(lane_addr + C_DS + 8 * c, d1);
+        tmem_st8(lane_addr + C_DS + 32 + 8 * c, d2);
       };
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        if (full) chunk(c, std::true_type{});
-        else chunk(c, std::false_type{});
-      }
+      if (full) chunk(std::true_type{});
+      else chunk(std::false_type{});
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&ms.p_full);
@@ -319,32 +327,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int64_t row = ((int64_t)b * a.Nk + (store ? j : 0)) * a.Hkv + gk;
       float4* dv4 = reinterpret_cast<float4*>(g.dv + row * 128);
       float4* dk4 = reinterpret_cast<float4*>(g.dk + row * 128);
+      const int c = wgr;  // this warpgroup's 32 columns of dV and dK
       if (n_steps > 0) {
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float x[32], y[32];
-          tmem_ld32f(lane_addr + C_DV + 32 * c, x);
-          tmem_ld32f(lane_addr + C_DK + 32 * c, y);
-          tmem_wait_ld();
-          if (store) {
+        float x[32], y[32];
+        tmem_ld32f(lane_addr + C_DV + 32 * c, x);
+        tmem_ld32f(lane_addr + C_DK + 32 * c, y);
+        tmem_wait_ld();
+        if (store) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              dv4[(32 * c + e) / 4] = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
-              dk4[(32 * c + e) / 4] = make_float4(y[e] * scale, y[e + 1] * scale,
-                                                  y[e + 2] * scale, y[e + 3] * scale);
-            }
+          for (int e = 0; e < 32; e += 4) {
+            dv4[(32 * c + e) / 4] = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+            dk4[(32 * c + e) / 4] = make_float4(y[e] * scale, y[e + 1] * scale,
+                                                y[e + 2] * scale, y[e + 3] * scale);
           }
         }
       } else if (store) {
-        for (int e = 0; e < 32; ++e) dv4[e] = dk4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int e = 0; e < 8; ++e) dv4[8 * c + e] = dk4[8 * c + e] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == W_MMA) {
     if (*abort_flag) {
       mbar_wait_drain(&ms.o_full, 0);
       if (lane == 0) report_status(a.dev_status, DIFFATTN_ERR_TIMEOUT);
@@ -408,12 +414,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&ms.kv_empty[s], 1);
     }
     mbar_init(&ms.s_full, 1);
-    mbar_init(&ms.p_full, 128);
+    mbar_init(&ms.p_full, 128 * RW);
     mbar_init(&ms.o_full, 1);
     ms.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == W_MMA) {
     tmem_alloc(&ms.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
@@ -432,7 +438,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = &ms.abort;
   const int rows = a.N + 64;
 
-  if (warp == 4) {
+  if (warp == W_TMA) {
     if (lane == 0) {
       tma_prefetch_desc(&maps.q);
       tma_prefetch_desc(&maps.k);
@@ -470,7 +476,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mbar_wait_drain(&ms.kv_full[t % STAGES], (t / STAGES) & 1);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == W_MMA) {
     if (lane == 0) {
       constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, false, true);
@@ -522,11 +528,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_commit(&ms.o_full);
     }
   } else {
-    // ----------------------- per-(query, branch) arithmetic (warps 0-3) ------------------
-    // row r: branch r / 64 of query q0 + r % 64 (rows 0-63 Q_1, 64-127 Q_2)
-    const int r = (int)threadIdx.x, br = r >> 6;
+    // ------------- per-(query, branch) arithmetic (warps 0 .. 4 RW - 1) ---------------
+    // row r (TMEM lane): branch r / 64 of query q0 + r % 64 (rows 0-63 Q_1, 64-127 Q_2);
+    // warpgroup wgr takes keys 32 wgr .. 32 wgr + 31 of every 128-key step
+    static_assert(RW == 4, "one 32-key chunk per row warpgroup");
+    const int wgr = warp >> 2;
+    const int r = (warp & 3) * 32 + lane, br = r >> 6;
     const int qi = q0 + (r & 63);
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sl2 = 1.4426950408889634f * rsqrtf((float)a.d);
     const float lam = a.lambda[u];
     bool ok = mbar_wait(&ms.q_full, 0, abort_flag);
@@ -557,11 +566,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tmem_st16(lane_addr + C_DS + 16 * c, ds);
       };
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        if (full) chunk(c, std::true_type{});
-        else chunk(c, std::false_type{});
-      }
+      if (full) chunk(wgr, std::true_type{});
+      else chunk(wgr, std::false_type{});
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&ms.p_full);
@@ -579,10 +585,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           V1 ? g.dq + (qrow * a.units + u) * 128 + 64 * br : g.dq + (qrow * a.Hq + 2 * u + br) * 128);
       const int n_ch = V1 ? 2 : 4;
       const uint32_t col0 = C_DQ + (V1 ? 64u * br : 0u);  // warp-uniform: br is per warp
-      if (n_kt > 0) {
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < n_ch; ++c) {
+      const int c = wgr;  // this warpgroup's 32 columns (warp-uniform)
+      if (c < n_ch) {
+        if (n_kt > 0) {
+          tc_fence_after();
           float x[32];
           tmem_ld32f(lane_addr + col0 + 32 * c, x);
           tmem_wait_ld();
@@ -592,16 +598,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               dq4[(32 * c + e) / 4] = make_float4(x[e] * scale, x[e + 1] * scale,
                                                   x[e + 2] * scale, x[e + 3] * scale);
           }
+        } else if (store) {
+          for (int e = 0; e < 8; ++e) dq4[8 * c + e] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-      } else if (store) {
-        for (int e = 0; e < 8 * n_ch; ++e) dq4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == W_MMA) {
     if (*abort_flag) {
       mbar_wait_drain(&ms.o_full, 0);
       if (lane == 0) report_status(a.dev_status, DIFFATTN_ERR_TIMEOUT);

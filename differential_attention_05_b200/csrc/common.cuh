@@ -319,6 +319,25 @@ __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float* f) {
       : "r"(taddr));
 }
 
+// 32 lanes x 32 bits, 16 consecutive columns, into 16 consecutive floats
+__device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float* f) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3]), "=f"(f[4]), "=f"(f[5]), "=f"(f[6]),
+        "=f"(f[7]), "=f"(f[8]), "=f"(f[9]), "=f"(f[10]), "=f"(f[11]), "=f"(f[12]), "=f"(f[13]),
+        "=f"(f[14]), "=f"(f[15])
+      : "r"(taddr));
+}
+
+// 32 lanes x 32 bits, 8 consecutive columns from 8 registers
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 // 16 lanes x 32 bits, twice, 32 consecutive columns: with `taddr` at lane L0 (a multiple of
 // 16), threads t and t + 16 of the warp both get lane L0 + t, columns col .. col+31 (the
 // second half's column offset is 0). Lets lanes 0-15 of a 32-lane group read lanes 16-31.
