@@ -74,6 +74,7 @@ constexpr int REGS_SOFTMAX = 200, REGS_OTHER = 104;
 constexpr int TMEM_COLS = 512;
 constexpr float RESCALE_LOG2 = 8.0f;
 constexpr int POLY_PAIRS = 1;          // of every 4 pairs of exponentials, on the FMA pipe
+constexpr int QBAND = 32;              // query tiles per band of the CTA order
 
 struct Misc {
   uint64_t q_full[2];
@@ -115,12 +116,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   Misc& ms = *reinterpret_cast<Misc*>(smem + MISC_OFF);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // tile -> (q-tile, unit, batch); the largest causal tiles are handed out first
+  // tile -> (q-tile, unit, batch). The query tiles go in bands of QBAND, the heaviest
+  // causal band first; inside a band, KV group by KV group (batch entry, KV head), each
+  // group's tiles heaviest first and the pairs of a tile together. So the CTAs in flight
+  // read the keys and values of one or two KV heads, which stay in L2, and the tiles that
+  // are handed out last are the lightest.
   const int n_qt = (a.N + BM - 1) / BM;
-  const int per_qt = a.units * a.B;
-  const int qt = a.causal ? (n_qt - 1 - (int)(blockIdx.x / per_qt)) : (int)(blockIdx.x / per_qt);
-  const int u = (int)(blockIdx.x % per_qt) % a.units;
-  const int b = (int)(blockIdx.x % per_qt) / a.units;
+  const int ppg = a.group / 2;                    // pairs per KV head
+  const int n_kvh = a.units / ppg;
+  const int per_band = QBAND * ppg * n_kvh * a.B;
+  const int band = (int)(blockIdx.x / per_band);
+  const int r_b = (int)(blockIdx.x - (unsigned)band * per_band);
+  const int band_len = min(QBAND, n_qt - QBAND * band);
+  const int grp = r_b / (band_len * ppg), r_g = r_b - grp * (band_len * ppg);
+  const int qt_i = QBAND * band + r_g / ppg;
+  const int qt = a.causal ? n_qt - 1 - qt_i : qt_i;
+  const int u = (grp % n_kvh) * ppg + r_g % ppg;
+  const int b = grp / n_kvh;
   const int q0 = qt * BM;
   // the sequence of this tile (a variable-length batch packs several into one tensor);
   // the whole CTA leaves before any setup when the tile lies past its sequence

@@ -88,3 +88,34 @@ def test_every_row_sees_a_key():
         if W and not causal:
             continue
         assert visible(N, Nk, causal, W).any(axis=1).all()
+
+
+def v2_cta_tile(idx, n_qt, units, group, B, causal, QBAND=32):
+    """The V2 prefill's CTA order, restated: bands of QBAND query tiles (heaviest first
+    when causal), then (batch entry, KV head) groups, then the band's tiles, then the pairs
+    of a tile. Returns (query tile, pair, batch entry)."""
+    ppg = group // 2
+    n_kvh = units // ppg
+    per_band = QBAND * ppg * n_kvh * B
+    band = idx // per_band
+    r_b = idx - band * per_band
+    band_len = min(QBAND, n_qt - QBAND * band)
+    grp = r_b // (band_len * ppg)
+    r_g = r_b - grp * (band_len * ppg)
+    qt_i = QBAND * band + r_g // ppg
+    return (n_qt - 1 - qt_i if causal else qt_i), (grp % n_kvh) * ppg + r_g % ppg, grp // n_kvh
+
+
+def test_v2_cta_order_covers_every_tile_once():
+    """The grid has n_qt * units * B CTAs; the order must hand out each (query tile, pair,
+    batch entry) exactly once, bands of partial length included, and keep the pairs of a
+    CTA's KV head together."""
+    for n_qt, Hq, Hkv, B in ((512, 64, 8, 1), (128, 64, 8, 1), (3, 16, 2, 2), (1, 8, 4, 3),
+                             (33, 4, 2, 1), (65, 32, 2, 2), (7, 64, 2, 1), (64, 8, 1, 2)):
+        units, group = Hq // 2, Hq // Hkv
+        for causal in (True, False):
+            got = [v2_cta_tile(i, n_qt, units, group, B, causal) for i in range(n_qt * units * B)]
+            assert len(set(got)) == len(got) == n_qt * units * B
+            assert all(0 <= t < n_qt and 0 <= u < units and 0 <= b < B for t, u, b in got)
+            if causal:  # the last CTAs take the lightest band
+                assert max(t for t, _, _ in got[-units * B:]) < 32
