@@ -90,6 +90,7 @@ constexpr int SMEM_BYTES = MISC_OFF + 1024 + 1024;
 constexpr int C_S = 0, C_DP = 128, C_PC = 128, C_DS = 192, C_DV = 256, C_DK = 384;
 struct Misc {
   uint64_t kv_full, q_full[STAGES], q_empty[STAGES], s_full, p_full, o_full;
+  uint64_t s_read;  // every row thread has read the step's S^T and dP^T columns
   uint32_t tmem_base;
   int abort;
 };
@@ -134,6 +135,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&ms.s_full, 1);
     mbar_init(&ms.p_full, 128 * RW);
     mbar_init(&ms.o_full, 1);
+    mbar_init(&ms.s_read, 128 * RW);
     ms.abort = 0;
     fence_barrier_init();
   }
@@ -205,15 +207,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t IDESC_ACC = idesc_bf16_f32(128, 128, false, true);
       const uint64_t kdesc = sw128_desc(smem_u32(smem + K_OFF), 16, 1024);
       const uint64_t vdesc = sw128_desc(smem_u32(smem + V_OFF), 16, 1024);
-      auto issue_s_dp = [&](int t) {
+      // S^T of step t (both branches stacked, N = 128) into columns 0..127
+      auto issue_st = [&](int t) {
         const uint32_t st = smem_u32(smem + STAGE_OFF + (t % STAGES) * STAGE_BYTES);
         const uint64_t qd = sw128_desc(st + QS, 16, 1024);
-        const uint64_t dd = sw128_desc(st + DO, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t o = (kk >> 2) * BLK + (kk & 3) * 32;
           umma_ss(tmem + C_S, desc_at(kdesc, o), desc_at(qd, o), IDESC_S, kk > 0);
         }
+      };
+      // dP^T of step t (N = 64) into columns 128..191, then the step is complete
+      auto issue_dp = [&](int t) {
+        const uint32_t st = smem_u32(smem + STAGE_OFF + (t % STAGES) * STAGE_BYTES);
+        const uint64_t dd = sw128_desc(st + DO, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t o = (kk >> 2) * BLK + (kk & 3) * 32;
@@ -237,23 +244,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&ms.q_empty[t % STAGES]);
       };
+      // Per step t: S^T(t+1) as soon as the row threads have read step t's columns (it
+      // overwrites only S^T), then dV, dK of step t once their operands are written, then
+      // dP^T(t+1) (its columns held P_1 - lambda P_2 of step t, which dV has read: the
+      // tensor core runs these in order).
       bool ok = mbar_wait(&ms.kv_full, 0, abort_flag);
       if (ok && n_steps > 0) {
         ok = mbar_wait(&ms.q_full[0], 0, abort_flag);
         if (ok) {
           tc_fence_after();
-          issue_s_dp(0);
+          issue_st(0);
+          issue_dp(0);
         }
       }
       for (int t = 0; t < n_steps && ok; ++t) {
+        const bool more = t + 1 < n_steps;
+        if (more) {
+          if (!(ok = mbar_wait(&ms.s_read, t & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(&ms.q_full[(t + 1) % STAGES], ((t + 1) / STAGES) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_st(t + 1);
+        }
         if (!(ok = mbar_wait(&ms.p_full, t & 1, abort_flag))) break;
         tc_fence_after();
         issue_dv_dk(t);
-        if (t + 1 < n_steps) {
-          if (!(ok = mbar_wait(&ms.q_full[(t + 1) % STAGES], ((t + 1) / STAGES) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_s_dp(t + 1);
-        }
+        if (more) issue_dp(t + 1);
       }
       // arrives once every MMA issued above has completed (also on an abort)
       tc_commit(&ms.o_full);
@@ -285,6 +300,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld16f(lane_addr + C_S + 64 + 16 * c, s2);
         tmem_ld16f(lane_addr + C_DP + 16 * c, dp);
         tmem_wait_ld();
+        // the next step's S^T may now overwrite columns 0..127
+        tc_fence_before();
+        mbar_arrive(&ms.s_read);
         uint32_t pc[8], d1[8], d2[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
@@ -375,6 +393,8 @@ constexpr int SMEM_BYTES = MISC_OFF + 1024 + 1024;
 constexpr int C_S = 0, C_DP = 128, C_DQ = 256, C_DS = 384;
 struct Misc {
   uint64_t q_full, kv_full[STAGES], kv_empty[STAGES], s_full, p_full, o_full;
+  uint64_t s_read;   // every row thread has read the step's S and dP columns
+  uint64_t dq_done;  // the dQ MMAs of a step have completed (they read its dS)
   uint32_t tmem_base;
   int abort;
 };
@@ -416,6 +436,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(&ms.s_full, 1);
     mbar_init(&ms.p_full, 128 * RW);
     mbar_init(&ms.o_full, 1);
+    mbar_init(&ms.s_read, 128 * RW);
+    mbar_init(&ms.dq_done, 1);
     ms.abort = 0;
     fence_barrier_init();
   }
@@ -505,6 +527,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tmem + C_DQ, tmem + C_DS + kk * 8, desc_at(kmn, kk * 2048), IDESC_ACC,
                   (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&ms.dq_done);
         tc_commit(&ms.kv_empty[t % STAGES]);
       };
       bool ok = mbar_wait(&ms.q_full, 0, abort_flag);
@@ -515,15 +538,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           issue_s_dp(0);
         }
       }
+      // Per step t: S, dP of step t+1 as soon as the row threads have read step t's (into
+      // the same columns), then dQ of step t once its dS is written.
       for (int t = 0; t < n_kt && ok; ++t) {
-        if (!(ok = mbar_wait(&ms.p_full, t & 1, abort_flag))) break;
-        tc_fence_after();
-        issue_dq(t);
         if (t + 1 < n_kt) {
+          if (!(ok = mbar_wait(&ms.s_read, t & 1, abort_flag))) break;
           if (!(ok = mbar_wait(&ms.kv_full[(t + 1) % STAGES], ((t + 1) / STAGES) & 1, abort_flag))) break;
           tc_fence_after();
           issue_s_dp(t + 1);
         }
+        if (!(ok = mbar_wait(&ms.p_full, t & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_dq(t);
       }
       tc_commit(&ms.o_full);
     }
@@ -547,12 +573,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const int kj0 = (j_lo + t) * KT;
       const bool full = tile_visible(a, q0, QT, kj0, KT);
+      uint32_t ds[16];
       auto chunk = [&](int c, auto all_visible) {
         float sv[32], dp[32];
         tmem_ld32f(lane_addr + C_S + 32 * c, sv);
         tmem_ld32f(lane_addr + C_DP + 32 * c, dp);
         tmem_wait_ld();
-        uint32_t ds[16];
+        // the next step's S and dP may now overwrite these columns
+        tc_fence_before();
+        mbar_arrive(&ms.s_read);
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float v2[2];
@@ -564,10 +593,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           ds[e / 2] = pack_bf16(v2[0], v2[1]);
         }
-        tmem_st16(lane_addr + C_DS + 16 * c, ds);
       };
       if (full) chunk(wgr, std::true_type{});
       else chunk(wgr, std::false_type{});
+      // dS of step t replaces that of step t - 1 once the dQ MMAs of t - 1 have read it
+      if (t > 0) {
+        if (ok) ok = mbar_wait(&ms.dq_done, (t - 1) & 1, abort_flag);
+        if (!(ok = __all_sync(FULL, ok))) break;
+        tc_fence_after();
+      }
+      tmem_st16(lane_addr + C_DS + 16 * wgr, ds);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&ms.p_full);
