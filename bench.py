@@ -519,7 +519,16 @@ def secondary(device, peaks, torch, da):
     ms = _timed(lambda: da.diffattn_fwd_prefill(q, k, v, lam, li, out=out, apply_norm=True,
                                                 norm_eps=inp.eps), torch)
     res["v1_layer"] = {"workload": inp.name, "inputs": seeded, **tflops(prefill_flops(inp), ms)}
-    del q, k, v, out
+    # its backward (V1 runs the exact-fp32 kernels). Algorithmic FLOPs per attended (query,
+    # key) pair and head: scores 2 x 2d, dP = dO V^T 4d (V is 2d wide), dV 4d, dK_1 + dK_2
+    # 4d, dQ_1 + dQ_2 4d: 20 d
+    dy = dev(synth.grad_out((inp.B, inp.N, inp.H, 2 * inp.d), 1001))
+    ms = _timed(lambda: da.diffattn_bwd_prefill(q, k, v, lam, dy, li, apply_norm=True,
+                                                norm_eps=inp.eps), torch, reps=3, warm=1)
+    res["v1_backward_exact_fp32"] = {
+        "workload": inp.name + " backward", "inputs": seeded, "path": "exact-fp32 SIMT kernels",
+        **tflops(20.0 * inp.d * inp.H * inp.B * visible_pairs(inp.N, inp.N), ms)}
+    del q, k, v, out, dy
     # ---- V2 prefill, its window and chunk forms
     inp = synth.config3()
     q, k, v = dev(inp.q), dev(inp.k), dev(inp.v)

@@ -195,10 +195,10 @@ int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t*
 }
 
 // the tensor-core backward serves bf16 V2 with d = 128; everything else runs on the
-// exact-fp32 SIMT kernels. (The tensor-core kernels also take V1, d = 64: its dQ, dK and dV
-// meet the bf16 bounds, but dlambda through the per-head norm's backward measured 0.5-1.1%
-// relative RMS off the float64 reference, above the 5e-3 the other outputs meet, so V1 stays
-// on the exact path.)
+// exact-fp32 SIMT kernels. (V1 is not given a tensor-core path: its dlambda goes through the
+// per-head norm's backward, which takes the forward's bf16-accumulated output as input; a
+// tensor-core version of V1 built this way measured 0.5-1.1% relative RMS off the float64
+// reference in dlambda, above the 5e-3 the other outputs meet.)
 static bool bwd_tensor_core(const diffattn_prefill_params* p) {
   return p->dtype == DIFFATTN_BF16 && p->variant == DIFFATTN_V2 && p->head_dim == 128;
 }
@@ -229,7 +229,7 @@ int diffattn_bwd_workspace_size(const diffattn_prefill_params* p, size_t* bytes)
   } else {
     return DIFFATTN_ERR_INVALID_ARG;
   }
-  *bytes = bwd_tensor_core(p) ? bwd_tc_workspace_bytes(p->variant, p->batch, p->seqlen, units)
+  *bytes = bwd_tensor_core(p) ? bwd_tc_workspace_bytes(p->batch, p->seqlen, units)
                               : bwd_workspace_bytes(p->batch, p->seqlen, units, dv);
   return DIFFATTN_OK;
 }
@@ -250,7 +250,7 @@ int diffattn_bwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return DIFFATTN_ERR_MISALIGNED;
   const PrefillArgs& a = g.f;
   const bool tc = bwd_tensor_core(p);
-  const size_t need = tc ? bwd_tc_workspace_bytes(a.variant, a.B, a.N, a.units)
+  const size_t need = tc ? bwd_tc_workspace_bytes(a.B, a.N, a.units)
                          : bwd_workspace_bytes(a.B, a.N, a.units, a.dv);
   if (!workspace || workspace_bytes < need) return DIFFATTN_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIFFATTN_ERR_MISALIGNED;

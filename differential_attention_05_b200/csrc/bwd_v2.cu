@@ -20,13 +20,9 @@
 //   3. bwd_v2_dq_kernel: one CTA per (64-query tile, pair, batch entry) walks the 128-key
 //      tiles its queries see: S = [Q_1; Q_2] K^T and dP = [dO; dO] V^T (branches stacked in
 //      the M = 128 rows), dS_b in bf16 into TMEM, dQ += dS K.
-// V1 (d = 64, branches with their own keys K_1, K_2 and one value of width 2d) runs the same
-// kernels: its key row is (K_1 | K_2), 128 wide, and the query tile is laid out zero-padded,
-// rows 0-63 = (Q_1 | 0), rows 64-127 = (0 | Q_2), so one K = 128 MMA chain gives both
-// branches' scores, dK = [dS_1^T | dS_2^T] [Q_1 0; 0 Q_2] is (dK_1 | dK_2) in the key layout,
-// and dQ_b is the branch's own half of dS [K_1 | K_2]. The statistics pass (the V1 forward
-// kernel) also writes the gradient reaching O through the per-head norm, in bf16, which the
-// kernels read in place of dy.
+// V1 runs the exact-fp32 kernels (backward.cu): its dlambda goes through the per-head norm's
+// backward, which takes the forward's bf16-accumulated output as input and amplifies its
+// rounding beyond the bf16 bound, so no tensor-core path is built for it.
 // No atomics: every dK/dV row and every dQ row is summed inside one CTA in a fixed order.
 // Warps 0-15 (four warpgroups, each taking a quarter of a step's columns) form the per-row
 // arithmetic, warp 16 issues the TMA loads (128-byte swizzle, no multicast) and the 1-D bulk
@@ -99,7 +95,6 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 }  // namespace kv
 }  // namespace
 
-template <bool V1>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_v2_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdArgs g) {
   using namespace kv;
@@ -123,7 +118,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   const int qt_lo = i_lo / QT;
   const int n_qt = i_hi >= i_lo ? i_hi / QT - qt_lo + 1 : 0;
-  const int pairs = V1 ? 1 : a.group / 2, u0 = gk * pairs;
+  const int pairs = a.group / 2, u0 = gk * pairs;
   const int n_steps = n_qt * pairs;  // step t: pair u0 + t / n_qt, query tile qt_lo + t % n_qt
 
   if (threadIdx.x == 0) {
@@ -142,15 +137,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == W_MMA) {
     tmem_alloc(&ms.tmem_base, TMEM_COLS);
     tmem_relinquish();
-  }
-  if (V1) {
-    // the zero quadrants of both stages' query tiles: block 1 rows 0-63, block 0 rows 64-127
-    for (int i = threadIdx.x; i < STAGES * 2 * (HBLK / 16); i += NUM_THREADS) {
-      const int st = i / (2 * (HBLK / 16)), r = i % (2 * (HBLK / 16));
-      const int off = (r < HBLK / 16) ? BLK + 16 * r : HBLK + 16 * (r - HBLK / 16);
-      *reinterpret_cast<uint4*>(smem + STAGE_OFF + st * STAGE_BYTES + QS + off) = make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async();
   }
   tc_fence_before();
   __syncthreads();
@@ -177,16 +163,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&ms.q_empty[s], ((t / STAGES) & 1) ^ 1, abort_flag)) break;
         const int u = u0 + t / n_qt, q0 = (qt_lo + t % n_qt) * QT;
         uint8_t* st = smem + STAGE_OFF + s * STAGE_BYTES;
-        mbar_arrive_expect_tx(&ms.q_full[s], (V1 ? 2 * HBLK : 2 * BLK) + 2 * HBLK + 1024);
+        mbar_arrive_expect_tx(&ms.q_full[s], 2 * BLK + 2 * HBLK + 1024);
         for (int hf = 0; hf < 2; ++hf) {
-          if (V1) {
-            // (Q_1 | 0) in rows 0-63, (0 | Q_2) in rows 64-127: block hf gets branch hf
-            tma_load_4d(st + QS + hf * BLK + hf * HBLK, &maps.q, &ms.q_full[s], 64 * hf, u, q0, b);
-          } else {
-            // [Q_1; Q_2]: rows 0-63 branch 1, rows 64-127 branch 2 of each 64-column block
-            tma_load_4d(st + QS + hf * BLK, &maps.q, &ms.q_full[s], 64 * hf, 2 * u, q0, b);
-            tma_load_4d(st + QS + hf * BLK + 64 * 128, &maps.q, &ms.q_full[s], 64 * hf, 2 * u + 1, q0, b);
-          }
+          // [Q_1; Q_2]: rows 0-63 branch 1, rows 64-127 branch 2 of each 64-column block
+          tma_load_4d(st + QS + hf * BLK, &maps.q, &ms.q_full[s], 64 * hf, 2 * u, q0, b);
+          tma_load_4d(st + QS + hf * BLK + 64 * 128, &maps.q, &ms.q_full[s], 64 * hf, 2 * u + 1, q0, b);
           tma_load_4d(st + DO + hf * HBLK, &maps.dy, &ms.q_full[s], 64 * hf, u, q0, b);
         }
         bulk_load(st + STS, g.w_st + (((int64_t)b * a.units + u) * rows + q0) * 4, 1024, &ms.q_full[s]);
@@ -403,7 +384,6 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 }  // namespace dqk
 }  // namespace
 
-template <bool V1>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_v2_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdArgs g) {
   using namespace dqk;
@@ -420,7 +400,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int u = (int)(blockIdx.x % per_qt) % a.units;
   const int b = (int)(blockIdx.x % per_qt) / a.units;
   const int q0 = qt * QT;
-  const int gk = V1 ? u : (2 * u) / a.group;
+  const int gk = (2 * u) / a.group;
   const int off = a.Nk - a.N;
   const int khi = a.causal ? min(q0 + QT - 1 + off, a.Nk - 1) : a.Nk - 1;
   const int klo = (a.causal && a.window > 0) ? max(0, q0 + off - a.window + 1) : 0;
@@ -445,14 +425,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tmem_alloc(&ms.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-  if (V1) {
-    // the zero quadrants of the query tile: block 1 rows 0-63, block 0 rows 64-127
-    for (int i = threadIdx.x; i < 2 * (HBLK / 16); i += NUM_THREADS) {
-      const int off = (i < HBLK / 16) ? BLK + 16 * i : HBLK + 16 * (i - HBLK / 16);
-      *reinterpret_cast<uint4*>(smem + QS_OFF + off) = make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -466,14 +438,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&maps.k);
       tma_prefetch_desc(&maps.v);
       tma_prefetch_desc(&maps.dy);
-      mbar_arrive_expect_tx(&ms.q_full, (V1 ? 2 * HBLK : 2 * BLK) + 2 * BLK + 1024);
+      mbar_arrive_expect_tx(&ms.q_full, 2 * BLK + 2 * BLK + 1024);
       for (int hf = 0; hf < 2; ++hf) {
-        if (V1) {
-          tma_load_4d(smem + QS_OFF + hf * BLK + hf * HBLK, &maps.q, &ms.q_full, 64 * hf, u, q0, b);
-        } else {
-          tma_load_4d(smem + QS_OFF + hf * BLK, &maps.q, &ms.q_full, 64 * hf, 2 * u, q0, b);
-          tma_load_4d(smem + QS_OFF + hf * BLK + 64 * 128, &maps.q, &ms.q_full, 64 * hf, 2 * u + 1, q0, b);
-        }
+        tma_load_4d(smem + QS_OFF + hf * BLK, &maps.q, &ms.q_full, 64 * hf, 2 * u, q0, b);
+        tma_load_4d(smem + QS_OFF + hf * BLK + 64 * 128, &maps.q, &ms.q_full, 64 * hf, 2 * u + 1, q0, b);
         // dO in both halves: the branch-2 rows need dP = dO V^T as well
         tma_load_4d(smem + DO_OFF + hf * BLK, &maps.dy, &ms.q_full, 64 * hf, u, q0, b);
         tma_load_4d(smem + DO_OFF + hf * BLK + 64 * 128, &maps.dy, &ms.q_full, 64 * hf, u, q0, b);
@@ -614,14 +582,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float scale = rsqrtf((float)a.d);
       const bool store = qi < a.N;
       const int64_t qrow = (int64_t)b * a.N + (store ? qi : 0);
-      // V2: the 128 columns of query head 2u + br; V1: branch br's own half (columns 64 br ..)
-      // of dS [K_1 | K_2], into q's [.., H, 2, d] layout
-      float4* dq4 = reinterpret_cast<float4*>(
-          V1 ? g.dq + (qrow * a.units + u) * 128 + 64 * br : g.dq + (qrow * a.Hq + 2 * u + br) * 128);
-      const int n_ch = V1 ? 2 : 4;
-      const uint32_t col0 = C_DQ + (V1 ? 64u * br : 0u);  // warp-uniform: br is per warp
+      // the 128 columns of query head 2u + br
+      float4* dq4 = reinterpret_cast<float4*>(g.dq + (qrow * a.Hq + 2 * u + br) * 128);
+      const uint32_t col0 = C_DQ;
       const int c = wgr;  // this warpgroup's 32 columns (warp-uniform)
-      if (c < n_ch) {
+      {
         if (n_kt > 0) {
           tc_fence_after();
           float x[32];
@@ -656,25 +621,20 @@ namespace {
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 }  // namespace
 
-// statistics rows (N + 64 per entry and unit), dlambda shares, and for V1 the bf16 dO
-size_t bwd_tc_workspace_bytes(int variant, int B, int N, int units) {
-  size_t n = up256((size_t)B * units * (N + 64) * 4 * sizeof(float)) +
-             up256((size_t)B * units * N * sizeof(float));
-  if (variant == DIFFATTN_V1) n += up256((size_t)B * N * units * 128 * 2);
-  return n;
+// statistics rows (N + 64 per entry and pair) and the dlambda shares
+size_t bwd_tc_workspace_bytes(int B, int N, int units) {
+  return up256((size_t)B * units * (N + 64) * 4 * sizeof(float)) +
+         up256((size_t)B * units * N * sizeof(float));
 }
 
 cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream) {
   const PrefillArgs& a = g.f;
-  const bool v1 = a.variant == DIFFATTN_V1;
-  if (a.cu_q || (v1 ? a.d != 64 : a.d != 128)) return cudaErrorNotSupported;
+  if (a.cu_q || a.variant != DIFFATTN_V2 || a.d != 128) return cudaErrorNotSupported;
   uint8_t* w = static_cast<uint8_t*>(workspace);
   const size_t st_bytes = up256((size_t)a.B * a.units * (a.N + 64) * 4 * sizeof(float));
-  const size_t dl_bytes = up256((size_t)a.B * a.units * a.N * sizeof(float));
   g.w_st = reinterpret_cast<float*>(w);
   g.w_dl = reinterpret_cast<float*>(w + st_bytes);
   g.w_do = nullptr;
-  g.w_do16 = v1 ? static_cast<void*>(w + st_bytes + dl_bytes) : nullptr;
   // 1. statistics: the forward kernel in its statistics mode
   PrefillArgs fa = a;
   fa.out = nullptr;
@@ -683,51 +643,32 @@ cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream) 
   fa.st = g.w_st;
   fa.st_dl = g.w_dl;
   fa.st_rows = a.N + 64;
-  fa.st_do = g.w_do16;
-  cudaError_t e = v1 ? launch_prefill_v1_stats(fa, stream) : launch_prefill_v2_stats(fa, stream);
+  cudaError_t e = launch_prefill_v2_stats(fa, stream);
   if (e != cudaSuccess) return e;
-  // 2, 3. dK/dV and dQ. V1: q [B, N, H, 128] (Q_1 | Q_2), k, v [B, N, H, 128], dO the bf16
-  // workspace [B, N, H, 128]; V2: q [B, N, Hq, 128], k, v [B, N, Hkv, 128], dO = dy.
+  // 2, 3. dK/dV and dQ: q [B, N, Hq, 128], k, v [B, N, Hkv, 128], dO = dy [B, N, Hq/2, 128]
   BwdMaps maps;
-  const int qheads = v1 ? a.units : a.Hq;
-  if (!make_map(&maps.q, a.q, 128, qheads, a.N, a.B, a.qs, 64)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.q, a.q, 128, a.Hq, a.N, a.B, a.qs, 64)) return cudaErrorInvalidValue;
   if (!make_map(&maps.k, a.k, 128, a.Hkv, a.Nk, a.B, a.ks, 128)) return cudaErrorInvalidValue;
   if (!make_map(&maps.v, a.v, 128, a.Hkv, a.Nk, a.B, a.vs, 128)) return cudaErrorInvalidValue;
-  if (v1) {
-    const int64_t ds[3] = {(int64_t)a.N * a.units * 128, (int64_t)a.units * 128, 128};
-    if (!make_map(&maps.dy, g.w_do16, 128, a.units, a.N, a.B, ds, 64)) return cudaErrorInvalidValue;
-  } else {
-    if (!make_map(&maps.dy, g.dy, 128, a.units, a.N, a.B, g.dys, 64)) return cudaErrorInvalidValue;
-  }
+  if (!make_map(&maps.dy, g.dy, 128, a.units, a.N, a.B, g.dys, 64)) return cudaErrorInvalidValue;
   int dev = 0;
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   if (dev >= 64 || !attr_set[dev]) {
-    const void* kv_fns[2] = {(const void*)bwd_v2_dkdv_kernel<false>, (const void*)bwd_v2_dkdv_kernel<true>};
-    const void* dq_fns[2] = {(const void*)bwd_v2_dq_kernel<false>, (const void*)bwd_v2_dq_kernel<true>};
-    for (int i = 0; i < 2; ++i) {
-      e = cudaFuncSetAttribute(kv_fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, kv::SMEM_BYTES);
-      if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(dq_fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::SMEM_BYTES);
-      if (e != cudaSuccess) return e;
-    }
+    e = cudaFuncSetAttribute(bwd_v2_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(bwd_v2_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     if (dev < 64) attr_set[dev] = true;
   }
   const long long kv_ctas = (long long)((a.Nk + kv::KT - 1) / kv::KT) * a.Hkv * a.B;
   const long long dq_ctas = (long long)((a.N + dqk::QT - 1) / dqk::QT) * a.units * a.B;
   if (kv_ctas > 0x7fffffffLL || dq_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  if (v1) {
-    bwd_v2_dkdv_kernel<true><<<(unsigned)kv_ctas, NUM_THREADS, kv::SMEM_BYTES, stream>>>(maps, g);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    bwd_v2_dq_kernel<true><<<(unsigned)dq_ctas, NUM_THREADS, dqk::SMEM_BYTES, stream>>>(maps, g);
-  } else {
-    bwd_v2_dkdv_kernel<false><<<(unsigned)kv_ctas, NUM_THREADS, kv::SMEM_BYTES, stream>>>(maps, g);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    bwd_v2_dq_kernel<false><<<(unsigned)dq_ctas, NUM_THREADS, dqk::SMEM_BYTES, stream>>>(maps, g);
-  }
+  bwd_v2_dkdv_kernel<<<(unsigned)kv_ctas, NUM_THREADS, kv::SMEM_BYTES, stream>>>(maps, g);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_v2_dq_kernel<<<(unsigned)dq_ctas, NUM_THREADS, dqk::SMEM_BYTES, stream>>>(maps, g);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_dlambda_reduce(g, stream);

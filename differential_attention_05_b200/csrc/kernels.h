@@ -42,7 +42,6 @@ struct PrefillArgs {
   float* st;
   float* st_dl;
   int st_rows;
-  void* st_do;  // V1: the gradient reaching O (through the norm), bf16 [B, N, H, 2d] dense
 };
 
 // Resolved backward problem: the forward's arguments plus the incoming gradient dy (the
@@ -60,7 +59,6 @@ struct BwdArgs {
   float* w_do;               // [B, N, units, dv] gradient reaching O
   float* w_st;               // [B, N, units, 4] lse_1, lse_2, delta_1, delta_2
   float* w_dl;               // [B, units, N] per-row dlambda shares
-  void* w_do16;              // V1 tensor-core path: dO in bf16 [B, N, H, 2d]
 };
 
 #ifdef __CUDACC__
@@ -125,7 +123,6 @@ cudaError_t launch_prefill_f32(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_v1(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_v2_stats(const PrefillArgs& a, cudaStream_t stream);
-cudaError_t launch_prefill_v1_stats(const PrefillArgs& a, cudaStream_t stream);
 
 // split-KV decode (V2, bf16, d = 128, 8 query heads per KV head)
 constexpr int kDecodeChunk = 64;  // keys per pipeline stage
@@ -139,7 +136,7 @@ cudaError_t launch_decode_v1(const DecodeArgs& a, cudaStream_t stream);
 size_t bwd_workspace_bytes(int B, int N, int units, int dv);
 cudaError_t launch_backward(BwdArgs g, void* workspace, cudaStream_t stream);
 cudaError_t launch_dlambda_reduce(const BwdArgs& g, cudaStream_t stream);
-size_t bwd_tc_workspace_bytes(int variant, int B, int N, int units);
+size_t bwd_tc_workspace_bytes(int B, int N, int units);
 cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream);
 cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* lq2,
                               const float* lk2, int n_heads, int dim, const float* dlam,

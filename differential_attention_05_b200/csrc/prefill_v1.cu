@@ -92,8 +92,6 @@ struct Misc {
   float ex_l[2][BM];      // epilogue: [branch][row] row sums
   float ex_c[BM];         // epilogue: c
   float ssx[2][BM];       // V1 norm: partial sums of squares
-  float ex_m[2][BM];      // statistics pass: [branch][row] maxima
-  float ex_s[2][BM];      //                  partial dot products
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -106,10 +104,7 @@ __device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 256;" 
 // only an upper end; that case compiles without the lower-end and unset-row checks.
 // VARLEN: a variable-length batch (a.cu_q != nullptr); the fixed-length instantiation
 // takes its sizes from the parameters alone.
-// STATS: the statistics pass of the backward (fixed length only): instead of the output
-// the epilogue writes the gradient reaching O through the norm (PrefillArgs::st_do), the
-// log-sum-exps, the deltas and the dlambda share (PrefillArgs::st).
-template <bool WINDOW, bool VARLEN, bool STATS = false>
+template <bool WINDOW, bool VARLEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_v1_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -455,101 +450,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int e = 0; e < 64; ++e) ss = fmaf(y[e], y[e], ss);
     }
-    if constexpr (STATS) {
-      // dy over this thread's 64 channels and (dy . o) over them
-      float gr[64];
-      float sdy = 0.f;
-      if (ok && qi < a.N) {
-        const uint4* g4 = reinterpret_cast<const uint4*>(
-            static_cast<const __nv_bfloat16*>(a.st_dy) + (int64_t)b * a.st_dys[0] +
-            (int64_t)qi * a.st_dys[1] + (int64_t)u * a.st_dys[2] + wg * 64);
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          const uint4 w = g4[v];
-          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            gr[v * 8 + 2 * e] = __uint_as_float(wv[e] << 16);
-            gr[v * 8 + 2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 64; ++e) gr[e] = 0.f;
-      }
-#pragma unroll
-      for (int e = 0; e < 64; ++e) sdy = fmaf(gr[e], y[e], sdy);
-      ms.ssx[wg][row] = ss;
-      ms.ex_s[wg][row] = sdy;
-      ms.ex_m[wg][row] = m;
-      bar_softmax();
-      const float ss_t = ms.ssx[0][row] + ms.ssx[1][row];
-      const float sdy_t = ms.ex_s[0][row] + ms.ex_s[1][row];
-      const float m1 = ms.ex_m[0][row], m2 = ms.ex_m[1][row];
-      if (a.apply_norm) {
-        // y = s o / r with r^2 = mean o^2 + eps: dO = s/r (dy - o (dy . o) / (n r^2))
-        const float r2 = ss_t * (1.f / 128.f) + a.eps;
-        const float f = (1.f - a.lambda_init[0]) * rsqrtf(r2);
-        const float proj = sdy_t / (128.f * r2);
-#pragma unroll
-        for (int e = 0; e < 64; ++e) gr[e] = f * (gr[e] - y[e] * proj);
-      }
-      // delta_b partials against O_1 = (D + c O_2) / l_1 and O_2 / l_2 (reloaded from TMEM)
-      float e1 = 0.f, e2 = 0.f;
-      if (ok) {
-        const float c1 = c * inv1;
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          float dv[32], ov[32];
-          tmem_ld32f(lane_addr + COL_D + wg * 64 + ch * 32, dv);
-          tmem_ld32f(lane_addr + COL_O2 + wg * 64 + ch * 32, ov);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            e1 = fmaf(gr[ch * 32 + e], __fmaf_rn(ov[e], c1, dv[e] * inv1), e1);
-            e2 = fmaf(gr[ch * 32 + e], ov[e] * inv2, e2);
-          }
-        }
-      }
-      bar_softmax();  // both warpgroups have read the first exchange
-      ms.ex_s[wg][row] = e1;
-      ms.ssx[wg][row] = e2;
-      bar_softmax();
-      const float d1 = ms.ex_s[0][row] + ms.ex_s[1][row];
-      const float d2 = ms.ssx[0][row] + ms.ssx[1][row];
-      if (ok && qi < a.N) {
-        uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.st_do) +
-                                             (((int64_t)b * a.N + qi) * a.units + u) * 128 + wg * 64);
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          uint4 w;
-          w.x = pack_bf16(gr[v * 8 + 0], gr[v * 8 + 1]);
-          w.y = pack_bf16(gr[v * 8 + 2], gr[v * 8 + 3]);
-          w.z = pack_bf16(gr[v * 8 + 4], gr[v * 8 + 5]);
-          w.w = pack_bf16(gr[v * 8 + 6], gr[v * 8 + 7]);
-          o4[v] = w;
-        }
-        if (wg == 0) {
-          const int64_t r = ((int64_t)b * a.units + u) * a.st_rows + qi;
-          *reinterpret_cast<float4*>(a.st + r * 4) =
-              make_float4(m1 + log2f(L1), m2 + log2f(L2), d1, d2);
-          a.st_dl[((int64_t)b * a.units + u) * a.N + qi] = -d2;
-        }
-      }
-    }
     float sc = 1.f;
-    if constexpr (!STATS) {
-      ms.ssx[wg][row] = ss;
-      bar_softmax();
-      if (a.apply_norm)
-        sc = rsqrtf((ms.ssx[0][row] + ms.ssx[1][row]) * (1.f / 128.f) + a.eps) *
-             (1.f - a.lambda_init[0]);
-    }
+    ms.ssx[wg][row] = ss;
+    bar_softmax();
+    if (a.apply_norm)
+      sc = rsqrtf((ms.ssx[0][row] + ms.ssx[1][row]) * (1.f / 128.f) + a.eps) *
+           (1.f - a.lambda_init[0]);
     // (a variable-length tile reads its sequence back from shared memory, keeping the
     // registers of the key loop free)
     const int o_nq = VARLEN ? ms.seq_nq : a.N, o_b = VARLEN ? ms.seq_bc : b;
     const int o_q0 = VARLEN ? ms.seq_q0 : 0;
-    if (!STATS && ok && qi < o_nq) {
+    if (ok && qi < o_nq) {
       __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)o_b * a.os[0] +
                           (int64_t)(o_q0 + qi) * a.os[1] + (int64_t)u * a.os[2] + wg * 64;
       uint4* o4 = reinterpret_cast<uint4*>(ob);
@@ -611,38 +522,6 @@ cudaError_t launch_prefill_v1(const PrefillArgs& a, cudaStream_t stream) {
     if (window) prefill_v1_kernel<true, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
     else prefill_v1_kernel<false, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   }
-  return cudaGetLastError();
-}
-
-// The backward's statistics pass over the same tiles (fixed-length batches): st, st_dl,
-// st_do and st_dy must be set; out is not written.
-cudaError_t launch_prefill_v1_stats(const PrefillArgs& a, cudaStream_t stream) {
-  if (a.variant != DIFFATTN_V1 || a.d != 64 || a.cu_q) return cudaErrorNotSupported;
-  if (!a.st || !a.st_dl || !a.st_dy || !a.st_do) return cudaErrorInvalidValue;
-  TcMaps maps;
-  if (!make_map(&maps.q, a.q, 128, a.units, a.N, a.B, a.qs, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.k, a.k, 128, a.units, a.Nk, a.B, a.ks, BN)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.v, a.v, 128, a.units, a.Nk, a.B, a.vs, BN)) return cudaErrorInvalidValue;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  static bool attr_set[64] = {};
-  if (dev >= 64 || !attr_set[dev]) {
-    const void* fns[2] = {(const void*)prefill_v1_kernel<false, false, true>,
-                          (const void*)prefill_v1_kernel<true, false, true>};
-    for (const void* fn : fns) {
-      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-      if (e != cudaSuccess) return e;
-    }
-    if (dev < 64) attr_set[dev] = true;
-  }
-  const long long tiles = (long long)((a.N + BM - 1) / BM) * a.units * a.B;
-  if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const dim3 grid((unsigned)tiles);
-  if (a.causal && a.window > 0)
-    prefill_v1_kernel<true, false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
-  else
-    prefill_v1_kernel<false, false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   return cudaGetLastError();
 }
 
