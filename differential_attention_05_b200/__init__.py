@@ -29,6 +29,7 @@ from ._binding import (  # noqa: F401
     diffattn_fwd_decode_paged,
     diffattn_selftest_timeout,
     diffattn_selftest_exp2,
+    diffattn_debug_bounds_violations,
     diffattn_decode_workspace_size,
     diffattn_status_string,
     library_path,
@@ -49,6 +50,7 @@ __all__ = [
     "diffattn_fwd_decode_paged",
     "diffattn_selftest_timeout",
     "diffattn_selftest_exp2",
+    "diffattn_debug_bounds_violations",
     "diffattn_decode_workspace_size",
     "diffattn_status_string",
     "library_path",

@@ -43,6 +43,7 @@ EXPORTS = (
     "diffattn_fwd_decode_paged",
     "diffattn_selftest_timeout",
     "diffattn_selftest_exp2",
+    "diffattn_debug_bounds_violations",
 )
 
 
@@ -148,6 +149,8 @@ def load_library():
     lib.diffattn_selftest_timeout.argtypes = [vp, i32, vp]
     lib.diffattn_selftest_exp2.restype = i32
     lib.diffattn_selftest_exp2.argtypes = [vp, vp, vp, i32, vp]
+    lib.diffattn_debug_bounds_violations.restype = i32
+    lib.diffattn_debug_bounds_violations.argtypes = [ctypes.POINTER(ctypes.c_int32)]
     _lib = lib
     return lib
 
@@ -530,3 +533,15 @@ def diffattn_selftest_exp2(x, stream=None):
     rc = lib.diffattn_selftest_exp2(_ptr(x), _ptr(y), _ptr(y_ref), int(x.numel()), _stream(stream))
     _check("diffattn_selftest_exp2", rc)
     return y, y_ref
+
+
+def diffattn_debug_bounds_violations():
+    """The bounds-checked build's count of skipped out-of-range accesses since the last call
+    (see include/diffattn.h), or None when the loaded library is the normal build."""
+    lib = load_library()
+    n = ctypes.c_int32(0)
+    rc = lib.diffattn_debug_bounds_violations(ctypes.byref(n))
+    if rc == -2:  # DIFFATTN_ERR_UNSUPPORTED: the normal build
+        return None
+    _check("diffattn_debug_bounds_violations", rc)
+    return int(n.value)

@@ -28,11 +28,44 @@ inline bool strides_ok(const int64_t* s, int n) {
   return true;
 }
 
+// One past the largest element offset of a [nb, rows, heads, width] view with element
+// strides {batch, token, head}; 0 for an empty view.
+inline int64_t extent(int64_t nb, int64_t rows, int64_t heads, int64_t width, const int64_t* s) {
+  if (nb <= 0 || rows <= 0 || heads <= 0 || width <= 0) return 0;
+  return (nb - 1) * s[0] + (rows - 1) * s[1] + (heads - 1) * s[2] + width;
+}
+
+#ifdef DIFFATTN_DEBUG
+// the bounds-checked build's own status word: the number of accesses its checks skipped
+__device__ int g_bounds_violations;
+int* debug_status_word() {
+  void* p = nullptr;
+  return cudaGetSymbolAddress(&p, g_bounds_violations) == cudaSuccess ? static_cast<int*>(p) : nullptr;
+}
+#else
+int* debug_status_word() { return nullptr; }
+#endif
+
 }  // namespace
 
 extern "C" {
 
 int diffattn_version(void) { return kAbiVersion; }
+
+int diffattn_debug_bounds_violations(int* count) {
+  if (!count) return DIFFATTN_ERR_INVALID_ARG;
+  *count = 0;
+#ifdef DIFFATTN_DEBUG
+  int* p = debug_status_word();
+  if (!p) return DIFFATTN_ERR_CUDA;
+  if (cudaMemcpy(count, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  if (cudaMemset(p, 0, sizeof(int)) != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DIFFATTN_ERR_CUDA;
+  return DIFFATTN_OK;
+#else
+  return DIFFATTN_ERR_UNSUPPORTED;
+#endif
+}
 
 const char* diffattn_status_string(int status) {
   switch (status) {
@@ -153,6 +186,18 @@ static int prefill_setup(const diffattn_prefill_params* p, const int32_t* cu_q, 
   a.lambda_init = lambda_init;
   a.out = const_cast<void*>(out);
   a.dev_status = dev_status;
+  // element extents (checked by the bounds-checked build): a variable-length batch is one
+  // packed sequence of rows
+  {
+    const int64_t nb = varlen ? 1 : a.B;
+    const int64_t rq = varlen ? p->seqlen : a.N, rk = varlen ? nk : a.Nk;
+    const int v1 = a.variant == DIFFATTN_V1;
+    a.ext_q = extent(nb, rq, v1 ? a.units : a.Hq, v1 ? 2 * a.d : a.d, a.qs);
+    a.ext_k = extent(nb, rk, a.Hkv, v1 ? 2 * a.d : a.d, a.ks);
+    a.ext_v = extent(nb, rk, a.Hkv, a.dv, a.vs);
+    a.ext_out = extent(nb, rq, a.units, a.dv, a.os);
+    a.dbg_status = debug_status_word();
+  }
   return DIFFATTN_OK;
 }
 
@@ -261,6 +306,13 @@ int diffattn_bwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   g.dk = dk;
   g.dv = dv;
   g.dlambda = dlambda;
+  {
+    const int v1 = a.variant == DIFFATTN_V1;
+    g.ext_dq = (int64_t)a.B * a.N * (v1 ? a.units * 2 * a.d : a.Hq * a.d);
+    g.ext_dk = (int64_t)a.B * a.Nk * a.Hkv * (v1 ? 2 * a.d : a.d);
+    g.ext_dv = (int64_t)a.B * a.Nk * a.Hkv * a.dv;
+    g.ext_ws = (int64_t)(workspace_bytes / sizeof(float));
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return from_cuda(tc ? launch_backward_tc(g, workspace, s) : launch_backward(g, workspace, s));
 }
@@ -426,6 +478,20 @@ static int decode_run(const diffattn_decode_params* p, const diffattn_paged_kv* 
   a.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                      (((recs * rec_floats * sizeof(float)) + 255) & ~(size_t)255));
   a.dev_status = dev_status;
+  // element extents (checked by the bounds-checked build)
+  {
+    const int64_t qh[3] = {p->q_strides[0], 0, p->q_strides[1]};  // [B, 1, heads, width]
+    const int64_t oh[3] = {p->o_strides[0], 0, p->o_strides[1]};
+    const int width = v1 ? 2 * a.d : a.d;
+    a.ext_q = extent(a.B, 1, a.Hq, width, qh);
+    a.ext_kv = pk ? extent(pk->num_pages, pk->page_size, a.Hkv, width, kvs)
+                  : extent(a.B, a.L, a.Hkv, width, kvs);
+    a.ext_out = extent(a.B, 1, v1 ? a.Hq : a.Hq / 2, width, oh);
+    a.ext_ws_o = (int64_t)(recs * rec_floats);
+    a.ext_ws_ml = (int64_t)(recs * 2);
+    a.ext_bt = pk ? (int64_t)a.B * pk->max_pages_per_seq : 0;
+    a.dbg_status = debug_status_word();
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return from_cuda(v1 ? launch_decode_v1(a, s) : launch_decode(a, s));
 }

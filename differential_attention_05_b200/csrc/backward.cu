@@ -110,13 +110,38 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_rows_kernel(BwdArgs g) {
   const T* k = static_cast<const T*>(a.k) + b * a.ks[0];
   const T* v = static_cast<const T*>(a.v) + b * a.vs[0];
   const UnitRows ur = unit_rows(a, u);
+  int lo, hi;
+  key_range(a, i, lo, hi);
+  {
+    // (bounds-checked build) every row this warp reads or writes; the strides are
+    // non-negative, so the first and last key rows bound all the others
+    const int64_t qo = b * a.qs[0] + (int64_t)i * a.qs[1];
+    const int64_t row = ((int64_t)b * a.N + i) * a.units + u;
+    const int64_t dq_off = a.variant == DIFFATTN_V1 ? (((int64_t)b * a.N + i) * a.units + u) * 2 * d
+                                                    : (((int64_t)b * a.N + i) * a.Hq + 2 * u) * d;
+    bool ok = in_bounds(qo + ur.q1, d, a.ext_q, a.dev_status, a.dbg_status) &&
+              in_bounds(qo + ur.q2, d, a.ext_q, a.dev_status, a.dbg_status) &&
+              in_bounds(b * g.dys[0] + (int64_t)i * g.dys[1] + u * g.dys[2], dv, a.ext_out,
+                        a.dev_status, a.dbg_status) &&
+              in_bounds((g.w_do - g.w_base) + row * dv, dv, g.ext_ws, a.dev_status, a.dbg_status) &&
+              in_bounds((g.w_st - g.w_base) + row * 4, 4, g.ext_ws, a.dev_status, a.dbg_status) &&
+              in_bounds((g.w_dl - g.w_base) + ((int64_t)b * a.units + u) * a.N + i, 1, g.ext_ws,
+                        a.dev_status, a.dbg_status) &&
+              in_bounds(dq_off, 2 * d, g.ext_dq, a.dev_status, a.dbg_status);
+    if (lo <= hi)
+      for (int e = 0; e < 2; ++e) {
+        const int jj = e ? hi : lo;
+        ok = ok && in_bounds(b * a.ks[0] + (int64_t)jj * a.ks[1] + ur.k1, d, a.ext_k, a.dev_status, a.dbg_status) &&
+             in_bounds(b * a.ks[0] + (int64_t)jj * a.ks[1] + ur.k2, d, a.ext_k, a.dev_status, a.dbg_status) &&
+             in_bounds(b * a.vs[0] + (int64_t)jj * a.vs[1] + ur.v, dv, a.ext_v, a.dev_status, a.dbg_status);
+      }
+    if (!ok) return;
+  }
   for (int c = lane; c < d; c += 32) {
     qsm[warp][0][c] = ld1(q + ur.q1 + c);
     qsm[warp][1][c] = ld1(q + ur.q2 + c);
   }
   __syncwarp();
-  int lo, hi;
-  key_range(a, i, lo, hi);
   const float scale = 1.0f / sqrtf((float)d);
   const float lam = a.lambda[u];
 
@@ -280,8 +305,18 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_keys_kernel(BwdArgs g) {
   if (j >= a.Nk) return;
   const int d = a.d, dv = a.dv;
   const bool v1 = a.variant == DIFFATTN_V1;
-  const T* kr = static_cast<const T*>(a.k) + b * a.ks[0] + (int64_t)j * a.ks[1] + (int64_t)kh * a.ks[2];
-  const T* vr = static_cast<const T*>(a.v) + b * a.vs[0] + (int64_t)j * a.vs[1] + (int64_t)kh * a.vs[2];
+  const int64_t k_off = b * a.ks[0] + (int64_t)j * a.ks[1] + (int64_t)kh * a.ks[2];
+  const int64_t v_off = b * a.vs[0] + (int64_t)j * a.vs[1] + (int64_t)kh * a.vs[2];
+  const int nkh_ = v1 ? a.units : a.Hkv;
+  const int64_t krow_ = ((int64_t)b * a.Nk + j) * nkh_ + kh;
+  // (bounds-checked build) this key's rows and outputs
+  if (!(in_bounds(k_off, v1 ? 2 * d : d, a.ext_k, a.dev_status, a.dbg_status) &&
+        in_bounds(v_off, dv, a.ext_v, a.dev_status, a.dbg_status) &&
+        in_bounds(krow_ * (v1 ? 2 * d : d), v1 ? 2 * d : d, g.ext_dk, a.dev_status, a.dbg_status) &&
+        in_bounds(krow_ * dv, dv, g.ext_dv, a.dev_status, a.dbg_status)))
+    return;
+  const T* kr = static_cast<const T*>(a.k) + k_off;
+  const T* vr = static_cast<const T*>(a.v) + v_off;
   for (int c = lane; c < d; c += 32) {
     ksm[warp][0][c] = ld1(kr + c);
     ksm[warp][1][c] = ld1(kr + (v1 ? d : 0) + c);
@@ -310,6 +345,19 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_keys_kernel(BwdArgs g) {
     const float lam = a.lambda[u];
     const UnitRows ur = unit_rows(a, u);
     const T* q = static_cast<const T*>(a.q) + b * a.qs[0];
+    if (i_lo <= i_hi) {
+      // (bounds-checked build) the first and last query rows bound the ones in between
+      bool ok = true;
+      for (int e = 0; e < 2; ++e) {
+        const int ii = e ? i_hi : i_lo;
+        const int64_t row = ((int64_t)b * a.N + ii) * a.units + u;
+        ok = ok && in_bounds(b * a.qs[0] + (int64_t)ii * a.qs[1] + ur.q1, d, a.ext_q, a.dev_status, a.dbg_status) &&
+             in_bounds(b * a.qs[0] + (int64_t)ii * a.qs[1] + ur.q2, d, a.ext_q, a.dev_status, a.dbg_status) &&
+             in_bounds((g.w_st - g.w_base) + row * 4, 4, g.ext_ws, a.dev_status, a.dbg_status) &&
+             in_bounds((g.w_do - g.w_base) + row * dv, dv, g.ext_ws, a.dev_status, a.dbg_status);
+      }
+      if (!ok) return;
+    }
     for (int i0 = i_lo; i0 <= i_hi; i0 += 32) {
       const int i = i0 + lane;
       float pv = 0.f, ds1 = 0.f, ds2 = 0.f;
@@ -379,6 +427,7 @@ __global__ void __launch_bounds__(256) bwd_dlambda_kernel(BwdArgs g) {
   float s = 0.f;
   for (int b = 0; b < a.B; ++b) {
     const float* w = g.w_dl + ((int64_t)b * a.units + u) * a.N;
+    if (!in_bounds(w - g.w_base, a.N, g.ext_ws, a.dev_status, a.dbg_status)) continue;
     for (int i = threadIdx.x; i < a.N; i += 256) s += w[i];
   }
   red[threadIdx.x] = s;
@@ -404,6 +453,7 @@ cudaError_t launch_backward(BwdArgs g, void* workspace, cudaStream_t stream) {
   g.w_do = reinterpret_cast<float*>(w);
   g.w_st = reinterpret_cast<float*>(w + up(rows * a.dv * sizeof(float)));
   g.w_dl = reinterpret_cast<float*>(w + up(rows * a.dv * sizeof(float)) + up(rows * 4 * sizeof(float)));
+  g.w_base = g.w_do;
   const dim3 grid_rows((a.N + kWarps - 1) / kWarps, a.units, a.B);
   const int nkh = a.variant == DIFFATTN_V1 ? a.units : a.Hkv;
   const dim3 grid_keys((a.Nk + kWarps - 1) / kWarps, nkh, a.B);

@@ -163,14 +163,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&ms.q_empty[s], ((t / STAGES) & 1) ^ 1, abort_flag)) break;
         const int u = u0 + t / n_qt, q0 = (qt_lo + t % n_qt) * QT;
         uint8_t* st = smem + STAGE_OFF + s * STAGE_BYTES;
-        mbar_arrive_expect_tx(&ms.q_full[s], 2 * BLK + 2 * HBLK + 1024);
+        // (w_st starts the workspace, so its offsets are workspace offsets)
+        const int64_t st_off = (((int64_t)b * a.units + u) * rows + q0) * 4;
+        const bool st_ok = in_bounds((g.w_st - g.w_base) + st_off, 256, g.ext_ws, a.dev_status, a.dbg_status);
+        mbar_arrive_expect_tx(&ms.q_full[s], 2 * BLK + 2 * HBLK + (st_ok ? 1024 : 0));
         for (int hf = 0; hf < 2; ++hf) {
           // [Q_1; Q_2]: rows 0-63 branch 1, rows 64-127 branch 2 of each 64-column block
           tma_load_4d(st + QS + hf * BLK, &maps.q, &ms.q_full[s], 64 * hf, 2 * u, q0, b);
           tma_load_4d(st + QS + hf * BLK + 64 * 128, &maps.q, &ms.q_full[s], 64 * hf, 2 * u + 1, q0, b);
           tma_load_4d(st + DO + hf * HBLK, &maps.dy, &ms.q_full[s], 64 * hf, u, q0, b);
         }
-        bulk_load(st + STS, g.w_st + (((int64_t)b * a.units + u) * rows + q0) * 4, 1024, &ms.q_full[s]);
+        if (st_ok) bulk_load(st + STS, g.w_st + st_off, 1024, &ms.q_full[s]);
         issued = t + 1;
       }
       if (*abort_flag) {
@@ -322,8 +325,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // depend on the key being inside the sequence
     if (ok) {
       const float scale = rsqrtf((float)a.d);
-      const bool store = j < a.Nk;
-      const int64_t row = ((int64_t)b * a.Nk + (store ? j : 0)) * a.Hkv + gk;
+      const int64_t row = ((int64_t)b * a.Nk + (j < a.Nk ? j : 0)) * a.Hkv + gk;
+      const bool store = j < a.Nk && in_bounds(row * 128, 128, g.ext_dv, a.dev_status, a.dbg_status) &&
+                         in_bounds(row * 128, 128, g.ext_dk, a.dev_status, a.dbg_status);
       float4* dv4 = reinterpret_cast<float4*>(g.dv + row * 128);
       float4* dk4 = reinterpret_cast<float4*>(g.dk + row * 128);
       const int c = wgr;  // this warpgroup's 32 columns of dV and dK
@@ -438,7 +442,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&maps.k);
       tma_prefetch_desc(&maps.v);
       tma_prefetch_desc(&maps.dy);
-      mbar_arrive_expect_tx(&ms.q_full, 2 * BLK + 2 * BLK + 1024);
+      const int64_t st_off = (((int64_t)b * a.units + u) * rows + q0) * 4;  // (workspace offset)
+      const bool st_ok = in_bounds((g.w_st - g.w_base) + st_off, 256, g.ext_ws, a.dev_status, a.dbg_status);
+      mbar_arrive_expect_tx(&ms.q_full, 2 * BLK + 2 * BLK + (st_ok ? 1024 : 0));
       for (int hf = 0; hf < 2; ++hf) {
         tma_load_4d(smem + QS_OFF + hf * BLK, &maps.q, &ms.q_full, 64 * hf, 2 * u, q0, b);
         tma_load_4d(smem + QS_OFF + hf * BLK + 64 * 128, &maps.q, &ms.q_full, 64 * hf, 2 * u + 1, q0, b);
@@ -446,7 +452,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_load_4d(smem + DO_OFF + hf * BLK, &maps.dy, &ms.q_full, 64 * hf, u, q0, b);
         tma_load_4d(smem + DO_OFF + hf * BLK + 64 * 128, &maps.dy, &ms.q_full, 64 * hf, u, q0, b);
       }
-      bulk_load(smem + ST_OFF, g.w_st + (((int64_t)b * a.units + u) * rows + q0) * 4, 1024, &ms.q_full);
+      if (st_ok) bulk_load(smem + ST_OFF, g.w_st + st_off, 1024, &ms.q_full);
       int issued = 0;
       for (int t = 0; t < n_kt && !*abort_flag; ++t) {
         const int s = t % STAGES;
@@ -580,8 +586,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // warp-collective TMEM loads; only the stores depend on the query being in range
     if (ok) {
       const float scale = rsqrtf((float)a.d);
-      const bool store = qi < a.N;
-      const int64_t qrow = (int64_t)b * a.N + (store ? qi : 0);
+      const int64_t qrow = (int64_t)b * a.N + (qi < a.N ? qi : 0);
+      const bool store = qi < a.N && in_bounds((qrow * a.Hq + 2 * u + br) * 128, 128, g.ext_dq,
+                                               a.dev_status, a.dbg_status);
       // the 128 columns of query head 2u + br
       float4* dq4 = reinterpret_cast<float4*>(g.dq + (qrow * a.Hq + 2 * u + br) * 128);
       const uint32_t col0 = C_DQ;
@@ -635,6 +642,7 @@ cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream) 
   g.w_st = reinterpret_cast<float*>(w);
   g.w_dl = reinterpret_cast<float*>(w + st_bytes);
   g.w_do = nullptr;
+  g.w_base = g.w_st;
   // 1. statistics: the forward kernel in its statistics mode
   PrefillArgs fa = a;
   fa.out = nullptr;
@@ -643,6 +651,9 @@ cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream) 
   fa.st = g.w_st;
   fa.st_dl = g.w_dl;
   fa.st_rows = a.N + 64;
+  fa.ext_st_dy = a.ext_out;  // dy has the output's layout
+  fa.ext_st = (int64_t)a.B * a.units * (a.N + 64) * 4;
+  fa.ext_st_dl = (int64_t)a.B * a.units * a.N;
   cudaError_t e = launch_prefill_v2_stats(fa, stream);
   if (e != cudaSuccess) return e;
   // 2, 3. dK/dV and dQ: q [B, N, Hq, 128], k, v [B, N, Hkv, 128], dO = dy [B, N, Hq/2, 128]

@@ -32,6 +32,23 @@ __device__ __forceinline__ void report_status(int* dev_status, int code) {
   if (dev_status) atomicCAS(dev_status, 0, code);
 }
 
+// Bounds checks of the raw global accesses (the TMA loads are bounded by their tensor maps).
+// The bounds-checked build (DIFFATTN_DEBUG) tests that an access of n elements at element
+// offset off stays inside [0, ext); one that does not is skipped by the caller and recorded
+// as DIFFATTN_ERR_INVALID_ARG in the caller's status word and in the build's own one. It
+// never traps. The normal build compiles every check to true.
+#ifdef DIFFATTN_DEBUG
+__device__ __forceinline__ bool in_bounds(int64_t off, int64_t n, int64_t ext, int* dev_status,
+                                          int* dbg_status) {
+  if (off >= 0 && n >= 0 && off + n <= ext) return true;
+  report_status(dev_status, DIFFATTN_ERR_INVALID_ARG);
+  if (dbg_status) atomicAdd(dbg_status, 1);
+  return false;
+}
+#else
+__device__ __forceinline__ bool in_bounds(int64_t, int64_t, int64_t, int*, int*) { return true; }
+#endif
+
 // ---- small math ----------------------------------------------------------------------
 
 __device__ __forceinline__ float warp_sum(float v) {

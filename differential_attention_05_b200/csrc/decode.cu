@@ -78,7 +78,6 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
   const int n_chunks = t_end > t_begin ? (t_end - t_begin + CH - 1) / CH : 0;
 
   // paged cache: this entry's row of the block table; the page stride replaces the batch one
-  const int32_t* bt = PAGED ? a.block_table + (int64_t)b * a.bt_stride : nullptr;
   const int64_t boff = PAGED ? 0 : b * a.kvs[0];
   const __nv_bfloat16* kbase =
       static_cast<const __nv_bfloat16*>(a.k) + boff + (int64_t)g * a.kvs[2];
@@ -99,7 +98,9 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
 #pragma unroll
       for (int i = 0; i < ROWS_T; ++i) {
         const int tok = tok0 + RSTEP * i;
-        pid[i] = tok < t_end ? __ldg(bt + (tok >> a.page_shift)) : 0;
+        const int64_t bi = (int64_t)b * a.bt_stride + (tok >> a.page_shift);
+        pid[i] = (tok < t_end && in_bounds(bi, 1, a.ext_bt, a.dev_status, a.dbg_status))
+                     ? __ldg(a.block_table + bi) : 0;
       }
     }
   };
@@ -127,6 +128,8 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
       } else {
         roff = (int64_t)tok * a.kvs[1];
       }
+      const int64_t soff = boff + (int64_t)g * a.kvs[2] + (ok ? roff : 0) + c16 * 8;
+      ok = ok && in_bounds(soff, 8, a.ext_kv, a.dev_status, a.dbg_status);
       const __nv_bfloat16* src = (tensor ? vbase : kbase) + (ok ? roff : 0) + c16 * 8;
       cp_async_16(st + tensor * TILE_BYTES + swz(row, c16), src, ok ? 16u : 0u);
     }
@@ -135,13 +138,13 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
   // Q fragments of the 8 heads (A operand, rows 0..7), all 8 k-steps of d = 128
   uint32_t qa[8][2];
   {
-    const __nv_bfloat16* qrow =
-        static_cast<const __nv_bfloat16*>(a.q) + b * a.qs[0] + (int64_t)(g * G + gq) * a.qs[1];
-    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qrow);
+    const int64_t q_off = b * a.qs[0] + (int64_t)(g * G + gq) * a.qs[1];
+    const bool q_ok = in_bounds(q_off, D, a.ext_q, a.dev_status, a.dbg_status);
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(a.q) + q_off);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      qa[ks][0] = q32[(ks * 16 + 2 * tq) / 2];
-      qa[ks][1] = q32[(ks * 16 + 8 + 2 * tq) / 2];
+      qa[ks][0] = q_ok ? q32[(ks * 16 + 2 * tq) / 2] : 0u;
+      qa[ks][1] = q_ok ? q32[(ks * 16 + 8 + 2 * tq) / 2] : 0u;
     }
   }
 
@@ -270,8 +273,9 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
     const int hq = g * G + h;
     const int64_t rec = ((int64_t)b * a.Hq + hq) * a.splits + split;
     float4* dst = reinterpret_cast<float4*>(a.ws_o + rec * D + c0);
+    const bool w_ok = in_bounds(rec * D + c0, 8, a.ext_ws_o, a.dev_status, a.dbg_status);
 #pragma unroll
-    for (int v4 = 0; v4 < 2; ++v4) {
+    for (int v4 = 0; v4 < 2 && w_ok; ++v4) {
       float r[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -282,7 +286,7 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
       }
       dst[v4] = make_float4(r[0], r[1], r[2], r[3]);
     }
-    if ((tid % 16) == 0) {
+    if ((tid % 16) == 0 && in_bounds(rec * 2, 2, a.ext_ws_ml, a.dev_status, a.dbg_status)) {
       a.ws_ml[rec * 2 + 0] = M;
       a.ws_ml[rec * 2 + 1] = L;
     }
@@ -296,6 +300,11 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeArgs a) {
   for (int e = 0; e < 2; ++e) {
     const int hq = 2 * p + e;
     const int64_t rec0 = ((int64_t)b * a.Hq + hq) * a.splits;
+    if (!in_bounds(rec0 * 2, 2 * (int64_t)a.splits, a.ext_ws_ml, a.dev_status, a.dbg_status) ||
+        !in_bounds(rec0 * D, (int64_t)a.splits * D, a.ext_ws_o, a.dev_status, a.dbg_status)) {
+      res[e] = 0.f;
+      continue;
+    }
     float M = -INFINITY;
     for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.ws_ml[(rec0 + s) * 2]);
     float L = 0.f, O = 0.f;
@@ -309,8 +318,9 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeArgs a) {
     res[e] = L > 0.f ? O / L : 0.f;
   }
   const float y = res[0] - a.lambda[p] * res[1];
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out) + b * a.os[0] + (int64_t)p * a.os[1];
-  out[c] = __float2bfloat16_rn(y);
+  const int64_t o_off = b * a.os[0] + (int64_t)p * a.os[1];
+  if (in_bounds(o_off + c, 1, a.ext_out, a.dev_status, a.dbg_status))
+    static_cast<__nv_bfloat16*>(a.out)[o_off + c] = __float2bfloat16_rn(y);
 }
 
 int decode_default_splits(int B, int L, int Hkv) {

@@ -70,7 +70,6 @@ __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs 
   const int n_chunks = t_end > t_begin ? (t_end - t_begin + CH - 1) / CH : 0;
 
   // paged cache: this entry's row of the block table; the page stride replaces the batch one
-  const int32_t* bt = PAGED ? a.block_table + (int64_t)b * a.bt_stride : nullptr;
   const int64_t boff = PAGED ? 0 : b * a.kvs[0];
   const __nv_bfloat16* kbase =
       static_cast<const __nv_bfloat16*>(a.k) + boff + (int64_t)h * a.kvs[2];
@@ -91,7 +90,9 @@ __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs 
 #pragma unroll
       for (int i = 0; i < ROWS_T; ++i) {
         const int tok = tok0 + RSTEP * i;
-        pid[i] = tok < t_end ? __ldg(bt + (tok >> a.page_shift)) : 0;
+        const int64_t bi = (int64_t)b * a.bt_stride + (tok >> a.page_shift);
+        pid[i] = (tok < t_end && in_bounds(bi, 1, a.ext_bt, a.dev_status, a.dbg_status))
+                     ? __ldg(a.block_table + bi) : 0;
       }
     }
   };
@@ -119,6 +120,8 @@ __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs 
       } else {
         roff = (int64_t)tok * a.kvs[1];
       }
+      const int64_t soff = boff + (int64_t)h * a.kvs[2] + (ok ? roff : 0) + c16 * 8;
+      ok = ok && in_bounds(soff, 8, a.ext_kv, a.dev_status, a.dbg_status);
       const __nv_bfloat16* src = (tensor ? vbase : kbase) + (ok ? roff : 0) + c16 * 8;
       cp_async_16(st + tensor * TILE_BYTES + swz_v1(row, c16), src, ok ? 16u : 0u);
     }
@@ -127,11 +130,12 @@ __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs 
   // this thread's query branch (64 values) in fp32
   float q[D1];
   {
-    const uint4* q4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
-                                                     b * a.qs[0] + (int64_t)h * a.qs[1] + br * D1);
+    const int64_t q_off = b * a.qs[0] + (int64_t)h * a.qs[1] + br * D1;
+    const bool q_ok = in_bounds(q_off, D1, a.ext_q, a.dev_status, a.dbg_status);
+    const uint4* q4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) + q_off);
 #pragma unroll
     for (int i = 0; i < D1 / 8; ++i) {
-      const uint4 w = q4[i];
+      const uint4 w = q_ok ? q4[i] : make_uint4(0u, 0u, 0u, 0u);
       q[8 * i + 0] = bf16lo(w.x); q[8 * i + 1] = bf16hi(w.x);
       q[8 * i + 2] = bf16lo(w.y); q[8 * i + 3] = bf16hi(w.y);
       q[8 * i + 4] = bf16lo(w.z); q[8 * i + 5] = bf16hi(w.z);
@@ -227,9 +231,11 @@ __global__ void __launch_bounds__(THREADS, 2) decode_v1_split_kernel(DecodeArgs 
     const size_t rec = ((size_t)(b * gridDim.y + h) * gridDim.x + split) * 2;
     float* w1 = a.ws_o + rec * DV;
     float* w2 = w1 + DV;
-    w1[2 * cp] = o1x; w1[2 * cp + 1] = o1y;
-    w2[2 * cp] = o2x; w2[2 * cp + 1] = o2y;
-    if (cp == 0) {
+    if (in_bounds((int64_t)rec * DV + 2 * cp, DV + 2, a.ext_ws_o, a.dev_status, a.dbg_status)) {
+      w1[2 * cp] = o1x; w1[2 * cp + 1] = o1y;
+      w2[2 * cp] = o2x; w2[2 * cp + 1] = o2y;
+    }
+    if (cp == 0 && in_bounds((int64_t)rec * 2, 4, a.ext_ws_ml, a.dev_status, a.dbg_status)) {
       a.ws_ml[rec * 2 + 0] = m1; a.ws_ml[rec * 2 + 1] = l1;
       a.ws_ml[rec * 2 + 2] = m2; a.ws_ml[rec * 2 + 3] = l2;
     }
@@ -242,13 +248,15 @@ __global__ void __launch_bounds__(DV) decode_v1_combine_kernel(DecodeArgs a) {
   const int h = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
   const int S = a.splits;
   const size_t rec0 = (size_t)(b * gridDim.x + h) * S * 2;
+  const bool r_ok = in_bounds((int64_t)rec0 * 2, 4 * (int64_t)S, a.ext_ws_ml, a.dev_status, a.dbg_status) &&
+                    in_bounds((int64_t)rec0 * DV, 2 * (int64_t)S * DV, a.ext_ws_o, a.dev_status, a.dbg_status);
   float M1 = -INFINITY, M2 = -INFINITY;
-  for (int s = 0; s < S; ++s) {
+  for (int s = 0; s < S && r_ok; ++s) {
     M1 = fmaxf(M1, a.ws_ml[(rec0 + 2 * s) * 2]);
     M2 = fmaxf(M2, a.ws_ml[(rec0 + 2 * s + 1) * 2]);
   }
   float L1 = 0.f, L2 = 0.f, O1 = 0.f, O2 = 0.f;
-  for (int s = 0; s < S; ++s) {
+  for (int s = 0; s < S && r_ok; ++s) {
     const size_t r1 = rec0 + 2 * s, r2 = r1 + 1;
     const float ma = a.ws_ml[r1 * 2], mb = a.ws_ml[r2 * 2];
     // a split with no keys has m = -inf and l = 0; it contributes nothing
@@ -269,8 +277,9 @@ __global__ void __launch_bounds__(DV) decode_v1_combine_kernel(DecodeArgs a) {
     const float tot = (red[0] + red[1]) + (red[2] + red[3]);
     y = y * rsqrtf(tot * (1.f / DV) + a.eps) * (1.f - a.lambda_init[0]);
   }
-  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.out) + b * a.os[0] + (int64_t)h * a.os[1];
-  o[c] = __float2bfloat16_rn(y);
+  const int64_t o_off = b * a.os[0] + (int64_t)h * a.os[1];
+  if (in_bounds(o_off + c, 1, a.ext_out, a.dev_status, a.dbg_status))
+    static_cast<__nv_bfloat16*>(a.out)[o_off + c] = __float2bfloat16_rn(y);
 }
 
 int decode_v1_default_splits(int B, int L, int H) {

@@ -42,6 +42,11 @@ struct PrefillArgs {
   float* st;
   float* st_dl;
   int st_rows;
+  // element extents (one past the largest element offset the shapes and strides reach) of
+  // q, k, v, out and the statistics-pass tensors, and the bounds-checked build's own status
+  // word (see in_bounds in common.cuh; unused by the normal build)
+  int64_t ext_q, ext_k, ext_v, ext_out, ext_st_dy, ext_st, ext_st_dl;
+  int* dbg_status;
 };
 
 // Resolved backward problem: the forward's arguments plus the incoming gradient dy (the
@@ -59,6 +64,10 @@ struct BwdArgs {
   float* w_do;               // [B, N, units, dv] gradient reaching O
   float* w_st;               // [B, N, units, 4] lse_1, lse_2, delta_1, delta_2
   float* w_dl;               // [B, units, N] per-row dlambda shares
+  // element extents of dq, dk, dv (dense) and of the workspace in floats, which starts at
+  // w_base (bounds-checked build, see in_bounds in common.cuh)
+  int64_t ext_dq, ext_dk, ext_dv, ext_ws;
+  const float* w_base;
 };
 
 #ifdef __CUDACC__
@@ -109,6 +118,10 @@ struct DecodeArgs {
   float* ws_o;   // V2: [B, Hq, splits, d]; V1: [B, H, splits, 2 branches, 2d]
   float* ws_ml;  // V2: [B, Hq, splits, 2];  V1: [B, H, splits, 2 branches, 2]
   int* dev_status;
+  // element extents of q, the caches (or page pools), out, the two workspace parts and the
+  // block table, and the bounds-checked build's status word (see in_bounds in common.cuh)
+  int64_t ext_q, ext_kv, ext_out, ext_ws_o, ext_ws_ml, ext_bt;
+  int* dbg_status;
 };
 
 cudaError_t launch_lambda(const float* lq1, const float* lk1, const float* lq2, const float* lk2,

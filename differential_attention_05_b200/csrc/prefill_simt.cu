@@ -58,9 +58,11 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_f32_kernel(PrefillArgs a)
     k2 = k + krow0 + g2 * a.ks[2];
     vb = v + vrow0 + g1 * a.vs[2];
   }
+  const bool q_ok = in_bounds(q1 - q, d, a.ext_q, a.dev_status, a.dbg_status) &&
+                    in_bounds(q2 - q, d, a.ext_q, a.dev_status, a.dbg_status);
   for (int c = lane; c < d; c += 32) {
-    qs[warp][0][c] = q1[c];
-    qs[warp][1][c] = q2[c];
+    qs[warp][0][c] = q_ok ? q1[c] : 0.f;
+    qs[warp][1][c] = q_ok ? q2[c] : 0.f;
   }
   __syncwarp();
 
@@ -77,7 +79,8 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_f32_kernel(PrefillArgs a)
   for (int j0 = key_lo; j0 < n_keys; j0 += 32) {
     const int j = j0 + lane;
     float s1 = -INFINITY, s2 = -INFINITY;
-    if (j < n_keys) {
+    if (j < n_keys && in_bounds(k1 + (int64_t)j * a.ks[1] - k, d, a.ext_k, a.dev_status, a.dbg_status) &&
+        in_bounds(k2 + (int64_t)j * a.ks[1] - k, d, a.ext_k, a.dev_status, a.dbg_status)) {
       const float4* kr1 = reinterpret_cast<const float4*>(k1 + (int64_t)j * a.ks[1]);
       const float4* kr2 = reinterpret_cast<const float4*>(k2 + (int64_t)j * a.ks[1]);
       const float4* qa = reinterpret_cast<const float4*>(qs[warp][0]);
@@ -113,10 +116,11 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_f32_kernel(PrefillArgs a)
       const float w1 = __shfl_sync(0xffffffffu, p1, jj);
       const float w2 = __shfl_sync(0xffffffffu, p2, jj);
       const float* vr = vb + (int64_t)(j0 + jj) * a.vs[1];
+      const bool v_ok = in_bounds(vr - v, dv, a.ext_v, a.dev_status, a.dbg_status);
 #pragma unroll
       for (int t = 0; t < kPerLane; ++t) {
         const int c = lane + 32 * t;
-        if (c < dv) {
+        if (c < dv && v_ok) {
           const float x = vr[c];
           acc1[t] = fmaf(w1, x, acc1[t]);
           acc2[t] = fmaf(w2, x, acc2[t]);
@@ -140,12 +144,13 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_f32_kernel(PrefillArgs a)
 #pragma unroll
     for (int t = 0; t < kPerLane; ++t) o[t] = o[t] / r * sc;
   }
-  float* ob = static_cast<float*>(a.out) + (int64_t)sr.bc * a.os[0] +
-              (int64_t)(sr.qrow0 + i) * a.os[1] + u * a.os[2];
+  const int64_t o_off = (int64_t)sr.bc * a.os[0] + (int64_t)(sr.qrow0 + i) * a.os[1] + u * a.os[2];
+  float* ob = static_cast<float*>(a.out) + o_off;
+  const bool o_ok = in_bounds(o_off, dv, a.ext_out, a.dev_status, a.dbg_status);
 #pragma unroll
   for (int t = 0; t < kPerLane; ++t) {
     const int c = lane + 32 * t;
-    if (c < dv) ob[c] = o[t];
+    if (c < dv && o_ok) ob[c] = o[t];
   }
 }
 

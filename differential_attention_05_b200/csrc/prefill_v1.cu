@@ -460,9 +460,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // registers of the key loop free)
     const int o_nq = VARLEN ? ms.seq_nq : a.N, o_b = VARLEN ? ms.seq_bc : b;
     const int o_q0 = VARLEN ? ms.seq_q0 : 0;
-    if (ok && qi < o_nq) {
-      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)o_b * a.os[0] +
-                          (int64_t)(o_q0 + qi) * a.os[1] + (int64_t)u * a.os[2] + wg * 64;
+    const int64_t o_off = (int64_t)o_b * a.os[0] + (int64_t)(o_q0 + qi) * a.os[1] +
+                          (int64_t)u * a.os[2] + wg * 64;
+    if (ok && qi < o_nq && in_bounds(o_off, 64, a.ext_out, a.dev_status, a.dbg_status)) {
+      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + o_off;
       uint4* o4 = reinterpret_cast<uint4*>(ob);
 #pragma unroll
       for (int v = 0; v < 8; ++v) {

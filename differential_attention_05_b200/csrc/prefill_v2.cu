@@ -473,10 +473,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float y[64];  // the output, or (STATS) the incoming gradient dy of the same columns
     float e1 = 0.f, e2 = 0.f;
     if constexpr (STATS) {
-      if (ok && qi < a.N) {
+      const int64_t dy_off = (int64_t)b * a.st_dys[0] + (int64_t)qi * a.st_dys[1] +
+                             (int64_t)u * a.st_dys[2] + hh * 64;
+      if (ok && qi < a.N && in_bounds(dy_off, 64, a.ext_st_dy, a.dev_status, a.dbg_status)) {
         const uint4* g4 = reinterpret_cast<const uint4*>(
-            static_cast<const __nv_bfloat16*>(a.st_dy) + (int64_t)b * a.st_dys[0] +
-            (int64_t)qi * a.st_dys[1] + (int64_t)u * a.st_dys[2] + hh * 64);
+            static_cast<const __nv_bfloat16*>(a.st_dy) + dy_off);
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
           const uint4 w = g4[v];
@@ -519,18 +520,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       e2 += __shfl_xor_sync(FULL, e2, 16);
       if (ok && hh == 0 && qi < a.N) {
         const int64_t r = ((int64_t)b * a.units + u) * a.st_rows + qi;
-        *reinterpret_cast<float4*>(a.st + r * 4) =
-            make_float4(m1 + log2f(l1), m2 + log2f(l2), e1, e2);
-        a.st_dl[((int64_t)b * a.units + u) * a.N + qi] = -e2;
+        const int64_t rl = ((int64_t)b * a.units + u) * a.N + qi;
+        if (in_bounds(r * 4, 4, a.ext_st, a.dev_status, a.dbg_status))
+          *reinterpret_cast<float4*>(a.st + r * 4) =
+              make_float4(m1 + log2f(l1), m2 + log2f(l2), e1, e2);
+        if (in_bounds(rl, 1, a.ext_st_dl, a.dev_status, a.dbg_status)) a.st_dl[rl] = -e2;
       }
     }
     // (a variable-length tile reads its sequence back from shared memory, keeping the
     // registers of the key loop free)
     const int o_nq = VARLEN ? ms.seq_nq : a.N, o_b = VARLEN ? ms.seq_bc : b;
     const int o_q0 = VARLEN ? ms.seq_q0 : 0;
-    if (!STATS && ok && qi < o_nq) {
-      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + (int64_t)o_b * a.os[0] +
-                          (int64_t)(o_q0 + qi) * a.os[1] + (int64_t)u * a.os[2] + hh * 64;
+    const int64_t o_off = (int64_t)o_b * a.os[0] + (int64_t)(o_q0 + qi) * a.os[1] +
+                          (int64_t)u * a.os[2] + hh * 64;
+    if (!STATS && ok && qi < o_nq && in_bounds(o_off, 64, a.ext_out, a.dev_status, a.dbg_status)) {
+      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + o_off;
       uint4* o4 = reinterpret_cast<uint4*>(ob);
 #pragma unroll
       for (int v = 0; v < 8; ++v) {

@@ -27,7 +27,8 @@
  * diffattn_fwd_decode (V2), diffattn_fwd_decode_v1, diffattn_fwd_decode_paged (block
  * table), diffattn_fwd_decode_static, diffattn_decode_workspace_size; diffattn_bwd_prefill,
  * diffattn_bwd_workspace_size, diffattn_lambda_bwd (training); diffattn_selftest_timeout
- * (the bounded-wait path), diffattn_selftest_exp2 (the FMA-pipe 2^x); diffattn_version,
+ * (the bounded-wait path), diffattn_selftest_exp2 (the FMA-pipe 2^x),
+ * diffattn_debug_bounds_violations (the bounds-checked build); diffattn_version,
  * diffattn_status_string.
  *
  * Conventions for every entry point
@@ -431,6 +432,25 @@ int diffattn_selftest_timeout(int* dev_status, int timeout_ms, void* stream);
  * DIFFATTN_ERR_CUDA if the launch fails, else DIFFATTN_OK (asynchronous on `stream`).
  */
 int diffattn_selftest_exp2(const float* x, float* y, float* y_ref, int n, void* stream);
+
+/*
+ * diffattn_debug_bounds_violations -- the bounds-checked build's count of skipped accesses.
+ * (A diagnostic of this library, for tests; the pages have no counterpart.)
+ *
+ * The library can be built a second time with every raw global-memory access of its kernels
+ * (the ones that do not go through a TMA tensor map, which bounds its own copies) checked
+ * against the extent of the tensor it touches, as computed on the host from the call's
+ * shapes and strides: libdiffattn_debug.so (python -m differential_attention_05_b200.build
+ * --debug). An access outside its tensor is skipped, DIFFATTN_ERR_INVALID_ARG goes to the
+ * call's dev_status (when given), and a device-wide counter is incremented; nothing traps.
+ * This entry point copies that counter to *count (a HOST int) and resets it; it waits for
+ * the device to finish its work first (cudaMemcpy and cudaDeviceSynchronize).
+ *
+ * Returns DIFFATTN_OK in the bounds-checked build, DIFFATTN_ERR_UNSUPPORTED (with *count =
+ * 0) in the normal build, DIFFATTN_ERR_INVALID_ARG for a null count, DIFFATTN_ERR_CUDA if
+ * the copy fails.
+ */
+int diffattn_debug_bounds_violations(int* count);
 
 #ifdef __cplusplus
 }

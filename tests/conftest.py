@@ -27,3 +27,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    # Under the bounds-checked library (DIFFATTN_EXPECT_NO_VIOLATIONS=1, set by
+    # tests/test_gpu_bounds_checked.py for its child run), every kernel access must have
+    # stayed inside its tensor: a non-zero count fails the session.
+    if os.environ.get("DIFFATTN_EXPECT_NO_VIOLATIONS") != "1":
+        return
+    import differential_attention_05_b200 as da
+    n = da.diffattn_debug_bounds_violations()
+    print(f"\nbounds-checked library: {n} out-of-range accesses skipped")
+    if n is None or n != 0:
+        session.exitstatus = 1

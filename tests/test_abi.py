@@ -225,6 +225,13 @@ def test_selftest_exp2_rejects(lib):
     assert f(None, None, None, 0, None) == 0  # nothing to do, nothing launched
 
 
+def test_debug_bounds_violations_normal_build(lib):
+    f = lib.diffattn_debug_bounds_violations
+    assert f(None) == -1
+    n = ctypes.c_int32(7)
+    assert f(ctypes.byref(n)) == -2 and n.value == 0  # the normal build counts nothing
+
+
 def _paged(page_size=16, num_pages=64, max_pages=8, strides=(16 * 8 * 128, 8 * 128, 128)):
     pk = B.PagedKV()
     pk.page_size, pk.num_pages, pk.max_pages_per_seq = page_size, num_pages, max_pages
