@@ -16,6 +16,7 @@
 // ("Differential Attention (V2)", The Concept: DiffAttn = (A_1 - lambda A_2) V).
 #include "common.cuh"
 #include "kernels.h"
+#include "tma_host.cuh"
 
 namespace diffattn {
 
@@ -29,13 +30,17 @@ constexpr int STAGES = 3;
 constexpr int ROW_BYTES = D * 2;
 constexpr int TILE_BYTES = CH * ROW_BYTES;   // 16 KB
 constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K + V
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+constexpr int HALF_BYTES = CH * 128;         // one 64-column half of a tile: [64 rows x 128 B]
 constexpr int CHUNKS16_PER_ROW = ROW_BYTES / 16;  // 16
-static_assert(SMEM_BYTES >= WARPS * (G * D + 2 * G) * 4, "merge scratch must fit");
+static_assert(STAGES * STAGE_BYTES >= WARPS * (G * D + 2 * G) * 4, "merge scratch must fit");
 }  // namespace
 
+// A 64-key tile (K or V) in shared memory: two 64-column halves of [64 rows x 128 B] in
+// the 128-byte swizzle TMA writes (16-byte chunk j of row r at chunk position j ^ (r % 8)),
+// so the ldmatrix reads of 8 rows x 16 bytes hit 8 different bank groups.
 __device__ __forceinline__ uint32_t swz(int row, int c16) {
-  return (uint32_t)(row * ROW_BYTES + ((c16 ^ (row & 7)) << 4));
+  return (uint32_t)((c16 >> 3) * HALF_BYTES + row * 128 + (((c16 & 7) ^ (row & 7)) << 4));
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -62,11 +67,24 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a2
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
 }
 
-// PAGED: the cache is a page pool addressed through a block table (DecodeArgs); the
-// contiguous instantiation has none of that code.
-template <bool PAGED>
-__global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) {
-  extern __shared__ __align__(1024) uint8_t smem[];
+// MODE: the cache layout and how it is loaded.
+//   kContig   contiguous cache [B, L, Hkv, d]: TMA boxes of 64 rows (zero fill past L);
+//   kPagedTma page pool with pages of >= 8 tokens: TMA boxes of min(page size, 64) rows,
+//             one per page of the chunk, each landing on a 1024-byte boundary;
+//   kPagedCp  page pool with pages of 1, 2 or 4 tokens: 16-byte cp.async copies row by row.
+// Rows past the entry's keys are zeroed in shared memory before use (V rows enter the P.V
+// sums with weight 0, and 0 times a stale non-finite value would not be 0).
+constexpr int kContig = 0, kPagedTma = 1, kPagedCp = 2;
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 2)
+    decode_split_kernel(const __grid_constant__ TcMaps maps, DecodeArgs a) {
+  constexpr bool PAGED = MODE != kContig;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ uint64_t full[STAGES];   // TMA modes: the chunk in stage s has landed
+  __shared__ uint64_t bad_box[STAGES];  // kPagedTma: boxes of the chunk in stage s not loaded
+  __shared__ int abort_flag;
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, tq = lane & 3;  // mma fragment row / column-pair index
@@ -91,9 +109,9 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
   constexpr int RSTEP = THREADS / CHUNKS16_PER_ROW;               // rows covered by one pass of the block
   constexpr int ROWS_T = CH / RSTEP;                   // rows per thread and tensor
   static_assert(THREADS % CHUNKS16_PER_ROW == 0 && CH % RSTEP == 0, "copy layout");
-  int pid[PAGED ? ROWS_T : 1];
+  int pid[MODE == kPagedCp ? ROWS_T : 1];
   auto fetch_ids = [&](int c) {
-    if constexpr (PAGED) {
+    if constexpr (MODE == kPagedCp) {
       const int tok0 = t_begin + c * CH + tid / CHUNKS16_PER_ROW;
 #pragma unroll
       for (int i = 0; i < ROWS_T; ++i) {
@@ -105,8 +123,8 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
     }
   };
 
-  // issue the copies of chunk c into stage c % STAGES (zero-fill past t_end)
-  auto load_chunk = [&](int c) {
+  // kPagedCp: issue the copies of chunk c into stage c % STAGES (zero-fill past t_end)
+  auto load_chunk_cp = [&](int c) {
     uint8_t* st = smem + (c % STAGES) * STAGE_BYTES;
     const int tok0 = t_begin + c * CH;
 #pragma unroll
@@ -135,6 +153,108 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
     }
   };
 
+  // kPagedTma: lane i % 32 of warp 0 reads the page ids of box i of a chunk one chunk ahead
+  // of its copies (fetch_ids_tma), so the table reads overlap the work on the current chunk;
+  // -1 marks a box wholly past t_end
+  int pid_t[2] = {-1, -1};
+  auto fetch_ids_tma = [&](int c) {
+    if constexpr (MODE == kPagedTma) {
+      const int pshift = min(a.page_shift, 6), pr = 1 << pshift, nbox = CH >> pshift;
+      const int tok0 = t_begin + c * CH;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int i = lane + 32 * r;
+        const int t = tok0 + i * pr;
+        pid_t[r] = -1;
+        if (i < nbox && t < t_end) {
+          const int64_t bi = (int64_t)b * a.bt_stride + (t >> a.page_shift);
+          pid_t[r] = in_bounds(bi, 1, a.ext_bt, a.dev_status, a.dbg_status) ? __ldg(a.block_table + bi)
+                                                                             : a.num_pages;
+        }
+      }
+    }
+  };
+
+  // TMA modes: warp 0 issues the copies of chunk c into stage c % STAGES. Paged: box i
+  // (rows i * pr .. of the chunk) is one page's run of pr tokens; lane i % 32 issues its
+  // copies with the page id fetched before. A box wholly past t_end is not loaded (zeroed
+  // after the wait), nor is one whose page id lies outside the pool (zeroed and reported).
+  auto load_chunk_tma = [&](int c) {
+    uint8_t* st = smem + (c % STAGES) * STAGE_BYTES;
+    uint64_t* bar = &full[c % STAGES];
+    const int tok0 = t_begin + c * CH;
+    if constexpr (MODE == kContig) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar, 2 * TILE_BYTES);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          tma_load_4d(st + hf * HALF_BYTES, &maps.k, bar, 64 * hf, g, tok0, b);
+          tma_load_4d(st + TILE_BYTES + hf * HALF_BYTES, &maps.v, bar, 64 * hf, g, tok0, b);
+        }
+      }
+    } else if constexpr (MODE == kPagedTma) {
+      const int pr = 1 << min(a.page_shift, 6), nbox = CH / pr;
+      const int pmask = (1 << a.page_shift) - 1;
+      int ids[2];
+      bool load[2] = {false, false}, bad[2] = {false, false};
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int i = lane + 32 * r;
+        if (i < nbox && tok0 + i * pr < t_end) {
+          ids[r] = pid_t[r];
+          load[r] = (unsigned)ids[r] < (unsigned)a.num_pages;
+          bad[r] = !load[r];
+        }
+      }
+      const uint32_t lmask0 = __ballot_sync(0xffffffffu, load[0]), lmask1 = __ballot_sync(0xffffffffu, load[1]);
+      const uint32_t bmask0 = __ballot_sync(0xffffffffu, bad[0]), bmask1 = __ballot_sync(0xffffffffu, bad[1]);
+      if (lane == 0) {
+        bad_box[c % STAGES] = (uint64_t)bmask0 | ((uint64_t)bmask1 << 32);
+        const int nl = __popc(lmask0) + __popc(lmask1);
+        mbar_arrive_expect_tx(bar, (uint32_t)(nl * pr * 128 * 4));  // K and V, both halves
+      }
+      __syncwarp();
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        if (!load[r]) continue;
+        const int i = lane + 32 * r;
+        const int row = (tok0 + i * pr) & pmask;  // first row of the run inside its page
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          tma_load_4d(st + hf * HALF_BYTES + i * pr * 128, &maps.k, bar, 64 * hf, g, row, ids[r]);
+          tma_load_4d(st + TILE_BYTES + hf * HALF_BYTES + i * pr * 128, &maps.v, bar, 64 * hf, g, row, ids[r]);
+        }
+      }
+      if (bmask0 | bmask1) bad_page = true;
+    }
+  };
+
+  // TMA modes, after chunk c has landed: zero the V rows of the chunk past t_end (and, for a
+  // page outside the pool, its K and V rows), so that they add exactly 0 to the P.V sums
+  auto zero_rows = [&](int c) {
+    if constexpr (MODE != kPagedCp) {
+      uint8_t* st = smem + (c % STAGES) * STAGE_BYTES;
+      const int valid = t_end - (t_begin + c * CH);  // rows < valid are keys of the entry
+      uint64_t bad = 0;
+      int pr = CH;
+      if constexpr (MODE == kPagedTma) {
+        bad = bad_box[c % STAGES];
+        pr = 1 << min(a.page_shift, 6);
+      }
+      if (valid < CH || bad) {
+        for (int idx = tid; idx < 2 * CH * CHUNKS16_PER_ROW; idx += THREADS) {
+          const int tensor = idx / (CH * CHUNKS16_PER_ROW);
+          const int rem = idx % (CH * CHUNKS16_PER_ROW);
+          const int row = rem / CHUNKS16_PER_ROW, c16 = rem % CHUNKS16_PER_ROW;
+          const bool bad_row = (bad >> (row / pr)) & 1;
+          if ((tensor == 1 && row >= valid) || bad_row)
+            *reinterpret_cast<uint4*>(st + tensor * TILE_BYTES + swz(row, c16)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async();  // before a later TMA copy rewrites the stage
+      }
+    }
+  };
+
   // Q fragments of the 8 heads (A operand, rows 0..7), all 8 k-steps of d = 128
   uint32_t qa[8][2];
   {
@@ -154,24 +274,69 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
 #pragma unroll
   for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
 
+  if constexpr (MODE != kPagedCp) {
+    if (tid == 0) {
+      for (int st = 0; st < STAGES; ++st) mbar_init(&full[st], 1);
+      abort_flag = 0;
+      fence_barrier_init();
+    }
+    __syncthreads();
+  }
+  int issued = 0;  // TMA modes: chunks whose copies were issued
 #pragma unroll
   for (int c = 0; c < STAGES - 1; ++c) {
-    if (c < n_chunks) {
-      fetch_ids(c);
-      load_chunk(c);
+    if constexpr (MODE == kPagedCp) {
+      if (c < n_chunks) {
+        fetch_ids(c);
+        load_chunk_cp(c);
+      }
+      cp_async_commit();
+    } else if (c < n_chunks) {
+      if (warp == 0) {
+        fetch_ids_tma(c);
+        load_chunk_tma(c);
+      }
+      issued = c + 1;
     }
-    cp_async_commit();
   }
-  if (STAGES - 1 < n_chunks) fetch_ids(STAGES - 1);
+  if constexpr (MODE == kPagedCp) {
+    if (STAGES - 1 < n_chunks) fetch_ids(STAGES - 1);
+  } else {
+    if (STAGES - 1 < n_chunks && warp == 0) fetch_ids_tma(STAGES - 1);
+  }
 
   for (int c = 0; c < n_chunks; ++c) {
-    if (c + STAGES - 1 < n_chunks) {
-      load_chunk(c + STAGES - 1);
-      if (c + STAGES < n_chunks) fetch_ids(c + STAGES);
+    if constexpr (MODE == kPagedCp) {
+      if (c + STAGES - 1 < n_chunks) {
+        load_chunk_cp(c + STAGES - 1);
+        if (c + STAGES < n_chunks) fetch_ids(c + STAGES);
+      }
+      cp_async_commit();
+      cp_async_wait<STAGES - 1>();
+      __syncthreads();
+    } else {
+      // stage (c + 2) % STAGES was released by the __syncthreads ending iteration c - 1
+      if (c + STAGES - 1 < n_chunks) {
+        if (warp == 0) {
+          load_chunk_tma(c + STAGES - 1);
+          if (c + STAGES < n_chunks) fetch_ids_tma(c + STAGES);
+        }
+        issued = c + STAGES;
+      }
+      const bool ok = mbar_wait(&full[c % STAGES], (c / STAGES) & 1, &abort_flag);
+      if (!__syncthreads_and(ok)) {
+        // a copy that never landed: let the ones in flight finish before the shared memory
+        // is reused below, and report
+        if (tid == 0) {
+          for (int cc = c; cc < issued; ++cc) mbar_wait_drain(&full[cc % STAGES], (cc / STAGES) & 1);
+          report_status(a.dev_status, DIFFATTN_ERR_TIMEOUT);
+        }
+        __syncthreads();
+        break;
+      }
+      zero_rows(c);
+      __syncthreads();
     }
-    cp_async_commit();
-    cp_async_wait<STAGES - 1>();
-    __syncthreads();
 
     const uint32_t kst = smem_u32(smem + (c % STAGES) * STAGE_BYTES);
     const uint32_t vst = kst + TILE_BYTES;
@@ -238,7 +403,7 @@ __global__ void __launch_bounds__(THREADS, 2) decode_split_kernel(DecodeArgs a) 
     }
     __syncthreads();  // stage c % STAGES is refilled on the next iteration
   }
-  cp_async_wait<0>();
+  if constexpr (MODE == kPagedCp) cp_async_wait<0>();
   __syncthreads();
   if (bad_page) report_status(a.dev_status, DIFFATTN_ERR_INVALID_ARG);
 
@@ -339,19 +504,35 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   if (dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(decode_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(decode_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    const void* fns[3] = {(const void*)decode_split_kernel<kContig>, (const void*)decode_split_kernel<kPagedTma>,
+                          (const void*)decode_split_kernel<kPagedCp>};
+    for (const void* fn : fns) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+    }
     if (dev < 64) attr_set[dev] = true;
   }
+  // tensor maps: K and V as {d, Hkv, rows, batch entries} (contiguous) or {d, Hkv, page size,
+  // pages} (pool), 64-column boxes of 64 rows (contiguous) or of one page's run of up to 64
+  // rows, 128-byte swizzle, zero fill outside the tensor
+  TcMaps maps = {};
+  const int ps = 1 << a.page_shift;
+  const int mode = !a.block_table ? kContig : (ps >= 8 ? kPagedTma : kPagedCp);
+  if (mode == kContig) {
+    if (!make_map(&maps.k, a.k, D, a.Hkv, a.L, a.B, a.kvs, CH)) return cudaErrorInvalidValue;
+    if (!make_map(&maps.v, a.v, D, a.Hkv, a.L, a.B, a.kvs, CH)) return cudaErrorInvalidValue;
+  } else if (mode == kPagedTma) {
+    const int pr = ps < CH ? ps : CH;
+    if (!make_map(&maps.k, a.k, D, a.Hkv, ps, a.num_pages, a.kvs, pr)) return cudaErrorInvalidValue;
+    if (!make_map(&maps.v, a.v, D, a.Hkv, ps, a.num_pages, a.kvs, pr)) return cudaErrorInvalidValue;
+  }
   dim3 grid(a.splits, a.Hkv, a.B);
-  if (a.block_table)
-    decode_split_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(a);
+  if (mode == kContig)
+    decode_split_kernel<kContig><<<grid, THREADS, SMEM_BYTES, stream>>>(maps, a);
+  else if (mode == kPagedTma)
+    decode_split_kernel<kPagedTma><<<grid, THREADS, SMEM_BYTES, stream>>>(maps, a);
   else
-    decode_split_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(a);
+    decode_split_kernel<kPagedCp><<<grid, THREADS, SMEM_BYTES, stream>>>(maps, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 grid2(a.Hq / 2, a.B);

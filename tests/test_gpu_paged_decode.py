@@ -30,7 +30,7 @@ def _paged(inp, page_size, kv_len, fill="nan", seed=5):
     return dev_tensor(kp), dev_tensor(vp), torch.from_numpy(bt).cuda()
 
 
-@pytest.mark.parametrize("page_size", [1, 16, 64, 256])
+@pytest.mark.parametrize("page_size", [1, 4, 8, 16, 64, 256])
 def test_v2_paged(page_size):
     L = 1000
     kv_len = [1000, 1, 513]
