@@ -23,6 +23,8 @@ from ._binding import (  # noqa: F401
     diffattn_bwd_prefill,
     diffattn_bwd_workspace_size,
     diffattn_lambda_bwd,
+    diffattn_fwd_prefill_train,
+    diffattn_bwd_prefill_saved,
     diffattn_fwd_decode,
     diffattn_fwd_decode_static,
     diffattn_fwd_decode_v1,
@@ -44,6 +46,8 @@ __all__ = [
     "diffattn_bwd_prefill",
     "diffattn_bwd_workspace_size",
     "diffattn_lambda_bwd",
+    "diffattn_fwd_prefill_train",
+    "diffattn_bwd_prefill_saved",
     "diffattn_fwd_decode",
     "diffattn_fwd_decode_static",
     "diffattn_fwd_decode_v1",

@@ -36,6 +36,8 @@ EXPORTS = (
     "diffattn_bwd_workspace_size",
     "diffattn_bwd_prefill",
     "diffattn_lambda_bwd",
+    "diffattn_fwd_prefill_train",
+    "diffattn_bwd_prefill_saved",
     "diffattn_decode_workspace_size",
     "diffattn_fwd_decode",
     "diffattn_fwd_decode_static",
@@ -127,6 +129,12 @@ def load_library():
     lib.diffattn_bwd_prefill.restype = i32
     lib.diffattn_bwd_prefill.argtypes = [ctypes.POINTER(PrefillParams), vp, vp, vp, f32p, f32p, vp,
                                          vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
+    lib.diffattn_fwd_prefill_train.restype = i32
+    lib.diffattn_fwd_prefill_train.argtypes = [ctypes.POINTER(PrefillParams), vp, vp, vp, f32p, vp, vp,
+                                               f32p, vp, vp]
+    lib.diffattn_bwd_prefill_saved.restype = i32
+    lib.diffattn_bwd_prefill_saved.argtypes = [ctypes.POINTER(PrefillParams), vp, vp, vp, f32p, vp, vp,
+                                               f32p, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
     lib.diffattn_lambda_bwd.restype = i32
     lib.diffattn_lambda_bwd.argtypes = [f32p, f32p, f32p, f32p, i32, i32, f32p, vp, vp, vp, vp, vp]
     lib.diffattn_decode_workspace_size.restype = i32
@@ -332,6 +340,56 @@ def diffattn_bwd_prefill(q, k, v, lam, dout, lambda_init=None, causal=True, appl
                                   _ptr(dl), _ptr(workspace), ws_bytes, _ptr(dev_status),
                                   _stream(stream))
     _check("diffattn_bwd_prefill", rc)
+    return dq, dk, dv, dl
+
+
+def diffattn_fwd_prefill_train(q, k, v, lam, out=None, o2=None, lse=None, causal=True, window=0,
+                               dev_status=None, stream=None):
+    """diffattn_fwd_prefill for training (V2 bf16, d = 128; see include/diffattn.h): returns
+    (out, o2, lse) -- the output, the branch-2 output O_2 / l_2 in out's layout, and float32
+    [B, Hq/2, N, 2] log2-domain log-sum-exps of both branches."""
+    import torch
+    lib = load_library()
+    B, N, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, N, Hq // 2, d), dtype=q.dtype, device=q.device)
+    if o2 is None:
+        o2 = torch.empty_like(out)
+    if lse is None:
+        lse = torch.empty((B, Hq // 2, N, 2), dtype=torch.float32, device=q.device)
+    if o2.stride() != out.stride():
+        raise ValueError("o2 must have out's layout")
+    p = prefill_params(q, k, v, out, causal, None, 1e-5, window)
+    rc = lib.diffattn_fwd_prefill_train(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out),
+                                        _ptr(o2), _ptr(lse), _ptr(dev_status), _stream(stream))
+    _check("diffattn_fwd_prefill_train", rc)
+    return out, o2, lse
+
+
+def diffattn_bwd_prefill_saved(q, k, v, lam, out, o2, lse, dout, causal=True, window=0,
+                               workspace=None, dev_status=None, stream=None, grads=None):
+    """diffattn_bwd_prefill from diffattn_fwd_prefill_train's (out, o2, lse) (see
+    include/diffattn.h): no recompute of the forward. Returns float32 (dq, dk, dv, dlambda)."""
+    import torch
+    lib = load_library()
+    if out.stride() != dout.stride() or o2.stride() != dout.stride():
+        raise ValueError("out, o2 and dout must share one layout")
+    p = prefill_params(q, k, v, dout, causal, None, 1e-5, window)
+    if grads is None:
+        grads = (torch.empty(q.shape, dtype=torch.float32, device=q.device),
+                 torch.empty(k.shape, dtype=torch.float32, device=q.device),
+                 torch.empty(v.shape, dtype=torch.float32, device=q.device),
+                 torch.empty(lam.shape, dtype=torch.float32, device=q.device))
+    dq, dk, dv, dl = grads
+    need = diffattn_bwd_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib.diffattn_bwd_prefill_saved(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out),
+                                        _ptr(o2), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                        _ptr(dl), _ptr(workspace), ws_bytes, _ptr(dev_status),
+                                        _stream(stream))
+    _check("diffattn_bwd_prefill_saved", rc)
     return dq, dk, dv, dl
 
 

@@ -317,6 +317,61 @@ int diffattn_bwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   return from_cuda(tc ? launch_backward_tc(g, workspace, s) : launch_backward(g, workspace, s));
 }
 
+int diffattn_fwd_prefill_train(const diffattn_prefill_params* p, const void* q, const void* k,
+                               const void* v, const float* lambda, void* out, void* o2, float* lse,
+                               int* dev_status, void* stream) {
+  if (!p) return DIFFATTN_ERR_INVALID_ARG;
+  if (p->variant != DIFFATTN_V2 || p->dtype != DIFFATTN_BF16 || p->head_dim != 128)
+    return DIFFATTN_ERR_UNSUPPORTED;
+  PrefillArgs a;
+  bool empty = false;
+  int rc = prefill_setup(p, nullptr, nullptr, 0, q, k, v, lambda, nullptr, out, dev_status, &a, &empty);
+  if (rc != DIFFATTN_OK || empty) return rc;
+  if (!o2 || !lse) return DIFFATTN_ERR_INVALID_ARG;
+  if (o2 == out || o2 == q || o2 == k || o2 == v) return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(o2) || !aligned16(lse)) return DIFFATTN_ERR_MISALIGNED;
+  if (a.Nk > (1 << 24) || p->seqlen > (1 << 24)) return DIFFATTN_ERR_UNSUPPORTED;
+  a.tr_o2 = o2;
+  a.tr_lse = lse;
+  a.ext_tr_lse = (int64_t)a.B * a.units * a.N * 2;
+  return from_cuda(launch_prefill_v2_train(a, static_cast<cudaStream_t>(stream)));
+}
+
+int diffattn_bwd_prefill_saved(const diffattn_prefill_params* p, const void* q, const void* k,
+                               const void* v, const float* lambda, const void* out, const void* o2,
+                               const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                               float* dlambda, void* workspace, size_t workspace_bytes,
+                               int* dev_status, void* stream) {
+  int rc = bwd_check(p);
+  if (rc != DIFFATTN_OK) return rc;
+  if (p->variant != DIFFATTN_V2 || p->dtype != DIFFATTN_BF16 || p->head_dim != 128)
+    return DIFFATTN_ERR_UNSUPPORTED;
+  BwdArgs g;
+  memset(&g, 0, sizeof(g));
+  bool empty = false;
+  rc = prefill_setup(p, nullptr, nullptr, 0, q, k, v, lambda, nullptr, dout, dev_status, &g.f, &empty);
+  if (rc != DIFFATTN_OK || empty) return rc;
+  if (!out || !o2 || !lse || !dout || !dq || !dk || !dv || !dlambda) return DIFFATTN_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(o2) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return DIFFATTN_ERR_MISALIGNED;
+  const PrefillArgs& a = g.f;
+  const size_t need = bwd_tc_workspace_bytes(a.B, a.N, a.units);
+  if (!workspace || workspace_bytes < need) return DIFFATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIFFATTN_ERR_MISALIGNED;
+  g.bf16 = 1;
+  g.dy = dout;
+  memcpy(g.dys, p->o_strides, sizeof(g.dys));
+  g.dq = dq;
+  g.dk = dk;
+  g.dv = dv;
+  g.dlambda = dlambda;
+  g.ext_dq = (int64_t)a.B * a.N * a.Hq * a.d;
+  g.ext_dk = (int64_t)a.B * a.Nk * a.Hkv * a.d;
+  g.ext_dv = (int64_t)a.B * a.Nk * a.Hkv * a.dv;
+  g.ext_ws = (int64_t)(workspace_bytes / sizeof(float));
+  return from_cuda(launch_backward_tc_saved(g, out, o2, lse, workspace, static_cast<cudaStream_t>(stream)));
+}
+
 int diffattn_lambda_bwd(const float* lq1, const float* lk1, const float* lq2, const float* lk2,
                         int n_heads, int dim, const float* dlambda, float* dlq1, float* dlk1,
                         float* dlq2, float* dlk2, void* stream) {

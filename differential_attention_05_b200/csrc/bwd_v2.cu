@@ -634,36 +634,67 @@ size_t bwd_tc_workspace_bytes(int B, int N, int units) {
          up256((size_t)B * units * N * sizeof(float));
 }
 
-cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream) {
+namespace {
+
+// The statistics rows of the backward from a training forward's saved outputs instead of a
+// recompute: delta_2 = dy . (O_2 / l_2) and delta_1 = dy . (O_1 / l_1) with
+// O_1 / l_1 = out + lambda O_2 / l_2, per (batch entry, query, pair); one warp per row, four
+// columns per lane. Writes (lse_1, lse_2, delta_1, delta_2) and the dlambda share -delta_2 in
+// the layout of the statistics pass.
+__global__ void __launch_bounds__(256) bwd_saved_stats_kernel(BwdArgs g, const __nv_bfloat16* out,
+                                                             const __nv_bfloat16* o2, const float* lse) {
   const PrefillArgs& a = g.f;
-  if (a.cu_q || a.variant != DIFFATTN_V2 || a.d != 128) return cudaErrorNotSupported;
-  uint8_t* w = static_cast<uint8_t*>(workspace);
-  const size_t st_bytes = up256((size_t)a.B * a.units * (a.N + 64) * 4 * sizeof(float));
-  g.w_st = reinterpret_cast<float*>(w);
-  g.w_dl = reinterpret_cast<float*>(w + st_bytes);
-  g.w_do = nullptr;
-  g.w_base = g.w_st;
-  // 1. statistics: the forward kernel in its statistics mode
-  PrefillArgs fa = a;
-  fa.out = nullptr;
-  fa.st_dy = g.dy;
-  for (int i = 0; i < 3; ++i) fa.st_dys[i] = g.dys[i];
-  fa.st = g.w_st;
-  fa.st_dl = g.w_dl;
-  fa.st_rows = a.N + 64;
-  fa.ext_st_dy = a.ext_out;  // dy has the output's layout
-  fa.ext_st = (int64_t)a.B * a.units * (a.N + 64) * 4;
-  fa.ext_st_dl = (int64_t)a.B * a.units * a.N;
-  cudaError_t e = launch_prefill_v2_stats(fa, stream);
-  if (e != cudaSuccess) return e;
-  // 2, 3. dK/dV and dQ: q [B, N, Hq, 128], k, v [B, N, Hkv, 128], dO = dy [B, N, Hq/2, 128]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * 8 + warp;  // (b * N + i) * units + u
+  if (r >= (int64_t)a.B * a.N * a.units) return;
+  const int u = (int)(r % a.units);
+  const int64_t bi = r / a.units;
+  const int i = (int)(bi % a.N), b = (int)(bi / a.N);
+  // out, o2 and dy share the output layout (strides a.os)
+  const int64_t off = (int64_t)b * a.os[0] + (int64_t)i * a.os[1] + (int64_t)u * a.os[2] + 4 * lane;
+  float e1 = 0.f, e2 = 0.f;
+  if (in_bounds(off, 4, a.ext_out, a.dev_status, a.dbg_status)) {
+    const uint2 wy = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(g.dy) + off);
+    const uint2 wo = *reinterpret_cast<const uint2*>(out + off);
+    const uint2 w2 = *reinterpret_cast<const uint2*>(o2 + off);
+    const float lam = a.lambda[u];
+    const uint32_t y4[2] = {wy.x, wy.y}, o4[2] = {wo.x, wo.y}, q4[2] = {w2.x, w2.y};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float dy = __uint_as_float(e ? (y4[h] & 0xffff0000u) : (y4[h] << 16));
+        const float ov = __uint_as_float(e ? (o4[h] & 0xffff0000u) : (o4[h] << 16));
+        const float o2v = __uint_as_float(e ? (q4[h] & 0xffff0000u) : (q4[h] << 16));
+        e2 = fmaf(dy, o2v, e2);
+        e1 = fmaf(dy, fmaf(lam, o2v, ov), e1);
+      }
+    }
+  }
+  e1 = warp_sum(e1);
+  e2 = warp_sum(e2);
+  if (lane == 0) {
+    const int64_t unit_row = (int64_t)b * a.units + u;
+    const int64_t sr = (unit_row * (a.N + 64) + i) * 4, lr = (unit_row * a.N + i) * 2;
+    if (in_bounds((g.w_st - g.w_base) + sr, 4, g.ext_ws, a.dev_status, a.dbg_status) &&
+        in_bounds(lr, 2, a.ext_tr_lse, a.dev_status, a.dbg_status))
+      *reinterpret_cast<float4*>(g.w_st + sr) = make_float4(lse[lr], lse[lr + 1], e1, e2);
+    if (in_bounds((g.w_dl - g.w_base) + unit_row * a.N + i, 1, g.ext_ws, a.dev_status, a.dbg_status))
+      g.w_dl[unit_row * a.N + i] = -e2;
+  }
+}
+
+// steps 2-4 of the tensor-core backward, once the statistics rows are in the workspace
+cudaError_t backward_tc_kernels(const BwdArgs& g, cudaStream_t stream) {
+  const PrefillArgs& a = g.f;
+  // dK/dV and dQ: q [B, N, Hq, 128], k, v [B, N, Hkv, 128], dO = dy [B, N, Hq/2, 128]
   BwdMaps maps;
   if (!make_map(&maps.q, a.q, 128, a.Hq, a.N, a.B, a.qs, 64)) return cudaErrorInvalidValue;
   if (!make_map(&maps.k, a.k, 128, a.Hkv, a.Nk, a.B, a.ks, 128)) return cudaErrorInvalidValue;
   if (!make_map(&maps.v, a.v, 128, a.Hkv, a.Nk, a.B, a.vs, 128)) return cudaErrorInvalidValue;
   if (!make_map(&maps.dy, g.dy, 128, a.units, a.N, a.B, g.dys, 64)) return cudaErrorInvalidValue;
   int dev = 0;
-  e = cudaGetDevice(&dev);
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   if (dev >= 64 || !attr_set[dev]) {
@@ -683,6 +714,53 @@ cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream) 
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_dlambda_reduce(g, stream);
+}
+
+void set_tc_workspace(BwdArgs& g, void* workspace) {
+  const PrefillArgs& a = g.f;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  const size_t st_bytes = up256((size_t)a.B * a.units * (a.N + 64) * 4 * sizeof(float));
+  g.w_st = reinterpret_cast<float*>(w);
+  g.w_dl = reinterpret_cast<float*>(w + st_bytes);
+  g.w_do = nullptr;
+  g.w_base = g.w_st;
+}
+
+}  // namespace
+
+cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream) {
+  const PrefillArgs& a = g.f;
+  if (a.cu_q || a.variant != DIFFATTN_V2 || a.d != 128) return cudaErrorNotSupported;
+  set_tc_workspace(g, workspace);
+  // 1. statistics: the forward kernel in its statistics mode
+  PrefillArgs fa = a;
+  fa.out = nullptr;
+  fa.st_dy = g.dy;
+  for (int i = 0; i < 3; ++i) fa.st_dys[i] = g.dys[i];
+  fa.st = g.w_st;
+  fa.st_dl = g.w_dl;
+  fa.st_rows = a.N + 64;
+  fa.ext_st_dy = a.ext_out;  // dy has the output's layout
+  fa.ext_st = (int64_t)a.B * a.units * (a.N + 64) * 4;
+  fa.ext_st_dl = (int64_t)a.B * a.units * a.N;
+  cudaError_t e = launch_prefill_v2_stats(fa, stream);
+  if (e != cudaSuccess) return e;
+  return backward_tc_kernels(g, stream);
+}
+
+cudaError_t launch_backward_tc_saved(BwdArgs g, const void* out, const void* o2, const float* lse,
+                                     void* workspace, cudaStream_t stream) {
+  const PrefillArgs& a = g.f;
+  if (a.cu_q || a.variant != DIFFATTN_V2 || a.d != 128) return cudaErrorNotSupported;
+  set_tc_workspace(g, workspace);
+  g.f.ext_tr_lse = (int64_t)a.B * a.units * a.N * 2;
+  const long long rows = (long long)a.B * a.N * a.units;
+  if ((rows + 7) / 8 > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  bwd_saved_stats_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+      g, static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(o2), lse);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return backward_tc_kernels(g, stream);
 }
 
 }  // namespace diffattn

@@ -42,10 +42,15 @@ struct PrefillArgs {
   float* st;
   float* st_dl;
   int st_rows;
+  // training forward (launch_prefill_v2_train): the branch-2 output O_2 / l_2 of every
+  // (query, pair) in out's layout and dtype, and lse[((b * units + u) * N + i) * 2 + 0..1],
+  // the log2-domain log-sum-exps of both branches
+  void* tr_o2;
+  float* tr_lse;
   // element extents (one past the largest element offset the shapes and strides reach) of
   // q, k, v, out and the statistics-pass tensors, and the bounds-checked build's own status
   // word (see in_bounds in common.cuh; unused by the normal build)
-  int64_t ext_q, ext_k, ext_v, ext_out, ext_st_dy, ext_st, ext_st_dl;
+  int64_t ext_q, ext_k, ext_v, ext_out, ext_st_dy, ext_st, ext_st_dl, ext_tr_lse;
   int* dbg_status;
 };
 
@@ -136,6 +141,7 @@ cudaError_t launch_prefill_f32(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_v1(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_v2_stats(const PrefillArgs& a, cudaStream_t stream);
+cudaError_t launch_prefill_v2_train(const PrefillArgs& a, cudaStream_t stream);
 
 // split-KV decode (V2, bf16, d = 128, 8 query heads per KV head)
 constexpr int kDecodeChunk = 64;  // keys per pipeline stage
@@ -151,6 +157,9 @@ cudaError_t launch_backward(BwdArgs g, void* workspace, cudaStream_t stream);
 cudaError_t launch_dlambda_reduce(const BwdArgs& g, cudaStream_t stream);
 size_t bwd_tc_workspace_bytes(int B, int N, int units);
 cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream);
+// the same from a training forward's saved O_2 / l_2 and log-sum-exps (no recompute)
+cudaError_t launch_backward_tc_saved(BwdArgs g, const void* out, const void* o2, const float* lse,
+                                     void* workspace, cudaStream_t stream);
 cudaError_t launch_lambda_bwd(const float* lq1, const float* lk1, const float* lq2,
                               const float* lk2, int n_heads, int dim, const float* dlam,
                               float* dlq1, float* dlk1, float* dlq2, float* dlk2,

@@ -107,7 +107,9 @@ __device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t bytes) {
 // takes its sizes from the parameters alone.
 // STATS: the statistics pass of the backward (fixed length only): the epilogue writes the
 // log-sum-exps and deltas described at PrefillArgs::st instead of the output.
-template <bool WINDOW, bool VARLEN, bool STATS = false>
+// TRAIN: the training forward (fixed length only): the output, and for the backward the
+// branch-2 output O_2 / l_2 (PrefillArgs::tr_o2) and both log-sum-exps (tr_lse).
+template <bool WINDOW, bool VARLEN, bool STATS = false, bool TRAIN = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_v2_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -512,7 +514,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             y[ch * 32 + e] = __fmaf_rn(ov[e], coef, __fmul_rn(dv[e], inv1));
           }
         }
+        if constexpr (TRAIN) {
+          // O_2 / l_2 of these 32 columns, in out's layout
+          const int64_t o2_off = (int64_t)b * a.os[0] + (int64_t)qi * a.os[1] + (int64_t)u * a.os[2] +
+                                 hh * 64 + ch * 32;
+          if (qi < a.N && in_bounds(o2_off, 32, a.ext_out, a.dev_status, a.dbg_status)) {
+            uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.tr_o2) + o2_off);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 w;
+              w.x = pack_bf16(ov[v * 8 + 0] * inv2, ov[v * 8 + 1] * inv2);
+              w.y = pack_bf16(ov[v * 8 + 2] * inv2, ov[v * 8 + 3] * inv2);
+              w.z = pack_bf16(ov[v * 8 + 4] * inv2, ov[v * 8 + 5] * inv2);
+              w.w = pack_bf16(ov[v * 8 + 6] * inv2, ov[v * 8 + 7] * inv2);
+              o4[v] = w;
+            }
+          }
+        }
       }
+    }
+    if constexpr (TRAIN) {
+      const int64_t rl = (((int64_t)b * a.units + u) * a.N + qi) * 2;
+      if (ok && hh == 0 && qi < a.N && in_bounds(rl, 2, a.ext_tr_lse, a.dev_status, a.dbg_status))
+        *reinterpret_cast<float2*>(a.tr_lse + rl) = make_float2(m1 + log2f(l1), m2 + log2f(l2));
     }
     if constexpr (STATS) {
       // the query's two halves add their column ranges; lse_b = m_b + log2 l_b (log2 domain)
@@ -595,6 +619,38 @@ cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream) {
     if (window) prefill_v2_kernel<true, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
     else prefill_v2_kernel<false, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   }
+  return cudaGetLastError();
+}
+
+// The training forward over the same tiles (fixed-length batches): out, tr_o2 and tr_lse
+// must be set.
+cudaError_t launch_prefill_v2_train(const PrefillArgs& a, cudaStream_t stream) {
+  if (a.variant != DIFFATTN_V2 || a.d != 128 || a.group % 2 != 0 || a.cu_q) return cudaErrorNotSupported;
+  if (!a.out || !a.tr_o2 || !a.tr_lse) return cudaErrorInvalidValue;
+  TcMaps maps;
+  if (!make_map(&maps.q, a.q, 128, a.Hq, a.N, a.B, a.qs, 16)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, 128, a.Hkv, a.Nk, a.B, a.ks, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, 128, a.Hkv, a.Nk, a.B, a.vs, BN)) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  if (dev >= 64 || !attr_set[dev]) {
+    const void* fns[2] = {(const void*)prefill_v2_kernel<false, false, false, true>,
+                          (const void*)prefill_v2_kernel<true, false, false, true>};
+    for (const void* fn : fns) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+    }
+    if (dev < 64) attr_set[dev] = true;
+  }
+  const long long tiles = (long long)((a.N + BM - 1) / BM) * a.units * a.B;
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const dim3 grid((unsigned)tiles);
+  if (a.causal && a.window > 0)
+    prefill_v2_kernel<true, false, false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  else
+    prefill_v2_kernel<false, false, false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   return cudaGetLastError();
 }
 

@@ -26,7 +26,8 @@
  * chunked, sliding window) and diffattn_fwd_prefill_varlen (packed sequences);
  * diffattn_fwd_decode (V2), diffattn_fwd_decode_v1, diffattn_fwd_decode_paged (block
  * table), diffattn_fwd_decode_static, diffattn_decode_workspace_size; diffattn_bwd_prefill,
- * diffattn_bwd_workspace_size, diffattn_lambda_bwd (training); diffattn_selftest_timeout
+ * diffattn_bwd_workspace_size, diffattn_fwd_prefill_train, diffattn_bwd_prefill_saved,
+ * diffattn_lambda_bwd (training); diffattn_selftest_timeout
  * (the bounded-wait path), diffattn_selftest_exp2 (the FMA-pipe 2^x),
  * diffattn_debug_bounds_violations (the bounds-checked build); diffattn_version,
  * diffattn_status_string.
@@ -222,6 +223,44 @@ int diffattn_bwd_prefill(const diffattn_prefill_params* p, const void* q, const 
                          const void* v, const float* lambda, const float* lambda_init,
                          const void* dout, float* dq, float* dk, float* dv, float* dlambda,
                          void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+
+/*
+ * diffattn_fwd_prefill_train -- diffattn_fwd_prefill for training (V2, bf16, d = 128): the
+ * same output, plus what the backward needs so that diffattn_bwd_prefill_saved does not
+ * recompute the forward. (The pages' training setting: "Differential Attention (V2)", Key
+ * Terms, "lambda", and "V1 vs V2"; the statistics are the softmax's own, Build It, Step 1.)
+ *
+ * p, q, k, v, lambda, out : as for diffattn_fwd_prefill (fixed-length batches; causal, full,
+ *              chunked and sliding window as there)
+ * o2         : the branch-2 output O_2 / l_2 = A_2 V of every (query, pair), in out's
+ *              layout (p->o_strides) and dtype, 16-byte aligned, overwritten
+ * lse        : float32 [B, Hq/2, N, 2], dense, 16-byte aligned: per (batch entry, pair,
+ *              query) the log-sum-exps of both branches in the log2 domain,
+ *              log2 sum_j 2^(s_b,j log2(e) / sqrt(d)) with s_b the raw scores; overwritten
+ * Returns DIFFATTN_ERR_UNSUPPORTED for V1, fp32 or d != 128 (those train through
+ * diffattn_bwd_prefill, which recomputes); otherwise errors as for diffattn_fwd_prefill.
+ */
+int diffattn_fwd_prefill_train(const diffattn_prefill_params* p, const void* q, const void* k,
+                               const void* v, const float* lambda, void* out, void* o2, float* lse,
+                               int* dev_status, void* stream);
+
+/*
+ * diffattn_bwd_prefill_saved -- diffattn_bwd_prefill from diffattn_fwd_prefill_train's saved
+ * output: the per-row deltas are taken from out and o2 (delta_2 = dO . O_2 / l_2,
+ * delta_1 = dO . (out + lambda O_2 / l_2)) and the log-sum-exps from lse, instead of a
+ * recompute of the forward. Same gradients, layouts, workspace size
+ * (diffattn_bwd_workspace_size), arithmetic and determinism as the tensor-core path of
+ * diffattn_bwd_prefill; V2, bf16, d = 128 only.
+ *
+ * out, o2, lse : the training forward's outputs for the same p, q, k, v and lambda; out,
+ *              o2 and dout share the layout p->o_strides
+ * Errors as for diffattn_bwd_prefill; DIFFATTN_ERR_UNSUPPORTED outside V2 bf16 d = 128.
+ */
+int diffattn_bwd_prefill_saved(const diffattn_prefill_params* p, const void* q, const void* k,
+                               const void* v, const float* lambda, const void* out, const void* o2,
+                               const float* lse, const void* dout, float* dq, float* dk, float* dv,
+                               float* dlambda, void* workspace, size_t workspace_bytes,
+                               int* dev_status, void* stream);
 
 /*
  * diffattn_lambda_bwd -- gradients of the four lambda vectors from dL/dlambda:

@@ -225,6 +225,18 @@ def test_selftest_exp2_rejects(lib):
     assert f(None, None, None, 0, None) == 0  # nothing to do, nothing launched
 
 
+def test_train_and_saved_backward_reject(lib):
+    vp = ctypes.c_void_p
+    assert lib.diffattn_fwd_prefill_train(None, *([None] * 9)) == -1
+    assert lib.diffattn_bwd_prefill_saved(None, *([None] * 13), 0, None, None) == -1
+    p = B.PrefillParams()
+    p.variant, p.dtype, p.batch, p.seqlen, p.n_q_heads, p.n_kv_heads, p.head_dim = 1, 1, 1, 8, 2, 2, 64
+    p.causal = 1
+    assert lib.diffattn_fwd_prefill_train(ctypes.byref(p), *([vp(GOOD)] * 7), None, None) == -2  # V1
+    p.variant, p.n_q_heads, p.n_kv_heads, p.head_dim = 2, 4, 2, 64
+    assert lib.diffattn_fwd_prefill_train(ctypes.byref(p), *([vp(GOOD)] * 7), None, None) == -2  # d != 128
+
+
 def test_debug_bounds_violations_normal_build(lib):
     f = lib.diffattn_debug_bounds_violations
     assert f(None) == -1
