@@ -14,8 +14,10 @@ backward of a V2 prefill (N=4096, 64/8 heads; step = lambda + the whole backward
 decode over 16-token pages in a shuffled block table.
 Inputs are the seeded synthetic tensors of differential_attention_05_b200.synth. With the
 default workload the line also carries "secondary": the other rows timed alone (the V1
-layer, the V2 prefill, its window and chunk forms and its backward on the synth tensors; the
-decodes on same-shape seeded draws made on the device, each entry saying which).
+layer and its exact-fp32 backward, the V2 prefill, its window and chunk forms, the training
+forward and the backward from its saved outputs, and the backward that recomputes them, on
+the synth tensors; the decodes on same-shape seeded draws made on the device, each entry
+saying which).
 
 Timing: W untimed warm-up steps, then K steps between a barrier + synchronize on both
 sides; every step is bracketed by CUDA events on the launching stream and L2 is flushed
@@ -545,15 +547,30 @@ def secondary(device, peaks, torch, da):
         res[name] = {"workload": inp.name, "inputs": seeded, "queries": Nq, "keys": N,
                      "window": window, **tflops(4.0 * d * Hq * visible_pairs(Nq, N, True, window), ms)}
     del q, k, v, out, qq, oo
-    # ---- V2 backward (statistics pass, dK/dV, dQ, dlambda sum); algorithmic FLOPs per
-    # attended (query head, key) pair: 8 d (scores 2d, dP d per head, dQ 2d, dK 2d, dV d)
+    # ---- V2 backward; algorithmic FLOPs per attended (query head, key) pair: 8 d (scores
+    # 2d, dP d per head, dQ 2d, dK 2d, dV d). The training path: the forward that saves
+    # O_2 / l_2 and the log-sum-exps (timed as its own line), then the backward from them
+    # (statistics rows, dK/dV, dQ, dlambda sum); and the backward that recomputes the
+    # statistics with a forward pass of its own.
     inp = synth.v2_backward()
     q, k, v, dy = dev(inp.q), dev(inp.k), dev(inp.v), dev(inp.extra["dy"])
     lam, li = lam_of((inp.lq1, inp.lk1, inp.lq2, inp.lk2), inp.depth)
-    ms = _timed(lambda: da.diffattn_bwd_prefill(q, k, v, lam, dy), torch)
+    bwd_flops = 8.0 * inp.d * inp.H * visible_pairs(inp.N, inp.N)
+    o, o2, lse = da.diffattn_fwd_prefill_train(q, k, v, lam)
+    ms = _timed(lambda: da.diffattn_fwd_prefill_train(q, k, v, lam, out=o, o2=o2, lse=lse), torch)
+    res["v2_forward_train_n4096"] = {"workload": inp.name, "inputs": seeded,
+                                     "writes": "out, O_2 / l_2, log-sum-exps",
+                                     **tflops(4.0 * inp.d * inp.H * visible_pairs(inp.N, inp.N), ms)}
+    grads = tuple(torch.empty(t.shape, dtype=torch.float32, device=device) for t in (q, k, v)) + (
+        torch.empty(lam.shape, dtype=torch.float32, device=device),)
+    ms = _timed(lambda: da.diffattn_bwd_prefill_saved(q, k, v, lam, o, o2, lse, dy, grads=grads), torch)
     res["v2_backward_n4096"] = {"workload": inp.name, "inputs": seeded,
-                                **tflops(8.0 * inp.d * inp.H * visible_pairs(inp.N, inp.N), ms)}
-    del q, k, v, dy
+                                "path": "from the training forward's saved outputs", **tflops(bwd_flops, ms)}
+    ms = _timed(lambda: da.diffattn_bwd_prefill(q, k, v, lam, dy, grads=grads), torch)
+    res["v2_backward_recompute_n4096"] = {"workload": inp.name, "inputs": seeded,
+                                          "path": "statistics recomputed by a forward pass",
+                                          **tflops(bwd_flops, ms)}
+    del q, k, v, dy, o, o2, lse, grads
     torch.cuda.empty_cache()
     # ---- V2 decode: same-shape draws on the device
     g = torch.Generator(device=device)

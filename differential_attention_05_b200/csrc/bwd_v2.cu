@@ -13,10 +13,11 @@
 //   2. bwd_v2_dkdv_kernel: one CTA per (128-key tile, KV head, batch entry) walks the pairs
 //      of the GQA group and the 64-query tiles that see its keys. Per step the tensor core
 //      computes S^T = K [Q_1; Q_2]^T (both branches stacked, N = 128) and dP^T = V dO^T;
-//      one warpgroup (thread = key = TMEM lane) forms (P_1 - lambda P_2)^T and
-//      [dS_1^T | dS_2^T] in bf16 straight into TMEM, and the tensor core accumulates
-//      dV += (P_1 - lambda P_2)^T dO and dK += [dS_1^T | dS_2^T] [Q_1; Q_2] in TMEM (A from
-//      TMEM, B = the same shared tiles read MN-major);
+//      the row threads (thread = key = TMEM lane) write (P_1 - lambda P_2)^T in bf16 to a
+//      shared tile and [dS_1^T | dS_2^T] in bf16 to TMEM, and the tensor core accumulates
+//      dV += (P_1 - lambda P_2)^T dO and dK += [dS_1^T | dS_2^T] [Q_1; Q_2] in TMEM (B = the
+//      same shared tiles read MN-major). The next step's S^T and dP^T are issued as soon as
+//      the rows have read this step's, so they run while the rows work;
 //   3. bwd_v2_dq_kernel: one CTA per (64-query tile, pair, batch entry) walks the 128-key
 //      tiles its queries see: S = [Q_1; Q_2] K^T and dP = [dO; dO] V^T (branches stacked in
 //      the M = 128 rows), dS_b in bf16 into TMEM, dQ += dS K.
@@ -74,23 +75,32 @@ __device__ __forceinline__ bool tile_visible(const PrefillArgs& a, int q0, int n
 
 // ----------------------------------------------------------------------------- dK, dV
 namespace kv {
-constexpr int KT = 128, QT = 64, STAGES = 2;
+constexpr int KT = 128, QT = 64;
+// Two rings: [Q_1; Q_2] of a step (read by its first MMA, S^T, and its last, dK) three deep,
+// so that the next step's copy never waits for the step before it to finish; dO and the
+// statistics rows (read by dP^T, the row threads and dV) two deep.
+constexpr int Q_STAGES = 3, D_STAGES = 2;
 constexpr int K_OFF = 0, V_OFF = 2 * BLK;
-constexpr int STAGE_OFF = 4 * BLK;
-constexpr int QS = 0, DO = 2 * BLK, STS = 2 * BLK + 2 * HBLK;  // inside a stage
-constexpr int STAGE_BYTES = 2 * BLK + 2 * HBLK + 1024;         // 49 KB
-constexpr int MISC_OFF = STAGE_OFF + STAGES * STAGE_BYTES;
+constexpr int Q_OFF = 4 * BLK;                       // Q_STAGES x [Q_1; Q_2] (32 KB)
+constexpr int D_OFF = Q_OFF + Q_STAGES * 2 * BLK;    // D_STAGES x (dO 16 KB + statistics 1 KB)
+constexpr int STS = 2 * HBLK;                        // the statistics inside a dO stage
+constexpr int D_STAGE = 2 * HBLK + 1024;
+// (P_1 - lambda P_2)^T of a step in bf16, [128 keys x 64 queries] 128-byte swizzled: the A
+// operand of the dV MMA, written by the row threads
+constexpr int PC_OFF = D_OFF + D_STAGES * D_STAGE;
+constexpr int MISC_OFF = PC_OFF + BLK;
 constexpr int SMEM_BYTES = MISC_OFF + 1024 + 1024;
-// TMEM columns: S^T (both branches), dP^T (then P_1 - lambda P_2 in bf16 over its first
-// half), [dS_1^T | dS_2^T] in bf16, dV, dK
-constexpr int C_S = 0, C_DP = 128, C_PC = 128, C_DS = 192, C_DV = 256, C_DK = 384;
+// TMEM columns: S^T (both branches), dP^T, [dS_1^T | dS_2^T] in bf16, dV, dK
+constexpr int C_S = 0, C_DP = 128, C_DS = 192, C_DV = 256, C_DK = 384;
 struct Misc {
-  uint64_t kv_full, q_full[STAGES], q_empty[STAGES], s_full, p_full, o_full;
-  uint64_t s_read;  // every row thread has read the step's S^T and dP^T columns
+  uint64_t kv_full, q_full[Q_STAGES], q_empty[Q_STAGES], d_full[D_STAGES], d_empty[D_STAGES];
+  uint64_t s_full, p_full, o_full;
+  uint64_t s_read;    // every row thread has read the step's S^T and dP^T columns
+  uint64_t acc_done;  // the dV and dK MMAs of a step have completed (they read P and dS)
   uint32_t tmem_base;
   int abort;
 };
-static_assert(STAGE_BYTES % 1024 == 0 && sizeof(Misc) <= 1024, "layout");
+static_assert(D_STAGE % 1024 == 0 && PC_OFF % 1024 == 0 && sizeof(Misc) <= 1024, "layout");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 }  // namespace kv
 }  // namespace
@@ -123,14 +133,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&ms.kv_full, 1);
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < Q_STAGES; ++s) {
       mbar_init(&ms.q_full[s], 1);
       mbar_init(&ms.q_empty[s], 1);
     }
+    for (int s = 0; s < D_STAGES; ++s) {
+      mbar_init(&ms.d_full[s], 1);
+      mbar_init(&ms.d_empty[s], 1);
+    }
     mbar_init(&ms.s_full, 1);
-    mbar_init(&ms.p_full, 128 * RW);
+    mbar_init(&ms.p_full, 4 * RW);  // one arrival per row warp
     mbar_init(&ms.o_full, 1);
-    mbar_init(&ms.s_read, 128 * RW);
+    mbar_init(&ms.s_read, 4 * RW);
+    mbar_init(&ms.acc_done, 1);
     ms.abort = 0;
     fence_barrier_init();
   }
@@ -157,30 +172,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_load_4d(smem + K_OFF + hf * BLK, &maps.k, &ms.kv_full, 64 * hf, gk, k0, b);
         tma_load_4d(smem + V_OFF + hf * BLK, &maps.v, &ms.kv_full, 64 * hf, gk, k0, b);
       }
-      int issued = 0;
+      int q_issued = 0, d_issued = 0;
       for (int t = 0; t < n_steps && !*abort_flag; ++t) {
-        const int s = t % STAGES;
-        if (!mbar_wait(&ms.q_empty[s], ((t / STAGES) & 1) ^ 1, abort_flag)) break;
         const int u = u0 + t / n_qt, q0 = (qt_lo + t % n_qt) * QT;
-        uint8_t* st = smem + STAGE_OFF + s * STAGE_BYTES;
+        const int sq = t % Q_STAGES, sd = t % D_STAGES;
+        if (!mbar_wait(&ms.q_empty[sq], ((t / Q_STAGES) & 1) ^ 1, abort_flag)) break;
+        uint8_t* qs = smem + Q_OFF + sq * 2 * BLK;
+        mbar_arrive_expect_tx(&ms.q_full[sq], 2 * BLK);
+        for (int hf = 0; hf < 2; ++hf) {
+          // [Q_1; Q_2]: rows 0-63 branch 1, rows 64-127 branch 2 of each 64-column block
+          tma_load_4d(qs + hf * BLK, &maps.q, &ms.q_full[sq], 64 * hf, 2 * u, q0, b);
+          tma_load_4d(qs + hf * BLK + 64 * 128, &maps.q, &ms.q_full[sq], 64 * hf, 2 * u + 1, q0, b);
+        }
+        q_issued = t + 1;
+        if (!mbar_wait(&ms.d_empty[sd], ((t / D_STAGES) & 1) ^ 1, abort_flag)) break;
+        uint8_t* ds = smem + D_OFF + sd * D_STAGE;
         // (w_st starts the workspace, so its offsets are workspace offsets)
         const int64_t st_off = (((int64_t)b * a.units + u) * rows + q0) * 4;
         const bool st_ok = in_bounds((g.w_st - g.w_base) + st_off, 256, g.ext_ws, a.dev_status, a.dbg_status);
-        mbar_arrive_expect_tx(&ms.q_full[s], 2 * BLK + 2 * HBLK + (st_ok ? 1024 : 0));
-        for (int hf = 0; hf < 2; ++hf) {
-          // [Q_1; Q_2]: rows 0-63 branch 1, rows 64-127 branch 2 of each 64-column block
-          tma_load_4d(st + QS + hf * BLK, &maps.q, &ms.q_full[s], 64 * hf, 2 * u, q0, b);
-          tma_load_4d(st + QS + hf * BLK + 64 * 128, &maps.q, &ms.q_full[s], 64 * hf, 2 * u + 1, q0, b);
-          tma_load_4d(st + DO + hf * HBLK, &maps.dy, &ms.q_full[s], 64 * hf, u, q0, b);
-        }
-        if (st_ok) bulk_load(st + STS, g.w_st + st_off, 1024, &ms.q_full[s]);
-        issued = t + 1;
+        mbar_arrive_expect_tx(&ms.d_full[sd], 2 * HBLK + (st_ok ? 1024 : 0));
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_4d(ds + hf * HBLK, &maps.dy, &ms.d_full[sd], 64 * hf, u, q0, b);
+        if (st_ok) bulk_load(ds + STS, g.w_st + st_off, 1024, &ms.d_full[sd]);
+        d_issued = t + 1;
       }
       if (*abort_flag) {
         // let the copies in flight land before the CTA's shared memory goes away
         mbar_wait_drain(&ms.kv_full, 0);
-        for (int t = max(0, issued - STAGES); t < issued; ++t)
-          mbar_wait_drain(&ms.q_full[t % STAGES], (t / STAGES) & 1);
+        for (int t = max(0, q_issued - Q_STAGES); t < q_issued; ++t)
+          mbar_wait_drain(&ms.q_full[t % Q_STAGES], (t / Q_STAGES) & 1);
+        for (int t = max(0, d_issued - D_STAGES); t < d_issued; ++t)
+          mbar_wait_drain(&ms.d_full[t % D_STAGES], (t / D_STAGES) & 1);
       }
     }
   } else if (warp == W_MMA) {
@@ -193,18 +215,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t vdesc = sw128_desc(smem_u32(smem + V_OFF), 16, 1024);
       // S^T of step t (both branches stacked, N = 128) into columns 0..127
       auto issue_st = [&](int t) {
-        const uint32_t st = smem_u32(smem + STAGE_OFF + (t % STAGES) * STAGE_BYTES);
-        const uint64_t qd = sw128_desc(st + QS, 16, 1024);
+        const uint64_t qd = sw128_desc(smem_u32(smem + Q_OFF + (t % Q_STAGES) * 2 * BLK), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t o = (kk >> 2) * BLK + (kk & 3) * 32;
           umma_ss(tmem + C_S, desc_at(kdesc, o), desc_at(qd, o), IDESC_S, kk > 0);
         }
       };
+      const uint64_t pcdesc = sw128_desc(smem_u32(smem + PC_OFF), 16, 1024);
       // dP^T of step t (N = 64) into columns 128..191, then the step is complete
       auto issue_dp = [&](int t) {
-        const uint32_t st = smem_u32(smem + STAGE_OFF + (t % STAGES) * STAGE_BYTES);
-        const uint64_t dd = sw128_desc(st + DO, 16, 1024);
+        const uint64_t dd = sw128_desc(smem_u32(smem + D_OFF + (t % D_STAGES) * D_STAGE), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t o = (kk >> 2) * BLK + (kk & 3) * 32;
@@ -214,27 +235,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_commit(&ms.s_full);
       };
       auto issue_dv_dk = [&](int t) {
-        const uint32_t st = smem_u32(smem + STAGE_OFF + (t % STAGES) * STAGE_BYTES);
         // the same tiles read MN-major: K index = query (16 rows = 2048 B per step)
-        const uint64_t dmn = sw128_desc(st + DO, HBLK, 1024);
-        const uint64_t qmn = sw128_desc(st + QS, BLK, 1024);
+        const uint64_t dmn = sw128_desc(smem_u32(smem + D_OFF + (t % D_STAGES) * D_STAGE), HBLK, 1024);
+        const uint64_t qmn = sw128_desc(smem_u32(smem + Q_OFF + (t % Q_STAGES) * 2 * BLK), BLK, 1024);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_ts(tmem + C_DV, tmem + C_PC + kk * 16, desc_at(dmn, kk * 2048), IDESC_ACC,
+          umma_ss(tmem + C_DV, desc_at(pcdesc, kk * 32), desc_at(dmn, kk * 2048), IDESC_ACC,
                   (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&ms.d_empty[t % D_STAGES]);  // dO and the statistics of step t are done with
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tmem + C_DK, tmem + C_DS + kk * 8, desc_at(qmn, kk * 2048), IDESC_ACC,
                   (t > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&ms.q_empty[t % STAGES]);
+        tc_commit(&ms.q_empty[t % Q_STAGES]);
+        tc_commit(&ms.acc_done);
       };
-      // Per step t: S^T(t+1) as soon as the row threads have read step t's columns (it
-      // overwrites only S^T), then dV, dK of step t once their operands are written, then
-      // dP^T(t+1) (its columns held P_1 - lambda P_2 of step t, which dV has read: the
-      // tensor core runs these in order).
+      // Per step t: S^T(t+1) and dP^T(t+1) as soon as the row threads have read step t's
+      // columns, so that they run while the rows work on step t; then dV, dK of step t once
+      // their operands are written. (The issuing thread is held at the tensor core's pace,
+      // so this order is also the order the tensor core runs them in.)
       bool ok = mbar_wait(&ms.kv_full, 0, abort_flag);
       if (ok && n_steps > 0) {
-        ok = mbar_wait(&ms.q_full[0], 0, abort_flag);
+        ok = mbar_wait(&ms.q_full[0], 0, abort_flag) && mbar_wait(&ms.d_full[0], 0, abort_flag);
         if (ok) {
           tc_fence_after();
           issue_st(0);
@@ -242,17 +264,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       for (int t = 0; t < n_steps && ok; ++t) {
-        const bool more = t + 1 < n_steps;
-        if (more) {
+        if (t + 1 < n_steps) {
           if (!(ok = mbar_wait(&ms.s_read, t & 1, abort_flag))) break;
-          if (!(ok = mbar_wait(&ms.q_full[(t + 1) % STAGES], ((t + 1) / STAGES) & 1, abort_flag))) break;
+          const int n = t + 1;
+          if (!(ok = mbar_wait(&ms.q_full[n % Q_STAGES], (n / Q_STAGES) & 1, abort_flag))) break;
           tc_fence_after();
-          issue_st(t + 1);
+          issue_st(n);
+          if (!(ok = mbar_wait(&ms.d_full[n % D_STAGES], (n / D_STAGES) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_dp(n);
         }
         if (!(ok = mbar_wait(&ms.p_full, t & 1, abort_flag))) break;
         tc_fence_after();
         issue_dv_dk(t);
-        if (more) issue_dp(t + 1);
       }
       // arrives once every MMA issued above has completed (also on an abort)
       tc_commit(&ms.o_full);
@@ -263,18 +287,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     static_assert(RW == 4, "one 16-query chunk per row warpgroup");
     const int wgr = warp >> 2;
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const int j = k0 + (warp & 3) * 32 + lane;  // this thread's key (TMEM lane)
+    const int kr = (warp & 3) * 32 + lane;  // this thread's key row (TMEM lane)
+    const int j = k0 + kr;
+    // this warpgroup's 16 queries of the key row in the swizzled P tile: 16-byte chunks
+    // 2 wgr and 2 wgr + 1 of the row's 128 bytes
+    uint8_t* pc_row = smem + PC_OFF + kr * 128;
+    const int pc_c0 = ((2 * wgr) ^ (kr & 7)) << 4, pc_c1 = ((2 * wgr + 1) ^ (kr & 7)) << 4;
     const float sl2 = 1.4426950408889634f * rsqrtf((float)a.d);
     bool ok = true;
     for (int t = 0; t < n_steps; ++t) {
-      const int s = t % STAGES;
+      const int sd = t % D_STAGES;
       const int u = u0 + t / n_qt, q0 = (qt_lo + t % n_qt) * QT;
       const float lam = a.lambda[u];
-      if (ok) ok = mbar_wait(&ms.q_full[s], (t / STAGES) & 1, abort_flag);
+      if (ok) ok = mbar_wait(&ms.d_full[sd], (t / D_STAGES) & 1, abort_flag);
       if (ok) ok = mbar_wait(&ms.s_full, t & 1, abort_flag);
       if (!(ok = __all_sync(FULL, ok))) break;
       tc_fence_after();
-      const float4* sts = reinterpret_cast<const float4*>(smem + STAGE_OFF + s * STAGE_BYTES + STS);
+      const float4* sts = reinterpret_cast<const float4*>(smem + D_OFF + sd * D_STAGE + STS);
       // inside the visible region (most steps of a causal problem) no pair needs a mask
       const bool full = tile_visible(a, q0, QT, k0, KT);
       auto chunk = [&](auto all_visible) {
@@ -284,9 +313,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld16f(lane_addr + C_S + 64 + 16 * c, s2);
         tmem_ld16f(lane_addr + C_DP + 16 * c, dp);
         tmem_wait_ld();
-        // the next step's S^T may now overwrite columns 0..127
+        // the next step's S^T and dP^T may now overwrite their columns (one arrival per warp:
+        // 512 single-thread arrivals on one barrier serialise)
         tc_fence_before();
-        mbar_arrive(&ms.s_read);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ms.s_read);
         uint32_t pc[8], d1[8], d2[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
@@ -306,17 +337,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           d1[e / 2] = pack_bf16(vd1[0], vd1[1]);
           d2[e / 2] = pack_bf16(vd2[0], vd2[1]);
         }
-        // P_1 - lambda P_2 over this chunk's own dP columns (read above, by this warp only);
-        // dS_1, dS_2 into their 8-column slots of the dS block
-        tmem_st8(lane_addr + C_PC + 16 * c, pc);
+        // P and dS of step t replace those of step t - 1 once its dV, dK MMAs are done
+        if (t > 0) {
+          if (ok) ok = mbar_wait(&ms.acc_done, (t - 1) & 1, abort_flag);
+          if (!(ok = __all_sync(FULL, ok))) return;
+          tc_fence_after();
+        }
+        // P_1 - lambda P_2 into the shared tile; dS_1, dS_2 into their 8-column slots of the
+        // dS block
+        *reinterpret_cast<uint4*>(pc_row + pc_c0) = make_uint4(pc[0], pc[1], pc[2], pc[3]);
+        *reinterpret_cast<uint4*>(pc_row + pc_c1) = make_uint4(pc[4], pc[5], pc[6], pc[7]);
         tmem_st8(lane_addr + C_DS + 8 * c, d1);
         tmem_st8(lane_addr + C_DS + 32 + 8 * c, d2);
       };
       if (full) chunk(std::true_type{});
       else chunk(std::false_type{});
+      if (!ok) break;
       tmem_wait_st();
+      // the shared stores above become visible to the tensor core's operand reads
+      fence_proxy_async();
       tc_fence_before();
-      mbar_arrive(&ms.p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms.p_full);
     }
     // ------------------------------- epilogue ----------------------------------------
     if (ok) ok = mbar_wait(&ms.o_full, 0, abort_flag);
@@ -366,24 +408,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ----------------------------------------------------------------------------- dQ
 namespace {
 namespace dqk {
-constexpr int QT = 64, KT = 128, STAGES = 2;
+constexpr int QT = 64, KT = 128;
+// Two rings: a step's K tile (read by its first MMA, S, and its last, dQ) three deep, so
+// that the next step's copy never waits for the step before it to finish; its V tile (read
+// by dP only) two deep.
+constexpr int K_STAGES = 3, V_STAGES = 2;
 constexpr int QS_OFF = 0;                 // [Q_1; Q_2]: 2 blocks of [128 x 64]
 constexpr int DO_OFF = 2 * BLK;           // [dO; dO]
 constexpr int ST_OFF = 4 * BLK;           // 64 x (lse_1, lse_2, delta_1, delta_2)
-constexpr int KV_OFF = 4 * BLK + 1024;
-constexpr int KV_STAGE = 4 * BLK;         // K (2 blocks), V (2 blocks)
-constexpr int MISC_OFF = KV_OFF + STAGES * KV_STAGE;
+constexpr int K_OFF = 4 * BLK + 1024;     // K_STAGES x K (2 blocks)
+constexpr int V_OFF = K_OFF + K_STAGES * 2 * BLK;  // V_STAGES x V (2 blocks)
+constexpr int MISC_OFF = V_OFF + V_STAGES * 2 * BLK;
 constexpr int SMEM_BYTES = MISC_OFF + 1024 + 1024;
 // TMEM columns: S, dP, dQ, dS (bf16)
 constexpr int C_S = 0, C_DP = 128, C_DQ = 256, C_DS = 384;
 struct Misc {
-  uint64_t q_full, kv_full[STAGES], kv_empty[STAGES], s_full, p_full, o_full;
+  uint64_t q_full, k_full[K_STAGES], k_empty[K_STAGES], v_full[V_STAGES], v_empty[V_STAGES];
+  uint64_t s_full, p_full, o_full;
   uint64_t s_read;   // every row thread has read the step's S and dP columns
   uint64_t dq_done;  // the dQ MMAs of a step have completed (they read its dS)
   uint32_t tmem_base;
   int abort;
 };
-static_assert(KV_OFF % 1024 == 0 && sizeof(Misc) <= 1024, "layout");
+static_assert(K_OFF % 1024 == 0 && sizeof(Misc) <= 1024, "layout");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 }  // namespace dqk
 }  // namespace
@@ -413,14 +460,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&ms.q_full, 1);
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&ms.kv_full[s], 1);
-      mbar_init(&ms.kv_empty[s], 1);
+    for (int s = 0; s < K_STAGES; ++s) {
+      mbar_init(&ms.k_full[s], 1);
+      mbar_init(&ms.k_empty[s], 1);
+    }
+    for (int s = 0; s < V_STAGES; ++s) {
+      mbar_init(&ms.v_full[s], 1);
+      mbar_init(&ms.v_empty[s], 1);
     }
     mbar_init(&ms.s_full, 1);
-    mbar_init(&ms.p_full, 128 * RW);
+    mbar_init(&ms.p_full, 4 * RW);  // one arrival per row warp
     mbar_init(&ms.o_full, 1);
-    mbar_init(&ms.s_read, 128 * RW);
+    mbar_init(&ms.s_read, 4 * RW);
     mbar_init(&ms.dq_done, 1);
     ms.abort = 0;
     fence_barrier_init();
@@ -453,23 +504,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_load_4d(smem + DO_OFF + hf * BLK + 64 * 128, &maps.dy, &ms.q_full, 64 * hf, u, q0, b);
       }
       if (st_ok) bulk_load(smem + ST_OFF, g.w_st + st_off, 1024, &ms.q_full);
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       for (int t = 0; t < n_kt && !*abort_flag; ++t) {
-        const int s = t % STAGES;
-        if (!mbar_wait(&ms.kv_empty[s], ((t / STAGES) & 1) ^ 1, abort_flag)) break;
         const int kj = (j_lo + t) * KT;
-        uint8_t* st = smem + KV_OFF + s * KV_STAGE;
-        mbar_arrive_expect_tx(&ms.kv_full[s], 4 * BLK);
-        for (int hf = 0; hf < 2; ++hf) {
-          tma_load_4d(st + hf * BLK, &maps.k, &ms.kv_full[s], 64 * hf, gk, kj, b);
-          tma_load_4d(st + 2 * BLK + hf * BLK, &maps.v, &ms.kv_full[s], 64 * hf, gk, kj, b);
-        }
-        issued = t + 1;
+        const int sk = t % K_STAGES, sv = t % V_STAGES;
+        if (!mbar_wait(&ms.k_empty[sk], ((t / K_STAGES) & 1) ^ 1, abort_flag)) break;
+        uint8_t* ks = smem + K_OFF + sk * 2 * BLK;
+        mbar_arrive_expect_tx(&ms.k_full[sk], 2 * BLK);
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_4d(ks + hf * BLK, &maps.k, &ms.k_full[sk], 64 * hf, gk, kj, b);
+        k_issued = t + 1;
+        if (!mbar_wait(&ms.v_empty[sv], ((t / V_STAGES) & 1) ^ 1, abort_flag)) break;
+        uint8_t* vs = smem + V_OFF + sv * 2 * BLK;
+        mbar_arrive_expect_tx(&ms.v_full[sv], 2 * BLK);
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_4d(vs + hf * BLK, &maps.v, &ms.v_full[sv], 64 * hf, gk, kj, b);
+        v_issued = t + 1;
       }
       if (*abort_flag) {
         mbar_wait_drain(&ms.q_full, 0);
-        for (int t = max(0, issued - STAGES); t < issued; ++t)
-          mbar_wait_drain(&ms.kv_full[t % STAGES], (t / STAGES) & 1);
+        for (int t = max(0, k_issued - K_STAGES); t < k_issued; ++t)
+          mbar_wait_drain(&ms.k_full[t % K_STAGES], (t / K_STAGES) & 1);
+        for (int t = max(0, v_issued - V_STAGES); t < v_issued; ++t)
+          mbar_wait_drain(&ms.v_full[t % V_STAGES], (t / V_STAGES) & 1);
       }
     }
   } else if (warp == W_MMA) {
@@ -479,9 +536,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t qd = sw128_desc(smem_u32(smem + QS_OFF), 16, 1024);
       const uint64_t dd = sw128_desc(smem_u32(smem + DO_OFF), 16, 1024);
       auto issue_s_dp = [&](int t) {
-        const uint32_t st = smem_u32(smem + KV_OFF + (t % STAGES) * KV_STAGE);
-        const uint64_t kd = sw128_desc(st, 16, 1024);
-        const uint64_t vd = sw128_desc(st + 2 * BLK, 16, 1024);
+        const uint64_t kd = sw128_desc(smem_u32(smem + K_OFF + (t % K_STAGES) * 2 * BLK), 16, 1024);
+        const uint64_t vd = sw128_desc(smem_u32(smem + V_OFF + (t % V_STAGES) * 2 * BLK), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t o = (kk >> 2) * BLK + (kk & 3) * 32;
@@ -493,20 +549,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           umma_ss(tmem + C_DP, desc_at(dd, o), desc_at(vd, o), IDESC_SS, kk > 0);
         }
         tc_commit(&ms.s_full);
+        tc_commit(&ms.v_empty[t % V_STAGES]);
       };
       auto issue_dq = [&](int t) {
-        const uint32_t st = smem_u32(smem + KV_OFF + (t % STAGES) * KV_STAGE);
-        const uint64_t kmn = sw128_desc(st, BLK, 1024);  // K read MN-major: K index = key
+        // K read MN-major: K index = key
+        const uint64_t kmn = sw128_desc(smem_u32(smem + K_OFF + (t % K_STAGES) * 2 * BLK), BLK, 1024);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tmem + C_DQ, tmem + C_DS + kk * 8, desc_at(kmn, kk * 2048), IDESC_ACC,
                   (t > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&ms.dq_done);
-        tc_commit(&ms.kv_empty[t % STAGES]);
+        tc_commit(&ms.k_empty[t % K_STAGES]);
+      };
+      auto kv_ready = [&](int t) {
+        return mbar_wait(&ms.k_full[t % K_STAGES], (t / K_STAGES) & 1, abort_flag) &&
+               mbar_wait(&ms.v_full[t % V_STAGES], (t / V_STAGES) & 1, abort_flag);
       };
       bool ok = mbar_wait(&ms.q_full, 0, abort_flag);
       if (ok && n_kt > 0) {
-        ok = mbar_wait(&ms.kv_full[0], 0, abort_flag);
+        ok = kv_ready(0);
         if (ok) {
           tc_fence_after();
           issue_s_dp(0);
@@ -517,7 +578,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int t = 0; t < n_kt && ok; ++t) {
         if (t + 1 < n_kt) {
           if (!(ok = mbar_wait(&ms.s_read, t & 1, abort_flag))) break;
-          if (!(ok = mbar_wait(&ms.kv_full[(t + 1) % STAGES], ((t + 1) / STAGES) & 1, abort_flag))) break;
+          if (!(ok = kv_ready(t + 1))) break;
           tc_fence_after();
           issue_s_dp(t + 1);
         }
@@ -553,9 +614,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_ld32f(lane_addr + C_S + 32 * c, sv);
         tmem_ld32f(lane_addr + C_DP + 32 * c, dp);
         tmem_wait_ld();
-        // the next step's S and dP may now overwrite these columns
+        // the next step's S and dP may now overwrite these columns (one arrival per warp)
         tc_fence_before();
-        mbar_arrive(&ms.s_read);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ms.s_read);
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float v2[2];
@@ -579,7 +641,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tmem_st16(lane_addr + C_DS + 16 * wgr, ds);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&ms.p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms.p_full);
     }
     if (ok) ok = mbar_wait(&ms.o_full, 0, abort_flag);
     ok = __all_sync(FULL, ok);
