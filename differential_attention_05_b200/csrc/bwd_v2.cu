@@ -25,6 +25,7 @@
 // backward, which takes the forward's bf16-accumulated output as input and amplifies its
 // rounding beyond the bf16 bound, so no tensor-core path is built for it.
 // No atomics: every dK/dV row and every dQ row is summed inside one CTA in a fixed order.
+// The dQ kernel runs on a second stream beside the dK/dV kernel (see SideStream).
 // Warps 0-15 (four warpgroups, each taking a quarter of a step's columns) form the per-row
 // arithmetic, warp 16 issues the TMA loads (128-byte swizzle, no multicast) and the 1-D bulk
 // copy of the statistics, warp 17 owns TMEM and every MMA.
@@ -33,6 +34,7 @@
 #include "kernels.h"
 #include "tma_host.cuh"
 
+#include <mutex>
 #include <type_traits>
 
 namespace diffattn {
@@ -747,6 +749,35 @@ __global__ void __launch_bounds__(256) bwd_saved_stats_kernel(BwdArgs g, const _
   }
 }
 
+// A second stream per device for the dQ kernel: the dK/dV grid (one CTA per 128 keys and KV
+// head, the first key tiles of a causal problem the heaviest) ends in a partial wave, and the
+// short dQ CTAs fill the SMs it leaves idle. Forked from the caller's stream and joined back
+// to it with events, so the pair stays ordered with the caller's work and can be captured
+// into a CUDA graph; the mutex keeps the event records of concurrent callers apart.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool failed = false;
+};
+std::mutex g_side_mu;
+SideStream g_side[64];
+
+// the side stream of device dev, or nullptr (then both kernels run on the caller's stream)
+SideStream* side_stream(int dev) {
+  if (dev < 0 || dev >= 64) return nullptr;
+  SideStream& ss = g_side[dev];
+  if (!ss.s && !ss.failed) {
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      ss.failed = true;
+      cudaGetLastError();  // the fallback below needs no side stream; clear the error
+      return nullptr;
+    }
+  }
+  return ss.failed ? nullptr : &ss;
+}
+
 // steps 2-4 of the tensor-core backward, once the statistics rows are in the workspace
 cudaError_t backward_tc_kernels(const BwdArgs& g, cudaStream_t stream) {
   const PrefillArgs& a = g.f;
@@ -770,12 +801,24 @@ cudaError_t backward_tc_kernels(const BwdArgs& g, cudaStream_t stream) {
   const long long kv_ctas = (long long)((a.Nk + kv::KT - 1) / kv::KT) * a.Hkv * a.B;
   const long long dq_ctas = (long long)((a.N + dqk::QT - 1) / dqk::QT) * a.units * a.B;
   if (kv_ctas > 0x7fffffffLL || dq_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  SideStream* ss = side_stream(dev);
+  cudaStream_t dq_stream = stream;
+  if (ss) {
+    if ((e = cudaEventRecord(ss->fork, stream)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return e;
+    dq_stream = ss->s;
+  }
   bwd_v2_dkdv_kernel<<<(unsigned)kv_ctas, NUM_THREADS, kv::SMEM_BYTES, stream>>>(maps, g);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_v2_dq_kernel<<<(unsigned)dq_ctas, NUM_THREADS, dqk::SMEM_BYTES, stream>>>(maps, g);
+  bwd_v2_dq_kernel<<<(unsigned)dq_ctas, NUM_THREADS, dqk::SMEM_BYTES, dq_stream>>>(maps, g);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (ss) {
+    if ((e = cudaEventRecord(ss->join, ss->s)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(stream, ss->join, 0)) != cudaSuccess) return e;
+  }
   return launch_dlambda_reduce(g, stream);
 }
 

@@ -102,3 +102,39 @@ def test_train_rejects_other_variants():
     out = torch.empty((1, 64, 2, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(Exception):
         da.diffattn_fwd_prefill_train(q, k, v, lam, out=out)
+
+
+def test_backward_graph_capture_and_side_stream():
+    """The tensor-core backward runs its dQ kernel on a library-owned second stream, forked
+    from and joined back to the caller's stream. Captured into a CUDA graph on a non-default
+    stream and replayed, it gives the eager call's gradients bit for bit, and work queued on
+    the caller's stream after it sees the finished gradients."""
+    Nq = Nk = 520
+    inp = synth.v2_small(B=1, N=Nk, Hq=16, Hkv=2, seed=920, causal=True)
+    q, k, v = dev_tensor(inp.q), dev_tensor(inp.k), dev_tensor(inp.v)
+    lam, _ = lambda_on_device(inp)
+    out, o2, lse = da.diffattn_fwd_prefill_train(q, k, v, lam)
+    g = torch.Generator().manual_seed(921)
+    dy = torch.randn(out.shape, generator=g).bfloat16().cuda()
+    eager = da.diffattn_bwd_prefill_saved(q, k, v, lam, out, o2, lse, dy)
+    p = da._binding.prefill_params(q, k, v, out, causal=True)
+    ws = torch.empty(max(da._binding.diffattn_bwd_workspace_size(p), 1), dtype=torch.uint8, device="cuda")
+    grads = tuple(torch.full(t.shape, float("nan"), dtype=torch.float32, device="cuda") for t in eager)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        da.diffattn_bwd_prefill_saved(q, k, v, lam, out, o2, lse, dy, workspace=ws, grads=grads)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        da.diffattn_bwd_prefill_saved(q, k, v, lam, out, o2, lse, dy, workspace=ws, grads=grads)
+    for t in grads:
+        t.fill_(float("nan"))
+    graph.replay()
+    # read on the replay stream's successor: the copy is ordered after the joined graph
+    copies = [t.clone() for t in grads]
+    torch.cuda.synchronize()
+    for name, x, y in zip(("dq", "dk", "dv", "dlambda"), copies, eager):
+        assert torch.equal(x, y), name
+    del graph
