@@ -31,12 +31,16 @@
 //   * TMEM lane / operand row of (query t, branch b) in a 64-query sub-tile:
 //     (t % 16) + 32 (t / 16) + 16 b; the Q rows are loaded in this order (16-row boxes
 //     alternating the two heads of the pair).
-//   * Warp w of a softmax warpgroup owns queries 16w..16w+15: lanes 0-15 branch 1, lanes
-//     16-31 branch 2 of the same queries. Every lane writes its p (fp32) over its own score
-//     columns; the 16-lane paired TMEM load then hands lanes 0-15 the row of lane + 16
-//     (exact p2 of the same keys). Branch 1 writes p1 - c p2 as its bf16 P row, branch 2
-//     writes p2; the P.V MMA (A = P from TMEM) leaves D in the branch-1 lanes and O_2 in
-//     the branch-2 lanes.
+//   * Warp w of a softmax warpgroup owns queries 16w..16w+15; lane l takes query 16w + l % 16
+//     and half l / 16 of the key tile (64 keys) and of the value columns. The split 16-lane
+//     TMEM loads give it both branches' scores of its keys (the branch-1 row and the branch-2
+//     row 16 lanes further on), so p1 - c p2 is formed in registers; the two halves of a
+//     query exchange only their maxima and sums. It writes the bf16 P rows of both branches
+//     (p1 - c p2 over the branch-1 row, p2 over the branch-2 row); the P.V MMA (A = P from
+//     TMEM) leaves D in the branch-1 lanes and O_2 in the branch-2 lanes.
+//   * CTA order: bands of 32 query tiles, heaviest causal band first; inside a band KV group
+//     by KV group, so the CTAs in flight read the K/V of one or two KV heads, which stay in
+//     L2.
 //   * Two 64-query sub-tiles per CTA (128 queries share every K/V tile) ping-pong: while
 //     one warpgroup turns its scores into P, the tensor core runs the other sub-tile's
 //     products. TMEM: S/P of sub-tile 0 | O of sub-tile 0 | S/P of 1 | O of 1 (4 x 128
