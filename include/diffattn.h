@@ -34,7 +34,9 @@
  *
  * Conventions for every entry point
  *   - Pointers are DEVICE pointers unless marked "host". The caller owns every buffer;
- *     the library allocates nothing, frees nothing and keeps no pointer after a call.
+ *     the library allocates no device memory, frees nothing and keeps no pointer after a
+ *     call. (Its own objects: the 16 MiB array of diffattn_fwd_decode_static, and one CUDA
+ *     stream with two events per device for the tensor-core backward's second stream.)
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
  *     The library never synchronizes.
  *   - Arguments are validated on the host before anything is launched. On any error
@@ -216,6 +218,13 @@ int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t*
  * every other case (fp32 inputs, V1, other d) runs exact fp32 on the CUDA cores. Both are
  * deterministic (no atomics: dQ rows, dK/dV rows and dlambda are each summed by one thread
  * group in a fixed order).
+ * Streams (tensor-core path): the dK/dV and dQ kernels run side by side, the dQ kernel on a
+ * stream the library creates once per device, forked from `stream` and joined back to it
+ * (events) before the call's last kernel. The call therefore stays ordered on `stream` and
+ * can be captured into a CUDA graph. Host threads calling concurrently are serialized while
+ * they enqueue; while one thread captures such a call, other threads must not call the
+ * tensor-core backward on the same device until that capture ends (their dQ kernel would
+ * join the capture).
  * Errors as for diffattn_fwd_prefill, plus DIFFATTN_ERR_WORKSPACE.
  */
 int diffattn_bwd_workspace_size(const diffattn_prefill_params* p, size_t* bytes);
@@ -249,8 +258,8 @@ int diffattn_fwd_prefill_train(const diffattn_prefill_params* p, const void* q, 
  * output: the per-row deltas are taken from out and o2 (delta_2 = dO . O_2 / l_2,
  * delta_1 = dO . (out + lambda O_2 / l_2)) and the log-sum-exps from lse, instead of a
  * recompute of the forward. Same gradients, layouts, workspace size
- * (diffattn_bwd_workspace_size), arithmetic and determinism as the tensor-core path of
- * diffattn_bwd_prefill; V2, bf16, d = 128 only.
+ * (diffattn_bwd_workspace_size), arithmetic, determinism and second stream as the
+ * tensor-core path of diffattn_bwd_prefill; V2, bf16, d = 128 only.
  *
  * out, o2, lse : the training forward's outputs for the same p, q, k, v and lambda; out,
  *              o2 and dout share the layout p->o_strides
