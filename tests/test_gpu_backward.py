@@ -101,6 +101,36 @@ def test_backward_v2_medium():
     _case(2, 2048, 2048, "bf16", seed=770, Hq=16, Hkv=2)
 
 
+@pytest.mark.parametrize("path", ["recompute", "saved"])
+def test_backward_v2_full_size_one_kv_group(path):
+    """The bench's backward workload at full size (B=1, N=4096, 64 query heads over 8 KV
+    heads, d=128, the seeded synth.v2_backward tensors), run as the bench runs it (the
+    recomputing backward, and the training forward + the backward from its saved outputs).
+    The float64 oracle covers one seeded KV group: the dQ of its 8 query heads, its dK and
+    dV (summed over the group's 4 pairs) and its 4 dlambda."""
+    inp = synth.v2_backward()
+    q, k, v = dev_tensor(inp.q), dev_tensor(inp.k), dev_tensor(inp.v)
+    dy = dev_tensor(inp.extra["dy"])
+    lam, _ = lambda_on_device(inp)
+    if path == "recompute":
+        dq, dk, dv, dl = da.diffattn_bwd_prefill(q, k, v, lam, dy)
+    else:
+        o, o2, lse = da.diffattn_fwd_prefill_train(q, k, v, lam)
+        dq, dk, dv, dl = da.diffattn_bwd_prefill_saved(q, k, v, lam, o, o2, lse, dy)
+    torch.cuda.synchronize()
+    g = int(np.random.default_rng(1007).integers(inp.Hkv))
+    group = inp.H // inp.Hkv
+    h0, p0 = g * group, g * group // 2
+    lam64 = oracle.lambda_(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.depth)[p0:p0 + group // 2]
+    dy64 = synth.bf16_to_f32(inp.extra["dy"]).astype(np.float64)[:, :, p0:p0 + group // 2]
+    ref = OB.prefill_v2_bwd(inp.as_f64("q")[:, :, h0:h0 + group], inp.as_f64("k")[:, :, g:g + 1],
+                            inp.as_f64("v")[:, :, g:g + 1], lam64, dy64)
+    tag = f"V2 N=4096 {path} KV group {g}"
+    got = (dq[:, :, h0:h0 + group], dk[:, :, g:g + 1], dv[:, :, g:g + 1], dl[p0:p0 + group // 2])
+    for name, t, r in zip(("dq", "dk", "dv", "dlambda"), got, ref):
+        _check(t, r, f"{tag} {name}", tensor_core=True)
+
+
 def test_lambda_bwd():
     inp = synth.v2_small(B=1, N=4, Hq=64, Hkv=8, seed=780)
     vecs = [dev_tensor(getattr(inp, n)) for n in ("lq1", "lk1", "lq2", "lk2")]
