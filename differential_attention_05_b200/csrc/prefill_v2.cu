@@ -47,7 +47,7 @@
 //     columns). P (bf16) overwrites the first 64 columns of its S block; the next score
 //     MMA of that sub-tile is issued after its P.V MMA, and tcgen05 MMAs run in order.
 //   * Exponentials: in every 8 keys one pair is evaluated on the FMA pipe (exp2_fma2), the
-//     rest on the MUFU unit.
+//     rest on the MUFU unit; launches long enough to run under the power cap use MUFU only.
 //   * warp 8: TMA loads (128-byte swizzle, no multicast) of Q once and of K, V per 128-key
 //     tile into 2-stage rings; warp 9: TMEM allocation and every tcgen05.mma / commit.
 //     Registers are re-split after launch (setmaxnreg): 200 for the softmax warpgroups, 104
@@ -77,7 +77,11 @@ constexpr int NUM_THREADS = 384;
 constexpr int REGS_SOFTMAX = 200, REGS_OTHER = 104;
 constexpr int TMEM_COLS = 512;
 constexpr float RESCALE_LOG2 = 8.0f;
-constexpr int POLY_PAIRS = 1;          // of every 4 pairs of exponentials, on the FMA pipe
+// Of every 4 pairs of exponentials, POLY go to the FMA pipe (kernel template argument): 1
+// for launches that run at full clock, 0 for launches long enough to run under the power
+// cap, where the polynomial's extra instructions cost more energy than the MUFU work they
+// save (measured: N = 65536 1.1% faster with 0, N = 16384 1.3% slower).
+constexpr double kLongLaunchFlops = 2e13;
 constexpr int QBAND = 32;              // query tiles per band of the CTA order
 
 struct Misc {
@@ -113,7 +117,7 @@ __device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t bytes) {
 // log-sum-exps and deltas described at PrefillArgs::st instead of the output.
 // TRAIN: the training forward (fixed length only): the output, and for the backward the
 // branch-2 output O_2 / l_2 (PrefillArgs::tr_o2) and both log-sum-exps (tr_lse).
-template <bool WINDOW, bool VARLEN, bool STATS = false, bool TRAIN = false>
+template <bool WINDOW, bool VARLEN, bool STATS = false, bool TRAIN = false, int POLY = 1>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_v2_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -368,7 +372,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       m1 = n1;
       m2 = n2;
       // p = 2^(s sl2 - m), in place (0 for every key while the query has none visible); in
-      // every group of 8 keys the last POLY_PAIRS pairs go to the FMA pipe, the rest to MUFU
+      // every group of 8 keys the last POLY pairs go to the FMA pipe, the rest to MUFU
       const float nm1 = (WINDOW && m1 == -INFINITY) ? 0.f : -m1;
       const float nm2 = (WINDOW && m2 == -INFINITY) ? 0.f : -m2;
       float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
@@ -383,7 +387,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int i = 0; i < 8; i += 2) ffma2(xv[i], xv[i + 1], pb[i], pb[i + 1], sl2, sl2, nm, nm);
 #pragma unroll
           for (int i = 0; i < 8; i += 2) {
-            if (i >= 8 - 2 * POLY_PAIRS) {
+            if (i >= 8 - 2 * POLY) {
               exp2_fma2(pb[i], pb[i + 1], xv[i], xv[i + 1]);
             } else {
               pb[i] = ex2(xv[i]);
@@ -604,8 +608,9 @@ cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   if (dev >= 64 || !attr_set[dev]) {
-    const void* fns[4] = {(const void*)prefill_v2_kernel<false, false>, (const void*)prefill_v2_kernel<true, false>,
-                          (const void*)prefill_v2_kernel<false, true>, (const void*)prefill_v2_kernel<true, true>};
+    const void* fns[5] = {(const void*)prefill_v2_kernel<false, false>, (const void*)prefill_v2_kernel<true, false>,
+                          (const void*)prefill_v2_kernel<false, true>, (const void*)prefill_v2_kernel<true, true>,
+                          (const void*)prefill_v2_kernel<false, false, false, false, 0>};
     for (const void* fn : fns) {
       e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
       if (e != cudaSuccess) return e;
@@ -619,9 +624,17 @@ cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream) {
   if (varlen) {
     if (window) prefill_v2_kernel<true, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
     else prefill_v2_kernel<false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  } else if (window) {
+    prefill_v2_kernel<true, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   } else {
-    if (window) prefill_v2_kernel<true, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
-    else prefill_v2_kernel<false, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+    // algorithmic FLOPs of the launch: 4 d per attended (query, key) pair and query head
+    const double nq = a.N, nk = a.Nk;
+    const double pairs = a.causal ? nq * (nk - nq) + nq * (nq + 1) / 2 : nq * nk;
+    const double flops = 4.0 * a.d * a.Hq * (double)a.B * pairs;
+    if (flops >= kLongLaunchFlops)
+      prefill_v2_kernel<false, false, false, false, 0><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+    else
+      prefill_v2_kernel<false, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   }
   return cudaGetLastError();
 }
