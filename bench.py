@@ -313,14 +313,24 @@ def run_ours(args, rank, world, device):
     flush = in_bytes < 2 * L2_BYTES
     scratch = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device) if flush else None
 
-    def lambda_step():
-        da.diffattn_lambda(*vecs, depth=inp.depth, lambda_out=lam, lambda_init_out=li)
+    # the device tensors of one step; the end-to-end measurement below runs two such sets
+    # so that one step's copies overlap another step's kernels
+    S0 = {"q": q, "k": k, "v": v, "vecs": vecs, "lam": lam, "li": li, "out": out}
+    if backward:
+        S0.update(dy=dy, grads=grads)
 
-    def main_kernel():
+    def lambda_step(S=S0):
+        da.diffattn_lambda(*S["vecs"], depth=inp.depth, lambda_out=S["lam"], lambda_init_out=S["li"])
+
+    def main_kernel(S=S0):
+        q, k, v, lam, li, out = S["q"], S["k"], S["v"], S["lam"], S["li"], S["out"]
         if paged:
+            kp = k.view(inp.B * inp.N // ps, ps, inp.Hkv, inp.d)
+            vp = v.view(inp.B * inp.N // ps, ps, inp.Hkv, inp.d)
             da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws)
         elif backward:
-            da.diffattn_bwd_prefill(q, k, v, lam, dy, causal=inp.causal, workspace=ws, grads=grads)
+            da.diffattn_bwd_prefill(q, k, v, lam, S["dy"], causal=inp.causal, workspace=ws,
+                                    grads=S["grads"])
         elif decode and inp.variant == 1:
             da.diffattn_fwd_decode_v1(q, k, v, lam, li, out=out, apply_norm=inp.apply_norm,
                                       norm_eps=inp.eps, workspace=ws)
@@ -382,36 +392,87 @@ def run_ours(args, rank, world, device):
                 for n in ("lq1", "lk1", "lq2", "lk2")]
     if backward:
         host_in.append(torch.from_numpy(inp.extra["dy"].view(np.int16)).pin_memory())
-    dev_in = (q, k, v, dy) if backward else (q, k, v)
-    dev_out = grads if backward else (out,)
-    host_outs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dev_out]
+    dev_in_of = lambda S: (S["q"], S["k"], S["v"], S["dy"]) if backward else (S["q"], S["k"], S["v"])
+    dev_out_of = lambda S: S["grads"] if backward else (S["out"],)
+    S1 = {name: (torch.empty_like(t) if torch.is_tensor(t) else
+                 (tuple(torch.empty_like(x) for x in t) if isinstance(t, tuple) else
+                  [torch.empty_like(x) for x in t]))
+          for name, t in S0.items()}
+    sets = (S0, S1)
+    host_outs = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dev_out_of(S0)]
+                 for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host_in + host_vec)
-    d2h = sum(t.numel() * t.element_size() for t in host_outs)
+    d2h = sum(t.numel() * t.element_size() for t in host_outs[0])
     e2e_steps = max(3, min(args.steps, 10))
+    cs_in, cs_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
 
-    def e2e_step():
-        for src, dst in zip(host_in, dev_in):
+    def copy_in(S):
+        for src, dst in zip(host_in, dev_in_of(S)):
             dst.view(src.dtype).copy_(src, non_blocking=True)
-        for src, dst in zip(host_vec, vecs):
-            dst.copy_(src, non_blocking=True)
-        lambda_step()
-        main_kernel()
-        for dst, src in zip(host_outs, dev_out):
+        for src, dst in zip(host_vec, S["vecs"]):
             dst.copy_(src, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize(device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist is not None:
-        dist.barrier()
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    e2e_ms = e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_ms, dist, device)
-    e2e_val = job_rate(world, work, e2e_steps, e2e_ms, 1e9 if decode else 1e12)
+    def copy_out(S, ho):
+        for dst, src in zip(ho, dev_out_of(S)):
+            dst.copy_(src, non_blocking=True)
+
+    def e2e_serial(n):
+        # every step: inputs in, lambda + hot path, result out, one after the other
+        for _ in range(n):
+            copy_in(S0)
+            lambda_step()
+            main_kernel()
+            copy_out(S0, host_outs[0])
+
+    def e2e_pipelined(n):
+        # step i runs on buffer set i % 2 while step i + 1's inputs are copied in (cs_in) and
+        # step i - 1's result is copied out (cs_out); every step's bytes still cross the bus
+        ready = [torch.cuda.Event() for _ in range(n)]
+        done = [torch.cuda.Event() for _ in range(n)]
+        copied = [torch.cuda.Event() for _ in range(n)]
+        start = torch.cuda.Event()
+        start.record(stream)
+        cs_in.wait_event(start)
+        cs_out.wait_event(start)
+        with torch.cuda.stream(cs_in):
+            copy_in(sets[0])
+            ready[0].record(cs_in)
+        for i in range(n):
+            S = sets[i % 2]
+            stream.wait_event(ready[i])
+            if i >= 2:
+                stream.wait_event(copied[i - 2])  # set i % 2's result of step i - 2 is out
+            lambda_step(S)
+            main_kernel(S)
+            done[i].record(stream)
+            if i + 1 < n:
+                if i >= 1:
+                    cs_in.wait_event(done[i - 1])  # set (i + 1) % 2 is free once step i - 1 ran
+                with torch.cuda.stream(cs_in):
+                    copy_in(sets[(i + 1) % 2])
+                    ready[i + 1].record(cs_in)
+            cs_out.wait_event(done[i])
+            with torch.cuda.stream(cs_out):
+                copy_out(S, host_outs[i % 2])
+                copied[i].record(cs_out)
+        stream.wait_event(copied[n - 1])
+
+    def timed(fn):
+        fn(2)  # untimed: first use of the copy streams and the second buffer set
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist is not None:
+            dist.barrier()
+        e0.record(stream)
+        fn(e2e_steps)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+        return job_rate(world, work, e2e_steps, ms, 1e9 if decode else 1e12)
+
+    e2e_serial_val = timed(e2e_serial)
+    e2e_val = timed(e2e_pipelined)
+    del S1, sets
 
     kernel_name = (("decode_v1_split_kernel" if inp.variant == 1 else "decode_split_kernel")
                    if decode else f"prefill_v{inp.variant}_kernel")
@@ -453,12 +514,16 @@ def run_ours(args, rank, world, device):
                 "sustained_peak": peaks["bf16_tflops_sustained"]} if bound == "tensor" else {}),
         },
         "e2e": {"value": round(e2e_val, 3), "unit": unit, "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps},
+                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
+                "overlap": "step i on one of two device buffer sets while step i+1's inputs are "
+                           "copied in and step i-1's result copied out on two copy streams",
+                "serial_value": round(e2e_serial_val, 3)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "wall_s_timed": round(t_wall, 4),
     }
-    del q, k, v, out, dev_in, dev_out
+    S0.clear()  # the step closures keep the dict; release its tensors before the secondaries
+    del q, k, v, out, S0
     if backward:
         del dy, grads
     if paged:
