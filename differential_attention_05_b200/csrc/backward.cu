@@ -15,11 +15,13 @@
 // of dA_2 inside dS_2).
 //
 // Three launches, none with atomics (deterministic):
-//   bwd_rows_kernel : one warp per (query row, unit). Sweep 1 recomputes both branches'
+//   bwd_rows_kernel : one warp per (query row, unit), 8 rows per block sharing staged key
+//                     rows (see below). Sweep 1 recomputes both branches'
 //                     softmax statistics and O_1, O_2; it forms dO (the V1 norm backward),
 //                     delta_1, delta_2, the row's dlambda share, and stores them with the
 //                     log-sum-exps. Sweep 2 recomputes A_b row by row and accumulates dQ.
-//   bwd_keys_kernel : one warp per (key row, KV head): walks every query that sees the key,
+//   bwd_keys_kernel : one warp per (key row, KV head), 8 rows per block sharing staged
+//                     query rows: walks every query that sees the key,
 //                     for every unit that reads this KV head (V2: the pairs of the GQA
 //                     group, both branches), recomputing A_b from the stored log-sum-exps,
 //                     and accumulates dK and dV.
@@ -30,7 +32,6 @@
 namespace diffattn {
 
 namespace {
-constexpr int kWarps = 4;
 constexpr int kMaxD = 128;          // branch width
 constexpr int kMaxDv = 2 * kMaxD;   // value width (V1: 2d)
 constexpr int kPerLane = kMaxDv / 32;
@@ -96,50 +97,112 @@ __device__ __forceinline__ UnitRows unit_rows(const PrefillArgs& a, int u) {
 }
 }  // namespace
 
+// Both passes run kRowWarps rows per block, one per warp, over the same unit (row pass) or
+// KV head (key pass). Consecutive rows see nearly the same range of the other side, so the
+// block walks the union of its rows' ranges in blocks of 32 rows of the other side: all
+// warps stage those rows into shared memory as fp32 (one contiguous row per warp
+// instruction), then every warp reads them from there (row r at stride width + 4 floats, so
+// a quarter-warp reading 16 bytes from 8 different rows covers the 32 banks once). Warps
+// whose own row is out of range still stage and meet every block barrier.
+namespace {
+constexpr int kRowWarps = 8;
+constexpr int kBlk = 32;
+
+// dot product of two 16-byte-aligned shared fp32 rows, n a multiple of 4, in the order of
+// dot_row
+__device__ __forceinline__ float dot_sm(const float* x, const float* y, int n) {
+  float acc = 0.f;
+  for (int c = 0; c < n; c += 4) {
+    const float4 p = *reinterpret_cast<const float4*>(x + c);
+    const float4 q = *reinterpret_cast<const float4*>(y + c);
+    acc = fmaf(p.x, q.x, acc);
+    acc = fmaf(p.y, q.y, acc);
+    acc = fmaf(p.z, q.z, acc);
+    acc = fmaf(p.w, q.w, acc);
+  }
+  return acc;
+}
+
+// rows r0 .. r0 + n - 1 of a global tensor (row stride rs elements, first column at col0)
+// into shared rows of `width` floats at stride width + 4, by the block's warps
 template <typename T>
-__global__ void __launch_bounds__(kWarps * 32) bwd_rows_kernel(BwdArgs g) {
-  const PrefillArgs& a = g.f;
-  __shared__ __align__(16) float qsm[kWarps][2][kMaxD];
-  __shared__ __align__(16) float dsm[kWarps][kMaxDv];
+__device__ __forceinline__ void stage_rows(float* dst, const T* src, int64_t rs, int64_t col0,
+                                           int r0, int n, int width) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x * kWarps + warp;
-  const int u = blockIdx.y, b = blockIdx.z;
-  if (i >= a.N) return;
+  for (int r = warp; r < n; r += kRowWarps) {
+    const T* s = src + (int64_t)(r0 + r) * rs + col0;
+    float* t = dst + r * (width + 4);
+    for (int c = 4 * lane; c < width; c += 128) *reinterpret_cast<float4*>(t + c) = ld4(s + c);
+  }
+}
+
+size_t bwd_simt_smem_bytes(int d, int dv) {
+  const size_t stage = (size_t)kBlk * (2 * (d + 4) + (dv + 4)) + 4 * kBlk;
+  return (stage + (size_t)kRowWarps * (2 * d + dv)) * sizeof(float);
+}
+}  // namespace
+
+template <typename T>
+__global__ void __launch_bounds__(kRowWarps * 32) bwd_rows_kernel(BwdArgs g) {
+  const PrefillArgs& a = g.f;
   const int d = a.d, dv = a.dv;
-  const T* q = static_cast<const T*>(a.q) + b * a.qs[0] + (int64_t)i * a.qs[1];
+  extern __shared__ __align__(16) float sm[];
+  float* k1s = sm;                          // [kBlk][d + 1]
+  float* k2s = k1s + kBlk * (d + 4);        // [kBlk][d + 1]
+  float* vsb = k2s + kBlk * (d + 4);        // [kBlk][dv + 1]
+  float* qsm = vsb + kBlk * (dv + 4) + 4 * kBlk;  // [warp][2][d]
+  float* dsm = qsm + kRowWarps * 2 * d;     // [warp][dv]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ib = blockIdx.x * kRowWarps;
+  const int i = ib + warp;
+  const int u = blockIdx.y, b = blockIdx.z;
   const T* k = static_cast<const T*>(a.k) + b * a.ks[0];
   const T* v = static_cast<const T*>(a.v) + b * a.vs[0];
   const UnitRows ur = unit_rows(a, u);
-  int lo, hi;
-  key_range(a, i, lo, hi);
-  {
-    // (bounds-checked build) every row this warp reads or writes; the strides are
-    // non-negative, so the first and last key rows bound all the others
+  bool valid = i < a.N;
+  int lo = 0, hi = -1;
+  if (valid) key_range(a, i, lo, hi);
+  // the block's key range: key_range is monotone in the query row
+  int blo, bhi, t0, t1;
+  key_range(a, ib, blo, t0);
+  key_range(a, min(ib + kRowWarps, a.N) - 1, t1, bhi);
+  const int64_t row = ((int64_t)b * a.N + (valid ? i : 0)) * a.units + u;
+  if (valid) {
+    // (bounds-checked build) every row this warp reads or writes
     const int64_t qo = b * a.qs[0] + (int64_t)i * a.qs[1];
-    const int64_t row = ((int64_t)b * a.N + i) * a.units + u;
     const int64_t dq_off = a.variant == DIFFATTN_V1 ? (((int64_t)b * a.N + i) * a.units + u) * 2 * d
                                                     : (((int64_t)b * a.N + i) * a.Hq + 2 * u) * d;
-    bool ok = in_bounds(qo + ur.q1, d, a.ext_q, a.dev_status, a.dbg_status) &&
-              in_bounds(qo + ur.q2, d, a.ext_q, a.dev_status, a.dbg_status) &&
-              in_bounds(b * g.dys[0] + (int64_t)i * g.dys[1] + u * g.dys[2], dv, a.ext_out,
-                        a.dev_status, a.dbg_status) &&
-              in_bounds((g.w_do - g.w_base) + row * dv, dv, g.ext_ws, a.dev_status, a.dbg_status) &&
-              in_bounds((g.w_st - g.w_base) + row * 4, 4, g.ext_ws, a.dev_status, a.dbg_status) &&
-              in_bounds((g.w_dl - g.w_base) + ((int64_t)b * a.units + u) * a.N + i, 1, g.ext_ws,
-                        a.dev_status, a.dbg_status) &&
-              in_bounds(dq_off, 2 * d, g.ext_dq, a.dev_status, a.dbg_status);
-    if (lo <= hi)
-      for (int e = 0; e < 2; ++e) {
-        const int jj = e ? hi : lo;
-        ok = ok && in_bounds(b * a.ks[0] + (int64_t)jj * a.ks[1] + ur.k1, d, a.ext_k, a.dev_status, a.dbg_status) &&
-             in_bounds(b * a.ks[0] + (int64_t)jj * a.ks[1] + ur.k2, d, a.ext_k, a.dev_status, a.dbg_status) &&
-             in_bounds(b * a.vs[0] + (int64_t)jj * a.vs[1] + ur.v, dv, a.ext_v, a.dev_status, a.dbg_status);
-      }
-    if (!ok) return;
+    valid = in_bounds(qo + ur.q1, d, a.ext_q, a.dev_status, a.dbg_status) &&
+            in_bounds(qo + ur.q2, d, a.ext_q, a.dev_status, a.dbg_status) &&
+            in_bounds(b * g.dys[0] + (int64_t)i * g.dys[1] + u * g.dys[2], dv, a.ext_out,
+                      a.dev_status, a.dbg_status) &&
+            in_bounds((g.w_do - g.w_base) + row * dv, dv, g.ext_ws, a.dev_status, a.dbg_status) &&
+            in_bounds((g.w_st - g.w_base) + row * 4, 4, g.ext_ws, a.dev_status, a.dbg_status) &&
+            in_bounds((g.w_dl - g.w_base) + ((int64_t)b * a.units + u) * a.N + i, 1, g.ext_ws,
+                      a.dev_status, a.dbg_status) &&
+            in_bounds(dq_off, 2 * d, g.ext_dq, a.dev_status, a.dbg_status);
   }
-  for (int c = lane; c < d; c += 32) {
-    qsm[warp][0][c] = ld1(q + ur.q1 + c);
-    qsm[warp][1][c] = ld1(q + ur.q2 + c);
+  // (bounds-checked build) the block's first and last key rows bound the staged ones; the
+  // strides are non-negative
+  bool keys_ok = true;
+  if (blo <= bhi)
+    for (int e = 0; e < 2; ++e) {
+      const int jj = e ? bhi : blo;
+      keys_ok = keys_ok &&
+                in_bounds(b * a.ks[0] + (int64_t)jj * a.ks[1] + ur.k1, d, a.ext_k, a.dev_status, a.dbg_status) &&
+                in_bounds(b * a.ks[0] + (int64_t)jj * a.ks[1] + ur.k2, d, a.ext_k, a.dev_status, a.dbg_status) &&
+                in_bounds(b * a.vs[0] + (int64_t)jj * a.vs[1] + ur.v, dv, a.ext_v, a.dev_status, a.dbg_status);
+    }
+  if (!keys_ok) bhi = blo - 1;  // uniform over the block: stage nothing
+  valid = valid && keys_ok;
+  float* qw = qsm + warp * 2 * d;
+  float* dw = dsm + warp * dv;
+  if (valid) {
+    const T* q = static_cast<const T*>(a.q) + b * a.qs[0] + (int64_t)i * a.qs[1];
+    for (int c = lane; c < d; c += 32) {
+      qw[c] = ld1(q + ur.q1 + c);
+      qw[d + c] = ld1(q + ur.q2 + c);
+    }
   }
   __syncwarp();
   const float scale = 1.0f / sqrtf((float)d);
@@ -150,97 +213,108 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_rows_kernel(BwdArgs g) {
   float o1[kPerLane], o2[kPerLane];
 #pragma unroll
   for (int t = 0; t < kPerLane; ++t) o1[t] = o2[t] = 0.f;
-  for (int j0 = lo; j0 <= hi; j0 += 32) {
-    const int j = j0 + lane;
-    float s1 = -INFINITY, s2 = -INFINITY;
-    if (j <= hi) {
-      s1 = dot_row(k + (int64_t)j * a.ks[1] + ur.k1, qsm[warp][0], d) * scale;
-      s2 = dot_row(k + (int64_t)j * a.ks[1] + ur.k2, qsm[warp][1], d) * scale;
-    }
-    const float n1 = fmaxf(m1, warp_max(s1)), n2 = fmaxf(m2, warp_max(s2));
-    const float al1 = (m1 == -INFINITY) ? 0.f : expf(m1 - n1);
-    const float al2 = (m2 == -INFINITY) ? 0.f : expf(m2 - n2);
-    const float p1 = (j <= hi) ? expf(s1 - n1) : 0.f;
-    const float p2 = (j <= hi) ? expf(s2 - n2) : 0.f;
-    l1 = l1 * al1 + warp_sum(p1);
-    l2 = l2 * al2 + warp_sum(p2);
-    m1 = n1;
-    m2 = n2;
-#pragma unroll
-    for (int t = 0; t < kPerLane; ++t) {
-      o1[t] *= al1;
-      o2[t] *= al2;
-    }
-    const int jn = min(32, hi - j0 + 1);
-    for (int jj = 0; jj < jn; ++jj) {
-      const float w1 = __shfl_sync(0xffffffffu, p1, jj);
-      const float w2 = __shfl_sync(0xffffffffu, p2, jj);
-      const T* vr = v + (int64_t)(j0 + jj) * a.vs[1] + ur.v;
+  for (int j0 = blo; j0 <= bhi; j0 += kBlk) {
+    const int jn = min(kBlk, bhi - j0 + 1);
+    stage_rows(k1s, k, a.ks[1], ur.k1, j0, jn, d);
+    stage_rows(k2s, k, a.ks[1], ur.k2, j0, jn, d);
+    stage_rows(vsb, v, a.vs[1], ur.v, j0, jn, dv);
+    __syncthreads();
+    if (valid && j0 <= hi && j0 + jn - 1 >= lo) {
+      const int j = j0 + lane;
+      const bool vis = lane < jn && j >= lo && j <= hi;
+      float s1 = -INFINITY, s2 = -INFINITY;
+      if (vis) {
+        s1 = dot_sm(k1s + lane * (d + 4), qw, d) * scale;
+        s2 = dot_sm(k2s + lane * (d + 4), qw + d, d) * scale;
+      }
+      const float n1 = fmaxf(m1, warp_max(s1)), n2 = fmaxf(m2, warp_max(s2));
+      const float al1 = (m1 == -INFINITY) ? 0.f : expf(m1 - n1);
+      const float al2 = (m2 == -INFINITY) ? 0.f : expf(m2 - n2);
+      const float p1 = vis ? expf(s1 - n1) : 0.f;
+      const float p2 = vis ? expf(s2 - n2) : 0.f;
+      l1 = l1 * al1 + warp_sum(p1);
+      l2 = l2 * al2 + warp_sum(p2);
+      m1 = n1;
+      m2 = n2;
 #pragma unroll
       for (int t = 0; t < kPerLane; ++t) {
-        const int c = lane + 32 * t;
-        if (c < dv) {
-          const float x = ld1(vr + c);
-          o1[t] = fmaf(w1, x, o1[t]);
-          o2[t] = fmaf(w2, x, o2[t]);
+        o1[t] *= al1;
+        o2[t] *= al2;
+      }
+      for (int jj = 0; jj < jn; ++jj) {
+        const float w1 = __shfl_sync(0xffffffffu, p1, jj);
+        const float w2 = __shfl_sync(0xffffffffu, p2, jj);
+        const float* vr = vsb + jj * (dv + 4);
+#pragma unroll
+        for (int t = 0; t < kPerLane; ++t) {
+          const int c = lane + 32 * t;
+          if (c < dv) {
+            const float x = vr[c];
+            o1[t] = fmaf(w1, x, o1[t]);
+            o2[t] = fmaf(w2, x, o2[t]);
+          }
         }
       }
     }
+    __syncthreads();
   }
 
   // ---- dO (through the V1 norm), delta_1, delta_2, dlambda share
-  const T* dy = static_cast<const T*>(g.dy) + b * g.dys[0] + (int64_t)i * g.dys[1] + u * g.dys[2];
   float dO[kPerLane];
-  float so = 0.f, sdy = 0.f;
-#pragma unroll
-  for (int t = 0; t < kPerLane; ++t) {
-    const int c = lane + 32 * t;
-    o1[t] /= l1;
-    o2[t] /= l2;
-    const float o = o1[t] - lam * o2[t];
-    dO[t] = (c < dv) ? ld1(dy + c) : 0.f;
-    if (c < dv) {
-      so = fmaf(o, o, so);
-      sdy = fmaf(dO[t], o, sdy);
-    }
-  }
-  if (a.apply_norm) {
-    so = warp_sum(so);
-    sdy = warp_sum(sdy);
-    const float r2 = so / (float)dv + a.eps;
-    const float r = sqrtf(r2);
-    const float s = 1.0f - a.lambda_init[0];
-    const float proj = sdy / ((float)dv * r2);
+  float lse1 = 0.f, lse2 = 0.f, delta1 = 0.f, delta2 = 0.f;
+  if (valid) {
+    const T* dy = static_cast<const T*>(g.dy) + b * g.dys[0] + (int64_t)i * g.dys[1] + u * g.dys[2];
+    float so = 0.f, sdy = 0.f;
 #pragma unroll
     for (int t = 0; t < kPerLane; ++t) {
+      const int c = lane + 32 * t;
+      o1[t] /= l1;
+      o2[t] /= l2;
       const float o = o1[t] - lam * o2[t];
-      dO[t] = s / r * (dO[t] - o * proj);
+      dO[t] = (c < dv) ? ld1(dy + c) : 0.f;
+      if (c < dv) {
+        so = fmaf(o, o, so);
+        sdy = fmaf(dO[t], o, sdy);
+      }
     }
-  }
-  float e1 = 0.f, e2 = 0.f;
+    if (a.apply_norm) {
+      so = warp_sum(so);
+      sdy = warp_sum(sdy);
+      const float r2 = so / (float)dv + a.eps;
+      const float r = sqrtf(r2);
+      const float s = 1.0f - a.lambda_init[0];
+      const float proj = sdy / ((float)dv * r2);
 #pragma unroll
-  for (int t = 0; t < kPerLane; ++t) {
-    if (lane + 32 * t < dv) {
-      e1 = fmaf(dO[t], o1[t], e1);
-      e2 = fmaf(dO[t], o2[t], e2);
+      for (int t = 0; t < kPerLane; ++t) {
+        const float o = o1[t] - lam * o2[t];
+        dO[t] = s / r * (dO[t] - o * proj);
+      }
     }
-  }
-  const float delta1 = warp_sum(e1), delta2 = warp_sum(e2);
-  const int64_t row = ((int64_t)b * a.N + i) * a.units + u;
-  float* wdo = g.w_do + row * dv;
+    float e1 = 0.f, e2 = 0.f;
 #pragma unroll
-  for (int t = 0; t < kPerLane; ++t) {
-    const int c = lane + 32 * t;
-    if (c < dv) {
-      dsm[warp][c] = dO[t];
-      wdo[c] = dO[t];
+    for (int t = 0; t < kPerLane; ++t) {
+      if (lane + 32 * t < dv) {
+        e1 = fmaf(dO[t], o1[t], e1);
+        e2 = fmaf(dO[t], o2[t], e2);
+      }
     }
-  }
-  const float lse1 = m1 + logf(l1), lse2 = m2 + logf(l2);
-  if (lane == 0) {
-    float4 st = make_float4(lse1, lse2, delta1, delta2);
-    *reinterpret_cast<float4*>(g.w_st + row * 4) = st;
-    g.w_dl[((int64_t)b * a.units + u) * a.N + i] = -delta2;
+    delta1 = warp_sum(e1);
+    delta2 = warp_sum(e2);
+    float* wdo = g.w_do + row * dv;
+#pragma unroll
+    for (int t = 0; t < kPerLane; ++t) {
+      const int c = lane + 32 * t;
+      if (c < dv) {
+        dw[c] = dO[t];
+        wdo[c] = dO[t];
+      }
+    }
+    lse1 = m1 + logf(l1);
+    lse2 = m2 + logf(l2);
+    if (lane == 0) {
+      *reinterpret_cast<float4*>(g.w_st + row * 4) = make_float4(lse1, lse2, delta1, delta2);
+      g.w_dl[((int64_t)b * a.units + u) * a.N + i] = -delta2;
+    }
   }
   __syncwarp();
 
@@ -248,31 +322,40 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_rows_kernel(BwdArgs g) {
   float dq1[kPerLaneD], dq2[kPerLaneD];
 #pragma unroll
   for (int t = 0; t < kPerLaneD; ++t) dq1[t] = dq2[t] = 0.f;
-  for (int j0 = lo; j0 <= hi; j0 += 32) {
-    const int j = j0 + lane;
-    float ds1 = 0.f, ds2 = 0.f;
-    if (j <= hi) {
-      const float s1 = dot_row(k + (int64_t)j * a.ks[1] + ur.k1, qsm[warp][0], d) * scale;
-      const float s2 = dot_row(k + (int64_t)j * a.ks[1] + ur.k2, qsm[warp][1], d) * scale;
-      const float dp = dot_row(v + (int64_t)j * a.vs[1] + ur.v, dsm[warp], dv);
-      ds1 = expf(s1 - lse1) * (dp - delta1);
-      ds2 = -lam * expf(s2 - lse2) * (dp - delta2);
-    }
-    const int jn = min(32, hi - j0 + 1);
-    for (int jj = 0; jj < jn; ++jj) {
-      const float w1 = __shfl_sync(0xffffffffu, ds1, jj);
-      const float w2 = __shfl_sync(0xffffffffu, ds2, jj);
-      const T* kr = k + (int64_t)(j0 + jj) * a.ks[1];
+  for (int j0 = blo; j0 <= bhi; j0 += kBlk) {
+    const int jn = min(kBlk, bhi - j0 + 1);
+    stage_rows(k1s, k, a.ks[1], ur.k1, j0, jn, d);
+    stage_rows(k2s, k, a.ks[1], ur.k2, j0, jn, d);
+    stage_rows(vsb, v, a.vs[1], ur.v, j0, jn, dv);
+    __syncthreads();
+    if (valid && j0 <= hi && j0 + jn - 1 >= lo) {
+      const int j = j0 + lane;
+      float ds1 = 0.f, ds2 = 0.f;
+      if (lane < jn && j >= lo && j <= hi) {
+        const float s1 = dot_sm(k1s + lane * (d + 4), qw, d) * scale;
+        const float s2 = dot_sm(k2s + lane * (d + 4), qw + d, d) * scale;
+        const float dp = dot_sm(vsb + lane * (dv + 4), dw, dv);
+        ds1 = expf(s1 - lse1) * (dp - delta1);
+        ds2 = -lam * expf(s2 - lse2) * (dp - delta2);
+      }
+      for (int jj = 0; jj < jn; ++jj) {
+        const float w1 = __shfl_sync(0xffffffffu, ds1, jj);
+        const float w2 = __shfl_sync(0xffffffffu, ds2, jj);
+        const float* r1 = k1s + jj * (d + 4);
+        const float* r2 = k2s + jj * (d + 4);
 #pragma unroll
-      for (int t = 0; t < kPerLaneD; ++t) {
-        const int c = lane + 32 * t;
-        if (c < d) {
-          dq1[t] = fmaf(w1, ld1(kr + ur.k1 + c), dq1[t]);
-          dq2[t] = fmaf(w2, ld1(kr + ur.k2 + c), dq2[t]);
+        for (int t = 0; t < kPerLaneD; ++t) {
+          const int c = lane + 32 * t;
+          if (c < d) {
+            dq1[t] = fmaf(w1, r1[c], dq1[t]);
+            dq2[t] = fmaf(w2, r2[c], dq2[t]);
+          }
         }
       }
     }
+    __syncthreads();
   }
+  if (!valid) return;
   // dq: dense fp32 in q's shape (V1 [B,N,H,2,d]; V2 [B,N,Hq,d])
   float* dq_1;
   float* dq_2;
@@ -294,43 +377,61 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_rows_kernel(BwdArgs g) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kWarps * 32) bwd_keys_kernel(BwdArgs g) {
+__global__ void __launch_bounds__(kRowWarps * 32) bwd_keys_kernel(BwdArgs g) {
   const PrefillArgs& a = g.f;
-  __shared__ __align__(16) float ksm[kWarps][2][kMaxD];
-  __shared__ __align__(16) float vsm[kWarps][kMaxDv];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = blockIdx.x * kWarps + warp;  // key row
-  const int kh = blockIdx.y;                 // V1 head / V2 KV head
-  const int b = blockIdx.z;
-  if (j >= a.Nk) return;
   const int d = a.d, dv = a.dv;
+  extern __shared__ __align__(16) float sm[];
+  float* q1s = sm;                          // [kBlk][d + 1]
+  float* q2s = q1s + kBlk * (d + 4);        // [kBlk][d + 1]
+  float* dos = q2s + kBlk * (d + 4);        // [kBlk][dv + 1]
+  float4* sts = reinterpret_cast<float4*>(dos + kBlk * (dv + 4));  // [kBlk]
+  float* ksm = reinterpret_cast<float*>(sts + kBlk);  // [warp][2][d]
+  float* vsm = ksm + kRowWarps * 2 * d;     // [warp][dv]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int jb = blockIdx.x * kRowWarps;
+  const int j = jb + warp;                  // key row
+  const int kh = blockIdx.y;                // V1 head / V2 KV head
+  const int b = blockIdx.z;
   const bool v1 = a.variant == DIFFATTN_V1;
-  const int64_t k_off = b * a.ks[0] + (int64_t)j * a.ks[1] + (int64_t)kh * a.ks[2];
-  const int64_t v_off = b * a.vs[0] + (int64_t)j * a.vs[1] + (int64_t)kh * a.vs[2];
-  const int nkh_ = v1 ? a.units : a.Hkv;
-  const int64_t krow_ = ((int64_t)b * a.Nk + j) * nkh_ + kh;
+  bool valid = j < a.Nk;
+  const int64_t k_off = b * a.ks[0] + (int64_t)(valid ? j : 0) * a.ks[1] + (int64_t)kh * a.ks[2];
+  const int64_t v_off = b * a.vs[0] + (int64_t)(valid ? j : 0) * a.vs[1] + (int64_t)kh * a.vs[2];
+  const int nkh = v1 ? a.units : a.Hkv;
+  const int64_t krow = ((int64_t)b * a.Nk + (valid ? j : 0)) * nkh + kh;
   // (bounds-checked build) this key's rows and outputs
-  if (!(in_bounds(k_off, v1 ? 2 * d : d, a.ext_k, a.dev_status, a.dbg_status) &&
-        in_bounds(v_off, dv, a.ext_v, a.dev_status, a.dbg_status) &&
-        in_bounds(krow_ * (v1 ? 2 * d : d), v1 ? 2 * d : d, g.ext_dk, a.dev_status, a.dbg_status) &&
-        in_bounds(krow_ * dv, dv, g.ext_dv, a.dev_status, a.dbg_status)))
-    return;
-  const T* kr = static_cast<const T*>(a.k) + k_off;
-  const T* vr = static_cast<const T*>(a.v) + v_off;
-  for (int c = lane; c < d; c += 32) {
-    ksm[warp][0][c] = ld1(kr + c);
-    ksm[warp][1][c] = ld1(kr + (v1 ? d : 0) + c);
+  if (valid)
+    valid = in_bounds(k_off, v1 ? 2 * d : d, a.ext_k, a.dev_status, a.dbg_status) &&
+            in_bounds(v_off, dv, a.ext_v, a.dev_status, a.dbg_status) &&
+            in_bounds(krow * (v1 ? 2 * d : d), v1 ? 2 * d : d, g.ext_dk, a.dev_status, a.dbg_status) &&
+            in_bounds(krow * dv, dv, g.ext_dv, a.dev_status, a.dbg_status);
+  float* kw = ksm + warp * 2 * d;
+  float* vw = vsm + warp * dv;
+  if (valid) {
+    const T* kr = static_cast<const T*>(a.k) + k_off;
+    const T* vr = static_cast<const T*>(a.v) + v_off;
+    for (int c = lane; c < d; c += 32) {
+      kw[c] = ld1(kr + c);
+      kw[d + c] = ld1(kr + (v1 ? d : 0) + c);
+    }
+    for (int c = lane; c < dv; c += 32) vw[c] = ld1(vr + c);
   }
-  for (int c = lane; c < dv; c += 32) vsm[warp][c] = ld1(vr + c);
   __syncwarp();
   const float scale = 1.0f / sqrtf((float)d);
-  // queries that see key j: i + off >= j (causal) and i + off - window < j (window)
+  // queries that see key j: i + off >= j (causal) and i + off - window < j (window); both
+  // ends are monotone in j, so the block's range is the first key's start to the last's end
   const int off = a.Nk - a.N;
-  int i_lo = 0, i_hi = a.N - 1;
-  if (a.causal) {
-    i_lo = max(0, j - off);
-    if (a.window > 0) i_hi = min(a.N - 1, j - off + a.window - 1);
-  }
+  auto query_range = [&](int jj, int& lo, int& hi) {
+    lo = 0;
+    hi = a.N - 1;
+    if (a.causal) {
+      lo = max(0, jj - off);
+      if (a.window > 0) hi = min(a.N - 1, jj - off + a.window - 1);
+    }
+  };
+  int i_lo = 0, i_hi = -1, bilo, bihi, t0, t1;
+  if (valid) query_range(j, i_lo, i_hi);
+  query_range(jb, bilo, t0);
+  query_range(min(jb + kRowWarps, a.Nk) - 1, t1, bihi);
   // units reading this KV head: V1 the head itself; V2 the pairs of its GQA group
   const int u_lo = v1 ? kh : kh * (a.group / 2);
   const int u_hi = v1 ? kh + 1 : (kh + 1) * (a.group / 2);
@@ -345,61 +446,74 @@ __global__ void __launch_bounds__(kWarps * 32) bwd_keys_kernel(BwdArgs g) {
     const float lam = a.lambda[u];
     const UnitRows ur = unit_rows(a, u);
     const T* q = static_cast<const T*>(a.q) + b * a.qs[0];
-    if (i_lo <= i_hi) {
-      // (bounds-checked build) the first and last query rows bound the ones in between
+    const float* wdo = g.w_do + ((int64_t)b * a.N) * a.units * dv;
+    const float* wst = g.w_st + ((int64_t)b * a.N) * a.units * 4;
+    int hi_u = bihi;
+    if (bilo <= bihi) {
+      // (bounds-checked build) the first and last query rows bound the staged ones
       bool ok = true;
       for (int e = 0; e < 2; ++e) {
-        const int ii = e ? i_hi : i_lo;
+        const int ii = e ? bihi : bilo;
         const int64_t row = ((int64_t)b * a.N + ii) * a.units + u;
         ok = ok && in_bounds(b * a.qs[0] + (int64_t)ii * a.qs[1] + ur.q1, d, a.ext_q, a.dev_status, a.dbg_status) &&
              in_bounds(b * a.qs[0] + (int64_t)ii * a.qs[1] + ur.q2, d, a.ext_q, a.dev_status, a.dbg_status) &&
              in_bounds((g.w_st - g.w_base) + row * 4, 4, g.ext_ws, a.dev_status, a.dbg_status) &&
              in_bounds((g.w_do - g.w_base) + row * dv, dv, g.ext_ws, a.dev_status, a.dbg_status);
       }
-      if (!ok) return;
-    }
-    for (int i0 = i_lo; i0 <= i_hi; i0 += 32) {
-      const int i = i0 + lane;
-      float pv = 0.f, ds1 = 0.f, ds2 = 0.f;
-      if (i <= i_hi) {
-        const int64_t row = ((int64_t)b * a.N + i) * a.units + u;
-        const float4 st = *reinterpret_cast<const float4*>(g.w_st + row * 4);
-        const float s1 = dot_row(q + (int64_t)i * a.qs[1] + ur.q1, ksm[warp][0], d) * scale;
-        const float s2 = dot_row(q + (int64_t)i * a.qs[1] + ur.q2, ksm[warp][1], d) * scale;
-        const float p1 = expf(s1 - st.x), p2 = expf(s2 - st.y);
-        const float dp = dot_row(g.w_do + row * dv, vsm[warp], dv);
-        pv = p1 - lam * p2;
-        ds1 = p1 * (dp - st.z);
-        ds2 = -lam * p2 * (dp - st.w);
+      if (!ok) {
+        hi_u = bilo - 1;  // uniform over the block: stage nothing for this unit
+        valid = false;
       }
-      const int in = min(32, i_hi - i0 + 1);
-      for (int ii = 0; ii < in; ++ii) {
-        const float w = __shfl_sync(0xffffffffu, pv, ii);
-        const float w1 = __shfl_sync(0xffffffffu, ds1, ii);
-        const float w2 = __shfl_sync(0xffffffffu, ds2, ii);
-        const int64_t row = ((int64_t)b * a.N + i0 + ii) * a.units + u;
-        const float* dor = g.w_do + row * dv;
-        const T* qr = q + (int64_t)(i0 + ii) * a.qs[1];
-#pragma unroll
-        for (int t = 0; t < kPerLane; ++t) {
-          const int c = lane + 32 * t;
-          if (c < dv) dvv[t] = fmaf(w, dor[c], dvv[t]);
+    }
+    for (int i0 = bilo; i0 <= hi_u; i0 += kBlk) {
+      const int in = min(kBlk, hi_u - i0 + 1);
+      stage_rows(q1s, q, a.qs[1], ur.q1, i0, in, d);
+      stage_rows(q2s, q, a.qs[1], ur.q2, i0, in, d);
+      stage_rows(dos, wdo, (int64_t)a.units * dv, (int64_t)u * dv, i0, in, dv);
+      if (threadIdx.x < in)
+        sts[threadIdx.x] = *reinterpret_cast<const float4*>(wst + ((int64_t)(i0 + threadIdx.x) * a.units + u) * 4);
+      __syncthreads();
+      if (valid && i0 <= i_hi && i0 + in - 1 >= i_lo) {
+        const int i = i0 + lane;
+        float pv = 0.f, ds1 = 0.f, ds2 = 0.f;
+        if (lane < in && i >= i_lo && i <= i_hi) {
+          const float4 st = sts[lane];
+          const float s1 = dot_sm(q1s + lane * (d + 4), kw, d) * scale;
+          const float s2 = dot_sm(q2s + lane * (d + 4), kw + d, d) * scale;
+          const float p1 = expf(s1 - st.x), p2 = expf(s2 - st.y);
+          const float dp = dot_sm(dos + lane * (dv + 4), vw, dv);
+          pv = p1 - lam * p2;
+          ds1 = p1 * (dp - st.z);
+          ds2 = -lam * p2 * (dp - st.w);
         }
+        for (int ii = 0; ii < in; ++ii) {
+          const float w = __shfl_sync(0xffffffffu, pv, ii);
+          const float w1 = __shfl_sync(0xffffffffu, ds1, ii);
+          const float w2 = __shfl_sync(0xffffffffu, ds2, ii);
+          const float* dor = dos + ii * (dv + 4);
+          const float* r1 = q1s + ii * (d + 4);
+          const float* r2 = q2s + ii * (d + 4);
 #pragma unroll
-        for (int t = 0; t < kPerLaneD; ++t) {
-          const int c = lane + 32 * t;
-          if (c < d) {
-            dk1[t] = fmaf(w1, ld1(qr + ur.q1 + c), dk1[t]);
-            dk2[t] = fmaf(w2, ld1(qr + ur.q2 + c), dk2[t]);
+          for (int t = 0; t < kPerLane; ++t) {
+            const int c = lane + 32 * t;
+            if (c < dv) dvv[t] = fmaf(w, dor[c], dvv[t]);
+          }
+#pragma unroll
+          for (int t = 0; t < kPerLaneD; ++t) {
+            const int c = lane + 32 * t;
+            if (c < d) {
+              dk1[t] = fmaf(w1, r1[c], dk1[t]);
+              dk2[t] = fmaf(w2, r2[c], dk2[t]);
+            }
           }
         }
       }
+      __syncthreads();
     }
   }
+  if (!valid) return;
   // dense fp32 outputs in k's and v's shapes (V1 k [B,Nk,H,2,d], v [B,Nk,H,2d];
   // V2 k, v [B,Nk,Hkv,d]); V2's two branches read the same K row, so their parts add
-  const int nkh = v1 ? a.units : a.Hkv;
-  const int64_t krow = ((int64_t)b * a.Nk + j) * nkh + kh;
 #pragma unroll
   for (int t = 0; t < kPerLaneD; ++t) {
     const int c = lane + 32 * t;
@@ -454,16 +568,34 @@ cudaError_t launch_backward(BwdArgs g, void* workspace, cudaStream_t stream) {
   g.w_st = reinterpret_cast<float*>(w + up(rows * a.dv * sizeof(float)));
   g.w_dl = reinterpret_cast<float*>(w + up(rows * a.dv * sizeof(float)) + up(rows * 4 * sizeof(float)));
   g.w_base = g.w_do;
-  const dim3 grid_rows((a.N + kWarps - 1) / kWarps, a.units, a.B);
+  const dim3 grid_rows((a.N + kRowWarps - 1) / kRowWarps, a.units, a.B);
   const int nkh = a.variant == DIFFATTN_V1 ? a.units : a.Hkv;
-  const dim3 grid_keys((a.Nk + kWarps - 1) / kWarps, nkh, a.B);
-  if (g.bf16) {
-    bwd_rows_kernel<__nv_bfloat16><<<grid_rows, kWarps * 32, 0, stream>>>(g);
-    bwd_keys_kernel<__nv_bfloat16><<<grid_keys, kWarps * 32, 0, stream>>>(g);
-  } else {
-    bwd_rows_kernel<float><<<grid_rows, kWarps * 32, 0, stream>>>(g);
-    bwd_keys_kernel<float><<<grid_keys, kWarps * 32, 0, stream>>>(g);
+  const dim3 grid_keys((a.Nk + kRowWarps - 1) / kRowWarps, nkh, a.B);
+  const size_t smem = bwd_simt_smem_bytes(a.d, a.dv);
+  // (d <= 128, dv <= 256: at most 85 KB, above the 48 KB default)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  if (dev >= 64 || !attr_set[dev]) {
+    const int max_smem = (int)bwd_simt_smem_bytes(kMaxD, kMaxDv);
+    const void* fns[4] = {(const void*)bwd_rows_kernel<__nv_bfloat16>, (const void*)bwd_keys_kernel<__nv_bfloat16>,
+                          (const void*)bwd_rows_kernel<float>, (const void*)bwd_keys_kernel<float>};
+    for (const void* fn : fns) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+      if (e != cudaSuccess) return e;
+    }
+    if (dev < 64) attr_set[dev] = true;
   }
+  if (g.bf16) {
+    bwd_rows_kernel<__nv_bfloat16><<<grid_rows, kRowWarps * 32, smem, stream>>>(g);
+    bwd_keys_kernel<__nv_bfloat16><<<grid_keys, kRowWarps * 32, smem, stream>>>(g);
+  } else {
+    bwd_rows_kernel<float><<<grid_rows, kRowWarps * 32, smem, stream>>>(g);
+    bwd_keys_kernel<float><<<grid_keys, kRowWarps * 32, smem, stream>>>(g);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   return launch_dlambda_reduce(g, stream);
 }
 
