@@ -556,8 +556,10 @@ def _timed(fn, torch, reps=10, warm=3):
 
 def secondary(device, peaks, torch, da):
     """Other rows of the hot path, each timed alone (median of 10 launches):
-      * the V1 bf16 layer (B=2, 16 heads, N=4096, d=64) and the V2 prefill (N=16384, 64/8
-        heads, d=128) on their seeded synth tensors, lambda from the lambda kernel; the
+      * the V1 bf16 layer (B=2, 16 heads, N=4096, d=64), its backward (tensor cores; and
+        widened to fp32 through the exact kernels, median of 3), and the V2 prefill
+        (N=16384, 64/8 heads, d=128) on their seeded synth tensors, lambda from the lambda
+        kernel; the
         V2 tensors also as a 4096-key sliding-window layer and as a 2048-query chunk, and
         the V2 backward on the seeded N=4096 backward workload;
       * the V2 decode (batch 64, cache 32768; contiguous and over 16/256-token pages) and
@@ -592,16 +594,26 @@ def secondary(device, peaks, torch, da):
     ms = _timed(lambda: da.diffattn_fwd_prefill(q, k, v, lam, li, out=out, apply_norm=True,
                                                 norm_eps=inp.eps), torch)
     res["v1_layer"] = {"workload": inp.name, "inputs": seeded, **tflops(prefill_flops(inp), ms)}
-    # its backward (V1 runs the exact-fp32 kernels). Algorithmic FLOPs per attended (query,
-    # key) pair and head: scores 2 x 2d, dP = dO V^T 4d (V is 2d wide), dV 4d, dK_1 + dK_2
-    # 4d, dQ_1 + dQ_2 4d: 20 d
+    # its backward: bf16 on the tensor cores, and the same values widened to fp32 through the
+    # exact-fp32 kernels. Algorithmic FLOPs per attended (query, key) pair and head: scores
+    # 2 x 2d, dP = dO V^T 4d (V is 2d wide), dV 4d, dK_1 + dK_2 4d, dQ_1 + dQ_2 4d: 20 d
+    bwd_flops = 20.0 * inp.d * inp.H * inp.B * visible_pairs(inp.N, inp.N)
     dy = dev(synth.grad_out((inp.B, inp.N, inp.H, 2 * inp.d), 1001))
+    grads = (torch.empty(q.shape, dtype=torch.float32, device=device),
+             torch.empty(k.shape, dtype=torch.float32, device=device),
+             torch.empty(v.shape, dtype=torch.float32, device=device),
+             torch.empty(lam.shape, dtype=torch.float32, device=device))
     ms = _timed(lambda: da.diffattn_bwd_prefill(q, k, v, lam, dy, li, apply_norm=True,
-                                                norm_eps=inp.eps), torch, reps=3, warm=1)
+                                                norm_eps=inp.eps, grads=grads), torch)
+    res["v1_backward"] = {"workload": inp.name + " backward", "inputs": seeded,
+                          "path": "tensor cores", **tflops(bwd_flops, ms)}
+    q32, k32, v32, dy32 = q.float(), k.float(), v.float(), dy.float()
+    ms = _timed(lambda: da.diffattn_bwd_prefill(q32, k32, v32, lam, dy32, li, apply_norm=True,
+                                                norm_eps=inp.eps, grads=grads), torch, reps=3, warm=1)
     res["v1_backward_exact_fp32"] = {
-        "workload": inp.name + " backward", "inputs": seeded, "path": "exact-fp32 SIMT kernels",
-        **tflops(20.0 * inp.d * inp.H * inp.B * visible_pairs(inp.N, inp.N), ms)}
-    del q, k, v, out, dy
+        "workload": inp.name + " backward, inputs widened to fp32", "inputs": seeded,
+        "path": "exact-fp32 SIMT kernels", **tflops(bwd_flops, ms)}
+    del q, k, v, out, dy, q32, k32, v32, dy32, grads
     # ---- V2 prefill, its window and chunk forms
     inp = synth.config3()
     q, k, v = dev(inp.q), dev(inp.k), dev(inp.v)

@@ -239,13 +239,11 @@ int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t*
                      out, dev_status, stream);
 }
 
-// the tensor-core backward serves bf16 V2 with d = 128; everything else runs on the
-// exact-fp32 SIMT kernels. (V1 is not given a tensor-core path: its dlambda goes through the
-// per-head norm's backward, which takes the forward's bf16-accumulated output as input; a
-// tensor-core version of V1 built this way measured 0.5-1.1% relative RMS off the float64
-// reference in dlambda, above the 5e-3 the other outputs meet.)
+// the tensor-core backward serves bf16 V2 with d = 128 and bf16 V1 with d = 64; everything
+// else (fp32 inputs, other d) runs on the exact-fp32 SIMT kernels
 static bool bwd_tensor_core(const diffattn_prefill_params* p) {
-  return p->dtype == DIFFATTN_BF16 && p->variant == DIFFATTN_V2 && p->head_dim == 128;
+  return p->dtype == DIFFATTN_BF16 &&
+         ((p->variant == DIFFATTN_V2 && p->head_dim == 128) || (p->variant == DIFFATTN_V1 && p->head_dim == 64));
 }
 
 // backward: any d <= 128 with d % 4 == 0, f32 or bf16 inputs, fixed-length batches
@@ -274,7 +272,7 @@ int diffattn_bwd_workspace_size(const diffattn_prefill_params* p, size_t* bytes)
   } else {
     return DIFFATTN_ERR_INVALID_ARG;
   }
-  *bytes = bwd_tensor_core(p) ? bwd_tc_workspace_bytes(p->batch, p->seqlen, units)
+  *bytes = bwd_tensor_core(p) ? bwd_tc_workspace_bytes(p->variant, p->batch, p->seqlen, units)
                               : bwd_workspace_bytes(p->batch, p->seqlen, units, dv);
   return DIFFATTN_OK;
 }
@@ -295,7 +293,7 @@ int diffattn_bwd_prefill(const diffattn_prefill_params* p, const void* q, const 
   if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return DIFFATTN_ERR_MISALIGNED;
   const PrefillArgs& a = g.f;
   const bool tc = bwd_tensor_core(p);
-  const size_t need = tc ? bwd_tc_workspace_bytes(a.B, a.N, a.units)
+  const size_t need = tc ? bwd_tc_workspace_bytes(a.variant, a.B, a.N, a.units)
                          : bwd_workspace_bytes(a.B, a.N, a.units, a.dv);
   if (!workspace || workspace_bytes < need) return DIFFATTN_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIFFATTN_ERR_MISALIGNED;
@@ -355,7 +353,7 @@ int diffattn_bwd_prefill_saved(const diffattn_prefill_params* p, const void* q, 
   if (!aligned16(out) || !aligned16(o2) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return DIFFATTN_ERR_MISALIGNED;
   const PrefillArgs& a = g.f;
-  const size_t need = bwd_tc_workspace_bytes(a.B, a.N, a.units);
+  const size_t need = bwd_tc_workspace_bytes(DIFFATTN_V2, a.B, a.N, a.units);
   if (!workspace || workspace_bytes < need) return DIFFATTN_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DIFFATTN_ERR_MISALIGNED;
   g.bf16 = 1;

@@ -21,9 +21,13 @@
 //   3. bwd_v2_dq_kernel: one CTA per (64-query tile, pair, batch entry) walks the 128-key
 //      tiles its queries see: S = [Q_1; Q_2] K^T and dP = [dO; dO] V^T (branches stacked in
 //      the M = 128 rows), dS_b in bf16 into TMEM, dQ += dS K.
-// V1 runs the exact-fp32 kernels (backward.cu): its dlambda goes through the per-head norm's
-// backward, which takes the forward's bf16-accumulated output as input and amplifies its
-// rounding beyond the bf16 bound, so no tensor-core path is built for it.
+// V1 (d = 64, branches with their own keys K_1, K_2 and one value of width 2d) runs the same
+// kernels: its key row is (K_1 | K_2), 128 wide, and the query tile is laid out zero-padded,
+// rows 0-63 = (Q_1 | 0), rows 64-127 = (0 | Q_2), so one K = 128 MMA chain gives both
+// branches' scores, dK = [dS_1^T | dS_2^T] [Q_1 0; 0 Q_2] is (dK_1 | dK_2) in the key layout,
+// and dQ_b is the branch's own half of dS [K_1 | K_2]. Its statistics pass (the V1 forward
+// kernel, prefill_v1.cu) also takes dy back through the per-head norm and writes that dO in
+// bf16, which the kernels read in place of dy.
 // No atomics: every dK/dV row and every dQ row is summed inside one CTA in a fixed order.
 // The dQ kernel runs on a second stream beside the dK/dV kernel (see SideStream).
 // Warps 0-15 (four warpgroups, each taking a quarter of a step's columns) form the per-row
@@ -107,6 +111,7 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 }  // namespace kv
 }  // namespace
 
+template <bool V1>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_v2_dkdv_kernel(const __grid_constant__ BwdMaps maps, const BwdArgs g) {
   using namespace kv;
@@ -130,7 +135,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   const int qt_lo = i_lo / QT;
   const int n_qt = i_hi >= i_lo ? i_hi / QT - qt_lo + 1 : 0;
-  const int pairs = a.group / 2, u0 = gk * pairs;
+  const int pairs = V1 ? 1 : a.group / 2, u0 = gk * pairs;
   const int n_steps = n_qt * pairs;  // step t: pair u0 + t / n_qt, query tile qt_lo + t % n_qt
 
   if (threadIdx.x == 0) {
@@ -155,12 +160,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tmem_alloc(&ms.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
+  if (V1) {
+    // the zero quadrants of every stage's query tile (block 0 rows 64-127, block 1 rows
+    // 0-63); the copies never write them
+    for (int i = threadIdx.x; i < Q_STAGES * 2 * (HBLK / 16); i += NUM_THREADS) {
+      const int st = i / (2 * (HBLK / 16)), r = i % (2 * (HBLK / 16));
+      const int o = r < HBLK / 16 ? HBLK + 16 * r : BLK + 16 * (r - HBLK / 16);
+      *reinterpret_cast<uint4*>(smem + Q_OFF + st * 2 * BLK + o) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms.tmem_base;
   volatile int* abort_flag = &ms.abort;
-  const int rows = a.N + 64;  // statistics rows per (batch entry, pair)
+  const int rows = a.N + 64;  // statistics rows per (batch entry, unit)
 
   if (warp == W_TMA) {
     if (lane == 0) {
@@ -180,11 +195,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int sq = t % Q_STAGES, sd = t % D_STAGES;
         if (!mbar_wait(&ms.q_empty[sq], ((t / Q_STAGES) & 1) ^ 1, abort_flag)) break;
         uint8_t* qs = smem + Q_OFF + sq * 2 * BLK;
-        mbar_arrive_expect_tx(&ms.q_full[sq], 2 * BLK);
+        mbar_arrive_expect_tx(&ms.q_full[sq], V1 ? 2 * HBLK : 2 * BLK);
         for (int hf = 0; hf < 2; ++hf) {
-          // [Q_1; Q_2]: rows 0-63 branch 1, rows 64-127 branch 2 of each 64-column block
-          tma_load_4d(qs + hf * BLK, &maps.q, &ms.q_full[sq], 64 * hf, 2 * u, q0, b);
-          tma_load_4d(qs + hf * BLK + 64 * 128, &maps.q, &ms.q_full[sq], 64 * hf, 2 * u + 1, q0, b);
+          if (V1) {
+            // (Q_1 | 0) in rows 0-63, (0 | Q_2) in rows 64-127: block hf gets branch hf
+            tma_load_4d(qs + hf * BLK + hf * HBLK, &maps.q, &ms.q_full[sq], 64 * hf, u, q0, b);
+          } else {
+            // [Q_1; Q_2]: rows 0-63 branch 1, rows 64-127 branch 2 of each 64-column block
+            tma_load_4d(qs + hf * BLK, &maps.q, &ms.q_full[sq], 64 * hf, 2 * u, q0, b);
+            tma_load_4d(qs + hf * BLK + 64 * 128, &maps.q, &ms.q_full[sq], 64 * hf, 2 * u + 1, q0, b);
+          }
         }
         q_issued = t + 1;
         if (!mbar_wait(&ms.d_empty[sd], ((t / D_STAGES) & 1) ^ 1, abort_flag)) break;
@@ -311,9 +331,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto chunk = [&](auto all_visible) {
         const int c = wgr;
         float s1[16], s2[16], dp[16];
-        tmem_ld16f(lane_addr + C_S + 16 * c, s1);
-        tmem_ld16f(lane_addr + C_S + 64 + 16 * c, s2);
-        tmem_ld16f(lane_addr + C_DP + 16 * c, dp);
+        tmem_ld16f(lane_addr + kv::C_S + 16 * c, s1);
+        tmem_ld16f(lane_addr + kv::C_S + 64 + 16 * c, s2);
+        tmem_ld16f(lane_addr + kv::C_DP + 16 * c, dp);
         tmem_wait_ld();
         // the next step's S^T and dP^T may now overwrite their columns (one arrival per warp:
         // 512 single-thread arrivals on one barrier serialise)
@@ -349,8 +369,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // dS block
         *reinterpret_cast<uint4*>(pc_row + pc_c0) = make_uint4(pc[0], pc[1], pc[2], pc[3]);
         *reinterpret_cast<uint4*>(pc_row + pc_c1) = make_uint4(pc[4], pc[5], pc[6], pc[7]);
-        tmem_st8(lane_addr + C_DS + 8 * c, d1);
-        tmem_st8(lane_addr + C_DS + 32 + 8 * c, d2);
+        tmem_st8(lane_addr + kv::C_DS + 8 * c, d1);
+        tmem_st8(lane_addr + kv::C_DS + 32 + 8 * c, d2);
       };
       if (full) chunk(std::true_type{});
       else chunk(std::false_type{});
@@ -437,6 +457,7 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 }  // namespace dqk
 }  // namespace
 
+template <bool V1>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     bwd_v2_dq_kernel(const __grid_constant__ BwdMaps maps, const BwdArgs g) {
   using namespace dqk;
@@ -453,7 +474,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int u = (int)(blockIdx.x % per_qt) % a.units;
   const int b = (int)(blockIdx.x % per_qt) / a.units;
   const int q0 = qt * QT;
-  const int gk = (2 * u) / a.group;
+  const int gk = V1 ? u : (2 * u) / a.group;
   const int off = a.Nk - a.N;
   const int khi = a.causal ? min(q0 + QT - 1 + off, a.Nk - 1) : a.Nk - 1;
   const int klo = (a.causal && a.window > 0) ? max(0, q0 + off - a.window + 1) : 0;
@@ -482,6 +503,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tmem_alloc(&ms.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
+  if (V1) {
+    // the zero quadrants of the query tile: block 0 rows 64-127, block 1 rows 0-63
+    for (int i = threadIdx.x; i < 2 * (HBLK / 16); i += NUM_THREADS) {
+      const int o = i < HBLK / 16 ? HBLK + 16 * i : BLK + 16 * (i - HBLK / 16);
+      *reinterpret_cast<uint4*>(smem + QS_OFF + o) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -497,10 +526,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&maps.dy);
       const int64_t st_off = (((int64_t)b * a.units + u) * rows + q0) * 4;  // (workspace offset)
       const bool st_ok = in_bounds((g.w_st - g.w_base) + st_off, 256, g.ext_ws, a.dev_status, a.dbg_status);
-      mbar_arrive_expect_tx(&ms.q_full, 2 * BLK + 2 * BLK + (st_ok ? 1024 : 0));
+      mbar_arrive_expect_tx(&ms.q_full, (V1 ? 2 * HBLK : 2 * BLK) + 2 * BLK + (st_ok ? 1024 : 0));
       for (int hf = 0; hf < 2; ++hf) {
-        tma_load_4d(smem + QS_OFF + hf * BLK, &maps.q, &ms.q_full, 64 * hf, 2 * u, q0, b);
-        tma_load_4d(smem + QS_OFF + hf * BLK + 64 * 128, &maps.q, &ms.q_full, 64 * hf, 2 * u + 1, q0, b);
+        if (V1) {
+          tma_load_4d(smem + QS_OFF + hf * BLK + hf * HBLK, &maps.q, &ms.q_full, 64 * hf, u, q0, b);
+        } else {
+          tma_load_4d(smem + QS_OFF + hf * BLK, &maps.q, &ms.q_full, 64 * hf, 2 * u, q0, b);
+          tma_load_4d(smem + QS_OFF + hf * BLK + 64 * 128, &maps.q, &ms.q_full, 64 * hf, 2 * u + 1, q0, b);
+        }
         // dO in both halves: the branch-2 rows need dP = dO V^T as well
         tma_load_4d(smem + DO_OFF + hf * BLK, &maps.dy, &ms.q_full, 64 * hf, u, q0, b);
         tma_load_4d(smem + DO_OFF + hf * BLK + 64 * 128, &maps.dy, &ms.q_full, 64 * hf, u, q0, b);
@@ -613,8 +646,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t ds[16];
       auto chunk = [&](int c, auto all_visible) {
         float sv[32], dp[32];
-        tmem_ld32f(lane_addr + C_S + 32 * c, sv);
-        tmem_ld32f(lane_addr + C_DP + 32 * c, dp);
+        tmem_ld32f(lane_addr + dqk::C_S + 32 * c, sv);
+        tmem_ld32f(lane_addr + dqk::C_DP + 32 * c, dp);
         tmem_wait_ld();
         // the next step's S and dP may now overwrite these columns (one arrival per warp)
         tc_fence_before();
@@ -652,13 +685,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (ok) {
       const float scale = rsqrtf((float)a.d);
       const int64_t qrow = (int64_t)b * a.N + (qi < a.N ? qi : 0);
-      const bool store = qi < a.N && in_bounds((qrow * a.Hq + 2 * u + br) * 128, 128, g.ext_dq,
-                                               a.dev_status, a.dbg_status);
-      // the 128 columns of query head 2u + br
-      float4* dq4 = reinterpret_cast<float4*>(g.dq + (qrow * a.Hq + 2 * u + br) * 128);
-      const uint32_t col0 = C_DQ;
+      // V2: the 128 columns of query head 2u + br; V1: branch br's own half (columns
+      // 64 br ..) of dS [K_1 | K_2], into q's [.., H, 2, d] layout
+      const int64_t dq_off = V1 ? (qrow * a.units + u) * 128 + 64 * br : (qrow * a.Hq + 2 * u + br) * 128;
+      const bool store = qi < a.N && in_bounds(dq_off, V1 ? 64 : 128, g.ext_dq, a.dev_status, a.dbg_status);
+      float4* dq4 = reinterpret_cast<float4*>(g.dq + dq_off);
+      const uint32_t col0 = C_DQ + (V1 ? 64u * br : 0u);  // br is warp-uniform
       const int c = wgr;  // this warpgroup's 32 columns (warp-uniform)
-      {
+      if (c < (V1 ? 2 : 4)) {
         if (n_kt > 0) {
           tc_fence_after();
           float x[32];
@@ -693,10 +727,12 @@ namespace {
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 }  // namespace
 
-// statistics rows (N + 64 per entry and pair) and the dlambda shares
-size_t bwd_tc_workspace_bytes(int B, int N, int units) {
-  return up256((size_t)B * units * (N + 64) * 4 * sizeof(float)) +
-         up256((size_t)B * units * N * sizeof(float));
+// statistics rows (N + 64 per entry and unit), the dlambda shares and, for V1, the bf16 dO
+size_t bwd_tc_workspace_bytes(int variant, int B, int N, int units) {
+  size_t n = up256((size_t)B * units * (N + 64) * 4 * sizeof(float)) +
+             up256((size_t)B * units * N * sizeof(float));
+  if (variant == DIFFATTN_V1) n += up256((size_t)B * N * units * 128 * 2);
+  return n;
 }
 
 namespace {
@@ -781,21 +817,33 @@ SideStream* side_stream(int dev) {
 // steps 2-4 of the tensor-core backward, once the statistics rows are in the workspace
 cudaError_t backward_tc_kernels(const BwdArgs& g, cudaStream_t stream) {
   const PrefillArgs& a = g.f;
-  // dK/dV and dQ: q [B, N, Hq, 128], k, v [B, N, Hkv, 128], dO = dy [B, N, Hq/2, 128]
+  const bool v1 = a.variant == DIFFATTN_V1;
+  // dK/dV and dQ. V2: q [B, N, Hq, 128], k, v [B, N, Hkv, 128], dO = dy [B, N, Hq/2, 128].
+  // V1: q, k, v [B, N, H, 128] ((Q_1 | Q_2), (K_1 | K_2), V), dO the bf16 workspace rows
+  // [B, N, H, 128].
   BwdMaps maps;
-  if (!make_map(&maps.q, a.q, 128, a.Hq, a.N, a.B, a.qs, 64)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.q, a.q, 128, v1 ? a.units : a.Hq, a.N, a.B, a.qs, 64)) return cudaErrorInvalidValue;
   if (!make_map(&maps.k, a.k, 128, a.Hkv, a.Nk, a.B, a.ks, 128)) return cudaErrorInvalidValue;
   if (!make_map(&maps.v, a.v, 128, a.Hkv, a.Nk, a.B, a.vs, 128)) return cudaErrorInvalidValue;
-  if (!make_map(&maps.dy, g.dy, 128, a.units, a.N, a.B, g.dys, 64)) return cudaErrorInvalidValue;
+  if (v1) {
+    const int64_t ds[3] = {(int64_t)a.N * a.units * 128, (int64_t)a.units * 128, 128};
+    if (!make_map(&maps.dy, g.w_do16, 128, a.units, a.N, a.B, ds, 64)) return cudaErrorInvalidValue;
+  } else {
+    if (!make_map(&maps.dy, g.dy, 128, a.units, a.N, a.B, g.dys, 64)) return cudaErrorInvalidValue;
+  }
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   static bool attr_set[64] = {};
   if (dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(bwd_v2_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kv::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(bwd_v2_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    const void* kv_fns[2] = {(const void*)bwd_v2_dkdv_kernel<false>, (const void*)bwd_v2_dkdv_kernel<true>};
+    const void* dq_fns[2] = {(const void*)bwd_v2_dq_kernel<false>, (const void*)bwd_v2_dq_kernel<true>};
+    for (int i = 0; i < 2; ++i) {
+      e = cudaFuncSetAttribute(kv_fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, kv::SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(dq_fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, dqk::SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+    }
     if (dev < 64) attr_set[dev] = true;
   }
   const long long kv_ctas = (long long)((a.Nk + kv::KT - 1) / kv::KT) * a.Hkv * a.B;
@@ -809,10 +857,12 @@ cudaError_t backward_tc_kernels(const BwdArgs& g, cudaStream_t stream) {
     if ((e = cudaStreamWaitEvent(ss->s, ss->fork, 0)) != cudaSuccess) return e;
     dq_stream = ss->s;
   }
-  bwd_v2_dkdv_kernel<<<(unsigned)kv_ctas, NUM_THREADS, kv::SMEM_BYTES, stream>>>(maps, g);
+  if (v1) bwd_v2_dkdv_kernel<true><<<(unsigned)kv_ctas, NUM_THREADS, kv::SMEM_BYTES, stream>>>(maps, g);
+  else bwd_v2_dkdv_kernel<false><<<(unsigned)kv_ctas, NUM_THREADS, kv::SMEM_BYTES, stream>>>(maps, g);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_v2_dq_kernel<<<(unsigned)dq_ctas, NUM_THREADS, dqk::SMEM_BYTES, dq_stream>>>(maps, g);
+  if (v1) bwd_v2_dq_kernel<true><<<(unsigned)dq_ctas, NUM_THREADS, dqk::SMEM_BYTES, dq_stream>>>(maps, g);
+  else bwd_v2_dq_kernel<false><<<(unsigned)dq_ctas, NUM_THREADS, dqk::SMEM_BYTES, dq_stream>>>(maps, g);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (ss) {
@@ -826,9 +876,11 @@ void set_tc_workspace(BwdArgs& g, void* workspace) {
   const PrefillArgs& a = g.f;
   uint8_t* w = static_cast<uint8_t*>(workspace);
   const size_t st_bytes = up256((size_t)a.B * a.units * (a.N + 64) * 4 * sizeof(float));
+  const size_t dl_bytes = up256((size_t)a.B * a.units * a.N * sizeof(float));
   g.w_st = reinterpret_cast<float*>(w);
   g.w_dl = reinterpret_cast<float*>(w + st_bytes);
   g.w_do = nullptr;
+  g.w_do16 = a.variant == DIFFATTN_V1 ? static_cast<void*>(w + st_bytes + dl_bytes) : nullptr;
   g.w_base = g.w_st;
 }
 
@@ -836,7 +888,8 @@ void set_tc_workspace(BwdArgs& g, void* workspace) {
 
 cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream) {
   const PrefillArgs& a = g.f;
-  if (a.cu_q || a.variant != DIFFATTN_V2 || a.d != 128) return cudaErrorNotSupported;
+  const bool v1 = a.variant == DIFFATTN_V1;
+  if (a.cu_q || (v1 ? a.d != 64 : a.d != 128)) return cudaErrorNotSupported;
   set_tc_workspace(g, workspace);
   // 1. statistics: the forward kernel in its statistics mode
   PrefillArgs fa = a;
@@ -849,7 +902,9 @@ cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream) 
   fa.ext_st_dy = a.ext_out;  // dy has the output's layout
   fa.ext_st = (int64_t)a.B * a.units * (a.N + 64) * 4;
   fa.ext_st_dl = (int64_t)a.B * a.units * a.N;
-  cudaError_t e = launch_prefill_v2_stats(fa, stream);
+  fa.st_do = g.w_do16;
+  fa.ext_st_do = (int64_t)a.B * a.N * a.units * 128;
+  cudaError_t e = v1 ? launch_prefill_v1_stats(fa, stream) : launch_prefill_v2_stats(fa, stream);
   if (e != cudaSuccess) return e;
   return backward_tc_kernels(g, stream);
 }

@@ -33,15 +33,19 @@ struct PrefillArgs {
   const int32_t* cu_q;
   const int32_t* cu_k;
   int total_q, total_k;
-  // V2 statistics pass of the backward (launch_prefill_v2_stats): instead of the output,
-  // per (query, pair) the log2-domain log-sum-exps of both branches and
-  // delta_b = dy . (A_b V) go to st[((b * units + u) * st_rows + i) * 4 + 0..3], and the
-  // row's dlambda share -delta_2 to dl[(b * units + u) * N + i]
+  // statistics pass of the backward (launch_prefill_v2_stats, launch_prefill_v1_stats):
+  // instead of the output, per (query, unit) the log2-domain log-sum-exps of both branches
+  // and delta_b = dO . (A_b V) go to st[((b * units + u) * st_rows + i) * 4 + 0..3], and
+  // the row's dlambda share -dO . (A_2 V) to dl[(b * units + u) * N + i]. V2: dO = dy. V1:
+  // dO is dy taken back through the per-head norm, written in bf16 to
+  // st_do[((b * N + i) * units + u) * 2d + ..] (dense [B, N, H, 2d]); the deltas take that
+  // bf16 dO, the dlambda share the fp32 one
   const void* st_dy;
   int64_t st_dys[3];
   float* st;
   float* st_dl;
   int st_rows;
+  void* st_do;
   // training forward (launch_prefill_v2_train): the branch-2 output O_2 / l_2 of every
   // (query, pair) in out's layout and dtype, and lse[((b * units + u) * N + i) * 2 + 0..1],
   // the log2-domain log-sum-exps of both branches
@@ -50,7 +54,7 @@ struct PrefillArgs {
   // element extents (one past the largest element offset the shapes and strides reach) of
   // q, k, v, out and the statistics-pass tensors, and the bounds-checked build's own status
   // word (see in_bounds in common.cuh; unused by the normal build)
-  int64_t ext_q, ext_k, ext_v, ext_out, ext_st_dy, ext_st, ext_st_dl, ext_tr_lse;
+  int64_t ext_q, ext_k, ext_v, ext_out, ext_st_dy, ext_st, ext_st_dl, ext_st_do, ext_tr_lse;
   int* dbg_status;
 };
 
@@ -69,6 +73,7 @@ struct BwdArgs {
   float* w_do;               // [B, N, units, dv] gradient reaching O
   float* w_st;               // [B, N, units, 4] lse_1, lse_2, delta_1, delta_2
   float* w_dl;               // [B, units, N] per-row dlambda shares
+  void* w_do16;              // V1 tensor-core path: dO in bf16 [B, N, H, 2d]
   // element extents of dq, dk, dv (dense) and of the workspace in floats, which starts at
   // w_base (bounds-checked build, see in_bounds in common.cuh)
   int64_t ext_dq, ext_dk, ext_dv, ext_ws;
@@ -141,6 +146,7 @@ cudaError_t launch_prefill_f32(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_v1(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_v2(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_v2_stats(const PrefillArgs& a, cudaStream_t stream);
+cudaError_t launch_prefill_v1_stats(const PrefillArgs& a, cudaStream_t stream);
 cudaError_t launch_prefill_v2_train(const PrefillArgs& a, cudaStream_t stream);
 
 // split-KV decode (V2, bf16, d = 128, 8 query heads per KV head)
@@ -155,7 +161,7 @@ cudaError_t launch_decode_v1(const DecodeArgs& a, cudaStream_t stream);
 size_t bwd_workspace_bytes(int B, int N, int units, int dv);
 cudaError_t launch_backward(BwdArgs g, void* workspace, cudaStream_t stream);
 cudaError_t launch_dlambda_reduce(const BwdArgs& g, cudaStream_t stream);
-size_t bwd_tc_workspace_bytes(int B, int N, int units);
+size_t bwd_tc_workspace_bytes(int variant, int B, int N, int units);
 cudaError_t launch_backward_tc(BwdArgs g, void* workspace, cudaStream_t stream);
 // the same from a training forward's saved O_2 / l_2 and log-sum-exps (no recompute)
 cudaError_t launch_backward_tc_saved(BwdArgs g, const void* out, const void* o2, const float* lse,

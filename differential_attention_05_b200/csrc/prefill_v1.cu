@@ -92,6 +92,8 @@ struct Misc {
   float ex_l[2][BM];      // epilogue: [branch][row] row sums
   float ex_c[BM];         // epilogue: c
   float ssx[2][BM];       // V1 norm: partial sums of squares
+  float ex_m[2][BM];      // statistics pass: [branch][row] maxima
+  float ex_s[3][2][BM];   //                  [quantity][half][row] partial dot products
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
@@ -104,7 +106,15 @@ __device__ __forceinline__ void bar_softmax() { asm volatile("bar.sync 1, 256;" 
 // only an upper end; that case compiles without the lower-end and unset-row checks.
 // VARLEN: a variable-length batch (a.cu_q != nullptr); the fixed-length instantiation
 // takes its sizes from the parameters alone.
-template <bool WINDOW, bool VARLEN>
+// STATS: the statistics pass of the backward (fixed length only). Instead of the output the
+// epilogue writes the gradient reaching o through the norm (PrefillArgs::st_do, bf16), the
+// log-sum-exps, the deltas and the dlambda share (PrefillArgs::st, st_dl). The backward
+// amplifies errors of o (the norm's backward projects dy against o, and on the usual inputs
+// O_1 and O_2 are nearly parallel, so dlambda = -sum dO . O_2 keeps only their small
+// difference), so here each P.V operand is split into a bf16 head and a bf16 remainder,
+// x = hi(x) + lo(x) with |x - hi - lo| <= 2^-18 |x|, and both parts go through the MMA: D
+// and O_2 come out as accurate as fp32 accumulation of fp32 probabilities.
+template <bool WINDOW, bool VARLEN, bool STATS = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefill_v1_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -246,6 +256,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
           umma_ts(tmem + COL_D, tmem + 128u * f + kk * 8, vd, IDESC_PV, acc);
           umma_ts(tmem + COL_O2, tmem + 128u * f + 32u + kk * 8, vd, IDESC_PV, acc);
+          if constexpr (STATS) {
+            // the remainders, over S_2's columns: keys 32 h .. 32 h + 31 at 64 + 32 h (x)
+            // and 64 + 32 h + 16 (p2)
+            const uint32_t lo = 128u * f + 64u + 32u * (kk >> 1) + 8u * (kk & 1);
+            umma_ts(tmem + COL_D, tmem + lo, vd, IDESC_PV, 1u);
+            umma_ts(tmem + COL_O2, tmem + lo + 16u, vd, IDESC_PV, 1u);
+          }
         }
         tc_commit(&ms.pv_done);
         tc_commit(&ms.v_empty[st]);
@@ -399,7 +416,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       c = cn;
-      // operands: p1 - c p2 -> columns 0..31, p2 -> columns 32..63 (bf16 over S_1)
+      // operands: p1 - c p2 -> columns 0..31, p2 -> columns 32..63 (bf16 over S_1); the
+      // statistics pass adds their remainders over the p2 columns of S_2 just read
       const float nc = -c;
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
@@ -413,9 +431,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ffma2(w0, w1, q2[e], q2[e + 1], nc, nc, p[ch * 32 + e], p[ch * 32 + e + 1]);
           pa[e / 2] = pack_bf16(w0, w1);
           pb[e / 2] = pack_bf16(q2[e], q2[e + 1]);
+          if constexpr (STATS) {
+            // the remainder x - hi(x) is exact in fp32; keep it in the registers of x
+            p[ch * 32 + e] = w0 - __uint_as_float(pa[e / 2] << 16);
+            p[ch * 32 + e + 1] = w1 - __uint_as_float(pa[e / 2] & 0xffff0000u);
+            q2[e] -= __uint_as_float(pb[e / 2] << 16);
+            q2[e + 1] -= __uint_as_float(pb[e / 2] & 0xffff0000u);
+          }
         }
         tmem_st16(sb + ch * 16, pa);
         tmem_st16(sb + 32 + ch * 16, pb);
+        if constexpr (STATS) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            pa[e / 2] = pack_bf16(p[ch * 32 + e], p[ch * 32 + e + 1]);
+            pb[e / 2] = pack_bf16(q2[e], q2[e + 1]);
+          }
+          tmem_st16(sb + 64 + ch * 32, pa);
+          tmem_st16(sb + 64 + ch * 32 + 16, pb);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -450,29 +484,117 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int e = 0; e < 64; ++e) ss = fmaf(y[e], y[e], ss);
     }
-    float sc = 1.f;
-    ms.ssx[wg][row] = ss;
-    bar_softmax();
-    if (a.apply_norm)
-      sc = rsqrtf((ms.ssx[0][row] + ms.ssx[1][row]) * (1.f / 128.f) + a.eps) *
-           (1.f - a.lambda_init[0]);
-    // (a variable-length tile reads its sequence back from shared memory, keeping the
-    // registers of the key loop free)
-    const int o_nq = VARLEN ? ms.seq_nq : a.N, o_b = VARLEN ? ms.seq_bc : b;
-    const int o_q0 = VARLEN ? ms.seq_q0 : 0;
-    const int64_t o_off = (int64_t)o_b * a.os[0] + (int64_t)(o_q0 + qi) * a.os[1] +
-                          (int64_t)u * a.os[2] + wg * 64;
-    if (ok && qi < o_nq && in_bounds(o_off, 64, a.ext_out, a.dev_status, a.dbg_status)) {
-      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + o_off;
-      uint4* o4 = reinterpret_cast<uint4*>(ob);
+    if constexpr (STATS) {
+      // dy over this thread's 64 channels (the output's layout)
+      float gr[64];
+      const int64_t dy_off = (int64_t)b * a.st_dys[0] + (int64_t)qi * a.st_dys[1] +
+                             (int64_t)u * a.st_dys[2] + wg * 64;
+      if (ok && qi < a.N && in_bounds(dy_off, 64, a.ext_st_dy, a.dev_status, a.dbg_status)) {
+        const uint4* g4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.st_dy) + dy_off);
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        uint4 w;
-        w.x = pack_bf16(y[v * 8 + 0] * sc, y[v * 8 + 1] * sc);
-        w.y = pack_bf16(y[v * 8 + 2] * sc, y[v * 8 + 3] * sc);
-        w.z = pack_bf16(y[v * 8 + 4] * sc, y[v * 8 + 5] * sc);
-        w.w = pack_bf16(y[v * 8 + 6] * sc, y[v * 8 + 7] * sc);
-        o4[v] = w;
+        for (int v = 0; v < 8; ++v) {
+          const uint4 w = g4[v];
+          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            gr[v * 8 + 2 * e] = __uint_as_float(wv[e] << 16);
+            gr[v * 8 + 2 * e + 1] = __uint_as_float(wv[e] & 0xffff0000u);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) gr[e] = 0.f;
+      }
+      float sdy = 0.f;
+#pragma unroll
+      for (int e = 0; e < 64; ++e) sdy = fmaf(gr[e], y[e], sdy);
+      ms.ssx[wg][row] = ss;
+      ms.ex_s[0][wg][row] = sdy;
+      ms.ex_m[wg][row] = m;
+      bar_softmax();
+      const float m1 = ms.ex_m[0][row], m2 = ms.ex_m[1][row];
+      if (a.apply_norm) {
+        // out = s o / r with r^2 = mean(o^2) + eps and s = 1 - lambda_init, so the gradient
+        // reaching o is s / r (dy - o (dy . o) / (n r^2)), n = 128
+        const float r2 = (ms.ssx[0][row] + ms.ssx[1][row]) * (1.f / 128.f) + a.eps;
+        const float f = (1.f - a.lambda_init[0]) * rsqrtf(r2);
+        const float proj = (ms.ex_s[0][0][row] + ms.ex_s[0][1][row]) / (128.f * r2);
+#pragma unroll
+        for (int e = 0; e < 64; ++e) gr[e] = f * fmaf(-y[e], proj, gr[e]);
+      }
+      // delta_b = dO . O_b / l_b with the bf16 dO the backward's MMAs read (so that the
+      // row's dS sums to zero over its operands), the dlambda share -dO . O_2 / l_2 with the
+      // fp32 one; O_1 / l_1 = (D + c O_2) / l_1
+      float e1 = 0.f, e2 = 0.f, e3 = 0.f;
+      if (ok) {
+        const float c1 = c * inv1;
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          float dv[32], ov[32];
+          tmem_ld32f(lane_addr + COL_D + wg * 64 + ch * 32, dv);
+          tmem_ld32f(lane_addr + COL_O2 + wg * 64 + ch * 32, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint32_t h = pack_bf16(gr[ch * 32 + e], gr[ch * 32 + e + 1]);
+            const float g0 = __uint_as_float(h << 16), g1 = __uint_as_float(h & 0xffff0000u);
+            const float o1a = __fmaf_rn(ov[e], c1, dv[e] * inv1), o1b = __fmaf_rn(ov[e + 1], c1, dv[e + 1] * inv1);
+            const float o2a = ov[e] * inv2, o2b = ov[e + 1] * inv2;
+            e1 = fmaf(g1, o1b, fmaf(g0, o1a, e1));
+            e2 = fmaf(g1, o2b, fmaf(g0, o2a, e2));
+            e3 = fmaf(gr[ch * 32 + e + 1], o2b, fmaf(gr[ch * 32 + e], o2a, e3));
+          }
+        }
+      }
+      ms.ex_s[1][wg][row] = e1;
+      ms.ex_s[2][wg][row] = e2;
+      ms.ex_s[3][wg][row] = e3;
+      bar_softmax();
+      if (ok && qi < a.N) {
+        const int64_t do_off = (((int64_t)b * a.N + qi) * a.units + u) * 128 + wg * 64;
+        if (in_bounds(do_off, 64, a.ext_st_do, a.dev_status, a.dbg_status)) {
+          uint4* o4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.st_do) + do_off);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            o4[v] = make_uint4(pack_bf16(gr[v * 8 + 0], gr[v * 8 + 1]), pack_bf16(gr[v * 8 + 2], gr[v * 8 + 3]),
+                               pack_bf16(gr[v * 8 + 4], gr[v * 8 + 5]), pack_bf16(gr[v * 8 + 6], gr[v * 8 + 7]));
+        }
+        if (wg == 0) {
+          const int64_t r = ((int64_t)b * a.units + u) * a.st_rows + qi;
+          const int64_t rl = ((int64_t)b * a.units + u) * a.N + qi;
+          if (in_bounds(r * 4, 4, a.ext_st, a.dev_status, a.dbg_status))
+            *reinterpret_cast<float4*>(a.st + r * 4) =
+                make_float4(m1 + log2f(L1), m2 + log2f(L2), ms.ex_s[1][0][row] + ms.ex_s[1][1][row],
+                            ms.ex_s[2][0][row] + ms.ex_s[2][1][row]);
+          if (in_bounds(rl, 1, a.ext_st_dl, a.dev_status, a.dbg_status))
+            a.st_dl[rl] = -(ms.ex_s[3][0][row] + ms.ex_s[3][1][row]);
+        }
+      }
+    } else {
+      float sc = 1.f;
+      ms.ssx[wg][row] = ss;
+      bar_softmax();
+      if (a.apply_norm)
+        sc = rsqrtf((ms.ssx[0][row] + ms.ssx[1][row]) * (1.f / 128.f) + a.eps) *
+             (1.f - a.lambda_init[0]);
+      // (a variable-length tile reads its sequence back from shared memory, keeping the
+      // registers of the key loop free)
+      const int o_nq = VARLEN ? ms.seq_nq : a.N, o_b = VARLEN ? ms.seq_bc : b;
+      const int o_q0 = VARLEN ? ms.seq_q0 : 0;
+      const int64_t o_off = (int64_t)o_b * a.os[0] + (int64_t)(o_q0 + qi) * a.os[1] +
+                            (int64_t)u * a.os[2] + wg * 64;
+      if (ok && qi < o_nq && in_bounds(o_off, 64, a.ext_out, a.dev_status, a.dbg_status)) {
+        __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.out) + o_off;
+        uint4* o4 = reinterpret_cast<uint4*>(ob);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          uint4 w;
+          w.x = pack_bf16(y[v * 8 + 0] * sc, y[v * 8 + 1] * sc);
+          w.y = pack_bf16(y[v * 8 + 2] * sc, y[v * 8 + 3] * sc);
+          w.z = pack_bf16(y[v * 8 + 4] * sc, y[v * 8 + 5] * sc);
+          w.w = pack_bf16(y[v * 8 + 6] * sc, y[v * 8 + 7] * sc);
+          o4[v] = w;
+        }
       }
     }
   }
@@ -523,6 +645,38 @@ cudaError_t launch_prefill_v1(const PrefillArgs& a, cudaStream_t stream) {
     if (window) prefill_v1_kernel<true, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
     else prefill_v1_kernel<false, false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   }
+  return cudaGetLastError();
+}
+
+// The backward's statistics pass over the same tiles (fixed-length batches): st, st_dl,
+// st_dy and st_do must be set; out is not written.
+cudaError_t launch_prefill_v1_stats(const PrefillArgs& a, cudaStream_t stream) {
+  if (a.variant != DIFFATTN_V1 || a.d != 64 || a.cu_q) return cudaErrorNotSupported;
+  if (!a.st || !a.st_dl || !a.st_dy || !a.st_do) return cudaErrorInvalidValue;
+  TcMaps maps;
+  if (!make_map(&maps.q, a.q, 128, a.units, a.N, a.B, a.qs, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, 128, a.units, a.Nk, a.B, a.ks, BN)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.v, a.v, 128, a.units, a.Nk, a.B, a.vs, BN)) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  if (dev >= 64 || !attr_set[dev]) {
+    const void* fns[2] = {(const void*)prefill_v1_kernel<false, false, true>,
+                          (const void*)prefill_v1_kernel<true, false, true>};
+    for (const void* fn : fns) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+    }
+    if (dev < 64) attr_set[dev] = true;
+  }
+  const long long tiles = (long long)((a.N + BM - 1) / BM) * a.units * a.B;
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const dim3 grid((unsigned)tiles);
+  if (a.causal && a.window > 0)
+    prefill_v1_kernel<true, false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
+  else
+    prefill_v1_kernel<false, false, true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(maps, a);
   return cudaGetLastError();
 }
 

@@ -3,13 +3,16 @@ float64 backward oracle (itself pinned to finite differences of the forward orac
 torch autograd).
 
 Tolerances, per tensor:
-  * exact-fp32 kernels (fp32 inputs, V1, other head widths): the kernels compute in fp32
-    from the same input values the oracle reads (bf16 inputs are widened exactly), so the
-    only error is fp32 rounding of sums over at most a few thousand terms and of expf/logf:
+  * exact-fp32 kernels (fp32 inputs, other head widths): the kernels compute in fp32 from
+    the same input values the oracle reads (bf16 inputs are widened exactly), so the only
+    error is fp32 rounding of sums over at most a few thousand terms and of expf/logf:
     max abs error <= 2e-5 x max|reference| + 1e-6;
-  * tensor-core kernels (bf16 V2 with d = 128): the MMA operands P_1 - lambda P_2 and dS_b
-    are rounded to bf16 (relative 2^-9 each, independent across terms), as in the forward:
-    relative RMS error <= 5e-3 and max abs error <= 2e-2 x max|reference|."""
+  * tensor-core kernels (bf16 V2 with d = 128, bf16 V1 with d = 64): the MMA operands
+    P_1 - lambda P_2 and dS_b (and V1's dO) are rounded to bf16 (relative 2^-9 each,
+    independent across terms), as in the forward: relative RMS error <= 5e-3 and max abs
+    error <= 2e-2 x max|reference|. V1's statistics pass forms O and the norm's backward
+    from probabilities split into two bf16 parts (error ~2^-18), so dlambda, which keeps
+    only the small part of O_2 orthogonal to O, meets the same bound."""
 import numpy as np
 import pytest
 import torch
@@ -41,9 +44,10 @@ def _check(got, ref, what, tensor_core=False):
     assert err <= bound, f"{what}: max abs err {err:.3e} > {bound:.3e}"
 
 
-def _case(variant, Nq, Nk, dtype, seed, causal=True, window=0, norm=True, Hq=8, Hkv=2, H=2):
+def _case(variant, Nq, Nk, dtype, seed, causal=True, window=0, norm=True, Hq=8, Hkv=2, H=2, d=None):
     if variant == 1:
-        inp = synth.v1_small(B=2, N=Nk, H=H, seed=seed, dtype=dtype, causal=causal, apply_norm=norm)
+        inp = synth.v1_small(B=2, N=Nk, H=H, d=d or 64, seed=seed, dtype=dtype, causal=causal,
+                             apply_norm=norm)
     else:
         inp = synth.v2_small(B=2, N=Nk, Hq=Hq, Hkv=Hkv, seed=seed, dtype=dtype, causal=causal)
     q = dev_tensor(inp.q)[:, Nk - Nq:].contiguous()
@@ -66,7 +70,7 @@ def _case(variant, Nq, Nk, dtype, seed, causal=True, window=0, norm=True, Hq=8, 
     else:
         ref = OB.prefill_v2_bwd(q64, k64, v64, lam64, dy64, causal=causal, window=window)
     tag = f"V{variant} {dtype} Nq={Nq} Nk={Nk} causal={causal} window={window}"
-    tc = variant == 2 and dtype == "bf16"
+    tc = dtype == "bf16" and inp.d == (64 if variant == 1 else 128)
     for name, t, r in zip(("dq", "dk", "dv", "dlambda"), (dq, dk, dv, dl), ref):
         _check(t, r, f"{tag} {name}", tensor_core=tc)
 
@@ -87,6 +91,33 @@ def test_backward_full_chunk_window(variant):
 
 def test_backward_v1_without_norm():
     _case(1, 120, 120, "bf16", seed=750, norm=False)
+
+
+def test_backward_v1_other_width_exact():
+    """bf16 V1 with d != 64 runs the exact-fp32 kernels (and meets their bound)."""
+    _case(1, 90, 90, "bf16", seed=752, d=32)
+
+
+def test_backward_v1_layer_full_size():
+    """The V1 layer at full size (B=2, 16 heads, N=4096, d=64, the seeded synth.config2
+    tensors, the norm on), as the bench runs its backward. The float64 oracle covers one
+    seeded head over both batch entries: its dQ, dK, dV and dlambda."""
+    inp = synth.config2()
+    q, k, v = dev_tensor(inp.q), dev_tensor(inp.k), dev_tensor(inp.v)
+    dy_bits = synth.grad_out((inp.B, inp.N, inp.H, 2 * inp.d), 1001)
+    dy = dev_tensor(dy_bits)
+    lam, li = lambda_on_device(inp)
+    dq, dk, dv, dl = da.diffattn_bwd_prefill(q, k, v, lam, dy, li, apply_norm=True, norm_eps=inp.eps)
+    torch.cuda.synchronize()
+    h = int(np.random.default_rng(1001).integers(inp.H))
+    lam64 = oracle.lambda_(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.depth)[h:h + 1]
+    dy64 = synth.bf16_to_f32(dy_bits).astype(np.float64)[:, :, h:h + 1]
+    ref = OB.prefill_v1_bwd(inp.as_f64("q")[:, :, h:h + 1], inp.as_f64("k")[:, :, h:h + 1],
+                            inp.as_f64("v")[:, :, h:h + 1], lam64, oracle.lambda_init(inp.depth), dy64,
+                            apply_norm=True, eps=inp.eps)
+    got = (dq[:, :, h:h + 1], dk[:, :, h:h + 1], dv[:, :, h:h + 1], dl[h:h + 1])
+    for name, t, r in zip(("dq", "dk", "dv", "dlambda"), got, ref):
+        _check(t, r, f"V1 layer N=4096 head {h} {name}", tensor_core=True)
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(4, 2), (8, 1), (16, 2)])
@@ -142,14 +173,21 @@ def test_lambda_bwd():
         _check(t, r, name)
 
 
-def test_backward_deterministic():
+@pytest.mark.parametrize("variant", [1, 2])
+def test_backward_deterministic(variant):
     """No atomics: two calls give identical bits."""
-    inp = synth.v2_small(B=1, N=300, Hq=16, Hkv=2, seed=790)
+    if variant == 1:
+        inp = synth.v1_small(B=1, N=300, H=4, seed=791)
+        oshape = (1, 300, 4, 128)
+    else:
+        inp = synth.v2_small(B=1, N=300, Hq=16, Hkv=2, seed=790)
+        oshape = (1, 300, 8, 128)
     q, k, v = (dev_tensor(getattr(inp, n)) for n in ("q", "k", "v"))
-    lam, _ = lambda_on_device(inp)
-    dy = torch.randn((1, 300, 8, 128), generator=torch.Generator().manual_seed(2)).bfloat16().cuda()
-    a = da.diffattn_bwd_prefill(q, k, v, lam, dy)
-    b = da.diffattn_bwd_prefill(q, k, v, lam, dy)
+    lam, li = lambda_on_device(inp)
+    dy = torch.randn(oshape, generator=torch.Generator().manual_seed(2)).bfloat16().cuda()
+    kw = dict(apply_norm=True) if variant == 1 else {}
+    a = da.diffattn_bwd_prefill(q, k, v, lam, dy, li, **kw)
+    b = da.diffattn_bwd_prefill(q, k, v, lam, dy, li, **kw)
     torch.cuda.synchronize()
     for x, y in zip(a, b):
         assert torch.equal(x, y)
