@@ -2,19 +2,20 @@
 """Benchmark of the differential attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload c2|c3|c4|c5|d1|b3|p4] [--no-secondary]
+                    [--workload c2|c3|c4|c5|d1|b1|b3|p4] [--no-secondary]
 
 A step is one pass of the hot path over one batch of synthetic input: the on-device
 lambda re-parameterisation followed by the fused prefill (or the split-KV decode for the
 decode workload). Default workload (the largest one-GPU workload): c5, the V2 long-context
 signal-plus-noise prefill (B=1, N=65536, 64 query heads over 8 KV heads, d=128, causal).
 Other workloads: c2 the V1 bf16 layer (B=2, 16 heads, N=4096, d=64), c3 V2 prefill
-(N=16384, 64/8 heads, d=128), c4 V2 decode (batch 64, cache 32768), d1 V1 decode, b3 the
-backward of a V2 prefill (N=4096, 64/8 heads; step = lambda + the whole backward), p4 the c4
-decode over 16-token pages in a shuffled block table.
+(N=16384, 64/8 heads, d=128), c4 V2 decode (batch 64, cache 32768), d1 V1 decode, b1 the
+backward of the V1 layer and b3 that of a V2 prefill (N=4096, 64/8 heads; step = lambda +
+the whole backward), p4 the c4 decode over 16-token pages in a shuffled block table.
 Inputs are the seeded synthetic tensors of differential_attention_05_b200.synth. With the
 default workload the line also carries "secondary": the other rows timed alone (the V1
-layer and its exact-fp32 backward, the V2 prefill, its window and chunk forms, the training
+layer and its backward, on the tensor cores and exact in fp32, the V2 prefill, its window
+and chunk forms, the training
 forward and the backward from its saved outputs, and the backward that recomputes them, on
 the synth tensors; the decodes on same-shape seeded draws made on the device, each entry
 saying which).
@@ -58,6 +59,8 @@ def workload_inputs(name: str, batch: int = 0):
         return synth.v2_decode(B=batch, name=f"v2_bf16_decode_b{batch}_l32768_hq64_hkv8_d128")
     if name == "d1":
         return synth.v1_decode(B=batch) if batch else synth.v1_decode()
+    if name == "b1":
+        return synth.v1_backward()
     if name == "b3":
         return synth.v2_backward()
     if name == "p4":
@@ -268,7 +271,7 @@ def run_ours(args, rank, world, device):
     li = torch.empty(1, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
     decode = inp.mode == "decode"
-    backward = args.workload == "b3"
+    backward = args.workload in ("b1", "b3")
     paged = args.workload == "p4"
     if paged:
         # the cache as a pool of 16-token pages in a seeded shuffled order (block table)
@@ -299,9 +302,7 @@ def run_ours(args, rank, world, device):
         p = da._binding.prefill_params(q, k, v, dy)
         ws = torch.empty(da._binding.diffattn_bwd_workspace_size(p), dtype=torch.uint8, device=device)
         out = grads[0]
-        # algorithmic FLOPs per attended (query head, key) pair: 8 d (scores 2d, dP d per
-        # head, dQ 2d, dK 2d, dV d per head)
-        work = 8.0 * inp.d * inp.H * inp.B * visible_pairs(inp.N, inp.N, inp.causal)
+        work = backward_flops(inp)
         unit, metric = "TFLOP/s", "diff-attn backward TFLOP/s (% bf16 peak)"
     else:
         out = (torch.empty((inp.B, inp.N, inp.H, 2 * inp.d), dtype=torch.bfloat16, device=device)
@@ -329,7 +330,8 @@ def run_ours(args, rank, world, device):
             vp = v.view(inp.B * inp.N // ps, ps, inp.Hkv, inp.d)
             da.diffattn_fwd_decode_paged(q, kp, vp, bt, lam, out=out, workspace=ws)
         elif backward:
-            da.diffattn_bwd_prefill(q, k, v, lam, S["dy"], causal=inp.causal, workspace=ws,
+            da.diffattn_bwd_prefill(q, k, v, lam, S["dy"], li, causal=inp.causal,
+                                    apply_norm=inp.apply_norm, norm_eps=inp.eps, workspace=ws,
                                     grads=S["grads"])
         elif decode and inp.variant == 1:
             da.diffattn_fwd_decode_v1(q, k, v, lam, li, out=out, apply_norm=inp.apply_norm,
@@ -489,7 +491,7 @@ def run_ours(args, rank, world, device):
                   float(in_bytes + out.numel() * out.element_size()))
     if backward:
         # the timed span is the whole backward call (its four launches)
-        kernel_name = ("prefill_v2_kernel (statistics mode) + bwd_v2_dkdv_kernel + "
+        kernel_name = (f"prefill_v{inp.variant}_kernel (statistics mode) + bwd_v2_dkdv_kernel + "
                        "bwd_v2_dq_kernel + bwd_dlambda_kernel")
         traffic = None
     line = {
@@ -777,33 +779,47 @@ def oracle_decode_sample(inp, seconds):
 
 
 def oracle_backward_sample(inp, seconds):
-    """The float64 backward oracle on whole query-head pairs (full sequence, every key) of
-    a backward workload, pair after pair until `seconds` have passed; returns (pairs, s)."""
+    """The float64 backward oracle on whole units (a V1 head, a V2 query-head pair; full
+    sequence, every key) of a backward workload's first batch entry, unit after unit until
+    `seconds` have passed; returns (units, s)."""
     import oracle
     from oracle import backward as OB
     from differential_attention_05_b200 import synth
     lam = oracle.lambda_(inp.lq1, inp.lk1, inp.lq2, inp.lk2, inp.depth)
+    f64 = lambda a: synth.bf16_to_f32(a).astype(np.float64)
     group = inp.H // inp.Hkv
     t0 = time.perf_counter()
     n = 0
     while True:
-        p = n % (inp.H // 2)
-        g = (2 * p) // group
-        q = synth.bf16_to_f32(inp.q[:1, :, 2 * p:2 * p + 2]).astype(np.float64)
-        k = synth.bf16_to_f32(inp.k[:1, :, g:g + 1]).astype(np.float64)
-        v = synth.bf16_to_f32(inp.v[:1, :, g:g + 1]).astype(np.float64)
-        dy = synth.bf16_to_f32(inp.extra["dy"][:1, :, p:p + 1]).astype(np.float64)
-        OB.prefill_v2_bwd(q, k, v, lam[p:p + 1], dy, causal=inp.causal)
+        if inp.variant == 1:
+            h = n % inp.H
+            OB.prefill_v1_bwd(f64(inp.q[:1, :, h:h + 1]), f64(inp.k[:1, :, h:h + 1]),
+                              f64(inp.v[:1, :, h:h + 1]), lam[h:h + 1], oracle.lambda_init(inp.depth),
+                              f64(inp.extra["dy"][:1, :, h:h + 1]), causal=inp.causal,
+                              apply_norm=inp.apply_norm, eps=inp.eps)
+        else:
+            p = n % (inp.H // 2)
+            g = (2 * p) // group
+            OB.prefill_v2_bwd(f64(inp.q[:1, :, 2 * p:2 * p + 2]), f64(inp.k[:1, :, g:g + 1]),
+                              f64(inp.v[:1, :, g:g + 1]), lam[p:p + 1],
+                              f64(inp.extra["dy"][:1, :, p:p + 1]), causal=inp.causal)
         n += 1
         if time.perf_counter() - t0 >= seconds:
             break
     return n, time.perf_counter() - t0
 
 
-def backward_pair_flops(inp) -> float:
-    """Algorithmic FLOPs of one pair's backward over one batch entry (8 d per attended
-    (query head, key) pair, two query heads)."""
-    return 8.0 * inp.d * 2 * visible_pairs(inp.N, inp.N, inp.causal)
+def backward_flops(inp) -> float:
+    """Algorithmic FLOPs of a backward workload: per attended (query, key) pair 20 d per V1
+    head (scores 2 x 2d, dP = dO V^T 4d with V 2d wide, dV 4d, dK_1 + dK_2 4d, dQ_1 + dQ_2
+    4d) and 8 d per V2 query head (scores 2d, dP d per head, dQ 2d, dK 2d, dV d per head)."""
+    per = 20.0 * inp.d if inp.variant == 1 else 8.0 * inp.d
+    return per * inp.H * inp.B * visible_pairs(inp.N, inp.N, inp.causal)
+
+
+def backward_unit_flops(inp) -> float:
+    """backward_flops of one unit (V1 head, V2 pair) over one batch entry."""
+    return backward_flops(inp) / inp.B / inp.n_units
 
 
 def cpu_baseline(inp, seconds=12.0):
@@ -811,9 +827,10 @@ def cpu_baseline(inp, seconds=12.0):
     cores = oracle.default_threads()
     if "dy" in inp.extra:
         n, dt = oracle_backward_sample(inp, seconds)
-        return {"value": round(n * backward_pair_flops(inp) / dt / 1e12, 6), "unit": "TFLOP/s",
+        return {"value": round(n * backward_unit_flops(inp) / dt / 1e12, 6), "unit": "TFLOP/s",
                 "cores": cores, "kind": "oracle",
-                "sample": f"{n} whole query-head pairs (every row and key) of {inp.name}, {dt:.1f} s"}
+                "sample": f"{n} whole {'heads' if inp.variant == 1 else 'query-head pairs'} (every row "
+                          f"and key) of {inp.name}, {dt:.1f} s"}
     if inp.mode == "decode":
         n, dt = oracle_decode_sample(inp, seconds)
         val = n * workload_decode_bytes(inp) / inp.B / dt / 1e9
@@ -843,9 +860,10 @@ def run_reference(args, rank, world):
                 times.append((n, dt))
         total_units = sum(n for n, _ in times)
         total_s = sum(dt for _, dt in times)
-        value = total_units * backward_pair_flops(inp) / total_s / 1e12
+        value = total_units * backward_unit_flops(inp) / total_s / 1e12
         unit, metric = "TFLOP/s", "diff-attn backward TFLOP/s (% bf16 peak)"
-        sample = f"whole query-head pairs of {inp.name} ({total_units} in {total_s:.1f} s)"
+        sample = (f"whole {'heads' if inp.variant == 1 else 'query-head pairs'} of {inp.name} "
+                  f"({total_units} in {total_s:.1f} s)")
     elif decode:
         times = []
         for i in range(args.warmup + args.steps):
@@ -895,7 +913,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", choices=("c2", "c3", "c4", "c5", "d1", "b3", "p4"), default="c5")
+    ap.add_argument("--workload", choices=("c2", "c3", "c4", "c5", "d1", "b1", "b3", "p4"), default="c5")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="decode workload only: smaller batch (profiling runs)")

@@ -166,6 +166,15 @@ def grad_out(shape, seed: int) -> np.ndarray:
     return _normal_sliced(seed, _T_V + 17, tuple(shape))
 
 
+def v1_backward() -> Inputs:
+    """Backward of the V1 layer: the config2 inputs plus dy [B,N,H,2d] N(0,1) in
+    extra["dy"] (seed 1001)."""
+    inp = config2()
+    inp.name = "v1_bf16_backward_b2_h16_n4096_d64"
+    inp.extra["dy"] = grad_out((inp.B, inp.N, inp.H, 2 * inp.d), 1001)
+    return inp
+
+
 def v2_backward(B=1, N=4096, Hq=64, Hkv=8, d=128, depth=24, seed=1007, name=None) -> Inputs:
     """Backward of a V2 prefill: the V2 prefill inputs (iid N(0,1)) plus dy [B,N,Hq/2,d]
     N(0,1) in extra["dy"]."""

@@ -211,13 +211,16 @@ int diffattn_fwd_prefill_varlen(const diffattn_prefill_params* p, const int32_t*
  *              16-byte aligned; fully overwritten
  * dlambda    : float32 [units] (V1 heads / V2 pairs), overwritten; feed it to
  *              diffattn_lambda_bwd for the four lambda vectors
- * workspace  : >= diffattn_bwd_workspace_size(p) bytes, 256-byte aligned (per row: dO in
- *              fp32, two log-sum-exps, two deltas, the row's dlambda share)
- * Arithmetic: bf16 V2 with d = 128 runs on the tensor cores (fp32 accumulation; the MMA
- * operands P_1 - lambda P_2 and dS_b rounded to bf16, as the forward rounds its P operand);
- * every other case (fp32 inputs, V1, other d) runs exact fp32 on the CUDA cores. Both are
- * deterministic (no atomics: dQ rows, dK/dV rows and dlambda are each summed by one thread
- * group in a fixed order).
+ * workspace  : >= diffattn_bwd_workspace_size(p) bytes, 256-byte aligned (per row: two
+ *              log-sum-exps, two deltas, the row's dlambda share, and dO: fp32 on the exact
+ *              path, bf16 for V1 on the tensor cores)
+ * Arithmetic: bf16 V2 with d = 128 and bf16 V1 with d = 64 run on the tensor cores (fp32
+ * accumulation; the MMA operands P_1 - lambda P_2, dS_b and, for V1, dO rounded to bf16, as
+ * the forward rounds its P operand). V1's statistics pass forms O and its norm's backward
+ * from probability operands split into two bf16 parts (error ~2^-18), because dlambda
+ * through the norm keeps only the small part of O_2 orthogonal to O. Every other case (fp32
+ * inputs, other d) runs exact fp32 on the CUDA cores. Both are deterministic (no atomics:
+ * dQ rows, dK/dV rows and dlambda are each summed by one thread group in a fixed order).
  * Streams (tensor-core path): the dK/dV and dQ kernels run side by side, the dQ kernel on a
  * stream the library creates once per device, forked from `stream` and joined back to it
  * (events) before the call's last kernel. The call therefore stays ordered on `stream` and
