@@ -93,7 +93,7 @@ struct Misc {
   float ex_c[BM];         // epilogue: c
   float ssx[2][BM];       // V1 norm: partial sums of squares
   float ex_m[2][BM];      // statistics pass: [branch][row] maxima
-  float ex_s[3][2][BM];   //                  [quantity][half][row] partial dot products
+  float ex_s[4][2][BM];   //                  [quantity][half][row] partial dot products
 };
 static_assert(sizeof(Misc) <= MISC_BYTES, "misc region");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
