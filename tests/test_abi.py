@@ -312,6 +312,18 @@ def test_backward_workspace_and_rejects(lib):
     assert n.value == up(rows * 128 * 4) + up(rows * 16) + up(rows * 4)
     big = _prefill_params(head_dim=256)
     assert lib.diffattn_bwd_workspace_size(ctypes.byref(big), ctypes.byref(n)) == -2
+    # V1 (H = 4 heads): bf16 with d = 64 takes the tensor-core path, whose workspace adds
+    # the bf16 dO through the norm [B, N, H, 2d]; bf16 with another d and fp32 take the
+    # exact kernels (fp32 dO rows of width 2d)
+    v1 = lambda **kw: _prefill_params(variant=B.DIFFATTN_V1, n_q_heads=4, n_kv_heads=4, apply_norm=1, **kw)
+    r1 = 256 * 4
+    assert lib.diffattn_bwd_workspace_size(ctypes.byref(v1(head_dim=64)), ctypes.byref(n)) == 0
+    assert n.value == up(4 * (256 + 64) * 16) + up(r1 * 4) + up(r1 * 128 * 2)
+    assert lib.diffattn_bwd_workspace_size(ctypes.byref(v1(head_dim=32)), ctypes.byref(n)) == 0
+    assert n.value == up(r1 * 64 * 4) + up(r1 * 16) + up(r1 * 4)
+    assert lib.diffattn_bwd_workspace_size(ctypes.byref(v1(head_dim=64, dtype=B.DIFFATTN_F32)),
+                                           ctypes.byref(n)) == 0
+    assert n.value == up(r1 * 128 * 4) + up(r1 * 16) + up(r1 * 4)
     f = lib.diffattn_bwd_prefill
     ptr = [vp(GOOD), vp(GOOD + 4096), vp(GOOD + 8192), vp(GOOD + 12288), None, vp(GOOD + 16384)]
     outs = [vp(GOOD + 20480), vp(GOOD + 24576), vp(GOOD + 28672), vp(GOOD + 32768)]
